@@ -1,0 +1,395 @@
+"""Oracle -- TEST INFRASTRUCTURE, not part of the product.
+
+A plain, slow, float64 CPU restatement of the partial-recompute denoising step
+of one bidirectional masked diffusion-LM layer.  Only ``tests/``,
+``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import
+it.  It shares no code with the CUDA library and never calls it.
+
+Pages followed (cited by title and section):
+
+[SL]  "Stopping Computation for Converged Tokens in Masked Diffusion-LM Decoding"
+      (SureLock).  Sec. 1 Problem Statement; Sec. 2 Methodology: "Locking
+      Condition", "Permanent Deactivation", "Continued Attention",
+      "Algorithmic Complexity"; Sec. 5 Significance.
+[SPA] "SPA-Cache: Singular Proxies for Adaptive Caching in Diffusion Language
+      Models".  Part 1 "low-resolution snapshot (Singular Proxies)"; part 2
+      "smart budget (Adaptive Caching)".
+[PS]  "Polestar: Drift-Aware Cache Calibration and Token Commitment for
+      Efficient Inference of Diffusion LLMs".  Polestar-Cache: refresh only the
+      positions whose representation drifted most.
+
+Readings taken where the pages are silent (each is listed in the design notes):
+
+R1  Layer form.  Pre-norm block  h = x + Attn(RMSNorm1(x)),
+    y = h + W_down (silu(W_g hn) * (W_u hn)),  hn = RMSNorm2(h).  Multi-head
+    attention with H heads of size hd, non-causal, scale 1/sqrt(hd), no RoPE,
+    no biases.  RMSNorm(x) = x / sqrt(mean(x^2) + eps) * g.
+R2  A locked row skips the whole block: its Q, K/V, FFN and output are frozen
+    ([SL] Sec. 2 "Permanent Deactivation").  Active rows get fresh K/V, which
+    are written into the cache *before* attention, so every active query sees
+    the current K/V of active keys and the cached K/V of locked keys ([SL]
+    Sec. 2 "Continued Attention").
+R3  Order inside a step: score -> lock -> compute on the rows still active.
+R4  The proxy of a row is p = U^T x on the layer *input* hidden state; the
+    proxy cache stores float32 and is refreshed only for recomputed rows.
+    cosine(a, b) = a.b / max(|a||b|, 1e-30); L2 = |a - b| (not squared).
+R5  Threshold rule: lock when score > tau (or < tau), strictly; a NaN score
+    never locks.  Budget rule: keep the k rows with the largest (or smallest)
+    score among the rows not yet locked; equal scores go to the lower index;
+    NaN is never preferred; +0 and -0 are equal.  Rows not kept are locked.
+R6  Precision policy "bf16": every tensor that the bf16 path stores in bf16
+    between operations is rounded to bf16 here as well -- the normalised
+    inputs of the projections (xn, hn), q, k, v (and so the K/V cache), the
+    attention output a, the SwiGLU product, and the layer output y.  The
+    residual stream h stays unrounded.  All arithmetic is float64.  Policy
+    "f64" rounds nothing.
+
+Parity unpinned: the pages print no tensor values, so nothing here is pinned to
+a printed example; every function is pinned instead to library routines,
+brute force, closed forms and invariants in ``tests/test_oracle_*.py``.
+"""
+from __future__ import annotations
+
+import contextlib
+import math
+
+import numpy as np
+
+__all__ = [
+    "to_bf16", "to_f32", "count_flops", "rmsnorm", "silu",
+    "proxy_project", "drift_cosine", "drift_l2", "score_drift",
+    "lock_threshold", "lock_topk", "compact",
+    "full_layer_step", "layer_step_partial", "proxy_commit",
+    "LayerState", "tiny_run",
+]
+
+# ---------------------------------------------------------------------------
+# rounding helpers (the precision policy R6)
+# ---------------------------------------------------------------------------
+_BF16_OVERFLOW = 2.0 ** 128
+
+
+def to_bf16(a) -> np.ndarray:
+    """Round float64 values to the nearest bf16 value, ties to even, as float64.
+
+    bf16 keeps 8 significant bits: a = m * 2**e with 0.5 <= |m| < 1 is rounded
+    to a multiple of 2**(e-8) (2**-133 below the normal range).
+    """
+    a = np.asarray(a, dtype=np.float64)
+    _, e = np.frexp(a)
+    q = np.ldexp(1.0, np.maximum(e - 8, -133))
+    with np.errstate(invalid="ignore", over="ignore"):
+        r = np.rint(a / q) * q
+    big = np.abs(r) >= _BF16_OVERFLOW
+    if np.any(big):
+        r = np.where(big, np.copysign(np.inf, a), r)
+    return r
+
+
+def to_f32(a) -> np.ndarray:
+    """Round to float32 storage (numpy's round-to-nearest-even) and return float64."""
+    return np.asarray(a, dtype=np.float64).astype(np.float32).astype(np.float64)
+
+
+def _store(a, policy):
+    return to_bf16(a) if policy == "bf16" else np.asarray(a, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# FLOP counting: every contraction goes through _mm
+# ---------------------------------------------------------------------------
+class _Counter:
+    def __init__(self):
+        self.flops = 0
+
+
+_counter: _Counter | None = None
+
+
+@contextlib.contextmanager
+def count_flops():
+    """Count 2*m*n*k for every product  a[m,k] @ b[n,k]^T  made inside the block."""
+    global _counter
+    prev, _counter = _counter, _Counter()
+    try:
+        yield _counter
+    finally:
+        _counter = prev
+
+
+def _mm(a, b):
+    """a [m, k] times b [n, k] transposed (nn.Linear weight layout)."""
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    if _counter is not None:
+        _counter.flops += 2 * a.shape[0] * b.shape[0] * a.shape[1]
+    return a @ b.T
+
+
+# ---------------------------------------------------------------------------
+# elementwise pieces of the layer (R1)
+# ---------------------------------------------------------------------------
+def rmsnorm(x, g, eps):
+    """x / sqrt(mean(x^2) + eps) * g over the last axis."""
+    x = np.asarray(x, dtype=np.float64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * np.asarray(g, dtype=np.float64)
+
+
+def silu(z):
+    """z * sigmoid(z) = z / (1 + exp(-z))."""
+    z = np.asarray(z, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return z / (1.0 + np.exp(-z))
+
+
+# ---------------------------------------------------------------------------
+# S1: drift score on the singular proxy ([SPA] part 1; [PS] drift)
+# ---------------------------------------------------------------------------
+def proxy_project(x_rows, Ut):
+    """p = U^T x for each row: x_rows [m, d], Ut [r, d] (rows = proxy directions) -> [m, r]."""
+    return _mm(x_rows, Ut)
+
+
+def drift_cosine(p, pc):
+    """cos(p, pc) per row with the 1e-30 floor of R4 (a zero vector gives 0)."""
+    p = np.asarray(p, dtype=np.float64)
+    pc = np.asarray(pc, dtype=np.float64)
+    dot = np.sum(p * pc, axis=-1)
+    den = np.sqrt(np.sum(p * p, axis=-1)) * np.sqrt(np.sum(pc * pc, axis=-1))
+    return dot / np.maximum(den, 1e-30)
+
+
+def drift_l2(p, pc):
+    """Euclidean distance |p - pc| per row (R4)."""
+    diff = np.asarray(p, dtype=np.float64) - np.asarray(pc, dtype=np.float64)
+    return np.sqrt(np.sum(diff * diff, axis=-1))
+
+
+def score_drift(X, Ut, proxy_cache, metric):
+    """S1 for every row of X [B, N, d]: returns (score [B, N], p [B, N, r]) in float64.
+
+    metric "cos": cosine similarity between the fresh proxy and the cached one
+    (high = converged); metric "l2": Euclidean drift (high = changed).
+    """
+    B, N, d = X.shape
+    p = proxy_project(np.asarray(X, dtype=np.float64).reshape(B * N, d), Ut)
+    pc = np.asarray(proxy_cache, dtype=np.float64).reshape(B * N, -1)
+    if metric == "cos":
+        s = drift_cosine(p, pc)
+    elif metric == "l2":
+        s = drift_l2(p, pc)
+    else:
+        raise ValueError(metric)
+    return s.reshape(B, N), p.reshape(B, N, -1)
+
+
+def proxy_commit(proxy_cache, p, idx):
+    """S10 (proxy half): rows in idx (flattened b*N+i) take the fresh proxy, stored as float32."""
+    out = np.array(proxy_cache, dtype=np.float64, copy=True)
+    flat = out.reshape(-1, out.shape[-1])
+    flat[np.asarray(idx, dtype=np.int64)] = to_f32(np.asarray(p).reshape(-1, out.shape[-1])[idx])
+    return out
+
+
+# ---------------------------------------------------------------------------
+# S2: lock rules ([SL] Sec. 2 "Locking Condition", "Permanent Deactivation";
+#     [SPA] part 2 budget; [PS] largest-drift refresh)
+# ---------------------------------------------------------------------------
+def lock_threshold(score, lock_in, tau, greater=True):
+    """Permanent threshold lock: lock' = lock or (score > tau) [or (score < tau)].
+
+    Once locked a row stays locked.  NaN compares false and never locks.
+    """
+    s = np.asarray(score, dtype=np.float64)
+    with np.errstate(invalid="ignore"):
+        hit = (s > tau) if greater else (s < tau)
+    return (np.asarray(lock_in).astype(bool) | hit).astype(np.uint8)
+
+
+def lock_topk(score, lock_in, k, largest=True):
+    """Budget rule: per sequence keep the k best-scoring unlocked rows active, lock the rest.
+
+    "Best" is the largest score (or the smallest); ties go to the lower index;
+    NaN is never preferred; a sequence with fewer than k unlocked rows keeps
+    them all.
+    """
+    s = np.asarray(score, dtype=np.float64)
+    lk = np.asarray(lock_in).astype(bool)
+    B, N = s.shape
+    out = np.ones((B, N), dtype=np.uint8)
+    for b in range(B):
+        cand = [i for i in range(N) if not lk[b, i]]
+
+        def key(i):
+            v = s[b, i]
+            if math.isnan(v):
+                return (1, 0.0, i)
+            return (0, -v if largest else v, i)
+
+        for i in sorted(cand, key=key)[: max(int(k), 0)]:
+            out[b, i] = 0
+    return out
+
+
+# ---------------------------------------------------------------------------
+# S3: compaction of the active set ([SL] Sec. 2: a locked row leaves A_t)
+# ---------------------------------------------------------------------------
+def compact(lock):
+    """Ascending flattened indices b*N+i of the active rows, and seg_ptr [B+1]."""
+    lk = np.asarray(lock).astype(bool)
+    B, N = lk.shape
+    idx, seg = [], [0]
+    for b in range(B):
+        for i in range(N):
+            if not lk[b, i]:
+                idx.append(b * N + i)
+        seg.append(len(idx))
+    return np.asarray(idx, dtype=np.int64), np.asarray(seg, dtype=np.int64)
+
+
+# ---------------------------------------------------------------------------
+# S4..S10: the layer block
+# ---------------------------------------------------------------------------
+class LayerState:
+    """Caller-owned caches of one layer: K, V, Y [B, N, d] (float64 values)."""
+
+    def __init__(self, K, V, Y):
+        self.K = np.asarray(K, dtype=np.float64)
+        self.V = np.asarray(V, dtype=np.float64)
+        self.Y = np.asarray(Y, dtype=np.float64)
+
+    def copy(self):
+        return LayerState(self.K.copy(), self.V.copy(), self.Y.copy())
+
+
+def _w(W, name):
+    return np.asarray(W[name], dtype=np.float64)
+
+
+def full_layer_step(dims, W, X, policy="f64"):
+    """Baseline sampler: recompute the block for all N rows ([SL] Sec. 1: O(N^2 d) + O(N d^2)).
+
+    Matrix form: every row of every sequence, attention as the full
+    softmax(Q K^T / sqrt(hd)) V matrix product per (sequence, head).
+    Returns the LayerState (K, V, Y) of all rows.
+    """
+    B, N, d, H, hd, F = dims.B, dims.N, dims.d, dims.H, dims.hd, dims.F
+    x = np.asarray(X, dtype=np.float64).reshape(B * N, d)
+    xn = _store(rmsnorm(x, W["g1"], dims.eps), policy)
+    qkv = _mm(xn, _w(W, "w_qkv"))
+    q = _store(qkv[:, :d], policy)
+    k = _store(qkv[:, d:2 * d], policy)
+    v = _store(qkv[:, 2 * d:], policy)
+    a = np.zeros((B * N, d))
+    scale = 1.0 / math.sqrt(hd)
+    for b in range(B):
+        rows = slice(b * N, (b + 1) * N)
+        for h in range(H):
+            cols = slice(h * hd, (h + 1) * hd)
+            S = _mm(q[rows, cols], k[rows, cols]) * scale          # [N, N]
+            S = S - S.max(axis=1, keepdims=True)
+            P = np.exp(S)
+            P = P / P.sum(axis=1, keepdims=True)
+            a[rows, cols] = _mm(P, v[rows, cols].T)                # [N, hd]
+    a = _store(a, policy)
+    hres = x + _mm(a, _w(W, "w_o"))
+    hn = _store(rmsnorm(hres, W["g2"], dims.eps), policy)
+    gu = _mm(hn, _w(W, "w_gu"))
+    act = _store(silu(gu[:, :F]) * gu[:, F:], policy)
+    y = _store(hres + _mm(act, _w(W, "w_down")), policy)
+    return LayerState(k.reshape(B, N, d), v.reshape(B, N, d), y.reshape(B, N, d))
+
+
+def layer_step_partial(dims, W, X, idx, seg_ptr, state, policy="f64", out_rows=None):
+    """Partial-recompute step ([SL] Sec. 2 "Permanent Deactivation", "Continued Attention").
+
+    Only the rows in ``idx`` (flattened b*N+i, ascending, grouped by seg_ptr)
+    go through the block.  Their fresh K/V replace the cached rows first (R2);
+    each active query then attends over all N cached keys of its sequence.
+    Cost: attention O(M N d), projections and FFN O(M d^2) ([SL] Sec. 2
+    "Algorithmic Complexity").
+
+    ``out_rows`` (positions into idx) restricts S7..S10 to a sample of the
+    active rows; K/V are still refreshed for every active row.
+    Returns a new LayerState; ``state`` is not modified.
+    """
+    B, N, d, H, hd, F = dims.B, dims.N, dims.d, dims.H, dims.hd, dims.F
+    idx = np.asarray(idx, dtype=np.int64)
+    seg_ptr = np.asarray(seg_ptr, dtype=np.int64)
+    out = state.copy()
+    M = idx.shape[0]
+    if M == 0:
+        return out
+    x_all = np.asarray(X, dtype=np.float64).reshape(B * N, d)
+    # S4 gather + RMSNorm1
+    x = x_all[idx]
+    xn = _store(rmsnorm(x, W["g1"], dims.eps), policy)
+    # S5 projections (Q only for active rows: [SL] Sec. 2 skips Q of locked rows)
+    qkv = _mm(xn, _w(W, "w_qkv"))
+    q = _store(qkv[:, :d], policy)
+    k = _store(qkv[:, d:2 * d], policy)
+    v = _store(qkv[:, 2 * d:], policy)
+    # S6 K/V scatter into the cache rows of the active positions
+    Kf = out.K.reshape(B * N, d)
+    Vf = out.V.reshape(B * N, d)
+    Kf[idx] = k
+    Vf[idx] = v
+    rows = np.arange(M) if out_rows is None else np.asarray(out_rows, dtype=np.int64)
+    # S7 attention of each active query over all N keys of its sequence
+    seq_of = np.searchsorted(seg_ptr, np.arange(M), side="right") - 1
+    scale = 1.0 / math.sqrt(hd)
+    a = np.zeros((rows.shape[0], d))
+    for t, j in enumerate(rows):
+        b = int(seq_of[j])
+        Kb = Kf[b * N:(b + 1) * N]
+        Vb = Vf[b * N:(b + 1) * N]
+        for h in range(H):
+            cols = slice(h * hd, (h + 1) * hd)
+            s = _mm(q[j:j + 1, cols], Kb[:, cols])[0] * scale     # [N]
+            s = s - s.max()
+            p = np.exp(s)
+            p = p / p.sum()
+            a[t, cols] = _mm(p[None, :], Vb[:, cols].T)[0]        # [hd]
+    a = _store(a, policy)
+    # S8 output projection + residual
+    hres = x[rows] + _mm(a, _w(W, "w_o"))
+    # S9 RMSNorm2 + SwiGLU + residual
+    hn = _store(rmsnorm(hres, W["g2"], dims.eps), policy)
+    gu = _mm(hn, _w(W, "w_gu"))
+    act = _store(silu(gu[:, :F]) * gu[:, F:], policy)
+    y = _store(hres + _mm(act, _w(W, "w_down")), policy)
+    # S10 output scatter (locked rows of Y untouched)
+    out.Y.reshape(B * N, d)[idx[rows]] = y
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Tiny fp32 workload driver: 20 denoising steps with the threshold lock
+# ---------------------------------------------------------------------------
+def tiny_run(dims, W, X0, Ut, lock0, noises, tau, perturb):
+    """The tiny fp32 workload, step by step, in float64.
+
+    Start: full step on X0 fills K/V/Y; proxy cache = fp32(U^T X0).  Then for
+    each noise tensor: (i) X += noise on the active rows (``perturb`` is the
+    harness's data-prep helper), (ii) cosine drift, (iii) threshold lock
+    (score > tau), (iv) compaction, (v) block on the rows still active,
+    (vi) proxy cache refresh for those rows.
+    Returns a list of per-step records.
+    """
+    state = full_layer_step(dims, W, X0, "f64")
+    x0 = np.asarray(X0, dtype=np.float64).reshape(dims.B * dims.N, dims.d)
+    pc = to_f32(proxy_project(x0, Ut)).reshape(dims.B, dims.N, -1)
+    lock = np.asarray(lock0, dtype=np.uint8).copy()
+    X = np.asarray(X0, dtype=np.float32).copy()
+    recs = []
+    for t, eps in enumerate(noises):
+        X = perturb(X, eps, lock == 0)
+        score, p = score_drift(X.astype(np.float64), Ut, pc, "cos")
+        lock = lock_threshold(score, lock, tau, greater=True)
+        idx, seg = compact(lock)
+        state = layer_step_partial(dims, W, X.astype(np.float64), idx, seg, state, "f64")
+        pc = proxy_commit(pc, p, idx)
+        recs.append(dict(X=X.copy(), score=score, lock=lock.copy(), idx=idx, seg_ptr=seg,
+                         K=state.K.copy(), V=state.V.copy(), Y=state.Y.copy(), proxy=pc.copy()))
+    return recs

@@ -1,0 +1,431 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test ties an oracle function to a library routine, a brute-force loop on a
+tiny input, a closed form from the SureLock page ("Stopping Computation for
+Converged Tokens in Masked Diffusion-LM Decoding", Sec. 2 "Algorithmic
+Complexity"), or an invariant the pages state.  The mutation tests at the end
+plant plausible mistakes in copies of the oracle and check that a pin fails.
+"""
+import hashlib
+import inspect
+import math
+import textwrap
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as Fnn
+
+import oracle
+import synth
+from oracle import plk_oracle as po
+
+
+def _dims(B=2, N=7, d=16, H=2, hd=8, F=24, dtype="f32"):
+    return synth.Dims(B=B, N=N, d=d, H=H, hd=hd, F=F, eps=1e-6, dtype=dtype)
+
+
+def _weights(dims, std=None, seed=0):
+    return synth.layer_weights(dims, std if std is not None else 1.0 / math.sqrt(dims.d), seed=seed)
+
+
+# ---------------------------------------------------------------------------
+# rounding
+# ---------------------------------------------------------------------------
+def test_to_bf16_matches_torch_rounding():
+    rng = np.random.default_rng(1)
+    v = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32) * 10.0 ** rng.integers(-30, 30, 20000),
+        np.array([0.0, -0.0, 1.0, 1.00390625, 1.01171875, 3.3895314e38, -3.3895314e38,
+                  3.4e38, 1e-40, -1e-41, 2.0 ** -133, 2.0 ** -134], dtype=np.float32),
+    ]).astype(np.float32)
+    # exact ties: 1 + 2^-8 (rounds down to even) and 1 + 3*2^-8 (rounds up)
+    got = oracle.to_bf16(v.astype(np.float64))
+    ref = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_to_f32_is_numpy_cast():
+    v = np.array([1.0 + 2.0 ** -30, 1e-50, 3.0], dtype=np.float64)
+    np.testing.assert_array_equal(oracle.to_f32(v), v.astype(np.float32).astype(np.float64))
+
+
+# ---------------------------------------------------------------------------
+# elementwise pieces against torch
+# ---------------------------------------------------------------------------
+def test_rmsnorm_matches_torch():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((5, 33))
+    g = rng.standard_normal(33)
+    ref = Fnn.rms_norm(torch.from_numpy(x), (33,), torch.from_numpy(g), eps=1e-6).numpy()
+    np.testing.assert_allclose(oracle.rmsnorm(x, g, 1e-6), ref, rtol=1e-13, atol=1e-14)
+
+
+def test_silu_matches_torch():
+    z = np.linspace(-50, 50, 1001)
+    np.testing.assert_allclose(oracle.silu(z), Fnn.silu(torch.from_numpy(z)).numpy(),
+                               rtol=1e-13, atol=1e-300)
+
+
+# ---------------------------------------------------------------------------
+# the full block against a composition of torch library routines
+# ---------------------------------------------------------------------------
+def torch_block(dims, W, X):
+    B, N, d, H, hd, F = dims.B, dims.N, dims.d, dims.H, dims.hd, dims.F
+    t = lambda a: torch.from_numpy(np.asarray(a, dtype=np.float64))
+    x = t(X)
+    xn = Fnn.rms_norm(x, (d,), t(W["g1"]), eps=dims.eps)
+    qkv = Fnn.linear(xn, t(W["w_qkv"]))
+    q, k, v = qkv.split(d, dim=-1)
+    heads = lambda z: z.reshape(B, N, H, hd).transpose(1, 2)
+    a = Fnn.scaled_dot_product_attention(heads(q), heads(k), heads(v), is_causal=False)
+    a = a.transpose(1, 2).reshape(B, N, d)
+    h = x + Fnn.linear(a, t(W["w_o"]))
+    hn = Fnn.rms_norm(h, (d,), t(W["g2"]), eps=dims.eps)
+    g, u = Fnn.linear(hn, t(W["w_gu"])).split(F, dim=-1)
+    y = h + Fnn.linear(Fnn.silu(g) * u, t(W["w_down"]))
+    return k.numpy(), v.numpy(), y.numpy()
+
+
+@pytest.mark.parametrize("shape", [dict(B=1, N=9, d=16, H=2, hd=8, F=24),
+                                   dict(B=3, N=5, d=12, H=3, hd=4, F=8),
+                                   dict(B=1, N=64, d=64, H=4, hd=16, F=256)])
+def test_full_step_matches_torch_composition(shape):
+    dims = _dims(**shape)
+    W = _weights(dims)
+    X = synth.hidden_states(dims)
+    st = oracle.full_layer_step(dims, W, X, "f64")
+    k, v, y = torch_block(dims, W, X)
+    np.testing.assert_allclose(st.K, k, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(st.V, v, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(st.Y, y, rtol=0, atol=1e-11)
+
+
+def test_attention_matches_sdpa_single_head():
+    # textbook softmax(Q K^T / sqrt(hd)) V through the oracle's full step with
+    # identity projections: d = hd, H = 1, w_qkv = [I; I; I], w_o = 0, FFN = 0
+    N, d = 11, 6
+    dims = _dims(B=1, N=N, d=d, H=1, hd=d, F=4)
+    rng = np.random.default_rng(3)
+    eye = np.eye(d)
+    W = dict(w_qkv=np.concatenate([eye, 2 * eye, -eye]), w_o=np.eye(d), w_gu=np.zeros((8, d)),
+             w_down=np.zeros((d, 4)), g1=np.ones(d), g2=np.ones(d))
+    X = rng.standard_normal((1, N, d))
+    st = oracle.full_layer_step(dims, W, X, "f64")
+    xn = oracle.rmsnorm(X[0], np.ones(d), 1e-6)
+    a = Fnn.scaled_dot_product_attention(torch.from_numpy(xn)[None], torch.from_numpy(2 * xn)[None],
+                                         torch.from_numpy(-xn)[None]).numpy()[0]
+    np.testing.assert_allclose(st.Y[0], X[0] + a, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# brute force: explicit scalar loops on a tiny input
+# ---------------------------------------------------------------------------
+def brute_block(dims, W, X, rows):
+    B, N, d, H, hd, F = dims.B, dims.N, dims.d, dims.H, dims.hd, dims.F
+    Wq = W["w_qkv"]
+    out = {}
+
+    def norm(vec, g):
+        ms = sum(z * z for z in vec) / len(vec)
+        r = 1.0 / math.sqrt(ms + dims.eps)
+        return [vec[i] * r * float(g[i]) for i in range(len(vec))]
+
+    def lin(wm, vec):
+        return [sum(float(wm[o][i]) * vec[i] for i in range(len(vec))) for o in range(len(wm))]
+
+    xs = {(b, n): [float(X[b][n][c]) for c in range(d)] for b in range(B) for n in range(N)}
+    kv = {}
+    for (b, n), vec in xs.items():
+        z = lin(Wq, norm(vec, W["g1"]))
+        kv[(b, n)] = (z[:d], z[d:2 * d], z[2 * d:])
+    for (b, n) in rows:
+        q = kv[(b, n)][0]
+        a = [0.0] * d
+        for h in range(H):
+            sc = []
+            for m in range(N):
+                kk = kv[(b, m)][1]
+                sc.append(sum(q[h * hd + c] * kk[h * hd + c] for c in range(hd)) / math.sqrt(hd))
+            mx = max(sc)
+            ex = [math.exp(s - mx) for s in sc]
+            tot = sum(ex)
+            for c in range(hd):
+                a[h * hd + c] = sum(ex[m] / tot * kv[(b, m)][2][h * hd + c] for m in range(N))
+        hres = [xs[(b, n)][c] + lin(W["w_o"], a)[c] for c in range(d)]
+        hn = norm(hres, W["g2"])
+        gu = lin(W["w_gu"], hn)
+        act = [gu[f] / (1.0 + math.exp(-gu[f])) * gu[F + f] for f in range(F)]
+        dn = lin(W["w_down"], act)
+        out[(b, n)] = [hres[c] + dn[c] for c in range(d)]
+    return kv, out
+
+
+def test_full_and_partial_match_brute_force():
+    dims = _dims(B=2, N=5, d=8, H=2, hd=4, F=12)
+    W = _weights(dims)
+    X = synth.hidden_states(dims, seed=4)
+    rows = [(b, n) for b in range(2) for n in range(5)]
+    kv, yb = brute_block(dims, W, X, rows)
+    st = oracle.full_layer_step(dims, W, X, "f64")
+    for (b, n) in rows:
+        np.testing.assert_allclose(st.K[b, n], kv[(b, n)][1], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(st.V[b, n], kv[(b, n)][2], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(st.Y[b, n], yb[(b, n)], rtol=0, atol=1e-12)
+    lock = np.zeros((2, 5), np.uint8)
+    idx, seg = oracle.compact(lock)
+    zero = oracle.LayerState(np.zeros_like(st.K), np.zeros_like(st.V), np.zeros_like(st.Y))
+    sp = oracle.layer_step_partial(dims, W, X, idx, seg, zero, "f64")
+    for (b, n) in rows:
+        np.testing.assert_allclose(sp.Y[b, n], yb[(b, n)], rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# invariants stated by the SureLock page (Sec. 2)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("policy", ["f64", "bf16"])
+def test_partial_with_all_rows_equals_full(policy):
+    dims = _dims(B=2, N=12, d=32, H=2, hd=16, F=48, dtype="bf16" if policy == "bf16" else "f32")
+    W = _weights(dims)
+    X = synth.hidden_states(dims, seed=5)
+    full = oracle.full_layer_step(dims, W, X, policy)
+    idx, seg = oracle.compact(np.zeros((2, 12), np.uint8))
+    zero = oracle.LayerState(np.zeros_like(full.K), np.zeros_like(full.V), np.zeros_like(full.Y))
+    part = oracle.layer_step_partial(dims, W, X, idx, seg, zero, policy)
+    if policy == "f64":
+        for a, b in ((part.K, full.K), (part.V, full.V), (part.Y, full.Y)):
+            np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+    else:
+        # same values; a bf16 rounding may flip on a 1e-16 difference in the
+        # two summation forms, so allow one bf16 ulp on a tiny fraction
+        for a, b in ((part.K, full.K), (part.V, full.V), (part.Y, full.Y)):
+            ulp = np.ldexp(1.0, np.frexp(np.abs(b) + 1e-30)[1] - 8)
+            assert np.all(np.abs(a - b) <= ulp)
+            assert np.mean(a != b) < 1e-2
+
+
+def test_unchanged_inputs_partial_rows_equal_full_rows():
+    dims = _dims(B=2, N=10, d=16, H=2, hd=8, F=32)
+    W = _weights(dims)
+    X = synth.hidden_states(dims, seed=6)
+    full = oracle.full_layer_step(dims, W, X, "f64")
+    lock = synth.bernoulli_active(2, 10, 0.4, seed=6)
+    idx, seg = oracle.compact(lock)
+    assert 0 < idx.size < 20
+    part = oracle.layer_step_partial(dims, W, X, idx, seg, full, "f64")
+    for a, b in ((part.K, full.K), (part.V, full.V), (part.Y, full.Y)):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+
+
+def _h(a):
+    return hashlib.sha256(np.ascontiguousarray(a).tobytes()).hexdigest()
+
+
+def test_locked_rows_untouched():
+    dims = _dims(B=2, N=10, d=16, H=2, hd=8, F=32)
+    W = _weights(dims)
+    X = synth.hidden_states(dims, seed=7)
+    rng = np.random.default_rng(7)
+    st = oracle.LayerState(rng.standard_normal((2, 10, 16)), rng.standard_normal((2, 10, 16)),
+                           rng.standard_normal((2, 10, 16)))
+    lock = synth.bernoulli_active(2, 10, 0.3, seed=8)
+    idx, seg = oracle.compact(lock)
+    out = oracle.layer_step_partial(dims, W, X, idx, seg, st, "f64")
+    locked = lock.astype(bool)
+    for new, old in ((out.K, st.K), (out.V, st.V), (out.Y, st.Y)):
+        assert _h(new[locked]) == _h(old[locked])
+        assert np.all(np.any(new[~locked] != old[~locked], axis=-1))
+
+
+def test_attention_depends_on_locked_keys():
+    # continued attention: an active row's output changes when a locked row's cached K changes
+    dims = _dims(B=1, N=6, d=8, H=2, hd=4, F=8)
+    W = _weights(dims)
+    X = synth.hidden_states(dims, seed=9)
+    st = oracle.full_layer_step(dims, W, X, "f64")
+    lock = np.array([[1, 1, 0, 1, 1, 1]], np.uint8)
+    idx, seg = oracle.compact(lock)
+    a = oracle.layer_step_partial(dims, W, X, idx, seg, st, "f64")
+    st2 = st.copy()
+    st2.K[0, 4] += 1.0
+    b = oracle.layer_step_partial(dims, W, X, idx, seg, st2, "f64")
+    assert np.max(np.abs(a.Y[0, 2] - b.Y[0, 2])) > 1e-6
+
+
+# ---------------------------------------------------------------------------
+# the complexity closed form (SureLock Sec. 2 "Algorithmic Complexity")
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("B,N,d,H,hd,F,p", [(1, 16, 16, 2, 8, 24, 0.25), (3, 9, 12, 3, 4, 20, 0.5)])
+def test_flop_count_closed_form(B, N, d, H, hd, F, p):
+    dims = _dims(B=B, N=N, d=d, H=H, hd=hd, F=F)
+    W = _weights(dims)
+    X = synth.hidden_states(dims, seed=10)
+    with oracle.count_flops() as cf:
+        full = oracle.full_layer_step(dims, W, X, "f64")
+    assert cf.flops == B * (N * (8 * d * d + 6 * d * F) + 4 * N * N * d)
+    lock = synth.bernoulli_active(B, N, p, seed=10)
+    idx, seg = oracle.compact(lock)
+    M = idx.size
+    with oracle.count_flops() as cp:
+        oracle.layer_step_partial(dims, W, X, idx, seg, full, "f64")
+    assert cp.flops == M * (8 * d * d + 6 * d * F) + 4 * M * N * d
+    # the 8B-shape per-row figure
+    assert 8 * 4096 ** 2 + 6 * 4096 * 12288 + 4 * 1024 * 4096 == 452_984_832
+
+
+# ---------------------------------------------------------------------------
+# S1 proxy and scores
+# ---------------------------------------------------------------------------
+def test_proxy_identity_basis_and_score_cases():
+    rng = np.random.default_rng(11)
+    d, r = 20, 5
+    Ut = np.eye(d)[:r]
+    X = rng.standard_normal((2, 4, d))
+    s, p = oracle.score_drift(X, Ut, np.zeros((2, 4, r)), "l2")
+    np.testing.assert_array_equal(p, X[..., :r])
+    np.testing.assert_allclose(s, np.linalg.norm(X[..., :r], axis=-1), rtol=1e-15)
+    s2, _ = oracle.score_drift(X, Ut, X[..., :r], "l2")
+    np.testing.assert_array_equal(s2, 0.0)
+    s3, _ = oracle.score_drift(X, Ut, X[..., :r], "cos")
+    np.testing.assert_allclose(s3, 1.0, rtol=1e-15)
+    s4, _ = oracle.score_drift(X, Ut, -3.0 * X[..., :r], "cos")
+    np.testing.assert_allclose(s4, -1.0, rtol=1e-15)
+    s5, _ = oracle.score_drift(X, Ut, np.zeros((2, 4, r)), "cos")
+    np.testing.assert_array_equal(s5, 0.0)
+    # orthonormal basis: |U^T x| <= |x|, and cosine against scipy's distance
+    from scipy.spatial.distance import cosine as sp_cos
+    U = synth.proxy_basis(d, r, dtype="f32").astype(np.float64)
+    np.testing.assert_allclose(U @ U.T, np.eye(r), atol=1e-6)
+    _, pu = oracle.score_drift(X, U, np.zeros((2, 4, r)), "l2")
+    assert np.all(np.linalg.norm(pu, axis=-1) <= np.linalg.norm(X, axis=-1) * (1 + 1e-6))
+    pc = rng.standard_normal((2, 4, r))
+    sc, _ = oracle.score_drift(X, U, pc, "cos")
+    for b in range(2):
+        for n in range(4):
+            assert abs(sc[b, n] - (1.0 - sp_cos(pu[b, n], pc[b, n]))) < 1e-13
+
+
+# ---------------------------------------------------------------------------
+# S2/S3 integer semantics against numpy sorts
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("ties", [False, True])
+@pytest.mark.parametrize("largest", [True, False])
+def test_topk_against_lexsort(ties, largest):
+    rng = np.random.default_rng(12)
+    B, N = 3, 200
+    s = rng.integers(0, 5, (B, N)).astype(np.float64) if ties else rng.standard_normal((B, N))
+    lock = (rng.random((B, N)) < 0.3).astype(np.uint8)
+    for k in (0, 1, 17, 140, 500):
+        got = oracle.lock_topk(s, lock, k, largest)
+        for b in range(B):
+            cand = np.nonzero(lock[b] == 0)[0]
+            key = -s[b, cand] if largest else s[b, cand]
+            order = cand[np.lexsort((cand, key))]
+            keep = np.zeros(N, bool)
+            keep[order[:k]] = True
+            np.testing.assert_array_equal(got[b], (~keep).astype(np.uint8))
+
+
+def test_topk_nan_and_signed_zero():
+    s = np.array([[np.nan, 0.0, -0.0, 1.0, np.nan, -1.0]])
+    lock = np.zeros((1, 6), np.uint8)
+    np.testing.assert_array_equal(oracle.lock_topk(s, lock, 3, True)[0], [1, 0, 0, 0, 1, 1])
+    np.testing.assert_array_equal(oracle.lock_topk(s, lock, 2, False)[0], [1, 0, 1, 1, 1, 0])
+    np.testing.assert_array_equal(oracle.lock_topk(s, lock, 6, True)[0], [0] * 6)
+
+
+def test_threshold_monotone_and_strict():
+    s = np.array([[0.99, 0.990001, np.nan, 1.0, -2.0]])
+    lock = np.array([[0, 0, 0, 0, 1]], np.uint8)
+    np.testing.assert_array_equal(oracle.lock_threshold(s, lock, 0.99, True), [[0, 1, 0, 1, 1]])
+    np.testing.assert_array_equal(oracle.lock_threshold(s, lock, 0.99, False), [[0, 0, 0, 0, 1]])
+    rng = np.random.default_rng(13)
+    lk = np.zeros((2, 50), np.uint8)
+    for _ in range(10):
+        new = oracle.lock_threshold(rng.random((2, 50)), lk, 0.8, True)
+        assert np.all(new >= lk)
+        lk = new
+
+
+def test_compact_against_nonzero():
+    rng = np.random.default_rng(14)
+    lock = (rng.random((4, 33)) < 0.6).astype(np.uint8)
+    idx, seg = oracle.compact(lock)
+    np.testing.assert_array_equal(idx, np.nonzero(lock.reshape(-1) == 0)[0])
+    np.testing.assert_array_equal(seg, np.concatenate([[0], np.cumsum((lock == 0).sum(1))]))
+    idx0, seg0 = oracle.compact(np.ones((2, 5), np.uint8))
+    assert idx0.size == 0 and list(seg0) == [0, 0, 0]
+
+
+# ---------------------------------------------------------------------------
+# mutation tests: plant a plausible mistake in a copy of the oracle; a pin must fail
+# ---------------------------------------------------------------------------
+_FULL_MUTANTS = [
+    ("hres = x + _mm(a", "hres = _mm(a"),                                  # dropped residual
+    ("* scale          ", "* 1.0            "),                            # wrong softmax scale
+    ("q = _store(qkv[:, :d]", "q = _store(qkv[:, d:2 * d]"),              # q taken from K rows
+    ("_mm(a, _w(W, \"w_o\"))", "_mm(a, _w(W, \"w_o\").T)"),               # transposed operand
+    ("silu(gu[:, :F]) * gu[:, F:]", "silu(gu[:, F:]) * gu[:, :F]"),       # gate/up swapped
+    ("S = S - S.max(axis=1, keepdims=True)", "S = S - S.max(axis=0, keepdims=True)"),
+    ("P = P / P.sum(axis=1, keepdims=True)", "P = P / P.sum(axis=0, keepdims=True)"),
+    ("hn = _store(rmsnorm(hres, W[\"g2\"]", "hn = _store(rmsnorm(x, W[\"g2\"]"),
+]
+
+
+def _mutant(func, old, new):
+    src = textwrap.dedent(inspect.getsource(func))
+    assert old in src, old
+    ns = dict(po.__dict__)
+    exec(compile(src.replace(old, new, 1), "<mutant>", "exec"), ns)
+    return ns[func.__name__]
+
+
+@pytest.mark.parametrize("old,new", _FULL_MUTANTS)
+def test_full_step_mutants_are_caught(old, new):
+    dims = _dims(B=2, N=9, d=16, H=2, hd=8, F=24)
+    W = _weights(dims)
+    X = synth.hidden_states(dims, seed=15)
+    W = dict(W, g2=np.linspace(0.5, 1.5, 16))
+    mut = _mutant(po.full_layer_step, old, new)
+    st = mut(dims, W, X, "f64")
+    k, v, y = torch_block(dims, W, X)
+    assert max(np.max(np.abs(st.K - k)), np.max(np.abs(st.V - v)), np.max(np.abs(st.Y - y))) > 1e-6
+
+
+_PARTIAL_MUTANTS = [
+    ("hres = x[rows] + _mm(a", "hres = _mm(a"),
+    ("Kf[idx] = k", "Kf[idx] = v"),
+    ("Vf[idx] = v", "pass"),
+    ("s = s - s.max()", "s = s - s.min()"),  # harmless shift: must NOT be caught (control)
+    ("* scale     # [N]", "           # [N]"),
+    ("q[j:j + 1, cols]", "q[0:1, cols]"),
+    ("Kb = Kf[b * N:(b + 1) * N]", "Kb = Kf[0:N]"),
+    ("a[t, cols] = _mm(p[None, :], Vb[:, cols].T)[0]", "a[t, cols] = _mm(p[None, :], Kb[:, cols].T)[0]"),
+    ("out.Y.reshape(B * N, d)[idx[rows]] = y", "out.Y.reshape(B * N, d)[idx[rows]] = hres"),
+]
+
+
+@pytest.mark.parametrize("old,new", _PARTIAL_MUTANTS)
+def test_partial_step_mutants_are_caught(old, new):
+    dims = _dims(B=2, N=8, d=16, H=2, hd=8, F=24)
+    W = _weights(dims)
+    X = synth.hidden_states(dims, seed=16)
+    full = oracle.full_layer_step(dims, W, X, "f64")
+    lock = synth.bernoulli_active(2, 8, 0.5, seed=16)
+    idx, seg = oracle.compact(lock)
+    assert idx.size > 2 and seg[1] > 0 and seg[2] > seg[1]
+    mut = _mutant(po.layer_step_partial, old, new)
+    # pin 1: unchanged inputs -> active rows equal full recompute
+    part = mut(dims, W, X, idx, seg, full, "f64")
+    err = max(np.max(np.abs(part.K - full.K)), np.max(np.abs(part.V - full.V)),
+              np.max(np.abs(part.Y - full.Y)))
+    # pin 2: from stale caches, active rows get exactly the fresh K/V of full recompute
+    rng = np.random.default_rng(17)
+    stale = oracle.LayerState(*(rng.standard_normal(full.K.shape) for _ in range(3)))
+    part2 = mut(dims, W, X, idx, seg, stale, "f64")
+    act = lock == 0
+    err = max(err, np.max(np.abs(part2.K[act] - full.K[act])), np.max(np.abs(part2.V[act] - full.V[act])))
+    if old == "s = s - s.max()":
+        assert err < 1e-12  # subtracting any constant leaves softmax unchanged
+    else:
+        assert err > 1e-6
