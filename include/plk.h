@@ -1,0 +1,197 @@
+/*
+ * plk.h -- C ABI of the partial-recompute K/V library (B200, sm_100a).
+ *
+ * The library runs the partial-recompute denoising step of one bidirectional
+ * masked diffusion-LM layer on one GPU:
+ *
+ *   score_drift      S1   per-token drift on a low-rank singular proxy
+ *   select_active    S2-3 lock converged rows, compact the M active rows
+ *   layer_step_partial S4-10 RMSNorm -> QKV -> attention of the M active
+ *                    queries over all N keys -> O -> SwiGLU FFN on the M rows,
+ *                    fresh K/V and outputs scattered into the caches
+ *   full_layer_step  the same block for all N rows (the baseline sampler)
+ *   proxy_commit     S10  refresh the proxy cache of the recomputed rows
+ *
+ * Sources (web pages, cited by title and section):
+ *   [SL]  "Stopping Computation for Converged Tokens in Masked Diffusion-LM
+ *         Decoding" (SureLock), Sec. 2 Methodology: Locking Condition,
+ *         Permanent Deactivation, Continued Attention, Algorithmic Complexity.
+ *   [SPA] "SPA-Cache: Singular Proxies for Adaptive Caching in Diffusion
+ *         Language Models", part 1 (singular proxies), part 2 (adaptive budget).
+ *   [PS]  "Polestar: Drift-Aware Cache Calibration and Token Commitment for
+ *         Efficient Inference of Diffusion LLMs" (refresh the most-drifted rows).
+ *
+ * Conventions for every call:
+ *   - All pointers are DEVICE pointers unless stated otherwise; the caller owns
+ *     all memory.  No call allocates device memory.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream) and returns PLK_OK after enqueueing.
+ *     Argument and shape errors are detected on the host before any launch and
+ *     return a negative code with nothing enqueued.  PLK_ERR_CUDA reports a
+ *     failed launch.  A device-side wait that exceeded its limit is reported
+ *     later by plk_get_status().
+ *   - Tensors are dense row-major.  Token row (b, i) of a [B, N, ...] tensor is
+ *     flattened row b*N + i.
+ *   - dtype PLK_BF16: hidden states, weights, Ut, K/V/Y caches are bf16;
+ *     proxies and scores are fp32; accumulation is fp32.  dtype PLK_F32: all
+ *     of those are fp32 (fp32 arithmetic, no tensor cores).
+ *   - The active set is never copied to the host: M = seg_ptr[B] lives on the
+ *     device and every kernel reads it there.
+ */
+#ifndef PLK_H
+#define PLK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* return codes */
+#define PLK_OK             0
+#define PLK_ERR_ARG       -1  /* null pointer, bad enum, k/r out of range      */
+#define PLK_ERR_SHAPE     -2  /* shape this build does not support             */
+#define PLK_ERR_DTYPE     -3  /* unknown dtype                                 */
+#define PLK_ERR_CUDA      -4  /* a CUDA runtime/driver call failed             */
+#define PLK_ERR_TIMEOUT   -5  /* a device wait gave up (from plk_get_status)   */
+#define PLK_ERR_WORKSPACE -6  /* workspace missing or smaller than required    */
+
+/* dtypes */
+#define PLK_F32  0
+#define PLK_BF16 1
+
+/* drift metrics of plk_score_drift */
+#define PLK_METRIC_COS 0  /* cosine similarity: high = converged            */
+#define PLK_METRIC_L2  1  /* Euclidean distance: high = drifted             */
+
+/* selection modes of plk_select_active */
+#define PLK_SEL_THRESH_GT     0  /* lock when score >  tau (permanent)         */
+#define PLK_SEL_THRESH_LT     1  /* lock when score <  tau (permanent)         */
+#define PLK_SEL_TOPK_LARGEST  2  /* keep the k largest scores active           */
+#define PLK_SEL_TOPK_SMALLEST 3  /* keep the k smallest scores active          */
+
+/* Shape of one layer: B sequences of N tokens, model dim d = H*hd, FFN dim F.
+ * PLK_BF16 requires hd == 128, d % 128 == 0, F % 64 == 0.
+ * PLK_F32 requires hd in {16, 32, 64, 128}.  B*N < 2^31. */
+typedef struct {
+  int B, N, d, H, hd, F;
+  float eps;    /* RMSNorm epsilon                                      */
+  int dtype;    /* PLK_F32 or PLK_BF16                                   */
+} plk_dims;
+
+/* Layer weights, nn.Linear layout [out_features, in_features], row-major:
+ *   g1, g2   [d]       RMSNorm gains
+ *   w_qkv    [3d, d]   rows 0..d-1 -> Q, d..2d-1 -> K, 2d..3d-1 -> V;
+ *                      head h of Q/K/V is columns h*hd .. h*hd+hd-1
+ *   w_o      [d, d]
+ *   w_gu     [2F, d]   rows 0..F-1 gate, F..2F-1 up
+ *   w_down   [d, F]
+ * Gains and weights have the layer dtype. */
+typedef struct {
+  const void *g1, *w_qkv, *w_o, *g2, *w_gu, *w_down;
+} plk_weights;
+
+/*
+ * S1  Drift score on the singular proxy ([SPA] part 1; [PS] drift signal).
+ *   p_i = Ut x_i  for every row i of X [B, N, d]   (Ut [r, d]: r proxy
+ *   directions as rows, layer dtype), then
+ *   PLK_METRIC_COS: score_i = p_i . c_i / max(|p_i| |c_i|, 1e-30)
+ *   PLK_METRIC_L2:  score_i = |p_i - c_i|
+ *   with c_i = proxy_cache[i] ([B, N, r] fp32).
+ * Outputs: score_out [B, N] fp32; proxy_out [B, N] x r fp32 (may be NULL;
+ * receives p).  proxy_out must not alias proxy_cache.
+ * PLK_BF16 requires r % 16 == 0 and 16 <= r <= 256; PLK_F32 1 <= r <= 256.
+ */
+int plk_score_drift(const plk_dims* dims, const void* X, const void* Ut, int r,
+                    const float* proxy_cache, int metric, float* proxy_out,
+                    float* score_out, void* stream);
+
+/*
+ * S2 + S3  Lock update and compaction of the active set.
+ *   lock_in, lock_out [B, N] uint8 (1 = locked, 0 = active); may be the same
+ *   buffer.  score [B, N] fp32 (unused by no mode may be NULL).
+ *   PLK_SEL_THRESH_GT/LT ([SL] Sec. 2 "Locking Condition" and "Permanent
+ *     Deactivation"):  lock_out = lock_in | (score > tau)  [or < tau].  A NaN
+ *     score never locks; a locked row never unlocks.
+ *   PLK_SEL_TOPK_LARGEST/SMALLEST ([SPA] part 2 budget; [PS] most-drifted
+ *     refresh):  per sequence, among the rows with lock_in == 0, the k rows
+ *     with the largest (smallest) score stay active and every other row gets
+ *     lock_out = 1.  Equal scores go to the lower index; +0 == -0; NaN is never
+ *     preferred; with fewer than k candidates all of them stay active.
+ *   Compaction: idx_out [B*N] int32 receives the flattened indices b*N + i of
+ *   the active rows, ascending; seg_ptr [B+1] int32 receives the prefix counts
+ *   (seg_ptr[0] = 0, M = seg_ptr[B]).  Entries of idx_out past M are not
+ *   written.  Results are bit-exact and deterministic.
+ */
+int plk_select_active(const plk_dims* dims, const float* score, const uint8_t* lock_in,
+                      uint8_t* lock_out, int mode, float tau, int k,
+                      int32_t* idx_out, int32_t* seg_ptr, void* stream);
+
+/*
+ * S4..S10  One partial-recompute layer step ([SL] Sec. 2 "Permanent
+ * Deactivation", "Continued Attention", "Algorithmic Complexity").
+ *   X [B, N, d]: layer input hidden states.  idx / seg_ptr: the active rows
+ *   as written by plk_select_active (M = seg_ptr[B], read on the device).
+ *   For every active row j (token row t = idx[j] of sequence b):
+ *     xn = RMSNorm(x_t) * g1;   [q|k|v] = xn W_qkv^T
+ *     K_cache[t] = k, V_cache[t] = v          (before attention)
+ *     a  = per head softmax(q K_cache[b]^T / sqrt(hd)) V_cache[b], over all N
+ *          keys of sequence b (non-causal)
+ *     h  = x_t + a W_o^T;  hn = RMSNorm(h) * g2
+ *     Y[t] = h + (silu(hn W_g^T) * (hn W_u^T)) W_down^T
+ *   Rows not in idx are not read as queries and their K_cache, V_cache and Y
+ *   rows are never written.  K_cache, V_cache, Y: [B, N, d], in/out.
+ *   PLK_BF16 stores xn, q, k, v, a, hn and the SwiGLU product in bf16 (the
+ *   residual stream h stays fp32).  M = 0 is a no-op.
+ *   workspace: device buffer of at least plk_workspace_bytes(dims) bytes, any
+ *   content, 256-byte aligned; it must not be used by another call that runs
+ *   concurrently.
+ */
+int plk_layer_step_partial(const plk_dims* dims, const plk_weights* w, const void* X,
+                           const int32_t* idx, const int32_t* seg_ptr,
+                           void* K_cache, void* V_cache, void* Y,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * The baseline sampler ([SL] Sec. 1): the same block for all N rows of every
+ * sequence; writes every row of K_cache, V_cache and Y.  Same workspace rule.
+ */
+int plk_full_layer_step(const plk_dims* dims, const plk_weights* w, const void* X,
+                        void* K_cache, void* V_cache, void* Y,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * S10 (proxy half)  proxy_cache[idx[j]] = proxy_new[idx[j]] for j < M = seg_ptr[B].
+ * Both [B, N, r] fp32; rows not in idx are untouched.
+ */
+int plk_proxy_commit(const plk_dims* dims, int r, const int32_t* idx, const int32_t* seg_ptr,
+                     const float* proxy_new, float* proxy_cache, void* stream);
+
+/* Bytes of workspace plk_layer_step_partial / plk_full_layer_step need for these
+ * dims on the current device (0 for invalid dims). */
+size_t plk_workspace_bytes(const plk_dims* dims);
+
+/* Synchronises `stream`, returns the device status word of the current device
+ * (PLK_OK or PLK_ERR_TIMEOUT) and clears it. */
+int plk_get_status(void* stream);
+
+/* Upper bound, in SM clock cycles, of every device-side wait (default 4e9,
+ * about two seconds).  Values < 1 are rejected. */
+int plk_set_wait_limit(long long cycles);
+
+/* Launches one block that waits on a device flag nothing ever sets, bounded by
+ * the current wait limit; the wait then records PLK_ERR_TIMEOUT in the status
+ * word.  Exists to test the timeout path without faulting or hanging a GPU. */
+int plk_selftest_wait_timeout(void* stream);
+
+/* Static description of a return code. */
+const char* plk_error_string(int code);
+
+/* Library version, 100*major + minor. */
+int plk_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PLK_H */

@@ -1,0 +1,165 @@
+"""Python binding of the partial-recompute K/V library (libplk.so, sm_100a).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  Tensors are torch CUDA tensors (contiguous); calls are asynchronous on
+torch's current stream unless ``stream`` is given.  There is no CPU fallback:
+importing this module fails if the compiled library is missing.
+
+The C contract of every call is documented in include/plk.h.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libplk.so")
+
+OK, ERR_ARG, ERR_SHAPE, ERR_DTYPE, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = 0, -1, -2, -3, -4, -5, -6
+F32, BF16 = 0, 1
+METRIC_COS, METRIC_L2 = 0, 1
+SEL_THRESH_GT, SEL_THRESH_LT, SEL_TOPK_LARGEST, SEL_TOPK_SMALLEST = 0, 1, 2, 3
+
+EXPORTED = (
+    "plk_score_drift", "plk_select_active", "plk_layer_step_partial", "plk_full_layer_step",
+    "plk_proxy_commit", "plk_workspace_bytes", "plk_get_status", "plk_set_wait_limit",
+    "plk_selftest_wait_timeout", "plk_error_string", "plk_version",
+)
+
+
+class PlkDims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("N", ctypes.c_int), ("d", ctypes.c_int), ("H", ctypes.c_int),
+                ("hd", ctypes.c_int), ("F", ctypes.c_int), ("eps", ctypes.c_float), ("dtype", ctypes.c_int)]
+
+
+class PlkWeights(ctypes.Structure):
+    _fields_ = [("g1", ctypes.c_void_p), ("w_qkv", ctypes.c_void_p), ("w_o", ctypes.c_void_p),
+                ("g2", ctypes.c_void_p), ("w_gu", ctypes.c_void_p), ("w_down", ctypes.c_void_p)]
+
+
+class PlkError(RuntimeError):
+    def __init__(self, code, where):
+        super().__init__(f"{where}: {error_string(code)} ({code})")
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m partial_recompute_kv_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, S, F, L, V = (ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_float, ctypes.c_longlong,
+                        ctypes.POINTER(PlkDims))
+    W = ctypes.POINTER(PlkWeights)
+    sig = {
+        "plk_score_drift": (I, [V, P, P, I, P, I, P, P, P]),
+        "plk_select_active": (I, [V, P, P, P, I, F, I, P, P, P]),
+        "plk_layer_step_partial": (I, [V, W, P, P, P, P, P, P, P, S, P]),
+        "plk_full_layer_step": (I, [V, W, P, P, P, P, P, S, P]),
+        "plk_proxy_commit": (I, [V, I, P, P, P, P, P]),
+        "plk_workspace_bytes": (S, [V]),
+        "plk_get_status": (I, [P]),
+        "plk_set_wait_limit": (I, [L]),
+        "plk_selftest_wait_timeout": (I, [P]),
+        "plk_error_string": (ctypes.c_char_p, [I]),
+        "plk_version": (I, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def error_string(code: int) -> str:
+    return lib.plk_error_string(int(code)).decode()
+
+
+def version() -> int:
+    return lib.plk_version()
+
+
+def _check(code, where):
+    if code != OK:
+        raise PlkError(code, where)
+
+
+def dims(B, N, d, H, hd, F, eps=1e-6, dtype=BF16) -> PlkDims:
+    return PlkDims(int(B), int(N), int(d), int(H), int(hd), int(F), float(eps), int(dtype))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch tensor")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("tensors must be contiguous CUDA tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def weights(w: dict) -> PlkWeights:
+    return PlkWeights(*(_ptr(w[k]) for k in ("g1", "w_qkv", "w_o", "g2", "w_gu", "w_down")))
+
+
+def workspace_bytes(dm: PlkDims) -> int:
+    return int(lib.plk_workspace_bytes(ctypes.byref(dm)))
+
+
+def score_drift(dm, X, Ut, r, proxy_cache, metric, score_out, proxy_out=None, stream=None):
+    _check(lib.plk_score_drift(ctypes.byref(dm), _ptr(X), _ptr(Ut), int(r), _ptr(proxy_cache), int(metric),
+                               _ptr(proxy_out), _ptr(score_out), _stream(stream)), "score_drift")
+
+
+def select_active(dm, score, lock_in, lock_out, mode, tau, k, idx_out, seg_ptr, stream=None):
+    _check(lib.plk_select_active(ctypes.byref(dm), _ptr(score), _ptr(lock_in), _ptr(lock_out), int(mode),
+                                 float(tau), int(k), _ptr(idx_out), _ptr(seg_ptr), _stream(stream)),
+           "select_active")
+
+
+def layer_step_partial(dm, w, X, idx, seg_ptr, K_cache, V_cache, Y, workspace, stream=None):
+    pw = w if isinstance(w, PlkWeights) else weights(w)
+    _check(lib.plk_layer_step_partial(ctypes.byref(dm), ctypes.byref(pw), _ptr(X), _ptr(idx), _ptr(seg_ptr),
+                                      _ptr(K_cache), _ptr(V_cache), _ptr(Y), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(stream)),
+           "layer_step_partial")
+
+
+def full_layer_step(dm, w, X, K_cache, V_cache, Y, workspace, stream=None):
+    pw = w if isinstance(w, PlkWeights) else weights(w)
+    _check(lib.plk_full_layer_step(ctypes.byref(dm), ctypes.byref(pw), _ptr(X), _ptr(K_cache), _ptr(V_cache),
+                                   _ptr(Y), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                   _stream(stream)), "full_layer_step")
+
+
+def proxy_commit(dm, r, idx, seg_ptr, proxy_new, proxy_cache, stream=None):
+    _check(lib.plk_proxy_commit(ctypes.byref(dm), int(r), _ptr(idx), _ptr(seg_ptr), _ptr(proxy_new),
+                                _ptr(proxy_cache), _stream(stream)), "proxy_commit")
+
+
+def get_status(stream=None) -> int:
+    return int(lib.plk_get_status(_stream(stream)))
+
+
+def set_wait_limit(cycles: int):
+    _check(lib.plk_set_wait_limit(int(cycles)), "set_wait_limit")
+
+
+def selftest_wait_timeout(stream=None):
+    _check(lib.plk_selftest_wait_timeout(_stream(stream)), "selftest_wait_timeout")
+
+
+def alloc_workspace(dm, device="cuda"):
+    n = workspace_bytes(dm)
+    if n == 0:
+        raise PlkError(ERR_SHAPE, "workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)

@@ -1,0 +1,135 @@
+// extern "C" boundary of the partial-recompute library: argument validation on
+// the host, then asynchronous launches on the caller's stream.  Declarations and
+// the contract of every call are in include/plk.h.
+#include "plk_common.cuh"
+#include "plk_internal.h"
+
+namespace plk {
+
+static int check_dims(const plk_dims* d) {
+  if (!d) return PLK_ERR_ARG;
+  if (d->dtype != PLK_F32 && d->dtype != PLK_BF16) return PLK_ERR_DTYPE;
+  if (d->B < 1 || d->N < 1 || d->d < 1 || d->H < 1 || d->hd < 1 || d->F < 1) return PLK_ERR_SHAPE;
+  if ((long long)d->H * d->hd != d->d) return PLK_ERR_SHAPE;
+  if ((long long)d->B * d->N >= (1LL << 31)) return PLK_ERR_SHAPE;
+  if (!(d->eps >= 0.f)) return PLK_ERR_ARG;
+  if (d->dtype == PLK_BF16) {
+    if (d->hd != 128 || d->d % 128 != 0 || d->F % 64 != 0) return PLK_ERR_SHAPE;
+  } else {
+    if (d->hd != 16 && d->hd != 32 && d->hd != 64 && d->hd != 128) return PLK_ERR_SHAPE;
+  }
+  return PLK_OK;
+}
+
+}  // namespace plk
+
+using namespace plk;
+
+extern "C" {
+
+int plk_version(void) { return 100; }
+
+const char* plk_error_string(int code) {
+  switch (code) {
+    case PLK_OK: return "ok";
+    case PLK_ERR_ARG: return "invalid argument";
+    case PLK_ERR_SHAPE: return "unsupported shape";
+    case PLK_ERR_DTYPE: return "unknown dtype";
+    case PLK_ERR_CUDA: return "CUDA call failed";
+    case PLK_ERR_TIMEOUT: return "device wait exceeded its limit";
+    case PLK_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown error code";
+  }
+}
+
+size_t plk_workspace_bytes(const plk_dims* dims) {
+  if (check_dims(dims) != PLK_OK) return 0;
+  const int nsm = device_sm_count();
+  if (nsm <= 0) return 0;
+  return workspace_layout(dims, nsm).total;
+}
+
+int plk_score_drift(const plk_dims* dims, const void* X, const void* Ut, int r, const float* proxy_cache,
+                    int metric, float* proxy_out, float* score_out, void* stream) {
+  const int e = check_dims(dims);
+  if (e != PLK_OK) return e;
+  if (!X || !Ut || !proxy_cache || !score_out) return PLK_ERR_ARG;
+  if (metric != PLK_METRIC_COS && metric != PLK_METRIC_L2) return PLK_ERR_ARG;
+  if (proxy_out && proxy_out == proxy_cache) return PLK_ERR_ARG;
+  if (dims->dtype == PLK_BF16) {
+    if (r < 16 || r > 256 || r % 16 != 0 || dims->d % 64 != 0) return PLK_ERR_ARG;
+  } else {
+    if (r < 1 || r > 256) return PLK_ERR_ARG;
+  }
+  return launch_score(dims, X, Ut, r, proxy_cache, metric, proxy_out, score_out, (cudaStream_t)stream);
+}
+
+int plk_select_active(const plk_dims* dims, const float* score, const uint8_t* lock_in, uint8_t* lock_out,
+                      int mode, float tau, int k, int32_t* idx_out, int32_t* seg_ptr, void* stream) {
+  if (!dims) return PLK_ERR_ARG;
+  if (dims->B < 1 || dims->N < 1 || (long long)dims->B * dims->N >= (1LL << 31)) return PLK_ERR_SHAPE;
+  if (!score || !lock_in || !lock_out || !idx_out || !seg_ptr) return PLK_ERR_ARG;
+  if (mode < PLK_SEL_THRESH_GT || mode > PLK_SEL_TOPK_SMALLEST) return PLK_ERR_ARG;
+  if ((mode == PLK_SEL_TOPK_LARGEST || mode == PLK_SEL_TOPK_SMALLEST) && k < 0) return PLK_ERR_ARG;
+  return launch_select(dims, score, lock_in, lock_out, mode, tau, k, idx_out, seg_ptr, (cudaStream_t)stream);
+}
+
+int plk_layer_step_partial(const plk_dims* dims, const plk_weights* w, const void* X, const int32_t* idx,
+                           const int32_t* seg_ptr, void* K_cache, void* V_cache, void* Y, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  const int e = check_dims(dims);
+  if (e != PLK_OK) return e;
+  if (!w || !w->g1 || !w->w_qkv || !w->w_o || !w->g2 || !w->w_gu || !w->w_down) return PLK_ERR_ARG;
+  if (!X || !idx || !seg_ptr || !K_cache || !V_cache || !Y) return PLK_ERR_ARG;
+  return run_layer(dims, w, X, idx, seg_ptr, false, K_cache, V_cache, Y, workspace, ws_bytes,
+                   (cudaStream_t)stream);
+}
+
+int plk_full_layer_step(const plk_dims* dims, const plk_weights* w, const void* X, void* K_cache, void* V_cache,
+                        void* Y, void* workspace, size_t ws_bytes, void* stream) {
+  const int e = check_dims(dims);
+  if (e != PLK_OK) return e;
+  if (!w || !w->g1 || !w->w_qkv || !w->w_o || !w->g2 || !w->w_gu || !w->w_down) return PLK_ERR_ARG;
+  if (!X || !K_cache || !V_cache || !Y) return PLK_ERR_ARG;
+  return run_layer(dims, w, X, nullptr, nullptr, true, K_cache, V_cache, Y, workspace, ws_bytes,
+                   (cudaStream_t)stream);
+}
+
+int plk_proxy_commit(const plk_dims* dims, int r, const int32_t* idx, const int32_t* seg_ptr,
+                     const float* proxy_new, float* proxy_cache, void* stream) {
+  if (!dims) return PLK_ERR_ARG;
+  if (dims->B < 1 || dims->N < 1) return PLK_ERR_SHAPE;
+  if (r < 1 || r > 256 || !idx || !seg_ptr || !proxy_new || !proxy_cache) return PLK_ERR_ARG;
+  return launch_proxy_commit(dims, r, idx, seg_ptr, proxy_new, proxy_cache, (cudaStream_t)stream);
+}
+
+int plk_get_status(void* stream) {
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return PLK_ERR_CUDA;
+  int v = PLK_OK;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return PLK_ERR_CUDA;
+  const int zero = PLK_OK;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return PLK_ERR_CUDA;
+  return v;
+}
+
+int plk_set_wait_limit(long long cycles) {
+  if (cycles < 1) return PLK_ERR_ARG;
+  return cudaMemcpyToSymbol(g_wait_limit, &cycles, sizeof(cycles)) == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;
+}
+
+}  // extern "C"
+
+namespace plk {
+__device__ uint32_t g_never_set = 0u;
+
+// One thread spins on a flag nothing writes; the bounded spin records
+// PLK_ERR_TIMEOUT and returns.
+__global__ void selftest_wait_kernel() {
+  if (threadIdx.x == 0) (void)spin_until_geq(&g_never_set, 1u);
+}
+}  // namespace plk
+
+extern "C" int plk_selftest_wait_timeout(void* stream) {
+  plk::selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>();
+  return cudaPeekAtLastError() == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;
+}

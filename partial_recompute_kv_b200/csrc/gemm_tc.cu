@@ -1,0 +1,369 @@
+// Persistent tcgen05 GEMM for the projections of the partial-recompute layer
+// step: out[token, f] = sum_k X[token, k] * W[f, k] on the M active rows only
+// (the SureLock page, "Stopping Computation for Converged Tokens in Masked
+// Diffusion-LM Decoding", Sec. 2: Q/K/V, output projection and FFN run for the
+// active subset, cost O(M d^2)).
+//
+// Design (sm_100a):
+//  * Weights are the UMMA A operand (M = 128 feature rows per tile) and the
+//    compacted activations the B operand (N = 64..256 tokens, chosen on the
+//    device from M = seg_ptr[B]); at M <= 256 every weight byte is read from HBM
+//    exactly once.  Both operands are K-major bf16 tiles loaded by TMA with a
+//    128-byte swizzle; accumulation is fp32 in TMEM (two 256-column buffers so
+//    the epilogue of one tile overlaps the main loop of the next).
+//  * Warp roles: warp 0 issues TMA, one thread of warp 1 issues tcgen05.mma,
+//    warps 2-5 drain TMEM (tcgen05.ld) and run the fused epilogue.
+//  * Stream-K: the (tile, k-block) iteration space is cut into gridDim.x equal
+//    contiguous ranges, one per CTA (one CTA per SM).  A tile whose k-range is
+//    split is finished by the CTA owning its k = 0 segment: the other CTAs
+//    (whose range starts inside the tile, so they reach it first) store fp32
+//    partials and release a flag; the owner waits for them (bounded), adds them
+//    to its accumulator and runs the epilogue.  Every output element is written
+//    once by a fused epilogue, no output buffer needs zeroing.
+//  * Epilogues: QKV (Q compact; K and V scattered straight into the cache rows,
+//    the K/V refresh of SureLock Sec. 2), O (+ residual, fp32 h), GU (tile =
+//    64 gate rows + 64 up rows of the same features; silu(g) * u), DOWN
+//    (+ fp32 residual, scattered into the output cache rows).
+#include "plk_common.cuh"
+#include "plk_internal.h"
+
+namespace plk {
+
+namespace {
+
+constexpr int kStageA = kGemmBM * kGemmBK * 2;     // 16 KB
+constexpr int kStageB = kGemmBNMax * kGemmBK * 2;  // 32 KB
+constexpr int kTileCols = 256;                     // TMEM columns per accumulator buffer
+constexpr int kSlotFloats = kGemmBNMax * kGemmBM;  // partial tile, [col][lane]
+constexpr int kXbufStride = 33;
+constexpr size_t kOffB = (size_t)kGemmStages * kStageA;
+constexpr size_t kOffBar = kOffB + (size_t)kGemmStages * kStageB;
+constexpr size_t kOffIdx = kOffBar + 128;
+constexpr size_t kOffXbuf = kOffIdx + kGemmBNMax * 4;
+constexpr size_t kSmemUsed = kOffXbuf + 64 * kXbufStride * 4;
+constexpr size_t kSmemBytes = kSmemUsed + 1024;  // slack for 1024-byte alignment
+
+struct Sched {
+  int M, ttiles, kblocks, total, L, begin, end;
+};
+
+__device__ __forceinline__ void sched_init(Sched& s, const GemmArgs& a) {
+  s.M = a.seg_ptr[a.B];
+  s.ttiles = ceil_div(s.M, kGemmBNMax);
+  s.kblocks = a.K / kGemmBK;
+  s.total = a.ftiles * s.ttiles * s.kblocks;
+  s.L = ceil_div(s.total, (int)gridDim.x);
+  s.begin = min((int)blockIdx.x * s.L, s.total);
+  s.end = min(s.begin + s.L, s.total);
+}
+
+struct Seg {
+  int t, k0, k1, ft, tok0, ntok, ncols;
+};
+
+__device__ __forceinline__ void seg_decode(Seg& g, const Sched& s, int it) {
+  g.t = it / s.kblocks;
+  g.k0 = it - g.t * s.kblocks;
+  g.k1 = min(s.kblocks, g.k0 + (s.end - it));
+  g.ft = g.t / s.ttiles;
+  const int tt = g.t - g.ft * s.ttiles;
+  g.tok0 = tt * kGemmBNMax;
+  g.ntok = min(kGemmBNMax, s.M - g.tok0);
+  g.ncols = (g.ntok + 63) & ~63;
+}
+
+// bounded mbarrier wait that also gives up as soon as another role aborted
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* s_abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  const long long lim = g_wait_limit;
+  while (!mbar_try_wait(bar, parity)) {
+    if (*s_abort) return false;
+    if (clock64() - t0 > lim) {
+      report_timeout();
+      *s_abort = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+
+}  // namespace
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                   const GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kOffB;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint64_t* full = bars;                  // [4] TMA -> MMA
+  uint64_t* empty = bars + 4;             // [4] MMA -> TMA
+  uint64_t* tfull = bars + 8;             // [2] MMA -> epilogue
+  uint64_t* tempty = bars + 10;           // [2] epilogue -> MMA
+  uint64_t* drain = bars + 12;            // MMA drain before TMEM release
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 13);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 14);
+  volatile int* s_epi_abort = reinterpret_cast<volatile int*>(bars + 15);
+  int* s_idx = reinterpret_cast<int*>(smem + kOffIdx);
+  float* xbuf = reinterpret_cast<float*>(smem + kOffXbuf);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  Sched s;
+  sched_init(s, args);
+  if (s.M <= 0 || s.begin >= s.end) return;  // uniform over the CTA; nobody waits on an empty range
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kGemmStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 128);
+    }
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    *s_epi_abort = 0;
+    fence_mbar_init();
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_parity[kGemmStages];
+      bool issued[kGemmStages];
+      for (int i = 0; i < kGemmStages; ++i) issued[i] = false;
+      Seg g;
+      for (int it = s.begin; it < s.end && !*s_abort; it += g.k1 - g.k0) {
+        seg_decode(g, s, it);
+        const int nbox = g.ncols >> 6;
+        const uint32_t bytes = kStageA + nbox * (64 * kGemmBK * 2);
+        const int yA0 = (args.epi == EPI_GU) ? g.ft * 64 : g.ft * kGemmBM;
+        const int yA1 = (args.epi == EPI_GU) ? args.gu_F + g.ft * 64 : g.ft * kGemmBM + 64;
+        for (int kb = g.k0; kb < g.k1; ++kb) {
+          if (!wait_or_abort(&empty[stage], phase ^ 1, s_abort)) break;
+          mbar_expect_tx(&full[stage], bytes);
+          uint8_t* a = sA + stage * kStageA;
+          uint8_t* b = sB + stage * kStageB;
+          const int x = kb * kGemmBK;
+          tma_load_2d(a, &tmW, x, yA0, &full[stage]);
+          tma_load_2d(a + 8192, &tmW, x, yA1, &full[stage]);
+          for (int j = 0; j < nbox; ++j) tma_load_2d(b + j * 8192, &tmX, x, g.tok0 + j * 64, &full[stage]);
+          issued[stage] = true;
+          issued_parity[stage] = phase;
+          if (++stage == kGemmStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (*s_abort) {
+        // let every copy this thread started land before the CTA exits
+        for (int i = 0; i < kGemmStages; ++i)
+          if (issued[i]) (void)mbar_wait(&full[i], issued_parity[i]);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, accph = 0;
+      Seg g;
+      for (int it = s.begin; it < s.end && !*s_abort; it += g.k1 - g.k0) {
+        seg_decode(g, s, it);
+        if (!wait_or_abort(&tempty[acc], accph ^ 1, s_abort)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * kTileCols);
+        const uint32_t idesc = idesc_bf16(kGemmBM, g.ncols);
+        bool ok = true;
+        for (int kb = g.k0; kb < g.k1; ++kb) {
+          if (!wait_or_abort(&full[stage], phase, s_abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = sdesc_sw128(smem_u32(sA + stage * kStageA));
+          const uint64_t bdesc = sdesc_sw128(smem_u32(sB + stage * kStageB));
+#pragma unroll
+          for (int k = 0; k < kGemmBK / 16; ++k) {
+            // +32 bytes of K per step, in 16-byte units of the descriptor address field
+            umma_bf16(d_tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > g.k0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == kGemmStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        acc ^= 1;
+        if (acc == 0) accph ^= 1;
+      }
+      // no MMA may still be running when TMEM is released
+      umma_commit(drain);
+      (void)mbar_wait(drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;           // TMEM lane quarter this warp may access
+    const int lr = q * 32 + lane;     // tile row = TMEM lane = feature row in tile
+    const int et = threadIdx.x - 64;  // 0..127
+    const int d = args.d;
+    int acc = 0;
+    uint32_t accph = 0;
+    Seg g;
+    for (int it = s.begin; it < s.end; it += g.k1 - g.k0) {
+      seg_decode(g, s, it);
+      const bool is_head = g.k0 == 0;
+      const bool is_full = is_head && g.k1 == s.kblocks;
+      named_bar_sync(1, 128);
+      for (int j = et; j < g.ntok; j += 128) s_idx[j] = args.idx[g.tok0 + j];
+      // The break decision must be the same in all four epilogue warps, so it is
+      // taken from a flag that is only written before this barrier.
+      bool bad = !wait_or_abort(&tfull[acc], accph, s_abort);
+      int c_last = (int)blockIdx.x;
+      if (is_head && !is_full) {
+        c_last = ((g.t + 1) * s.kblocks - 1) / s.L;
+        if (!bad) bad = !spin_until_geq(&args.flags[g.t], (uint32_t)(c_last - (int)blockIdx.x));
+      }
+      if (bad) {
+        *s_epi_abort = 1;
+        *s_abort = 1;
+      }
+      named_bar_sync(1, 128);
+      if (*s_epi_abort) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (uint32_t)(acc * kTileCols) + ((uint32_t)(q * 32) << 16);
+      const int nchunks = g.ncols >> 5;
+      for (int c = 0; c < nchunks; ++c) {
+        uint32_t r[32];
+        tmem_ld32(taddr + (uint32_t)(c * 32), r);
+        tmem_ld_wait();
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+        if (!is_head) {
+          float* slot = args.partials + (size_t)blockIdx.x * kSlotFloats;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) slot[(c * 32 + i) * kGemmBM + lr] = v[i];
+          continue;
+        }
+        if (!is_full) {
+          for (int sl = (int)blockIdx.x + 1; sl <= c_last; ++sl) {
+            const float* slot = args.partials + (size_t)sl * kSlotFloats;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] += __ldcg(&slot[(c * 32 + i) * kGemmBM + lr]);
+          }
+        }
+        const int jb = c * 32;
+        if (args.epi == EPI_QKV) {
+          const int f = g.ft * kGemmBM + lr;
+          const int part = f / d, col = f - part * d;
+          __nv_bfloat16* dst = part == 0 ? (__nv_bfloat16*)args.q_out
+                                         : (part == 1 ? (__nv_bfloat16*)args.k_cache : (__nv_bfloat16*)args.v_cache);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (jb + i < g.ntok) {
+              const size_t row = part == 0 ? (size_t)(g.tok0 + jb + i) : (size_t)s_idx[jb + i];
+              dst[row * d + col] = f2bf(v[i]);
+            }
+          }
+        } else if (args.epi == EPI_O) {
+          const int f = g.ft * kGemmBM + lr;
+          const __nv_bfloat16* x = (const __nv_bfloat16*)args.x_in;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (jb + i < g.ntok) {
+              const size_t tok = (size_t)(g.tok0 + jb + i);
+              args.h32[tok * d + f] = v[i] + bf2f(x[(size_t)s_idx[jb + i] * d + f]);
+            }
+          }
+        } else if (args.epi == EPI_GU) {
+          if (q >= 2) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) xbuf[(lr - 64) * kXbufStride + i] = v[i];
+          }
+          named_bar_sync(2, 128);
+          if (q < 2) {
+            const int F = args.gu_F;
+            const int f = g.ft * 64 + lr;
+            __nv_bfloat16* out = (__nv_bfloat16*)args.act_out;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              if (jb + i < g.ntok) {
+                const float u = xbuf[lr * kXbufStride + i];
+                out[(size_t)(g.tok0 + jb + i) * F + f] = f2bf(silu_f(v[i]) * u);
+              }
+            }
+          }
+          named_bar_sync(2, 128);
+        } else {  // EPI_DOWN
+          const int f = g.ft * kGemmBM + lr;
+          __nv_bfloat16* y = (__nv_bfloat16*)args.y_cache;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (jb + i < g.ntok) {
+              const size_t tok = (size_t)(g.tok0 + jb + i);
+              y[(size_t)s_idx[jb + i] * d + f] = f2bf(args.h32[tok * d + f] + v[i]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+      if (!is_head) {
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (et == 0) red_release_add_u32(&args.flags[g.t], 1u);
+      } else if (!is_full) {
+        named_bar_sync(1, 128);
+        if (et == 0) args.flags[g.t] = 0u;  // ready for the next GEMM of the step
+      }
+      acc ^= 1;
+      if (acc == 0) accph ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& a, cudaStream_t st) {
+  static int attr_done[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PLK_ERR_CUDA;
+  if (dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
+        cudaSuccess)
+      return PLK_ERR_CUDA;
+    attr_done[dev] = 1;
+  }
+  gemm_tc_kernel<<<a.nslots, kGemmThreads, kSmemBytes, st>>>(tmW, tmX, a);
+  return cudaPeekAtLastError() == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;
+}
+
+}  // namespace plk

@@ -1,0 +1,356 @@
+// S4..S10: one partial-recompute layer step on the M active rows (the SureLock
+// page, "Stopping Computation for Converged Tokens in Masked Diffusion-LM
+// Decoding", Sec. 2 "Permanent Deactivation", "Continued Attention",
+// "Algorithmic Complexity"), and the full-recompute baseline (Sec. 1).
+//
+// bf16 chain (7 launches, M read on the device, no host synchronisation):
+//   1 gather rows idx[j] of X, RMSNorm1 -> xn (bf16); clear the GEMM fix-up flags
+//   2 tcgen05 GEMM  xn W_qkv^T -> Q (compact), K and V scattered into the caches
+//   3 attention of the M queries over all N cached keys -> a (bf16)
+//   4 tcgen05 GEMM  a W_o^T + x -> h (fp32)
+//   5 RMSNorm2(h) -> hn (bf16)
+//   6 tcgen05 GEMM  hn [W_g; W_u]^T -> silu(g) * u (bf16)
+//   7 tcgen05 GEMM  act W_down^T + h -> Y rows idx[j] (bf16)
+// fp32 chain: the same steps with SIMT GEMMs into an fp32 scratch and
+// elementwise epilogue kernels.
+#include <math.h>
+
+#include <algorithm>
+
+#include "plk_common.cuh"
+#include "plk_internal.h"
+
+namespace plk {
+
+// ---------------------------------------------------------------------------
+// host helpers
+// ---------------------------------------------------------------------------
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+Workspace workspace_layout(const plk_dims* dm, int num_sms) {
+  Workspace w;
+  const size_t Mcap = (size_t)dm->B * dm->N, d = dm->d, F = dm->F;
+  const size_t es = dm->dtype == PLK_BF16 ? 2 : 4;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 1024);
+    return o;
+  };
+  w.iota = take(4 * Mcap);
+  w.seg = take(4 * ((size_t)dm->B + 1));
+  w.xn = take(es * Mcap * d);
+  w.q = take(es * Mcap * d);
+  w.a = take(es * Mcap * d);
+  w.h32 = take(4 * Mcap * d);
+  w.hn = take(es * Mcap * d);
+  w.act = take(es * Mcap * F);
+  if (dm->dtype == PLK_BF16) {
+    const size_t ttiles = (Mcap + kGemmBNMax - 1) / kGemmBNMax;
+    const size_t ft = std::max((size_t)3 * d / kGemmBM, F / 64);
+    w.nslots = num_sms;
+    w.nflags = (int)(ft * ttiles);
+    w.partials = take((size_t)num_sms * kGemmBNMax * kGemmBM * 4);
+    w.flags = take(4 * (size_t)w.nflags);
+  } else {
+    w.c32 = take(4 * Mcap * std::max((size_t)3 * d, 2 * F));
+  }
+  w.total = off;
+  return w;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+int make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return PLK_ERR_CUDA;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PLK_OK : PLK_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// elementwise kernels
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float block_sum_f(float v, float* sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) sh[warp] = v;
+  __syncthreads();
+  float t = (threadIdx.x < nw) ? sh[threadIdx.x] : 0.f;
+  if (warp == 0) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (lane == 0) sh[32] = t;
+  }
+  __syncthreads();
+  return sh[32];
+}
+
+// out[j] = RMSNorm(src_row(j)) * g for j < M.  src_row(j) = X[idx[j]] (gather)
+// or H[j] (idx == nullptr).  Block 0 also clears the GEMM fix-up flags.
+template <typename Tin, typename Tg, typename Tout>
+__global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const Tin* __restrict__ X, const int32_t* __restrict__ idx,
+                                                           const int32_t* __restrict__ seg_ptr, int B,
+                                                           const Tg* __restrict__ g, float eps, int d,
+                                                           Tout* __restrict__ out, uint32_t* flags, int nflags) {
+  __shared__ float sh[33];
+  if (flags && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < nflags; i += blockDim.x) flags[i] = 0u;
+  const int M = seg_ptr[B];
+  const int j = blockIdx.x;
+  if (j >= M) return;
+  const size_t row = idx ? (size_t)idx[j] : (size_t)j;
+  const Tin* x = X + row * d;
+  float ss = 0.f;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    const float v = to_f(x[c]);
+    ss = fmaf(v, v, ss);
+  }
+  ss = block_sum_f(ss, sh);
+  const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+  Tout* o = out + (size_t)j * d;
+  for (int c = threadIdx.x; c < d; c += blockDim.x) o[c] = from_f<Tout>(to_f(x[c]) * inv * to_f(g[c]));
+}
+
+__global__ void fill_identity_kernel(int32_t* iota, int32_t* seg, int B, int N) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < B * N) iota[i] = i;
+  if (i <= B) seg[i] = i * N;
+}
+
+// ---- fp32 path --------------------------------------------------------------
+// C[j, n] = sum_k A[j, k] W[n, k] for j < M (SIMT, 64x64 tiles)
+__global__ void __launch_bounds__(256) gemm_f32_kernel(const float* __restrict__ A, const float* __restrict__ W,
+                                                       float* __restrict__ C, int Nout, int K,
+                                                       const int32_t* __restrict__ seg_ptr, int B) {
+  __shared__ float As[16][65], Ws[16][65];
+  const int M = seg_ptr[B];
+  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
+  if (m0 >= M) return;
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    for (int e = threadIdx.x; e < 64 * 16; e += 256) {
+      const int r = e >> 4, kk = e & 15;
+      As[kk][r] = (m0 + r < M && k0 + kk < K) ? A[(size_t)(m0 + r) * K + k0 + kk] : 0.f;
+      Ws[kk][r] = (n0 + r < Nout && k0 + kk < K) ? W[(size_t)(n0 + r) * K + k0 + kk] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < 16; ++kk)
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) acc[i][jj] = fmaf(As[kk][ty * 4 + i], Ws[kk][tx * 4 + jj], acc[i][jj]);
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int m = m0 + ty * 4 + i, n = n0 + tx * 4 + jj;
+      if (m < M && n < Nout) C[(size_t)m * Nout + n] = acc[i][jj];
+    }
+}
+
+enum F32Epi { F32_QKV = 0, F32_O = 1, F32_GU = 2, F32_DOWN = 3 };
+
+// Epilogues of the fp32 chain, one CTA per active row j.
+__global__ void __launch_bounds__(256) epilogue_f32_kernel(int mode, const float* __restrict__ C,
+                                                           const int32_t* __restrict__ idx,
+                                                           const int32_t* __restrict__ seg_ptr, int B, int d, int F,
+                                                           float* q, float* kc, float* vc, const float* x, float* h32,
+                                                           float* act, float* y) {
+  const int M = seg_ptr[B];
+  const int j = blockIdx.x;
+  if (j >= M) return;
+  const size_t row = (size_t)idx[j];
+  if (mode == F32_QKV) {
+    const float* c = C + (size_t)j * 3 * d;
+    for (int t = threadIdx.x; t < d; t += blockDim.x) {
+      q[(size_t)j * d + t] = c[t];
+      kc[row * d + t] = c[d + t];
+      vc[row * d + t] = c[2 * d + t];
+    }
+  } else if (mode == F32_O) {
+    for (int t = threadIdx.x; t < d; t += blockDim.x)
+      h32[(size_t)j * d + t] = x[row * d + t] + C[(size_t)j * d + t];
+  } else if (mode == F32_GU) {
+    const float* c = C + (size_t)j * 2 * F;
+    for (int t = threadIdx.x; t < F; t += blockDim.x) {
+      const float gg = c[t];
+      act[(size_t)j * F + t] = gg / (1.0f + expf(-gg)) * c[F + t];
+    }
+  } else {
+    for (int t = threadIdx.x; t < d; t += blockDim.x)
+      y[row * d + t] = h32[(size_t)j * d + t] + C[(size_t)j * d + t];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// orchestration
+// ---------------------------------------------------------------------------
+#define PLK_TRY(x)                  \
+  do {                              \
+    const int _r = (x);             \
+    if (_r != PLK_OK) return _r;    \
+  } while (0)
+#define PLK_LAUNCHED() \
+  do { if (cudaPeekAtLastError() != cudaSuccess) return PLK_ERR_CUDA; } while (0)
+
+static int run_layer_f32(const plk_dims* dm, const plk_weights* w, const float* X, const int32_t* idx,
+                         const int32_t* seg, float* Kc, float* Vc, float* Y, uint8_t* ws, const Workspace& L,
+                         cudaStream_t st) {
+  const int B = dm->B, d = dm->d, F = dm->F, Mcap = dm->B * dm->N;
+  float* xn = (float*)(ws + L.xn);
+  float* q = (float*)(ws + L.q);
+  float* a = (float*)(ws + L.a);
+  float* h32 = (float*)(ws + L.h32);
+  float* hn = (float*)(ws + L.hn);
+  float* act = (float*)(ws + L.act);
+  float* c32 = (float*)(ws + L.c32);
+  const dim3 rows(Mcap);
+  auto gemm = [&](const float* A, const void* Wt, int Nout, int K) {
+    dim3 grid(ceil_div(Nout, 64), ceil_div(Mcap, 64));
+    gemm_f32_kernel<<<grid, 256, 0, st>>>(A, (const float*)Wt, c32, Nout, K, seg, B);
+  };
+  rmsnorm_rows_kernel<float, float, float><<<rows, 256, 0, st>>>(X, idx, seg, B, (const float*)w->g1, dm->eps, d, xn,
+                                                          nullptr, 0);
+  gemm(xn, w->w_qkv, 3 * d, d);
+  epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_QKV, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y);
+  PLK_LAUNCHED();
+  PLK_TRY(launch_attention_f32(dm, q, Kc, Vc, a, seg, Mcap, st));
+  gemm(a, w->w_o, d, d);
+  epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_O, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y);
+  rmsnorm_rows_kernel<float, float, float><<<rows, 256, 0, st>>>(h32, nullptr, seg, B, (const float*)w->g2, dm->eps, d,
+                                                          hn, nullptr, 0);
+  gemm(hn, w->w_gu, 2 * F, d);
+  epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_GU, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y);
+  gemm(act, w->w_down, d, F);
+  epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_DOWN, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y);
+  PLK_LAUNCHED();
+  return PLK_OK;
+}
+
+static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_bfloat16* X, const int32_t* idx,
+                          const int32_t* seg, void* Kc, void* Vc, void* Y, uint8_t* ws, const Workspace& L,
+                          cudaStream_t st) {
+  const int B = dm->B, d = dm->d, F = dm->F, Mcap = dm->B * dm->N;
+  __nv_bfloat16* xn = (__nv_bfloat16*)(ws + L.xn);
+  __nv_bfloat16* q = (__nv_bfloat16*)(ws + L.q);
+  __nv_bfloat16* a = (__nv_bfloat16*)(ws + L.a);
+  float* h32 = (float*)(ws + L.h32);
+  __nv_bfloat16* hn = (__nv_bfloat16*)(ws + L.hn);
+  __nv_bfloat16* act = (__nv_bfloat16*)(ws + L.act);
+  uint32_t* flags = (uint32_t*)(ws + L.flags);
+
+  CUtensorMap tW_qkv, tW_o, tW_gu, tW_down, tX_xn, tX_a, tX_hn, tX_act;
+  PLK_TRY(make_tmap_bf16(&tW_qkv, w->w_qkv, 3ull * d, d, 64));
+  PLK_TRY(make_tmap_bf16(&tW_o, w->w_o, (uint64_t)d, d, 64));
+  PLK_TRY(make_tmap_bf16(&tW_gu, w->w_gu, 2ull * F, d, 64));
+  PLK_TRY(make_tmap_bf16(&tW_down, w->w_down, (uint64_t)d, F, 64));
+  PLK_TRY(make_tmap_bf16(&tX_xn, xn, (uint64_t)Mcap, d, 64));
+  PLK_TRY(make_tmap_bf16(&tX_a, a, (uint64_t)Mcap, d, 64));
+  PLK_TRY(make_tmap_bf16(&tX_hn, hn, (uint64_t)Mcap, d, 64));
+  PLK_TRY(make_tmap_bf16(&tX_act, act, (uint64_t)Mcap, F, 64));
+
+  GemmArgs g{};
+  g.d = d;
+  g.Mcap = Mcap;
+  g.seg_ptr = seg;
+  g.B = B;
+  g.idx = idx;
+  g.partials = (float*)(ws + L.partials);
+  g.flags = flags;
+  g.nslots = L.nslots;
+
+  rmsnorm_rows_kernel<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16><<<Mcap, 256, 0, st>>>(
+      X, idx, seg, B, (const __nv_bfloat16*)w->g1, dm->eps, d, xn, flags, L.nflags);
+  PLK_LAUNCHED();
+
+  g.epi = EPI_QKV;
+  g.K = d;
+  g.ftiles = 3 * d / kGemmBM;
+  g.q_out = q;
+  g.k_cache = Kc;
+  g.v_cache = Vc;
+  PLK_TRY(launch_gemm_tc(tW_qkv, tX_xn, g, st));
+
+  PLK_TRY(launch_attention_bf16(dm, q, Kc, Vc, a, seg, st));
+
+  g.epi = EPI_O;
+  g.K = d;
+  g.ftiles = d / kGemmBM;
+  g.x_in = X;
+  g.h32 = h32;
+  PLK_TRY(launch_gemm_tc(tW_o, tX_a, g, st));
+
+  rmsnorm_rows_kernel<float, __nv_bfloat16, __nv_bfloat16><<<Mcap, 256, 0, st>>>(
+      h32, nullptr, seg, B, (const __nv_bfloat16*)w->g2, dm->eps, d, hn, nullptr, 0);
+  PLK_LAUNCHED();
+
+  g.epi = EPI_GU;
+  g.K = d;
+  g.ftiles = F / 64;
+  g.gu_F = F;
+  g.act_out = act;
+  PLK_TRY(launch_gemm_tc(tW_gu, tX_hn, g, st));
+
+  g.epi = EPI_DOWN;
+  g.K = F;
+  g.ftiles = d / kGemmBM;
+  g.y_cache = Y;
+  PLK_TRY(launch_gemm_tc(tW_down, tX_act, g, st));
+  return PLK_OK;
+}
+
+int run_layer(const plk_dims* dm, const plk_weights* w, const void* X, const int32_t* idx, const int32_t* seg_ptr,
+              bool full, void* Kc, void* Vc, void* Y, void* ws, size_t ws_bytes, cudaStream_t st) {
+  const int nsm = device_sm_count();
+  if (nsm <= 0) return PLK_ERR_CUDA;
+  const Workspace L = workspace_layout(dm, nsm);
+  if (!ws || ws_bytes < L.total) return PLK_ERR_WORKSPACE;
+  uint8_t* wsb = (uint8_t*)ws;
+  if (full) {
+    int32_t* iota = (int32_t*)(wsb + L.iota);
+    int32_t* seg = (int32_t*)(wsb + L.seg);
+    const int n = dm->B * dm->N + 1;
+    fill_identity_kernel<<<ceil_div(n, 256), 256, 0, st>>>(iota, seg, dm->B, dm->N);
+    PLK_LAUNCHED();
+    idx = iota;
+    seg_ptr = seg;
+  }
+  if (dm->dtype == PLK_F32)
+    return run_layer_f32(dm, w, (const float*)X, idx, seg_ptr, (float*)Kc, (float*)Vc, (float*)Y, wsb, L, st);
+  return run_layer_bf16(dm, w, (const __nv_bfloat16*)X, idx, seg_ptr, Kc, Vc, Y, wsb, L, st);
+}
+
+}  // namespace plk

@@ -1,0 +1,84 @@
+// Host-side internals of the partial-recompute library: launch functions of
+// each kernel family, the workspace layout and TMA descriptor helpers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/plk.h"
+
+namespace plk {
+
+// ---- tile constants of the tcgen05 GEMM ------------------------------------
+constexpr int kGemmBM = 128;      // feature rows per tile (UMMA M)
+constexpr int kGemmBNMax = 256;   // tokens per tile (UMMA N, runtime 64..256)
+constexpr int kGemmBK = 64;       // K per stage: one 128-byte swizzle row of bf16
+constexpr int kGemmStages = 4;
+constexpr int kGemmThreads = 192; // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+
+// ---- workspace layout -------------------------------------------------------
+struct Workspace {
+  size_t total = 0;
+  // offsets (bytes)
+  size_t iota = 0, seg = 0;              // identity active set for the full step
+  size_t xn = 0, q = 0, a = 0, h32 = 0, hn = 0, act = 0;
+  size_t c32 = 0;                        // fp32 path: GEMM output scratch [Mcap, max(3d, 2F)]
+  size_t partials = 0, flags = 0;        // stream-K fix-up of the tcgen05 GEMM
+  int nflags = 0, nslots = 0;
+};
+Workspace workspace_layout(const plk_dims* d, int num_sms);
+int device_sm_count();
+
+// ---- TMA descriptors ---------------------------------------------------------
+// 2D bf16 tensor [rows, cols] row-major (cols contiguous), 128-byte swizzle,
+// box {64 cols, box_rows rows}.
+int make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+
+// ---- launches (all asynchronous on `st`; return PLK_OK / PLK_ERR_CUDA) -------
+int launch_select(const plk_dims* dims, const float* score, const uint8_t* lock_in, uint8_t* lock_out,
+                  int mode, float tau, int k, int32_t* idx_out, int32_t* seg_ptr, cudaStream_t st);
+
+int launch_score(const plk_dims* dims, const void* X, const void* Ut, int r, const float* proxy_cache,
+                 int metric, float* proxy_out, float* score_out, cudaStream_t st);
+
+int launch_proxy_commit(const plk_dims* dims, int r, const int32_t* idx, const int32_t* seg_ptr,
+                        const float* proxy_new, float* proxy_cache, cudaStream_t st);
+
+int run_layer(const plk_dims* dims, const plk_weights* w, const void* X, const int32_t* idx,
+              const int32_t* seg_ptr, bool full, void* K_cache, void* V_cache, void* Y, void* ws,
+              size_t ws_bytes, cudaStream_t st);
+
+// epilogue modes of the tcgen05 GEMM
+enum GemmEpi { EPI_QKV = 0, EPI_O = 1, EPI_GU = 2, EPI_DOWN = 3 };
+
+struct GemmArgs {
+  int epi;
+  int K;                   // reduction length, multiple of 64
+  int ftiles;              // 128-row feature tiles
+  int gu_F;                // EPI_GU: F (tile f = gate rows f*64.. and up rows F + f*64..)
+  int d;                   // model dim
+  int Mcap;                // token capacity of the activation buffer
+  const int32_t* seg_ptr;  // M = seg_ptr[B]
+  int B;
+  const int32_t* idx;      // compact token -> flattened row
+  void* q_out;             // EPI_QKV: Q compact [Mcap, d] bf16
+  void* k_cache;           // EPI_QKV
+  void* v_cache;           // EPI_QKV
+  const void* x_in;        // EPI_O residual source X [B*N, d] bf16
+  float* h32;              // EPI_O output, EPI_DOWN residual [Mcap, d]
+  void* act_out;           // EPI_GU: [Mcap, F] bf16
+  void* y_cache;           // EPI_DOWN
+  float* partials;         // [nslots][256][128]
+  uint32_t* flags;         // [nflags]
+  int nslots;
+};
+int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& a, cudaStream_t st);
+
+int launch_attention_bf16(const plk_dims* dims, const void* q, const void* K_cache, const void* V_cache,
+                          void* a_out, const int32_t* seg_ptr, cudaStream_t st);
+int launch_attention_f32(const plk_dims* dims, const float* q, const float* K_cache, const float* V_cache,
+                         float* a_out, const int32_t* seg_ptr, int Mcap, cudaStream_t st);
+
+}  // namespace plk

@@ -1,0 +1,249 @@
+// S1: drift score on the singular proxy (the SPA-Cache page, "SPA-Cache:
+// Singular Proxies for Adaptive Caching in Diffusion Language Models", part 1:
+// compare a low-dimensional snapshot instead of the full hidden state; the
+// Polestar page uses the same drift signal to pick rows to refresh).
+//
+//   p_i = Ut x_i (rank r),  score_i = cos(p_i, c_i)  or  |p_i - c_i|
+//
+// bf16: one CTA per 128 rows, X tile (128 x 64) and Ut tile (r x 64) staged by
+// TMA, tcgen05.mma into an fp32 TMEM accumulator of r columns, and the row-wise
+// distance computed straight from TMEM (thread = row) against the cached proxy.
+// The kernel streams X once from HBM; Ut stays in L2.
+// fp32: a SIMT kernel, one warp per row.
+#include "plk_common.cuh"
+#include "plk_internal.h"
+
+namespace plk {
+
+namespace {
+constexpr int kScStages = 4;
+constexpr int kScA = 128 * 64 * 2;  // 16 KB of X per stage
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+}  // namespace
+
+__global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ CUtensorMap tmX,
+                                                       const __grid_constant__ CUtensorMap tmU, int rows, int d,
+                                                       int r, int tmem_cols, const float* __restrict__ cache,
+                                                       float* __restrict__ pout, float* __restrict__ score,
+                                                       int metric) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const int stageB = r * 128;
+  const int stage_bytes = kScA + ((stageB + 1023) & ~1023);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kScStages * stage_bytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kScStages;
+  uint64_t* done = bars + 2 * kScStages;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * kScStages + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 2 * kScStages + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int row0 = blockIdx.x * 128;
+  const int nkb = d / 64;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kScStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    mbar_init(done, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(s_tmem, (uint32_t)tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  if (warp == 0) {
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1)) {
+          *s_abort = 1;
+          break;
+        }
+        uint8_t* a = smem + stage * stage_bytes;
+        mbar_expect_tx(&full[stage], (uint32_t)(kScA + stageB));
+        tma_load_2d(a, &tmX, kb * 64, row0, &full[stage]);
+        tma_load_2d(a + kScA, &tmU, kb * 64, 0, &full[stage]);
+        ++issued;
+        if (++stage == kScStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (*s_abort) {  // let started copies land before exit
+        for (int i = 0; i < kScStages && i < issued; ++i) {
+          const int kb = issued - 1 - i;
+          (void)mbar_wait(&full[kb % kScStages], (uint32_t)((kb / kScStages) & 1));
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (elect_one()) {
+      int stage = 0;
+      uint32_t phase = 0;
+      const uint32_t idesc = idesc_bf16(128, r);
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait(&full[stage], phase)) {
+          *s_abort = 1;
+          break;
+        }
+        tc_fence_after();
+        uint8_t* a = smem + stage * stage_bytes;
+        const uint64_t adesc = sdesc_sw128(smem_u32(a));
+        const uint64_t bdesc = sdesc_sw128(smem_u32(a + kScA));
+#pragma unroll
+        for (int k = 0; k < 4; ++k) umma_bf16(tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) ? 1u : 0u);
+        umma_commit(&empty[stage]);
+        if (++stage == kScStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      umma_commit(done);  // also the drain: arrives when every MMA above is complete
+    }
+    __syncwarp();
+  }
+
+  // epilogue: thread = row (TMEM lane)
+  const bool ok = mbar_wait(done, 0);
+  tc_fence_after();
+  const int row = row0 + warp * 32 + lane;
+  float dot = 0.f, pp = 0.f, cc = 0.f, dd = 0.f;
+  // tcgen05.ld is warp-collective: take the decision once per warp
+  if (__all_sync(0xffffffffu, ok && !*s_abort)) {
+    for (int c0 = 0; c0 < r; c0 += 16) {
+      uint32_t v[16];
+      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+      tmem_ld_wait();
+      if (row < rows) {
+        const float4* cp = reinterpret_cast<const float4*>(cache + (size_t)row * r + c0);
+        float cv[16];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float4 t = __ldg(cp + u);
+          cv[4 * u] = t.x;
+          cv[4 * u + 1] = t.y;
+          cv[4 * u + 2] = t.z;
+          cv[4 * u + 3] = t.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p = __uint_as_float(v[i]);
+          dot = fmaf(p, cv[i], dot);
+          pp = fmaf(p, p, pp);
+          cc = fmaf(cv[i], cv[i], cc);
+          const float df = p - cv[i];
+          dd = fmaf(df, df, dd);
+        }
+        if (pout) {
+          float4* op = reinterpret_cast<float4*>(pout + (size_t)row * r + c0);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            op[u] = make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
+                                __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3]));
+        }
+      }
+    }
+    if (row < rows) {
+      score[row] = metric == PLK_METRIC_COS ? dot / fmaxf(sqrtf(pp) * sqrtf(cc), 1e-30f) : sqrtf(dd);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, (uint32_t)tmem_cols);
+  }
+}
+
+__global__ void __launch_bounds__(256) score_f32_kernel(const float* __restrict__ X, const float* __restrict__ Ut,
+                                                        int rows, int d, int r, const float* __restrict__ cache,
+                                                        float* __restrict__ pout, float* __restrict__ score,
+                                                        int metric) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const float* x = X + (size_t)row * d;
+  float dot = 0.f, pp = 0.f, cc = 0.f, dd = 0.f;
+  for (int c = 0; c < r; ++c) {
+    float s = 0.f;
+    for (int k = lane; k < d; k += 32) s = fmaf(x[k], Ut[(size_t)c * d + k], s);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float cv = cache[(size_t)row * r + c];
+    dot = fmaf(s, cv, dot);
+    pp = fmaf(s, s, pp);
+    cc = fmaf(cv, cv, cc);
+    dd = fmaf(s - cv, s - cv, dd);
+    if (pout && lane == 0) pout[(size_t)row * r + c] = s;
+  }
+  if (lane == 0) score[row] = metric == PLK_METRIC_COS ? dot / fmaxf(sqrtf(pp) * sqrtf(cc), 1e-30f) : sqrtf(dd);
+}
+
+__global__ void proxy_commit_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ seg_ptr, int B,
+                                    int r, const float* __restrict__ pnew, float* __restrict__ pc) {
+  const int M = seg_ptr[B];
+  const int j = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (j >= M) return;
+  const size_t row = (size_t)idx[j];
+  for (int c = threadIdx.x & 31; c < r; c += 32) pc[row * r + c] = pnew[row * r + c];
+}
+
+static int score_tc_smem(int r) {
+  const int stage_bytes = kScA + ((r * 128 + 1023) & ~1023);
+  return kScStages * stage_bytes + 128 + 1024;
+}
+
+int launch_score(const plk_dims* dims, const void* X, const void* Ut, int r, const float* proxy_cache,
+                 int metric, float* proxy_out, float* score_out, cudaStream_t st) {
+  const int rows = dims->B * dims->N, d = dims->d;
+  if (dims->dtype == PLK_F32) {
+    score_f32_kernel<<<ceil_div(rows, 8), 256, 0, st>>>((const float*)X, (const float*)Ut, rows, d, r,
+                                                         proxy_cache, proxy_out, score_out, metric);
+    return cudaPeekAtLastError() == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;
+  }
+  CUtensorMap tmX, tmU;
+  if (make_tmap_bf16(&tmX, X, (uint64_t)rows, (uint64_t)d, 128) != PLK_OK) return PLK_ERR_CUDA;
+  if (make_tmap_bf16(&tmU, Ut, (uint64_t)r, (uint64_t)d, (uint32_t)r) != PLK_OK) return PLK_ERR_CUDA;
+  int tcols = 32;
+  while (tcols < r) tcols <<= 1;
+  const int smem = score_tc_smem(r);
+  static int attr_smem[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PLK_ERR_CUDA;
+  if (dev < 64 && attr_smem[dev] < smem) {
+    if (cudaFuncSetAttribute(score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return PLK_ERR_CUDA;
+    attr_smem[dev] = smem;
+  }
+  score_tc_kernel<<<ceil_div(rows, 128), 128, smem, st>>>(tmX, tmU, rows, d, r, tcols, proxy_cache, proxy_out,
+                                                          score_out, metric);
+  return cudaPeekAtLastError() == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;
+}
+
+int launch_proxy_commit(const plk_dims* dims, int r, const int32_t* idx, const int32_t* seg_ptr,
+                        const float* proxy_new, float* proxy_cache, cudaStream_t st) {
+  const int rows = dims->B * dims->N;
+  proxy_commit_kernel<<<ceil_div(rows, 8), 256, 0, st>>>(idx, seg_ptr, dims->B, r, proxy_new, proxy_cache);
+  return cudaPeekAtLastError() == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;
+}
+
+}  // namespace plk

@@ -1,0 +1,204 @@
+// S2 + S3: lock rules and active-set compaction.
+//
+// Lock rules: the threshold lock of the SureLock page ("Stopping Computation
+// for Converged Tokens in Masked Diffusion-LM Decoding", Sec. 2 "Locking
+// Condition", "Permanent Deactivation") and the top-k budget of the SPA-Cache
+// page ("SPA-Cache: Singular Proxies for Adaptive Caching in Diffusion Language
+// Models", part 2) / Polestar-Cache's most-drifted refresh.
+//
+// Compaction: one CTA per sequence.  A CTA first counts the active rows of the
+// sequences before it (re-deriving their lock state, which is idempotent, so no
+// inter-CTA wait and no scratch memory is needed), then compacts its own
+// sequence chunk by chunk with warp ballots, popcounts and a block scan of the
+// 32 warp counts.  Indices come out ascending and deterministic.
+#include "plk_common.cuh"
+#include "plk_internal.h"
+
+namespace plk {
+
+constexpr int kSelThreads = 1024;
+
+__device__ __forceinline__ uint8_t derive_lock(int mode, const float* score, const uint8_t* lock_src,
+                                               float tau, long long i) {
+  uint8_t l = lock_src[i];
+  if (!l && mode == PLK_SEL_THRESH_GT) l = (score[i] > tau) ? 1 : 0;  // NaN compares false
+  if (!l && mode == PLK_SEL_THRESH_LT) l = (score[i] < tau) ? 1 : 0;
+  return l;
+}
+
+__device__ __forceinline__ int block_sum(int v, int* sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if (lane == 0) sh[warp] = v;
+  __syncthreads();
+  int t = (threadIdx.x < nw) ? sh[threadIdx.x] : 0;
+  if (warp == 0) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (lane == 0) sh[32] = t;
+  }
+  __syncthreads();
+  return sh[32];
+}
+
+// Exclusive block scan of a 0/1 flag; returns this thread's rank and the chunk total.
+__device__ __forceinline__ int block_rank(int flag, int* sh, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const unsigned bal = __ballot_sync(0xffffffffu, flag);
+  const int wpre = __popc(bal & ((1u << lane) - 1u));
+  if (lane == 0) sh[warp] = __popc(bal);
+  __syncthreads();
+  if (warp == 0) {
+    const int v = (lane < nw) ? sh[lane] : 0;
+    int inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += n;
+    }
+    sh[lane] = inc - v;
+    if (lane == 31) sh[32] = inc;
+  }
+  __syncthreads();
+  const int r = sh[warp] + wpre;
+  *total = sh[32];
+  __syncthreads();
+  return r;
+}
+
+// mode: PLK_SEL_THRESH_GT / PLK_SEL_THRESH_LT derive lock_out from lock_in and
+// the score; any other value takes lock_src as the final lock (after top-k).
+__global__ void __launch_bounds__(kSelThreads) compact_kernel(int mode, const float* __restrict__ score,
+                                                              const uint8_t* lock_src, uint8_t* lock_out,
+                                                              int N, float tau, int32_t* __restrict__ idx_out,
+                                                              int32_t* __restrict__ seg_ptr) {
+  __shared__ int sh[33];
+  const int b = blockIdx.x;
+  const bool writes_lock = (mode == PLK_SEL_THRESH_GT || mode == PLK_SEL_THRESH_LT);
+  // active rows of the sequences before this one
+  int cnt = 0;
+  const long long before = (long long)b * N;
+  for (long long i = threadIdx.x; i < before; i += blockDim.x)
+    cnt += derive_lock(mode, score, lock_src, tau, i) ? 0 : 1;
+  const int offset = block_sum(cnt, sh);
+  int running = 0;
+  for (int c0 = 0; c0 < N; c0 += blockDim.x) {
+    const int i = c0 + threadIdx.x;
+    int act = 0;
+    if (i < N) {
+      const uint8_t l = derive_lock(mode, score, lock_src, tau, before + i);
+      if (writes_lock) lock_out[before + i] = l;
+      act = l ? 0 : 1;
+    }
+    int total;
+    const int r = block_rank(act, sh, &total);
+    if (act) idx_out[offset + running + r] = (int32_t)(before + i);
+    running += total;
+  }
+  if (threadIdx.x == 0) {
+    seg_ptr[b + 1] = offset + running;
+    if (b == 0) seg_ptr[0] = 0;
+  }
+}
+
+// Order-preserving key: larger key = more preferred.  NaN maps to 0, below
+// every other key; -0 maps like +0.
+__device__ __forceinline__ uint32_t pref_key(float s, bool largest) {
+  uint32_t u = __float_as_uint(s);
+  if ((u & 0x7FFFFFFFu) > 0x7F800000u) return 0u;  // NaN
+  if ((u & 0x7FFFFFFFu) == 0u) u = 0u;               // -0 -> +0
+  uint32_t k = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return largest ? k : ~k;
+}
+
+// One CTA per sequence: among rows with lock_in == 0 keep the k most preferred
+// (ties to the lower index) and lock every other row.  Radix select on 8-bit
+// digits finds the k-th key; an ordered block scan breaks ties.
+__global__ void __launch_bounds__(kSelThreads) topk_kernel(const float* __restrict__ score,
+                                                           const uint8_t* lock_in, uint8_t* lock_out, int N,
+                                                           int k, int largest) {
+  __shared__ int hist[256];
+  __shared__ int sh[33];
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_remaining;
+  const long long base = (long long)blockIdx.x * N;
+  const bool lg = largest != 0;
+  int c = 0;
+  for (int i = threadIdx.x; i < N; i += blockDim.x) c += lock_in[base + i] ? 0 : 1;
+  const int ncand = block_sum(c, sh);
+  if (k >= ncand || k <= 0) {
+    // every candidate kept (k >= ncand) or none (k <= 0)
+    __syncthreads();
+    for (int i = threadIdx.x; i < N; i += blockDim.x) {
+      const uint8_t l = lock_in[base + i];
+      lock_out[base + i] = (k > 0 && !l) ? 0 : 1;
+    }
+    return;
+  }
+  uint32_t prefix = 0, pmask = 0;
+  int remaining = k;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int t = threadIdx.x; t < 256; t += blockDim.x) hist[t] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < N; i += blockDim.x) {
+      if (lock_in[base + i]) continue;
+      const uint32_t key = pref_key(score[base + i], lg);
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int above = 0, bin = 255;
+      for (; bin > 0; --bin) {
+        if (above + hist[bin] >= remaining) break;
+        above += hist[bin];
+      }
+      s_prefix = prefix | ((uint32_t)bin << shift);
+      s_remaining = remaining - above;
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    remaining = s_remaining;
+    pmask |= 0xFFu << shift;
+    __syncthreads();
+  }
+  // prefix = k-th most preferred key; remaining = how many rows equal to it to keep
+  const uint32_t kth = prefix;
+  int taken_eq = 0;
+  for (int c0 = 0; c0 < N; c0 += blockDim.x) {
+    const int i = c0 + threadIdx.x;
+    bool cand = false, eq = false, gt = false;
+    if (i < N) {
+      cand = lock_in[base + i] == 0;
+      if (cand) {
+        const uint32_t key = pref_key(score[base + i], lg);
+        gt = key > kth;
+        eq = key == kth;
+      }
+    }
+    int total;
+    const int r = block_rank(eq ? 1 : 0, sh, &total);
+    if (i < N) {
+      const bool keep = cand && (gt || (eq && taken_eq + r < remaining));
+      lock_out[base + i] = keep ? 0 : 1;
+    }
+    taken_eq += total;
+  }
+}
+
+int launch_select(const plk_dims* dims, const float* score, const uint8_t* lock_in, uint8_t* lock_out,
+                  int mode, float tau, int k, int32_t* idx_out, int32_t* seg_ptr, cudaStream_t st) {
+  const int B = dims->B, N = dims->N;
+  if (mode == PLK_SEL_TOPK_LARGEST || mode == PLK_SEL_TOPK_SMALLEST) {
+    topk_kernel<<<B, kSelThreads, 0, st>>>(score, lock_in, lock_out, N, k, mode == PLK_SEL_TOPK_LARGEST);
+    if (cudaPeekAtLastError() != cudaSuccess) return PLK_ERR_CUDA;
+    compact_kernel<<<B, kSelThreads, 0, st>>>(-1, score, lock_out, lock_out, N, tau, idx_out, seg_ptr);
+  } else {
+    compact_kernel<<<B, kSelThreads, 0, st>>>(mode, score, lock_in, lock_out, N, tau, idx_out, seg_ptr);
+  }
+  return cudaPeekAtLastError() == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;
+}
+
+}  // namespace plk

@@ -1,0 +1,68 @@
+"""The C-ABI library loads and exports every entry point declared in include/plk.h.
+
+Runs without a GPU: only symbol lookup and host-side argument validation (which
+returns before any CUDA call) are exercised.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "plk.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(plk_[a-z_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def built():
+    from partial_recompute_kv_b200 import build
+    return build.build()
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("plk_score_drift", "plk_select_active", "plk_layer_step_partial", "plk_full_layer_step"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(built):
+    lib = ctypes.CDLL(built)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_binding_covers_every_declared_symbol(built):
+    import partial_recompute_kv_b200 as plk
+    assert sorted(plk.EXPORTED) == declared_functions()
+
+
+def test_host_validation_without_gpu(built):
+    import partial_recompute_kv_b200 as plk
+    lib = plk.lib
+    assert plk.version() == 100
+    assert plk.error_string(plk.ERR_TIMEOUT) == "device wait exceeded its limit"
+    # null dims / bad enums / bad shapes are rejected before any CUDA call
+    assert lib.plk_score_drift(None, None, None, 8, None, 0, None, None, None) == plk.ERR_ARG
+    bad_dtype = plk.dims(1, 8, 64, 4, 16, 64, dtype=7)
+    assert lib.plk_score_drift(ctypes.byref(bad_dtype), None, None, 8, None, 0, None, None, None) == plk.ERR_DTYPE
+    bad_hd = plk.dims(1, 8, 512, 8, 64, 256, dtype=plk.BF16)  # bf16 needs hd == 128
+    assert lib.plk_full_layer_step(ctypes.byref(bad_hd), None, None, None, None, None, None, 0, None) == \
+        plk.ERR_SHAPE
+    bad_split = plk.dims(1, 8, 64, 3, 16, 64, dtype=plk.F32)  # d != H * hd
+    assert lib.plk_workspace_bytes(ctypes.byref(bad_split)) == 0
+    ok = plk.dims(2, 8, 64, 4, 16, 64, dtype=plk.F32)
+    p = ctypes.c_void_p(16)
+    assert lib.plk_select_active(ctypes.byref(ok), p, p, p, 9, 0.5, 1, p, p, None) == plk.ERR_ARG
+    assert lib.plk_select_active(ctypes.byref(ok), p, p, p, plk.SEL_TOPK_LARGEST, 0.5, -1, p, p, None) == \
+        plk.ERR_ARG
+    assert lib.plk_score_drift(ctypes.byref(ok), p, p, 300, p, 0, None, p, None) == plk.ERR_ARG
+    assert lib.plk_score_drift(ctypes.byref(ok), p, p, 8, p, 5, None, p, None) == plk.ERR_ARG
+    assert lib.plk_score_drift(ctypes.byref(ok), p, p, 8, p, 0, p, p, None) == plk.ERR_ARG  # out aliases cache
+    assert lib.plk_set_wait_limit(0) == plk.ERR_ARG
+    assert lib.plk_proxy_commit(ctypes.byref(ok), 0, p, p, p, p, None) == plk.ERR_ARG

@@ -1,0 +1,406 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Integer results (lock, idx, seg_ptr) must match bit-exactly when both sides get
+the same scores; floating-point results use the tolerances of parity_util.
+Every input is seeded synthetic data from `synth`; the oracle never sees a value
+produced by the GPU.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests.parity_util import (assert_bf16_close, assert_f32_close, dev, host, metrics, tdtype,
+                               weights_dev)
+
+pytestmark = pytest.mark.gpu
+
+BF = torch.bfloat16
+
+
+@pytest.fixture(scope="module")
+def plk():
+    import partial_recompute_kv_b200 as m
+    return m
+
+
+def pdims(plk, D):
+    return plk.dims(D.B, D.N, D.d, D.H, D.hd, D.F, D.eps, plk.BF16 if D.dtype == "bf16" else plk.F32)
+
+
+def int_dev(a, n):
+    t = torch.full((n,), -1, dtype=torch.int32, device="cuda")
+    if len(a):
+        t[: len(a)] = torch.from_numpy(np.asarray(a, dtype=np.int32)).cuda()
+    return t
+
+
+def sel_bufs(B, N):
+    idx = torch.full((B * N,), -1, dtype=torch.int32, device="cuda")
+    seg = torch.full((B + 1,), -7, dtype=torch.int32, device="cuda")
+    return idx, seg
+
+
+def check_compaction(idx, seg, ref_lock):
+    ref_idx, ref_seg = oracle.compact(ref_lock)
+    assert np.array_equal(host(seg), ref_seg)
+    M = int(ref_seg[-1])
+    hi = host(idx)
+    assert np.array_equal(hi[:M], ref_idx)
+    assert np.all(hi[M:] == -1), "nothing past M is written"
+
+
+# ---------------------------------------------------------------------------
+# S2/S3 select + compaction: bit-exact
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("B,N", [(1, 1), (3, 1000), (2, 3000)])
+@pytest.mark.parametrize("gt", [True, False])
+@pytest.mark.parametrize("inplace", [False, True])
+def test_select_threshold_bitexact(plk, B, N, gt, inplace):
+    rng = np.random.default_rng(100 + N)
+    s = rng.random((B, N)).astype(np.float32)
+    s[rng.random((B, N)) < 0.02] = np.nan
+    s[0, 0] = 0.5  # exactly tau: strict comparison never locks it
+    lock = (rng.random((B, N)) < 0.3).astype(np.uint8)
+    tau = np.float32(0.5)
+    ref = oracle.lock_threshold(s.astype(np.float64), lock, float(tau), greater=gt)
+    dm = plk.dims(B, N, 64, 4, 16, 64, dtype=plk.F32)
+    score, lin = dev(s, torch.float32), dev(lock, torch.uint8)
+    lout = lin if inplace else torch.full_like(lin, 9)
+    idx, seg = sel_bufs(B, N)
+    plk.select_active(dm, score, lin, lout, plk.SEL_THRESH_GT if gt else plk.SEL_THRESH_LT, float(tau), 0,
+                      idx, seg)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(lout), ref)
+    check_compaction(idx, seg, ref)
+
+
+@pytest.mark.parametrize("B,N", [(1, 5), (2, 777), (8, 4096)])
+@pytest.mark.parametrize("kind", ["random", "ties", "nan"])
+@pytest.mark.parametrize("largest", [True, False])
+def test_select_topk_bitexact(plk, B, N, kind, largest):
+    rng = np.random.default_rng(200 + N)
+    if kind == "ties":
+        s = rng.integers(-2, 3, (B, N)).astype(np.float32)
+        z = s == 0
+        s[z & (rng.random((B, N)) < 0.5)] = -0.0
+    else:
+        s = rng.standard_normal((B, N)).astype(np.float32)
+        if kind == "nan":
+            s[rng.random((B, N)) < 0.05] = np.nan
+    lock = (rng.random((B, N)) < 0.2).astype(np.uint8)
+    dm = plk.dims(B, N, 64, 4, 16, 64, dtype=plk.F32)
+    score, lin = dev(s, torch.float32), dev(lock, torch.uint8)
+    for k in sorted({0, 1, max(N // 10, 1), N // 2, N, N + 5}):
+        ref = oracle.lock_topk(s.astype(np.float64), lock, k, largest)
+        lout = torch.full_like(lin, 9)
+        idx, seg = sel_bufs(B, N)
+        plk.select_active(dm, score, lin, lout, plk.SEL_TOPK_LARGEST if largest else plk.SEL_TOPK_SMALLEST,
+                          0.0, k, idx, seg)
+        torch.cuda.synchronize()
+        assert np.array_equal(host(lout), ref), f"k={k}"
+        check_compaction(idx, seg, ref)
+
+
+# ---------------------------------------------------------------------------
+# S1 score_drift and S10 proxy commit
+# ---------------------------------------------------------------------------
+def _score_case(dtype):
+    if dtype == "f32":
+        return synth.Dims(B=2, N=100, d=64, H=4, hd=16, F=64, dtype="f32"), 8
+    return synth.Dims(B=2, N=300, d=512, H=4, hd=128, F=512, dtype="bf16"), 128
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("metric", ["cos", "l2"])
+def test_score_drift(plk, dtype, metric):
+    D, r = _score_case(dtype)
+    X = synth.hidden_states(D, seed=3)
+    Ut = synth.proxy_basis(D.d, r, seed=3, dtype=dtype)
+    p_exact = oracle.proxy_project(X.reshape(-1, D.d).astype(np.float64), Ut.astype(np.float64))
+    rng = np.random.default_rng(3)
+    moved = rng.random(D.B * D.N) < 0.3
+    pc = p_exact + moved[:, None] * rng.standard_normal(p_exact.shape) * 0.5
+    pc = pc.astype(np.float32).reshape(D.B, D.N, r)
+    ref_s, ref_p = oracle.score_drift(X.astype(np.float64), Ut.astype(np.float64), pc, metric)
+    dm = pdims(plk, D)
+    score = torch.empty((D.B, D.N), dtype=torch.float32, device="cuda")
+    pout = torch.empty((D.B, D.N, r), dtype=torch.float32, device="cuda")
+    plk.score_drift(dm, dev(X, tdtype(D)), dev(Ut, tdtype(D)), r, dev(pc, torch.float32),
+                    plk.METRIC_COS if metric == "cos" else plk.METRIC_L2, score, proxy_out=pout)
+    torch.cuda.synchronize()
+    assert_f32_close(host(pout), ref_p, "proxy", tol=1e-5)
+    assert_f32_close(host(score), ref_s, "score", tol=1e-4)
+
+
+def test_proxy_commit(plk):
+    B, N, r = 3, 50, 16
+    rng = np.random.default_rng(4)
+    pc = rng.standard_normal((B, N, r)).astype(np.float32)
+    pn = rng.standard_normal((B, N, r)).astype(np.float32)
+    lock = (rng.random((B, N)) < 0.6).astype(np.uint8)
+    idx, seg = oracle.compact(lock)
+    ref = oracle.proxy_commit(pc, pn, idx)
+    dm = plk.dims(B, N, 64, 4, 16, 64, dtype=plk.F32)
+    pcd = dev(pc, torch.float32)
+    plk.proxy_commit(dm, r, int_dev(idx, B * N), int_dev(seg, B + 1), dev(pn, torch.float32), pcd)
+    torch.cuda.synchronize()
+    assert np.array_equal(host(pcd), ref)
+
+
+# ---------------------------------------------------------------------------
+# S4..S10 layer steps, bf16
+# ---------------------------------------------------------------------------
+SMALL = synth.Dims(B=2, N=320, d=512, H=4, hd=128, F=1536, dtype="bf16")
+
+
+def _run_partial(plk, D, W, X, idx, seg, st):
+    dm = pdims(plk, D)
+    K, V, Y = dev(st.K, BF), dev(st.V, BF), dev(st.Y, BF)
+    ws = plk.alloc_workspace(dm)
+    plk.layer_step_partial(dm, weights_dev(W, D), dev(X, BF), int_dev(idx, D.B * D.N), int_dev(seg, D.B + 1),
+                           K, V, Y, ws)
+    assert plk.get_status() == plk.OK
+    return host(K), host(V), host(Y)
+
+
+def test_full_layer_step_bf16(plk):
+    D = SMALL
+    W = synth.layer_weights(D, 0.02, seed=1)
+    X = synth.hidden_states(D, seed=1)
+    ref = oracle.full_layer_step(D, W, X, "bf16")
+    dm = pdims(plk, D)
+    K = torch.zeros((D.B, D.N, D.d), dtype=BF, device="cuda")
+    V, Y = torch.zeros_like(K), torch.zeros_like(K)
+    ws = plk.alloc_workspace(dm)
+    plk.full_layer_step(dm, weights_dev(W, D), dev(X, BF), K, V, Y, ws)
+    assert plk.get_status() == plk.OK
+    assert_bf16_close(host(K), ref.K, "K")
+    assert_bf16_close(host(V), ref.V, "V")
+    assert_bf16_close(host(Y), ref.Y, "Y")
+
+
+@pytest.mark.parametrize("p_active", [0.05, 0.3, 1.0])
+def test_partial_step_bf16(plk, p_active):
+    D = SMALL
+    W = synth.layer_weights(D, 0.02, seed=2)
+    X = synth.hidden_states(D, seed=2)
+    base = oracle.full_layer_step(D, W, X, "bf16")
+    lock = synth.bernoulli_active(D.B, D.N, p_active, seed=7)
+    if p_active == 1.0:
+        lock[:] = 0
+    idx, seg = oracle.compact(lock)
+    X2 = synth.perturb_rows(X, synth.step_noise((D.B, D.N, D.d), 0.01, seed=7), lock == 0, "bf16")
+    ref = oracle.layer_step_partial(D, W, X2, idx, seg, base, "bf16")
+    K, V, Y = _run_partial(plk, D, W, X2, idx, seg, base)
+    locked = lock.astype(bool)
+    for g, o0, name in ((K, base.K, "K"), (V, base.V, "V"), (Y, base.Y, "Y")):
+        assert np.array_equal(g[locked], o0[locked]), f"{name}: a locked row was written"
+    act = ~locked
+    assert_bf16_close(K[act], ref.K[act], "K active")
+    assert_bf16_close(V[act], ref.V[act], "V active")
+    assert_bf16_close(Y[act], ref.Y[act], "Y active")
+
+
+def test_partial_step_m_zero_is_noop(plk):
+    D = SMALL
+    W = synth.layer_weights(D, 0.02, seed=3)
+    X = synth.hidden_states(D, seed=3)
+    rng = np.random.default_rng(3)
+    st = oracle.LayerState(*(synth.round_bf16(rng.standard_normal((D.B, D.N, D.d)).astype(np.float32))
+                             .astype(np.float64) for _ in range(3)))
+    idx, seg = oracle.compact(np.ones((D.B, D.N), np.uint8))
+    K, V, Y = _run_partial(plk, D, W, X, idx, seg, st)
+    assert np.array_equal(K, st.K) and np.array_equal(V, st.V) and np.array_equal(Y, st.Y)
+
+
+def test_workspace_too_small_is_rejected(plk):
+    D = SMALL
+    dm = pdims(plk, D)
+    W = weights_dev(synth.layer_weights(D, 0.02), D)
+    X = torch.zeros((D.B, D.N, D.d), dtype=BF, device="cuda")
+    small = torch.empty(1024, dtype=torch.uint8, device="cuda")
+    with pytest.raises(plk.PlkError) as e:
+        plk.full_layer_step(dm, W, X, X.clone(), X.clone(), X.clone(), small)
+    assert e.value.code == plk.ERR_WORKSPACE
+
+
+# ---------------------------------------------------------------------------
+# the tiny fp32 workload: 20 denoising steps, every step checked
+# ---------------------------------------------------------------------------
+def test_tiny_fp32_driver(plk):
+    D = synth.TINY
+    r = synth.TINY_RANK
+    W = synth.layer_weights(D, 1.0 / math.sqrt(D.d))
+    X0 = synth.hidden_states(D)
+    Ut = synth.proxy_basis(D.d, r, dtype="f32")
+    lock0 = synth.bernoulli_active(D.B, D.N, synth.TINY_P_ACTIVE)
+    noises = [synth.step_noise((D.B, D.N, D.d), synth.TINY_NOISE_VAR, step=t) for t in range(synth.TINY_STEPS)]
+    perturb = lambda X, e, m: synth.perturb_rows(X, e, m, "f32")
+    recs = oracle.tiny_run(D, W, X0, Ut.astype(np.float64), lock0, noises, synth.TINY_TAU, perturb)
+
+    dm = pdims(plk, D)
+    f32 = torch.float32
+    Wd = weights_dev(W, D)
+    Utd = dev(Ut, f32)
+    K = torch.zeros((D.B, D.N, D.d), dtype=f32, device="cuda")
+    V, Y = torch.zeros_like(K), torch.zeros_like(K)
+    ws = plk.alloc_workspace(dm)
+    plk.full_layer_step(dm, Wd, dev(X0, f32), K, V, Y, ws)
+    score = torch.empty((D.B, D.N), dtype=f32, device="cuda")
+    pnew = torch.empty((D.B, D.N, r), dtype=f32, device="cuda")
+    pc = torch.zeros_like(pnew)
+    plk.score_drift(dm, dev(X0, f32), Utd, r, pc, plk.METRIC_L2, score, proxy_out=pnew)
+    pc.copy_(pnew)
+    lock = dev(lock0, torch.uint8)
+    idx, seg = sel_bufs(D.B, D.N)
+    X = X0.copy()
+    for t, eps in enumerate(noises):
+        X = perturb(X, eps, host(lock) == 0)
+        Xd = dev(X, f32)
+        plk.score_drift(dm, Xd, Utd, r, pc, plk.METRIC_COS, score, proxy_out=pnew)
+        plk.select_active(dm, score, lock, lock, plk.SEL_THRESH_GT, synth.TINY_TAU, 0, idx, seg)
+        plk.layer_step_partial(dm, Wd, Xd, idx, seg, K, V, Y, ws)
+        plk.proxy_commit(dm, r, idx, seg, pnew, pc)
+        assert plk.get_status() == plk.OK
+        rec = recs[t]
+        assert np.array_equal(host(lock), rec["lock"]), f"step {t}: lock"
+        M = int(rec["seg_ptr"][-1])
+        assert np.array_equal(host(seg), rec["seg_ptr"]) and np.array_equal(host(idx)[:M], rec["idx"])
+        assert_f32_close(host(score), rec["score"], f"step {t}: score")
+        for name, g in (("K", K), ("V", V), ("Y", Y), ("proxy", pc)):
+            assert_f32_close(host(g), rec[name], f"step {t}: {name}")
+
+
+# ---------------------------------------------------------------------------
+# the 8B-shape layer at M/N = 0.25 (the benchmarked launch), sampled rows
+# ---------------------------------------------------------------------------
+@pytest.mark.slow
+def test_layer_8b_quarter_sampled(plk):
+    D = synth.LAYER_8B
+    W = synth.layer_weights(D, synth.LAYER_8B_WSTD)
+    X = synth.hidden_states(D)
+    base = oracle.full_layer_step(D, W, X, "bf16")
+    pos = synth.layer_8b_positions(D.N, 0.25)
+    lock = np.ones((1, D.N), np.uint8)
+    lock[0, pos] = 0
+    idx, seg = oracle.compact(lock)
+    assert idx.size == 256
+    X2 = synth.perturb_rows(X, synth.step_noise((1, D.N, D.d), 0.01), lock == 0, "bf16")
+    sample = np.arange(0, 256, 8)
+    ref = oracle.layer_step_partial(D, W, X2, idx, seg, base, "bf16", out_rows=sample)
+    K, V, Y = _run_partial(plk, D, W, X2, idx, seg, base)
+    locked = lock.astype(bool)
+    assert np.array_equal(K[locked], base.K[locked]) and np.array_equal(Y[locked], base.Y[locked])
+    act = ~locked
+    assert_bf16_close(K[act], ref.K[act], "K active")
+    assert_bf16_close(V[act], ref.V[act], "V active")
+    rows = idx[sample]
+    assert_bf16_close(Y.reshape(-1, D.d)[rows], ref.Y.reshape(-1, D.d)[rows], "Y sampled")
+
+
+# ---------------------------------------------------------------------------
+# long-context block decode (N = 8192, M from the seeded geometric draw), reduced width
+# ---------------------------------------------------------------------------
+def test_long_context_blocks_reduced_width(plk):
+    D = synth.Dims(B=1, N=8192, d=256, H=2, hd=128, F=512, dtype="bf16")
+    W = synth.layer_weights(D, 0.02, seed=4)
+    X = synth.hidden_states(D, seed=4)
+    rng = np.random.default_rng(4)
+    st = oracle.LayerState(*(synth.round_bf16(rng.standard_normal((1, D.N, D.d)).astype(np.float32))
+                             .astype(np.float64) for _ in range(3)))
+    Ms = synth.geometric_block_m(8)
+    prompt = 7936
+    dm = pdims(plk, D)
+    Wd = weights_dev(W, D)
+    ws = plk.alloc_workspace(dm)
+    K, V, Y = dev(st.K, BF), dev(st.V, BF), dev(st.Y, BF)
+    for blk in (0, 7):
+        M = int(Ms[blk])
+        b0 = prompt + 32 * blk
+        extra = synth.uniform_positions(0, b0, M - 32, tag=100 + blk)
+        lock = np.ones((1, D.N), np.uint8)
+        lock[0, np.arange(b0, b0 + 32)] = 0
+        lock[0, extra] = 0
+        idx, seg = oracle.compact(lock)
+        assert idx.size == M
+        ref = oracle.layer_step_partial(D, W, X, idx, seg, st, "bf16")
+        before = [host(K), host(V), host(Y)]
+        plk.layer_step_partial(dm, Wd, dev(X, BF), int_dev(idx, D.N), int_dev(seg, 2), K, V, Y, ws)
+        assert plk.get_status() == plk.OK
+        act = lock == 0
+        for g, g0, o, name in ((K, before[0], ref.K, "K"), (V, before[1], ref.V, "V"), (Y, before[2], ref.Y, "Y")):
+            gh = host(g)
+            assert np.array_equal(gh[~act], g0[~act]), f"{name}: locked rows changed"
+            assert_bf16_close(gh[act], o[act], f"block {blk} {name}")
+        st = ref
+
+
+# ---------------------------------------------------------------------------
+# B = 4 multi-layer stack with the linear schedule, reduced width: score -> top-k
+# among unlocked rows -> partial step, layer output feeding the next layer
+# ---------------------------------------------------------------------------
+def test_stack_b4_two_layers_reduced_width(plk):
+    D = synth.Dims(B=4, N=2048, d=256, H=2, hd=128, F=512, dtype="bf16")
+    r = 128
+    sched = synth.linear_schedule(D.N)
+    dm = pdims(plk, D)
+    ws = plk.alloc_workspace(dm)
+    layers = [synth.layer_weights(D, 0.02, seed=0, layer=l) for l in range(2)]
+    Ut = synth.proxy_basis(D.d, r, seed=5)
+    rng = np.random.default_rng(5)
+    for t in (0, 128, 255):
+        M_prev = int(sched[t - 1]) if t else D.N
+        lock = np.ones((D.B, D.N), np.uint8)
+        for b in range(D.B):
+            lock[b, rng.choice(D.N, M_prev, replace=False)] = 0
+        X = synth.hidden_states(D, seed=10 + t)
+        for l, W in enumerate(layers):
+            st = oracle.LayerState(*(synth.round_bf16(rng.standard_normal((D.B, D.N, D.d)).astype(np.float32))
+                                     .astype(np.float64) for _ in range(3)))
+            pc = rng.standard_normal((D.B, D.N, r)).astype(np.float32)
+            ref_s, _ = oracle.score_drift(X.astype(np.float64), Ut.astype(np.float64), pc, "l2")
+            score = torch.empty((D.B, D.N), dtype=torch.float32, device="cuda")
+            plk.score_drift(dm, dev(X, BF), dev(Ut, BF), r, dev(pc, torch.float32), plk.METRIC_L2, score)
+            assert_f32_close(host(score), ref_s, f"t{t} l{l} score")
+            # top-k selection, both sides on the same (oracle's, fp32-rounded) scores
+            s32 = ref_s.astype(np.float32)
+            k = int(sched[t])
+            ref_lock = oracle.lock_topk(s32.astype(np.float64), lock, k, True)
+            lk_in, lk = dev(lock, torch.uint8), torch.empty((D.B, D.N), dtype=torch.uint8, device="cuda")
+            idx_d, seg_d = sel_bufs(D.B, D.N)
+            plk.select_active(dm, dev(s32, torch.float32), lk_in, lk, plk.SEL_TOPK_LARGEST, 0.0, k, idx_d, seg_d)
+            torch.cuda.synchronize()
+            assert np.array_equal(host(lk), ref_lock)
+            check_compaction(idx_d, seg_d, ref_lock)
+            idx, seg = oracle.compact(ref_lock)
+            ref = oracle.layer_step_partial(D, W, X, idx, seg, st, "bf16")
+            K, V, Y = dev(st.K, BF), dev(st.V, BF), dev(st.Y, BF)
+            plk.layer_step_partial(dm, weights_dev(W, D), dev(X, BF), idx_d, seg_d, K, V, Y, ws)
+            assert plk.get_status() == plk.OK
+            act = ref_lock == 0
+            for g, o, name in ((K, ref.K, "K"), (V, ref.V, "V"), (Y, ref.Y, "Y")):
+                gh = host(g)
+                assert np.array_equal(gh[~act], o[~act]), f"{name}: locked rows changed"
+                assert_bf16_close(gh[act], o[act], f"t{t} l{l} {name}")
+            lock = ref_lock
+            X = ref.Y.astype(np.float32)  # next layer's input: this layer's output cache
+
+
+# ---------------------------------------------------------------------------
+# the device wait limit: a wait that nothing satisfies returns an error status
+# ---------------------------------------------------------------------------
+def test_wait_timeout_reports_status(plk):
+    assert plk.get_status() == plk.OK
+    plk.set_wait_limit(2_000_000)  # about a millisecond
+    try:
+        plk.selftest_wait_timeout()
+        assert plk.get_status() == plk.ERR_TIMEOUT
+        assert plk.get_status() == plk.OK  # cleared by the read
+    finally:
+        plk.set_wait_limit(4_000_000_000)
+    x = torch.ones(4, device="cuda")
+    assert float((x + 1).sum()) == 8.0  # the context is still usable
