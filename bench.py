@@ -1,0 +1,448 @@
+#!/usr/bin/env python
+"""Throughput of the partial-recompute denoising step on B200.
+
+Workload: one 8B-shape bidirectional layer (d=4096, 32 heads x 128, SwiGLU
+F=12288), N=1024 tokens, batch 1, active fraction M/N = 0.25 (256 rows), as in
+the SureLock page's setting ("Stopping Computation for Converged Tokens in
+Masked Diffusion-LM Decoding", Sec. 4: LLaDA-8B).  One step is the whole hot
+path: S1 drift score (rank-128 singular proxy, L2), S2/S3 top-k selection and
+compaction, S4-S10 partial layer step, S10 proxy refresh.  The 256 perturbed
+rows are exactly the ones the top-k picks; the proxy cache is restored between
+steps (untimed) so that every step does the same work.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl plk|reference]
+
+Prints one JSON line (rank 0).  --impl reference times the CPU oracle instead.
+Multi-GPU: one process per GPU under torchrun; every rank runs its own
+replica (independent sequences, no collective on the data path), time is the
+max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "active-token-layers/sec at 8B-shape, M/N=0.25; % of bf16 tensor peak"
+UNIT = "active-token-layers/s"
+PROFILE_TXT = os.path.join(ROOT, "profiles", "gemm_tc_8b_quarter.txt")
+GEMM_SRC = os.path.join(ROOT, "partial_recompute_kv_b200", "csrc", "gemm_tc.cu")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# workload (seeded synthetic inputs shared by both arms)
+# ---------------------------------------------------------------------------
+class Workload:
+    def __init__(self, frac=0.25, rank=128, seed=0):
+        import synth
+        self.D = synth.LAYER_8B
+        self.frac, self.r = frac, rank
+        self.M = synth.active_count(self.D.N, frac)
+        self.W = synth.layer_weights(self.D, synth.LAYER_8B_WSTD, seed=seed)
+        self.X = synth.hidden_states(self.D, seed=seed)
+        self.Ut = synth.proxy_basis(self.D.d, rank, seed=seed)
+        self.pos = synth.layer_8b_positions(self.D.N, frac, seed=seed)
+        mask = np.zeros((self.D.B, self.D.N), bool)
+        mask[0, self.pos] = True
+        noise = synth.step_noise((self.D.B, self.D.N, self.D.d), 0.01, seed=seed)
+        self.Xp = synth.perturb_rows(self.X, noise, mask, "bf16")
+
+    def flops_per_row(self):
+        D = self.D
+        return 8 * D.d * D.d + 6 * D.d * D.F + 4 * D.N * D.d
+
+    def gemm_flops_per_row(self):
+        D = self.D
+        return 8 * D.d * D.d + 6 * D.d * D.F
+
+    def config(self):
+        D = self.D
+        return {"workload": (f"single 8B-shape layer, d={D.d}, {D.H} heads x {D.hd}, SwiGLU F={D.F}, "
+                             f"N={D.N}, batch {D.B}, M/N={self.frac} ({self.M} active rows); step = drift "
+                             f"score (rank-{self.r} proxy, L2) + top-k select + partial layer step + "
+                             f"proxy refresh"),
+                "B": D.B, "N": D.N, "d": D.d, "heads": D.H, "head_dim": D.hd, "F": D.F,
+                "active_rows": self.M, "proxy_rank": self.r,
+                "l2": "flushed before every timed step (256 MiB write)",
+                "inputs": "resident in HBM for value; host pinned buffers for e2e"}
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    except Exception:
+        return dict(FALLBACK_PEAKS)
+
+
+def gemm_traffic_per_launch():
+    """dram read+write bytes per GEMM launch from the committed ncu summary, or None
+    when the summary is missing or was taken on a different kernel source."""
+    try:
+        src_hash = hashlib.sha256(open(GEMM_SRC, "rb").read()).hexdigest()[:16]
+        kv = {}
+        for line in open(PROFILE_TXT):
+            if ":" in line:
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+        if kv.get("kernel_source_sha256_16") != src_hash:
+            return None
+        return float(kv["dram_bytes_per_launch_avg"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    def __init__(self, device_index, period=0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period, self._stop = period, threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            pass
+
+    def _run(self):
+        nv = self.nv
+        names = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+                 "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for n, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(n)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def aggregate(dist, value_local, device=None):
+    """Max of a float over ranks (identity when not distributed)."""
+    if dist is None or not dist.is_initialized():
+        return value_local
+    import torch
+    t = torch.tensor([value_local], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline of the GPU arm, and the reference arm)
+# ---------------------------------------------------------------------------
+class OracleRunner:
+    """The CPU oracle on the same workload: caches from a full step (untimed), then
+    partial steps.  A step on `rows` active rows is a complete partial-recompute
+    step with that active set (S1 for all N rows, S2 top-k, S3, S4-S10, proxy refresh)."""
+
+    def __init__(self, wl):
+        import oracle
+        self.o, self.wl = oracle, wl
+        D = wl.D
+        self.base = oracle.full_layer_step(D, wl.W, wl.X, "bf16")
+        x = wl.X.reshape(-1, D.d).astype(np.float64)
+        self.pc = oracle.to_f32(oracle.proxy_project(x, wl.Ut.astype(np.float64))).reshape(D.B, D.N, -1)
+        self.Utd = wl.Ut.astype(np.float64)
+
+    def step(self, rows):
+        o, wl, D = self.o, self.wl, self.wl.D
+        # only the chosen `rows` of the perturbed positions differ from the cached proxies
+        keep = np.zeros((D.B, D.N), bool)
+        keep[0, wl.pos[:rows]] = True
+        Xs = np.where(keep[..., None], wl.Xp, wl.X)
+        score, p = o.score_drift(Xs.astype(np.float64), self.Utd, self.pc, "l2")
+        lock = o.lock_topk(score, np.zeros((D.B, D.N), np.uint8), rows, True)
+        idx, seg = o.compact(lock)
+        o.layer_step_partial(D, wl.W, Xs, idx, seg, self.base, "bf16")
+        o.proxy_commit(self.pc, p, idx)
+        return int(idx.size)
+
+
+def run_reference(args, wl):
+    cfg = wl.config()
+    run = OracleRunner(wl)
+    t0 = time.perf_counter()
+    run.step(8)
+    per_row = (time.perf_counter() - t0) / 8
+    budget = 150.0
+    rows = int(max(1, min(wl.M, budget / max(args.steps + args.warmup, 1) / per_row)))
+    for _ in range(args.warmup):
+        run.step(rows)
+    t0 = time.perf_counter()
+    units = 0
+    for _ in range(args.steps):
+        units += run.step(rows)
+    el = time.perf_counter() - t0
+    value = units / el
+    sample = (f"{args.steps} oracle steps of the same layer and cache state with {rows} of the "
+              f"{wl.M} active rows per step (complete partial steps at that active count)")
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": cfg,
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(wl, budget_s=15.0):
+    run = OracleRunner(wl)
+    t0 = time.perf_counter()
+    units, steps = 0, 0
+    while True:
+        units += run.step(wl.M)
+        steps += 1
+        if time.perf_counter() - t0 > budget_s or steps >= 20:
+            break
+    el = time.perf_counter() - t0
+    return {"value": units / el, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{steps} complete oracle steps of this workload ({wl.M} active rows each), "
+                      f"caches from an untimed oracle full step"}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_gpu(args, wl, dist, rank, world, local_rank):
+    import torch
+    import partial_recompute_kv_b200 as plk
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    D, r, M = wl.D, wl.r, wl.M
+    bf = torch.bfloat16
+    up = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(dt)
+    dm = plk.dims(D.B, D.N, D.d, D.H, D.hd, D.F, D.eps, plk.BF16)
+    W = {k: up(v, bf) for k, v in wl.W.items()}
+    pw = plk.weights(W)
+    X, Xp, Ut = up(wl.X, bf), up(wl.Xp, bf), up(wl.Ut, bf)
+    K = torch.zeros((D.B, D.N, D.d), dtype=bf, device=dev)
+    V, Y = torch.zeros_like(K), torch.zeros_like(K)
+    ws = plk.alloc_workspace(dm, device=dev)
+    score = torch.empty((D.B, D.N), dtype=torch.float32, device=dev)
+    pnew = torch.empty((D.B, D.N, r), dtype=torch.float32, device=dev)
+    pc = torch.zeros_like(pnew)
+    lock_in = torch.zeros((D.B, D.N), dtype=torch.uint8, device=dev)
+    lock = torch.empty_like(lock_in)
+    idx = torch.empty(D.B * D.N, dtype=torch.int32, device=dev)
+    seg = torch.empty(D.B + 1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    # state: caches from a full step on X, cached proxies of X
+    plk.full_layer_step(dm, pw, X, K, V, Y, ws)
+    plk.score_drift(dm, X, Ut, r, pc, plk.METRIC_L2, score, proxy_out=pnew)
+    pc0 = pnew.clone()
+    pc.copy_(pc0)
+
+    def step(xin):
+        plk.score_drift(dm, xin, Ut, r, pc, plk.METRIC_L2, score, proxy_out=pnew)
+        plk.select_active(dm, score, lock_in, lock, plk.SEL_TOPK_LARGEST, 0.0, M, idx, seg)
+        plk.layer_step_partial(dm, pw, xin, idx, seg, K, V, Y, ws)
+        plk.proxy_commit(dm, r, idx, seg, pnew, pc)
+
+    def prep():
+        pc.copy_(pc0)
+        flush.zero_()
+
+    prep()
+    step(Xp)
+    st = plk.get_status()
+    if st != plk.OK:
+        raise RuntimeError(f"device status {plk.error_string(st)}")
+    got = idx[:M].cpu().numpy()
+    if int(seg[-1]) != M or not np.array_equal(np.sort(got), np.sort(wl.pos)):
+        raise RuntimeError("the top-k did not select the perturbed rows")
+    if args.profile:
+        for _ in range(args.steps):
+            prep()
+            step(Xp)
+        torch.cuda.synchronize()
+        return None
+    for _ in range(args.warmup):
+        prep()
+        step(Xp)
+    torch.cuda.synchronize()
+
+    K_ = args.steps
+    E = lambda: torch.cuda.Event(enable_timing=True)
+    ev = [[E() for _ in range(12)] for _ in range(K_)]  # 0 start, 1 score, 2 select, 3..10 layer, 11 end
+    if dist is not None:
+        dist.barrier(device_ids=[local_rank])
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        for i in range(K_):
+            prep()
+            e = ev[i]
+            plk.trace_events(e[3:11])
+            e[0].record()
+            plk.score_drift(dm, Xp, Ut, r, pc, plk.METRIC_L2, score, proxy_out=pnew)
+            e[1].record()
+            plk.select_active(dm, score, lock_in, lock, plk.SEL_TOPK_LARGEST, 0.0, M, idx, seg)
+            e[2].record()
+            plk.layer_step_partial(dm, pw, Xp, idx, seg, K, V, Y, ws)
+            plk.proxy_commit(dm, r, idx, seg, pnew, pc)
+            e[11].record()
+        torch.cuda.synchronize()
+    plk.trace_events([])
+    if dist is not None:
+        dist.barrier(device_ids=[local_rank])
+    st = plk.get_status()
+    if st != plk.OK:
+        raise RuntimeError(f"device status {plk.error_string(st)}")
+
+    step_ms = [e[0].elapsed_time(e[11]) for e in ev]
+    names = ["score", "select", "rmsnorm1", "gemm_qkv", "attention", "gemm_o", "rmsnorm2", "gemm_gu",
+             "gemm_down", "proxy_commit"]
+    bounds = [(0, 1), (1, 2), (3, 4), (4, 5), (5, 6), (6, 7), (7, 8), (8, 9), (9, 10), (10, 11)]
+    per = {n: statistics.mean(e[a].elapsed_time(e[b]) for e in ev) * 1e3 for n, (a, b) in zip(names, bounds)}
+    total_ms = sum(step_ms)
+    total_ms_max = aggregate(dist, total_ms, dev)
+    ms_per_step = total_ms_max / K_
+    value = world * M * K_ / (total_ms_max / 1e3)
+
+    # roofline of the dominant kernel: the tcgen05 GEMM (4 launches per step)
+    pk = peaks()
+    gemm_us = per["gemm_qkv"] + per["gemm_o"] + per["gemm_gu"] + per["gemm_down"]
+    gemm_flops_launch = M * wl.gemm_flops_per_row() / 4
+    achieved = gemm_flops_launch / (gemm_us / 4 * 1e-6) / 1e12
+    peak = float(pk["bf16_tflops"])
+    traffic = gemm_traffic_per_launch()
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": traffic, "kernel": "gemm_tc_kernel",
+                "launches_per_step": 4, "peak_source": f"{pk.get('source')} bf16_tflops (burst)"}
+
+    # e2e through the public API: H2D of the step's input, the step, D2H of the output cache
+    e2e_steps = min(K_, 50)
+    Xp_host = torch.from_numpy(np.ascontiguousarray(wl.Xp)).to(bf).pin_memory()
+    Y_host = torch.empty(Y.shape, dtype=bf).pin_memory()
+    xin = torch.empty_like(Xp)
+    ee = [(E(), E()) for _ in range(e2e_steps)]
+    torch.cuda.synchronize()
+    for i in range(e2e_steps):
+        prep()
+        ee[i][0].record()
+        xin.copy_(Xp_host, non_blocking=True)
+        step(xin)
+        Y_host.copy_(Y, non_blocking=True)
+        ee[i][1].record()
+    torch.cuda.synchronize()
+    e2e_ms = aggregate(dist, sum(a.elapsed_time(b) for a, b in ee), dev) / e2e_steps
+    e2e = {"value": world * M / (e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": Xp_host.numel() * Xp_host.element_size(),
+           "d2h_bytes_per_step": Y_host.numel() * Y_host.element_size(), "ms_per_step": e2e_ms}
+    step_flops = M * wl.flops_per_row()
+    return {"value": value, "ms_per_step": ms_per_step, "per_kernel_us": per, "roofline": roofline,
+            "e2e": e2e, "clocks": clk.summary(), "step_tflops": step_flops / (ms_per_step * 1e-3) / 1e12,
+            "peaks": pk}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["plk", "reference"], default="plk")
+    ap.add_argument("--profile", action="store_true",
+                    help="set up and run --steps steps without timing or output (for ncu)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3) if not args.profile else args.warmup
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        run_reference(args, Workload())
+        return 0
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    wl = Workload()
+    try:
+        res = run_gpu(args, wl, dist, rank, world, local_rank)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+    if res is None or rank != 0:
+        return 0
+    launches_per_step = 1 + 2 + 7 + 1
+    line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(wl.config(), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+            "roofline": res["roofline"],
+            "step_tflops": res["step_tflops"],
+            "step_frac_of_bf16_peak": res["step_tflops"] / float(res["peaks"]["bf16_tflops"]),
+            "per_kernel_us": res["per_kernel_us"],
+            "e2e": res["e2e"], "gpu_launches": launches_per_step * args.steps, "clocks": res["clocks"]}
+    if world == 1:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

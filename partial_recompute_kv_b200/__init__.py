@@ -25,7 +25,7 @@ SEL_THRESH_GT, SEL_THRESH_LT, SEL_TOPK_LARGEST, SEL_TOPK_SMALLEST = 0, 1, 2, 3
 EXPORTED = (
     "plk_score_drift", "plk_select_active", "plk_layer_step_partial", "plk_full_layer_step",
     "plk_proxy_commit", "plk_workspace_bytes", "plk_get_status", "plk_set_wait_limit",
-    "plk_selftest_wait_timeout", "plk_error_string", "plk_version",
+    "plk_selftest_wait_timeout", "plk_trace_events", "plk_error_string", "plk_version",
 )
 
 
@@ -62,6 +62,7 @@ def _load():
         "plk_get_status": (I, [P]),
         "plk_set_wait_limit": (I, [L]),
         "plk_selftest_wait_timeout": (I, [P]),
+        "plk_trace_events": (I, [ctypes.POINTER(ctypes.c_void_p), I]),
         "plk_error_string": (ctypes.c_char_p, [I]),
         "plk_version": (I, []),
     }
@@ -72,7 +73,25 @@ def _load():
     return lib
 
 
-lib = _load()
+class _Lib:
+    """The loaded libplk.so, opened on first use (so that the in-package build
+    script can run before the library exists).  Raises ImportError if the
+    library is missing: there is no fallback."""
+
+    _cdll = None
+
+    def __getattr__(self, name):
+        if _Lib._cdll is None:
+            _Lib._cdll = _load()
+        return getattr(_Lib._cdll, name)
+
+
+lib = _Lib()
+
+
+def load():
+    """Open the library now (raises ImportError if it is missing)."""
+    return lib.plk_version()
 
 
 def error_string(code: int) -> str:
@@ -152,6 +171,19 @@ def get_status(stream=None) -> int:
 
 def set_wait_limit(cycles: int):
     _check(lib.plk_set_wait_limit(int(cycles)), "set_wait_limit")
+
+
+def trace_events(events):
+    """Register torch.cuda.Event objects (timing enabled) to be recorded between the
+    layer step's kernels; an empty list unregisters.  Each event is recorded once
+    first so that its CUDA handle exists."""
+    handles = []
+    for e in events:
+        if e.cuda_event == 0:
+            e.record()
+        handles.append(e.cuda_event)
+    arr = (ctypes.c_void_p * max(len(handles), 1))(*handles)
+    _check(lib.plk_trace_events(arr, len(handles)), "trace_events")
 
 
 def selftest_wait_timeout(stream=None):

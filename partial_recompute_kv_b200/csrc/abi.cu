@@ -112,6 +112,13 @@ int plk_get_status(void* stream) {
   return v;
 }
 
+int plk_trace_events(void* const* events, int n) {
+  if (n < 0 || n > 16 || (n > 0 && !events)) return PLK_ERR_ARG;
+  for (int i = 0; i < 16; ++i) g_trace[i] = (i < n) ? (cudaEvent_t)events[i] : nullptr;
+  g_ntrace = n;
+  return PLK_OK;
+}
+
 int plk_set_wait_limit(long long cycles) {
   if (cycles < 1) return PLK_ERR_ARG;
   return cudaMemcpyToSymbol(g_wait_limit, &cycles, sizeof(cycles)) == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;

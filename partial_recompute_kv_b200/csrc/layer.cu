@@ -25,6 +25,13 @@ namespace plk {
 // ---------------------------------------------------------------------------
 // host helpers
 // ---------------------------------------------------------------------------
+// events registered by plk_trace_events, recorded between the step's kernels
+cudaEvent_t g_trace[16];
+int g_ntrace = 0;
+static inline void trace_mark(int i, cudaStream_t st) {
+  if (i < g_ntrace && g_trace[i]) cudaEventRecord(g_trace[i], st);
+}
+
 int device_sm_count() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -292,9 +299,11 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   g.flags = flags;
   g.nslots = L.nslots;
 
+  trace_mark(0, st);
   rmsnorm_rows_kernel<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16><<<Mcap, 256, 0, st>>>(
       X, idx, seg, B, (const __nv_bfloat16*)w->g1, dm->eps, d, xn, flags, L.nflags);
   PLK_LAUNCHED();
+  trace_mark(1, st);
 
   g.epi = EPI_QKV;
   g.K = d;
@@ -303,8 +312,10 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   g.k_cache = Kc;
   g.v_cache = Vc;
   PLK_TRY(launch_gemm_tc(tW_qkv, tX_xn, g, st));
+  trace_mark(2, st);
 
   PLK_TRY(launch_attention_bf16(dm, q, Kc, Vc, a, seg, st));
+  trace_mark(3, st);
 
   g.epi = EPI_O;
   g.K = d;
@@ -312,10 +323,12 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   g.x_in = X;
   g.h32 = h32;
   PLK_TRY(launch_gemm_tc(tW_o, tX_a, g, st));
+  trace_mark(4, st);
 
   rmsnorm_rows_kernel<float, __nv_bfloat16, __nv_bfloat16><<<Mcap, 256, 0, st>>>(
       h32, nullptr, seg, B, (const __nv_bfloat16*)w->g2, dm->eps, d, hn, nullptr, 0);
   PLK_LAUNCHED();
+  trace_mark(5, st);
 
   g.epi = EPI_GU;
   g.K = d;
@@ -323,12 +336,14 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   g.gu_F = F;
   g.act_out = act;
   PLK_TRY(launch_gemm_tc(tW_gu, tX_hn, g, st));
+  trace_mark(6, st);
 
   g.epi = EPI_DOWN;
   g.K = F;
   g.ftiles = d / kGemmBM;
   g.y_cache = Y;
   PLK_TRY(launch_gemm_tc(tW_down, tX_act, g, st));
+  trace_mark(7, st);
   return PLK_OK;
 }
 
