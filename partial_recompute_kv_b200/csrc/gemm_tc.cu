@@ -38,7 +38,9 @@ constexpr int kSlotFloats = kGemmBNMax * kGemmBM;  // partial tile, [col][lane]
 constexpr int kXbufStride = 33;
 constexpr size_t kOffB = (size_t)kGemmStages * kStageA;
 constexpr size_t kOffBar = kOffB + (size_t)kGemmStages * kStageB;
-constexpr size_t kOffIdx = kOffBar + 128;
+constexpr size_t kOffIdx = kOffBar + 256;
+constexpr int kRing = 8;                           // fix-up ring: 8 x 16 KB in the idle stage buffers
+constexpr int kPieceFloats = 32 * kGemmBM;         // one chunk (32 columns x 128 lanes) of a partial
 constexpr size_t kOffXbuf = kOffIdx + kGemmBNMax * 4;
 constexpr size_t kSmemUsed = kOffXbuf + 64 * kXbufStride * 4;
 constexpr size_t kSmemBytes = kSmemUsed + 1024;  // slack for 1024-byte alignment
@@ -109,6 +111,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 13);
   volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 14);
   volatile int* s_epi_abort = reinterpret_cast<volatile int*>(bars + 15);
+  uint64_t* fixbar = bars + 16;           // [8] fix-up ring
+  float* ring = reinterpret_cast<float*>(smem);
   int* s_idx = reinterpret_cast<int*>(smem + kOffIdx);
   float* xbuf = reinterpret_cast<float*>(smem + kOffXbuf);
 
@@ -127,6 +131,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[i], 128);
     }
     mbar_init(drain, 1);
+    for (int i = 0; i < kRing; ++i) mbar_init(&fixbar[i], 1);
     *s_abort = 0;
     *s_epi_abort = 0;
     fence_mbar_init();
@@ -255,7 +260,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t)(acc * kTileCols) + ((uint32_t)(q * 32) << 16);
       const int nchunks = g.ncols >> 5;
+      // Split tile owned here: the other CTAs' partials stream through a ring of
+      // 16 KB shared-memory buffers (bulk async copies, up to 128 KB in flight).
+      // This is the CTA's last segment, so the stage buffers are idle.
+      const int nother = (is_head && !is_full) ? c_last - (int)blockIdx.x : 0;
+      const int npieces = nchunks * nother;
+      auto issue_piece = [&](int p) {
+        const int c = p / nother, sl = (int)blockIdx.x + 1 + p % nother;
+        const int b = p % kRing;
+        mbar_expect_tx(&fixbar[b], kPieceFloats * 4);
+        bulk_load(ring + b * kPieceFloats, args.partials + (size_t)sl * kSlotFloats + (size_t)c * kPieceFloats,
+                  kPieceFloats * 4, &fixbar[b]);
+      };
+      int issued_hi = 0, consumed = 0;  // issued_hi is tracked by the issuing thread only
+      if (npieces > 0 && et == 0) {
+        fence_proxy_async_global();
+        for (int p = 0; p < npieces && p < kRing; ++p) issue_piece(p);
+        issued_hi = npieces < kRing ? npieces : kRing;
+      }
       for (int c = 0; c < nchunks; ++c) {
+        const int jb = c * 32;
+        // residual operands first, so their latency overlaps the TMEM drain
+        float res[32];
+        if (args.epi == EPI_O || args.epi == EPI_DOWN) {
+          const int f = g.ft * kGemmBM + lr;
+          const __nv_bfloat16* x = (const __nv_bfloat16*)args.x_in;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            res[i] = 0.f;
+            if (jb + i < g.ntok) {
+              res[i] = args.epi == EPI_O ? bf2f(x[(size_t)s_idx[jb + i] * d + f])
+                                         : __ldcg(&args.h32[(size_t)(g.tok0 + jb + i) * d + f]);
+            }
+          }
+        }
         uint32_t r[32];
         tmem_ld32(taddr + (uint32_t)(c * 32), r);
         tmem_ld_wait();
@@ -268,14 +306,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int i = 0; i < 32; ++i) slot[(c * 32 + i) * kGemmBM + lr] = v[i];
           continue;
         }
-        if (!is_full) {
-          for (int sl = (int)blockIdx.x + 1; sl <= c_last; ++sl) {
-            const float* slot = args.partials + (size_t)sl * kSlotFloats;
+        for (int so = 0; so < nother; ++so) {
+          const int p = c * nother + so, b = p % kRing;
+          if (!*s_abort && !mbar_wait(&fixbar[b], (uint32_t)((p / kRing) & 1))) *s_abort = 1;
+          if (!*s_abort) {
+            consumed = p + 1;
+            const float* buf = ring + b * kPieceFloats;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] += __ldcg(&slot[(c * 32 + i) * kGemmBM + lr]);
+            for (int i = 0; i < 32; ++i) v[i] += buf[i * kGemmBM + lr];
+          }
+          named_bar_sync(1, 128);  // every thread is done with buffer b
+          if (et == 0 && p + kRing < npieces && !*s_abort) {
+            issue_piece(p + kRing);
+            issued_hi = p + kRing + 1;
           }
         }
-        const int jb = c * 32;
         if (args.epi == EPI_QKV) {
           const int f = g.ft * kGemmBM + lr;
           const int part = f / d, col = f - part * d;
@@ -290,14 +335,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         } else if (args.epi == EPI_O) {
           const int f = g.ft * kGemmBM + lr;
-          const __nv_bfloat16* x = (const __nv_bfloat16*)args.x_in;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (jb + i < g.ntok) {
-              const size_t tok = (size_t)(g.tok0 + jb + i);
-              args.h32[tok * d + f] = v[i] + bf2f(x[(size_t)s_idx[jb + i] * d + f]);
-            }
-          }
+          for (int i = 0; i < 32; ++i)
+            if (jb + i < g.ntok) args.h32[(size_t)(g.tok0 + jb + i) * d + f] = v[i] + res[i];
         } else if (args.epi == EPI_GU) {
           if (q >= 2) {
 #pragma unroll
@@ -321,18 +361,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int f = g.ft * kGemmBM + lr;
           __nv_bfloat16* y = (__nv_bfloat16*)args.y_cache;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (jb + i < g.ntok) {
-              const size_t tok = (size_t)(g.tok0 + jb + i);
-              y[(size_t)s_idx[jb + i] * d + f] = f2bf(args.h32[tok * d + f] + v[i]);
-            }
-          }
+          for (int i = 0; i < 32; ++i)
+            if (jb + i < g.ntok) y[(size_t)s_idx[jb + i] * d + f] = f2bf(res[i] + v[i]);
         }
+      }
+      if (et == 0 && *s_abort) {
+        // bounded wait for the fix-up copies still in flight before the CTA exits
+        for (int p = consumed; p < issued_hi; ++p) (void)mbar_wait(&fixbar[p % kRing], (uint32_t)((p / kRing) & 1));
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
       if (!is_head) {
         __threadfence();
+        fence_proxy_async_global();  // the owner reads this partial with bulk copies
         named_bar_sync(1, 128);
         if (et == 0) red_release_add_u32(&args.flags[g.t], 1u);
       } else if (!is_full) {

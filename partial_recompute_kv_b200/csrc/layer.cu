@@ -147,6 +147,123 @@ __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const Tin* __restrict
   for (int c = threadIdx.x; c < d; c += blockDim.x) o[c] = from_f<Tout>(to_f(x[c]) * inv * to_f(g[c]));
 }
 
+// Same as rmsnorm_rows_kernel with the row held in registers: each thread loads
+// up to NV 16-byte vectors in one batch (so the loads overlap), squares and sums
+// them, and writes its outputs from registers.  Requires d % (16/sizeof(Tin)) == 0
+// and d <= NV * 256 * (16/sizeof(Tin)).
+template <typename T>
+struct Vec16;
+template <>
+struct Vec16<__nv_bfloat16> {
+  static constexpr int E = 8;
+  __device__ static void unpack(const uint4& u, float* f) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 t = __bfloat1622float2(h[i]);
+      f[2 * i] = t.x;
+      f[2 * i + 1] = t.y;
+    }
+  }
+};
+template <>
+struct Vec16<float> {
+  static constexpr int E = 4;
+  __device__ static void unpack(const uint4& u, float* f) {
+    f[0] = __uint_as_float(u.x);
+    f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z);
+    f[3] = __uint_as_float(u.w);
+  }
+};
+
+// Stores E consecutive outputs with one (or two) vector stores.
+template <typename T, int E>
+__device__ __forceinline__ void store_vec(T* dst, const float* y);
+template <>
+__device__ __forceinline__ void store_vec<__nv_bfloat16, 8>(__nv_bfloat16* dst, const float* y) {
+  uint4 u;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(y[2 * i], y[2 * i + 1]);
+  *reinterpret_cast<uint4*>(dst) = u;
+}
+template <>
+__device__ __forceinline__ void store_vec<__nv_bfloat16, 4>(__nv_bfloat16* dst, const float* y) {
+  uint2 u;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+  h[0] = __floats2bfloat162_rn(y[0], y[1]);
+  h[1] = __floats2bfloat162_rn(y[2], y[3]);
+  *reinterpret_cast<uint2*>(dst) = u;
+}
+template <>
+__device__ __forceinline__ void store_vec<float, 4>(float* dst, const float* y) {
+  *reinterpret_cast<float4*>(dst) = make_float4(y[0], y[1], y[2], y[3]);
+}
+template <>
+__device__ __forceinline__ void store_vec<float, 8>(float* dst, const float* y) {
+  reinterpret_cast<float4*>(dst)[0] = make_float4(y[0], y[1], y[2], y[3]);
+  reinterpret_cast<float4*>(dst)[1] = make_float4(y[4], y[5], y[6], y[7]);
+}
+
+template <typename Tin, typename Tg, typename Tout, int NV>
+__global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict__ X, const int32_t* __restrict__ idx,
+                                                          const int32_t* __restrict__ seg_ptr, int B,
+                                                          const Tg* __restrict__ g, float eps, int d,
+                                                          Tout* __restrict__ out, uint32_t* flags, int nflags) {
+  constexpr int E = Vec16<Tin>::E;
+  __shared__ float sh[33];
+  if (flags && blockIdx.x == 0)
+    for (int i = threadIdx.x; i < nflags; i += blockDim.x) flags[i] = 0u;
+  const int M = seg_ptr[B];
+  const int j = blockIdx.x;
+  if (j >= M) return;
+  const size_t row = idx ? (size_t)idx[j] : (size_t)j;
+  const uint4* xv = reinterpret_cast<const uint4*>(X + row * d);
+  const int nvec = d / E;
+  uint4 buf[NV];
+#pragma unroll
+  for (int u = 0; u < NV; ++u) {
+    const int vi = threadIdx.x + u * 256;
+    if (vi < nvec) buf[u] = __ldg(xv + vi);
+  }
+  float ss = 0.f;
+#pragma unroll
+  for (int u = 0; u < NV; ++u) {
+    if (threadIdx.x + u * 256 < nvec) {
+      float f[E];
+      Vec16<Tin>::unpack(buf[u], f);
+#pragma unroll
+      for (int e = 0; e < E; ++e) ss = fmaf(f[e], f[e], ss);
+    }
+  }
+  ss = block_sum_f(ss, sh);
+  const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+  Tout* o = out + (size_t)j * d;
+#pragma unroll
+  for (int u = 0; u < NV; ++u) {
+    const int vi = threadIdx.x + u * 256;
+    if (vi < nvec) {
+      float f[E];
+      Vec16<Tin>::unpack(buf[u], f);
+#pragma unroll
+      for (int e = 0; e < E; ++e) f[e] = f[e] * inv * to_f(g[vi * E + e]);
+      store_vec<Tout, E>(o + vi * E, f);
+    }
+  }
+}
+
+// Picks the register-resident kernel when the row fits, else the looping one.
+template <typename Tin, typename Tg, typename Tout>
+static void launch_rmsnorm(const Tin* X, const int32_t* idx, const int32_t* seg, int B, const Tg* g, float eps,
+                           int d, Tout* out, uint32_t* flags, int nflags, int grid, cudaStream_t st) {
+  constexpr int E = Vec16<Tin>::E;
+  if (d % E == 0 && d <= 4 * 256 * E)
+    rmsnorm_vec_kernel<Tin, Tg, Tout, 4><<<grid, 256, 0, st>>>(X, idx, seg, B, g, eps, d, out, flags, nflags);
+  else
+    rmsnorm_rows_kernel<Tin, Tg, Tout><<<grid, 256, 0, st>>>(X, idx, seg, B, g, eps, d, out, flags, nflags);
+}
+
 __global__ void fill_identity_kernel(int32_t* iota, int32_t* seg, int B, int N) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i < B * N) iota[i] = i;
@@ -249,16 +366,15 @@ static int run_layer_f32(const plk_dims* dm, const plk_weights* w, const float* 
     dim3 grid(ceil_div(Nout, 64), ceil_div(Mcap, 64));
     gemm_f32_kernel<<<grid, 256, 0, st>>>(A, (const float*)Wt, c32, Nout, K, seg, B);
   };
-  rmsnorm_rows_kernel<float, float, float><<<rows, 256, 0, st>>>(X, idx, seg, B, (const float*)w->g1, dm->eps, d, xn,
-                                                          nullptr, 0);
+  launch_rmsnorm<float, float, float>(X, idx, seg, B, (const float*)w->g1, dm->eps, d, xn, nullptr, 0, Mcap, st);
   gemm(xn, w->w_qkv, 3 * d, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_QKV, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y);
   PLK_LAUNCHED();
   PLK_TRY(launch_attention_f32(dm, q, Kc, Vc, a, seg, Mcap, st));
   gemm(a, w->w_o, d, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_O, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y);
-  rmsnorm_rows_kernel<float, float, float><<<rows, 256, 0, st>>>(h32, nullptr, seg, B, (const float*)w->g2, dm->eps, d,
-                                                          hn, nullptr, 0);
+  launch_rmsnorm<float, float, float>(h32, nullptr, seg, B, (const float*)w->g2, dm->eps, d, hn, nullptr, 0, Mcap,
+                                      st);
   gemm(hn, w->w_gu, 2 * F, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_GU, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y);
   gemm(act, w->w_down, d, F);
@@ -300,8 +416,8 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   g.nslots = L.nslots;
 
   trace_mark(0, st);
-  rmsnorm_rows_kernel<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16><<<Mcap, 256, 0, st>>>(
-      X, idx, seg, B, (const __nv_bfloat16*)w->g1, dm->eps, d, xn, flags, L.nflags);
+  launch_rmsnorm<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(X, idx, seg, B, (const __nv_bfloat16*)w->g1, dm->eps, d,
+                                                              xn, flags, L.nflags, Mcap, st);
   PLK_LAUNCHED();
   trace_mark(1, st);
 
@@ -325,8 +441,8 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   PLK_TRY(launch_gemm_tc(tW_o, tX_a, g, st));
   trace_mark(4, st);
 
-  rmsnorm_rows_kernel<float, __nv_bfloat16, __nv_bfloat16><<<Mcap, 256, 0, st>>>(
-      h32, nullptr, seg, B, (const __nv_bfloat16*)w->g2, dm->eps, d, hn, nullptr, 0);
+  launch_rmsnorm<float, __nv_bfloat16, __nv_bfloat16>(h32, nullptr, seg, B, (const __nv_bfloat16*)w->g2, dm->eps, d, hn,
+                                                      nullptr, 0, Mcap, st);
   PLK_LAUNCHED();
   trace_mark(5, st);
 

@@ -8,7 +8,11 @@
 // bf16: one CTA per 128 rows, X tile (128 x 64) and Ut tile (r x 64) staged by
 // TMA, tcgen05.mma into an fp32 TMEM accumulator of r columns, and the row-wise
 // distance computed straight from TMEM (thread = row) against the cached proxy.
-// The kernel streams X once from HBM; Ut stays in L2.
+// The kernel streams X once from HBM; Ut stays in L2.  When there are too few
+// 128-row tiles to fill the GPU, the K dimension is split over a thread-block
+// cluster of S CTAs: each CTA parks its partial projection in its own shared
+// memory and then finishes 128/S of the rows, summing the S partials through
+// distributed shared memory (no global scratch).
 // fp32: a SIMT kernel, one warp per row.
 #include "plk_common.cuh"
 #include "plk_internal.h"
@@ -16,7 +20,7 @@
 namespace plk {
 
 namespace {
-constexpr int kScStages = 4;
+constexpr int kScStages = 3;
 constexpr int kScA = 128 * 64 * 2;  // 16 KB of X per stage
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
@@ -48,7 +52,10 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row0 = blockIdx.x * 128;
-  const int nkb = d / 64;
+  const int S = gridDim.y, ks = blockIdx.y;  // K slices = cluster size (1 = no cluster)
+  const int nkb_all = d / 64;
+  const int kb0 = ks * nkb_all / S;
+  const int nkb = (ks + 1) * nkb_all / S - kb0;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kScStages; ++i) {
       mbar_init(&full[i], 1);
@@ -79,8 +86,8 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
         }
         uint8_t* a = smem + stage * stage_bytes;
         mbar_expect_tx(&full[stage], (uint32_t)(kScA + stageB));
-        tma_load_2d(a, &tmX, kb * 64, row0, &full[stage]);
-        tma_load_2d(a + kScA, &tmU, kb * 64, 0, &full[stage]);
+        tma_load_2d(a, &tmX, (kb0 + kb) * 64, row0, &full[stage]);
+        tma_load_2d(a + kScA, &tmU, (kb0 + kb) * 64, 0, &full[stage]);
         ++issued;
         if (++stage == kScStages) {
           stage = 0;
@@ -122,9 +129,58 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
     __syncwarp();
   }
 
-  // epilogue: thread = row (TMEM lane)
   const bool ok = mbar_wait(done, 0);
   tc_fence_after();
+  if (S > 1) {
+    // split-K over the cluster: partial [128 rows][r] (stride r+1) in the idle stage buffers
+    float* part = reinterpret_cast<float*>(smem);
+    const int pstride = r + 1;
+    const int rl = warp * 32 + lane;
+    const bool good = __all_sync(0xffffffffu, ok && !*s_abort);
+    for (int c0 = 0; c0 < r; c0 += 16) {
+      uint32_t v[16];
+      if (good) {
+        tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
+        tmem_ld_wait();
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) part[rl * pstride + c0 + i] = good ? __uint_as_float(v[i]) : 0.f;
+    }
+    tc_fence_before();
+    cluster_sync_all();
+    const int rows_per = 128 / S, tpr = 128 / rows_per;
+    const int lrow = ks * rows_per + (int)threadIdx.x / tpr, sub = (int)threadIdx.x % tpr;
+    const int row = row0 + lrow;
+    const uint32_t pbase = smem_u32(part + lrow * pstride);
+    float dot = 0.f, pp = 0.f, cc = 0.f, dd = 0.f;
+    for (int c = sub; c < r; c += tpr) {
+      float p = 0.f;
+      for (int sr = 0; sr < S; ++sr) p += ld_dsmem_f32(dsmem_addr(pbase + 4u * c, (uint32_t)sr));
+      if (row < rows) {
+        const float cv = __ldg(cache + (size_t)row * r + c);
+        dot = fmaf(p, cv, dot);
+        pp = fmaf(p, p, pp);
+        cc = fmaf(cv, cv, cc);
+        dd = fmaf(p - cv, p - cv, dd);
+        if (pout) pout[(size_t)row * r + c] = p;
+      }
+    }
+    for (int o = 1; o < tpr; o <<= 1) {
+      dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      pp += __shfl_xor_sync(0xffffffffu, pp, o);
+      cc += __shfl_xor_sync(0xffffffffu, cc, o);
+      dd += __shfl_xor_sync(0xffffffffu, dd, o);
+    }
+    if (sub == 0 && row < rows)
+      score[row] = metric == PLK_METRIC_COS ? dot / fmaxf(sqrtf(pp) * sqrtf(cc), 1e-30f) : sqrtf(dd);
+    cluster_sync_all();  // peers may still be reading this CTA's partial
+    if (warp == 2) {
+      tc_fence_after();
+      tmem_dealloc(tmem, (uint32_t)tmem_cols);
+    }
+    return;
+  }
+  // epilogue: thread = row (TMEM lane)
   const int row = row0 + warp * 32 + lane;
   float dot = 0.f, pp = 0.f, cc = 0.f, dd = 0.f;
   // tcgen05.ld is warp-collective: take the decision once per warp
@@ -234,8 +290,30 @@ int launch_score(const plk_dims* dims, const void* X, const void* Ut, int r, con
       return PLK_ERR_CUDA;
     attr_smem[dev] = smem;
   }
-  score_tc_kernel<<<ceil_div(rows, 128), 128, smem, st>>>(tmX, tmU, rows, d, r, tcols, proxy_cache, proxy_out,
-                                                          score_out, metric);
+  // K slices: grow the cluster while it still fits the GPU and leaves >= 2 k-blocks per slice
+  const int tiles = ceil_div(rows, 128), nkb = d / 64;
+  int S = 1;
+  while (S < 8 && tiles * S * 2 <= device_sm_count() && nkb % (S * 2) == 0 && nkb / (S * 2) >= 2) S *= 2;
+  if (S == 1) {
+    score_tc_kernel<<<tiles, 128, smem, st>>>(tmX, tmU, rows, d, r, tcols, proxy_cache, proxy_out, score_out,
+                                              metric);
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(tiles, S, 1);
+    cfg.blockDim = dim3(128, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 1;
+    at[0].val.clusterDim.y = S;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, score_tc_kernel, tmX, tmU, rows, d, r, tcols, proxy_cache, proxy_out, score_out,
+                           metric) != cudaSuccess)
+      return PLK_ERR_CUDA;
+  }
   return cudaPeekAtLastError() == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;
 }
 

@@ -114,65 +114,98 @@ __device__ __forceinline__ uint32_t pref_key(float s, bool largest) {
 }
 
 // One CTA per sequence: among rows with lock_in == 0 keep the k most preferred
-// (ties to the lower index) and lock every other row.  Radix select on 8-bit
-// digits finds the k-th key; an ordered block scan breaks ties.
-__global__ void __launch_bounds__(kSelThreads) topk_kernel(const float* __restrict__ score,
-                                                           const uint8_t* lock_in, uint8_t* lock_out, int N,
-                                                           int k, int largest) {
+// (ties to the lower index), lock every other row, and compact the kept rows.
+// Radix select on 8-bit digits finds the k-th key (warp-parallel bin search);
+// an ordered block scan breaks ties and produces the ascending indices.  The
+// output offset of sequence b is sum_{b'<b} min(k, candidates(b')), which each
+// CTA computes from lock_in itself; when lock_in and lock_out alias, a
+// sequence's min(k, unlocked) count is the same before, during and after its
+// CTA rewrites it, so no inter-CTA ordering is needed.
+__global__ void __launch_bounds__(kSelThreads) topk_compact_kernel(const float* __restrict__ score,
+                                                                   const uint8_t* lock_in, uint8_t* lock_out,
+                                                                   int N, int k, int largest,
+                                                                   int32_t* __restrict__ idx_out,
+                                                                   int32_t* __restrict__ seg_ptr) {
   __shared__ int hist[256];
   __shared__ int sh[33];
   __shared__ uint32_t s_prefix;
   __shared__ int s_remaining;
-  const long long base = (long long)blockIdx.x * N;
+  const int b = blockIdx.x;
+  const long long base = (long long)b * N;
   const bool lg = largest != 0;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int offset = 0;
+  if (k > 0) {
+    for (int bp = 0; bp < b; ++bp) {
+      int c = 0;
+      for (int i = threadIdx.x; i < N; i += blockDim.x) c += lock_in[(long long)bp * N + i] ? 0 : 1;
+      offset += min(k, block_sum(c, sh));
+    }
+  }
   int c = 0;
   for (int i = threadIdx.x; i < N; i += blockDim.x) c += lock_in[base + i] ? 0 : 1;
   const int ncand = block_sum(c, sh);
-  if (k >= ncand || k <= 0) {
-    // every candidate kept (k >= ncand) or none (k <= 0)
-    __syncthreads();
-    for (int i = threadIdx.x; i < N; i += blockDim.x) {
-      const uint8_t l = lock_in[base + i];
-      lock_out[base + i] = (k > 0 && !l) ? 0 : 1;
-    }
-    return;
-  }
-  uint32_t prefix = 0, pmask = 0;
-  int remaining = k;
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int t = threadIdx.x; t < 256; t += blockDim.x) hist[t] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < N; i += blockDim.x) {
-      if (lock_in[base + i]) continue;
-      const uint32_t key = pref_key(score[base + i], lg);
-      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
-    }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      int above = 0, bin = 255;
-      for (; bin > 0; --bin) {
-        if (above + hist[bin] >= remaining) break;
-        above += hist[bin];
+  const int keep_n = k <= 0 ? 0 : min(k, ncand);
+  uint32_t kth = 0u;  // every candidate has key > 0 or == 0 (NaN); with keep-all, take all
+  int remaining = 0;
+  const bool keep_all = keep_n == ncand;
+  if (!keep_all) {
+    uint32_t prefix = 0, pmask = 0;
+    remaining = keep_n;
+    for (int pass = 0; pass < 4; ++pass) {
+      const int shift = 24 - 8 * pass;
+      for (int t = threadIdx.x; t < 256; t += blockDim.x) hist[t] = 0;
+      __syncthreads();
+      for (int i = threadIdx.x; i < N; i += blockDim.x) {
+        if (lock_in[base + i]) continue;
+        const uint32_t key = pref_key(score[base + i], lg);
+        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
       }
-      s_prefix = prefix | ((uint32_t)bin << shift);
-      s_remaining = remaining - above;
+      __syncthreads();
+      if (warp == 0) {
+        // lane l owns bins 255-8l .. 248-8l (descending); find the bin holding the
+        // remaining-th most preferred key
+        int cnt[8], tot = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          cnt[j] = hist[255 - 8 * lane - j];
+          tot += cnt[j];
+        }
+        int inc = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int n = __shfl_up_sync(0xffffffffu, inc, o);
+          if (lane >= o) inc += n;
+        }
+        int above = inc - tot;
+        if (above < remaining && remaining <= inc) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (above + cnt[j] >= remaining) {
+              s_prefix = prefix | ((uint32_t)(255 - 8 * lane - j) << shift);
+              s_remaining = remaining - above;
+              break;
+            }
+            above += cnt[j];
+          }
+        }
+      }
+      __syncthreads();
+      prefix = s_prefix;
+      remaining = s_remaining;
+      pmask |= 0xFFu << shift;
+      __syncthreads();
     }
-    __syncthreads();
-    prefix = s_prefix;
-    remaining = s_remaining;
-    pmask |= 0xFFu << shift;
-    __syncthreads();
+    kth = prefix;
   }
-  // prefix = k-th most preferred key; remaining = how many rows equal to it to keep
-  const uint32_t kth = prefix;
-  int taken_eq = 0;
+  // keep: candidates with key > kth, plus the first `remaining` with key == kth
+  int taken_eq = 0, running = 0;
   for (int c0 = 0; c0 < N; c0 += blockDim.x) {
     const int i = c0 + threadIdx.x;
     bool cand = false, eq = false, gt = false;
     if (i < N) {
       cand = lock_in[base + i] == 0;
-      if (cand) {
+      if (cand && !keep_all) {
         const uint32_t key = pref_key(score[base + i], lg);
         gt = key > kth;
         eq = key == kth;
@@ -180,11 +213,17 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(const float* __restri
     }
     int total;
     const int r = block_rank(eq ? 1 : 0, sh, &total);
-    if (i < N) {
-      const bool keep = cand && (gt || (eq && taken_eq + r < remaining));
-      lock_out[base + i] = keep ? 0 : 1;
-    }
+    const bool keep = cand && (keep_all ? keep_n > 0 : (gt || (eq && taken_eq + r < remaining)));
     taken_eq += total;
+    if (i < N) lock_out[base + i] = keep ? 0 : 1;
+    int kt;
+    const int kr = block_rank(keep ? 1 : 0, sh, &kt);
+    if (keep) idx_out[offset + running + kr] = (int32_t)(base + i);
+    running += kt;
+  }
+  if (threadIdx.x == 0) {
+    seg_ptr[b + 1] = offset + running;
+    if (b == 0) seg_ptr[0] = 0;
   }
 }
 
@@ -192,9 +231,8 @@ int launch_select(const plk_dims* dims, const float* score, const uint8_t* lock_
                   int mode, float tau, int k, int32_t* idx_out, int32_t* seg_ptr, cudaStream_t st) {
   const int B = dims->B, N = dims->N;
   if (mode == PLK_SEL_TOPK_LARGEST || mode == PLK_SEL_TOPK_SMALLEST) {
-    topk_kernel<<<B, kSelThreads, 0, st>>>(score, lock_in, lock_out, N, k, mode == PLK_SEL_TOPK_LARGEST);
-    if (cudaPeekAtLastError() != cudaSuccess) return PLK_ERR_CUDA;
-    compact_kernel<<<B, kSelThreads, 0, st>>>(-1, score, lock_out, lock_out, N, tau, idx_out, seg_ptr);
+    topk_compact_kernel<<<B, kSelThreads, 0, st>>>(score, lock_in, lock_out, N, k, mode == PLK_SEL_TOPK_LARGEST,
+                                                   idx_out, seg_ptr);
   } else {
     compact_kernel<<<B, kSelThreads, 0, st>>>(mode, score, lock_in, lock_out, N, tau, idx_out, seg_ptr);
   }
