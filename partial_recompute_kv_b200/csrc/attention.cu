@@ -17,6 +17,8 @@
 // fp32: one thread per (query row, head), online softmax, SIMT.
 #include <math.h>
 
+#include <algorithm>
+
 #include "plk_common.cuh"
 #include "plk_internal.h"
 
@@ -63,16 +65,37 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uin
 }
 }  // namespace
 
+// Number of key splits for the current active set: enough CTAs to cover the
+// GPU twice, at most smax.  Computed identically by the attention and combine
+// kernels from seg_ptr (device-side M, no host synchronisation).
+__device__ __forceinline__ int attn_splits(const int32_t* seg_ptr, int B, int H, int smax, int nsm) {
+  int qtiles = 0;
+  for (int b = 0; b < B; ++b) qtiles += ceil_div(seg_ptr[b + 1] - seg_ptr[b], kAttBQ);
+  if (qtiles == 0) return 1;
+  const int want = ceil_div(2 * nsm, qtiles * H);
+  return max(1, min(smax, want));
+}
+
+// Split partials: o_part[s][row][d] (unnormalised, fp32) and ml[s][row][h] = (max, sum)
+// in the log2 domain; rows are compact active-row indices below part_rows.
+struct AttnSplit {
+  float* o_part;
+  float2* ml;
+  int smax, part_rows, nsm;
+};
+
 __global__ void __launch_bounds__(kAttThreads) attn_bf16_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                 const __grid_constant__ CUtensorMap tmV,
                                                                 const __nv_bfloat16* __restrict__ Q,
                                                                 __nv_bfloat16* __restrict__ Aout,
-                                                                const int32_t* __restrict__ seg_ptr, int N, int d,
-                                                                float scale_log2) {
-  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+                                                                const int32_t* __restrict__ seg_ptr, int B, int N,
+                                                                int d, float scale_log2, AttnSplit sp) {
+  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z / sp.smax, split = blockIdx.z % sp.smax;
   const int seg0 = seg_ptr[b], seg1 = seg_ptr[b + 1];
   const int r0 = seg0 + qt * kAttBQ;
   if (r0 >= seg1) return;
+  const int S = attn_splits(seg_ptr, B, gridDim.y, sp.smax, sp.nsm);
+  if (split >= S) return;
   const int nrows = min(kAttBQ, seg1 - r0);
 
   extern __shared__ uint8_t smem_raw[];
@@ -85,7 +108,9 @@ __global__ void __launch_bounds__(kAttThreads) attn_bf16_kernel(const __grid_con
   volatile int* s_bad = reinterpret_cast<volatile int*>(full + 2);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int ntiles = ceil_div(N, kAttBK);
+  const int ntiles_all = ceil_div(N, kAttBK);
+  const int t0 = split * ntiles_all / S;                 // this split's key tiles [t0, t0 + ntiles)
+  const int ntiles = (split + 1) * ntiles_all / S - t0;
   const int hcol = h * kAttHD;
 
   if (tid == 0) {
@@ -96,7 +121,7 @@ __global__ void __launch_bounds__(kAttThreads) attn_bf16_kernel(const __grid_con
   }
   __syncthreads();
   auto issue = [&](int j, int s) {
-    const int y = b * N + j * kAttBK;
+    const int y = b * N + (t0 + j) * kAttBK;
     mbar_expect_tx(&full[s], 2 * kAttTile);
     tma_load_2d(sK + s * kAttTile, &tmK, hcol, y, &full[s]);
     tma_load_2d(sK + s * kAttTile + 8192, &tmK, hcol + 64, y, &full[s]);
@@ -157,7 +182,7 @@ __global__ void __launch_bounds__(kAttThreads) attn_bf16_kernel(const __grid_con
         mma16816(sc[2 * np + 1], qa[ks], kr[2], kr[3]);
       }
     }
-    const int key0 = j * kAttBK;
+    const int key0 = (t0 + j) * kAttBK;
     if (key0 + kAttBK > N) {
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt)
@@ -225,14 +250,51 @@ __global__ void __launch_bounds__(kAttThreads) attn_bf16_kernel(const __grid_con
     float l = l_r[hf];
     l += __shfl_xor_sync(0xffffffffu, l, 1);
     l += __shfl_xor_sync(0xffffffffu, l, 2);
-    const float inv = 1.0f / l;
     const int row = warp * 16 + (lane >> 2) + 8 * hf;
-    if (row < nrows) {
+    if (row >= nrows) continue;
+    if (S == 1) {
+      const float inv = 1.0f / l;
       __nv_bfloat16* dst = Aout + (size_t)(r0 + row) * d + hcol + 2 * cq;
 #pragma unroll
       for (int nt = 0; nt < 16; ++nt)
         *reinterpret_cast<uint32_t*>(dst + nt * 8) = pack_bf16(o[nt][2 * hf] * inv, o[nt][2 * hf + 1] * inv);
+    } else {
+      float* dst = sp.o_part + ((size_t)split * sp.part_rows + (r0 + row)) * d + hcol + 2 * cq;
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt)
+        *reinterpret_cast<float2*>(dst + nt * 8) = make_float2(o[nt][2 * hf], o[nt][2 * hf + 1]);
+      if (cq == 0) sp.ml[((size_t)split * sp.part_rows + (r0 + row)) * gridDim.y + h] = make_float2(m_r[hf], l);
     }
+  }
+}
+
+// out[row, h] = sum_s 2^(m_s - m) o_s / sum_s 2^(m_s - m) l_s, one CTA per active row.
+__global__ void __launch_bounds__(256) attn_combine_kernel(const int32_t* __restrict__ seg_ptr, int B, int H,
+                                                           int d, AttnSplit sp, __nv_bfloat16* __restrict__ Aout) {
+  const int j = blockIdx.x;
+  if (j >= seg_ptr[B]) return;
+  const int S = attn_splits(seg_ptr, B, H, sp.smax, sp.nsm);
+  if (S == 1) return;
+  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+    const int h = c / kAttHD;
+    float m = -INFINITY;
+    for (int s = 0; s < S; ++s) m = fmaxf(m, sp.ml[((size_t)s * sp.part_rows + j) * H + h].x);
+    float l = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < S; ++s) {
+      const float2 ml = sp.ml[((size_t)s * sp.part_rows + j) * H + h];
+      const float w = exp2f(ml.x - m);
+      l = fmaf(w, ml.y, l);
+      const float4 o = *reinterpret_cast<const float4*>(sp.o_part + ((size_t)s * sp.part_rows + j) * d + c);
+      acc[0] = fmaf(w, o.x, acc[0]);
+      acc[1] = fmaf(w, o.y, acc[1]);
+      acc[2] = fmaf(w, o.z, acc[2]);
+      acc[3] = fmaf(w, o.w, acc[3]);
+    }
+    const float inv = 1.0f / l;
+    uint2 u;
+    u.x = pack_bf16(acc[0] * inv, acc[1] * inv);
+    u.y = pack_bf16(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(Aout + (size_t)j * d + c) = u;
   }
 }
 
@@ -272,8 +334,15 @@ __global__ void attn_f32_kernel(const float* __restrict__ Q, const float* __rest
   for (int c = 0; c < HD; ++c) A[(size_t)j * d + h * HD + c] = o[c] * inv;
 }
 
+int attn_split_rows(const plk_dims* dims, int num_sms) {
+  // splits are used only while q-tiles x heads < 2 x SMs, so fewer active rows
+  const int rows = ceil_div(2 * num_sms, dims->H) * kAttBQ;
+  return std::min(dims->B * dims->N, rows);
+}
+
 int launch_attention_bf16(const plk_dims* dims, const void* q, const void* K_cache, const void* V_cache,
-                          void* a_out, const int32_t* seg_ptr, cudaStream_t st) {
+                          void* a_out, const int32_t* seg_ptr, float* o_part, void* ml, int smax, int part_rows,
+                          int num_sms, cudaStream_t st) {
   const int B = dims->B, N = dims->N, d = dims->d, H = dims->H;
   CUtensorMap tmK, tmV;
   if (make_tmap_bf16(&tmK, K_cache, (uint64_t)B * N, (uint64_t)d, 64) != PLK_OK) return PLK_ERR_CUDA;
@@ -288,9 +357,14 @@ int launch_attention_bf16(const plk_dims* dims, const void* q, const void* K_cac
     attr_done[dev] = 1;
   }
   const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->hd));
-  dim3 grid(ceil_div(N, kAttBQ), H, B);
+  AttnSplit sp{o_part, (float2*)ml, std::max(1, std::min(smax, ceil_div(N, kAttBK))), part_rows, num_sms};
+  dim3 grid(ceil_div(N, kAttBQ), H, B * sp.smax);
   attn_bf16_kernel<<<grid, kAttThreads, kAttSmem, st>>>(tmK, tmV, (const __nv_bfloat16*)q, (__nv_bfloat16*)a_out,
-                                                        seg_ptr, N, d, scale_log2);
+                                                        seg_ptr, B, N, d, scale_log2, sp);
+  if (cudaPeekAtLastError() != cudaSuccess) return PLK_ERR_CUDA;
+  if (sp.smax > 1) {
+    attn_combine_kernel<<<part_rows, 256, 0, st>>>(seg_ptr, B, H, d, sp, (__nv_bfloat16*)a_out);
+  }
   return cudaPeekAtLastError() == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;
 }
 

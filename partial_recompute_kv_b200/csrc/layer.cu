@@ -66,6 +66,9 @@ Workspace workspace_layout(const plk_dims* dm, int num_sms) {
     w.nflags = (int)(ft * ttiles);
     w.partials = take((size_t)num_sms * kGemmBNMax * kGemmBM * 4);
     w.flags = take(4 * (size_t)w.nflags);
+    w.att_rows = attn_split_rows(dm, num_sms);
+    w.att_o = take((size_t)kAttSplitMax * w.att_rows * d * 4);
+    w.att_ml = take((size_t)kAttSplitMax * w.att_rows * dm->H * 8);
   } else {
     w.c32 = take(4 * Mcap * std::max((size_t)3 * d, 2 * F));
   }
@@ -430,7 +433,8 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   PLK_TRY(launch_gemm_tc(tW_qkv, tX_xn, g, st));
   trace_mark(2, st);
 
-  PLK_TRY(launch_attention_bf16(dm, q, Kc, Vc, a, seg, st));
+  PLK_TRY(launch_attention_bf16(dm, q, Kc, Vc, a, seg, (float*)(ws + L.att_o), ws + L.att_ml, kAttSplitMax,
+                                L.att_rows, L.nslots, st));
   trace_mark(3, st);
 
   g.epi = EPI_O;

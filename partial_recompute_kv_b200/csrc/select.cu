@@ -146,10 +146,11 @@ __global__ void __launch_bounds__(kSelThreads) topk_compact_kernel(const float* 
   for (int i = threadIdx.x; i < N; i += blockDim.x) c += lock_in[base + i] ? 0 : 1;
   const int ncand = block_sum(c, sh);
   const int keep_n = k <= 0 ? 0 : min(k, ncand);
-  uint32_t kth = 0u;  // every candidate has key > 0 or == 0 (NaN); with keep-all, take all
+  uint32_t kth = 0u;
   int remaining = 0;
-  const bool keep_all = keep_n == ncand;
-  if (!keep_all) {
+  const bool keep_none = keep_n == 0;
+  const bool keep_all = !keep_none && keep_n == ncand;
+  if (!keep_none && !keep_all) {
     uint32_t prefix = 0, pmask = 0;
     remaining = keep_n;
     for (int pass = 0; pass < 4; ++pass) {
@@ -205,7 +206,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_compact_kernel(const float* 
     bool cand = false, eq = false, gt = false;
     if (i < N) {
       cand = lock_in[base + i] == 0;
-      if (cand && !keep_all) {
+      if (cand && !keep_all && !keep_none) {
         const uint32_t key = pref_key(score[base + i], lg);
         gt = key > kth;
         eq = key == kth;
@@ -213,7 +214,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_compact_kernel(const float* 
     }
     int total;
     const int r = block_rank(eq ? 1 : 0, sh, &total);
-    const bool keep = cand && (keep_all ? keep_n > 0 : (gt || (eq && taken_eq + r < remaining)));
+    const bool keep = cand && !keep_none && (keep_all || gt || (eq && taken_eq + r < remaining));
     taken_eq += total;
     if (i < N) lock_out[base + i] = keep ? 0 : 1;
     int kt;
