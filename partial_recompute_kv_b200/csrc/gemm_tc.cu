@@ -21,7 +21,7 @@
 //    to its accumulator and runs the epilogue.  Every output element is written
 //    once by a fused epilogue, no output buffer needs zeroing.
 //  * Epilogues: QKV (Q compact; K and V scattered straight into the cache rows,
-//    the K/V refresh of SureLock Sec. 2), O (+ residual, fp32 h), GU (tile =
+//    the K/V refresh of SureLock Sec. 2), O (h += a W_o^T, fp32), GU (tile =
 //    64 gate rows + 64 up rows of the same features; silu(g) * u), DOWN
 //    (+ fp32 residual, scattered into the output cache rows).
 #include "plk_common.cuh"
@@ -34,15 +34,16 @@ namespace {
 constexpr int kStageA = kGemmBM * kGemmBK * 2;     // 16 KB
 constexpr int kStageB = kGemmBNMax * kGemmBK * 2;  // 32 KB
 constexpr int kTileCols = 256;                     // TMEM columns per accumulator buffer
-constexpr int kSlotFloats = kGemmBNMax * kGemmBM;  // partial tile, [col][lane]
+constexpr int kSlotFloats = kGemmBNMax * kGemmBM;  // partial tile, [lane quarter][col][32 lanes]
 constexpr int kXbufStride = 33;
 constexpr size_t kOffB = (size_t)kGemmStages * kStageA;
 constexpr size_t kOffBar = kOffB + (size_t)kGemmStages * kStageB;
-constexpr size_t kOffIdx = kOffBar + 256;
-constexpr int kRing = 8;                           // fix-up ring: 8 x 16 KB in the idle stage buffers
-constexpr int kPieceFloats = 32 * kGemmBM;         // one chunk (32 columns x 128 lanes) of a partial
+constexpr size_t kOffIdx = kOffBar + 512;
+constexpr int kRing = 8;                           // fix-up ring per epilogue warp: 8 pieces of 4 KB
+constexpr int kPieceFloats = 32 * 32;              // one warp's chunk (32 columns x 32 lanes) of a partial
+constexpr int kQuarterFloats = kGemmBNMax * 32;    // one lane quarter of a partial slot
 constexpr size_t kOffXbuf = kOffIdx + kGemmBNMax * 4;
-constexpr size_t kSmemUsed = kOffXbuf + 64 * kXbufStride * 4;
+constexpr size_t kSmemUsed = kOffXbuf + 2 * 64 * kXbufStride * 4;  // double-buffered gate/up exchange
 constexpr size_t kSmemBytes = kSmemUsed + 1024;  // slack for 1024-byte alignment
 
 struct Sched {
@@ -111,7 +112,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 13);
   volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 14);
   volatile int* s_epi_abort = reinterpret_cast<volatile int*>(bars + 15);
-  uint64_t* fixbar = bars + 16;           // [8] fix-up ring
+  uint64_t* fixbar = bars + 16;           // [4 warps][8] fix-up rings
+  uint64_t* epi_done = bars + 48;         // epilogue warps finished with TMEM
   float* ring = reinterpret_cast<float*>(smem);
   int* s_idx = reinterpret_cast<int*>(smem + kOffIdx);
   float* xbuf = reinterpret_cast<float*>(smem + kOffXbuf);
@@ -131,7 +133,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&tempty[i], 128);
     }
     mbar_init(drain, 1);
-    for (int i = 0; i < kRing; ++i) mbar_init(&fixbar[i], 1);
+    for (int i = 0; i < 4 * kRing; ++i) mbar_init(&fixbar[i], 1);
+    mbar_init(epi_done, 128);
     *s_abort = 0;
     *s_epi_abort = 0;
     fence_mbar_init();
@@ -260,38 +263,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_after();
       const uint32_t taddr = tmem_base + (uint32_t)(acc * kTileCols) + ((uint32_t)(q * 32) << 16);
       const int nchunks = g.ncols >> 5;
-      // Split tile owned here: the other CTAs' partials stream through a ring of
-      // 16 KB shared-memory buffers (bulk async copies, up to 128 KB in flight).
-      // This is the CTA's last segment, so the stage buffers are idle.
+      // Split tile owned here: each warp streams its lane quarter of the other
+      // CTAs' partials (4 KB per chunk and slot, contiguous) through its own ring
+      // in the idle stage buffers; no cross-warp synchronisation is needed.
       const int nother = (is_head && !is_full) ? c_last - (int)blockIdx.x : 0;
       const int npieces = nchunks * nother;
+      float* wring = ring + q * (kRing * kPieceFloats);
+      uint64_t* wbar = fixbar + q * kRing;
       auto issue_piece = [&](int p) {
-        const int c = p / nother, sl = (int)blockIdx.x + 1 + p % nother;
-        const int b = p % kRing;
-        mbar_expect_tx(&fixbar[b], kPieceFloats * 4);
-        bulk_load(ring + b * kPieceFloats, args.partials + (size_t)sl * kSlotFloats + (size_t)c * kPieceFloats,
-                  kPieceFloats * 4, &fixbar[b]);
+        const int c = p / nother, sl = (int)blockIdx.x + 1 + p % nother, b = p % kRing;
+        mbar_expect_tx(&wbar[b], kPieceFloats * 4);
+        bulk_load(wring + b * kPieceFloats,
+                  args.partials + (size_t)sl * kSlotFloats + (size_t)q * kQuarterFloats + (size_t)c * kPieceFloats,
+                  kPieceFloats * 4, &wbar[b]);
       };
-      int issued_hi = 0, consumed = 0;  // issued_hi is tracked by the issuing thread only
-      if (npieces > 0 && et == 0) {
+      int issued_hi = 0, consumed = 0;
+      if (npieces > 0 && lane == 0) {
         fence_proxy_async_global();
-        for (int p = 0; p < npieces && p < kRing; ++p) issue_piece(p);
         issued_hi = npieces < kRing ? npieces : kRing;
+        for (int p = 0; p < issued_hi; ++p) issue_piece(p);
       }
+      const bool resid = is_head && (args.epi == EPI_O || args.epi == EPI_DOWN);
+      const int f128 = g.ft * kGemmBM + lr;
       for (int c = 0; c < nchunks; ++c) {
         const int jb = c * 32;
-        // residual operands first, so their latency overlaps the TMEM drain
+        // residual operand (fp32 h, contiguous rows): every load issued before any
+        // use; rows past ntok are clamped to a valid row and never stored
         float res[32];
-        if (args.epi == EPI_O || args.epi == EPI_DOWN) {
-          const int f = g.ft * kGemmBM + lr;
-          const __nv_bfloat16* x = (const __nv_bfloat16*)args.x_in;
+        if (resid) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            res[i] = 0.f;
-            if (jb + i < g.ntok) {
-              res[i] = args.epi == EPI_O ? bf2f(x[(size_t)s_idx[jb + i] * d + f])
-                                         : __ldcg(&args.h32[(size_t)(g.tok0 + jb + i) * d + f]);
-            }
+            const int jj = min(jb + i, g.ntok - 1);
+            res[i] = __ldcg(&args.h32[(size_t)(g.tok0 + jj) * d + f128]);
           }
         }
         uint32_t r[32];
@@ -301,74 +304,76 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
         if (!is_head) {
-          float* slot = args.partials + (size_t)blockIdx.x * kSlotFloats;
+          float* slot = args.partials + (size_t)blockIdx.x * kSlotFloats + (size_t)q * kQuarterFloats + jb * 32;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) slot[(c * 32 + i) * kGemmBM + lr] = v[i];
+          for (int i = 0; i < 32; ++i) slot[i * 32 + lane] = v[i];
           continue;
         }
         for (int so = 0; so < nother; ++so) {
           const int p = c * nother + so, b = p % kRing;
-          if (!*s_abort && !mbar_wait(&fixbar[b], (uint32_t)((p / kRing) & 1))) *s_abort = 1;
+          if (!*s_abort && !mbar_wait(&wbar[b], (uint32_t)((p / kRing) & 1))) *s_abort = 1;
           if (!*s_abort) {
             consumed = p + 1;
-            const float* buf = ring + b * kPieceFloats;
+            const float* buf = wring + b * kPieceFloats;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] += buf[i * kGemmBM + lr];
+            for (int i = 0; i < 32; ++i) v[i] += buf[i * 32 + lane];
           }
-          named_bar_sync(1, 128);  // every thread is done with buffer b
-          if (et == 0 && p + kRing < npieces && !*s_abort) {
+          __syncwarp();  // the whole warp is done with buffer b
+          if (lane == 0 && p + kRing < npieces && !*s_abort) {
             issue_piece(p + kRing);
             issued_hi = p + kRing + 1;
           }
         }
+        const int nval = g.ntok - jb;  // valid tokens in this chunk (may exceed 32)
         if (args.epi == EPI_QKV) {
-          const int f = g.ft * kGemmBM + lr;
-          const int part = f / d, col = f - part * d;
+          const int part = f128 / d, col = f128 - part * d;
           __nv_bfloat16* dst = part == 0 ? (__nv_bfloat16*)args.q_out
                                          : (part == 1 ? (__nv_bfloat16*)args.k_cache : (__nv_bfloat16*)args.v_cache);
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            if (jb + i < g.ntok) {
+            if (i < nval) {
               const size_t row = part == 0 ? (size_t)(g.tok0 + jb + i) : (size_t)s_idx[jb + i];
               dst[row * d + col] = f2bf(v[i]);
             }
           }
         } else if (args.epi == EPI_O) {
-          const int f = g.ft * kGemmBM + lr;
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (jb + i < g.ntok) args.h32[(size_t)(g.tok0 + jb + i) * d + f] = v[i] + res[i];
+            if (i < nval) args.h32[(size_t)(g.tok0 + jb + i) * d + f128] = v[i] + res[i];
         } else if (args.epi == EPI_GU) {
+          // gate rows are TMEM lanes 0-63 (warps with q = 0, 1), up rows lanes 64-127
+          // (q = 2, 3): warp q+2 hands its values to warp q through a
+          // double-buffered exchange, one 64-thread barrier per chunk and pair
+          float* xb = xbuf + (c & 1) * (64 * kXbufStride);
           if (q >= 2) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) xbuf[(lr - 64) * kXbufStride + i] = v[i];
+            for (int i = 0; i < 32; ++i) xb[(lr - 64) * kXbufStride + i] = v[i];
           }
-          named_bar_sync(2, 128);
+          named_bar_sync(2 + (q & 1), 64);
           if (q < 2) {
             const int F = args.gu_F;
             const int f = g.ft * 64 + lr;
             __nv_bfloat16* out = (__nv_bfloat16*)args.act_out;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-              if (jb + i < g.ntok) {
-                const float u = xbuf[lr * kXbufStride + i];
+              if (i < nval) {
+                const float u = xb[lr * kXbufStride + i];
                 out[(size_t)(g.tok0 + jb + i) * F + f] = f2bf(silu_f(v[i]) * u);
               }
             }
           }
-          named_bar_sync(2, 128);
         } else {  // EPI_DOWN
-          const int f = g.ft * kGemmBM + lr;
           __nv_bfloat16* y = (__nv_bfloat16*)args.y_cache;
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (jb + i < g.ntok) y[(size_t)s_idx[jb + i] * d + f] = f2bf(res[i] + v[i]);
+            if (i < nval) y[(size_t)s_idx[jb + i] * d + f128] = f2bf(res[i] + v[i]);
         }
       }
-      if (et == 0 && *s_abort) {
-        // bounded wait for the fix-up copies still in flight before the CTA exits
-        for (int p = consumed; p < issued_hi; ++p) (void)mbar_wait(&fixbar[p % kRing], (uint32_t)((p / kRing) & 1));
+      if (lane == 0 && *s_abort) {
+        // bounded wait for this warp's fix-up copies still in flight before exit
+        for (int p = consumed; p < issued_hi; ++p) (void)mbar_wait(&wbar[p % kRing], (uint32_t)((p / kRing) & 1));
       }
+      __syncwarp();
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
       if (!is_head) {
@@ -383,11 +388,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       acc ^= 1;
       if (acc == 0) accph ^= 1;
     }
+    tc_fence_before();
+    mbar_arrive(epi_done);  // every epilogue thread is done with TMEM
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
+    // the epilogue warps signal their last TMEM read on their own barrier, so
+    // the columns are released only after it
+    (void)mbar_wait(epi_done, 0);
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }

@@ -4,10 +4,11 @@
 // "Algorithmic Complexity"), and the full-recompute baseline (Sec. 1).
 //
 // bf16 chain (7 launches, M read on the device, no host synchronisation):
-//   1 gather rows idx[j] of X, RMSNorm1 -> xn (bf16); clear the GEMM fix-up flags
+//   1 gather rows idx[j] of X, RMSNorm1 -> xn (bf16), x -> h (fp32); clear the
+//     GEMM fix-up flags
 //   2 tcgen05 GEMM  xn W_qkv^T -> Q (compact), K and V scattered into the caches
 //   3 attention of the M queries over all N cached keys -> a (bf16)
-//   4 tcgen05 GEMM  a W_o^T + x -> h (fp32)
+//   4 tcgen05 GEMM  h += a W_o^T (fp32)
 //   5 RMSNorm2(h) -> hn (bf16)
 //   6 tcgen05 GEMM  hn [W_g; W_u]^T -> silu(g) * u (bf16)
 //   7 tcgen05 GEMM  act W_down^T + h -> Y rows idx[j] (bf16)
@@ -130,7 +131,8 @@ template <typename Tin, typename Tg, typename Tout>
 __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const Tin* __restrict__ X, const int32_t* __restrict__ idx,
                                                            const int32_t* __restrict__ seg_ptr, int B,
                                                            const Tg* __restrict__ g, float eps, int d,
-                                                           Tout* __restrict__ out, uint32_t* flags, int nflags) {
+                                                           Tout* __restrict__ out, uint32_t* flags, int nflags,
+                                                           float* __restrict__ res_out) {
   __shared__ float sh[33];
   if (flags && blockIdx.x == 0)
     for (int i = threadIdx.x; i < nflags; i += blockDim.x) flags[i] = 0u;
@@ -143,6 +145,7 @@ __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const Tin* __restrict
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
     const float v = to_f(x[c]);
     ss = fmaf(v, v, ss);
+    if (res_out) res_out[(size_t)j * d + c] = v;
   }
   ss = block_sum_f(ss, sh);
   const float inv = 1.0f / sqrtf(ss / (float)d + eps);
@@ -213,7 +216,8 @@ template <typename Tin, typename Tg, typename Tout, int NV>
 __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict__ X, const int32_t* __restrict__ idx,
                                                           const int32_t* __restrict__ seg_ptr, int B,
                                                           const Tg* __restrict__ g, float eps, int d,
-                                                          Tout* __restrict__ out, uint32_t* flags, int nflags) {
+                                                          Tout* __restrict__ out, uint32_t* flags, int nflags,
+                                                          float* __restrict__ res_out) {
   constexpr int E = Vec16<Tin>::E;
   __shared__ float sh[33];
   if (flags && blockIdx.x == 0)
@@ -249,6 +253,7 @@ __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict_
     if (vi < nvec) {
       float f[E];
       Vec16<Tin>::unpack(buf[u], f);
+      if (res_out) store_vec<float, E>(res_out + (size_t)j * d + vi * E, f);
 #pragma unroll
       for (int e = 0; e < E; ++e) f[e] = f[e] * inv * to_f(g[vi * E + e]);
       store_vec<Tout, E>(o + vi * E, f);
@@ -259,12 +264,15 @@ __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict_
 // Picks the register-resident kernel when the row fits, else the looping one.
 template <typename Tin, typename Tg, typename Tout>
 static void launch_rmsnorm(const Tin* X, const int32_t* idx, const int32_t* seg, int B, const Tg* g, float eps,
-                           int d, Tout* out, uint32_t* flags, int nflags, int grid, cudaStream_t st) {
+                           int d, Tout* out, uint32_t* flags, int nflags, int grid, cudaStream_t st,
+                           float* res_out = nullptr) {
   constexpr int E = Vec16<Tin>::E;
   if (d % E == 0 && d <= 4 * 256 * E)
-    rmsnorm_vec_kernel<Tin, Tg, Tout, 4><<<grid, 256, 0, st>>>(X, idx, seg, B, g, eps, d, out, flags, nflags);
+    rmsnorm_vec_kernel<Tin, Tg, Tout, 4><<<grid, 256, 0, st>>>(X, idx, seg, B, g, eps, d, out, flags, nflags,
+                                                               res_out);
   else
-    rmsnorm_rows_kernel<Tin, Tg, Tout><<<grid, 256, 0, st>>>(X, idx, seg, B, g, eps, d, out, flags, nflags);
+    rmsnorm_rows_kernel<Tin, Tg, Tout><<<grid, 256, 0, st>>>(X, idx, seg, B, g, eps, d, out, flags, nflags,
+                                                             res_out);
 }
 
 __global__ void fill_identity_kernel(int32_t* iota, int32_t* seg, int B, int N) {
@@ -419,8 +427,9 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   g.nslots = L.nslots;
 
   trace_mark(0, st);
+  // also stages x (fp32) in h32: the O projection's epilogue adds its residual there
   launch_rmsnorm<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(X, idx, seg, B, (const __nv_bfloat16*)w->g1, dm->eps, d,
-                                                              xn, flags, L.nflags, Mcap, st);
+                                                              xn, flags, L.nflags, Mcap, st, h32);
   PLK_LAUNCHED();
   trace_mark(1, st);
 
