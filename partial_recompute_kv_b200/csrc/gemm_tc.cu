@@ -35,15 +35,15 @@ constexpr int kStageA = kGemmBM * kGemmBK * 2;     // 16 KB
 constexpr int kStageB = kGemmBNMax * kGemmBK * 2;  // 32 KB
 constexpr int kTileCols = 256;                     // TMEM columns per accumulator buffer
 constexpr int kSlotFloats = kGemmBNMax * kGemmBM;  // partial tile, [lane quarter][col][32 lanes]
-constexpr int kXbufStride = 33;
 constexpr size_t kOffB = (size_t)kGemmStages * kStageA;
 constexpr size_t kOffBar = kOffB + (size_t)kGemmStages * kStageB;
 constexpr size_t kOffIdx = kOffBar + 512;
 constexpr int kRing = 8;                           // fix-up ring per epilogue warp: 8 pieces of 4 KB
 constexpr int kPieceFloats = 32 * 32;              // one warp's chunk (32 columns x 32 lanes) of a partial
 constexpr int kQuarterFloats = kGemmBNMax * 32;    // one lane quarter of a partial slot
-constexpr size_t kOffXbuf = kOffIdx + kGemmBNMax * 4;
-constexpr size_t kSmemUsed = kOffXbuf + 2 * 64 * kXbufStride * 4;  // double-buffered gate/up exchange
+constexpr size_t kOffStg = kOffIdx + kGemmBNMax * 4;
+constexpr int kStgFloats = 32 * 32;                // per epilogue warp: 32 tokens x 32 features
+constexpr size_t kSmemUsed = kOffStg + 4 * kStgFloats * 4;
 constexpr size_t kSmemBytes = kSmemUsed + 1024;  // slack for 1024-byte alignment
 
 struct Sched {
@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* epi_done = bars + 48;         // epilogue warps finished with TMEM
   float* ring = reinterpret_cast<float*>(smem);
   int* s_idx = reinterpret_cast<int*>(smem + kOffIdx);
-  float* xbuf = reinterpret_cast<float*>(smem + kOffXbuf);
+  float* stg_all = reinterpret_cast<float*>(smem + kOffStg);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   Sched s;
@@ -324,49 +324,73 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             issued_hi = p + kRing + 1;
           }
         }
+        // Output: the warp's 32 features x 32 tokens go through its staging buffer
+        // and leave token-major as 16-byte stores (64 B of each token row).
         const int nval = g.ntok - jb;  // valid tokens in this chunk (may exceed 32)
-        if (args.epi == EPI_QKV) {
-          const int part = f128 / d, col = f128 - part * d;
-          __nv_bfloat16* dst = part == 0 ? (__nv_bfloat16*)args.q_out
-                                         : (part == 1 ? (__nv_bfloat16*)args.k_cache : (__nv_bfloat16*)args.v_cache);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (i < nval) {
-              const size_t row = part == 0 ? (size_t)(g.tok0 + jb + i) : (size_t)s_idx[jb + i];
-              dst[row * d + col] = f2bf(v[i]);
-            }
-          }
-        } else if (args.epi == EPI_O) {
+        float* stg = stg_all + q * kStgFloats;
+        __nv_bfloat16* stg_h = reinterpret_cast<__nv_bfloat16*>(stg);
+        const int fbase = g.ft * kGemmBM + q * 32;  // first feature of this warp
+        if (args.epi == EPI_QKV || args.epi == EPI_DOWN) {
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (i < nval) args.h32[(size_t)(g.tok0 + jb + i) * d + f128] = v[i] + res[i];
-        } else if (args.epi == EPI_GU) {
-          // gate rows are TMEM lanes 0-63 (warps with q = 0, 1), up rows lanes 64-127
-          // (q = 2, 3): warp q+2 hands its values to warp q through a
-          // double-buffered exchange, one 64-thread barrier per chunk and pair
-          float* xb = xbuf + (c & 1) * (64 * kXbufStride);
+            stg_h[i * 32 + lane] = f2bf(args.epi == EPI_DOWN ? res[i] + v[i] : v[i]);
+          __syncwarp();
+          const int part = fbase / d, col = fbase - part * d;
+          __nv_bfloat16* dst = args.epi == EPI_DOWN
+                                   ? (__nv_bfloat16*)args.y_cache
+                                   : (part == 0 ? (__nv_bfloat16*)args.q_out
+                                                : (part == 1 ? (__nv_bfloat16*)args.k_cache
+                                                             : (__nv_bfloat16*)args.v_cache));
+          const bool compact = args.epi == EPI_QKV && part == 0;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int tk = k * 8 + (lane >> 2);
+            if (tk < nval) {
+              const size_t row = compact ? (size_t)(g.tok0 + jb + tk) : (size_t)s_idx[jb + tk];
+              *reinterpret_cast<uint4*>(dst + row * d + col + (lane & 3) * 8) =
+                  reinterpret_cast<const uint4*>(stg_h)[tk * 4 + (lane & 3)];
+            }
+          }
+          __syncwarp();
+        } else if (args.epi == EPI_O) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) stg[i * 32 + lane] = v[i] + res[i];
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int tk = k * 4 + (lane >> 3);
+            if (tk < nval)
+              *reinterpret_cast<float4*>(args.h32 + (size_t)(g.tok0 + jb + tk) * d + fbase + (lane & 7) * 4) =
+                  reinterpret_cast<const float4*>(stg)[tk * 8 + (lane & 7)];
+          }
+          __syncwarp();
+        } else {  // EPI_GU
+          // gate rows are TMEM lanes 0-63 (warps q = 0, 1), up rows lanes 64-127
+          // (q = 2, 3): warp q+2 parks its values in its staging buffer, warp q
+          // reads them, forms silu(g) * u and stores it; two 64-thread barriers
+          // per chunk and pair
           if (q >= 2) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) xb[(lr - 64) * kXbufStride + i] = v[i];
+            for (int i = 0; i < 32; ++i) stg[i * 32 + lane] = v[i];
           }
           named_bar_sync(2 + (q & 1), 64);
           if (q < 2) {
+            const float* up = stg_all + (q + 2) * kStgFloats;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) stg_h[i * 32 + lane] = f2bf(silu_f(v[i]) * up[i * 32 + lane]);
+            __syncwarp();
             const int F = args.gu_F;
-            const int f = g.ft * 64 + lr;
-            __nv_bfloat16* out = (__nv_bfloat16*)args.act_out;
+            __nv_bfloat16* out = (__nv_bfloat16*)args.act_out + g.ft * 64 + q * 32;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              if (i < nval) {
-                const float u = xb[lr * kXbufStride + i];
-                out[(size_t)(g.tok0 + jb + i) * F + f] = f2bf(silu_f(v[i]) * u);
-              }
+            for (int k = 0; k < 4; ++k) {
+              const int tk = k * 8 + (lane >> 2);
+              if (tk < nval)
+                *reinterpret_cast<uint4*>(out + (size_t)(g.tok0 + jb + tk) * F + (lane & 3) * 8) =
+                    reinterpret_cast<const uint4*>(stg_h)[tk * 4 + (lane & 3)];
             }
+            __syncwarp();
           }
-        } else {  // EPI_DOWN
-          __nv_bfloat16* y = (__nv_bfloat16*)args.y_cache;
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (i < nval) y[(size_t)s_idx[jb + i] * d + f128] = f2bf(res[i] + v[i]);
+          named_bar_sync(2 + (q & 1), 64);  // warp q+2 may refill its buffer
         }
       }
       if (lane == 0 && *s_abort) {
