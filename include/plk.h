@@ -168,6 +168,30 @@ int plk_full_layer_step(const plk_dims* dims, const plk_weights* w, const void* 
 int plk_proxy_commit(const plk_dims* dims, int r, const int32_t* idx, const int32_t* seg_ptr,
                      const float* proxy_new, float* proxy_cache, void* stream);
 
+/*
+ * plk_layer_step_partial without a caller workspace.  (The pages have no
+ * counterpart: this is a deployment variant of the layer step above.)
+ * Some callers cannot call cudaMalloc -- code running inside a global-mode
+ * stream capture (an allocation there breaks the capture), real-time paths that
+ * cannot absorb an allocation's latency, and plugins whose host runtime owns
+ * every device allocation.  This entry point runs the same kernels as
+ * plk_layer_step_partial with its scratch in a file-scope device array of
+ * PLK_STATIC_WS_BYTES, which every GPU that loads the library holds until the
+ * process exits.  Arguments and results are those of plk_layer_step_partial.
+ *   - It calls no cudaMalloc, cudaFree or allocating library routine.
+ *   - Returns PLK_ERR_WORKSPACE, enqueueing nothing, when plk_workspace_bytes(dims)
+ *     exceeds PLK_STATIC_WS_BYTES.
+ *   - The first call on a device resolves the array's device address
+ *     (cudaGetSymbolAddress); make that first call outside any stream capture.
+ *   - All calls on a device share the array, which keeps the last call's
+ *     contents (every kernel initialises what it reads): calls that overlap on
+ *     the GPU, e.g. on two streams, race and must be serialised by the caller.
+ */
+#define PLK_STATIC_WS_BYTES (32u << 20)
+int plk_layer_step_partial_static(const plk_dims* dims, const plk_weights* w, const void* X,
+                                  const int32_t* idx, const int32_t* seg_ptr,
+                                  void* K_cache, void* V_cache, void* Y, void* stream);
+
 /* Bytes of workspace plk_layer_step_partial / plk_full_layer_step need for these
  * dims on the current device (0 for invalid dims). */
 size_t plk_workspace_bytes(const plk_dims* dims);

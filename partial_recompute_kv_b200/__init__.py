@@ -24,7 +24,8 @@ SEL_THRESH_GT, SEL_THRESH_LT, SEL_TOPK_LARGEST, SEL_TOPK_SMALLEST = 0, 1, 2, 3
 
 EXPORTED = (
     "plk_score_drift", "plk_select_active", "plk_layer_step_partial", "plk_full_layer_step",
-    "plk_proxy_commit", "plk_workspace_bytes", "plk_get_status", "plk_set_wait_limit",
+    "plk_proxy_commit", "plk_layer_step_partial_static", "plk_workspace_bytes", "plk_get_status",
+    "plk_set_wait_limit",
     "plk_selftest_wait_timeout", "plk_trace_events", "plk_error_string", "plk_version",
 )
 
@@ -57,6 +58,7 @@ def _load():
         "plk_select_active": (I, [V, P, P, P, I, F, I, P, P, P]),
         "plk_layer_step_partial": (I, [V, W, P, P, P, P, P, P, P, S, P]),
         "plk_full_layer_step": (I, [V, W, P, P, P, P, P, S, P]),
+        "plk_layer_step_partial_static": (I, [V, W, P, P, P, P, P, P, P]),
         "plk_proxy_commit": (I, [V, I, P, P, P, P, P]),
         "plk_workspace_bytes": (S, [V]),
         "plk_get_status": (I, [P]),
@@ -151,6 +153,18 @@ def layer_step_partial(dm, w, X, idx, seg_ptr, K_cache, V_cache, Y, workspace, s
                                       _ptr(K_cache), _ptr(V_cache), _ptr(Y), _ptr(workspace),
                                       workspace.numel() * workspace.element_size(), _stream(stream)),
            "layer_step_partial")
+
+
+STATIC_WS_BYTES = 32 << 20
+
+
+def layer_step_partial_static(dm, w, X, idx, seg_ptr, K_cache, V_cache, Y, stream=None):
+    """layer_step_partial with the library's own device-array scratch (no workspace,
+    no allocation); see plk_layer_step_partial_static in include/plk.h."""
+    pw = w if isinstance(w, PlkWeights) else weights(w)
+    _check(lib.plk_layer_step_partial_static(ctypes.byref(dm), ctypes.byref(pw), _ptr(X), _ptr(idx),
+                                             _ptr(seg_ptr), _ptr(K_cache), _ptr(V_cache), _ptr(Y),
+                                             _stream(stream)), "layer_step_partial_static")
 
 
 def full_layer_step(dm, w, X, K_cache, V_cache, Y, workspace, stream=None):

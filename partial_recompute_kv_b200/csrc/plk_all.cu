@@ -6,3 +6,4 @@
 #include "gemm_tc.cu"
 #include "attention.cu"
 #include "abi.cu"
+#include "static_ws.cu"
