@@ -4,8 +4,7 @@
 // "Algorithmic Complexity"), and the full-recompute baseline (Sec. 1).
 //
 // bf16 chain (7 launches, M read on the device, no host synchronisation):
-//   1 gather rows idx[j] of X, RMSNorm1 -> xn (bf16), x -> h (fp32); clear the
-//     GEMM fix-up flags
+//   1 gather rows idx[j] of X, RMSNorm1 -> xn (bf16), x -> h (fp32)
 //   2 tcgen05 GEMM  xn W_qkv^T -> Q (compact), K and V scattered into the caches
 //   3 attention of the M queries over all N cached keys -> a (bf16)
 //   4 tcgen05 GEMM  h += a W_o^T (fp32)
@@ -60,13 +59,8 @@ Workspace workspace_layout(const plk_dims* dm, int num_sms) {
   w.h32 = take(4 * Mcap * d);
   w.hn = take(es * Mcap * d);
   w.act = take(es * Mcap * F);
+  w.num_sms = num_sms;
   if (dm->dtype == PLK_BF16) {
-    const size_t ttiles = (Mcap + kGemmBNMax - 1) / kGemmBNMax;
-    const size_t ft = std::max((size_t)3 * d / kGemmBM, F / 64);
-    w.nslots = num_sms;
-    w.nflags = (int)(ft * ttiles);
-    w.partials = take((size_t)num_sms * kGemmBNMax * kGemmBM * 4);
-    w.flags = take(4 * (size_t)w.nflags);
     w.att_rows = attn_split_rows(dm, num_sms);
     w.att_o = take((size_t)kAttSplitMax * w.att_rows * d * 4);
     w.att_ml = take((size_t)kAttSplitMax * w.att_rows * dm->H * 8);
@@ -126,16 +120,13 @@ __device__ __forceinline__ float block_sum_f(float v, float* sh) {
 }
 
 // out[j] = RMSNorm(src_row(j)) * g for j < M.  src_row(j) = X[idx[j]] (gather)
-// or H[j] (idx == nullptr).  Block 0 also clears the GEMM fix-up flags.
+// or H[j] (idx == nullptr); res_out (optional) receives the fp32 source row.
 template <typename Tin, typename Tg, typename Tout>
 __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const Tin* __restrict__ X, const int32_t* __restrict__ idx,
                                                            const int32_t* __restrict__ seg_ptr, int B,
                                                            const Tg* __restrict__ g, float eps, int d,
-                                                           Tout* __restrict__ out, uint32_t* flags, int nflags,
-                                                           float* __restrict__ res_out) {
+                                                           Tout* __restrict__ out, float* __restrict__ res_out) {
   __shared__ float sh[33];
-  if (flags && blockIdx.x == 0)
-    for (int i = threadIdx.x; i < nflags; i += blockDim.x) flags[i] = 0u;
   const int M = seg_ptr[B];
   const int j = blockIdx.x;
   if (j >= M) return;
@@ -216,12 +207,9 @@ template <typename Tin, typename Tg, typename Tout, int NV>
 __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict__ X, const int32_t* __restrict__ idx,
                                                           const int32_t* __restrict__ seg_ptr, int B,
                                                           const Tg* __restrict__ g, float eps, int d,
-                                                          Tout* __restrict__ out, uint32_t* flags, int nflags,
-                                                          float* __restrict__ res_out) {
+                                                          Tout* __restrict__ out, float* __restrict__ res_out) {
   constexpr int E = Vec16<Tin>::E;
   __shared__ float sh[33];
-  if (flags && blockIdx.x == 0)
-    for (int i = threadIdx.x; i < nflags; i += blockDim.x) flags[i] = 0u;
   const int M = seg_ptr[B];
   const int j = blockIdx.x;
   if (j >= M) return;
@@ -264,15 +252,12 @@ __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict_
 // Picks the register-resident kernel when the row fits, else the looping one.
 template <typename Tin, typename Tg, typename Tout>
 static void launch_rmsnorm(const Tin* X, const int32_t* idx, const int32_t* seg, int B, const Tg* g, float eps,
-                           int d, Tout* out, uint32_t* flags, int nflags, int grid, cudaStream_t st,
-                           float* res_out = nullptr) {
+                           int d, Tout* out, int grid, cudaStream_t st, float* res_out = nullptr) {
   constexpr int E = Vec16<Tin>::E;
   if (d % E == 0 && d <= 4 * 256 * E)
-    rmsnorm_vec_kernel<Tin, Tg, Tout, 4><<<grid, 256, 0, st>>>(X, idx, seg, B, g, eps, d, out, flags, nflags,
-                                                               res_out);
+    rmsnorm_vec_kernel<Tin, Tg, Tout, 4><<<grid, 256, 0, st>>>(X, idx, seg, B, g, eps, d, out, res_out);
   else
-    rmsnorm_rows_kernel<Tin, Tg, Tout><<<grid, 256, 0, st>>>(X, idx, seg, B, g, eps, d, out, flags, nflags,
-                                                             res_out);
+    rmsnorm_rows_kernel<Tin, Tg, Tout><<<grid, 256, 0, st>>>(X, idx, seg, B, g, eps, d, out, res_out);
 }
 
 __global__ void fill_identity_kernel(int32_t* iota, int32_t* seg, int B, int N) {
@@ -377,15 +362,14 @@ static int run_layer_f32(const plk_dims* dm, const plk_weights* w, const float* 
     dim3 grid(ceil_div(Nout, 64), ceil_div(Mcap, 64));
     gemm_f32_kernel<<<grid, 256, 0, st>>>(A, (const float*)Wt, c32, Nout, K, seg, B);
   };
-  launch_rmsnorm<float, float, float>(X, idx, seg, B, (const float*)w->g1, dm->eps, d, xn, nullptr, 0, Mcap, st);
+  launch_rmsnorm<float, float, float>(X, idx, seg, B, (const float*)w->g1, dm->eps, d, xn, Mcap, st);
   gemm(xn, w->w_qkv, 3 * d, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_QKV, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y);
   PLK_LAUNCHED();
   PLK_TRY(launch_attention_f32(dm, q, Kc, Vc, a, seg, Mcap, st));
   gemm(a, w->w_o, d, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_O, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y);
-  launch_rmsnorm<float, float, float>(h32, nullptr, seg, B, (const float*)w->g2, dm->eps, d, hn, nullptr, 0, Mcap,
-                                      st);
+  launch_rmsnorm<float, float, float>(h32, nullptr, seg, B, (const float*)w->g2, dm->eps, d, hn, Mcap, st);
   gemm(hn, w->w_gu, 2 * F, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_GU, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y);
   gemm(act, w->w_down, d, F);
@@ -404,7 +388,6 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   float* h32 = (float*)(ws + L.h32);
   __nv_bfloat16* hn = (__nv_bfloat16*)(ws + L.hn);
   __nv_bfloat16* act = (__nv_bfloat16*)(ws + L.act);
-  uint32_t* flags = (uint32_t*)(ws + L.flags);
 
   CUtensorMap tW_qkv, tW_o, tW_gu, tW_down, tX_xn, tX_a, tX_hn, tX_act;
   PLK_TRY(make_tmap_bf16(&tW_qkv, w->w_qkv, 3ull * d, d, 64));
@@ -422,14 +405,13 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   g.seg_ptr = seg;
   g.B = B;
   g.idx = idx;
-  g.partials = (float*)(ws + L.partials);
-  g.flags = flags;
-  g.nslots = L.nslots;
+  g.ttiles_max = ceil_div(Mcap, kGemmBNMax);
+  g.num_sms = L.num_sms;
 
   trace_mark(0, st);
   // also stages x (fp32) in h32: the O projection's epilogue adds its residual there
   launch_rmsnorm<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(X, idx, seg, B, (const __nv_bfloat16*)w->g1, dm->eps, d,
-                                                              xn, flags, L.nflags, Mcap, st, h32);
+                                                              xn, Mcap, st, h32);
   PLK_LAUNCHED();
   trace_mark(1, st);
 
@@ -443,7 +425,7 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   trace_mark(2, st);
 
   PLK_TRY(launch_attention_bf16(dm, q, Kc, Vc, a, seg, (float*)(ws + L.att_o), ws + L.att_ml, kAttSplitMax,
-                                L.att_rows, L.nslots, st));
+                                L.att_rows, L.num_sms, st));
   trace_mark(3, st);
 
   g.epi = EPI_O;
@@ -455,7 +437,7 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   trace_mark(4, st);
 
   launch_rmsnorm<float, __nv_bfloat16, __nv_bfloat16>(h32, nullptr, seg, B, (const __nv_bfloat16*)w->g2, dm->eps, d, hn,
-                                                      nullptr, 0, Mcap, st);
+                                                      Mcap, st);
   PLK_LAUNCHED();
   trace_mark(5, st);
 

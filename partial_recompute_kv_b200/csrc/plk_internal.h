@@ -25,8 +25,7 @@ struct Workspace {
   size_t iota = 0, seg = 0;              // identity active set for the full step
   size_t xn = 0, q = 0, a = 0, h32 = 0, hn = 0, act = 0;
   size_t c32 = 0;                        // fp32 path: GEMM output scratch [Mcap, max(3d, 2F)]
-  size_t partials = 0, flags = 0;        // stream-K fix-up of the tcgen05 GEMM
-  int nflags = 0, nslots = 0;
+  int num_sms = 0;
   size_t att_o = 0, att_ml = 0;          // split-KV attention partials
   int att_rows = 0;
 };
@@ -72,9 +71,8 @@ struct GemmArgs {
   float* h32;              // EPI_O output, EPI_DOWN residual [Mcap, d]
   void* act_out;           // EPI_GU: [Mcap, F] bf16
   void* y_cache;           // EPI_DOWN
-  float* partials;         // [nslots][256][128]
-  uint32_t* flags;         // [nflags]
-  int nslots;
+  int ttiles_max;          // token tiles of Mcap (grid rows; tiles past M exit at once)
+  int num_sms;             // SM count, for the split-K choice
 };
 int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& a, cudaStream_t st);
 
