@@ -204,6 +204,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   };
 
+  float res[32];  // epilogue warps: residuals of the chunk being finished
+
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (elect_one()) {
@@ -275,7 +277,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const bool have_acc = !*s_epi_abort && !*s_abort && kb1 > kb0;
     const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
     if (CS == 1) {
-      float res[32], res_nx[32];
+      float res_nx[32];
       if (resid) load_res(0, res_nx);
       for (int c = 0; c < nchunks && have_acc; ++c) {
         if (resid) {
@@ -292,6 +294,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         apply(c, v, res);
       }
     } else {
+      // residuals of the first chunk this CTA will finish, in flight across the barrier
+      if (resid && kr < nchunks) load_res(kr, res);
       // park this CTA's partial for the cluster reduction
       for (int c = 0; c < nchunks; ++c) {
         uint32_t r[32];
@@ -324,22 +328,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp >= 2) {
       // ---------------------------------------------------------- epilogue, part 2
       // this CTA finishes chunks c = kr, kr + CS, ... summing the CS partials
-      float res[32];
       const uint32_t mine = smem_u32(rb + q * kRbQuarter + lane * kRbLane);
       for (int c = kr; c < nchunks; c += CS) {
-        if (resid) load_res(c, res);
+        if (resid && c != kr) load_res(c, res);  // the first chunk's were loaded before the barrier
         float v[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = 0.f;
         for (int p = 0; p < CS; ++p) {
           const uint32_t src = dsmem_addr(mine + (uint32_t)(c * kRbChunk * 4), (uint32_t)p);
+          float4 t[8];  // all of a peer's loads in flight before the first add
+#pragma unroll
+          for (int i = 0; i < 8; ++i) t[i] = ld_dsmem_v4(src + 16u * i);
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float4 t = ld_dsmem_v4(src + 16u * i);
-            v[4 * i] += t.x;
-            v[4 * i + 1] += t.y;
-            v[4 * i + 2] += t.z;
-            v[4 * i + 3] += t.w;
+            v[4 * i] += t[i].x;
+            v[4 * i + 1] += t[i].y;
+            v[4 * i + 2] += t[i].z;
+            v[4 * i + 3] += t[i].w;
           }
         }
         apply(c, v, res);

@@ -154,8 +154,14 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
     const uint32_t pbase = smem_u32(part + lrow * pstride);
     float dot = 0.f, pp = 0.f, cc = 0.f, dd = 0.f;
     for (int c = sub; c < r; c += tpr) {
+      float pk[8];  // the S loads of this column in flight before the sum
+#pragma unroll
+      for (int sr = 0; sr < 8; ++sr)
+        if (sr < S) pk[sr] = ld_dsmem_f32(dsmem_addr(pbase + 4u * c, (uint32_t)sr));
       float p = 0.f;
-      for (int sr = 0; sr < S; ++sr) p += ld_dsmem_f32(dsmem_addr(pbase + 4u * c, (uint32_t)sr));
+#pragma unroll
+      for (int sr = 0; sr < 8; ++sr)
+        if (sr < S) p += pk[sr];
       if (row < rows) {
         const float cv = __ldg(cache + (size_t)row * r + c);
         dot = fmaf(p, cv, dot);
