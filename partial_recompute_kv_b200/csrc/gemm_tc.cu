@@ -21,12 +21,14 @@
 //    that tiles x CS fills the SMs (at M <= 256 the O and down projections have
 //    only 32 tiles of 128 features).  CS = 1 drains TMEM straight into the
 //    epilogue.
-//  * Epilogues: QKV (Q compact; K and V scattered straight into the cache rows,
-//    the K/V refresh of SureLock Sec. 2), O (h += a W_o^T, fp32), GU (tile =
-//    64 gate rows + 64 up rows of the same features; silu(g) * u), DOWN
-//    (h + act W_down^T, scattered into the output cache rows).  Each warp's
-//    32 features x 32 tokens leave through a small staging buffer as 16-byte
-//    token-major stores.
+//  * Epilogues (one kernel instantiation each): QKV (Q compact; K and V
+//    scattered straight into the cache rows, the K/V refresh of SureLock
+//    Sec. 2), O (h += a W_o^T, fp32), GU (tile = 64 gate rows + 64 up rows of
+//    the same features; silu(g) * u), DOWN (h + act W_down^T, scattered into
+//    the output cache rows).  Each warp's 32 tokens x 32 features are staged
+//    token-major in shared memory and leave as 16-byte stores; the parked
+//    partial uses the same token-major layout, so every remote read of the
+//    reduction is 512 contiguous bytes per warp instruction.
 #include "plk_common.cuh"
 #include "plk_internal.h"
 
@@ -40,15 +42,12 @@ constexpr size_t kOffB = (size_t)kGemmStages * kStageA;
 constexpr size_t kOffBar = kOffB + (size_t)kGemmStages * kStageB;
 constexpr size_t kOffIdx = kOffBar + 128;
 constexpr size_t kOffStg = kOffIdx + kGemmBNMax * 4;
-constexpr int kStgFloats = 32 * 32;                // per epilogue warp: 32 tokens x 32 features
-constexpr size_t kSmemUsed = kOffStg + 4 * kStgFloats * 4;
+constexpr int kBlk = 32 * 32;                      // a warp's block: 32 tokens x 32 features (fp32)
+constexpr size_t kSmemUsed = kOffStg + 4 * kBlk * 4;
 constexpr size_t kSmemBytes = kSmemUsed + 1024;    // slack for 1024-byte alignment
 // Partial parked for the cluster reduction, in the stage area once the main loop
-// is over: [chunk][lane quarter][lane][36] fp32 (36 = 32 + padding: 16-byte
-// accesses of 8 consecutive lanes hit distinct banks).
-constexpr int kRbLane = 36;
-constexpr int kRbQuarter = 32 * kRbLane;
-constexpr int kRbChunk = 4 * kRbQuarter;
+// is over: [chunk][lane quarter][token][feature] fp32.
+constexpr int kRbChunk = 4 * kBlk;
 static_assert((size_t)8 * kRbChunk * 4 <= kOffBar, "partial must fit the stage buffers");
 
 // silu(g) = g / (1 + e^-g) with the fast exp and divide intrinsics: their ~1e-6
@@ -64,8 +63,114 @@ __device__ __forceinline__ float4 ld_dsmem_v4(uint32_t addr) {
   return v;
 }
 
+__device__ __forceinline__ float4 add4(float4 a, float4 b) {
+  return make_float4(a.x + b.x, a.y + b.y, a.z + b.z, a.w + b.w);
+}
+
+__device__ __forceinline__ uint4 pack8_bf16(float4 a, float4 b) {
+  uint4 u;
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+  h[0] = __floats2bfloat162_rn(a.x, a.y);
+  h[1] = __floats2bfloat162_rn(a.z, a.w);
+  h[2] = __floats2bfloat162_rn(b.x, b.y);
+  h[3] = __floats2bfloat162_rn(b.z, b.w);
+  return u;
+}
+
+// Epilogue of one warp block.  The block (32 tokens x 32 features, fp32,
+// token-major) sits in shared memory at `blk`; token t of the block is token
+// tok0 + jb + t of the tile, feature j is feature fbase + j.
+//   Items for bf16 outputs: lane l handles 8 features (group l & 3) of tokens
+//   k*8 + (l >> 2), k = 0..3.  Items for the fp32 output: 4 features (group
+//   l & 7) of tokens k*4 + (l >> 3), k = 0..7.  Residuals for those items are
+//   loaded by load_res into r[8] (float4).
+struct EpiCtx {
+  int tok0, jb, nval, fbase, d, lane;
+  const int* s_idx;
+};
+
+template <int EPI>
+__device__ __forceinline__ void load_res(const GemmArgs& a, const EpiCtx& e, int ntok, float4 (&r)[8]) {
+  if (EPI == EPI_O) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int tk = min(e.jb + k * 4 + (e.lane >> 3), ntok - 1);  // clamped: always a valid row
+      r[k] = __ldcg(reinterpret_cast<const float4*>(a.h32 + (size_t)(e.tok0 + tk) * e.d + e.fbase +
+                                                    (e.lane & 7) * 4));
+    }
+  } else if (EPI == EPI_DOWN) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int tk = min(e.jb + k * 8 + (e.lane >> 2), ntok - 1);
+      const float4* src =
+          reinterpret_cast<const float4*>(a.h32 + (size_t)(e.tok0 + tk) * e.d + e.fbase + (e.lane & 3) * 8);
+      r[2 * k] = __ldcg(src);
+      r[2 * k + 1] = __ldcg(src + 1);
+    }
+  }
+}
+
 }  // namespace
 
+namespace {
+
+template <int EPI>
+__device__ __forceinline__ void finish_block(const GemmArgs& a, const EpiCtx& e, const float* blk,
+                                             const float* up_blk, const float4 (&r)[8]) {
+  const int l = e.lane;
+  if (EPI == EPI_O) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int t = k * 4 + (l >> 3);
+      if (t < e.nval) {
+        const float4 x = add4(reinterpret_cast<const float4*>(blk)[t * 8 + (l & 7)], r[k]);
+        *reinterpret_cast<float4*>(a.h32 + (size_t)(e.tok0 + e.jb + t) * e.d + e.fbase + (l & 7) * 4) = x;
+      }
+    }
+    return;
+  }
+  __nv_bfloat16* dst;
+  int col = 0;
+  size_t ld = (size_t)e.d;
+  bool compact = false;
+  if (EPI == EPI_QKV) {
+    const int part = e.fbase / e.d;
+    col = e.fbase - part * e.d;
+    dst = (__nv_bfloat16*)(part == 0 ? a.q_out : (part == 1 ? a.k_cache : a.v_cache));
+    compact = part == 0;
+  } else if (EPI == EPI_DOWN) {
+    dst = (__nv_bfloat16*)a.y_cache;
+    col = e.fbase;
+  } else {  // EPI_GU: features fbase index the [gate | up] tile rows; output column ft*64 + j
+    dst = (__nv_bfloat16*)a.act_out;
+    col = e.fbase;  // caller passes the output column of this warp's gate features
+    ld = (size_t)a.gu_F;
+    compact = true;
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int t = k * 8 + (l >> 2);
+    if (t < e.nval) {
+      const float4* src = reinterpret_cast<const float4*>(blk) + t * 8 + (l & 3) * 2;
+      float4 x0 = src[0], x1 = src[1];
+      if (EPI == EPI_DOWN) {
+        x0 = add4(x0, r[2 * k]);
+        x1 = add4(x1, r[2 * k + 1]);
+      } else if (EPI == EPI_GU) {
+        const float4* u = reinterpret_cast<const float4*>(up_blk) + t * 8 + (l & 3) * 2;
+        const float4 u0 = u[0], u1 = u[1];
+        x0 = make_float4(silu_f(x0.x) * u0.x, silu_f(x0.y) * u0.y, silu_f(x0.z) * u0.z, silu_f(x0.w) * u0.w);
+        x1 = make_float4(silu_f(x1.x) * u1.x, silu_f(x1.y) * u1.y, silu_f(x1.z) * u1.z, silu_f(x1.w) * u1.w);
+      }
+      const size_t row = compact ? (size_t)(e.tok0 + e.jb + t) : (size_t)e.s_idx[e.jb + t];
+      *reinterpret_cast<uint4*>(dst + row * ld + col + (l & 3) * 8) = pack8_bf16(x0, x1);
+    }
+  }
+}
+
+}  // namespace
+
+template <int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                    const GemmArgs args) {
@@ -117,94 +222,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
 
-  // epilogue state shared by the direct (CS = 1) and reduced (CS > 1) paths
-  const int q = warp & 3;           // TMEM lane quarter this warp may access
-  const int lr = q * 32 + lane;     // tile row = TMEM lane = feature row in tile
-  const int et = threadIdx.x - 64;  // 0..127 in the epilogue warps
-  const int d = args.d;
-  const bool resid = args.epi == EPI_O || args.epi == EPI_DOWN;
-  const int f128 = ft * kGemmBM + lr;
-  float* stg = stg_all + q * kStgFloats;
-  __nv_bfloat16* stg_h = reinterpret_cast<__nv_bfloat16*>(stg);
-  const int fbase = ft * kGemmBM + q * 32;  // first feature of this warp
-
-  // residual operand (fp32 h, contiguous rows); rows past ntok are clamped to a
-  // valid row and never stored, so every load is issued unconditionally
-  auto load_res = [&](int c, float (&dst)[32]) {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int jj = min(c * 32 + i, ntok - 1);
-      dst[i] = __ldcg(&args.h32[(size_t)(tok0 + jj) * d + f128]);
+  // epilogue state
+  const int q = warp & 3;  // TMEM lane quarter this warp may access (warps 2-5)
+  float* stg = stg_all + q * kBlk;
+  EpiCtx e;
+  e.tok0 = tok0;
+  e.jb = 0;
+  e.nval = 0;
+  e.fbase = EPI == EPI_GU ? ft * 64 + (q & 1) * 32 : ft * kGemmBM + q * 32;
+  e.d = args.d;
+  e.lane = lane;
+  e.s_idx = s_idx;
+  const bool gate_warp = EPI != EPI_GU || q < 2;  // GU: warps q >= 2 hold the up rows
+  float4 res[8];
+  auto at_chunk = [&](int c) {
+    e.jb = c * 32;
+    e.nval = ntok - e.jb;
+  };
+  // the warp's block of chunk c is in stg; finish it (GU: pair with warp q^2)
+  auto finish = [&]() {
+    if (EPI == EPI_GU) {
+      named_bar_sync(2 + (q & 1), 64);  // both halves of the pair are staged
+      if (gate_warp) finish_block<EPI>(args, e, stg, stg_all + (q + 2) * kBlk, res);
+      named_bar_sync(2 + (q & 1), 64);  // warp q+2 may overwrite its block
+    } else {
+      finish_block<EPI>(args, e, stg, nullptr, res);
+      __syncwarp();
     }
   };
-  // fused epilogue of token chunk c (tokens tok0 + 32c ..) from this thread's
-  // accumulator row v and residuals res
-  auto apply = [&](int c, const float (&v)[32], const float (&res)[32]) {
-    const int jb = c * 32;
-    const int nval = ntok - jb;
-    if (args.epi == EPI_QKV || args.epi == EPI_DOWN) {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) stg_h[i * 32 + lane] = f2bf(args.epi == EPI_DOWN ? res[i] + v[i] : v[i]);
-      __syncwarp();
-      const int part = fbase / d, col = fbase - part * d;
-      __nv_bfloat16* dst =
-          args.epi == EPI_DOWN
-              ? (__nv_bfloat16*)args.y_cache
-              : (part == 0 ? (__nv_bfloat16*)args.q_out
-                           : (part == 1 ? (__nv_bfloat16*)args.k_cache : (__nv_bfloat16*)args.v_cache));
-      const bool compact = args.epi == EPI_QKV && part == 0;
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int tk = k * 8 + (lane >> 2);
-        if (tk < nval) {
-          const size_t row = compact ? (size_t)(tok0 + jb + tk) : (size_t)s_idx[jb + tk];
-          *reinterpret_cast<uint4*>(dst + row * d + col + (lane & 3) * 8) =
-              reinterpret_cast<const uint4*>(stg_h)[tk * 4 + (lane & 3)];
-        }
-      }
-      __syncwarp();
-    } else if (args.epi == EPI_O) {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) stg[i * 32 + lane] = v[i] + res[i];
-      __syncwarp();
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int tk = k * 4 + (lane >> 3);
-        if (tk < nval)
-          *reinterpret_cast<float4*>(args.h32 + (size_t)(tok0 + jb + tk) * d + fbase + (lane & 7) * 4) =
-              reinterpret_cast<const float4*>(stg)[tk * 8 + (lane & 7)];
-      }
-      __syncwarp();
-    } else {  // EPI_GU
-      // gate rows are TMEM lanes 0-63 (warps q = 0, 1), up rows lanes 64-127
-      // (q = 2, 3): warp q+2 parks its values in its staging buffer, warp q reads
-      // them, forms silu(g) * u and stores it; two 64-thread barriers per chunk
-      if (q >= 2) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) stg[i * 32 + lane] = v[i];
-      }
-      named_bar_sync(2 + (q & 1), 64);
-      if (q < 2) {
-        const float* up = stg_all + (q + 2) * kStgFloats;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) stg_h[i * 32 + lane] = f2bf(silu_f(v[i]) * up[i * 32 + lane]);
-        __syncwarp();
-        const int F = args.gu_F;
-        __nv_bfloat16* out = (__nv_bfloat16*)args.act_out + ft * 64 + q * 32;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int tk = k * 8 + (lane >> 2);
-          if (tk < nval)
-            *reinterpret_cast<uint4*>(out + (size_t)(tok0 + jb + tk) * F + (lane & 3) * 8) =
-                reinterpret_cast<const uint4*>(stg_h)[tk * 4 + (lane & 3)];
-        }
-        __syncwarp();
-      }
-      named_bar_sync(2 + (q & 1), 64);  // warp q+2 may refill its buffer
-    }
-  };
-
-  float res[32];  // epilogue warps: residuals of the chunk being finished
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -214,8 +259,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int issued = 0;
       const int nbox = ncols >> 6;
       const uint32_t bytes = kStageA + nbox * (64 * kGemmBK * 2);
-      const int yA0 = (args.epi == EPI_GU) ? ft * 64 : ft * kGemmBM;
-      const int yA1 = (args.epi == EPI_GU) ? args.gu_F + ft * 64 : ft * kGemmBM + 64;
+      const int yA0 = (EPI == EPI_GU) ? ft * 64 : ft * kGemmBM;
+      const int yA1 = (EPI == EPI_GU) ? args.gu_F + ft * 64 : ft * kGemmBM + 64;
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1)) {
           *s_abort = 1;
@@ -269,6 +314,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue, part 1
+    const int et = threadIdx.x - 64;
     for (int j = et; j < ntok; j += 128) s_idx[j] = args.idx[tok0 + j];
     if (!mbar_wait(tfull, 0)) *s_epi_abort = 1;
     named_bar_sync(1, 128);
@@ -276,42 +322,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // a K range of zero length (more slices than k-blocks) leaves TMEM unwritten
     const bool have_acc = !*s_epi_abort && !*s_abort && kb1 > kb0;
     const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
-    if (CS == 1) {
-      float res_nx[32];
-      if (resid) load_res(0, res_nx);
-      for (int c = 0; c < nchunks && have_acc; ++c) {
-        if (resid) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) res[i] = res_nx[i];
-          if (c + 1 < nchunks) load_res(c + 1, res_nx);
-        }
-        uint32_t r[32];
+    // TMEM chunk c -> token-major block at dst (this lane = feature, 32 tokens)
+    auto drain_chunk = [&](int c, float* dst) {
+      uint32_t r[32];
+      if (have_acc) {
         tmem_ld32(taddr + (uint32_t)(c * 32), r);
         tmem_ld_wait();
-        float v[32];
+      } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-        apply(c, v, res);
+        for (int i = 0; i < 32; ++i) r[i] = 0u;
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) dst[i * 32 + lane] = __uint_as_float(r[i]);
+    };
+    if (CS == 1) {
+      for (int c = 0; c < nchunks; ++c) {
+        at_chunk(c);
+        if (gate_warp) load_res<EPI>(args, e, ntok, res);
+        drain_chunk(c, stg);
+        __syncwarp();
+        finish();
       }
     } else {
-      // residuals of the first chunk this CTA will finish, in flight across the barrier
-      if (resid && kr < nchunks) load_res(kr, res);
-      // park this CTA's partial for the cluster reduction
-      for (int c = 0; c < nchunks; ++c) {
-        uint32_t r[32];
-        if (have_acc) {
-          tmem_ld32(taddr + (uint32_t)(c * 32), r);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = 0u;
-        }
-        float4* dst = reinterpret_cast<float4*>(rb + c * kRbChunk + q * kRbQuarter + lane * kRbLane);
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                               __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+      // residuals of the first chunk this CTA finishes, in flight across the barrier
+      if (kr < nchunks) {
+        at_chunk(kr);
+        load_res<EPI>(args, e, ntok, res);
       }
+      for (int c = 0; c < nchunks; ++c) drain_chunk(c, rb + c * kRbChunk + q * kBlk);
     }
   }
 
@@ -327,27 +365,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (CS > 1) {
     if (warp >= 2) {
       // ---------------------------------------------------------- epilogue, part 2
-      // this CTA finishes chunks c = kr, kr + CS, ... summing the CS partials
-      const uint32_t mine = smem_u32(rb + q * kRbQuarter + lane * kRbLane);
+      // this CTA finishes chunks c = kr, kr + CS, ...: lane l sums float4 l + 32j
+      // (j = 0..7) of the warp's block over the CS partials, into its own block
       for (int c = kr; c < nchunks; c += CS) {
-        if (resid && c != kr) load_res(c, res);  // the first chunk's were loaded before the barrier
-        float v[32];
+        at_chunk(c);
+        if (c != kr) load_res<EPI>(args, e, ntok, res);
+        const uint32_t base = smem_u32(rb + c * kRbChunk + q * kBlk) + 16u * lane;
+        float4 acc[8];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        for (int j = 0; j < 8; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int p = 0; p < CS; ++p) {
-          const uint32_t src = dsmem_addr(mine + (uint32_t)(c * kRbChunk * 4), (uint32_t)p);
-          float4 t[8];  // all of a peer's loads in flight before the first add
+          const uint32_t src = dsmem_addr(base, (uint32_t)p);
+          float4 t[8];  // a peer's eight loads in flight before the first add
 #pragma unroll
-          for (int i = 0; i < 8; ++i) t[i] = ld_dsmem_v4(src + 16u * i);
+          for (int j = 0; j < 8; ++j) t[j] = ld_dsmem_v4(src + 512u * j);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            v[4 * i] += t[i].x;
-            v[4 * i + 1] += t[i].y;
-            v[4 * i + 2] += t[i].z;
-            v[4 * i + 3] += t[i].w;
-          }
+          for (int j = 0; j < 8; ++j) acc[j] = add4(acc[j], t[j]);
         }
-        apply(c, v, res);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) reinterpret_cast<float4*>(stg)[lane + 32 * j] = acc[j];
+        __syncwarp();
+        finish();
       }
     }
     cluster_sync_all();  // peers are done reading this CTA's partial
@@ -373,17 +411,18 @@ static int choose_cluster(int ftiles, int kblocks, int nsm) {
   return best;
 }
 
-int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& a, cudaStream_t st) {
+template <int EPI>
+static int launch_epi(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& a, int cs,
+                      cudaStream_t st) {
   static int attr_done[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PLK_ERR_CUDA;
   if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemBytes) != cudaSuccess)
       return PLK_ERR_CUDA;
     attr_done[dev] = 1;
   }
-  const int cs = choose_cluster(a.ftiles, a.K / kGemmBK, a.num_sms);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs, a.ftiles * a.ttiles_max, 1);
   cfg.blockDim = dim3(kGemmThreads, 1, 1);
@@ -396,8 +435,19 @@ int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArg
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = cs > 1 ? 1 : 0;
-  if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel, tmW, tmX, a) != cudaSuccess) return PLK_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel<EPI>, tmW, tmX, a) != cudaSuccess) return PLK_ERR_CUDA;
   return cudaPeekAtLastError() == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;
+}
+
+int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& a, cudaStream_t st) {
+  const int cs = choose_cluster(a.ftiles, a.K / kGemmBK, a.num_sms);
+  switch (a.epi) {
+    case EPI_QKV: return launch_epi<EPI_QKV>(tmW, tmX, a, cs, st);
+    case EPI_O: return launch_epi<EPI_O>(tmW, tmX, a, cs, st);
+    case EPI_GU: return launch_epi<EPI_GU>(tmW, tmX, a, cs, st);
+    case EPI_DOWN: return launch_epi<EPI_DOWN>(tmW, tmX, a, cs, st);
+    default: return PLK_ERR_ARG;
+  }
 }
 
 }  // namespace plk
