@@ -320,7 +320,7 @@ def run_gpu(args, wl, dist, rank, world, local_rank):
 
     K_ = args.steps
     E = lambda: torch.cuda.Event(enable_timing=True)
-    ev = [[E() for _ in range(12)] for _ in range(K_)]  # 0 start, 1 score, 2 select, 3..10 layer, 11 end
+    ev = [[E() for _ in range(15)] for _ in range(K_)]  # 0 start, 1 score, 2 select, 3..13 layer, 14 end
     if dist is not None:
         dist.barrier(device_ids=[local_rank])
     torch.cuda.synchronize()
@@ -328,7 +328,7 @@ def run_gpu(args, wl, dist, rank, world, local_rank):
         for i in range(K_):
             prep()
             e = ev[i]
-            plk.trace_events(e[3:11])
+            plk.trace_events(e[3:14])
             e[0].record()
             plk.score_drift(dm, Xp, Ut, r, pc, plk.METRIC_L2, score, proxy_out=pnew)
             e[1].record()
@@ -336,7 +336,7 @@ def run_gpu(args, wl, dist, rank, world, local_rank):
             e[2].record()
             plk.layer_step_partial(dm, pw, Xp, idx, seg, K, V, Y, ws)
             plk.proxy_commit(dm, r, idx, seg, pnew, pc)
-            e[11].record()
+            e[14].record()
         torch.cuda.synchronize()
     plk.trace_events([])
     if dist is not None:
@@ -345,10 +345,10 @@ def run_gpu(args, wl, dist, rank, world, local_rank):
     if st != plk.OK:
         raise RuntimeError(f"device status {plk.error_string(st)}")
 
-    step_ms = [e[0].elapsed_time(e[11]) for e in ev]
-    names = ["score", "select", "rmsnorm1", "gemm_qkv", "attention", "gemm_o", "rmsnorm2", "gemm_gu",
-             "gemm_down", "proxy_commit"]
-    bounds = [(0, 1), (1, 2), (3, 4), (4, 5), (5, 6), (6, 7), (7, 8), (8, 9), (9, 10), (10, 11)]
+    step_ms = [e[0].elapsed_time(e[14]) for e in ev]
+    names = ["score", "select", "rmsnorm1", "gemm_qkv", "finish_qkv", "attention", "gemm_o", "rmsnorm2",
+             "gemm_gu", "finish_gu", "gemm_down", "finish_y", "proxy_commit"]
+    bounds = [(0, 1), (1, 2)] + [(i, i + 1) for i in range(3, 14)]
     per = {n: statistics.mean(e[a].elapsed_time(e[b]) for e in ev) * 1e3 for n, (a, b) in zip(names, bounds)}
     total_ms = sum(step_ms)
     total_ms_max = aggregate(dist, total_ms, dev)
@@ -428,7 +428,7 @@ def main():
             dist.destroy_process_group()
     if res is None or rank != 0:
         return 0
-    launches_per_step = 1 + 2 + 7 + 1
+    launches_per_step = 1 + 1 + 11 + 1  # score, select, layer (attention + combine), commit
     line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",

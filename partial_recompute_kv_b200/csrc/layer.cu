@@ -3,14 +3,17 @@
 // Decoding", Sec. 2 "Permanent Deactivation", "Continued Attention",
 // "Algorithmic Complexity"), and the full-recompute baseline (Sec. 1).
 //
-// bf16 chain (7 launches, M read on the device, no host synchronisation):
-//   1 gather rows idx[j] of X, RMSNorm1 -> xn (bf16), x -> h (fp32)
-//   2 tcgen05 GEMM  xn W_qkv^T -> Q (compact), K and V scattered into the caches
-//   3 attention of the M queries over all N cached keys -> a (bf16)
-//   4 tcgen05 GEMM  h += a W_o^T (fp32)
-//   5 RMSNorm2(h) -> hn (bf16)
-//   6 tcgen05 GEMM  hn [W_g; W_u]^T -> silu(g) * u (bf16)
-//   7 tcgen05 GEMM  act W_down^T + h -> Y rows idx[j] (bf16)
+// bf16 chain (10 launches, M read on the device, no host synchronisation):
+//   1 gather rows idx[j] of X, RMSNorm1 -> xn (bf16), x -> h (fp32), zero the QKV sums
+//   2 tcgen05 GEMM  xn W_qkv^T -> QKV sums (fp32, split-K reduce-adds)
+//   3 QKV sums -> Q (compact bf16), K and V scattered into the cache rows idx[j]
+//   4 attention of the M queries over all N cached keys -> a (bf16)
+//   5 tcgen05 GEMM  h += a W_o^T (fp32)
+//   6 RMSNorm2(h) -> hn (bf16), zero the gate/up sums
+//   7 tcgen05 GEMM  hn [W_g; W_u]^T -> gate/up sums (fp32)
+//   8 act = silu(g) * u (bf16)
+//   9 tcgen05 GEMM  h += act W_down^T (fp32)
+//  10 h -> Y rows idx[j] (bf16)
 // fp32 chain: the same steps with SIMT GEMMs into an fp32 scratch and
 // elementwise epilogue kernels.
 #include <math.h>
@@ -64,9 +67,8 @@ Workspace workspace_layout(const plk_dims* dm, int num_sms) {
     w.att_rows = attn_split_rows(dm, num_sms);
     w.att_o = take((size_t)kAttSplitMax * w.att_rows * d * 4);
     w.att_ml = take((size_t)kAttSplitMax * w.att_rows * dm->H * 8);
-  } else {
-    w.c32 = take(4 * Mcap * std::max((size_t)3 * d, 2 * F));
   }
+  w.c32 = take(4 * Mcap * std::max((size_t)3 * d, 2 * F));
   w.total = off;
   return w;
 }
@@ -85,6 +87,19 @@ static EncodeTiledFn encode_fn() {
       fn = reinterpret_cast<EncodeTiledFn>(p);
   }
   return fn;
+}
+
+int make_tmap_f32(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return PLK_ERR_CUDA;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 4};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PLK_OK : PLK_ERR_CUDA;
 }
 
 int make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
@@ -119,17 +134,27 @@ __device__ __forceinline__ float block_sum_f(float v, float* sh) {
   return sh[32];
 }
 
+// zcols % 4 == 0, row 16-byte aligned
+__device__ __forceinline__ void clear_row(float* row, int zcols) {
+  float4* r4 = reinterpret_cast<float4*>(row);
+  for (int c = threadIdx.x; c < (zcols >> 2); c += blockDim.x) r4[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
 // out[j] = RMSNorm(src_row(j)) * g for j < M.  src_row(j) = X[idx[j]] (gather)
-// or H[j] (idx == nullptr); res_out (optional) receives the fp32 source row.
+// or H[j] (idx == nullptr); res_out (optional) receives the fp32 source row;
+// zero_out (optional) gets row j of a [Mcap, zcols] fp32 buffer cleared for the
+// reduce-adds of the GEMM that follows.
 template <typename Tin, typename Tg, typename Tout>
 __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const Tin* __restrict__ X, const int32_t* __restrict__ idx,
                                                            const int32_t* __restrict__ seg_ptr, int B,
                                                            const Tg* __restrict__ g, float eps, int d,
-                                                           Tout* __restrict__ out, float* __restrict__ res_out) {
+                                                           Tout* __restrict__ out, float* __restrict__ res_out,
+                                                           float* __restrict__ zero_out, int zcols) {
   __shared__ float sh[33];
   const int M = seg_ptr[B];
   const int j = blockIdx.x;
   if (j >= M) return;
+  if (zero_out) clear_row(zero_out + (size_t)j * zcols, zcols);
   const size_t row = idx ? (size_t)idx[j] : (size_t)j;
   const Tin* x = X + row * d;
   float ss = 0.f;
@@ -207,12 +232,14 @@ template <typename Tin, typename Tg, typename Tout, int NV>
 __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict__ X, const int32_t* __restrict__ idx,
                                                           const int32_t* __restrict__ seg_ptr, int B,
                                                           const Tg* __restrict__ g, float eps, int d,
-                                                          Tout* __restrict__ out, float* __restrict__ res_out) {
+                                                          Tout* __restrict__ out, float* __restrict__ res_out,
+                                                          float* __restrict__ zero_out, int zcols) {
   constexpr int E = Vec16<Tin>::E;
   __shared__ float sh[33];
   const int M = seg_ptr[B];
   const int j = blockIdx.x;
   if (j >= M) return;
+  if (zero_out) clear_row(zero_out + (size_t)j * zcols, zcols);
   const size_t row = idx ? (size_t)idx[j] : (size_t)j;
   const uint4* xv = reinterpret_cast<const uint4*>(X + row * d);
   const int nvec = d / E;
@@ -252,12 +279,83 @@ __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict_
 // Picks the register-resident kernel when the row fits, else the looping one.
 template <typename Tin, typename Tg, typename Tout>
 static void launch_rmsnorm(const Tin* X, const int32_t* idx, const int32_t* seg, int B, const Tg* g, float eps,
-                           int d, Tout* out, int grid, cudaStream_t st, float* res_out = nullptr) {
+                           int d, Tout* out, int grid, cudaStream_t st, float* res_out = nullptr,
+                           float* zero_out = nullptr, int zcols = 0) {
   constexpr int E = Vec16<Tin>::E;
   if (d % E == 0 && d <= 4 * 256 * E)
-    rmsnorm_vec_kernel<Tin, Tg, Tout, 4><<<grid, 256, 0, st>>>(X, idx, seg, B, g, eps, d, out, res_out);
+    rmsnorm_vec_kernel<Tin, Tg, Tout, 4><<<grid, 256, 0, st>>>(X, idx, seg, B, g, eps, d, out, res_out, zero_out,
+                                                                zcols);
   else
-    rmsnorm_rows_kernel<Tin, Tg, Tout><<<grid, 256, 0, st>>>(X, idx, seg, B, g, eps, d, out, res_out);
+    rmsnorm_rows_kernel<Tin, Tg, Tout><<<grid, 256, 0, st>>>(X, idx, seg, B, g, eps, d, out, res_out, zero_out, zcols);
+}
+
+// ---------------------------------------------------------------------------
+// finishing kernels of the bf16 path: the tcgen05 GEMM leaves fp32 sums; these
+// apply the nonlinearity or scatter and store bf16.  One block per compact row
+// (grid-stride over the M live rows), 8 features per thread and step.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+
+__device__ __forceinline__ void load8(const float* p, float* f) {
+  const float4 a = __ldcs(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+  f[0] = a.x, f[1] = a.y, f[2] = a.z, f[3] = a.w, f[4] = b.x, f[5] = b.y, f[6] = b.z, f[7] = b.w;
+}
+
+// [q | k | v] sums of compact row j -> Q[j] (compact), K/V cache rows idx[j]
+__global__ void __launch_bounds__(256) finish_qkv_kernel(const float* __restrict__ qkv32,
+                                                         const int32_t* __restrict__ idx,
+                                                         const int32_t* __restrict__ seg_ptr, int B, int d,
+                                                         __nv_bfloat16* __restrict__ q, __nv_bfloat16* __restrict__ Kc,
+                                                         __nv_bfloat16* __restrict__ Vc) {
+  const int M = seg_ptr[B];
+  const int nv = 3 * d / 8;
+  for (int j = blockIdx.x; j < M; j += gridDim.x) {
+    const size_t row = (size_t)idx[j];
+    const float* src = qkv32 + (size_t)j * 3 * d;
+    for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+      const int c = v * 8, part = c / d, col = c - part * d;
+      float f[8];
+      load8(src + c, f);
+      __nv_bfloat16* dst = part == 0 ? q + (size_t)j * d : (part == 1 ? Kc : Vc) + row * d;
+      store_vec<__nv_bfloat16, 8>(dst + col, f);
+    }
+  }
+}
+
+// [g | u] sums of compact row j -> act[j] = silu(g) * u
+__global__ void __launch_bounds__(256) finish_gu_kernel(const float* __restrict__ gu32,
+                                                        const int32_t* __restrict__ seg_ptr, int B, int F,
+                                                        __nv_bfloat16* __restrict__ act) {
+  const int M = seg_ptr[B];
+  const int nv = F / 8;
+  for (int j = blockIdx.x; j < M; j += gridDim.x) {
+    const float* src = gu32 + (size_t)j * 2 * F;
+    for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+      float g[8], u[8];
+      load8(src + v * 8, g);
+      load8(src + F + v * 8, u);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) g[e] = silu_f(g[e]) * u[e];
+      store_vec<__nv_bfloat16, 8>(act + (size_t)j * F + v * 8, g);
+    }
+  }
+}
+
+// residual-stream sums of compact row j -> Y cache row idx[j]
+__global__ void __launch_bounds__(256) finish_y_kernel(const float* __restrict__ h32, const int32_t* __restrict__ idx,
+                                                       const int32_t* __restrict__ seg_ptr, int B, int d,
+                                                       __nv_bfloat16* __restrict__ Y) {
+  const int M = seg_ptr[B];
+  const int nv = d / 8;
+  for (int j = blockIdx.x; j < M; j += gridDim.x) {
+    const size_t row = (size_t)idx[j];
+    for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+      float f[8];
+      load8(h32 + (size_t)j * d + v * 8, f);
+      store_vec<__nv_bfloat16, 8>(Y + row * d + v * 8, f);
+    }
+  }
 }
 
 __global__ void fill_identity_kernel(int32_t* iota, int32_t* seg, int B, int N) {
@@ -389,7 +487,9 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   __nv_bfloat16* hn = (__nv_bfloat16*)(ws + L.hn);
   __nv_bfloat16* act = (__nv_bfloat16*)(ws + L.act);
 
-  CUtensorMap tW_qkv, tW_o, tW_gu, tW_down, tX_xn, tX_a, tX_hn, tX_act;
+  float* c32 = (float*)(ws + L.c32);  // [Mcap, 3d] QKV sums, later [Mcap, 2F] gate/up sums
+
+  CUtensorMap tW_qkv, tW_o, tW_gu, tW_down, tX_xn, tX_a, tX_hn, tX_act, tO_qkv, tO_h, tO_gu;
   PLK_TRY(make_tmap_bf16(&tW_qkv, w->w_qkv, 3ull * d, d, 64));
   PLK_TRY(make_tmap_bf16(&tW_o, w->w_o, (uint64_t)d, d, 64));
   PLK_TRY(make_tmap_bf16(&tW_gu, w->w_gu, 2ull * F, d, 64));
@@ -398,63 +498,67 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   PLK_TRY(make_tmap_bf16(&tX_a, a, (uint64_t)Mcap, d, 64));
   PLK_TRY(make_tmap_bf16(&tX_hn, hn, (uint64_t)Mcap, d, 64));
   PLK_TRY(make_tmap_bf16(&tX_act, act, (uint64_t)Mcap, F, 64));
+  PLK_TRY(make_tmap_f32(&tO_qkv, c32, (uint64_t)Mcap, 3ull * d));
+  PLK_TRY(make_tmap_f32(&tO_h, h32, (uint64_t)Mcap, d));
+  PLK_TRY(make_tmap_f32(&tO_gu, c32, (uint64_t)Mcap, 2ull * F));
 
   GemmArgs g{};
-  g.d = d;
-  g.Mcap = Mcap;
   g.seg_ptr = seg;
   g.B = B;
-  g.idx = idx;
   g.ttiles_max = ceil_div(Mcap, kGemmBNMax);
   g.num_sms = L.num_sms;
+  const int rgrid = std::min(Mcap, 2 * L.num_sms);  // finishing kernels: grid-stride over M rows
 
   trace_mark(0, st);
-  // also stages x (fp32) in h32: the O projection's epilogue adds its residual there
+  // x (fp32) staged in h32 takes the O projection's adds; the QKV sums start at 0
   launch_rmsnorm<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(X, idx, seg, B, (const __nv_bfloat16*)w->g1, dm->eps, d,
-                                                              xn, Mcap, st, h32);
+                                                              xn, Mcap, st, h32, c32, 3 * d);
   PLK_LAUNCHED();
   trace_mark(1, st);
 
-  g.epi = EPI_QKV;
   g.K = d;
   g.ftiles = 3 * d / kGemmBM;
-  g.q_out = q;
-  g.k_cache = Kc;
-  g.v_cache = Vc;
-  PLK_TRY(launch_gemm_tc(tW_qkv, tX_xn, g, st));
+  g.gu_F = 0;
+  PLK_TRY(launch_gemm_tc(tW_qkv, tX_xn, tO_qkv, g, st));
   trace_mark(2, st);
+
+  finish_qkv_kernel<<<rgrid, 256, 0, st>>>(c32, idx, seg, B, d, q, (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc);
+  PLK_LAUNCHED();
+  trace_mark(3, st);
 
   PLK_TRY(launch_attention_bf16(dm, q, Kc, Vc, a, seg, (float*)(ws + L.att_o), ws + L.att_ml, kAttSplitMax,
                                 L.att_rows, L.num_sms, st));
-  trace_mark(3, st);
-
-  g.epi = EPI_O;
-  g.K = d;
-  g.ftiles = d / kGemmBM;
-  g.x_in = X;
-  g.h32 = h32;
-  PLK_TRY(launch_gemm_tc(tW_o, tX_a, g, st));
   trace_mark(4, st);
 
-  launch_rmsnorm<float, __nv_bfloat16, __nv_bfloat16>(h32, nullptr, seg, B, (const __nv_bfloat16*)w->g2, dm->eps, d, hn,
-                                                      Mcap, st);
-  PLK_LAUNCHED();
+  g.K = d;
+  g.ftiles = d / kGemmBM;
+  PLK_TRY(launch_gemm_tc(tW_o, tX_a, tO_h, g, st));  // h = x + a W_o^T
   trace_mark(5, st);
 
-  g.epi = EPI_GU;
+  launch_rmsnorm<float, __nv_bfloat16, __nv_bfloat16>(h32, nullptr, seg, B, (const __nv_bfloat16*)w->g2, dm->eps, d, hn,
+                                                      Mcap, st, nullptr, c32, 2 * F);
+  PLK_LAUNCHED();
+  trace_mark(6, st);
+
   g.K = d;
   g.ftiles = F / 64;
   g.gu_F = F;
-  g.act_out = act;
-  PLK_TRY(launch_gemm_tc(tW_gu, tX_hn, g, st));
-  trace_mark(6, st);
+  PLK_TRY(launch_gemm_tc(tW_gu, tX_hn, tO_gu, g, st));
+  trace_mark(7, st);
 
-  g.epi = EPI_DOWN;
+  finish_gu_kernel<<<rgrid, 256, 0, st>>>(c32, seg, B, F, act);
+  PLK_LAUNCHED();
+  trace_mark(8, st);
+
   g.K = F;
   g.ftiles = d / kGemmBM;
-  g.y_cache = Y;
-  PLK_TRY(launch_gemm_tc(tW_down, tX_act, g, st));
-  trace_mark(7, st);
+  g.gu_F = 0;
+  PLK_TRY(launch_gemm_tc(tW_down, tX_act, tO_h, g, st));  // y = h + act W_down^T
+  trace_mark(9, st);
+
+  finish_y_kernel<<<rgrid, 256, 0, st>>>(h32, idx, seg, B, d, (__nv_bfloat16*)Y);
+  PLK_LAUNCHED();
+  trace_mark(10, st);
   return PLK_OK;
 }
 

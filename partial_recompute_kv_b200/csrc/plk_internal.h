@@ -17,6 +17,7 @@ constexpr int kGemmBNMax = 256;   // tokens per tile (UMMA N, runtime 64..256)
 constexpr int kGemmBK = 64;       // K per stage: one 128-byte swizzle row of bf16
 constexpr int kGemmStages = 4;
 constexpr int kGemmThreads = 192; // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int kGemmSplitMax = 16; // most K slices of one GEMM
 
 // ---- workspace layout -------------------------------------------------------
 struct Workspace {
@@ -24,7 +25,7 @@ struct Workspace {
   // offsets (bytes)
   size_t iota = 0, seg = 0;              // identity active set for the full step
   size_t xn = 0, q = 0, a = 0, h32 = 0, hn = 0, act = 0;
-  size_t c32 = 0;                        // fp32 path: GEMM output scratch [Mcap, max(3d, 2F)]
+  size_t c32 = 0;                        // fp32 GEMM sums [Mcap, max(3d, 2F)] (QKV, then gate/up)
   int num_sms = 0;
   size_t att_o = 0, att_ml = 0;          // split-KV attention partials
   int att_rows = 0;
@@ -36,6 +37,9 @@ int device_sm_count();
 // 2D bf16 tensor [rows, cols] row-major (cols contiguous), 128-byte swizzle,
 // box {64 cols, box_rows rows}.
 int make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// 2D fp32 tensor [rows, cols] row-major, no swizzle, box {32 cols, 32 rows}:
+// the target of the GEMM's bulk reduce-adds.
+int make_tmap_f32(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols);
 
 // ---- launches (all asynchronous on `st`; return PLK_OK / PLK_ERR_CUDA) -------
 int launch_select(const plk_dims* dims, const float* score, const uint8_t* lock_in, uint8_t* lock_out,
@@ -51,30 +55,19 @@ int run_layer(const plk_dims* dims, const plk_weights* w, const void* X, const i
               const int32_t* seg_ptr, bool full, void* K_cache, void* V_cache, void* Y, void* ws,
               size_t ws_bytes, cudaStream_t st);
 
-// epilogue modes of the tcgen05 GEMM
-enum GemmEpi { EPI_QKV = 0, EPI_O = 1, EPI_GU = 2, EPI_DOWN = 3 };
-
+// Arguments of the tcgen05 GEMM out[t, f] += sum_k X[t, k] W[f, k] over the
+// M = seg_ptr[B] compact tokens (fp32 out, added with bulk reduce-adds).
 struct GemmArgs {
-  int epi;
   int K;                   // reduction length, multiple of 64
   int ftiles;              // 128-row feature tiles
-  int gu_F;                // EPI_GU: F (tile f = gate rows f*64.. and up rows F + f*64..)
-  int d;                   // model dim
-  int Mcap;                // token capacity of the activation buffer
+  int gu_F;                // gate/up GEMM: F (tile f = gate rows f*64.. and up rows F + f*64..), else 0
   const int32_t* seg_ptr;  // M = seg_ptr[B]
   int B;
-  const int32_t* idx;      // compact token -> flattened row
-  void* q_out;             // EPI_QKV: Q compact [Mcap, d] bf16
-  void* k_cache;           // EPI_QKV
-  void* v_cache;           // EPI_QKV
-  const void* x_in;        // EPI_O residual source X [B*N, d] bf16
-  float* h32;              // EPI_O output, EPI_DOWN residual [Mcap, d]
-  void* act_out;           // EPI_GU: [Mcap, F] bf16
-  void* y_cache;           // EPI_DOWN
   int ttiles_max;          // token tiles of Mcap (grid rows; tiles past M exit at once)
   int num_sms;             // SM count, for the split-K choice
 };
-int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const GemmArgs& a, cudaStream_t st);
+int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const CUtensorMap& tmOut, const GemmArgs& a,
+                   cudaStream_t st);
 
 constexpr int kAttSplitMax = 4;
 int attn_split_rows(const plk_dims* dims, int num_sms);
