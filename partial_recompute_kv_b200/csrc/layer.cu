@@ -505,7 +505,6 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   GemmArgs g{};
   g.seg_ptr = seg;
   g.B = B;
-  g.ttiles_max = ceil_div(Mcap, kGemmBNMax);
   g.num_sms = L.num_sms;
   const int rgrid = std::min(Mcap, 2 * L.num_sms);  // finishing kernels: grid-stride over M rows
 

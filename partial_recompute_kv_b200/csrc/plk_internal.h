@@ -17,7 +17,6 @@ constexpr int kGemmBNMax = 256;   // tokens per tile (UMMA N, runtime 64..256)
 constexpr int kGemmBK = 64;       // K per stage: one 128-byte swizzle row of bf16
 constexpr int kGemmStages = 4;
 constexpr int kGemmThreads = 192; // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
-constexpr int kGemmSplitMax = 16; // most K slices of one GEMM
 
 // ---- workspace layout -------------------------------------------------------
 struct Workspace {
@@ -63,8 +62,7 @@ struct GemmArgs {
   int gu_F;                // gate/up GEMM: F (tile f = gate rows f*64.. and up rows F + f*64..), else 0
   const int32_t* seg_ptr;  // M = seg_ptr[B]
   int B;
-  int ttiles_max;          // token tiles of Mcap (grid rows; tiles past M exit at once)
-  int num_sms;             // SM count, for the split-K choice
+  int num_sms;             // SM count: one persistent CTA per SM
 };
 int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const CUtensorMap& tmOut, const GemmArgs& a,
                    cudaStream_t st);
