@@ -320,36 +320,47 @@ def run_gpu(args, wl, dist, rank, world, local_rank):
 
     K_ = args.steps
     E = lambda: torch.cuda.Event(enable_timing=True)
-    ev = [[E() for _ in range(15)] for _ in range(K_)]  # 0 start, 1 score, 2 select, 3..13 layer, 14 end
+    ev = [(E(), E()) for _ in range(K_)]
     if dist is not None:
         dist.barrier(device_ids=[local_rank])
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
         for i in range(K_):
             prep()
-            e = ev[i]
-            plk.trace_events(e[3:14])
-            e[0].record()
-            plk.score_drift(dm, Xp, Ut, r, pc, plk.METRIC_L2, score, proxy_out=pnew)
-            e[1].record()
-            plk.select_active(dm, score, lock_in, lock, plk.SEL_TOPK_LARGEST, 0.0, M, idx, seg)
-            e[2].record()
-            plk.layer_step_partial(dm, pw, Xp, idx, seg, K, V, Y, ws)
-            plk.proxy_commit(dm, r, idx, seg, pnew, pc)
-            e[14].record()
+            ev[i][0].record()
+            step(Xp)
+            ev[i][1].record()
         torch.cuda.synchronize()
-    plk.trace_events([])
     if dist is not None:
         dist.barrier(device_ids=[local_rank])
     st = plk.get_status()
     if st != plk.OK:
         raise RuntimeError(f"device status {plk.error_string(st)}")
+    step_ms = [a.elapsed_time(b) for a, b in ev]
 
-    step_ms = [e[0].elapsed_time(e[14]) for e in ev]
+    # per-kernel breakdown: separate, untimed-for-value steps with an event between
+    # every kernel (the events themselves add a little time to each gap)
+    nb = min(K_, 20)
+    bev = [[E() for _ in range(15)] for _ in range(nb)]  # 0 start, 1 score, 2 select, 3..13 layer, 14 end
+    for i in range(nb):
+        prep()
+        e = bev[i]
+        plk.trace_events(e[3:14])
+        e[0].record()
+        plk.score_drift(dm, Xp, Ut, r, pc, plk.METRIC_L2, score, proxy_out=pnew)
+        e[1].record()
+        plk.select_active(dm, score, lock_in, lock, plk.SEL_TOPK_LARGEST, 0.0, M, idx, seg)
+        e[2].record()
+        plk.layer_step_partial(dm, pw, Xp, idx, seg, K, V, Y, ws)
+        plk.proxy_commit(dm, r, idx, seg, pnew, pc)
+        e[14].record()
+    torch.cuda.synchronize()
+    plk.trace_events([])
     names = ["score", "select", "rmsnorm1", "gemm_qkv", "finish_qkv", "attention", "gemm_o", "rmsnorm2",
              "gemm_gu", "finish_gu", "gemm_down", "finish_y", "proxy_commit"]
     bounds = [(0, 1), (1, 2)] + [(i, i + 1) for i in range(3, 14)]
-    per = {n: statistics.mean(e[a].elapsed_time(e[b]) for e in ev) * 1e3 for n, (a, b) in zip(names, bounds)}
+    per = {n: statistics.mean(e[a].elapsed_time(e[b]) for e in bev) * 1e3 for n, (a, b) in zip(names, bounds)}
+    per["traced_step"] = statistics.mean(e[0].elapsed_time(e[14]) for e in bev) * 1e3
     total_ms = sum(step_ms)
     total_ms_max = aggregate(dist, total_ms, dev)
     ms_per_step = total_ms_max / K_

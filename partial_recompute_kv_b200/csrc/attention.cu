@@ -90,6 +90,8 @@ __global__ void __launch_bounds__(kAttThreads) attn_bf16_kernel(const __grid_con
                                                                 __nv_bfloat16* __restrict__ Aout,
                                                                 const int32_t* __restrict__ seg_ptr, int B, int N,
                                                                 int d, float scale_log2, AttnSplit sp) {
+  pdl_wait();
+  pdl_trigger();
   const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z / sp.smax, split = blockIdx.z % sp.smax;
   const int seg0 = seg_ptr[b], seg1 = seg_ptr[b + 1];
   const int r0 = seg0 + qt * kAttBQ;
@@ -271,6 +273,8 @@ __global__ void __launch_bounds__(kAttThreads) attn_bf16_kernel(const __grid_con
 // out[row, h] = sum_s 2^(m_s - m) o_s / sum_s 2^(m_s - m) l_s, one CTA per active row.
 __global__ void __launch_bounds__(256) attn_combine_kernel(const int32_t* __restrict__ seg_ptr, int B, int H,
                                                            int d, AttnSplit sp, __nv_bfloat16* __restrict__ Aout) {
+  pdl_wait();
+  pdl_trigger();
   const int j = blockIdx.x;
   if (j >= seg_ptr[B]) return;
   const int S = attn_splits(seg_ptr, B, H, sp.smax, sp.nsm);
@@ -359,13 +363,11 @@ int launch_attention_bf16(const plk_dims* dims, const void* q, const void* K_cac
   const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->hd));
   AttnSplit sp{o_part, (float2*)ml, std::max(1, std::min(smax, ceil_div(N, kAttBK))), part_rows, num_sms};
   dim3 grid(ceil_div(N, kAttBQ), H, B * sp.smax);
-  attn_bf16_kernel<<<grid, kAttThreads, kAttSmem, st>>>(tmK, tmV, (const __nv_bfloat16*)q, (__nv_bfloat16*)a_out,
-                                                        seg_ptr, B, N, d, scale_log2, sp);
-  if (cudaPeekAtLastError() != cudaSuccess) return PLK_ERR_CUDA;
-  if (sp.smax > 1) {
-    attn_combine_kernel<<<part_rows, 256, 0, st>>>(seg_ptr, B, H, d, sp, (__nv_bfloat16*)a_out);
-  }
-  return cudaPeekAtLastError() == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;
+  const int rc = launch_pdl(attn_bf16_kernel, grid, dim3(kAttThreads), kAttSmem, st, tmK, tmV,
+                            (const __nv_bfloat16*)q, (__nv_bfloat16*)a_out, seg_ptr, B, N, d, scale_log2, sp);
+  if (rc != PLK_OK || sp.smax == 1) return rc;
+  return launch_pdl(attn_combine_kernel, dim3(part_rows), dim3(256), 0, st, seg_ptr, B, H, d, sp,
+                    (__nv_bfloat16*)a_out);
 }
 
 int launch_attention_f32(const plk_dims* dims, const float* q, const float* K_cache, const float* V_cache,

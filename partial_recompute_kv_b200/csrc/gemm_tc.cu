@@ -121,12 +121,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   float* stg_all = reinterpret_cast<float*>(smem + kOffStg);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // seg_ptr comes from a kernel before the predecessor: already complete (see pdl_wait)
   const int M = args.seg_ptr[args.B];
-  if (M <= 0) return;
-  const int ttiles = ceil_div(M, kGemmBNMax);
+  const int ttiles = ceil_div(max(M, 0), kGemmBNMax);
   const int tiles = args.ftiles * ttiles;
   const int KB = args.K / kGemmBK;
-  if (SegWalk(blockIdx.x, gridDim.x, tiles, KB).done()) return;  // no iterations for this CTA
+  if (M <= 0 || SegWalk(blockIdx.x, gridDim.x, tiles, KB).done()) {  // no iterations for this CTA
+    pdl_wait();
+    return;
+  }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kGemmStages; ++i) {
@@ -152,32 +155,57 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
+  if (warp != 0) {
+    pdl_wait();
+    pdl_trigger();
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (elect_one()) {
+      // weight rows of tile t (gate/up tile: 64 gate rows, then the 64 up rows)
+      auto load_a = [&](int stage, const TileGeom& t, int kb) {
+        const int yA0 = args.gu_F ? t.ft * 64 : t.ft * kGemmBM;
+        const int yA1 = args.gu_F ? args.gu_F + t.ft * 64 : t.ft * kGemmBM + 64;
+        uint8_t* a = sA + stage * kStageA;
+        tma_load_2d(a, &tmW, kb * kGemmBK, yA0, &full[stage]);
+        tma_load_2d(a + 8192, &tmW, kb * kGemmBK, yA1, &full[stage]);
+      };
+      auto stage_bytes = [](const TileGeom& t) { return (uint32_t)(kStageA + (t.ncols >> 6) * (64 * kGemmBK * 2)); };
       SegWalk w(blockIdx.x, gridDim.x, tiles, KB);
       int u, kb0, kb1, stage = 0;
+      // The weights are no kernel's output: the first stages' weight loads start
+      // before the wait for the predecessor, overlapping its tail.
+      int pre = 0;
+      {
+        SegWalk w2 = w;
+        while (pre < kGemmStages && w2.next(u, kb0, kb1)) {
+          const TileGeom t(u, ttiles, M);
+          for (int kb = kb0; kb < kb1 && pre < kGemmStages; ++kb, ++pre) {
+            mbar_expect_tx(&full[pre], stage_bytes(t));
+            load_a(pre, t, kb);
+          }
+        }
+      }
+      pdl_wait();
+      pdl_trigger();
       uint32_t phase = 0;
       long long issued = 0;
       while (!*s_abort && w.next(u, kb0, kb1)) {
         const TileGeom t(u, ttiles, M);
         const int nbox = t.ncols >> 6;
-        const uint32_t bytes = kStageA + nbox * (64 * kGemmBK * 2);
-        const int yA0 = args.gu_F ? t.ft * 64 : t.ft * kGemmBM;
-        const int yA1 = args.gu_F ? args.gu_F + t.ft * 64 : t.ft * kGemmBM + 64;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1)) {
-            *s_abort = 1;
-            break;
+          if (issued >= pre) {  // stages past the prefetched ones: wait for a free slot
+            if (!mbar_wait(&empty[stage], phase ^ 1)) {
+              *s_abort = 1;
+              break;
+            }
+            mbar_expect_tx(&full[stage], stage_bytes(t));
+            load_a(stage, t, kb);
           }
-          mbar_expect_tx(&full[stage], bytes);
-          uint8_t* a = sA + stage * kStageA;
           uint8_t* b = sB + stage * kStageB;
-          const int x = kb * kGemmBK;
-          tma_load_2d(a, &tmW, x, yA0, &full[stage]);
-          tma_load_2d(a + 8192, &tmW, x, yA1, &full[stage]);
-          for (int j = 0; j < nbox; ++j) tma_load_2d(b + j * 8192, &tmX, x, t.tok0 + j * 64, &full[stage]);
+          for (int j = 0; j < nbox; ++j)
+            tma_load_2d(b + j * 8192, &tmX, kb * kGemmBK, t.tok0 + j * 64, &full[stage]);
           ++issued;
           if (++stage == kGemmStages) {
             stage = 0;
@@ -313,8 +341,7 @@ int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const CUtenso
     attr_done[dev] = 1;
   }
   // persistent: one CTA per SM, each owning an equal share of the k-block iterations
-  gemm_tc_kernel<<<a.num_sms, kGemmThreads, kSmemBytes, st>>>(tmW, tmX, tmOut, a);
-  return cudaPeekAtLastError() == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;
+  return launch_pdl(gemm_tc_kernel, dim3(a.num_sms), dim3(kGemmThreads), kSmemBytes, st, tmW, tmX, tmOut, a);
 }
 
 }  // namespace plk

@@ -151,6 +151,8 @@ __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const Tin* __restrict
                                                            Tout* __restrict__ out, float* __restrict__ res_out,
                                                            float* __restrict__ zero_out, int zcols) {
   __shared__ float sh[33];
+  pdl_wait();
+  pdl_trigger();
   const int M = seg_ptr[B];
   const int j = blockIdx.x;
   if (j >= M) return;
@@ -236,6 +238,8 @@ __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict_
                                                           float* __restrict__ zero_out, int zcols) {
   constexpr int E = Vec16<Tin>::E;
   __shared__ float sh[33];
+  pdl_wait();
+  pdl_trigger();
   const int M = seg_ptr[B];
   const int j = blockIdx.x;
   if (j >= M) return;
@@ -278,15 +282,15 @@ __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict_
 
 // Picks the register-resident kernel when the row fits, else the looping one.
 template <typename Tin, typename Tg, typename Tout>
-static void launch_rmsnorm(const Tin* X, const int32_t* idx, const int32_t* seg, int B, const Tg* g, float eps,
+static int launch_rmsnorm(const Tin* X, const int32_t* idx, const int32_t* seg, int B, const Tg* g, float eps,
                            int d, Tout* out, int grid, cudaStream_t st, float* res_out = nullptr,
                            float* zero_out = nullptr, int zcols = 0) {
   constexpr int E = Vec16<Tin>::E;
   if (d % E == 0 && d <= 4 * 256 * E)
-    rmsnorm_vec_kernel<Tin, Tg, Tout, 4><<<grid, 256, 0, st>>>(X, idx, seg, B, g, eps, d, out, res_out, zero_out,
-                                                                zcols);
-  else
-    rmsnorm_rows_kernel<Tin, Tg, Tout><<<grid, 256, 0, st>>>(X, idx, seg, B, g, eps, d, out, res_out, zero_out, zcols);
+    return launch_pdl(rmsnorm_vec_kernel<Tin, Tg, Tout, 4>, dim3(grid), dim3(256), 0, st, X, idx, seg, B, g, eps, d,
+                      out, res_out, zero_out, zcols);
+  return launch_pdl(rmsnorm_rows_kernel<Tin, Tg, Tout>, dim3(grid), dim3(256), 0, st, X, idx, seg, B, g, eps, d, out,
+                    res_out, zero_out, zcols);
 }
 
 // ---------------------------------------------------------------------------
@@ -308,6 +312,8 @@ __global__ void __launch_bounds__(256) finish_qkv_kernel(const float* __restrict
                                                          const int32_t* __restrict__ seg_ptr, int B, int d,
                                                          __nv_bfloat16* __restrict__ q, __nv_bfloat16* __restrict__ Kc,
                                                          __nv_bfloat16* __restrict__ Vc) {
+  pdl_wait();
+  pdl_trigger();
   const int M = seg_ptr[B];
   const int nv = 3 * d / 8;
   for (int j = blockIdx.x; j < M; j += gridDim.x) {
@@ -327,6 +333,8 @@ __global__ void __launch_bounds__(256) finish_qkv_kernel(const float* __restrict
 __global__ void __launch_bounds__(256) finish_gu_kernel(const float* __restrict__ gu32,
                                                         const int32_t* __restrict__ seg_ptr, int B, int F,
                                                         __nv_bfloat16* __restrict__ act) {
+  pdl_wait();
+  pdl_trigger();
   const int M = seg_ptr[B];
   const int nv = F / 8;
   for (int j = blockIdx.x; j < M; j += gridDim.x) {
@@ -346,6 +354,8 @@ __global__ void __launch_bounds__(256) finish_gu_kernel(const float* __restrict_
 __global__ void __launch_bounds__(256) finish_y_kernel(const float* __restrict__ h32, const int32_t* __restrict__ idx,
                                                        const int32_t* __restrict__ seg_ptr, int B, int d,
                                                        __nv_bfloat16* __restrict__ Y) {
+  pdl_wait();
+  pdl_trigger();
   const int M = seg_ptr[B];
   const int nv = d / 8;
   for (int j = blockIdx.x; j < M; j += gridDim.x) {
@@ -436,9 +446,9 @@ __global__ void __launch_bounds__(256) epilogue_f32_kernel(int mode, const float
 // ---------------------------------------------------------------------------
 // orchestration
 // ---------------------------------------------------------------------------
-#define PLK_TRY(x)                  \
+#define PLK_TRY(...)                \
   do {                              \
-    const int _r = (x);             \
+    const int _r = (__VA_ARGS__);   \
     if (_r != PLK_OK) return _r;    \
   } while (0)
 #define PLK_LAUNCHED() \
@@ -460,14 +470,14 @@ static int run_layer_f32(const plk_dims* dm, const plk_weights* w, const float* 
     dim3 grid(ceil_div(Nout, 64), ceil_div(Mcap, 64));
     gemm_f32_kernel<<<grid, 256, 0, st>>>(A, (const float*)Wt, c32, Nout, K, seg, B);
   };
-  launch_rmsnorm<float, float, float>(X, idx, seg, B, (const float*)w->g1, dm->eps, d, xn, Mcap, st);
+  PLK_TRY(launch_rmsnorm<float, float, float>(X, idx, seg, B, (const float*)w->g1, dm->eps, d, xn, Mcap, st));
   gemm(xn, w->w_qkv, 3 * d, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_QKV, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y);
   PLK_LAUNCHED();
   PLK_TRY(launch_attention_f32(dm, q, Kc, Vc, a, seg, Mcap, st));
   gemm(a, w->w_o, d, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_O, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y);
-  launch_rmsnorm<float, float, float>(h32, nullptr, seg, B, (const float*)w->g2, dm->eps, d, hn, Mcap, st);
+  PLK_TRY(launch_rmsnorm<float, float, float>(h32, nullptr, seg, B, (const float*)w->g2, dm->eps, d, hn, Mcap, st));
   gemm(hn, w->w_gu, 2 * F, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_GU, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y);
   gemm(act, w->w_down, d, F);
@@ -510,9 +520,8 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
 
   trace_mark(0, st);
   // x (fp32) staged in h32 takes the O projection's adds; the QKV sums start at 0
-  launch_rmsnorm<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(X, idx, seg, B, (const __nv_bfloat16*)w->g1, dm->eps, d,
-                                                              xn, Mcap, st, h32, c32, 3 * d);
-  PLK_LAUNCHED();
+  PLK_TRY(launch_rmsnorm<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(X, idx, seg, B, (const __nv_bfloat16*)w->g1,
+                                                                      dm->eps, d, xn, Mcap, st, h32, c32, 3 * d));
   trace_mark(1, st);
 
   g.K = d;
@@ -521,8 +530,8 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   PLK_TRY(launch_gemm_tc(tW_qkv, tX_xn, tO_qkv, g, st));
   trace_mark(2, st);
 
-  finish_qkv_kernel<<<rgrid, 256, 0, st>>>(c32, idx, seg, B, d, q, (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc);
-  PLK_LAUNCHED();
+  PLK_TRY(launch_pdl(finish_qkv_kernel, dim3(rgrid), dim3(256), 0, st, (const float*)c32, idx, seg, B, d, q,
+                     (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc));
   trace_mark(3, st);
 
   PLK_TRY(launch_attention_bf16(dm, q, Kc, Vc, a, seg, (float*)(ws + L.att_o), ws + L.att_ml, kAttSplitMax,
@@ -534,9 +543,8 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   PLK_TRY(launch_gemm_tc(tW_o, tX_a, tO_h, g, st));  // h = x + a W_o^T
   trace_mark(5, st);
 
-  launch_rmsnorm<float, __nv_bfloat16, __nv_bfloat16>(h32, nullptr, seg, B, (const __nv_bfloat16*)w->g2, dm->eps, d, hn,
-                                                      Mcap, st, nullptr, c32, 2 * F);
-  PLK_LAUNCHED();
+  PLK_TRY(launch_rmsnorm<float, __nv_bfloat16, __nv_bfloat16>(h32, nullptr, seg, B, (const __nv_bfloat16*)w->g2,
+                                                              dm->eps, d, hn, Mcap, st, nullptr, c32, 2 * F));
   trace_mark(6, st);
 
   g.K = d;
@@ -545,8 +553,7 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   PLK_TRY(launch_gemm_tc(tW_gu, tX_hn, tO_gu, g, st));
   trace_mark(7, st);
 
-  finish_gu_kernel<<<rgrid, 256, 0, st>>>(c32, seg, B, F, act);
-  PLK_LAUNCHED();
+  PLK_TRY(launch_pdl(finish_gu_kernel, dim3(rgrid), dim3(256), 0, st, (const float*)c32, seg, B, F, act));
   trace_mark(8, st);
 
   g.K = F;
@@ -555,8 +562,8 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   PLK_TRY(launch_gemm_tc(tW_down, tX_act, tO_h, g, st));  // y = h + act W_down^T
   trace_mark(9, st);
 
-  finish_y_kernel<<<rgrid, 256, 0, st>>>(h32, idx, seg, B, d, (__nv_bfloat16*)Y);
-  PLK_LAUNCHED();
+  PLK_TRY(launch_pdl(finish_y_kernel, dim3(rgrid), dim3(256), 0, st, (const float*)h32, idx, seg, B, d,
+                     (__nv_bfloat16*)Y));
   trace_mark(10, st);
   return PLK_OK;
 }

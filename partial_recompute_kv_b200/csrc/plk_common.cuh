@@ -22,6 +22,16 @@ __device__ long long g_wait_limit = 4000000000LL;  // cycles, about 2 s
 
 __device__ __forceinline__ void report_timeout() { atomicCAS(&g_status, PLK_OK, PLK_ERR_TIMEOUT); }
 
+// Programmatic dependent launch.  Every kernel of the step is launched with
+// programmatic stream serialization; each CTA calls pdl_wait() before it reads
+// or writes global memory that an earlier kernel of the stream touches, and
+// before any return, and calls pdl_trigger() only after that wait.  So while a
+// kernel runs, every kernel before its immediate predecessor has completed, and
+// a kernel completes only after its predecessor has.  Without a programmatic
+// dependency both instructions are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "../../include/plk.h"
 
 namespace plk {
@@ -17,6 +19,25 @@ constexpr int kGemmBNMax = 256;   // tokens per tile (UMMA N, runtime 64..256)
 constexpr int kGemmBK = 64;       // K per stage: one 128-byte swizzle row of bf16
 constexpr int kGemmStages = 4;
 constexpr int kGemmThreads = 192; // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+
+// ---- launch with programmatic stream serialization ---------------------------
+// The kernel may start while its predecessor in the stream finishes; it orders
+// itself with pdl_wait() (plk_common.cuh).
+template <typename... KArgs, typename... Args>
+inline int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                      Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;
+}
 
 // ---- workspace layout -------------------------------------------------------
 struct Workspace {

@@ -50,6 +50,8 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * kScStages + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 2 * kScStages + 2);
 
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row0 = blockIdx.x * 128;
   const int S = gridDim.y, ks = blockIdx.y;  // K slices = cluster size (1 = no cluster)
@@ -262,6 +264,8 @@ __global__ void __launch_bounds__(256) score_f32_kernel(const float* __restrict_
 
 __global__ void proxy_commit_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ seg_ptr, int B,
                                     int r, const float* __restrict__ pnew, float* __restrict__ pc) {
+  pdl_wait();
+  pdl_trigger();
   const int M = seg_ptr[B];
   const int j = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (j >= M) return;
@@ -301,21 +305,23 @@ int launch_score(const plk_dims* dims, const void* X, const void* Ut, int r, con
   int S = 1;
   while (S < 8 && tiles * S * 2 <= device_sm_count() && nkb % (S * 2) == 0 && nkb / (S * 2) >= 2) S *= 2;
   if (S == 1) {
-    score_tc_kernel<<<tiles, 128, smem, st>>>(tmX, tmU, rows, d, r, tcols, proxy_cache, proxy_out, score_out,
-                                              metric);
+    return launch_pdl(score_tc_kernel, dim3(tiles), dim3(128), smem, st, tmX, tmU, rows, d, r, tcols, proxy_cache,
+                      proxy_out, score_out, metric);
   } else {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(tiles, S, 1);
     cfg.blockDim = dim3(128, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute at[1];
+    cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeClusterDimension;
     at[0].val.clusterDim.x = 1;
     at[0].val.clusterDim.y = S;
     at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, score_tc_kernel, tmX, tmU, rows, d, r, tcols, proxy_cache, proxy_out, score_out,
                            metric) != cudaSuccess)
       return PLK_ERR_CUDA;
@@ -326,8 +332,8 @@ int launch_score(const plk_dims* dims, const void* X, const void* Ut, int r, con
 int launch_proxy_commit(const plk_dims* dims, int r, const int32_t* idx, const int32_t* seg_ptr,
                         const float* proxy_new, float* proxy_cache, cudaStream_t st) {
   const int rows = dims->B * dims->N;
-  proxy_commit_kernel<<<ceil_div(rows, 8), 256, 0, st>>>(idx, seg_ptr, dims->B, r, proxy_new, proxy_cache);
-  return cudaPeekAtLastError() == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;
+  return launch_pdl(proxy_commit_kernel, dim3(ceil_div(rows, 8)), dim3(256), 0, st, idx, seg_ptr, dims->B, r,
+                    proxy_new, proxy_cache);
 }
 
 }  // namespace plk

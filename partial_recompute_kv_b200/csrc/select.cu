@@ -75,6 +75,8 @@ __global__ void __launch_bounds__(kSelThreads) compact_kernel(int mode, const fl
                                                               int N, float tau, int32_t* __restrict__ idx_out,
                                                               int32_t* __restrict__ seg_ptr) {
   __shared__ int sh[33];
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.x;
   const bool writes_lock = (mode == PLK_SEL_THRESH_GT || mode == PLK_SEL_THRESH_LT);
   // active rows of the sequences before this one
@@ -130,6 +132,8 @@ __global__ void __launch_bounds__(kSelThreads) topk_compact_kernel(const float* 
   __shared__ int sh[33];
   __shared__ uint32_t s_prefix;
   __shared__ int s_remaining;
+  pdl_wait();
+  pdl_trigger();
   const int b = blockIdx.x;
   const long long base = (long long)b * N;
   const bool lg = largest != 0;
@@ -232,12 +236,11 @@ int launch_select(const plk_dims* dims, const float* score, const uint8_t* lock_
                   int mode, float tau, int k, int32_t* idx_out, int32_t* seg_ptr, cudaStream_t st) {
   const int B = dims->B, N = dims->N;
   if (mode == PLK_SEL_TOPK_LARGEST || mode == PLK_SEL_TOPK_SMALLEST) {
-    topk_compact_kernel<<<B, kSelThreads, 0, st>>>(score, lock_in, lock_out, N, k, mode == PLK_SEL_TOPK_LARGEST,
-                                                   idx_out, seg_ptr);
-  } else {
-    compact_kernel<<<B, kSelThreads, 0, st>>>(mode, score, lock_in, lock_out, N, tau, idx_out, seg_ptr);
+    return launch_pdl(topk_compact_kernel, dim3(B), dim3(kSelThreads), 0, st, score, lock_in, lock_out, N, k,
+                      (int)(mode == PLK_SEL_TOPK_LARGEST), idx_out, seg_ptr);
   }
-  return cudaPeekAtLastError() == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;
+  return launch_pdl(compact_kernel, dim3(B), dim3(kSelThreads), 0, st, mode, score, lock_in, lock_out, N, tau, idx_out,
+                    seg_ptr);
 }
 
 }  // namespace plk
