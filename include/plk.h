@@ -72,7 +72,8 @@ extern "C" {
 #define PLK_SEL_TOPK_SMALLEST 3  /* keep the k smallest scores active          */
 
 /* Shape of one layer: B sequences of N tokens, model dim d = H*hd, FFN dim F.
- * PLK_BF16 requires hd == 128, d % 128 == 0, F % 64 == 0.
+ * PLK_BF16 requires hd == 128, d % 256 == 0, F % 128 == 0 (the projection GEMM
+ * computes 256-feature tiles on pairs of SMs).
  * PLK_F32 requires hd in {16, 32, 64, 128}.  B*N < 2^31. */
 typedef struct {
   int B, N, d, H, hd, F;

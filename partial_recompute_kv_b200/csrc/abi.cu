@@ -14,7 +14,7 @@ static int check_dims(const plk_dims* d) {
   if ((long long)d->B * d->N >= (1LL << 31)) return PLK_ERR_SHAPE;
   if (!(d->eps >= 0.f)) return PLK_ERR_ARG;
   if (d->dtype == PLK_BF16) {
-    if (d->hd != 128 || d->d % 128 != 0 || d->F % 64 != 0) return PLK_ERR_SHAPE;
+    if (d->hd != 128 || d->d % 256 != 0 || d->F % 128 != 0) return PLK_ERR_SHAPE;
   } else {
     if (d->hd != 16 && d->hd != 32 && d->hd != 64 && d->hd != 128) return PLK_ERR_SHAPE;
   }

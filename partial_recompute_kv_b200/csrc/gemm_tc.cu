@@ -5,32 +5,37 @@
 // active subset, cost O(M d^2)).
 //
 // Design (sm_100a):
-//  * Weights are the UMMA A operand (M = 128 feature rows per tile) and the
-//    compacted activations the B operand (N = 64..256 tokens, chosen on the
-//    device from M = seg_ptr[B]); at M <= 256 every weight byte is read from HBM
-//    once.  Both operands are K-major bf16 tiles loaded by TMA with a 128-byte
-//    swizzle into a 4-stage ring; accumulation is fp32 in TMEM.
-//  * Warp roles: warp 0 issues TMA, one thread of warp 1 issues tcgen05.mma,
-//    warps 2-5 drain TMEM (tcgen05.ld).
-//  * Persistent stream-K without inter-CTA waiting: one CTA per SM owns an
-//    equal, contiguous share of the tiles x k-blocks iteration space and adds
-//    the fp32 partial of each tile piece it covers into the fp32 output with
-//    TMA bulk reduce-add (cp.reduce.async.bulk.tensor ... .add.f32), which the
-//    L2 applies atomically.  The output is either the residual stream h (the O
-//    and down projections: h += a W_o^T, then h += act W_down^T) or a zeroed
-//    fp32 buffer whose finishing kernel applies the nonlinear or scattering
-//    epilogue (QKV -> Q and the K/V cache rows; gate/up -> silu(g) * u).  At
-//    M <= 256 the O and down projections have only 32 tiles of 128 features;
-//    stream-K keeps all SMs busy regardless.  The order of the reduce-adds is
-//    not fixed, so results may differ in the last fp32 bit between runs.
-//  * Two 256-column TMEM accumulators: the epilogue drains one tile piece while
-//    the MMA fills the next, and the TMA producer runs ahead across pieces.
+//  * CTA pairs (cta_group::2): the even CTA issues one tcgen05.mma of
+//    M = 256 feature rows x N = 128 or 256 tokens that runs on the tensor cores
+//    of both SMs.  Each CTA stages its own 128 weight rows and HALF of the
+//    token tile, so an SM ingests 32 KB per 64-deep k-block instead of 48 KB
+//    for a one-CTA 128 x 256 tile: the operand feed (L2 -> SM), not the tensor
+//    pipe, bounds this GEMM at M <= 256 tokens.  Accumulation is fp32 in TMEM;
+//    each CTA's TMEM holds its 128 rows x N columns.
+//  * Weights are the A operand and the compacted activations the B operand;
+//    at M <= 256 every weight byte is read from HBM once.  Both are K-major
+//    bf16 tiles loaded by TMA with a 128-byte swizzle into a 6-stage ring.
+//  * Warp roles: warp 0 issues TMA in both CTAs, every load counting its bytes
+//    on the even CTA's stage barrier; one thread of warp 1 of the even CTA
+//    issues the pair MMAs; warps 2-5 of both CTAs drain their TMEM.
+//  * Persistent stream-K without inter-CTA waiting: each pair owns an equal,
+//    contiguous share of the (256-feature tile) x (k-block) iteration space
+//    and adds the fp32 partial of each tile piece it covers into the fp32
+//    output with TMA bulk reduce-add (cp.reduce.async.bulk.tensor .add.f32),
+//    which the L2 applies atomically.  The output is the residual stream h
+//    (O and down projections) or a zeroed fp32 buffer that a finishing kernel
+//    turns into bf16 (QKV -> Q and the K/V cache rows; gate/up -> silu(g) u).
+//    The order of the adds is not fixed: results may differ in the last fp32
+//    bit between runs.
+//  * Two 256-column TMEM accumulators per CTA: the epilogue drains one tile
+//    piece while the MMA fills the next; the producers run ahead across
+//    pieces.
 //  * Each epilogue warp stages its 32 tokens x 32 features token-major in a
 //    double-buffered shared-memory block (rows past M zeroed) and issues one
 //    bulk reduce per block; the CTA's last piece stages all its blocks in the
 //    then idle operand ring so that every reduce is in flight at once.  A
-//    gate/up tile (64 gate + 64 up rows of the same features) lands in the
-//    gate and up halves of its [M, 2F] buffer.
+//    gate/up tile of a CTA (64 gate + 64 up rows of the same features) lands
+//    in the gate and up halves of its [M, 2F] buffer.
 #include "plk_common.cuh"
 #include "plk_internal.h"
 
@@ -38,15 +43,17 @@ namespace plk {
 
 namespace {
 
-constexpr int kStageA = kGemmBM * kGemmBK * 2;     // 16 KB
-constexpr int kStageB = kGemmBNMax * kGemmBK * 2;  // 32 KB
+constexpr int kHalfTok = kGemmBNMax / 2;            // token rows of B staged per CTA
+constexpr int kStageA = kGemmBM * kGemmBK * 2;      // 16 KB
+constexpr int kStageB = kHalfTok * kGemmBK * 2;     // 16 KB
 constexpr size_t kOffB = (size_t)kGemmStages * kStageA;
 constexpr size_t kOffBar = kOffB + (size_t)kGemmStages * kStageB;
-constexpr size_t kOffStg = kOffBar + 128;
-constexpr int kBlk = 32 * 32;                      // a warp's block: 32 tokens x 32 features (fp32)
+constexpr size_t kOffStg = kOffBar + 256;
+constexpr int kBlk = 32 * 32;                       // a warp's block: 32 tokens x 32 features (fp32)
 constexpr size_t kSmemUsed = kOffStg + 4 * 2 * kBlk * 4;
-constexpr size_t kSmemBytes = kSmemUsed + 1024;    // slack for 1024-byte alignment
+constexpr size_t kSmemBytes = kSmemUsed + 1024;     // slack for 1024-byte alignment
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert((size_t)4 * 8 * kBlk * 4 <= kOffBar, "the last piece's blocks fit the operand ring");
 
 // bulk reduce-add of a [32 rows][32 fp32] smem block into the tensor at (x, y)
 __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* tm, int x, int y, const void* smem_src) {
@@ -69,17 +76,17 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 }  // namespace
 
-// The flattened iteration space of one GEMM: tiles x KB k-blocks, tile u =
-// ft * ttiles + tt (token tiles fastest, so CTAs that run at the same time share
-// a weight tile in L2).  CTA c owns iterations [c*T/G, (c+1)*T/G); a segment is
-// the part of that range inside one tile.
+// The flattened iteration space of one GEMM: tiles x KB k-blocks, pair tile
+// u = pt * ttiles + tt (token tiles fastest, so pairs that run at the same
+// time share a weight tile in L2).  Pair c owns iterations [c*T/G, (c+1)*T/G);
+// a segment is the part of that range inside one tile.
 struct SegWalk {
   long long i, iend;
   int KB;
-  __device__ SegWalk(int cta, int nctas, int tiles, int KB_) : KB(KB_) {
+  __device__ SegWalk(int pair, int npairs, int tiles, int KB_) : KB(KB_) {
     const long long T = (long long)tiles * KB_;
-    i = T * cta / nctas;
-    iend = T * (cta + 1) / nctas;
+    i = T * pair / npairs;
+    iend = T * (pair + 1) / npairs;
   }
   __device__ bool next(int& u, int& kb0, int& kb1) {
     if (i >= iend) return false;
@@ -92,13 +99,18 @@ struct SegWalk {
   __device__ bool done() const { return i >= iend; }
 };
 
+// Geometry of pair tile u as seen by CTA `rank` of the pair.
 struct TileGeom {
-  int ft, tok0, ntok, ncols;
-  __device__ TileGeom(int u, int ttiles, int M) {
-    ft = u / ttiles;
-    tok0 = (u - ft * ttiles) * kGemmBNMax;
+  int ft;     // this CTA's 128-row feature tile (pair tile pt covers 2 pt and 2 pt + 1)
+  int tok0;   // first token of the tile
+  int ntok;   // valid tokens
+  int ncols;  // UMMA N: 128 or 256 (each CTA stages ncols / 2 token rows)
+  __device__ TileGeom(int u, int ttiles, int M, int rank) {
+    const int pt = u / ttiles;
+    ft = 2 * pt + rank;
+    tok0 = (u - pt * ttiles) * kGemmBNMax;
     ntok = min(kGemmBNMax, M - tok0);
-    ncols = (ntok + 63) & ~63;  // UMMA N: whole 64-token boxes
+    ncols = (ntok + 127) & ~127;
   }
 };
 
@@ -107,38 +119,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                    const __grid_constant__ CUtensorMap tmOut, const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
-  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // same offset in both CTAs of a pair
   uint8_t* sA = smem;
   uint8_t* sB = smem + kOffB;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* full = bars;            // [4] TMA -> MMA
-  uint64_t* empty = bars + 4;       // [4] MMA -> TMA
-  uint64_t* tfull = bars + 8;       // [2] MMA -> epilogue, per TMEM accumulator
-  uint64_t* tempty = bars + 10;     // [2] epilogue -> MMA
-  uint64_t* drain = bars + 12;      // MMA completion on the abort path
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 13);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 14);
+  uint64_t* full = bars;                        // [6] stage landed, both halves (even CTA's used)
+  uint64_t* empty = bars + kGemmStages;         // [6] stage consumed by the pair MMA
+  uint64_t* tfull = bars + 2 * kGemmStages;     // [2] accumulator ready for the epilogue
+  uint64_t* tempty = bars + 2 * kGemmStages + 2;  // [2] accumulator drained (even CTA: 8 warps)
+  uint64_t* drain = bars + 2 * kGemmStages + 4;   // MMA completion on the abort path
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * kGemmStages + 5);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 2 * kGemmStages + 6);
   float* stg_all = reinterpret_cast<float*>(smem + kOffStg);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = (int)cluster_ctarank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   // seg_ptr comes from a kernel before the predecessor: already complete (see pdl_wait)
   const int M = args.seg_ptr[args.B];
   const int ttiles = ceil_div(max(M, 0), kGemmBNMax);
-  const int tiles = args.ftiles * ttiles;
+  const int tiles = (args.ftiles >> 1) * ttiles;
   const int KB = args.K / kGemmBK;
-  if (M <= 0 || SegWalk(blockIdx.x, gridDim.x, tiles, KB).done()) {  // no iterations for this CTA
+  if (M <= 0 || SegWalk(pair, npairs, tiles, KB).done()) {  // the same for both CTAs of the pair
     pdl_wait();
     return;
   }
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kGemmStages; ++i) {
-      mbar_init(&full[i], 1);
+      mbar_init(&full[i], 1);  // the even CTA's expect-arrive; both CTAs' loads complete on it
       mbar_init(&empty[i], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 4);  // one arrival per epilogue warp
+      mbar_init(&tempty[b], 8);  // one arrival per epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -148,11 +162,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&tmOut);
   }
   if (warp == 1) {
-    tmem_alloc(s_tmem, 512);  // two 256-column fp32 accumulators
-    tmem_relinquish();
+    tmem_alloc_pair(s_tmem, 512);  // two 256-column fp32 accumulators in each CTA
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // barriers initialised and TMEM allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
   if (warp != 0) {
@@ -161,18 +175,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producer (both CTAs)
     if (elect_one()) {
-      // weight rows of tile t (gate/up tile: 64 gate rows, then the 64 up rows)
+      // this CTA's 128 weight rows of tile t (gate/up tile: 64 gate rows, then the 64 up rows)
+      const uint32_t lead_full0 = dsmem_addr(smem_u32(&full[0]), 0);
       auto load_a = [&](int stage, const TileGeom& t, int kb) {
         const int yA0 = args.gu_F ? t.ft * 64 : t.ft * kGemmBM;
         const int yA1 = args.gu_F ? args.gu_F + t.ft * 64 : t.ft * kGemmBM + 64;
         uint8_t* a = sA + stage * kStageA;
-        tma_load_2d(a, &tmW, kb * kGemmBK, yA0, &full[stage]);
-        tma_load_2d(a + 8192, &tmW, kb * kGemmBK, yA1, &full[stage]);
+        const uint32_t fb = lead_full0 + (uint32_t)(stage * 8);
+        tma_load_2d_pair(a, &tmW, kb * kGemmBK, yA0, fb);
+        tma_load_2d_pair(a + 8192, &tmW, kb * kGemmBK, yA1, fb);
       };
-      auto stage_bytes = [](const TileGeom& t) { return (uint32_t)(kStageA + (t.ncols >> 6) * (64 * kGemmBK * 2)); };
-      SegWalk w(blockIdx.x, gridDim.x, tiles, KB);
+      // bytes of one stage, both CTAs: 2 x (A rows + half of the token rows)
+      auto stage_bytes = [](const TileGeom& t) {
+        return (uint32_t)(2 * (kStageA + (t.ncols >> 7) * (64 * kGemmBK * 2)));
+      };
+      SegWalk w(pair, npairs, tiles, KB);
       int u, kb0, kb1, stage = 0;
       // The weights are no kernel's output: the first stages' weight loads start
       // before the wait for the predecessor, overlapping its tail.
@@ -180,9 +199,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       {
         SegWalk w2 = w;
         while (pre < kGemmStages && w2.next(u, kb0, kb1)) {
-          const TileGeom t(u, ttiles, M);
+          const TileGeom t(u, ttiles, M, rank);
           for (int kb = kb0; kb < kb1 && pre < kGemmStages; ++kb, ++pre) {
-            mbar_expect_tx(&full[pre], stage_bytes(t));
+            if (rank == 0) mbar_expect_tx(&full[pre], stage_bytes(t));
             load_a(pre, t, kb);
           }
         }
@@ -192,20 +211,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       long long issued = 0;
       while (!*s_abort && w.next(u, kb0, kb1)) {
-        const TileGeom t(u, ttiles, M);
-        const int nbox = t.ncols >> 6;
+        const TileGeom t(u, ttiles, M, rank);
+        const int half = t.ncols >> 1, nbox = half >> 6;
+        const int trow = t.tok0 + rank * half;  // this CTA's token rows: MMA columns rank*half ..
         for (int kb = kb0; kb < kb1; ++kb) {
           if (issued >= pre) {  // stages past the prefetched ones: wait for a free slot
             if (!mbar_wait(&empty[stage], phase ^ 1)) {
               *s_abort = 1;
               break;
             }
-            mbar_expect_tx(&full[stage], stage_bytes(t));
+            if (rank == 0) mbar_expect_tx(&full[stage], stage_bytes(t));
             load_a(stage, t, kb);
           }
           uint8_t* b = sB + stage * kStageB;
           for (int j = 0; j < nbox; ++j)
-            tma_load_2d(b + j * 8192, &tmX, kb * kGemmBK, t.tok0 + j * 64, &full[stage]);
+            tma_load_2d_pair(b + j * 8192, &tmX, kb * kGemmBK, trow + j * 64, lead_full0 + (uint32_t)(stage * 8));
           ++issued;
           if (++stage == kGemmStages) {
             stage = 0;
@@ -213,66 +233,74 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
-      if (*s_abort) {
-        // let the copies this thread started land before the CTA moves on
+      if (*s_abort && rank == 0) {
+        // let the pair's copies land before the CTAs move on (bounded; the odd
+        // CTA's copies complete on these barriers too)
         for (long long i = issued > kGemmStages ? issued - kGemmStages : 0; i < issued; ++i)
           (void)mbar_wait(&full[i % kGemmStages], (uint32_t)((i / kGemmStages) & 1));
       }
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (elect_one()) {
-      SegWalk w(blockIdx.x, gridDim.x, tiles, KB);
-      int u, kb0, kb1, stage = 0, j = 0;
-      uint32_t phase = 0;
-      bool any = false;
-      while (!*s_abort && w.next(u, kb0, kb1)) {
-        const TileGeom t(u, ttiles, M);
-        const int b = j & 1;
-        if (!mbar_wait(&tempty[b], ((j >> 1) & 1) ^ 1)) {  // the epilogue has drained this accumulator
-          *s_abort = 1;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t acc = tmem_base + (uint32_t)(b * 256);
-        const uint32_t idesc = idesc_bf16(kGemmBM, t.ncols);
-        for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase)) {
+    if (rank == 0) {
+      // ---------------------------------------------------------- pair MMA issuer (even CTA)
+      if (elect_one()) {
+        const uint32_t peer_empty0 = dsmem_addr(smem_u32(&empty[0]), 1);
+        const uint32_t peer_tfull0 = dsmem_addr(smem_u32(&tfull[0]), 1);
+        SegWalk w(pair, npairs, tiles, KB);
+        int u, kb0, kb1, stage = 0, j = 0;
+        uint32_t phase = 0;
+        bool any = false;
+        while (!*s_abort && w.next(u, kb0, kb1)) {
+          const TileGeom t(u, ttiles, M, rank);
+          const int b = j & 1;
+          if (!mbar_wait_cluster(&tempty[b], ((j >> 1) & 1) ^ 1)) {  // both epilogues have drained it
             *s_abort = 1;
             break;
           }
           tc_fence_after();
-          const uint64_t adesc = sdesc_sw128(smem_u32(sA + stage * kStageA));
-          const uint64_t bdesc = sdesc_sw128(smem_u32(sB + stage * kStageB));
+          const uint32_t acc = tmem_base + (uint32_t)(b * 256);
+          const uint32_t idesc = idesc_bf16(2 * kGemmBM, t.ncols);
+          for (int kb = kb0; kb < kb1; ++kb) {
+            if (!mbar_wait(&full[stage], phase)) {  // both CTAs' halves of the stage landed
+              *s_abort = 1;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t adesc = sdesc_sw128(smem_u32(sA + stage * kStageA));
+            const uint64_t bdesc = sdesc_sw128(smem_u32(sB + stage * kStageB));
 #pragma unroll
-          for (int k = 0; k < kGemmBK / 16; ++k)  // +32 bytes of K per step = 2 descriptor units
-            umma_bf16(acc, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
-          any = true;
-          umma_commit(&empty[stage]);
-          if (++stage == kGemmStages) {
-            stage = 0;
-            phase ^= 1;
+            for (int k = 0; k < kGemmBK / 16; ++k)  // +32 bytes of K per step = 2 descriptor units
+              umma_bf16_pair(acc, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            any = true;
+            umma_commit_pair(smem_u32(&empty[stage]));  // the stage is free in both CTAs
+            umma_commit_pair(peer_empty0 + (uint32_t)(stage * 8));
+            if (++stage == kGemmStages) {
+              stage = 0;
+              phase ^= 1;
+            }
           }
+          if (*s_abort) break;
+          umma_commit_pair(smem_u32(&tfull[b]));  // the accumulators are complete in both CTAs
+          umma_commit_pair(peer_tfull0 + (uint32_t)(b * 8));
+          ++j;
         }
-        if (*s_abort) break;
-        umma_commit(&tfull[b]);  // arrives once every MMA of this segment is complete
-        ++j;
-      }
-      if (*s_abort && any) {
-        umma_commit(drain);  // wait for the MMAs in flight before TMEM is freed
-        (void)mbar_wait(drain, 0);
+        if (*s_abort && any) {
+          umma_commit_pair(smem_u32(drain));  // wait for the MMAs in flight before TMEM is freed
+          (void)mbar_wait(drain, 0);
+        }
       }
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;  // a warp reads TMEM lanes 32 * (warp % 4) ..
-    SegWalk w(blockIdx.x, gridDim.x, tiles, KB);
+    const uint32_t lead_tempty0 = rank == 0 ? 0u : dsmem_addr(smem_u32(&tempty[0]), 0);
+    SegWalk w(pair, npairs, tiles, KB);
     int u, kb0, kb1, j = 0, n = 0;
     while (w.next(u, kb0, kb1)) {
       const bool last = w.done();  // no MMA or TMA follows: the stage buffers are free for staging
-      const TileGeom t(u, ttiles, M);
+      const TileGeom t(u, ttiles, M, rank);
       const int b = j & 1;
       const bool ok = mbar_wait(&tfull[b], (j >> 1) & 1) && !*s_abort;
       if (!__all_sync(0xffffffffu, ok)) {
@@ -300,10 +328,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         uint32_t r[32];
         tmem_ld32(taddr + (uint32_t)(c * 32), r);
         tmem_ld_wait();
-        if (c == nchunks - 1) {  // accumulator b drained: the MMA may reuse it
+        if (c == nchunks - 1) {  // accumulator b drained: the pair MMA may reuse it
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[b]);
+          if (lane == 0) {
+            if (rank == 0)
+              mbar_arrive(&tempty[b]);
+            else
+              mbar_arrive_remote(lead_tempty0 + (uint32_t)(b * 8));
+          }
         }
         const int nval = t.ntok - c * 32;  // tokens past M contribute zeros
 #pragma unroll
@@ -321,16 +354,43 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   }
 
+  // Neither CTA may leave while the pair MMA can still read its shared memory
+  // or the other CTA can still arrive on its barriers.
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    tmem_dealloc_pair(tmem_base, 512);
   }
+}
+
+// Pairs that can be resident at once (cluster of 2, one CTA per SM), per device.
+static int resident_pairs(int num_sms) {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_sms & ~1);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel, &cfg) != cudaSuccess || n <= 0) return 0;
+  n = std::min(n, num_sms / 2);
+  if (dev < 64) cached[dev] = n;
+  return n;
 }
 
 int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const CUtensorMap& tmOut, const GemmArgs& a,
                    cudaStream_t st) {
+  if (a.ftiles <= 0 || (a.ftiles & 1) || a.K % kGemmBK != 0) return PLK_ERR_SHAPE;
   static int attr_done[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PLK_ERR_CUDA;
@@ -340,8 +400,25 @@ int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const CUtenso
       return PLK_ERR_CUDA;
     attr_done[dev] = 1;
   }
-  // persistent: one CTA per SM, each owning an equal share of the k-block iterations
-  return launch_pdl(gemm_tc_kernel, dim3(a.num_sms), dim3(kGemmThreads), kSmemBytes, st, tmW, tmX, tmOut, a);
+  // persistent: every resident CTA pair owns an equal share of the k-block iterations
+  const int pairs = resident_pairs(a.num_sms);
+  if (pairs <= 0) return PLK_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel, tmW, tmX, tmOut, a) != cudaSuccess) return PLK_ERR_CUDA;
+  return PLK_OK;
 }
 
 }  // namespace plk

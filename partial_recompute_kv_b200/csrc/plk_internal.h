@@ -14,10 +14,10 @@
 namespace plk {
 
 // ---- tile constants of the tcgen05 GEMM ------------------------------------
-constexpr int kGemmBM = 128;      // feature rows per tile (UMMA M)
-constexpr int kGemmBNMax = 256;   // tokens per tile (UMMA N, runtime 64..256)
+constexpr int kGemmBM = 128;      // feature rows per CTA (a CTA pair computes 256)
+constexpr int kGemmBNMax = 256;   // tokens per tile (UMMA N, runtime 128 or 256; each CTA loads half)
 constexpr int kGemmBK = 64;       // K per stage: one 128-byte swizzle row of bf16
-constexpr int kGemmStages = 4;
+constexpr int kGemmStages = 6;
 constexpr int kGemmThreads = 192; // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 
 // ---- launch with programmatic stream serialization ---------------------------
@@ -79,11 +79,11 @@ int run_layer(const plk_dims* dims, const plk_weights* w, const void* X, const i
 // M = seg_ptr[B] compact tokens (fp32 out, added with bulk reduce-adds).
 struct GemmArgs {
   int K;                   // reduction length, multiple of 64
-  int ftiles;              // 128-row feature tiles
+  int ftiles;              // 128-row feature tiles (even: a CTA pair takes two)
   int gu_F;                // gate/up GEMM: F (tile f = gate rows f*64.. and up rows F + f*64..), else 0
   const int32_t* seg_ptr;  // M = seg_ptr[B]
   int B;
-  int num_sms;             // SM count: one persistent CTA per SM
+  int num_sms;             // SM count: at most one persistent CTA per SM, in pairs
 };
 int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const CUtensorMap& tmOut, const GemmArgs& a,
                    cudaStream_t st);

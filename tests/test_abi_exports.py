@@ -54,6 +54,10 @@ def test_host_validation_without_gpu(built):
     bad_hd = plk.dims(1, 8, 512, 8, 64, 256, dtype=plk.BF16)  # bf16 needs hd == 128
     assert lib.plk_full_layer_step(ctypes.byref(bad_hd), None, None, None, None, None, None, 0, None) == \
         plk.ERR_SHAPE
+    bad_width = plk.dims(1, 8, 384, 3, 128, 256, dtype=plk.BF16)  # bf16 needs d % 256 == 0
+    assert lib.plk_workspace_bytes(ctypes.byref(bad_width)) == 0
+    bad_ffn = plk.dims(1, 8, 512, 4, 128, 320, dtype=plk.BF16)  # bf16 needs F % 128 == 0
+    assert lib.plk_workspace_bytes(ctypes.byref(bad_ffn)) == 0
     bad_split = plk.dims(1, 8, 64, 3, 16, 64, dtype=plk.F32)  # d != H * hd
     assert lib.plk_workspace_bytes(ctypes.byref(bad_split)) == 0
     ok = plk.dims(2, 8, 64, 4, 16, 64, dtype=plk.F32)
