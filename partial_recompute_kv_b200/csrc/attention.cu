@@ -4,16 +4,20 @@
 // active tokens keep attending to locked tokens through their cached K/V; cost
 // O(M N d) instead of O(N^2 d), Sec. 2 "Algorithmic Complexity").
 //
-// bf16, hd = 128: one CTA per (64-query tile, head, sequence), 4 warps of 16
-// query rows.  K/V tiles of 64 keys x 128 dims are staged by TMA (128-byte
-// swizzle, two boxes of 64 dims each) into a double-buffered shared-memory
-// ring; Q fragments stay in registers; S = Q K^T and O += P V run on the tensor
-// cores (mma.sync m16n8k16, fp32 accumulate) with an online softmax in
-// registers (quad shuffles for the row max and sum).  P is split into a bf16
-// high part and a bf16 residual and both are multiplied with V, so the softmax
-// weights enter P V with ~16 significant bits: a bf16-rounded P would perturb
-// the attention output by ~1e-3 relative, which later bf16 roundings amplify.
-// Rows past the sequence's last active row and keys past N are masked.
+// bf16, hd = 128, on the tcgen05 tensor cores: a CTA takes 128 active queries
+// of one sequence and one head and a contiguous range of 64-key chunks.  Warp
+// 0 stages Q once and K, V chunk by chunk with TMA (128-byte swizzle, 3-stage
+// rings); one thread of warp 1 issues S = Q K^T into TMEM (double-buffered,
+// 64 columns each) and O += P V into TMEM (128 columns); warps 2-5 own one
+// query row per thread: they read the row's scores from TMEM, keep the running
+// row max and sum (online softmax), and write P to shared memory as a bf16 high
+// part and a bf16 residual, both multiplied with V, so the softmax weights
+// enter P V with ~16 significant bits (a bf16-rounded P would perturb the
+// attention output by ~1e-3 relative, which later bf16 roundings amplify).  A
+// row keeps a stale max until the new one exceeds it by 2^8 (the weights stay
+// below 256, exact in fp32); only then is its O row rescaled in TMEM.  Keys are
+// split over CTAs when the query tiles alone leave SMs idle; a combine kernel
+// merges the splits.  Keys past N are masked.
 // fp32: one thread per (query row, head), online softmax, SIMT.
 #include <math.h>
 
@@ -25,31 +29,22 @@
 namespace plk {
 
 namespace {
-constexpr int kAttBQ = 64, kAttBK = 64, kAttHD = 128, kAttThreads = 128;
-constexpr int kAttTile = kAttBK * kAttHD * 2;  // 16 KB
-constexpr int kAttSmem = 5 * kAttTile + 128 + 1024;
+constexpr int kAttHD = 128;
+constexpr int kAttBQ = 128;                    // queries per CTA (UMMA M, one TMEM lane each)
+constexpr int kAttBK = 64;                     // keys per chunk (UMMA N of S, K of P V)
+constexpr int kAttStages = 3;                  // K and V ring depth
+constexpr int kAttThreads = 192;               // warp 0 TMA, warp 1 MMA, warps 2-5 softmax
+constexpr int kAttQBytes = kAttBQ * kAttHD * 2;   // 32 KB
+constexpr int kAttKVBytes = kAttBK * kAttHD * 2;  // 16 KB
+constexpr int kAttPBytes = kAttBQ * kAttBK * 2;   // 16 KB (high or low part)
+constexpr size_t kAttOffK = kAttQBytes;
+constexpr size_t kAttOffV = kAttOffK + (size_t)kAttStages * kAttKVBytes;
+constexpr size_t kAttOffP = kAttOffV + (size_t)kAttStages * kAttKVBytes;  // [2 buffers][high, low]
+constexpr size_t kAttOffBar = kAttOffP + 4 * (size_t)kAttPBytes;
+constexpr int kAttSmem = (int)kAttOffBar + 256 + 1024;
+constexpr uint32_t kAttTmemCols = 256;         // O: 0..127, S buffers: 128..191, 192..255
+constexpr float kAttStaleMax = 8.f;            // log2 headroom before a row's O is rescaled
 
-__device__ __forceinline__ uint32_t sw_addr(uint32_t base, int row, int col) {
-  // [64 rows][128 cols] bf16 stored as two 64-column boxes with 128-byte swizzle
-  return base + (uint32_t)((col >> 6) * 8192 + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4));
-}
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-      "{%0, %1, %2, %3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -63,17 +58,45 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uin
   hi = *reinterpret_cast<uint32_t*>(&hv);
   lo = pack_bf16(x0 - __bfloat162float(h0), x1 - __bfloat162float(h1));
 }
+
+// Shared-memory descriptor of an MN-major operand tile with 128-byte swizzle:
+// rows of 64 MN-elements (128 B), 8-row groups 1024 B apart along K, 64-wide MN
+// blocks `mn_block_bytes` apart.  The V chunk [64 keys][128 dims], stored as two
+// 64-dim TMA boxes, is the B operand of P V in this form (K = keys, N = dims).
+__device__ __forceinline__ uint64_t sdesc_sw128_mn(uint32_t saddr, uint32_t mn_block_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((mn_block_bytes >> 4) & 0x3FFFu) << 16;  // leading byte offset: next MN block
+  d |= (uint64_t)(1024 >> 4) << 32;                          // stride byte offset: next 8 K-rows
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
 }  // namespace
 
-// Number of key splits for the current active set: enough CTAs to cover the
-// GPU twice, at most smax.  Computed identically by the attention and combine
-// kernels from seg_ptr (device-side M, no host synchronisation).
-__device__ __forceinline__ int attn_splits(const int32_t* seg_ptr, int B, int H, int smax, int nsm) {
-  int qtiles = 0;
-  for (int b = 0; b < B; ++b) qtiles += ceil_div(seg_ptr[b + 1] - seg_ptr[b], kAttBQ);
-  if (qtiles == 0) return 1;
-  const int want = ceil_div(2 * nsm, qtiles * H);
-  return max(1, min(smax, want));
+// Key splits for the current active set (device-side M, no host sync): the
+// split count s <= smax minimising whole waves of CTAs x chunks per CTA, one
+// CTA per SM, plus one chunk's worth for the combine when s > 1.  Splits are
+// considered only while the query tiles x heads leave SMs idle.  Computed
+// identically by the attention and combine kernels.
+__device__ __forceinline__ int attn_qtiles(const int32_t* seg_ptr, int B) {
+  int qt = 0;
+  for (int b = 0; b < B; ++b) qt += ceil_div(seg_ptr[b + 1] - seg_ptr[b], kAttBQ);
+  return qt;
+}
+__device__ __forceinline__ int attn_splits(const int32_t* seg_ptr, int B, int H, int N, int smax, int nsm) {
+  const int items = attn_qtiles(seg_ptr, B) * H;
+  if (items == 0 || items >= nsm) return 1;
+  const int nch = ceil_div(N, kAttBK);
+  int best = 1, best_cost = 1 << 30;
+  for (int s = 1; s <= smax && s <= nch; ++s) {
+    const int cost = ceil_div(items * s, nsm) * ceil_div(nch, s) * 2 + (s > 1 ? 1 : 0);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = s;
+    }
+  }
+  return best;
 }
 
 // Split partials: o_part[s][row][d] (unnormalised, fp32) and ml[s][row][h] = (max, sum)
@@ -84,200 +107,369 @@ struct AttnSplit {
   int smax, part_rows, nsm;
 };
 
-__global__ void __launch_bounds__(kAttThreads) attn_bf16_kernel(const __grid_constant__ CUtensorMap tmK,
-                                                                const __grid_constant__ CUtensorMap tmV,
-                                                                const __nv_bfloat16* __restrict__ Q,
-                                                                __nv_bfloat16* __restrict__ Aout,
-                                                                const int32_t* __restrict__ seg_ptr, int B, int N,
-                                                                int d, float scale_log2, AttnSplit sp) {
-  pdl_wait();
-  pdl_trigger();
-  const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z / sp.smax, split = blockIdx.z % sp.smax;
-  const int seg0 = seg_ptr[b], seg1 = seg_ptr[b + 1];
-  const int r0 = seg0 + qt * kAttBQ;
-  if (r0 >= seg1) return;
-  const int S = attn_splits(seg_ptr, B, gridDim.y, sp.smax, sp.nsm);
-  if (split >= S) return;
-  const int nrows = min(kAttBQ, seg1 - r0);
+// One work item: 128 queries [r0, r0 + nrows) of sequence b, head h, chunks [c0, c1).
+struct AttnItem {
+  int b, h, split, r0, nrows, c0, c1;
+};
+__device__ __forceinline__ AttnItem attn_item(int i, const int32_t* seg_ptr, int B, int H, int N, int S) {
+  AttnItem it;
+  it.split = i % S;
+  const int rest = i / S;
+  it.h = rest % H;
+  int qi = rest / H, b = 0;
+  for (; b < B; ++b) {
+    const int qt = ceil_div(seg_ptr[b + 1] - seg_ptr[b], kAttBQ);
+    if (qi < qt) break;
+    qi -= qt;
+  }
+  it.b = b;
+  it.r0 = seg_ptr[b] + qi * kAttBQ;
+  it.nrows = min(kAttBQ, seg_ptr[b + 1] - it.r0);
+  const int nch = ceil_div(N, kAttBK);
+  it.c0 = it.split * nch / S;
+  it.c1 = (it.split + 1) * nch / S;
+  return it;
+}
 
+__global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                               const __grid_constant__ CUtensorMap tmK,
+                                                               const __grid_constant__ CUtensorMap tmV,
+                                                               __nv_bfloat16* __restrict__ Aout,
+                                                               const int32_t* __restrict__ seg_ptr, int B, int N,
+                                                               int H, int d, float scale_log2, AttnSplit sp) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   uint8_t* sQ = smem;
-  uint8_t* sK = smem + kAttTile;          // [2] stages
-  uint8_t* sV = smem + 3 * kAttTile;      // [2] stages
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + 5 * kAttTile);
-  volatile int* s_bad = reinterpret_cast<volatile int*>(full + 2);
+  uint8_t* sK = smem + kAttOffK;
+  uint8_t* sV = smem + kAttOffV;
+  uint8_t* sP = smem + kAttOffP;  // buffer x: high part at 2x, low part at 2x + 1 (16 KB each)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAttOffBar);
+  uint64_t* q_full = bars + 0;
+  uint64_t* q_free = bars + 1;
+  uint64_t* k_full = bars + 2;    // [3]
+  uint64_t* k_empty = bars + 5;   // [3]
+  uint64_t* v_full = bars + 8;    // [3]
+  uint64_t* v_empty = bars + 11;  // [3]
+  uint64_t* s_full = bars + 14;   // [2] scores of a chunk in TMEM
+  uint64_t* s_free = bars + 16;   // [2] scores read by the 4 softmax warps
+  uint64_t* p_full = bars + 18;   // [2] P of a chunk in shared memory (4 softmax warps)
+  uint64_t* pv_done = bars + 20;  // one phase per chunk: its P V has completed
+  uint64_t* o_free = bars + 21;   // O read out by the 4 softmax warps
+  uint64_t* drain = bars + 22;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 23);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 24);
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int ntiles_all = ceil_div(N, kAttBK);
-  const int t0 = split * ntiles_all / S;                 // this split's key tiles [t0, t0 + ntiles)
-  const int ntiles = (split + 1) * ntiles_all / S - t0;
-  const int hcol = h * kAttHD;
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = attn_splits(seg_ptr, B, H, N, sp.smax, sp.nsm);
+  const int nitems = attn_qtiles(seg_ptr, B) * H * S;
+  if ((int)blockIdx.x >= nitems) return;
 
-  if (tid == 0) {
-    mbar_init(&full[0], 1);
-    mbar_init(&full[1], 1);
-    *s_bad = 0;
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_free, 1);
+    for (int i = 0; i < kAttStages; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);
+      mbar_init(&p_full[i], 4);
+    }
+    mbar_init(pv_done, 1);
+    mbar_init(o_free, 4);
+    mbar_init(drain, 1);
+    *s_abort = 0;
     fence_mbar_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
   }
+  if (warp == 1) {
+    tmem_alloc(s_tmem, kAttTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
-  auto issue = [&](int j, int s) {
-    const int y = b * N + (t0 + j) * kAttBK;
-    mbar_expect_tx(&full[s], 2 * kAttTile);
-    tma_load_2d(sK + s * kAttTile, &tmK, hcol, y, &full[s]);
-    tma_load_2d(sK + s * kAttTile + 8192, &tmK, hcol + 64, y, &full[s]);
-    tma_load_2d(sV + s * kAttTile, &tmV, hcol, y, &full[s]);
-    tma_load_2d(sV + s * kAttTile + 8192, &tmV, hcol + 64, y, &full[s]);
-  };
-  int last_issued = -1;  // meaningful in thread 0, which issues every copy
-  if (tid == 0) {
-    issue(0, 0);
-    last_issued = 0;
-    if (ntiles > 1) {
-      issue(1, 1);
-      last_issued = 1;
-    }
-  }
-  // Q tile -> shared memory in the same swizzled layout (zeros past the last row)
-  for (int e = tid; e < kAttBQ * 16; e += kAttThreads) {
-    const int row = e >> 4, ch = e & 15;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (row < nrows) v = *reinterpret_cast<const uint4*>(Q + (size_t)(r0 + row) * d + hcol + ch * 8);
-    *reinterpret_cast<uint4*>(sQ + ((ch >> 3) * 8192 + row * 128 + (((ch & 7) ^ (row & 7)) << 4))) = v;
-  }
-  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
 
-  const uint32_t qbase = smem_u32(sQ), kbase0 = smem_u32(sK), vbase0 = smem_u32(sV);
-  const int mi = lane >> 3, ri = lane & 7;
-  uint32_t qa[8][4];
-#pragma unroll
-  for (int ks = 0; ks < 8; ++ks)
-    ldsm_x4(qa[ks], sw_addr(qbase, warp * 16 + (mi & 1) * 8 + ri, ks * 16 + (mi >> 1) * 8));
-
-  float o[16][4];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
-  const int cq = lane & 3;
-
-  int jfail = ntiles;
-  for (int j = 0; j < ntiles; ++j) {
-    const int s = j & 1;
-    if (!mbar_wait(&full[s], (uint32_t)((j >> 1) & 1))) *s_bad = 1;
-    __syncthreads();
-    if (*s_bad) {
-      jfail = j;
-      break;
-    }
-    const uint32_t kb = kbase0 + s * kAttTile, vb = vbase0 + s * kAttTile;
-    float sc[8][4];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) sc[i][0] = sc[i][1] = sc[i][2] = sc[i][3] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < 8; ++ks) {
-#pragma unroll
-      for (int np = 0; np < 4; ++np) {
-        uint32_t kr[4];
-        ldsm_x4(kr, sw_addr(kb, (2 * np + (mi >> 1)) * 8 + ri, ks * 16 + (mi & 1) * 8));
-        mma16816(sc[2 * np], qa[ks], kr[0], kr[1]);
-        mma16816(sc[2 * np + 1], qa[ks], kr[2], kr[3]);
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (elect_one()) {
+      long long g = 0;  // chunk counter over this CTA's items
+      int t = 0;        // item counter
+      for (int i = blockIdx.x; i < nitems && !*s_abort; i += gridDim.x, ++t) {
+        const AttnItem it = attn_item(i, seg_ptr, B, H, N, S);
+        const int hc = it.h * kAttHD;
+        if (!mbar_wait(q_free, (uint32_t)((t & 1) ^ 1))) {
+          *s_abort = 1;
+          break;
+        }
+        mbar_expect_tx(q_full, kAttQBytes);
+        tma_load_2d(sQ, &tmQ, hc, it.r0, q_full);
+        tma_load_2d(sQ + kAttQBytes / 2, &tmQ, hc + 64, it.r0, q_full);
+        for (int c = it.c0; c < it.c1; ++c, ++g) {
+          const int st = (int)(g % kAttStages);
+          const uint32_t ph = (uint32_t)((g / kAttStages) & 1);
+          const int y = it.b * N + c * kAttBK;
+          if (!mbar_wait(&k_empty[st], ph ^ 1)) {
+            *s_abort = 1;
+            break;
+          }
+          mbar_expect_tx(&k_full[st], kAttKVBytes);
+          tma_load_2d(sK + st * kAttKVBytes, &tmK, hc, y, &k_full[st]);
+          tma_load_2d(sK + st * kAttKVBytes + kAttKVBytes / 2, &tmK, hc + 64, y, &k_full[st]);
+          if (!mbar_wait(&v_empty[st], ph ^ 1)) {
+            *s_abort = 1;
+            break;
+          }
+          mbar_expect_tx(&v_full[st], kAttKVBytes);
+          tma_load_2d(sV + st * kAttKVBytes, &tmV, hc, y, &v_full[st]);
+          tma_load_2d(sV + st * kAttKVBytes + kAttKVBytes / 2, &tmV, hc + 64, y, &v_full[st]);
+        }
       }
     }
-    const int key0 = (t0 + j) * kAttBK;
-    if (key0 + kAttBK > N) {
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      const uint32_t idesc_s = idesc_bf16(kAttBQ, kAttBK);
+      const uint32_t idesc_pv = idesc_bf16(kAttBQ, kAttHD) | (1u << 16);  // B = V chunk, MN-major
+      const uint32_t q0 = smem_u32(sQ);
+      long long g = 0;
+      int t = 0;
+      bool any = false;
+      // O += P_hi V + P_lo V for global chunk gj (first: the item's first chunk overwrites O)
+      auto issue_pv = [&](long long gj, bool first) -> bool {
+        const int pb = (int)(gj & 1), st = (int)(gj % kAttStages);
+        if (first && !mbar_wait(o_free, (uint32_t)((t & 1) ^ 1))) return false;  // last item's O read
+        if (!mbar_wait(&p_full[pb], (uint32_t)((gj >> 1) & 1))) return false;
+        if (!mbar_wait(&v_full[st], (uint32_t)((gj / kAttStages) & 1))) return false;
+        tc_fence_after();
+        const uint32_t vb = smem_u32(sV + st * kAttKVBytes);
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
+        for (int part = 0; part < 2; ++part) {
+          const uint64_t pdesc = sdesc_sw128(smem_u32(sP + (2 * pb + part) * kAttPBytes));
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (key0 + nt * 8 + 2 * cq + (e & 1) >= N) sc[nt][e] = -INFINITY;
-    }
+          for (int k = 0; k < kAttBK / 16; ++k)  // 16 keys per step: +32 B of P rows, +2 KB of V rows
+            umma_bf16(tmem_base, pdesc + 2 * k, sdesc_sw128_mn(vb + k * 2048, kAttKVBytes / 2), idesc_pv,
+                      (!first || part > 0 || k > 0) ? 1u : 0u);
+        }
+        umma_commit(&v_empty[st]);
+        umma_commit(pv_done);
+        return true;
+      };
+      for (int i = blockIdx.x; i < nitems && !*s_abort; i += gridDim.x, ++t) {
+        const AttnItem it = attn_item(i, seg_ptr, B, H, N, S);
+        const int n = it.c1 - it.c0;
+        bool ok = mbar_wait(q_full, (uint32_t)(t & 1));
+        tc_fence_after();
+        for (int j = 0; j < n && ok; ++j) {
+          const long long gj = g + j;
+          const int sb = (int)(gj & 1), st = (int)(gj % kAttStages);
+          ok = mbar_wait(&s_free[sb], (uint32_t)(((gj >> 1) & 1) ^ 1)) &&
+               mbar_wait(&k_full[st], (uint32_t)((gj / kAttStages) & 1));
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t kb = smem_u32(sK + st * kAttKVBytes);
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      float mx = -INFINITY;
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) mx = fmaxf(mx, fmaxf(sc[nt][2 * hf], sc[nt][2 * hf + 1]));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      const float m_new = fmaxf(m_r[hf], mx * scale_log2);
-      const float alpha = exp2f(m_r[hf] - m_new);
-      m_r[hf] = m_new;
-      float rs = 0.f;
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        const float p0 = exp2f(fmaf(sc[nt][2 * hf], scale_log2, -m_new));
-        const float p1 = exp2f(fmaf(sc[nt][2 * hf + 1], scale_log2, -m_new));
-        sc[nt][2 * hf] = p0;
-        sc[nt][2 * hf + 1] = p1;
-        rs += p0 + p1;
+          for (int k = 0; k < kAttHD / 16; ++k) {  // 16 dims per step: box k / 4, +32 B within it
+            const uint32_t qa = q0 + (k >> 2) * (kAttQBytes / 2), ka = kb + (k >> 2) * (kAttKVBytes / 2);
+            umma_bf16(tmem_base + 128 + sb * 64, sdesc_sw128(qa) + 2 * (k & 3), sdesc_sw128(ka) + 2 * (k & 3),
+                      idesc_s, k > 0 ? 1u : 0u);
+          }
+          any = true;
+          umma_commit(&s_full[sb]);
+          umma_commit(&k_empty[st]);
+          if (j >= 1) ok = issue_pv(gj - 1, j == 1);  // P V of the previous chunk overlaps this softmax
+        }
+        if (ok) ok = issue_pv(g + n - 1, n == 1);
+        if (!ok) {
+          *s_abort = 1;
+          break;
+        }
+        umma_commit(q_free);  // every MMA reading this Q has completed
+        g += n;
       }
-      l_r[hf] = l_r[hf] * alpha + rs;
-#pragma unroll
-      for (int nt = 0; nt < 16; ++nt) {
-        o[nt][2 * hf] *= alpha;
-        o[nt][2 * hf + 1] *= alpha;
+      if (*s_abort && any) {
+        umma_commit(drain);
+        (void)mbar_wait(drain, 0);
       }
     }
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      uint32_t ah[4], al[4];
-      split_pair(sc[2 * kk][0], sc[2 * kk][1], ah[0], al[0]);
-      split_pair(sc[2 * kk][2], sc[2 * kk][3], ah[1], al[1]);
-      split_pair(sc[2 * kk + 1][0], sc[2 * kk + 1][1], ah[2], al[2]);
-      split_pair(sc[2 * kk + 1][2], sc[2 * kk + 1][3], ah[3], al[3]);
-#pragma unroll
-      for (int np = 0; np < 8; ++np) {
-        uint32_t vr[4];
-        ldsm_x4_t(vr, sw_addr(vb, kk * 16 + (mi & 1) * 8 + ri, (2 * np + (mi >> 1)) * 8));
-        mma16816(o[2 * np], ah, vr[0], vr[1]);
-        mma16816(o[2 * np], al, vr[0], vr[1]);
-        mma16816(o[2 * np + 1], ah, vr[2], vr[3]);
-        mma16816(o[2 * np + 1], al, vr[2], vr[3]);
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax: one query row per thread
+    const int q = warp & 3;  // a warp reads TMEM lanes 32 * (warp % 4) ..
+    const int row = q * 32 + lane;
+    const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
+    const int nch = ceil_div(N, kAttBK);
+    long long g = 0, pv_waited = 0;
+    int t = 0;
+    bool ok = true;
+    // waits for the P V of every chunk up to global chunk k, in order (one phase at a time)
+    auto wait_pv_upto = [&](long long k) -> bool {
+      while (pv_waited <= k) {
+        if (!mbar_wait(pv_done, (uint32_t)(pv_waited & 1))) return false;
+        ++pv_waited;
       }
-    }
-    __syncthreads();  // every warp is done with stage s
-    if (tid == 0 && j + 2 < ntiles) {
-      issue(j + 2, s);
-      last_issued = j + 2;
-    }
-  }
-  if (*s_bad) {
-    // bounded wait for the copies this CTA started, then leave without writing
-    if (tid == 0)
-      for (int t = jfail; t <= last_issued; ++t) (void)mbar_wait(&full[t & 1], (uint32_t)((t >> 1) & 1));
-    return;
-  }
+      return true;
+    };
+    for (int i = blockIdx.x; i < nitems && ok; i += gridDim.x, ++t) {
+      const AttnItem it = attn_item(i, seg_ptr, B, H, N, S);
+      const int n = it.c1 - it.c0;
+      float m_used = -INFINITY, l = 0.f;
+      for (int j = 0; j < n; ++j) {
+        const long long gj = g + j;
+        const int sb = (int)(gj & 1);
+        ok = mbar_wait(&s_full[sb], (uint32_t)((gj >> 1) & 1)) && !*s_abort;
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t ra[32], rb[32];
+        tmem_ld32(lane_base + 128 + sb * 64, ra);
+        tmem_ld32(lane_base + 128 + sb * 64 + 32, rb);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[sb]);
+        float sc[kAttBK];
 #pragma unroll
-  for (int hf = 0; hf < 2; ++hf) {
-    float l = l_r[hf];
-    l += __shfl_xor_sync(0xffffffffu, l, 1);
-    l += __shfl_xor_sync(0xffffffffu, l, 2);
-    const int row = warp * 16 + (lane >> 2) + 8 * hf;
-    if (row >= nrows) continue;
-    if (S == 1) {
+        for (int e = 0; e < 32; ++e) {
+          sc[e] = __uint_as_float(ra[e]);
+          sc[32 + e] = __uint_as_float(rb[e]);
+        }
+        const int key0 = (it.c0 + j) * kAttBK;
+        if (key0 + kAttBK > N) {
+#pragma unroll
+          for (int e = 0; e < kAttBK; ++e)
+            if (key0 + e >= N) sc[e] = -INFINITY;
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < kAttBK; ++e) mx = fmaxf(mx, sc[e]);
+        const float mc = mx * scale_log2;  // every chunk holds at least one key < N
+        const bool need = mc > m_used + kAttStaleMax;
+        float factor = 1.f;
+        if (need) {
+          factor = exp2f(m_used - mc);  // 0 for the first chunk
+          m_used = mc;
+        }
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          // the previous chunks' P V must be complete before O rows are rescaled
+          ok = wait_pv_upto(gj - 1);
+          if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int cb = 0; cb < kAttHD / 32; ++cb) {
+            uint32_t o[32];
+            tmem_ld32(lane_base + cb * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+            tmem_st32(lane_base + cb * 32, o);
+          }
+          tmem_st_wait();
+        }
+        l *= factor;
+        ok = wait_pv_upto(gj - 2);  // the P V that read P buffer sb has completed
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        // P = 2^(s * scale - m_used) <= 2^8, as bf16 high + low parts, K-major with 128-byte swizzle
+        uint8_t* ph = sP + (2 * sb) * kAttPBytes;
+        uint8_t* pl = ph + kAttPBytes;
+        const uint32_t rowoff = (uint32_t)((row >> 3) * 1024 + (row & 7) * 128);
+#pragma unroll
+        for (int c = 0; c < kAttBK / 8; ++c) {
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float p0 = exp2f(fmaf(sc[c * 8 + 2 * e], scale_log2, -m_used));
+            const float p1 = exp2f(fmaf(sc[c * 8 + 2 * e + 1], scale_log2, -m_used));
+            l += p0 + p1;
+            split_pair(p0, p1, hi[e], lo[e]);
+          }
+          const uint32_t off = rowoff + ((uint32_t)(c ^ (row & 7)) << 4);
+          *reinterpret_cast<uint4*>(ph + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(pl + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+        fence_proxy_async_smem();  // P visible to the tensor cores
+        tc_fence_before();         // and any O rescale ordered before the next P V
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[sb]);
+      }
+      if (!ok) break;
+      ok = wait_pv_upto(g + n - 1);  // O is final
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const bool whole = (n == nch);  // no key split: normalise and store bf16
+      const int grow = it.r0 + row;
       const float inv = 1.0f / l;
-      __nv_bfloat16* dst = Aout + (size_t)(r0 + row) * d + hcol + 2 * cq;
 #pragma unroll
-      for (int nt = 0; nt < 16; ++nt)
-        *reinterpret_cast<uint32_t*>(dst + nt * 8) = pack_bf16(o[nt][2 * hf] * inv, o[nt][2 * hf + 1] * inv);
-    } else {
-      float* dst = sp.o_part + ((size_t)split * sp.part_rows + (r0 + row)) * d + hcol + 2 * cq;
+      for (int cb = 0; cb < kAttHD / 32; ++cb) {
+        uint32_t o[32];
+        tmem_ld32(lane_base + cb * 32, o);
+        tmem_ld_wait();
+        if (row < it.nrows) {
+          if (whole) {
+            uint4* dst = reinterpret_cast<uint4*>(Aout + (size_t)grow * d + it.h * kAttHD + cb * 32);
 #pragma unroll
-      for (int nt = 0; nt < 16; ++nt)
-        *reinterpret_cast<float2*>(dst + nt * 8) = make_float2(o[nt][2 * hf], o[nt][2 * hf + 1]);
-      if (cq == 0) sp.ml[((size_t)split * sp.part_rows + (r0 + row)) * gridDim.y + h] = make_float2(m_r[hf], l);
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(pack_bf16(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv),
+                                  pack_bf16(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv),
+                                  pack_bf16(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv),
+                                  pack_bf16(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(sp.o_part + ((size_t)it.split * sp.part_rows + grow) * d +
+                                                    it.h * kAttHD + cb * 32);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
+                                   __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
+          }
+        }
+      }
+      if (!whole && row < it.nrows) sp.ml[((size_t)it.split * sp.part_rows + grow) * H + it.h] = make_float2(m_used, l);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(o_free);
+      g += n;
     }
+    if (!ok && lane == 0) *s_abort = 1;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kAttTmemCols);
   }
 }
 
 // out[row, h] = sum_s 2^(m_s - m) o_s / sum_s 2^(m_s - m) l_s, one CTA per active row.
 __global__ void __launch_bounds__(256) attn_combine_kernel(const int32_t* __restrict__ seg_ptr, int B, int H,
-                                                           int d, AttnSplit sp, __nv_bfloat16* __restrict__ Aout) {
+                                                           int N, int d, AttnSplit sp,
+                                                           __nv_bfloat16* __restrict__ Aout) {
   pdl_wait();
   pdl_trigger();
   const int j = blockIdx.x;
   if (j >= seg_ptr[B]) return;
-  const int S = attn_splits(seg_ptr, B, H, sp.smax, sp.nsm);
+  const int S = attn_splits(seg_ptr, B, H, N, sp.smax, sp.nsm);
   if (S == 1) return;
   for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
     const int h = c / kAttHD;
@@ -339,8 +531,8 @@ __global__ void attn_f32_kernel(const float* __restrict__ Q, const float* __rest
 }
 
 int attn_split_rows(const plk_dims* dims, int num_sms) {
-  // splits are used only while q-tiles x heads < 2 x SMs, so fewer active rows
-  const int rows = ceil_div(2 * num_sms, dims->H) * kAttBQ;
+  // keys are split only while query tiles x heads < SMs, so fewer active rows than this
+  const int rows = ceil_div(num_sms, dims->H) * kAttBQ;
   return std::min(dims->B * dims->N, rows);
 }
 
@@ -348,25 +540,25 @@ int launch_attention_bf16(const plk_dims* dims, const void* q, const void* K_cac
                           void* a_out, const int32_t* seg_ptr, float* o_part, void* ml, int smax, int part_rows,
                           int num_sms, cudaStream_t st) {
   const int B = dims->B, N = dims->N, d = dims->d, H = dims->H;
-  CUtensorMap tmK, tmV;
-  if (make_tmap_bf16(&tmK, K_cache, (uint64_t)B * N, (uint64_t)d, 64) != PLK_OK) return PLK_ERR_CUDA;
-  if (make_tmap_bf16(&tmV, V_cache, (uint64_t)B * N, (uint64_t)d, 64) != PLK_OK) return PLK_ERR_CUDA;
+  CUtensorMap tmQ, tmK, tmV;
+  if (make_tmap_bf16(&tmQ, q, (uint64_t)B * N, (uint64_t)d, kAttBQ) != PLK_OK) return PLK_ERR_CUDA;
+  if (make_tmap_bf16(&tmK, K_cache, (uint64_t)B * N, (uint64_t)d, kAttBK) != PLK_OK) return PLK_ERR_CUDA;
+  if (make_tmap_bf16(&tmV, V_cache, (uint64_t)B * N, (uint64_t)d, kAttBK) != PLK_OK) return PLK_ERR_CUDA;
   static int attr_done[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PLK_ERR_CUDA;
   if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(attn_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttSmem) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttSmem) != cudaSuccess)
       return PLK_ERR_CUDA;
     attr_done[dev] = 1;
   }
   const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->hd));
   AttnSplit sp{o_part, (float2*)ml, std::max(1, std::min(smax, ceil_div(N, kAttBK))), part_rows, num_sms};
-  dim3 grid(ceil_div(N, kAttBQ), H, B * sp.smax);
-  const int rc = launch_pdl(attn_bf16_kernel, grid, dim3(kAttThreads), kAttSmem, st, tmK, tmV,
-                            (const __nv_bfloat16*)q, (__nv_bfloat16*)a_out, seg_ptr, B, N, d, scale_log2, sp);
+  // persistent: one CTA per SM walks the (query tile, head, key split) items
+  const int rc = launch_pdl(attn_tc_kernel, dim3(num_sms), dim3(kAttThreads), kAttSmem, st, tmQ, tmK, tmV,
+                            (__nv_bfloat16*)a_out, seg_ptr, B, N, H, d, scale_log2, sp);
   if (rc != PLK_OK || sp.smax == 1) return rc;
-  return launch_pdl(attn_combine_kernel, dim3(part_rows), dim3(256), 0, st, seg_ptr, B, H, d, sp,
+  return launch_pdl(attn_combine_kernel, dim3(part_rows), dim3(256), 0, st, seg_ptr, B, H, N, d, sp,
                     (__nv_bfloat16*)a_out);
 }
 
