@@ -154,11 +154,11 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
   uint64_t* s_full = bars + 14;   // [2] scores of a chunk in TMEM
   uint64_t* s_free = bars + 16;   // [2] scores read by the 4 softmax warps
   uint64_t* p_full = bars + 18;   // [2] P of a chunk in shared memory (4 softmax warps)
-  uint64_t* pv_done = bars + 20;  // one phase per chunk: its P V has completed
-  uint64_t* o_free = bars + 21;   // O read out by the 4 softmax warps
-  uint64_t* drain = bars + 22;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 23);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 24);
+  uint64_t* p_free = bars + 20;   // [2] the P V that read P buffer x has completed
+  uint64_t* o_free = bars + 22;   // O read out by the 4 softmax warps
+  uint64_t* drain = bars + 23;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 24);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 25);
 
   pdl_wait();
   pdl_trigger();
@@ -180,8 +180,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
       mbar_init(&s_full[i], 1);
       mbar_init(&s_free[i], 4);
       mbar_init(&p_full[i], 4);
+      mbar_init(&p_free[i], 1);
     }
-    mbar_init(pv_done, 1);
     mbar_init(o_free, 4);
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -262,7 +262,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
                       (!first || part > 0 || k > 0) ? 1u : 0u);
         }
         umma_commit(&v_empty[st]);
-        umma_commit(pv_done);
+        umma_commit(&p_free[pb]);  // also: every earlier MMA, so O holds chunks <= gj
         return true;
       };
       for (int i = blockIdx.x; i < nitems && !*s_abort; i += gridDim.x, ++t) {
@@ -309,16 +309,13 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
     const int row = q * 32 + lane;
     const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
     const int nch = ceil_div(N, kAttBK);
-    long long g = 0, pv_waited = 0;
+    long long g = 0;
     int t = 0;
     bool ok = true;
-    // waits for the P V of every chunk up to global chunk k, in order (one phase at a time)
-    auto wait_pv_upto = [&](long long k) -> bool {
-      while (pv_waited <= k) {
-        if (!mbar_wait(pv_done, (uint32_t)(pv_waited & 1))) return false;
-        ++pv_waited;
-      }
-      return true;
+    // waits until the P V of global chunk k (and every MMA before it) has completed; k's
+    // buffer cannot have moved on, its next P V needs P of chunk k + 2 from these warps
+    auto wait_pv = [&](long long k) -> bool {
+      return k < 0 || mbar_wait(&p_free[k & 1], (uint32_t)((k >> 1) & 1));
     };
     for (int i = blockIdx.x; i < nitems && ok; i += gridDim.x, ++t) {
       const AttnItem it = attn_item(i, seg_ptr, B, H, N, S);
@@ -364,7 +361,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
         }
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           // the previous chunks' P V must be complete before O rows are rescaled
-          ok = wait_pv_upto(gj - 1);
+          ok = wait_pv(gj - 1);
           if (!__all_sync(0xffffffffu, ok)) {
             ok = false;
             break;
@@ -382,7 +379,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
           tmem_st_wait();
         }
         l *= factor;
-        ok = wait_pv_upto(gj - 2);  // the P V that read P buffer sb has completed
+        ok = wait_pv(gj - 2);  // the P V that read P buffer sb has completed
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
@@ -411,7 +408,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
         if (lane == 0) mbar_arrive(&p_full[sb]);
       }
       if (!ok) break;
-      ok = wait_pv_upto(g + n - 1);  // O is final
+      ok = wait_pv(g + n - 1);  // O is final
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
         break;
