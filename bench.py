@@ -449,7 +449,7 @@ def main():
             dist.destroy_process_group()
     if res is None or rank != 0:
         return 0
-    launches_per_step = 1 + 1 + 11 + 1  # score, select, layer (attention + combine), commit
+    launches_per_step = 1 + 1 + 10 + 1  # score, select, layer, commit
     line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",

@@ -213,9 +213,9 @@ int plk_selftest_wait_timeout(void* stream);
 /* Tracing.  Registers up to 16 cudaEvent_t handles (passed as void*).  While
  * registered, plk_layer_step_partial and plk_full_layer_step record events[0]
  * on their stream before their first kernel and events[i] after their i-th
- * step of the chain (the bf16 step has 10: RMSNorm1, QKV GEMM, QKV finish,
- * attention (one or two kernels), O GEMM, RMSNorm2, gate/up GEMM, SwiGLU
- * finish, down GEMM, output finish), so a caller can time every kernel with
+ * kernel of the chain (the bf16 step has 10: RMSNorm1, QKV GEMM, QKV finish,
+ * attention, O GEMM, RMSNorm2, gate/up GEMM, SwiGLU finish, down GEMM, output
+ * finish), so a caller can time every kernel with
  * cudaEventElapsedTime on the launching stream.  n = 0 unregisters.  The events
  * must outlive their registration.  Host-side state, not thread-safe. */
 int plk_trace_events(void* const* events, int n);

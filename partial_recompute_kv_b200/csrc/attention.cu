@@ -33,17 +33,22 @@ constexpr int kAttHD = 128;
 constexpr int kAttBQ = 128;                    // queries per CTA (UMMA M, one TMEM lane each)
 constexpr int kAttBK = 64;                     // keys per chunk (UMMA N of S, K of P V)
 constexpr int kAttStages = 3;                  // K and V ring depth
-constexpr int kAttThreads = 192;               // warp 0 TMA, warp 1 MMA, warps 2-5 softmax
+constexpr int kAttSoftWarps = 8;               // two warps per TMEM lane quarter, one per half row
+constexpr int kAttThreads = 32 * (2 + kAttSoftWarps);  // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
 constexpr int kAttQBytes = kAttBQ * kAttHD * 2;   // 32 KB
 constexpr int kAttKVBytes = kAttBK * kAttHD * 2;  // 16 KB
 constexpr int kAttPBytes = kAttBQ * kAttBK * 2;   // 16 KB (high or low part)
 constexpr size_t kAttOffK = kAttQBytes;
 constexpr size_t kAttOffV = kAttOffK + (size_t)kAttStages * kAttKVBytes;
 constexpr size_t kAttOffP = kAttOffV + (size_t)kAttStages * kAttKVBytes;  // [2 buffers][high, low]
-constexpr size_t kAttOffBar = kAttOffP + 4 * (size_t)kAttPBytes;
-constexpr int kAttSmem = (int)kAttOffBar + 256 + 1024;
+constexpr size_t kAttOffML = kAttOffP + 4 * (size_t)kAttPBytes;            // [128] (max, sum) of the odd CTA
+constexpr size_t kAttOffXM = kAttOffML + kAttBQ * 8;                       // [2][2 halves][128] row max
+constexpr size_t kAttOffXL = kAttOffXM + 2 * 2 * kAttBQ * 4;               // [2 halves][128] row sum
+constexpr size_t kAttOffBar = kAttOffXL + 2 * kAttBQ * 4;
+constexpr int kAttSmem = (int)kAttOffBar + 512 + 1024;
 constexpr uint32_t kAttTmemCols = 256;         // O: 0..127, S buffers: 128..191, 192..255
 constexpr float kAttStaleMax = 8.f;            // log2 headroom before a row's O is rescaled
+static_assert(4 * kAttPBytes == kAttBQ * kAttHD * 4, "the P region holds one fp32 O tile");
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -72,51 +77,30 @@ __device__ __forceinline__ uint64_t sdesc_sw128_mn(uint32_t saddr, uint32_t mn_b
   d |= (uint64_t)2 << 61;
   return d;
 }
+__device__ __forceinline__ void st_dsmem_v4(uint32_t addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void st_dsmem_v2(uint32_t addr, float2 v) {
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(v.x), "f"(v.y) : "memory");
+}
 }  // namespace
 
-// Key splits for the current active set (device-side M, no host sync): the
-// split count s <= smax minimising whole waves of CTAs x chunks per CTA, one
-// CTA per SM, plus one chunk's worth for the combine when s > 1.  Splits are
-// considered only while the query tiles x heads leave SMs idle.  Computed
-// identically by the attention and combine kernels.
-__device__ __forceinline__ int attn_qtiles(const int32_t* seg_ptr, int B) {
+// Work units: (128-query tile of one sequence, head).  Computed on the device
+// from seg_ptr (no host synchronisation).
+__device__ __forceinline__ int attn_units(const int32_t* seg_ptr, int B, int H) {
   int qt = 0;
   for (int b = 0; b < B; ++b) qt += ceil_div(seg_ptr[b + 1] - seg_ptr[b], kAttBQ);
-  return qt;
+  return qt * H;
 }
-__device__ __forceinline__ int attn_splits(const int32_t* seg_ptr, int B, int H, int N, int smax, int nsm) {
-  const int items = attn_qtiles(seg_ptr, B) * H;
-  if (items == 0 || items >= nsm) return 1;
-  const int nch = ceil_div(N, kAttBK);
-  int best = 1, best_cost = 1 << 30;
-  for (int s = 1; s <= smax && s <= nch; ++s) {
-    const int cost = ceil_div(items * s, nsm) * ceil_div(nch, s) * 2 + (s > 1 ? 1 : 0);
-    if (cost < best_cost) {
-      best_cost = cost;
-      best = s;
-    }
-  }
-  return best;
-}
-
-// Split partials: o_part[s][row][d] (unnormalised, fp32) and ml[s][row][h] = (max, sum)
-// in the log2 domain; rows are compact active-row indices below part_rows.
-struct AttnSplit {
-  float* o_part;
-  float2* ml;
-  int smax, part_rows, nsm;
+struct AttnUnit {
+  int b, h, r0, nrows;
 };
-
-// One work item: 128 queries [r0, r0 + nrows) of sequence b, head h, chunks [c0, c1).
-struct AttnItem {
-  int b, h, split, r0, nrows, c0, c1;
-};
-__device__ __forceinline__ AttnItem attn_item(int i, const int32_t* seg_ptr, int B, int H, int N, int S) {
-  AttnItem it;
-  it.split = i % S;
-  const int rest = i / S;
-  it.h = rest % H;
-  int qi = rest / H, b = 0;
+__device__ __forceinline__ AttnUnit attn_unit(int u, const int32_t* seg_ptr, int B, int H) {
+  AttnUnit it;
+  it.h = u % H;
+  int qi = u / H, b = 0;
   for (; b < B; ++b) {
     const int qt = ceil_div(seg_ptr[b + 1] - seg_ptr[b], kAttBQ);
     if (qi < qt) break;
@@ -125,10 +109,31 @@ __device__ __forceinline__ AttnItem attn_item(int i, const int32_t* seg_ptr, int
   it.b = b;
   it.r0 = seg_ptr[b] + qi * kAttBQ;
   it.nrows = min(kAttBQ, seg_ptr[b + 1] - it.r0);
-  const int nch = ceil_div(N, kAttBK);
-  it.c0 = it.split * nch / S;
-  it.c1 = (it.split + 1) * nch / S;
   return it;
+}
+
+// The grid is clusters of two CTAs.  When every unit fits on a CTA pair at once
+// (2 x units <= CTAs) the two CTAs of a cluster split the unit's keys in halves
+// and the odd CTA hands its partial (O, max, sum) to the even one through
+// distributed shared memory; otherwise every CTA takes whole units on its own.
+struct AttnPlan {
+  int split;   // 1 or 2
+  int first;   // first unit of this CTA
+  int stride;  // unit stride
+  int units;
+};
+__device__ __forceinline__ AttnPlan attn_plan(const int32_t* seg_ptr, int B, int H, int N) {
+  AttnPlan p;
+  p.units = attn_units(seg_ptr, B, H);
+  p.split = (2 * p.units <= (int)gridDim.x && ceil_div(N, kAttBK) >= 2) ? 2 : 1;
+  if (p.split == 2) {
+    p.first = blockIdx.x >> 1;
+    p.stride = gridDim.x >> 1;
+  } else {
+    p.first = blockIdx.x;
+    p.stride = gridDim.x;
+  }
+  return p;
 }
 
 __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -136,14 +141,16 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
                                                                const __grid_constant__ CUtensorMap tmV,
                                                                __nv_bfloat16* __restrict__ Aout,
                                                                const int32_t* __restrict__ seg_ptr, int B, int N,
-                                                               int H, int d, float scale_log2, AttnSplit sp) {
+                                                               int H, int d, float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
-  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // same offset in both CTAs
   uint8_t* sQ = smem;
   uint8_t* sK = smem + kAttOffK;
   uint8_t* sV = smem + kAttOffV;
   uint8_t* sP = smem + kAttOffP;  // buffer x: high part at 2x, low part at 2x + 1 (16 KB each)
+  float* xmax = reinterpret_cast<float*>(smem + kAttOffXM);  // [chunk parity][half][row]
+  float* xl = reinterpret_cast<float*>(smem + kAttOffXL);    // [half][row]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAttOffBar);
   uint64_t* q_full = bars + 0;
   uint64_t* q_free = bars + 1;
@@ -152,20 +159,30 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
   uint64_t* v_full = bars + 8;    // [3]
   uint64_t* v_empty = bars + 11;  // [3]
   uint64_t* s_full = bars + 14;   // [2] scores of a chunk in TMEM
-  uint64_t* s_free = bars + 16;   // [2] scores read by the 4 softmax warps
-  uint64_t* p_full = bars + 18;   // [2] P of a chunk in shared memory (4 softmax warps)
+  uint64_t* s_free = bars + 16;   // [2] scores read by the 8 softmax warps
+  uint64_t* p_full = bars + 18;   // [2] P of a chunk in shared memory (8 softmax warps)
   uint64_t* p_free = bars + 20;   // [2] the P V that read P buffer x has completed
-  uint64_t* o_free = bars + 22;   // O read out by the 4 softmax warps
+  uint64_t* o_free = bars + 22;   // O read out by the 8 softmax warps
   uint64_t* drain = bars + 23;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 24);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 25);
+  uint64_t* xo_full = bars + 24;  // even CTA: the odd CTA's partial is in my P region (8 warps)
+  uint64_t* xo_free = bars + 25;  // odd CTA: the even CTA's P region is free for my partial (8 warps)
+  uint64_t* xmb = bars + 26;      // [4 quarters][2] row-max exchange of the two warps of a quarter
+  uint64_t* xlb = bars + 34;      // [4 quarters] row-sum exchange
+  uint64_t* xo_read = bars + 38;  // even CTA: all 8 softmax warps have read the odd CTA's partial
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 39);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 40);
 
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int S = attn_splits(seg_ptr, B, H, N, sp.smax, sp.nsm);
-  const int nitems = attn_qtiles(seg_ptr, B) * H * S;
-  if ((int)blockIdx.x >= nitems) return;
+  const int rank = (int)cluster_ctarank();
+  const AttnPlan plan = attn_plan(seg_ptr, B, H, N);
+  const int nch = ceil_div(N, kAttBK);
+  const int c0 = plan.split == 2 ? rank * nch / 2 : 0;  // this CTA's key chunks of every unit
+  const int c1 = plan.split == 2 ? (rank + 1) * nch / 2 : nch;
+  const int n = c1 - c0;
+  // the two CTAs of a cluster see the same plan; with a split they also see the same units
+  if (plan.first >= plan.units) return;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -178,12 +195,17 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
-      mbar_init(&p_full[i], 4);
+      mbar_init(&s_free[i], kAttSoftWarps);
+      mbar_init(&p_full[i], kAttSoftWarps);
       mbar_init(&p_free[i], 1);
     }
-    mbar_init(o_free, 4);
+    mbar_init(o_free, kAttSoftWarps);
     mbar_init(drain, 1);
+    mbar_init(xo_full, kAttSoftWarps);
+    mbar_init(xo_free, kAttSoftWarps);
+    for (int i = 0; i < 8; ++i) mbar_init(&xmb[i], 2);
+    for (int i = 0; i < 4; ++i) mbar_init(&xlb[i], 2);
+    mbar_init(xo_read, kAttSoftWarps);
     *s_abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -195,17 +217,20 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
     tmem_relinquish();
   }
   tc_fence_before();
-  __syncthreads();
+  if (plan.split == 2)
+    cluster_sync_all();  // the partner's exchange barriers are initialised
+  else
+    __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (elect_one()) {
-      long long g = 0;  // chunk counter over this CTA's items
-      int t = 0;        // item counter
-      for (int i = blockIdx.x; i < nitems && !*s_abort; i += gridDim.x, ++t) {
-        const AttnItem it = attn_item(i, seg_ptr, B, H, N, S);
+      long long g = 0;  // chunk counter over this CTA's units
+      int t = 0;        // unit counter
+      for (int u = plan.first; u < plan.units && !*s_abort; u += plan.stride, ++t) {
+        const AttnUnit it = attn_unit(u, seg_ptr, B, H);
         const int hc = it.h * kAttHD;
         if (!mbar_wait(q_free, (uint32_t)((t & 1) ^ 1))) {
           *s_abort = 1;
@@ -214,7 +239,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
         mbar_expect_tx(q_full, kAttQBytes);
         tma_load_2d(sQ, &tmQ, hc, it.r0, q_full);
         tma_load_2d(sQ + kAttQBytes / 2, &tmQ, hc + 64, it.r0, q_full);
-        for (int c = it.c0; c < it.c1; ++c, ++g) {
+        for (int c = c0; c < c1; ++c, ++g) {
           const int st = (int)(g % kAttStages);
           const uint32_t ph = (uint32_t)((g / kAttStages) & 1);
           const int y = it.b * N + c * kAttBK;
@@ -245,10 +270,10 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
       long long g = 0;
       int t = 0;
       bool any = false;
-      // O += P_hi V + P_lo V for global chunk gj (first: the item's first chunk overwrites O)
+      // O += P_hi V + P_lo V for global chunk gj (first: the unit's first chunk overwrites O)
       auto issue_pv = [&](long long gj, bool first) -> bool {
         const int pb = (int)(gj & 1), st = (int)(gj % kAttStages);
-        if (first && !mbar_wait(o_free, (uint32_t)((t & 1) ^ 1))) return false;  // last item's O read
+        if (first && !mbar_wait(o_free, (uint32_t)((t & 1) ^ 1))) return false;  // last unit's O read
         if (!mbar_wait(&p_full[pb], (uint32_t)((gj >> 1) & 1))) return false;
         if (!mbar_wait(&v_full[st], (uint32_t)((gj / kAttStages) & 1))) return false;
         tc_fence_after();
@@ -265,9 +290,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
         umma_commit(&p_free[pb]);  // also: every earlier MMA, so O holds chunks <= gj
         return true;
       };
-      for (int i = blockIdx.x; i < nitems && !*s_abort; i += gridDim.x, ++t) {
-        const AttnItem it = attn_item(i, seg_ptr, B, H, N, S);
-        const int n = it.c1 - it.c0;
+      for (int u = plan.first; u < plan.units && !*s_abort; u += plan.stride, ++t) {
         bool ok = mbar_wait(q_full, (uint32_t)(t & 1));
         tc_fence_after();
         for (int j = 0; j < n && ok; ++j) {
@@ -304,11 +327,19 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax: one query row per thread
-    const int q = warp & 3;  // a warp reads TMEM lanes 32 * (warp % 4) ..
+    // ------------------------------------------------------------ softmax: half a query row per thread
+    const int q = warp & 3;              // a warp reads TMEM lanes 32 * (warp % 4) ..
+    const int hf = (warp - 2) >> 2;      // warps 2-5 take keys 0-31 of a chunk (O dims 0-63), 6-9 the rest
     const int row = q * 32 + lane;
     const uint32_t lane_base = tmem_base + ((uint32_t)(q * 32) << 16);
-    const int nch = ceil_div(N, kAttBK);
+    // the two warps sharing these rows exchange through shared memory; lane 0 of each arrives
+    // on an mbarrier (count 2) after the warp's writes, and both warps wait on it (bounded)
+    auto pair_exchange = [&](uint64_t* bar, uint32_t parity) -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
+      return mbar_wait(bar, parity);
+    };
+    float* ml = reinterpret_cast<float*>(smem + kAttOffML);
     long long g = 0;
     int t = 0;
     bool ok = true;
@@ -317,9 +348,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
     auto wait_pv = [&](long long k) -> bool {
       return k < 0 || mbar_wait(&p_free[k & 1], (uint32_t)((k >> 1) & 1));
     };
-    for (int i = blockIdx.x; i < nitems && ok; i += gridDim.x, ++t) {
-      const AttnItem it = attn_item(i, seg_ptr, B, H, N, S);
-      const int n = it.c1 - it.c0;
+    for (int u = plan.first; u < plan.units && ok; u += plan.stride, ++t) {
+      const AttnUnit it = attn_unit(u, seg_ptr, B, H);
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < n; ++j) {
         const long long gj = g + j;
@@ -330,30 +360,35 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
           break;
         }
         tc_fence_after();
-        uint32_t ra[32], rb[32];
-        tmem_ld32(lane_base + 128 + sb * 64, ra);
-        tmem_ld32(lane_base + 128 + sb * 64 + 32, rb);
+        uint32_t ra[32];
+        tmem_ld32(lane_base + 128 + sb * 64 + hf * 32, ra);
         tmem_ld_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_free[sb]);
-        float sc[kAttBK];
+        float sc[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          sc[e] = __uint_as_float(ra[e]);
-          sc[32 + e] = __uint_as_float(rb[e]);
-        }
-        const int key0 = (it.c0 + j) * kAttBK;
-        if (key0 + kAttBK > N) {
+        for (int e = 0; e < 32; ++e) sc[e] = __uint_as_float(ra[e]);
+        const int key0 = (c0 + j) * kAttBK + hf * 32;
+        if (key0 + 32 > N) {
 #pragma unroll
-          for (int e = 0; e < kAttBK; ++e)
+          for (int e = 0; e < 32; ++e)
             if (key0 + e >= N) sc[e] = -INFINITY;
         }
         float mx = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < kAttBK; ++e) mx = fmaxf(mx, sc[e]);
+        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, sc[e]);
+        // the row max over both halves (double-buffered by chunk parity)
+        float* xm = xmax + (size_t)(gj & 1) * 2 * kAttBQ;
+        xm[hf * kAttBQ + row] = mx;
+        ok = pair_exchange(&xmb[q * 2 + (int)(gj & 1)], (uint32_t)((gj >> 1) & 1));
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        mx = fmaxf(mx, xm[(1 - hf) * kAttBQ + row]);
         const float mc = mx * scale_log2;  // every chunk holds at least one key < N
-        const bool need = mc > m_used + kAttStaleMax;
+        const bool need = mc > m_used + kAttStaleMax;  // identical in both halves of the row
         float factor = 1.f;
         if (need) {
           factor = exp2f(m_used - mc);  // 0 for the first chunk
@@ -368,18 +403,20 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
           }
           tc_fence_after();
 #pragma unroll
-          for (int cb = 0; cb < kAttHD / 32; ++cb) {
+          for (int cb = 0; cb < 2; ++cb) {
             uint32_t o[32];
-            tmem_ld32(lane_base + cb * 32, o);
+            tmem_ld32(lane_base + hf * 64 + cb * 32, o);
             tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-            tmem_st32(lane_base + cb * 32, o);
+            tmem_st32(lane_base + hf * 64 + cb * 32, o);
           }
           tmem_st_wait();
         }
         l *= factor;
         ok = wait_pv(gj - 2);  // the P V that read P buffer sb has completed
+        // even CTA with a split: the odd CTA's last partial, which sat in the P region, is consumed
+        if (plan.split == 2 && rank == 0 && j == 0 && t > 0) ok = ok && mbar_wait(xo_read, (uint32_t)((t - 1) & 1));
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
@@ -389,16 +426,16 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
         uint8_t* pl = ph + kAttPBytes;
         const uint32_t rowoff = (uint32_t)((row >> 3) * 1024 + (row & 7) * 128);
 #pragma unroll
-        for (int c = 0; c < kAttBK / 8; ++c) {
+        for (int cc = 0; cc < 4; ++cc) {
           uint32_t hi[4], lo[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float p0 = exp2f(fmaf(sc[c * 8 + 2 * e], scale_log2, -m_used));
-            const float p1 = exp2f(fmaf(sc[c * 8 + 2 * e + 1], scale_log2, -m_used));
+            const float p0 = exp2f(fmaf(sc[cc * 8 + 2 * e], scale_log2, -m_used));
+            const float p1 = exp2f(fmaf(sc[cc * 8 + 2 * e + 1], scale_log2, -m_used));
             l += p0 + p1;
             split_pair(p0, p1, hi[e], lo[e]);
           }
-          const uint32_t off = rowoff + ((uint32_t)(c ^ (row & 7)) << 4);
+          const uint32_t off = rowoff + ((uint32_t)((hf * 4 + cc) ^ (row & 7)) << 4);
           *reinterpret_cast<uint4*>(ph + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
           *reinterpret_cast<uint4*>(pl + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
         }
@@ -414,80 +451,89 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
         break;
       }
       tc_fence_after();
-      const bool whole = (n == nch);  // no key split: normalise and store bf16
-      const int grow = it.r0 + row;
-      const float inv = 1.0f / l;
-#pragma unroll
-      for (int cb = 0; cb < kAttHD / 32; ++cb) {
-        uint32_t o[32];
-        tmem_ld32(lane_base + cb * 32, o);
-        tmem_ld_wait();
-        if (row < it.nrows) {
-          if (whole) {
-            uint4* dst = reinterpret_cast<uint4*>(Aout + (size_t)grow * d + it.h * kAttHD + cb * 32);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(pack_bf16(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv),
-                                  pack_bf16(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv),
-                                  pack_bf16(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv),
-                                  pack_bf16(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv));
-          } else {
-            float4* dst = reinterpret_cast<float4*>(sp.o_part + ((size_t)it.split * sp.part_rows + grow) * d +
-                                                    it.h * kAttHD + cb * 32);
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(__uint_as_float(o[4 * v]), __uint_as_float(o[4 * v + 1]),
-                                   __uint_as_float(o[4 * v + 2]), __uint_as_float(o[4 * v + 3]));
-          }
-        }
+      xl[hf * kAttBQ + row] = l;
+      ok = pair_exchange(&xlb[q], (uint32_t)(t & 1));
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
       }
-      if (!whole && row < it.nrows) sp.ml[((size_t)it.split * sp.part_rows + grow) * H + it.h] = make_float2(m_used, l);
+      const float l_row = xl[row] + xl[kAttBQ + row];
+      float o[64];
+#pragma unroll
+      for (int cb = 0; cb < 2; ++cb) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + hf * 64 + cb * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[cb * 32 + e] = __uint_as_float(r[e]);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(o_free);
+      const int grow = it.r0 + row;
+      if (plan.split == 2 && rank == 1) {
+        // hand (O, max, sum) of my key half to the even CTA, into its P region
+        ok = mbar_wait_cluster(xo_free, (uint32_t)(t & 1));
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        const uint32_t xo = dsmem_addr(smem_u32(sP), 0) + (uint32_t)(row * kAttHD + hf * 64) * 4;
+#pragma unroll
+        for (int v = 0; v < 16; ++v)
+          st_dsmem_v4(xo + v * 16, make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]));
+        if (hf == 0) st_dsmem_v2(dsmem_addr(smem_u32(ml), 0) + row * 8, make_float2(m_used, l_row));
+        asm volatile("fence.acq_rel.cluster;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(dsmem_addr(smem_u32(xo_full), 0));
+      } else {
+        float w_own = 1.f, inv;
+        if (plan.split == 2) {
+          // my P region is free (every P V of this unit is done): the odd CTA may write its partial
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(dsmem_addr(smem_u32(xo_free), 1));
+          ok = mbar_wait_cluster(xo_full, (uint32_t)(t & 1));
+          if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
+          }
+          const float2 pm = reinterpret_cast<const float2*>(ml)[row];  // odd CTA's (max, sum)
+          const float m = fmaxf(m_used, pm.x);
+          w_own = exp2f(m_used - m);
+          const float w_odd = exp2f(pm.x - m);
+          inv = 1.0f / (w_own * l_row + w_odd * pm.y);
+          const float* xo = reinterpret_cast<const float*>(sP) + row * kAttHD + hf * 64;
+#pragma unroll
+          for (int e = 0; e < 64; ++e) o[e] = fmaf(w_own, o[e], w_odd * xo[e]);
+          // the next unit's P may overwrite the partial once every softmax warp has read it
+          __syncwarp();
+          if (lane == 0) mbar_arrive(xo_read);
+        } else {
+          inv = 1.0f / l_row;
+        }
+        if (row < it.nrows) {
+          uint4* dst = reinterpret_cast<uint4*>(Aout + (size_t)grow * d + it.h * kAttHD + hf * 64);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[v] = make_uint4(pack_bf16(o[8 * v + 0] * inv, o[8 * v + 1] * inv),
+                                pack_bf16(o[8 * v + 2] * inv, o[8 * v + 3] * inv),
+                                pack_bf16(o[8 * v + 4] * inv, o[8 * v + 5] * inv),
+                                pack_bf16(o[8 * v + 6] * inv, o[8 * v + 7] * inv));
+        }
+      }
       g += n;
     }
     if (!ok && lane == 0) *s_abort = 1;
   }
 
   tc_fence_before();
-  __syncthreads();
+  if (plan.split == 2)
+    cluster_sync_all();  // no CTA leaves while its partner may still touch its shared memory
+  else
+    __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kAttTmemCols);
-  }
-}
-
-// out[row, h] = sum_s 2^(m_s - m) o_s / sum_s 2^(m_s - m) l_s, one CTA per active row.
-__global__ void __launch_bounds__(256) attn_combine_kernel(const int32_t* __restrict__ seg_ptr, int B, int H,
-                                                           int N, int d, AttnSplit sp,
-                                                           __nv_bfloat16* __restrict__ Aout) {
-  pdl_wait();
-  pdl_trigger();
-  const int j = blockIdx.x;
-  if (j >= seg_ptr[B]) return;
-  const int S = attn_splits(seg_ptr, B, H, N, sp.smax, sp.nsm);
-  if (S == 1) return;
-  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
-    const int h = c / kAttHD;
-    float m = -INFINITY;
-    for (int s = 0; s < S; ++s) m = fmaxf(m, sp.ml[((size_t)s * sp.part_rows + j) * H + h].x);
-    float l = 0.f, acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int s = 0; s < S; ++s) {
-      const float2 ml = sp.ml[((size_t)s * sp.part_rows + j) * H + h];
-      const float w = exp2f(ml.x - m);
-      l = fmaf(w, ml.y, l);
-      const float4 o = *reinterpret_cast<const float4*>(sp.o_part + ((size_t)s * sp.part_rows + j) * d + c);
-      acc[0] = fmaf(w, o.x, acc[0]);
-      acc[1] = fmaf(w, o.y, acc[1]);
-      acc[2] = fmaf(w, o.z, acc[2]);
-      acc[3] = fmaf(w, o.w, acc[3]);
-    }
-    const float inv = 1.0f / l;
-    uint2 u;
-    u.x = pack_bf16(acc[0] * inv, acc[1] * inv);
-    u.y = pack_bf16(acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<uint2*>(Aout + (size_t)j * d + c) = u;
   }
 }
 
@@ -527,15 +573,8 @@ __global__ void attn_f32_kernel(const float* __restrict__ Q, const float* __rest
   for (int c = 0; c < HD; ++c) A[(size_t)j * d + h * HD + c] = o[c] * inv;
 }
 
-int attn_split_rows(const plk_dims* dims, int num_sms) {
-  // keys are split only while query tiles x heads < SMs, so fewer active rows than this
-  const int rows = ceil_div(num_sms, dims->H) * kAttBQ;
-  return std::min(dims->B * dims->N, rows);
-}
-
 int launch_attention_bf16(const plk_dims* dims, const void* q, const void* K_cache, const void* V_cache,
-                          void* a_out, const int32_t* seg_ptr, float* o_part, void* ml, int smax, int part_rows,
-                          int num_sms, cudaStream_t st) {
+                          void* a_out, const int32_t* seg_ptr, int num_sms, cudaStream_t st) {
   const int B = dims->B, N = dims->N, d = dims->d, H = dims->H;
   CUtensorMap tmQ, tmK, tmV;
   if (make_tmap_bf16(&tmQ, q, (uint64_t)B * N, (uint64_t)d, kAttBQ) != PLK_OK) return PLK_ERR_CUDA;
@@ -550,13 +589,25 @@ int launch_attention_bf16(const plk_dims* dims, const void* q, const void* K_cac
     attr_done[dev] = 1;
   }
   const float scale_log2 = (float)(1.4426950408889634 / sqrt((double)dims->hd));
-  AttnSplit sp{o_part, (float2*)ml, std::max(1, std::min(smax, ceil_div(N, kAttBK))), part_rows, num_sms};
-  // persistent: one CTA per SM walks the (query tile, head, key split) items
-  const int rc = launch_pdl(attn_tc_kernel, dim3(num_sms), dim3(kAttThreads), kAttSmem, st, tmQ, tmK, tmV,
-                            (__nv_bfloat16*)a_out, seg_ptr, B, N, H, d, scale_log2, sp);
-  if (rc != PLK_OK || sp.smax == 1) return rc;
-  return launch_pdl(attn_combine_kernel, dim3(part_rows), dim3(256), 0, st, seg_ptr, B, H, N, d, sp,
-                    (__nv_bfloat16*)a_out);
+  // persistent clusters of two CTAs, one CTA per SM, over the (query tile, head) units
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(num_sms & ~1));
+  cfg.blockDim = dim3(kAttThreads);
+  cfg.dynamicSmemBytes = kAttSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 2;
+  if (cudaLaunchKernelEx(&cfg, attn_tc_kernel, tmQ, tmK, tmV, (__nv_bfloat16*)a_out, seg_ptr, B, N, H, d,
+                         scale_log2) != cudaSuccess)
+    return PLK_ERR_CUDA;
+  return PLK_OK;
 }
 
 int launch_attention_f32(const plk_dims* dims, const float* q, const float* K_cache, const float* V_cache,

@@ -63,11 +63,6 @@ Workspace workspace_layout(const plk_dims* dm, int num_sms) {
   w.hn = take(es * Mcap * d);
   w.act = take(es * Mcap * F);
   w.num_sms = num_sms;
-  if (dm->dtype == PLK_BF16) {
-    w.att_rows = attn_split_rows(dm, num_sms);
-    w.att_o = take((size_t)kAttSplitMax * w.att_rows * d * 4);
-    w.att_ml = take((size_t)kAttSplitMax * w.att_rows * dm->H * 8);
-  }
   w.c32 = take(4 * Mcap * std::max((size_t)3 * d, 2 * F));
   w.total = off;
   return w;
@@ -534,8 +529,7 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
                      (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc));
   trace_mark(3, st);
 
-  PLK_TRY(launch_attention_bf16(dm, q, Kc, Vc, a, seg, (float*)(ws + L.att_o), ws + L.att_ml, kAttSplitMax,
-                                L.att_rows, L.num_sms, st));
+  PLK_TRY(launch_attention_bf16(dm, q, Kc, Vc, a, seg, L.num_sms, st));
   trace_mark(4, st);
 
   g.K = d;

@@ -47,8 +47,6 @@ struct Workspace {
   size_t xn = 0, q = 0, a = 0, h32 = 0, hn = 0, act = 0;
   size_t c32 = 0;                        // fp32 GEMM sums [Mcap, max(3d, 2F)] (QKV, then gate/up)
   int num_sms = 0;
-  size_t att_o = 0, att_ml = 0;          // split-KV attention partials
-  int att_rows = 0;
 };
 Workspace workspace_layout(const plk_dims* d, int num_sms);
 int device_sm_count();
@@ -88,11 +86,8 @@ struct GemmArgs {
 int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const CUtensorMap& tmOut, const GemmArgs& a,
                    cudaStream_t st);
 
-constexpr int kAttSplitMax = 4;
-int attn_split_rows(const plk_dims* dims, int num_sms);
 int launch_attention_bf16(const plk_dims* dims, const void* q, const void* K_cache, const void* V_cache,
-                          void* a_out, const int32_t* seg_ptr, float* o_part, void* ml, int smax, int part_rows,
-                          int num_sms, cudaStream_t st);
+                          void* a_out, const int32_t* seg_ptr, int num_sms, cudaStream_t st);
 int launch_attention_f32(const plk_dims* dims, const float* q, const float* K_cache, const float* V_cache,
                          float* a_out, const int32_t* seg_ptr, int Mcap, cudaStream_t st);
 
