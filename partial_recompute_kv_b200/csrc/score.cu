@@ -10,9 +10,10 @@
 // distance computed straight from TMEM (thread = row) against the cached proxy.
 // The kernel streams X once from HBM; Ut stays in L2.  When there are too few
 // 128-row tiles to fill the GPU, the K dimension is split over a thread-block
-// cluster of S CTAs: each CTA parks its partial projection in its own shared
-// memory and then finishes 128/S of the rows, summing the S partials through
-// distributed shared memory (no global scratch).
+// cluster of S CTAs: each CTA pushes the row slices of its partial projection
+// into the shared memory of the CTA that finishes those rows (distributed
+// shared memory stores), and after one cluster barrier every CTA sums its S
+// slices locally (no global scratch, no remote loads).
 // fp32: a SIMT kernel, one warp per row.
 #include "plk_common.cuh"
 #include "plk_internal.h"
@@ -20,8 +21,17 @@
 namespace plk {
 
 namespace {
-constexpr int kScStages = 3;
+constexpr int kScStagesMax = 6;
 constexpr int kScA = 128 * 64 * 2;  // 16 KB of X per stage
+constexpr int kScRingBudget = 200 * 1024;
+
+// Ring depth for proxy rank r: as many (X, U) stages as fit 200 KB, 2..6.  The
+// X loads are HBM-latency bound, so the more stages in flight the better.
+__host__ __device__ inline int sc_stages(int r) {
+  const int stage_bytes = kScA + ((r * 128 + 1023) & ~1023);
+  const int n = kScRingBudget / stage_bytes;
+  return n < 2 ? 2 : (n > kScStagesMax ? kScStagesMax : n);
+}
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
@@ -43,12 +53,13 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   const int stageB = r * 128;
   const int stage_bytes = kScA + ((stageB + 1023) & ~1023);
+  const int kScStages = sc_stages(r);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kScStages * stage_bytes);
   uint64_t* full = bars;
-  uint64_t* empty = bars + kScStages;
-  uint64_t* done = bars + 2 * kScStages;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * kScStages + 1);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 2 * kScStages + 2);
+  uint64_t* empty = bars + kScStagesMax;
+  uint64_t* done = bars + 2 * kScStagesMax;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * kScStagesMax + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 2 * kScStagesMax + 2);
 
   pdl_wait();
   pdl_trigger();
@@ -134,10 +145,14 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
   const bool ok = mbar_wait(done, 0);
   tc_fence_after();
   if (S > 1) {
-    // split-K over the cluster: partial [128 rows][r] (stride r+1) in the idle stage buffers
-    float* part = reinterpret_cast<float*>(smem);
-    const int pstride = r + 1;
+    // split-K over the cluster: every CTA pushes the row slices of its partial projection to
+    // the CTA that finishes those rows (distributed shared memory stores, nothing waits on a
+    // round trip); the receiver's idle stage buffers hold slots [sender][rows_per][r]
+    const int rows_per = 128 / S, tpr = 128 / rows_per;
+    float* slots = reinterpret_cast<float*>(smem);
     const int rl = warp * 32 + lane;
+    const uint32_t dst = dsmem_addr(smem_u32(slots + ((size_t)ks * rows_per + rl % rows_per) * r),
+                                    (uint32_t)(rl / rows_per));
     const bool good = __all_sync(0xffffffffu, ok && !*s_abort);
     for (int c0 = 0; c0 < r; c0 += 16) {
       uint32_t v[16];
@@ -146,31 +161,38 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
         tmem_ld_wait();
       }
 #pragma unroll
-      for (int i = 0; i < 16; ++i) part[rl * pstride + c0 + i] = good ? __uint_as_float(v[i]) : 0.f;
+      for (int u = 0; u < 4; ++u)
+        st_dsmem_f32x4(dst + 4u * (c0 + 4 * u),
+                       good ? make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
+                                          __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3]))
+                            : make_float4(0.f, 0.f, 0.f, 0.f));
     }
     tc_fence_before();
-    cluster_sync_all();
-    const int rows_per = 128 / S, tpr = 128 / rows_per;
-    const int lrow = ks * rows_per + (int)threadIdx.x / tpr, sub = (int)threadIdx.x % tpr;
-    const int row = row0 + lrow;
-    const uint32_t pbase = smem_u32(part + lrow * pstride);
+    cluster_sync_all();  // every slice has landed; nobody touches another CTA's memory after this
+    const int lrow = (int)threadIdx.x / tpr, sub = (int)threadIdx.x % tpr;
+    const int row = row0 + ks * rows_per + lrow;
     float dot = 0.f, pp = 0.f, cc = 0.f, dd = 0.f;
-    for (int c = sub; c < r; c += tpr) {
-      float pk[8];  // the S loads of this column in flight before the sum
-#pragma unroll
-      for (int sr = 0; sr < 8; ++sr)
-        if (sr < S) pk[sr] = ld_dsmem_f32(dsmem_addr(pbase + 4u * c, (uint32_t)sr));
-      float p = 0.f;
-#pragma unroll
-      for (int sr = 0; sr < 8; ++sr)
-        if (sr < S) p += pk[sr];
+    for (int c = sub * 4; c < r; c += 4 * tpr) {
+      float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int sr = 0; sr < S; ++sr) {
+        const float4 x = *reinterpret_cast<const float4*>(slots + ((size_t)sr * rows_per + lrow) * r + c);
+        p.x += x.x;
+        p.y += x.y;
+        p.z += x.z;
+        p.w += x.w;
+      }
       if (row < rows) {
-        const float cv = __ldg(cache + (size_t)row * r + c);
-        dot = fmaf(p, cv, dot);
-        pp = fmaf(p, p, pp);
-        cc = fmaf(cv, cv, cc);
-        dd = fmaf(p - cv, p - cv, dd);
-        if (pout) pout[(size_t)row * r + c] = p;
+        const float4 cv = __ldg(reinterpret_cast<const float4*>(cache + (size_t)row * r + c));
+        const float pv[4] = {p.x, p.y, p.z, p.w};
+        const float cvv[4] = {cv.x, cv.y, cv.z, cv.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          dot = fmaf(pv[e], cvv[e], dot);
+          pp = fmaf(pv[e], pv[e], pp);
+          cc = fmaf(cvv[e], cvv[e], cc);
+          dd = fmaf(pv[e] - cvv[e], pv[e] - cvv[e], dd);
+        }
+        if (pout) *reinterpret_cast<float4*>(pout + (size_t)row * r + c) = p;
       }
     }
     for (int o = 1; o < tpr; o <<= 1) {
@@ -181,7 +203,6 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
     }
     if (sub == 0 && row < rows)
       score[row] = metric == PLK_METRIC_COS ? dot / fmaxf(sqrtf(pp) * sqrtf(cc), 1e-30f) : sqrtf(dd);
-    cluster_sync_all();  // peers may still be reading this CTA's partial
     if (warp == 2) {
       tc_fence_after();
       tmem_dealloc(tmem, (uint32_t)tmem_cols);
@@ -275,7 +296,7 @@ __global__ void proxy_commit_kernel(const int32_t* __restrict__ idx, const int32
 
 static int score_tc_smem(int r) {
   const int stage_bytes = kScA + ((r * 128 + 1023) & ~1023);
-  return kScStages * stage_bytes + 128 + 1024;
+  return sc_stages(r) * stage_bytes + 128 + 1024;
 }
 
 int launch_score(const plk_dims* dims, const void* X, const void* Ut, int r, const float* proxy_cache,
