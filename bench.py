@@ -331,13 +331,32 @@ def run_gpu(args, wl, dist, rank, world, local_rank):
     if dist is not None:
         dist.barrier(device_ids=[local_rank])
     torch.cuda.synchronize()
+    graph = None
+    if args.graph:
+        # the whole step (score, select, layer step, commit) as one CUDA graph: every call is
+        # capture-safe (no allocation, no host synchronisation, launch attributes kept)
+        graph = torch.cuda.CUDAGraph()
+        prep()
+        with torch.cuda.graph(graph):
+            step(Xp)
+        torch.cuda.synchronize()
+        for _ in range(3):
+            prep()
+            graph.replay()
+        torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
+        h0 = time.perf_counter()
         for i in range(K_):
             prep()
             ev[i][0].record()
-            step(Xp)
+            if graph is not None:
+                graph.replay()
+            else:
+                step(Xp)
             ev[i][1].record()
+        h1 = time.perf_counter()
         torch.cuda.synchronize()
+    host_us = (h1 - h0) / K_ * 1e6
     if dist is not None:
         dist.barrier(device_ids=[local_rank])
     st = plk.get_status()
@@ -405,6 +424,7 @@ def run_gpu(args, wl, dist, rank, world, local_rank):
            "d2h_bytes_per_step": Y_host.numel() * Y_host.element_size(), "ms_per_step": e2e_ms}
     step_flops = M * wl.flops_per_row()
     return {"value": value, "ms_per_step": ms_per_step, "per_kernel_us": per, "roofline": roofline,
+            "host_enqueue_us_per_step": host_us,
             "e2e": e2e, "clocks": clk.summary(), "step_tflops": step_flops / (ms_per_step * 1e-3) / 1e12,
             "peaks": pk}
 
@@ -418,6 +438,10 @@ def main():
     ap.add_argument("--l2", choices=["stream", "flush"], default="stream",
                     help="stream: no flush between steps (the weights alone are 3.4x L2); "
                          "flush: write 256 MiB before every step")
+    ap.add_argument("--graph", dest="graph", action="store_true", default=True,
+                    help="replay the step as one captured CUDA graph (default)")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="enqueue the step's library calls directly every step")
     ap.add_argument("--profile", action="store_true",
                     help="set up and run --steps steps without timing or output (for ncu)")
     args = ap.parse_args()
@@ -457,7 +481,8 @@ def main():
             "roofline": res["roofline"],
             "step_tflops": res["step_tflops"],
             "step_frac_of_bf16_peak": res["step_tflops"] / float(res["peaks"]["bf16_tflops"]),
-            "per_kernel_us": res["per_kernel_us"],
+            "per_kernel_us": res["per_kernel_us"], "host_enqueue_us_per_step": res["host_enqueue_us_per_step"],
+            "launch": "cuda graph" if args.graph else "stream",
             "e2e": res["e2e"], "gpu_launches": launches_per_step * args.steps, "clocks": res["clocks"]}
     if world == 1:
         line["cpu_baseline"] = cpu_baseline(wl)

@@ -10,10 +10,11 @@
 // distance computed straight from TMEM (thread = row) against the cached proxy.
 // The kernel streams X once from HBM; Ut stays in L2.  When there are too few
 // 128-row tiles to fill the GPU, the K dimension is split over a thread-block
-// cluster of S CTAs: each CTA pushes the row slices of its partial projection
-// into the shared memory of the CTA that finishes those rows (distributed
-// shared memory stores), and after one cluster barrier every CTA sums its S
-// slices locally (no global scratch, no remote loads).
+// cluster of S CTAs: once every CTA's loads and MMAs are done (a cluster
+// barrier), each CTA pushes the row slices of its partial projection into the
+// idle stage buffers of the CTA that finishes those rows (distributed shared
+// memory stores), and after a second barrier every CTA sums its S slices
+// locally (no global scratch, no remote loads).
 // fp32: a SIMT kernel, one warp per row.
 #include "plk_common.cuh"
 #include "plk_internal.h"
@@ -154,6 +155,8 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
     const uint32_t dst = dsmem_addr(smem_u32(slots + ((size_t)ks * rows_per + rl % rows_per) * r),
                                     (uint32_t)(rl / rows_per));
     const bool good = __all_sync(0xffffffffu, ok && !*s_abort);
+    // the receivers' stage buffers must be idle: every CTA's loads and MMAs are done
+    cluster_sync_all();
     for (int c0 = 0; c0 < r; c0 += 16) {
       uint32_t v[16];
       if (good) {

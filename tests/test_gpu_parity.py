@@ -136,6 +136,29 @@ def test_score_drift(plk, dtype, metric):
     assert_f32_close(host(score), ref_s, "score", tol=1e-4)
 
 
+def test_score_drift_8b_shape_repeated(plk):
+    """The scoring launch the benchmark times (1024 rows x 4096, rank 128, K split over a
+    cluster of 8 CTAs), run several times on the same inputs: every run must match."""
+    D = synth.Dims(B=1, N=1024, d=4096, H=32, hd=128, F=12288, dtype="bf16")
+    r = 128
+    X = synth.hidden_states(D, seed=5)
+    Ut = synth.proxy_basis(D.d, r, seed=5, dtype="bf16")
+    p_exact = oracle.proxy_project(X.reshape(-1, D.d).astype(np.float64), Ut.astype(np.float64))
+    rng = np.random.default_rng(5)
+    pc = (p_exact + (rng.random(D.N) < 0.25)[:, None] * rng.standard_normal(p_exact.shape) * 0.5)
+    pc = pc.astype(np.float32).reshape(D.B, D.N, r)
+    ref_s, ref_p = oracle.score_drift(X.astype(np.float64), Ut.astype(np.float64), pc, "l2")
+    dm = pdims(plk, D)
+    Xd, Ud, pcd = dev(X, torch.bfloat16), dev(Ut, torch.bfloat16), dev(pc, torch.float32)
+    for run in range(6):
+        score = torch.full((D.B, D.N), float("nan"), dtype=torch.float32, device="cuda")
+        pout = torch.full((D.B, D.N, r), float("nan"), dtype=torch.float32, device="cuda")
+        plk.score_drift(dm, Xd, Ud, r, pcd, plk.METRIC_L2, score, proxy_out=pout)
+        torch.cuda.synchronize()
+        assert_f32_close(host(pout), ref_p, f"proxy, run {run}", tol=1e-5)
+        assert_f32_close(host(score), ref_s, f"score, run {run}", tol=1e-4)
+
+
 def test_proxy_commit(plk):
     B, N, r = 3, 50, 16
     rng = np.random.default_rng(4)
