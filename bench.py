@@ -401,7 +401,19 @@ def run_gpu(args, wl, dist, rank, world, local_rank):
     traffic = gemm_traffic_per_launch()
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic, "kernel": "gemm_tc_kernel",
-                "launches_per_step": 4, "peak_source": f"{pk.get('source')} bf16_tflops (burst)"}
+                "launches_per_step": 4, "peak_source": f"{pk.get('source')} bf16_tflops (burst)",
+                "frac_of_sustained": achieved / float(pk.get("bf16_tflops_sustained", peak))}
+
+    # the memory-bound kernels: algorithmic bytes / traced time against the measured HBM copy rate
+    d_, F_, r_, BN = D.d, D.F, r, D.B * D.N
+    alg_bytes = {"score": 2 * BN * d_ + 8 * BN * r_ + 2 * d_ * r_,
+                 "select": 6 * BN + 4 * M,
+                 "rmsnorm1": 20 * M * d_, "finish_qkv": 18 * M * d_,
+                 "rmsnorm2": 6 * M * d_ + 8 * M * F_, "finish_gu": 10 * M * F_,
+                 "finish_y": 6 * M * d_, "proxy_commit": 8 * M * r_}
+    hbm = float(pk["hbm_gbs"])
+    hbm_kernels = {k: {"bytes": v, "GB/s": v / (per[k] * 1e-6) / 1e9, "frac": v / (per[k] * 1e-6) / 1e9 / hbm}
+                   for k, v in alg_bytes.items()}
 
     # e2e through the public API: H2D of the step's input, the step, D2H of the output cache
     e2e_steps = min(K_, 50)
@@ -424,7 +436,8 @@ def run_gpu(args, wl, dist, rank, world, local_rank):
            "d2h_bytes_per_step": Y_host.numel() * Y_host.element_size(), "ms_per_step": e2e_ms}
     step_flops = M * wl.flops_per_row()
     return {"value": value, "ms_per_step": ms_per_step, "per_kernel_us": per, "roofline": roofline,
-            "host_enqueue_us_per_step": host_us,
+            "host_enqueue_us_per_step": host_us, "hbm_kernels": hbm_kernels,
+            "ms_per_step_median": statistics.median(step_ms),
             "e2e": e2e, "clocks": clk.summary(), "step_tflops": step_flops / (ms_per_step * 1e-3) / 1e12,
             "peaks": pk}
 
@@ -482,6 +495,7 @@ def main():
             "step_tflops": res["step_tflops"],
             "step_frac_of_bf16_peak": res["step_tflops"] / float(res["peaks"]["bf16_tflops"]),
             "per_kernel_us": res["per_kernel_us"], "host_enqueue_us_per_step": res["host_enqueue_us_per_step"],
+            "ms_per_step_median": res["ms_per_step_median"], "hbm_kernels": res["hbm_kernels"],
             "launch": "cuda graph" if args.graph else "stream",
             "e2e": res["e2e"], "gpu_launches": launches_per_step * args.steps, "clocks": res["clocks"]}
     if world == 1:
