@@ -37,6 +37,12 @@ R5  Threshold rule: lock when score > tau (or < tau), strictly; a NaN score
     never locks.  Budget rule: keep the k rows with the largest (or smallest)
     score among the rows not yet locked; equal scores go to the lower index;
     NaN is never preferred; +0 and -0 are equal.  Rows not kept are locked.
+R7  KL lock ([SL] Sec. 2 "Locking Condition"): p_t = softmax over the
+    vocabulary of a position's logits at step t; a still-active position
+    locks when KL(p_t || p_{t-1}) <= eps (inclusive).  The optional
+    "confidence gate" (low entropy) is read as H(p_t) <= h_max in nats; with
+    h_max = +inf the gate is off.  The caller supplies the logits of both
+    steps; rows already locked are not examined and stay locked.
 R6  Precision policy "bf16": every tensor that the bf16 path stores in bf16
     between operations is rounded to bf16 here as well -- the normalised
     inputs of the projections (xn, hn), q, k, v (and so the K/V cache), the
@@ -58,7 +64,7 @@ import numpy as np
 __all__ = [
     "to_bf16", "to_f32", "count_flops", "rmsnorm", "silu",
     "proxy_project", "drift_cosine", "drift_l2", "score_drift",
-    "lock_threshold", "lock_topk", "compact",
+    "lock_threshold", "lock_topk", "compact", "log_softmax", "kl_divergence", "entropy", "kl_lock",
     "full_layer_step", "layer_step_partial", "proxy_commit",
     "LayerState", "tiny_run",
 ]
@@ -230,6 +236,48 @@ def lock_topk(score, lock_in, k, largest=True):
         for i in sorted(cand, key=key)[: max(int(k), 0)]:
             out[b, i] = 0
     return out
+
+
+def log_softmax(z):
+    """log p_v = z_v - log sum_w exp(z_w) along the last axis (max-shifted, float64)."""
+    z = np.asarray(z, dtype=np.float64)
+    m = np.max(z, axis=-1, keepdims=True)
+    return z - (m + np.log(np.sum(np.exp(z - m), axis=-1, keepdims=True)))
+
+
+def kl_divergence(z_t, z_prev):
+    """KL(p_t || p_prev) = sum_v p_t,v (log p_t,v - log p_prev,v), p = softmax of the logits."""
+    lt, lp = log_softmax(z_t), log_softmax(z_prev)
+    return np.sum(np.exp(lt) * (lt - lp), axis=-1)
+
+
+def entropy(z):
+    """H(p) = -sum_v p_v log p_v in nats, p = softmax of the logits."""
+    lt = log_softmax(z)
+    return -np.sum(np.exp(lt) * lt, axis=-1)
+
+
+def kl_lock(logits_t, logits_prev, lock_in, eps, h_max=math.inf):
+    """SureLock locking condition ([SL] Sec. 2 "Locking Condition", R7).
+
+    A row with lock_in = 0 locks when KL(p_t || p_{t-1}) <= eps and, with the
+    confidence gate on, H(p_t) <= h_max.  Locked rows stay locked and are not
+    examined.  Returns (lock_out [B, N] u8, kl [B, N], H [B, N]) with NaN in kl
+    and H at rows that were already locked.
+    """
+    lk = np.asarray(lock_in).astype(bool)
+    B, N = lk.shape
+    kl = np.full((B, N), np.nan)
+    ent = np.full((B, N), np.nan)
+    out = lk.copy()
+    for b in range(B):
+        for i in range(N):
+            if lk[b, i]:
+                continue
+            kl[b, i] = kl_divergence(logits_t[b, i], logits_prev[b, i])
+            ent[b, i] = entropy(logits_t[b, i])
+            out[b, i] = kl[b, i] <= eps and ent[b, i] <= h_max
+    return out.astype(np.uint8), kl, ent
 
 
 # ---------------------------------------------------------------------------

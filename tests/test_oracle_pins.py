@@ -429,3 +429,86 @@ def test_partial_step_mutants_are_caught(old, new):
         assert err < 1e-12  # subtracting any constant leaves softmax unchanged
     else:
         assert err > 1e-6
+
+
+# ---------------------------------------------------------------------------
+# KL lock rule (SureLock "Locking Condition": KL(p_t || p_{t-1}) <= eps, optional low-entropy gate)
+# ---------------------------------------------------------------------------
+def _sigmoid(a):
+    return 1.0 / (1.0 + math.exp(-a))
+
+
+def test_log_softmax_matches_torch():
+    z = np.random.default_rng(30).standard_normal((5, 7, 33)) * 4.0
+    ref = Fnn.log_softmax(torch.from_numpy(z), dim=-1).numpy()
+    np.testing.assert_allclose(oracle.log_softmax(z), ref, rtol=0, atol=1e-12)
+
+
+def test_kl_matches_torch_kl_div_in_the_stated_direction():
+    rng = np.random.default_rng(31)
+    zt, zp = rng.standard_normal((6, 40)) * 3, rng.standard_normal((6, 40)) * 3
+    lt = torch.from_numpy(oracle.log_softmax(zt))
+    lp = torch.from_numpy(oracle.log_softmax(zp))
+    # torch: kl_div(input = log q, target = log p, log_target) = sum p (log p - log q) = KL(p || q)
+    ref = Fnn.kl_div(lp, lt, reduction="none", log_target=True).sum(-1).numpy()
+    np.testing.assert_allclose(oracle.kl_divergence(zt, zp), ref, rtol=1e-12, atol=1e-14)
+    # the reverse direction differs: a swapped argument order would fail the line above
+    assert np.max(np.abs(oracle.kl_divergence(zp, zt) - ref)) > 1e-3
+
+
+@pytest.mark.parametrize("a,b", [(0.3, -1.2), (2.0, 2.5), (-4.0, 1.0)])
+def test_kl_and_entropy_two_point_closed_form(a, b):
+    p, q = _sigmoid(a), _sigmoid(b)
+    kl = p * math.log(p / q) + (1 - p) * math.log((1 - p) / (1 - q))
+    h = -p * math.log(p) - (1 - p) * math.log(1 - p)
+    assert abs(oracle.kl_divergence(np.array([a, 0.0]), np.array([b, 0.0])) - kl) < 1e-14
+    assert abs(oracle.entropy(np.array([a, 0.0])) - h) < 1e-14
+
+
+def test_kl_invariants():
+    rng = np.random.default_rng(32)
+    z = rng.standard_normal((50, 64)) * 2
+    assert np.max(np.abs(oracle.kl_divergence(z, z))) < 1e-14
+    assert np.max(np.abs(oracle.kl_divergence(z + 7.5, z))) < 1e-12  # softmax ignores a shift
+    zp = z + rng.standard_normal(z.shape) * 0.3
+    assert np.all(oracle.kl_divergence(z, zp) > 0)  # Gibbs' inequality
+    np.testing.assert_allclose(oracle.entropy(np.zeros((3, 64))), math.log(64), rtol=1e-14)
+    spike = np.zeros(64)
+    spike[5] = 1000.0
+    assert oracle.entropy(spike) < 1e-12
+
+
+def test_kl_brute_force_tiny():
+    rng = np.random.default_rng(33)
+    zt, zp = rng.standard_normal(9), rng.standard_normal(9)
+    et, ep = [math.exp(x) for x in zt], [math.exp(x) for x in zp]
+    st, sp = sum(et), sum(ep)
+    kl = sum((et[v] / st) * math.log((et[v] / st) / (ep[v] / sp)) for v in range(9))
+    h = -sum((et[v] / st) * math.log(et[v] / st) for v in range(9))
+    assert abs(oracle.kl_divergence(zt, zp) - kl) < 1e-14
+    assert abs(oracle.entropy(zt) - h) < 1e-14
+
+
+def test_kl_lock_semantics():
+    rng = np.random.default_rng(34)
+    B, N, V = 2, 6, 16
+    zp = rng.standard_normal((B, N, V))
+    zt = zp + rng.standard_normal((B, N, V)) * np.linspace(0.0, 0.5, N)[None, :, None]
+    lock_in = np.zeros((B, N), np.uint8)
+    lock_in[1, 2] = 1
+    kl = oracle.kl_divergence(zt, zp)
+    eps = float(np.median(kl))
+    out, klo, ho = oracle.kl_lock(zt, zp, lock_in, eps)
+    assert out[1, 2] == 1 and np.isnan(klo[1, 2]) and np.isnan(ho[1, 2])  # permanent, not examined
+    act = lock_in == 0
+    np.testing.assert_array_equal(out[act], (kl[act] <= eps).astype(np.uint8))
+    # inclusive threshold: eps equal to a row's KL locks it
+    j = np.argmax(np.where(act, kl, -1))
+    out2, _, _ = oracle.kl_lock(zt, zp, lock_in, float(kl.flat[j]))
+    assert out2.flat[j] == 1
+    # the gate can only keep rows active; h_max = +inf is "off"
+    h = oracle.entropy(zt)
+    hm = float(np.median(h[act]))
+    out3, _, _ = oracle.kl_lock(zt, zp, lock_in, eps, hm)
+    np.testing.assert_array_equal(out3[act], ((kl[act] <= eps) & (h[act] <= hm)).astype(np.uint8))
+    assert np.all(out3 <= out)
