@@ -163,6 +163,23 @@ int plk_full_layer_step(const plk_dims* dims, const plk_weights* w, const void* 
                         void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * S2' SureLock's locking condition on logits ([SL] Sec. 2 "Locking
+ * Condition"): for every row i with lock_in[i] == 0,
+ *   KL_i = KL(p_t || p_{t-1}),  p = softmax over the V vocabulary logits,
+ *   H_i  = entropy of p_t in nats (the optional "confidence gate"),
+ *   lock_out[i] = (KL_i <= eps && H_i <= h_max)   (h_max = +INFINITY: gate off).
+ * Rows with lock_in[i] == 1 are not read and get lock_out[i] = 1.
+ * logits_t, logits_prev: [B, N, V] in the layer dtype (dims->dtype), row-major,
+ * the logits of the current and the previous step.  kl_out, h_out: [B, N] fp32
+ * or NULL; written only at examined rows.  lock_in and lock_out may alias.
+ * Only dims->B, dims->N and dims->dtype are used.  Errors: PLK_ERR_ARG for a
+ * NULL input, V < 1 or a NaN eps / h_max; PLK_ERR_SHAPE for B*N >= 2^31.
+ */
+int plk_kl_lock(const plk_dims* dims, int V, const void* logits_t, const void* logits_prev,
+                const uint8_t* lock_in, uint8_t* lock_out, float eps, float h_max,
+                float* kl_out, float* h_out, void* stream);
+
+/*
  * S10 (proxy half)  proxy_cache[idx[j]] = proxy_new[idx[j]] for j < M = seg_ptr[B].
  * Both [B, N, r] fp32; rows not in idx are untouched.
  */

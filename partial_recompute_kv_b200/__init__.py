@@ -10,6 +10,7 @@ The C contract of every call is documented in include/plk.h.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 
 import torch
@@ -24,7 +25,7 @@ SEL_THRESH_GT, SEL_THRESH_LT, SEL_TOPK_LARGEST, SEL_TOPK_SMALLEST = 0, 1, 2, 3
 
 EXPORTED = (
     "plk_score_drift", "plk_select_active", "plk_layer_step_partial", "plk_full_layer_step",
-    "plk_proxy_commit", "plk_layer_step_partial_static", "plk_workspace_bytes", "plk_get_status",
+    "plk_proxy_commit", "plk_layer_step_partial_static", "plk_kl_lock", "plk_workspace_bytes", "plk_get_status",
     "plk_set_wait_limit",
     "plk_selftest_wait_timeout", "plk_trace_events", "plk_error_string", "plk_version",
 )
@@ -60,6 +61,7 @@ def _load():
         "plk_full_layer_step": (I, [V, W, P, P, P, P, P, S, P]),
         "plk_layer_step_partial_static": (I, [V, W, P, P, P, P, P, P, P]),
         "plk_proxy_commit": (I, [V, I, P, P, P, P, P]),
+        "plk_kl_lock": (I, [V, I, P, P, P, P, F, F, P, P, P]),
         "plk_workspace_bytes": (S, [V]),
         "plk_get_status": (I, [P]),
         "plk_set_wait_limit": (I, [L]),
@@ -177,6 +179,14 @@ def full_layer_step(dm, w, X, K_cache, V_cache, Y, workspace, stream=None):
 def proxy_commit(dm, r, idx, seg_ptr, proxy_new, proxy_cache, stream=None):
     _check(lib.plk_proxy_commit(ctypes.byref(dm), int(r), _ptr(idx), _ptr(seg_ptr), _ptr(proxy_new),
                                 _ptr(proxy_cache), _stream(stream)), "proxy_commit")
+
+
+def kl_lock(dm, V, logits_t, logits_prev, lock_in, lock_out, eps, h_max=math.inf, kl_out=None, h_out=None,
+            stream=None):
+    opt = lambda t: None if t is None else _ptr(t)
+    _check(lib.plk_kl_lock(ctypes.byref(dm), int(V), _ptr(logits_t), _ptr(logits_prev), _ptr(lock_in),
+                           _ptr(lock_out), float(eps), float(h_max), opt(kl_out), opt(h_out), _stream(stream)),
+           "kl_lock")
 
 
 def get_status(stream=None) -> int:

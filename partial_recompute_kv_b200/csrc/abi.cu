@@ -74,6 +74,17 @@ int plk_select_active(const plk_dims* dims, const float* score, const uint8_t* l
   return launch_select(dims, score, lock_in, lock_out, mode, tau, k, idx_out, seg_ptr, (cudaStream_t)stream);
 }
 
+int plk_kl_lock(const plk_dims* dims, int V, const void* logits_t, const void* logits_prev, const uint8_t* lock_in,
+                uint8_t* lock_out, float eps, float h_max, float* kl_out, float* h_out, void* stream) {
+  if (!dims) return PLK_ERR_ARG;
+  if (dims->dtype != PLK_F32 && dims->dtype != PLK_BF16) return PLK_ERR_DTYPE;
+  if (dims->B < 1 || dims->N < 1 || (long long)dims->B * dims->N >= (1LL << 31)) return PLK_ERR_SHAPE;
+  if (V < 1 || !logits_t || !logits_prev || !lock_in || !lock_out) return PLK_ERR_ARG;
+  if (eps != eps || h_max != h_max) return PLK_ERR_ARG;
+  return launch_kl_lock(dims, V, logits_t, logits_prev, lock_in, lock_out, eps, h_max, kl_out, h_out,
+                        (cudaStream_t)stream);
+}
+
 int plk_layer_step_partial(const plk_dims* dims, const plk_weights* w, const void* X, const int32_t* idx,
                            const int32_t* seg_ptr, void* K_cache, void* V_cache, void* Y, void* workspace,
                            size_t ws_bytes, void* stream) {

@@ -7,3 +7,4 @@
 #include "attention.cu"
 #include "abi.cu"
 #include "static_ws.cu"
+#include "kl_lock.cu"

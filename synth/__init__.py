@@ -28,6 +28,7 @@ S_MASK = 3
 S_NOISE = 4
 S_POS = 5
 S_PROXY = 6
+S_LOGITS = 7
 
 
 def round_bf16(a) -> np.ndarray:
@@ -169,6 +170,24 @@ def linear_schedule(N: int, steps: int = 256) -> np.ndarray:
 # ---------------------------------------------------------------------------
 # Named workloads (shapes and distributions of the pages' experiments)
 # ---------------------------------------------------------------------------
+def logits_pair(B: int, N: int, V: int, seed: int = 0, std: float = 2.0, drift=(0.0, 0.3),
+                dtype: str = "f32"):
+    """Two steps of vocabulary logits [B, N, V]: z_prev ~ N(0, std^2) per entry, and
+    z_t = z_prev + N(0, s_i^2) with s_i spread uniformly over `drift` across rows, so that
+    some rows barely move and others change a lot.  Rounded to bf16 for "bf16"."""
+    rng = _rng(seed, S_LOGITS)
+    zp = rng.standard_normal((B, N, V)).astype(np.float32) * np.float32(std)
+    s = np.linspace(drift[0], drift[1], B * N, dtype=np.float32).reshape(B, N, 1)
+    zt = zp + rng.standard_normal((B, N, V)).astype(np.float32) * s
+    if dtype == "bf16":
+        return round_bf16(zt), round_bf16(zp)
+    return zt, zp
+
+
+# vocabulary size of the 8B model the pages name, for the KL-lock measurement
+VOCAB_8B = 126464
+
+
 TINY = Dims(B=1, N=64, d=64, H=4, hd=16, F=256, eps=1e-6, dtype="f32")
 LAYER_8B = Dims(B=1, N=1024, d=4096, H=32, hd=128, F=12288, eps=1e-6, dtype="bf16")
 STACK_8B = Dims(B=4, N=2048, d=4096, H=32, hd=128, F=12288, eps=1e-6, dtype="bf16")
