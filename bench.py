@@ -442,6 +442,67 @@ def run_gpu(args, wl, dist, rank, world, local_rank):
             "peaks": pk}
 
 
+# ---------------------------------------------------------------------------
+# the KL lock rule (SureLock's locking condition) on its own: not part of the
+# headline step, measured with --kernel kl_lock
+# ---------------------------------------------------------------------------
+def run_kl_lock(args):
+    import torch
+    import partial_recompute_kv_b200 as plk
+    import oracle
+    import synth
+
+    B, N, V, M = 1, 1024, synth.VOCAB_8B, 256
+    dev = torch.device("cuda", 0)
+    zt, zp = synth.logits_pair(B, N, V, seed=0, drift=(0.0, 0.3), dtype="bf16")
+    lock0 = np.ones((B, N), np.uint8)
+    lock0[0, synth.layer_8b_positions(N, M / N)] = 0
+    bf = torch.bfloat16
+    Zt = torch.from_numpy(zt).to(dev).to(bf)
+    Zp = torch.from_numpy(zp).to(dev).to(bf)
+    lk0 = torch.from_numpy(lock0).to(dev)
+    lk = torch.empty_like(lk0)
+    kl = torch.empty((B, N), dtype=torch.float32, device=dev)
+    dm = plk.dims(B, N, 256, 2, 128, 512, dtype=plk.BF16)
+    eps = 1e-3
+    call = lambda: plk.kl_lock(dm, V, Zt, Zp, lk0, lk, eps, math.inf, kl_out=kl)
+    for _ in range(max(args.warmup, 3)):
+        call()
+    torch.cuda.synchronize()
+    E = lambda: torch.cuda.Event(enable_timing=True)
+    ev = [(E(), E()) for _ in range(args.steps)]
+    with ClockSampler(0) as clk:
+        for a, b in ev:
+            a.record()
+            call()
+            b.record()
+        torch.cuda.synchronize()
+    st = plk.get_status()
+    if st != plk.OK:
+        raise RuntimeError(f"device status {plk.error_string(st)}")
+    us = statistics.mean(a.elapsed_time(b) for a, b in ev) * 1e3
+    pk = peaks()
+    alg = 2 * M * V * 2  # both steps' bf16 logits of the active rows, read once
+    gbs = alg / (us * 1e-6) / 1e9
+    # cpu baseline: the oracle on 8 of the active rows
+    rows = np.flatnonzero(lock0[0] == 0)[:8]
+    t0 = time.perf_counter()
+    oracle.kl_lock(zt[:, rows], zp[:, rows], np.zeros((1, rows.size), np.uint8), eps)
+    cpu_s = time.perf_counter() - t0
+    line = {"metric": "KL-lock rows/s (8B vocabulary, bf16 logits)", "value": M / (us * 1e-6),
+            "unit": "rows/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "us_per_call": us,
+            "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"kl_lock, B={B}, N={N}, V={V}, {M} active rows, eps={eps}, gate off"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": float(pk["hbm_gbs"]), "unit": "GB/s",
+                         "frac": gbs / float(pk["hbm_gbs"]), "traffic": None,
+                         "kernel": "kl_lock_kernel", "alg_bytes_per_call": alg},
+            "clocks": clk.summary(),
+            "cpu_baseline": {"value": rows.size / cpu_s, "unit": "rows/s", "cores": os.cpu_count(),
+                             "kind": "oracle", "sample": f"{rows.size} active rows of the same workload"}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -455,6 +516,8 @@ def main():
                     help="replay the step as one captured CUDA graph (default)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="enqueue the step's library calls directly every step")
+    ap.add_argument("--kernel", choices=["step", "kl_lock"], default="step",
+                    help="step: the headline layer step; kl_lock: the KL lock rule alone")
     ap.add_argument("--profile", action="store_true",
                     help="set up and run --steps steps without timing or output (for ncu)")
     args = ap.parse_args()
@@ -463,6 +526,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.kernel == "kl_lock":
+        return run_kl_lock(args) if rank == 0 else 0
     if args.impl == "reference":
         if rank != 0:
             return 0
