@@ -16,8 +16,11 @@
 // cancellation of two large log-sum-exps, which keeps the small KL values near a
 // locking threshold accurate in fp32; when some z_t is so far above max z_p that
 // the u form would overflow, the plain difference of log-sum-exps is used.
-// Three exp2 per element put the kernel on the MUFU pipe at about the same
-// time as the HBM stream of the two logit rows.
+// Two exp2 per element (ex2.approx; the third factor 2^(m_t - m_p) is one per
+// chunk) keep the MUFU pipe near the time of the HBM stream of the two rows.
+// Measured alternatives: a 4-CTA cluster per row and a shared-memory ring of
+// bulk copies were both slower (the row's dependent instruction stream, not the
+// memory system, sets the pace).
 #include <math.h>
 
 #include "plk_common.cuh"
@@ -37,6 +40,13 @@ struct KlAcc {
   float mp, sp, u;     // previous step: max y_p, sums
   int far;             // some y_t - m_p > kKlFar
 };
+
+// 2^x on the MUFU pipe (PTX ex2.approx: ~2 ulp, flushes results below 2^-126 to 0)
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __device__ __forceinline__ void kl_init(KlAcc& c) {
   c.mt = -INFINITY, c.st = 0.f, c.a = 0.f, c.e = 0.f;
@@ -65,18 +75,18 @@ __device__ __forceinline__ void kl_add(KlAcc& c, const float (&zt)[8], const flo
     c.sp *= f, c.u *= f;
     c.mp = cmp;
   }
+  // 2^(y_t - m_p) = 2^(y_t - m_t) 2^(m_t - m_p): one exp2 per chunk instead of per element
+  const float cexp = c.mt - c.mp;
+  c.far |= cexp > kKlFar;
+  const float scale = ex2(fminf(cexp, kKlFar));
 #pragma unroll
   for (int k = 0; k < n; ++k) {
-    const float yt = zt[k] * kLog2e, yp = zp[k] * kLog2e;
-    const float wt = exp2f(yt - c.mt), wp = exp2f(yp - c.mp);
-    const float dx = yt - c.mp;
-    c.far |= dx > kKlFar;
-    const float wx = exp2f(fminf(dx, kKlFar));
+    const float wt = ex2(fmaf(zt[k], kLog2e, -c.mt)), wp = ex2(fmaf(zp[k], kLog2e, -c.mp));
     c.st += wt;
     c.sp += wp;
     c.a = fmaf(wt, zt[k] - zp[k], c.a);
     c.e = fmaf(wt, zt[k], c.e);
-    c.u += wx - wp;
+    c.u += fmaf(wt, scale, -wp);
   }
 }
 
