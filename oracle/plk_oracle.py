@@ -43,6 +43,11 @@ R7  KL lock ([SL] Sec. 2 "Locking Condition"): p_t = softmax over the
     "confidence gate" (low entropy) is read as H(p_t) <= h_max in nats; with
     h_max = +inf the gate is off.  The caller supplies the logits of both
     steps; rows already locked are not examined and stay locked.
+R8  Rotary position embedding (an optional layer variant; the pages name the
+    8B model but not its positional encoding): with dims.rope_theta > 0, q and
+    k of the token at position n of its sequence are rotated per head before
+    they are stored or attended: for i < hd/2 the pair (x_i, x_{i+hd/2}) turns
+    by the angle n * theta^(-2i/hd).  K is cached after the rotation.
 R6  Precision policy "bf16": every tensor that the bf16 path stores in bf16
     between operations is rounded to bf16 here as well -- the normalised
     inputs of the projections (xn, hn), q, k, v (and so the K/V cache), the
@@ -64,7 +69,7 @@ import numpy as np
 __all__ = [
     "to_bf16", "to_f32", "count_flops", "rmsnorm", "silu",
     "proxy_project", "drift_cosine", "drift_l2", "score_drift",
-    "lock_threshold", "lock_topk", "compact", "log_softmax", "kl_divergence", "entropy", "kl_lock",
+    "lock_threshold", "lock_topk", "compact", "log_softmax", "kl_divergence", "entropy", "kl_lock", "rope",
     "full_layer_step", "layer_step_partial", "proxy_commit",
     "LayerState", "tiny_run",
 ]
@@ -311,6 +316,29 @@ class LayerState:
         return LayerState(self.K.copy(), self.V.copy(), self.Y.copy())
 
 
+def rope(x, pos, H, hd, theta):
+    """R8: rows x [R, H*hd] at sequence positions pos [R]; per head the pair (x_i, x_{i+hd/2}),
+    i < hd/2, turns by pos * theta^(-2i/hd) (float64)."""
+    x = np.asarray(x, dtype=np.float64).reshape(-1, H, hd)
+    half = hd // 2
+    inv = theta ** (-2.0 * np.arange(half) / hd)
+    ang = np.asarray(pos, dtype=np.float64)[:, None] * inv[None, :]
+    c, s = np.cos(ang)[:, None, :], np.sin(ang)[:, None, :]
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x1 * s + x2 * c], axis=-1).reshape(-1, H * hd)
+
+
+def _qk(qkv, dims, pos):
+    """q and k of the projection output, rotated when the layer uses RoPE (R8)."""
+    d = dims.d
+    q, k = qkv[:, :d], qkv[:, d:2 * d]
+    theta = getattr(dims, "rope_theta", 0.0)
+    if theta and theta > 0:
+        q = rope(q, pos, dims.H, dims.hd, theta)
+        k = rope(k, pos, dims.H, dims.hd, theta)
+    return q, k
+
+
 def _w(W, name):
     return np.asarray(W[name], dtype=np.float64)
 
@@ -326,8 +354,8 @@ def full_layer_step(dims, W, X, policy="f64"):
     x = np.asarray(X, dtype=np.float64).reshape(B * N, d)
     xn = _store(rmsnorm(x, W["g1"], dims.eps), policy)
     qkv = _mm(xn, _w(W, "w_qkv"))
-    q = _store(qkv[:, :d], policy)
-    k = _store(qkv[:, d:2 * d], policy)
+    q, k = _qk(qkv, dims, np.arange(B * N) % N)
+    q, k = _store(q, policy), _store(k, policy)
     v = _store(qkv[:, 2 * d:], policy)
     a = np.zeros((B * N, d))
     scale = 1.0 / math.sqrt(hd)
@@ -375,8 +403,8 @@ def layer_step_partial(dims, W, X, idx, seg_ptr, state, policy="f64", out_rows=N
     xn = _store(rmsnorm(x, W["g1"], dims.eps), policy)
     # S5 projections (Q only for active rows: [SL] Sec. 2 skips Q of locked rows)
     qkv = _mm(xn, _w(W, "w_qkv"))
-    q = _store(qkv[:, :d], policy)
-    k = _store(qkv[:, d:2 * d], policy)
+    q, k = _qk(qkv, dims, idx % N)
+    q, k = _store(q, policy), _store(k, policy)
     v = _store(qkv[:, 2 * d:], policy)
     # S6 K/V scatter into the cache rows of the active positions
     Kf = out.K.reshape(B * N, d)

@@ -63,6 +63,7 @@ class Dims:
     F: int
     eps: float = 1e-6
     dtype: str = "bf16"  # "bf16" or "f32"
+    rope_theta: float = 0.0  # RoPE base for q and k; 0 = no rotary embedding
 
     def __post_init__(self):
         assert self.d == self.H * self.hd, "d must equal H*hd"

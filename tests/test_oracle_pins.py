@@ -363,7 +363,7 @@ def test_compact_against_nonzero():
 _FULL_MUTANTS = [
     ("hres = x + _mm(a", "hres = _mm(a"),                                  # dropped residual
     ("* scale          ", "* 1.0            "),                            # wrong softmax scale
-    ("q = _store(qkv[:, :d]", "q = _store(qkv[:, d:2 * d]"),              # q taken from K rows
+    ("q, k = _qk(qkv, dims", "k, q = _qk(qkv, dims"),                     # q and k swapped
     ("_mm(a, _w(W, \"w_o\"))", "_mm(a, _w(W, \"w_o\").T)"),               # transposed operand
     ("silu(gu[:, :F]) * gu[:, F:]", "silu(gu[:, F:]) * gu[:, :F]"),       # gate/up swapped
     ("S = S - S.max(axis=1, keepdims=True)", "S = S - S.max(axis=0, keepdims=True)"),
@@ -512,3 +512,56 @@ def test_kl_lock_semantics():
     out3, _, _ = oracle.kl_lock(zt, zp, lock_in, eps, hm)
     np.testing.assert_array_equal(out3[act], ((kl[act] <= eps) & (h[act] <= hm)).astype(np.uint8))
     assert np.all(out3 <= out)
+
+
+# ---------------------------------------------------------------------------
+# RoPE layer variant (reading R8)
+# ---------------------------------------------------------------------------
+def test_rope_matches_complex_rotation():
+    rng = np.random.default_rng(40)
+    H, hd, theta = 3, 16, 10000.0
+    x = rng.standard_normal((5, H * hd))
+    pos = np.array([0, 1, 7, 100, 4095])
+    got = oracle.rope(x, pos, H, hd, theta).reshape(5, H, hd)
+    z = x.reshape(5, H, hd)
+    zc = z[..., : hd // 2] + 1j * z[..., hd // 2:]                      # pair (i, i + hd/2) as a + ib
+    w = np.exp(1j * pos[:, None, None] * theta ** (-np.arange(hd // 2) * 2.0 / hd))
+    ref = zc * w
+    np.testing.assert_allclose(got[..., : hd // 2], ref.real, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got[..., hd // 2:], ref.imag, rtol=0, atol=1e-12)
+
+
+def test_rope_invariants():
+    rng = np.random.default_rng(41)
+    H, hd, theta = 2, 8, 500.0
+    q, k = rng.standard_normal((1, H * hd)), rng.standard_normal((1, H * hd))
+    np.testing.assert_array_equal(oracle.rope(q, [0], H, hd, theta), q)  # position 0: identity
+    r = oracle.rope(q, [37], H, hd, theta)
+    np.testing.assert_allclose(np.linalg.norm(r.reshape(H, hd), axis=1),
+                               np.linalg.norm(q.reshape(H, hd), axis=1), rtol=1e-13)
+    # scores depend on the relative position only
+    def score(m, n):
+        a = oracle.rope(q, [m], H, hd, theta).reshape(H, hd)
+        b = oracle.rope(k, [n], H, hd, theta).reshape(H, hd)
+        return np.sum(a * b, axis=1)
+    np.testing.assert_allclose(score(9, 4), score(109, 104), rtol=0, atol=1e-12)
+    assert np.max(np.abs(score(9, 4) - score(4, 9))) > 1e-3
+
+
+def test_rope_partial_equals_full_and_keeps_locked_rows():
+    dims = synth.Dims(B=2, N=7, d=16, H=2, hd=8, F=24, eps=1e-6, dtype="f32", rope_theta=100.0)
+    W = _weights(dims)
+    X = synth.hidden_states(dims, seed=42)
+    full = oracle.full_layer_step(dims, W, X, "f64")
+    plain = oracle.full_layer_step(synth.Dims(**{**dims.__dict__, "rope_theta": 0.0}), W, X, "f64")
+    assert np.max(np.abs(full.Y - plain.Y)) > 1e-3  # the rotation changes the layer
+    np.testing.assert_array_equal(full.V, plain.V)   # and leaves V alone
+    idx, seg = oracle.compact(np.zeros((2, 7), np.uint8))
+    part = oracle.layer_step_partial(dims, W, X, idx, seg, oracle.LayerState(*(np.zeros_like(full.K),) * 3), "f64")
+    for a, b in ((part.K, full.K), (part.V, full.V), (part.Y, full.Y)):
+        assert np.max(np.abs(a - b)) < 1e-12
+    lock = synth.bernoulli_active(2, 7, 0.5, seed=42)
+    idx, seg = oracle.compact(lock)
+    part = oracle.layer_step_partial(dims, W, X, idx, seg, full, "f64")  # unchanged inputs
+    for a, b in ((part.K, full.K), (part.V, full.V), (part.Y, full.Y)):
+        assert np.max(np.abs(a - b)) < 1e-12
