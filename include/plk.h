@@ -79,6 +79,11 @@ typedef struct {
   int B, N, d, H, hd, F;
   float eps;    /* RMSNorm epsilon                                      */
   int dtype;    /* PLK_F32 or PLK_BF16                                   */
+  float rope_theta; /* rotary position embedding base for q and k; 0 = none.
+                     * With theta > 0 the pair (x_i, x_{i+hd/2}) of every
+                     * head of q and k of the token at position n of its
+                     * sequence turns by n * theta^(-2i/hd) before it is
+                     * stored (K is cached after the rotation).            */
 } plk_dims;
 
 /* Layer weights, nn.Linear layout [out_features, in_features], row-major:

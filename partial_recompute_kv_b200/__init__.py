@@ -33,7 +33,8 @@ EXPORTED = (
 
 class PlkDims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("N", ctypes.c_int), ("d", ctypes.c_int), ("H", ctypes.c_int),
-                ("hd", ctypes.c_int), ("F", ctypes.c_int), ("eps", ctypes.c_float), ("dtype", ctypes.c_int)]
+                ("hd", ctypes.c_int), ("F", ctypes.c_int), ("eps", ctypes.c_float), ("dtype", ctypes.c_int),
+                ("rope_theta", ctypes.c_float)]
 
 
 class PlkWeights(ctypes.Structure):
@@ -111,8 +112,8 @@ def _check(code, where):
         raise PlkError(code, where)
 
 
-def dims(B, N, d, H, hd, F, eps=1e-6, dtype=BF16) -> PlkDims:
-    return PlkDims(int(B), int(N), int(d), int(H), int(hd), int(F), float(eps), int(dtype))
+def dims(B, N, d, H, hd, F, eps=1e-6, dtype=BF16, rope_theta=0.0) -> PlkDims:
+    return PlkDims(int(B), int(N), int(d), int(H), int(hd), int(F), float(eps), int(dtype), float(rope_theta))
 
 
 def _ptr(t):

@@ -13,6 +13,7 @@ static int check_dims(const plk_dims* d) {
   if ((long long)d->H * d->hd != d->d) return PLK_ERR_SHAPE;
   if ((long long)d->B * d->N >= (1LL << 31)) return PLK_ERR_SHAPE;
   if (!(d->eps >= 0.f)) return PLK_ERR_ARG;
+  if (!(d->rope_theta >= 0.f) || d->rope_theta > 3.0e38f) return PLK_ERR_ARG;
   if (d->dtype == PLK_BF16) {
     if (d->hd != 128 || d->d % 256 != 0 || d->F % 128 != 0) return PLK_ERR_SHAPE;
   } else {

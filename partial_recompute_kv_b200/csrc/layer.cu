@@ -301,20 +301,55 @@ __device__ __forceinline__ void load8(const float* p, float* f) {
   f[0] = a.x, f[1] = a.y, f[2] = a.z, f[3] = a.w, f[4] = b.x, f[5] = b.y, f[6] = b.z, f[7] = b.w;
 }
 
-// [q | k | v] sums of compact row j -> Q[j] (compact), K/V cache rows idx[j]
+// Rotary position embedding: cos and sin of pos * theta^(-2i/hd) for the pair
+// (x_i, x_{i+hd/2}) of a head.  The angle is formed and reduced modulo 2 pi in
+// double, so that large positions keep full fp32 accuracy in sincosf.
+__device__ __forceinline__ void rope_cs(int pos, int i, int hd, float log2_theta, float& c, float& s) {
+  const double inv = exp2(-(2.0 * i / hd) * (double)log2_theta);
+  double a = (double)pos * inv;
+  const double two_pi = 6.283185307179586;
+  a -= floor(a / two_pi) * two_pi;
+  sincosf((float)a, &s, &c);
+}
+
+// [q | k | v] sums of compact row j -> Q[j] (compact), K/V cache rows idx[j];
+// with RoPE (log2_theta > 0) q and k are rotated by the row's position idx[j] % N
 __global__ void __launch_bounds__(256) finish_qkv_kernel(const float* __restrict__ qkv32,
                                                          const int32_t* __restrict__ idx,
-                                                         const int32_t* __restrict__ seg_ptr, int B, int d,
-                                                         __nv_bfloat16* __restrict__ q, __nv_bfloat16* __restrict__ Kc,
+                                                         const int32_t* __restrict__ seg_ptr, int B, int N, int d,
+                                                         int hd, float log2_theta, __nv_bfloat16* __restrict__ q,
+                                                         __nv_bfloat16* __restrict__ Kc,
                                                          __nv_bfloat16* __restrict__ Vc) {
   pdl_wait();
   pdl_trigger();
   const int M = seg_ptr[B];
+  const bool rope = log2_theta > 0.f;
+  const int npair = rope ? d / 8 : 0;  // q and k: 8 pairs (x_i, x_{i+hd/2}) per unit
   const int nv = 3 * d / 8;
   for (int j = blockIdx.x; j < M; j += gridDim.x) {
     const size_t row = (size_t)idx[j];
     const float* src = qkv32 + (size_t)j * 3 * d;
-    for (int v = threadIdx.x; v < nv; v += blockDim.x) {
+    const int pos = (int)(row % (size_t)N);
+    for (int u = threadIdx.x; u < npair; u += blockDim.x) {
+      const int per_part = d / 16, part = u / per_part, rem = u - part * per_part;
+      const int h = rem / (hd / 16), i0 = (rem - h * (hd / 16)) * 8;
+      const int c1 = h * hd + i0, c2 = c1 + hd / 2;
+      float x1[8], x2[8];
+      load8(src + part * d + c1, x1);
+      load8(src + part * d + c2, x2);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        float cs, sn;
+        rope_cs(pos, i0 + e, hd, log2_theta, cs, sn);
+        const float a = x1[e], b = x2[e];
+        x1[e] = a * cs - b * sn;
+        x2[e] = a * sn + b * cs;
+      }
+      __nv_bfloat16* dst = part == 0 ? q + (size_t)j * d : Kc + row * d;
+      store_vec<__nv_bfloat16, 8>(dst + c1, x1);
+      store_vec<__nv_bfloat16, 8>(dst + c2, x2);
+    }
+    for (int v = threadIdx.x + (rope ? d / 4 : 0); v < nv; v += blockDim.x) {  // with RoPE: v only
       const int c = v * 8, part = c / d, col = c - part * d;
       float f[8];
       load8(src + c, f);
@@ -411,13 +446,27 @@ __global__ void __launch_bounds__(256) epilogue_f32_kernel(int mode, const float
                                                            const int32_t* __restrict__ idx,
                                                            const int32_t* __restrict__ seg_ptr, int B, int d, int F,
                                                            float* q, float* kc, float* vc, const float* x, float* h32,
-                                                           float* act, float* y) {
+                                                           float* act, float* y, int N, int hd, float log2_theta) {
   const int M = seg_ptr[B];
   const int j = blockIdx.x;
   if (j >= M) return;
   const size_t row = (size_t)idx[j];
   if (mode == F32_QKV) {
     const float* c = C + (size_t)j * 3 * d;
+    if (log2_theta > 0.f) {  // RoPE on q and k: pair (t, t + hd/2) of a head
+      const int pos = (int)(row % (size_t)N), half = hd / 2;
+      for (int u = threadIdx.x; u < d / 2; u += blockDim.x) {
+        const int h = u / half, i = u - h * half, t1 = h * hd + i, t2 = t1 + half;
+        float cs, sn;
+        rope_cs(pos, i, hd, log2_theta, cs, sn);
+        q[(size_t)j * d + t1] = c[t1] * cs - c[t2] * sn;
+        q[(size_t)j * d + t2] = c[t1] * sn + c[t2] * cs;
+        kc[row * d + t1] = c[d + t1] * cs - c[d + t2] * sn;
+        kc[row * d + t2] = c[d + t1] * sn + c[d + t2] * cs;
+      }
+      for (int t = threadIdx.x; t < d; t += blockDim.x) vc[row * d + t] = c[2 * d + t];
+      return;
+    }
     for (int t = threadIdx.x; t < d; t += blockDim.x) {
       q[(size_t)j * d + t] = c[t];
       kc[row * d + t] = c[d + t];
@@ -467,16 +516,17 @@ static int run_layer_f32(const plk_dims* dm, const plk_weights* w, const float* 
   };
   PLK_TRY(launch_rmsnorm<float, float, float>(X, idx, seg, B, (const float*)w->g1, dm->eps, d, xn, Mcap, st));
   gemm(xn, w->w_qkv, 3 * d, d);
-  epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_QKV, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y);
+  epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_QKV, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, dm->N,
+                                            dm->hd, dm->rope_theta > 0.f ? log2f(dm->rope_theta) : 0.f);
   PLK_LAUNCHED();
   PLK_TRY(launch_attention_f32(dm, q, Kc, Vc, a, seg, Mcap, st));
   gemm(a, w->w_o, d, d);
-  epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_O, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y);
+  epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_O, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, 0, 0, 0.f);
   PLK_TRY(launch_rmsnorm<float, float, float>(h32, nullptr, seg, B, (const float*)w->g2, dm->eps, d, hn, Mcap, st));
   gemm(hn, w->w_gu, 2 * F, d);
-  epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_GU, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y);
+  epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_GU, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, 0, 0, 0.f);
   gemm(act, w->w_down, d, F);
-  epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_DOWN, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y);
+  epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_DOWN, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, 0, 0, 0.f);
   PLK_LAUNCHED();
   return PLK_OK;
 }
@@ -525,8 +575,9 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   PLK_TRY(launch_gemm_tc(tW_qkv, tX_xn, tO_qkv, g, st));
   trace_mark(2, st);
 
-  PLK_TRY(launch_pdl(finish_qkv_kernel, dim3(rgrid), dim3(256), 0, st, (const float*)c32, idx, seg, B, d, q,
-                     (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc));
+  const float log2_theta = dm->rope_theta > 0.f ? log2f(dm->rope_theta) : 0.f;
+  PLK_TRY(launch_pdl(finish_qkv_kernel, dim3(rgrid), dim3(256), 0, st, (const float*)c32, idx, seg, B, dm->N, d,
+                     dm->hd, log2_theta, q, (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc));
   trace_mark(3, st);
 
   PLK_TRY(launch_attention_bf16(dm, q, Kc, Vc, a, seg, L.num_sms, st));

@@ -28,7 +28,8 @@ def plk():
 
 
 def pdims(plk, D):
-    return plk.dims(D.B, D.N, D.d, D.H, D.hd, D.F, D.eps, plk.BF16 if D.dtype == "bf16" else plk.F32)
+    return plk.dims(D.B, D.N, D.d, D.H, D.hd, D.F, D.eps, plk.BF16 if D.dtype == "bf16" else plk.F32,
+                    getattr(D, "rope_theta", 0.0))
 
 
 def int_dev(a, n):
@@ -226,6 +227,52 @@ def test_partial_step_bf16(plk, p_active):
     assert_bf16_close(K[act], ref.K[act], "K active")
     assert_bf16_close(V[act], ref.V[act], "V active")
     assert_bf16_close(Y[act], ref.Y[act], "Y active")
+
+
+@pytest.mark.parametrize("theta", [10000.0, 500000.0])
+def test_rope_layer_bf16(plk, theta):
+    """RoPE variant: full step, then a partial step on perturbed active rows (positions up to
+    N - 1 = 319 in each of two sequences)."""
+    D = synth.Dims(**{**SMALL.__dict__, "rope_theta": theta})
+    W = synth.layer_weights(D, 0.02, seed=8)
+    X = synth.hidden_states(D, seed=8)
+    base = oracle.full_layer_step(D, W, X, "bf16")
+    dm = pdims(plk, D)
+    K = torch.zeros((D.B, D.N, D.d), dtype=BF, device="cuda")
+    V, Y = torch.zeros_like(K), torch.zeros_like(K)
+    plk.full_layer_step(dm, weights_dev(W, D), dev(X, BF), K, V, Y, plk.alloc_workspace(dm))
+    assert plk.get_status() == plk.OK
+    assert_bf16_close(host(K), base.K, "K full")
+    assert_bf16_close(host(Y), base.Y, "Y full")
+    lock = synth.bernoulli_active(D.B, D.N, 0.3, seed=8)
+    idx, seg = oracle.compact(lock)
+    X2 = synth.perturb_rows(X, synth.step_noise((D.B, D.N, D.d), 0.01, seed=8), lock == 0, "bf16")
+    ref = oracle.layer_step_partial(D, W, X2, idx, seg, base, "bf16")
+    K, V, Y = _run_partial(plk, D, W, X2, idx, seg, base)
+    locked = lock.astype(bool)
+    assert np.array_equal(K[locked], base.K[locked]) and np.array_equal(Y[locked], base.Y[locked])
+    act = ~locked
+    assert_bf16_close(K[act], ref.K[act], "K active")
+    assert_bf16_close(Y[act], ref.Y[act], "Y active")
+
+
+def test_rope_layer_fp32(plk):
+    D = synth.Dims(B=2, N=100, d=64, H=4, hd=16, F=64, eps=1e-6, dtype="f32", rope_theta=10000.0)
+    W = synth.layer_weights(D, 1.0 / math.sqrt(D.d), seed=9)
+    X = synth.hidden_states(D, seed=9)
+    base = oracle.full_layer_step(D, W, X, "f64")
+    lock = synth.bernoulli_active(D.B, D.N, 0.4, seed=9)
+    idx, seg = oracle.compact(lock)
+    X2 = synth.perturb_rows(X, synth.step_noise((D.B, D.N, D.d), 0.01, seed=9), lock == 0, "f32")
+    ref = oracle.layer_step_partial(D, W, X2, idx, seg, base, "f64")
+    dm = pdims(plk, D)
+    K, V, Y = (dev(a, torch.float32) for a in (base.K, base.V, base.Y))
+    plk.layer_step_partial(dm, weights_dev(W, D), dev(X2, torch.float32), int_dev(idx, D.B * D.N),
+                           int_dev(seg, D.B + 1), K, V, Y, plk.alloc_workspace(dm))
+    assert plk.get_status() == plk.OK
+    act = lock == 0
+    assert_f32_close(host(K)[act], ref.K[act], "K active")
+    assert_f32_close(host(Y)[act], ref.Y[act], "Y active")
 
 
 def test_partial_step_m_zero_is_noop(plk):
