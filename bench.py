@@ -503,6 +503,105 @@ def run_kl_lock(args):
     return 0
 
 
+# ---------------------------------------------------------------------------
+# kernels at the configurations where their rooflines are judged (not the
+# headline): scoring at the 8 x 4096 scoring shape (HBM-bound), and the layer
+# step with every row active at B = 4, N = 2048 (step 0 of the 32-layer stack:
+# compute-bound GEMMs and attention, the K/V scatter at 67 MB)
+# ---------------------------------------------------------------------------
+def _timed(torch, fn, steps, warmup):
+    for _ in range(max(warmup, 3)):
+        fn()
+    torch.cuda.synchronize()
+    E = lambda: torch.cuda.Event(enable_timing=True)
+    ev = [(E(), E()) for _ in range(steps)]
+    for a, b in ev:
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
+
+
+def run_kernel_configs(args):
+    import torch
+    import partial_recompute_kv_b200 as plk
+    import synth
+
+    dev = torch.device("cuda", 0)
+    bf = torch.bfloat16
+    pk = peaks()
+    hbm, tfl = float(pk["hbm_gbs"]), float(pk["bf16_tflops"])
+    up = lambda a, dt: torch.from_numpy(np.ascontiguousarray(a)).to(dev).to(dt)
+    out = []
+    # scoring shape: X [8, 4096, 4096] bf16, rank 128, L2; top-k 10% per sequence
+    D, r = synth.SCORE_8B, synth.PROXY_RANK_8B
+    dm = plk.dims(D.B, D.N, D.d, D.H, D.hd, D.F, D.eps, plk.BF16)
+    X = torch.randn((D.B, D.N, D.d), device=dev).to(bf)
+    Ut = up(synth.proxy_basis(D.d, r, seed=0), bf)
+    pc = torch.randn((D.B, D.N, r), device=dev)
+    pnew, score = torch.empty_like(pc), torch.empty((D.B, D.N), device=dev)
+    us = _timed(torch, lambda: plk.score_drift(dm, X, Ut, r, pc, plk.METRIC_L2, score, proxy_out=pnew),
+                args.steps, args.warmup)
+    by = 2 * D.B * D.N * D.d + 8 * D.B * D.N * r + 2 * D.d * r
+    out.append({"kernel": "score_tc_kernel", "config": f"B={D.B} N={D.N} d={D.d} r={r} L2", "us": us,
+                "GB/s": by / (us * 1e-6) / 1e9, "frac_of_hbm": by / (us * 1e-6) / 1e9 / hbm})
+    k = D.N * 10 // 100
+    lk_in = torch.zeros((D.B, D.N), dtype=torch.uint8, device=dev)
+    lk, idx = torch.empty_like(lk_in), torch.empty(D.B * D.N, dtype=torch.int32, device=dev)
+    seg = torch.empty(D.B + 1, dtype=torch.int32, device=dev)
+    us = _timed(torch, lambda: plk.select_active(dm, score, lk_in, lk, plk.SEL_TOPK_LARGEST, 0.0, k, idx, seg),
+                args.steps, args.warmup)
+    by = 6 * D.B * D.N + 4 * D.B * k
+    out.append({"kernel": "topk_compact_kernel", "config": f"B={D.B} N={D.N} k={k}", "us": us,
+                "GB/s": by / (us * 1e-6) / 1e9, "frac_of_hbm": by / (us * 1e-6) / 1e9 / hbm})
+    del X, pc, pnew
+    # stack step 0: B = 4, N = 2048, every row active
+    D = synth.STACK_8B
+    dm = plk.dims(D.B, D.N, D.d, D.H, D.hd, D.F, D.eps, plk.BF16)
+    W = {kk: (torch.randn(sh, device=dev) * 0.02).to(bf) if len(sh) == 2 else torch.ones(sh, device=dev).to(bf)
+         for kk, sh in (("g1", (D.d,)), ("w_qkv", (3 * D.d, D.d)), ("w_o", (D.d, D.d)), ("g2", (D.d,)),
+                        ("w_gu", (2 * D.F, D.d)), ("w_down", (D.d, D.F)))}
+    pw = plk.weights(W)
+    X = torch.randn((D.B, D.N, D.d), device=dev).to(bf)
+    K, V, Y = (torch.zeros((D.B, D.N, D.d), dtype=bf, device=dev) for _ in range(3))
+    M = D.B * D.N
+    idx = torch.arange(M, dtype=torch.int32, device=dev)
+    seg = torch.tensor([b * D.N for b in range(D.B + 1)], dtype=torch.int32, device=dev)
+    ws = plk.alloc_workspace(dm, device=dev)
+    step = lambda: plk.layer_step_partial(dm, pw, X, idx, seg, K, V, Y, ws)
+    us_step = _timed(torch, step, max(args.steps // 10, 5), args.warmup)
+    E = lambda: torch.cuda.Event(enable_timing=True)
+    tr = [[E() for _ in range(11)] for _ in range(5)]
+    for e in tr:
+        plk.trace_events(e)
+        step()
+    torch.cuda.synchronize()
+    plk.trace_events([])
+    names = ["rmsnorm1", "gemm_qkv", "finish_qkv", "attention", "gemm_o", "rmsnorm2", "gemm_gu", "finish_gu",
+             "gemm_down", "finish_y"]
+    per = {n: statistics.median(e[i].elapsed_time(e[i + 1]) for e in tr) * 1e3 for i, n in enumerate(names)}
+    gemm_flops = M * (8 * D.d * D.d + 6 * D.d * D.F)
+    gemm_us = per["gemm_qkv"] + per["gemm_o"] + per["gemm_gu"] + per["gemm_down"]
+    att_flops = 4 * D.B * D.N * D.N * D.d  # QK^T and PV over every (query, key) pair of a sequence
+    scat = 18 * M * D.d
+    out.append({"kernel": "layer step, every row active", "config": f"B={D.B} N={D.N} (stack step 0)",
+                "us": us_step, "active_token_layers_per_s": M / (us_step * 1e-6),
+                "gemm_tc_kernel": {"us": gemm_us, "TFLOP/s": gemm_flops / (gemm_us * 1e-6) / 1e12,
+                                   "frac_of_peak": gemm_flops / (gemm_us * 1e-6) / 1e12 / tfl},
+                "attn_tc_kernel": {"us": per["attention"], "TFLOP/s": att_flops / (per["attention"] * 1e-6) / 1e12,
+                                   "frac_of_peak": att_flops / (per["attention"] * 1e-6) / 1e12 / tfl},
+                "finish_qkv_kernel (K/V scatter)": {"us": per["finish_qkv"], "GB/s": scat / (per["finish_qkv"] * 1e-6) / 1e9,
+                                                    "frac_of_hbm": scat / (per["finish_qkv"] * 1e-6) / 1e9 / hbm},
+                "per_kernel_us_traced": per})
+    st = plk.get_status()
+    if st != plk.OK:
+        raise RuntimeError(f"device status {plk.error_string(st)}")
+    for o in out:
+        print(json.dumps(o), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -516,8 +615,9 @@ def main():
                     help="replay the step as one captured CUDA graph (default)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="enqueue the step's library calls directly every step")
-    ap.add_argument("--kernel", choices=["step", "kl_lock"], default="step",
-                    help="step: the headline layer step; kl_lock: the KL lock rule alone")
+    ap.add_argument("--kernel", choices=["step", "kl_lock", "configs"], default="step",
+                    help="step: the headline layer step; kl_lock: the KL lock rule alone; configs: scoring "
+                         "and the all-active stack step at the shapes where their rooflines are judged")
     ap.add_argument("--profile", action="store_true",
                     help="set up and run --steps steps without timing or output (for ncu)")
     args = ap.parse_args()
@@ -528,6 +628,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.kernel == "kl_lock":
         return run_kl_lock(args) if rank == 0 else 0
+    if args.kernel == "configs":
+        return run_kernel_configs(args) if rank == 0 else 0
     if args.impl == "reference":
         if rank != 0:
             return 0
