@@ -57,9 +57,12 @@ static_assert((size_t)4 * 8 * kBlk * 4 <= kOffBar, "the last piece's blocks fit 
 // Longest run of k-blocks accumulated in one TMEM chain before its partial is
 // added into the fp32 output.  The tensor core's fp32 accumulation loses a
 // little precision per step (measured: 0.14% of bf16-rounded q values differ
-// from an fp64 reference over 256 steps, against 0.017% for fp32 in sequence
-// on the CPU); shorter chains summed by the L2 in fp32 keep that loss small.
-constexpr int kGemmChainKB = 16;
+// from an fp64 reference over 256 steps, 0.06% over 64, against 0.017% for
+// fp32 in sequence on the CPU); shorter chains summed by the L2 in fp32 keep
+// that loss small, but every chain is one more fp32 read-modify-write of its
+// tile (measured over the four projections: 16 k-blocks cost 5% at 256 tokens
+// and 15% at 2048 tokens against no limit).
+constexpr int kGemmChainKB = 32;
 
 // bulk reduce-add of a [32 rows][32 fp32] smem block into the tensor at (x, y)
 __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* tm, int x, int y, const void* smem_src) {

@@ -381,13 +381,14 @@ def test_layer_8b_quarter_sampled(layer_8b_quarter):
     assert np.all(np.isfinite(g))
     mr, ma = metrics(g, o)
     assert mr <= BF16_MAX_REL, f"Y sampled: max_rel {mr:.3e}"
-    # regression guard at the level measured on B200 (1.17e-3); the 1e-3 bound is the next test
+    # regression guard at the level measured on B200 (1.17e-3 to 1.29e-3 with accumulation chains of
+    # 16 k-blocks to unlimited); the 1e-3 bound is the next test
     assert ma <= 1.3e-3, f"Y sampled: mae/rms {ma:.3e}"
 
 
 @pytest.mark.slow
 @pytest.mark.xfail(strict=False, reason=(
-    "Y mean absolute error at d=4096, F=12288 is 1.17e-3 of rms(y) against the 1e-3 bound: the "
+    "Y mean absolute error at d=4096, F=12288 is 1.2e-3 of rms(y) against the 1e-3 bound: the "
     "tensor cores' fp32 accumulation drifts a little per MMA step over K=4096 and 12288, and the "
     "bf16 storage points (q, a, hn, act) amplify single-ulp flips; an fp32-exact pipeline reaches "
     "7.6e-4 at this shape.  Every smaller shape meets the bound."))
