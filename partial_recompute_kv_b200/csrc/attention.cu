@@ -15,9 +15,11 @@
 // enter P V with ~16 significant bits (a bf16-rounded P would perturb the
 // attention output by ~1e-3 relative, which later bf16 roundings amplify).  A
 // row keeps a stale max until the new one exceeds it by 2^8 (the weights stay
-// below 256, exact in fp32); only then is its O row rescaled in TMEM.  Keys are
-// split over CTAs when the query tiles alone leave SMs idle; a combine kernel
-// merges the splits.  Keys past N are masked.
+// below 256, exact in fp32); only then is its O row rescaled in TMEM.  When the
+// query tiles alone leave SMs idle, the two CTAs of a cluster pair split a
+// tile's keys: the odd CTA hands its partial O, row max and row sum to the even
+// CTA through distributed shared memory, which merges and writes the tile.
+// Keys past N are masked.
 // fp32: one thread per (query row, head), online softmax, SIMT.
 #include <math.h>
 
