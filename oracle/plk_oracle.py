@@ -17,6 +17,11 @@ Pages followed (cited by title and section):
 [PS]  "Polestar: Drift-Aware Cache Calibration and Token Commitment for
       Efficient Inference of Diffusion LLMs".  Polestar-Cache: refresh only the
       positions whose representation drifted most.
+[SF]  "Accelerating Diffusion Large Language Models with SlowFast Sampling: The
+      Three Golden Principles".  Part 2 "Methodology": the two-stage pipeline
+      (exploratory stage with its stability check, accelerated stage with
+      in-span parallel decoding, out-of-span caching and the top-k fallback);
+      part 4 "Ablation Studies" (K_max = 8, W_hist = 2, variance threshold 1.0).
 
 Readings taken where the pages are silent (each is listed in the design notes):
 
@@ -48,6 +53,30 @@ R8  Rotary position embedding (an optional layer variant; the pages name the
     k of the token at position n of its sequence are rotated per head before
     they are stored or attended: for i < hd/2 the pair (x_i, x_{i+hd/2}) turns
     by the angle n * theta^(-2i/hd).  K is cached after the rotation.
+R9  SlowFast span policy ([SF] part 2), per sequence and per decoding step,
+    on the caller's confidences c_i (fp32) of the still-masked positions:
+    - A cycle starts in the slow phase at s = the first masked position.  A
+      slow step unmasks the k most confident masked positions at or after s
+      (larger c first, NaN last, ties to the lower index) and records the
+      convergence end point e_t = the largest masked position >= s with
+      c_i > tau_conv (e_t = s when there is none), taken on this step's
+      confidences before its unmasking.
+    - After a slow step the cycle turns fast with the span [s, e_t] when at
+      least W_hist end points were recorded in this cycle and the population
+      variance of the last W_hist of them is < var_stable (strictly), or when
+      the cycle has taken K_max slow steps.
+    - A fast step unmasks every masked position in [s, e] with c_i > tau_high;
+      when none qualifies it unmasks the k most confident masked positions of
+      the span instead (the fallback, "insufficient" read as "none").
+    - When no masked position is left in the span (after a fast step, or at
+      once after the switch), the cycle ends: the state returns to its initial
+      value (slow, s = e = 0, no end points).  A fast step that finds no masked
+      position in its span unmasks nothing and ends the cycle.  A state with
+      an unknown phase or a negative step count is read as the initial state.
+    - lock_out says which rows the next forward pass may skip (the out-of-span
+      caching): in the fast phase every row outside [s, e]; in the slow phase
+      none; once nothing is masked, every row.  A sequence with nothing masked
+      is left as it is.
 R6  Precision policy "bf16": every tensor that the bf16 path stores in bf16
     between operations is rounded to bf16 here as well -- the normalised
     inputs of the projections (xn, hn), q, k, v (and so the K/V cache), the
@@ -63,6 +92,7 @@ from __future__ import annotations
 
 import contextlib
 import math
+from fractions import Fraction
 
 import numpy as np
 
@@ -70,6 +100,7 @@ __all__ = [
     "to_bf16", "to_f32", "count_flops", "rmsnorm", "silu",
     "proxy_project", "drift_cosine", "drift_l2", "score_drift",
     "lock_threshold", "lock_topk", "compact", "log_softmax", "kl_divergence", "entropy", "kl_lock", "rope",
+    "SpanParams", "SpanState", "population_variance", "slowfast_step_seq", "slowfast_step",
     "full_layer_step", "layer_step_partial", "proxy_commit",
     "LayerState", "tiny_run",
 ]
@@ -283,6 +314,116 @@ def kl_lock(logits_t, logits_prev, lock_in, eps, h_max=math.inf):
             ent[b, i] = entropy(logits_t[b, i])
             out[b, i] = kl[b, i] <= eps and ent[b, i] <= h_max
     return out.astype(np.uint8), kl, ent
+
+
+# ---------------------------------------------------------------------------
+# SlowFast span policy ([SF] part 2 "Methodology"; part 4 "Ablation Studies"; R9)
+# ---------------------------------------------------------------------------
+SF_SLOW, SF_FAST = 0, 1
+
+
+class SpanParams:
+    """Knobs of the policy.  k: positions per slow step and per fallback;
+    tau_conv: confidence that marks a converged position (end point);
+    tau_high: the in-span threshold tau_high_conf; var_stable: sigma^2_stable;
+    w_hist: W_hist; k_max: K_max.  Thresholds are fp32 values, as on the device."""
+
+    def __init__(self, k=1, tau_conv=0.5, tau_high=0.9, var_stable=1.0, w_hist=2, k_max=8):
+        self.k, self.w_hist, self.k_max = int(k), int(w_hist), int(k_max)
+        self.tau_conv = float(np.float32(tau_conv))
+        self.tau_high = float(np.float32(tau_high))
+        self.var_stable = float(np.float32(var_stable))
+
+
+class SpanState:
+    """One sequence's policy state: phase, cycle start s, span end e, slow steps
+    taken in this cycle and their end points (oldest first)."""
+
+    def __init__(self, phase=SF_SLOW, s=0, e=0, nslow=0, hist=()):
+        self.phase, self.s, self.e, self.nslow = int(phase), int(s), int(e), int(nslow)
+        self.hist = [int(v) for v in hist]
+
+    def copy(self):
+        return SpanState(self.phase, self.s, self.e, self.nslow, self.hist)
+
+
+def population_variance(values):
+    """Exact population variance, (1/n) sum (v - mean)^2, as a Fraction."""
+    n = len(values)
+    mean = Fraction(sum(values), n)
+    return sum((Fraction(v) - mean) ** 2 for v in values) / n
+
+
+def _most_confident(conf, cand, k):
+    """The k most confident positions of cand: larger confidence first, NaN last, ties to the lower index."""
+    def key(i):
+        v = float(conf[i])
+        return (1, 0.0, i) if math.isnan(v) else (0, -v, i)
+    return sorted(cand, key=key)[:k]
+
+
+def slowfast_step_seq(conf, masked, state, p):
+    """One decoding step of the SlowFast policy on one sequence (R9).
+
+    conf [N] fp32 confidences of this step; masked [N] (1 = still masked);
+    state: SpanState; p: SpanParams.  Returns (masked' [N] u8, unmask [N] u8,
+    lock [N] u8, state').  The inputs are not modified.
+    """
+    conf = np.asarray(conf, dtype=np.float32)
+    N = conf.shape[0]
+    masked = np.asarray(masked).astype(bool).copy()
+    st = state.copy()
+    if st.phase not in (SF_SLOW, SF_FAST) or st.nslow < 0:
+        st = SpanState()
+    unmask = np.zeros(N, dtype=bool)
+    pending = [i for i in range(N) if masked[i]]
+    if not pending:
+        return masked.astype(np.uint8), unmask.astype(np.uint8), np.ones(N, np.uint8), st
+
+    chosen = []
+    if st.phase == SF_FAST:
+        cand = [i for i in pending if st.s <= i <= st.e]
+        if not cand:
+            st = SpanState()
+        else:
+            hot = [i for i in cand if float(conf[i]) > p.tau_high]
+            chosen = hot if hot else _most_confident(conf, cand, p.k)
+    else:
+        if st.nslow == 0:
+            st.s = pending[0]
+        cand = [i for i in pending if i >= st.s]
+        converged = [i for i in cand if float(conf[i]) > p.tau_conv]
+        end = max(converged) if converged else st.s
+        chosen = _most_confident(conf, cand, p.k)
+        st.hist.append(end)
+        st.nslow += 1
+        stable = (st.nslow >= p.w_hist
+                  and population_variance(st.hist[-p.w_hist:]) < Fraction(p.var_stable))
+        if stable or st.nslow >= p.k_max:
+            st.phase, st.e = SF_FAST, end
+
+    for i in chosen:
+        masked[i] = False
+        unmask[i] = True
+    if st.phase == SF_FAST and not any(masked[i] for i in range(max(st.s, 0), min(st.e, N - 1) + 1)):
+        st = SpanState()  # the span is decoded: the cycle ends
+
+    if not masked.any():
+        lock = np.ones(N, dtype=np.uint8)
+    elif st.phase == SF_FAST:
+        lock = np.array([0 if st.s <= i <= st.e else 1 for i in range(N)], dtype=np.uint8)
+    else:
+        lock = np.zeros(N, dtype=np.uint8)
+    return masked.astype(np.uint8), unmask.astype(np.uint8), lock, st
+
+
+def slowfast_step(conf, masked, states, p):
+    """slowfast_step_seq on every sequence of conf / masked [B, N]; states: list of B SpanState."""
+    conf = np.asarray(conf, dtype=np.float32)
+    B, N = conf.shape
+    out = [slowfast_step_seq(conf[b], np.asarray(masked)[b], states[b], p) for b in range(B)]
+    return (np.stack([o[0] for o in out]), np.stack([o[1] for o in out]), np.stack([o[2] for o in out]),
+            [o[3] for o in out])
 
 
 # ---------------------------------------------------------------------------

@@ -29,6 +29,7 @@ S_NOISE = 4
 S_POS = 5
 S_PROXY = 6
 S_LOGITS = 7
+S_CONF = 8
 
 
 def round_bf16(a) -> np.ndarray:
@@ -183,6 +184,32 @@ def logits_pair(B: int, N: int, V: int, seed: int = 0, std: float = 2.0, drift=(
     if dtype == "bf16":
         return round_bf16(zt), round_bf16(zp)
     return zt, zp
+
+
+def span_confidences(B: int, N: int, step: int, seed: int = 0, prompt: int = 0, rate: float = 16.0,
+                     width: float = 24.0, noise: float = 0.75, levels: int = 256) -> np.ndarray:
+    """Per-position confidences [B, N] fp32 in [0, 1] at decoding step `step`.
+
+    A confident region grows from the prompt end by about `rate` positions a
+    step (each sequence with its own jitter): position i gets the logistic of
+    (front - i) / width plus N(0, noise^2) per position, which leaves
+    scattered confident positions ahead of the front and doubtful ones behind
+    it.  Values are rounded to multiples of 1/levels so that equal confidences
+    occur (ties).
+    """
+    rng = _rng(seed, S_CONF, step)
+    i = np.arange(N, dtype=np.float64)
+    front = prompt + rate * (step + 1) + rng.normal(0.0, 4.0, size=(B, 1))
+    z = (front - i[None, :]) / width + rng.normal(0.0, noise, size=(B, N))
+    c = 1.0 / (1.0 + np.exp(-z))
+    return (np.round(c * levels) / levels).astype(np.float32)
+
+
+def generation_mask(B: int, N: int, prompt: int) -> np.ndarray:
+    """masked [B, N] u8: the prompt (first `prompt` positions) is given, the rest is masked."""
+    m = np.ones((B, N), dtype=np.uint8)
+    m[:, :prompt] = 0
+    return m
 
 
 # vocabulary size of the 8B model the pages name, for the KL-lock measurement
