@@ -354,6 +354,13 @@ def population_variance(values):
     return sum((Fraction(v) - mean) ** 2 for v in values) / n
 
 
+def _below(v, x):
+    """v < x for an exact rational v and a float threshold x that may be infinite."""
+    if math.isinf(x):
+        return x > 0
+    return v < Fraction(x)
+
+
 def _most_confident(conf, cand, k):
     """The k most confident positions of cand: larger confidence first, NaN last, ties to the lower index."""
     def key(i):
@@ -397,8 +404,7 @@ def slowfast_step_seq(conf, masked, state, p):
         chosen = _most_confident(conf, cand, p.k)
         st.hist.append(end)
         st.nslow += 1
-        stable = (st.nslow >= p.w_hist
-                  and population_variance(st.hist[-p.w_hist:]) < Fraction(p.var_stable))
+        stable = st.nslow >= p.w_hist and _below(population_variance(st.hist[-p.w_hist:]), p.var_stable)
         if stable or st.nslow >= p.k_max:
             st.phase, st.e = SF_FAST, end
 

@@ -262,6 +262,16 @@ def test_invariants_on_random_trajectories(seed, k, w, kmax, var):
     assert _invariants_hold(po.slowfast_step_seq, seed, p)
 
 
+def test_infinite_variance_threshold():
+    # +inf: every window is stable, so W_hist = 1 switches after each slow step;
+    # -inf: no window is, so only K_max ends the slow phase
+    conf = np.array([.9, .2, .7, .1], dtype=np.float32)
+    for var, k_max, want in ((np.inf, 8, po.SF_FAST), (-np.inf, 8, po.SF_SLOW), (-np.inf, 1, po.SF_FAST)):
+        p = po.SpanParams(k=1, tau_conv=0.5, var_stable=var, w_hist=1, k_max=k_max)
+        st = po.slowfast_step_seq(conf, np.ones(4, np.uint8), po.SpanState(), p)[3]
+        assert st.phase == want and (st.e == 2 if want == po.SF_FAST else True)
+
+
 def test_invalid_state_reads_as_initial_and_inputs_untouched():
     conf = np.array([.9, .2, .7, .1], dtype=np.float32)
     masked = np.ones(4, dtype=np.uint8)
@@ -282,7 +292,7 @@ _MUTANTS = [
     ("slowfast_step_seq", "float(conf[i]) > p.tau_high", "float(conf[i]) >= p.tau_high"),
     ("slowfast_step_seq", "float(conf[i]) > p.tau_conv", "float(conf[i]) >= p.tau_conv"),
     ("slowfast_step_seq", "max(converged)", "min(converged)"),
-    ("slowfast_step_seq", "< Fraction(p.var_stable)", "<= Fraction(p.var_stable)"),
+    ("_below", "v < Fraction(x)", "v <= Fraction(x)"),
     ("slowfast_step_seq", "st.hist[-p.w_hist:]", "st.hist[:p.w_hist]"),
     ("slowfast_step_seq", "chosen = hot if hot else _most_confident(conf, cand, p.k)", "chosen = hot"),
     ("slowfast_step_seq", "st = SpanState()  # the span is decoded", "pass  #"),
