@@ -185,6 +185,62 @@ int plk_kl_lock(const plk_dims* dims, int V, const void* logits_t, const void* l
                 float* kl_out, float* h_out, void* stream);
 
 /*
+ * SlowFast span policy ("Accelerating Diffusion Large Language Models with
+ * SlowFast Sampling: The Three Golden Principles", part 2 "Methodology": the
+ * two-stage pipeline of an exploratory (slow) and an accelerated (fast) stage;
+ * part 4 "Ablation Studies": K_max = 8, W_hist = 2, variance threshold 1.0).
+ * One decoding step per call, per sequence b, on conf [B, N] fp32 (the
+ * confidence of each position's prediction at this step) and masked [B, N]
+ * uint8 (1 = still masked; in/out):
+ *   slow phase: a cycle starts at s = the first masked position.  The k most
+ *     confident masked positions >= s are unmasked (larger first, NaN last,
+ *     equal values to the lower index).  The end point e_t = the largest masked
+ *     position >= s with conf > tau_conv (s when none), taken before this
+ *     step's unmasking, is recorded.  When the cycle has W_hist end points and
+ *     the population variance of the last W_hist is < var_stable, or after
+ *     K_max slow steps, the phase turns fast with the span [s, e_t].
+ *   fast phase: every masked position of [s, e] with conf > tau_high is
+ *     unmasked; when there is none, the k most confident masked positions of
+ *     the span are (the fallback).  A span without masked positions unmasks
+ *     nothing.
+ *   When the span holds no masked position after the step, the cycle ends and
+ *     the state returns to all zeros.  A sequence with nothing masked is left
+ *     unchanged.
+ * Outputs (may be NULL; must not alias masked):
+ *   unmask_out [B, N] uint8: 1 at the positions unmasked by this step.
+ *   lock_out   [B, N] uint8: the rows the next forward pass may skip (the
+ *     out-of-span caching): in the fast phase those outside [s, e], in the slow
+ *     phase none, once nothing is masked all of them.  It is a lock_in for
+ *     plk_select_active(PLK_SEL_THRESH_GT, tau = +INFINITY), which compacts
+ *     the remaining rows.
+ * state [B] plk_sf_state (device, in/out): all zeros before the first step of
+ *   a sequence.  Other contents give unspecified decisions (never an
+ *   out-of-bounds access); a phase other than 0/1 or nslow < 0 reads as zeros.
+ * params (host): k >= 1, 1 <= w_hist <= PLK_SF_HIST_MAX, k_max >= 1,
+ *   thresholds not NaN.  Only dims->B and dims->N are used; N <= 2^20 keeps the
+ *   variance test exact.  Decisions are bit-exact and deterministic.
+ * Errors: PLK_ERR_ARG (NULL input, bad params, aliasing), PLK_ERR_SHAPE.
+ */
+#define PLK_SF_HIST_MAX 16
+typedef struct {
+  int32_t phase;                  /* 0 slow, 1 fast                           */
+  int32_t s, e;                   /* cycle start; span end (fast phase)       */
+  int32_t nslow;                  /* slow steps taken in this cycle           */
+  int32_t hist[PLK_SF_HIST_MAX];  /* end point of slow step n at n % w_hist   */
+} plk_sf_state;
+typedef struct {
+  int k;             /* positions per slow step and per fallback         */
+  int w_hist;        /* W_hist: end points in the variance window        */
+  int k_max;         /* K_max: slow steps after which the span is taken  */
+  float tau_conv;    /* confidence of a converged position (end point)   */
+  float tau_high;    /* tau_high_conf: in-span parallel unmasking        */
+  float var_stable;  /* sigma^2_stable                                   */
+} plk_sf_params;
+int plk_slowfast_step(const plk_dims* dims, const plk_sf_params* params, const float* conf,
+                      uint8_t* masked, plk_sf_state* state, uint8_t* unmask_out,
+                      uint8_t* lock_out, void* stream);
+
+/*
  * S10 (proxy half)  proxy_cache[idx[j]] = proxy_new[idx[j]] for j < M = seg_ptr[B].
  * Both [B, N, r] fp32; rows not in idx are untouched.
  */

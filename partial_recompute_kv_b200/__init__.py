@@ -25,7 +25,8 @@ SEL_THRESH_GT, SEL_THRESH_LT, SEL_TOPK_LARGEST, SEL_TOPK_SMALLEST = 0, 1, 2, 3
 
 EXPORTED = (
     "plk_score_drift", "plk_select_active", "plk_layer_step_partial", "plk_full_layer_step",
-    "plk_proxy_commit", "plk_layer_step_partial_static", "plk_kl_lock", "plk_workspace_bytes", "plk_get_status",
+    "plk_proxy_commit", "plk_layer_step_partial_static", "plk_kl_lock", "plk_slowfast_step", "plk_workspace_bytes",
+    "plk_get_status",
     "plk_set_wait_limit",
     "plk_selftest_wait_timeout", "plk_trace_events", "plk_error_string", "plk_version",
 )
@@ -40,6 +41,15 @@ class PlkDims(ctypes.Structure):
 class PlkWeights(ctypes.Structure):
     _fields_ = [("g1", ctypes.c_void_p), ("w_qkv", ctypes.c_void_p), ("w_o", ctypes.c_void_p),
                 ("g2", ctypes.c_void_p), ("w_gu", ctypes.c_void_p), ("w_down", ctypes.c_void_p)]
+
+
+SF_HIST_MAX = 16
+SF_STATE_WORDS = 4 + SF_HIST_MAX  # plk_sf_state: phase, s, e, nslow, hist[16] (int32)
+
+
+class PlkSfParams(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_int), ("w_hist", ctypes.c_int), ("k_max", ctypes.c_int),
+                ("tau_conv", ctypes.c_float), ("tau_high", ctypes.c_float), ("var_stable", ctypes.c_float)]
 
 
 class PlkError(RuntimeError):
@@ -63,6 +73,7 @@ def _load():
         "plk_layer_step_partial_static": (I, [V, W, P, P, P, P, P, P, P]),
         "plk_proxy_commit": (I, [V, I, P, P, P, P, P]),
         "plk_kl_lock": (I, [V, I, P, P, P, P, F, F, P, P, P]),
+        "plk_slowfast_step": (I, [V, ctypes.POINTER(PlkSfParams), P, P, P, P, P, P]),
         "plk_workspace_bytes": (S, [V]),
         "plk_get_status": (I, [P]),
         "plk_set_wait_limit": (I, [L]),
@@ -188,6 +199,24 @@ def kl_lock(dm, V, logits_t, logits_prev, lock_in, lock_out, eps, h_max=math.inf
     _check(lib.plk_kl_lock(ctypes.byref(dm), int(V), _ptr(logits_t), _ptr(logits_prev), _ptr(lock_in),
                            _ptr(lock_out), float(eps), float(h_max), opt(kl_out), opt(h_out), _stream(stream)),
            "kl_lock")
+
+
+def sf_params(k=1, w_hist=2, k_max=8, tau_conv=0.5, tau_high=0.9, var_stable=1.0) -> PlkSfParams:
+    return PlkSfParams(int(k), int(w_hist), int(k_max), float(tau_conv), float(tau_high), float(var_stable))
+
+
+def sf_state(B, device="cuda"):
+    """Initial SlowFast state of B sequences: int32 [B, SF_STATE_WORDS] zeros (plk_sf_state rows)."""
+    return torch.zeros((int(B), SF_STATE_WORDS), dtype=torch.int32, device=device)
+
+
+def slowfast_step(dm, params, conf, masked, state, unmask_out=None, lock_out=None, stream=None):
+    """One SlowFast decoding step: conf [B, N] fp32, masked [B, N] uint8 (in/out),
+    state int32 [B, SF_STATE_WORDS] (in/out); unmask_out / lock_out [B, N] uint8 or None."""
+    if state.dtype != torch.int32 or state.shape[-1] != SF_STATE_WORDS:
+        raise ValueError("state must be int32 [B, %d]" % SF_STATE_WORDS)
+    _check(lib.plk_slowfast_step(ctypes.byref(dm), ctypes.byref(params), _ptr(conf), _ptr(masked), _ptr(state),
+                                 _ptr(unmask_out), _ptr(lock_out), _stream(stream)), "slowfast_step")
 
 
 def get_status(stream=None) -> int:

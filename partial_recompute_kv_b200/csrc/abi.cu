@@ -86,6 +86,21 @@ int plk_kl_lock(const plk_dims* dims, int V, const void* logits_t, const void* l
                         (cudaStream_t)stream);
 }
 
+int plk_slowfast_step(const plk_dims* dims, const plk_sf_params* params, const float* conf, uint8_t* masked,
+                      plk_sf_state* state, uint8_t* unmask_out, uint8_t* lock_out, void* stream) {
+  if (!dims || !params) return PLK_ERR_ARG;
+  if (dims->B < 1 || dims->N < 1 || dims->N > (1 << 20) || (long long)dims->B * dims->N >= (1LL << 31))
+    return PLK_ERR_SHAPE;
+  if (!conf || !masked || !state) return PLK_ERR_ARG;
+  if (params->k < 1 || params->w_hist < 1 || params->w_hist > PLK_SF_HIST_MAX || params->k_max < 1)
+    return PLK_ERR_ARG;
+  if (params->tau_conv != params->tau_conv || params->tau_high != params->tau_high ||
+      params->var_stable != params->var_stable)
+    return PLK_ERR_ARG;
+  if (unmask_out == masked || lock_out == masked || (unmask_out && unmask_out == lock_out)) return PLK_ERR_ARG;
+  return launch_slowfast(dims, params, conf, masked, state, unmask_out, lock_out, (cudaStream_t)stream);
+}
+
 int plk_layer_step_partial(const plk_dims* dims, const plk_weights* w, const void* X, const int32_t* idx,
                            const int32_t* seg_ptr, void* K_cache, void* V_cache, void* Y, void* workspace,
                            size_t ws_bytes, void* stream) {

@@ -8,3 +8,4 @@
 #include "abi.cu"
 #include "static_ws.cu"
 #include "kl_lock.cu"
+#include "slowfast.cu"

@@ -72,6 +72,9 @@ int launch_proxy_commit(const plk_dims* dims, int r, const int32_t* idx, const i
 int launch_kl_lock(const plk_dims* dims, int V, const void* logits_t, const void* logits_prev, const uint8_t* lock_in,
                    uint8_t* lock_out, float eps, float h_max, float* kl_out, float* h_out, cudaStream_t st);
 
+int launch_slowfast(const plk_dims* dims, const plk_sf_params* prm, const float* conf, uint8_t* masked,
+                    plk_sf_state* state, uint8_t* unmask_out, uint8_t* lock_out, cudaStream_t st);
+
 int run_layer(const plk_dims* dims, const plk_weights* w, const void* X, const int32_t* idx,
               const int32_t* seg_ptr, bool full, void* K_cache, void* V_cache, void* Y, void* ws,
               size_t ws_bytes, cudaStream_t st);

@@ -115,6 +115,65 @@ __device__ __forceinline__ uint32_t pref_key(float s, bool largest) {
   return largest ? k : ~k;
 }
 
+// Block-wide radix select on 8-bit digits of pref_key: the key *kth of the
+// keep_n-th most preferred candidate (cand(i) true, i < N) and the number
+// *remaining of candidates with exactly that key that are kept (the lowest
+// indices first).  Requires 0 < keep_n < candidates; every thread of the block
+// calls it.  hist[256], s_prefix and s_remaining are shared scratch.
+template <typename Cand>
+__device__ void block_radix_kth(const float* __restrict__ score, int N, int keep_n, bool largest, Cand cand,
+                                int* hist, uint32_t* s_prefix, int* s_remaining, uint32_t* kth, int* remaining) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t prefix = 0, pmask = 0;
+  int rem = keep_n;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int t = threadIdx.x; t < 256; t += blockDim.x) hist[t] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < N; i += blockDim.x) {
+      if (!cand(i)) continue;
+      const uint32_t key = pref_key(score[i], largest);
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l owns bins 255-8l .. 248-8l (descending); find the bin holding the
+      // rem-th most preferred key
+      int cnt[8], tot = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        cnt[j] = hist[255 - 8 * lane - j];
+        tot += cnt[j];
+      }
+      int inc = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += n;
+      }
+      int above = inc - tot;
+      if (above < rem && rem <= inc) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (above + cnt[j] >= rem) {
+            *s_prefix = prefix | ((uint32_t)(255 - 8 * lane - j) << shift);
+            *s_remaining = rem - above;
+            break;
+          }
+          above += cnt[j];
+        }
+      }
+    }
+    __syncthreads();
+    prefix = *s_prefix;
+    rem = *s_remaining;
+    pmask |= 0xFFu << shift;
+    __syncthreads();
+  }
+  *kth = prefix;
+  *remaining = rem;
+}
+
 // One CTA per sequence: among rows with lock_in == 0 keep the k most preferred
 // (ties to the lower index), lock every other row, and compact the kept rows.
 // Radix select on 8-bit digits finds the k-th key (warp-parallel bin search);
@@ -137,7 +196,6 @@ __global__ void __launch_bounds__(kSelThreads) topk_compact_kernel(const float* 
   const int b = blockIdx.x;
   const long long base = (long long)b * N;
   const bool lg = largest != 0;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int offset = 0;
   if (k > 0) {
     for (int bp = 0; bp < b; ++bp) {
@@ -155,53 +213,9 @@ __global__ void __launch_bounds__(kSelThreads) topk_compact_kernel(const float* 
   const bool keep_none = keep_n == 0;
   const bool keep_all = !keep_none && keep_n == ncand;
   if (!keep_none && !keep_all) {
-    uint32_t prefix = 0, pmask = 0;
-    remaining = keep_n;
-    for (int pass = 0; pass < 4; ++pass) {
-      const int shift = 24 - 8 * pass;
-      for (int t = threadIdx.x; t < 256; t += blockDim.x) hist[t] = 0;
-      __syncthreads();
-      for (int i = threadIdx.x; i < N; i += blockDim.x) {
-        if (lock_in[base + i]) continue;
-        const uint32_t key = pref_key(score[base + i], lg);
-        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
-      }
-      __syncthreads();
-      if (warp == 0) {
-        // lane l owns bins 255-8l .. 248-8l (descending); find the bin holding the
-        // remaining-th most preferred key
-        int cnt[8], tot = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          cnt[j] = hist[255 - 8 * lane - j];
-          tot += cnt[j];
-        }
-        int inc = tot;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const int n = __shfl_up_sync(0xffffffffu, inc, o);
-          if (lane >= o) inc += n;
-        }
-        int above = inc - tot;
-        if (above < remaining && remaining <= inc) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (above + cnt[j] >= remaining) {
-              s_prefix = prefix | ((uint32_t)(255 - 8 * lane - j) << shift);
-              s_remaining = remaining - above;
-              break;
-            }
-            above += cnt[j];
-          }
-        }
-      }
-      __syncthreads();
-      prefix = s_prefix;
-      remaining = s_remaining;
-      pmask |= 0xFFu << shift;
-      __syncthreads();
-    }
-    kth = prefix;
+    const uint8_t* lk = lock_in + base;
+    block_radix_kth(score + base, N, keep_n, lg, [lk](int i) { return lk[i] == 0; }, hist, &s_prefix,
+                    &s_remaining, &kth, &remaining);
   }
   // keep: candidates with key > kth, plus the first `remaining` with key == kth
   int taken_eq = 0, running = 0;

@@ -70,3 +70,27 @@ def test_host_validation_without_gpu(built):
     assert lib.plk_score_drift(ctypes.byref(ok), p, p, 8, p, 0, p, p, None) == plk.ERR_ARG  # out aliases cache
     assert lib.plk_set_wait_limit(0) == plk.ERR_ARG
     assert lib.plk_proxy_commit(ctypes.byref(ok), 0, p, p, p, p, None) == plk.ERR_ARG
+    # SlowFast policy: bad params, shapes and aliasing are refused before any launch
+    q = ctypes.c_void_p(32)
+    sfp = plk.sf_params()
+    assert lib.plk_slowfast_step(ctypes.byref(ok), None, p, p, p, None, None, None) == plk.ERR_ARG
+    assert lib.plk_slowfast_step(ctypes.byref(ok), ctypes.byref(sfp), None, p, p, None, None, None) == plk.ERR_ARG
+    for bad in (dict(k=0), dict(w_hist=0), dict(w_hist=plk.SF_HIST_MAX + 1), dict(k_max=0),
+                dict(tau_conv=float("nan")), dict(tau_high=float("nan")), dict(var_stable=float("nan"))):
+        bp = plk.sf_params(**bad)
+        assert lib.plk_slowfast_step(ctypes.byref(ok), ctypes.byref(bp), p, q, p, None, None, None) == \
+            plk.ERR_ARG, bad
+    assert lib.plk_slowfast_step(ctypes.byref(ok), ctypes.byref(sfp), p, q, p, q, None, None) == plk.ERR_ARG
+    assert lib.plk_slowfast_step(ctypes.byref(ok), ctypes.byref(sfp), p, q, p, None, q, None) == plk.ERR_ARG
+    assert lib.plk_slowfast_step(ctypes.byref(ok), ctypes.byref(sfp), p, q, p, p, p, None) == plk.ERR_ARG
+    long_seq = plk.dims(1, (1 << 20) + 1, 64, 4, 16, 64, dtype=plk.F32)
+    assert lib.plk_slowfast_step(ctypes.byref(long_seq), ctypes.byref(sfp), p, q, p, None, None, None) == \
+        plk.ERR_SHAPE
+
+
+def test_slowfast_state_layout_matches_header():
+    import partial_recompute_kv_b200 as plk
+    src = open(HEADER).read()
+    assert "#define PLK_SF_HIST_MAX %d" % plk.SF_HIST_MAX in src
+    assert plk.SF_STATE_WORDS == 4 + plk.SF_HIST_MAX
+    assert ctypes.sizeof(plk.PlkSfParams) == 24
