@@ -602,6 +602,106 @@ def run_kernel_configs(args):
     return 0
 
 
+# ---------------------------------------------------------------------------
+# the SlowFast span policy on its own (one call per decoding step), measured with
+# --kernel slowfast over whole decoding trajectories at the 32-layer stack's
+# batch (4 x 2048, 1024 generated) and the long-context sequence (1 x 8192, 256
+# generated), with K_max = 8, W_hist = 2, variance threshold 1.0
+# ---------------------------------------------------------------------------
+SF_SHAPES = ((4, 2048, 1024), (1, 8192, 7936))
+SF_PARAMS = dict(k=2, tau_conv=0.7, tau_high=0.9, var_stable=1.0, w_hist=2, k_max=8)
+
+
+def run_slowfast(args):
+    import torch
+    import partial_recompute_kv_b200 as plk
+    import oracle
+    import synth
+
+    dev = torch.device("cuda", 0)
+    pk = peaks()
+    hbm = float(pk["hbm_gbs"])
+    params, op = plk.sf_params(**SF_PARAMS), oracle.SpanParams(**SF_PARAMS)
+    lines = []
+    for B, N, prompt in SF_SHAPES:
+        dm = plk.dims(B, N, 64, 4, 16, 64, dtype=plk.F32)
+        m0 = torch.from_numpy(synth.generation_mask(B, N, prompt)).to(dev)
+        m, st = torch.empty_like(m0), plk.sf_state(B, device=dev)
+        un, lk = torch.empty_like(m0), torch.empty_like(m0)
+        confs = [torch.from_numpy(synth.span_confidences(B, N, t, seed=1, prompt=prompt)).to(dev)
+                 for t in range(N - prompt)]
+
+        def trajectory(events=None):
+            m.copy_(m0)
+            st.zero_()
+            for t, c in enumerate(confs):
+                if events is not None:
+                    events[t][0].record()
+                plk.slowfast_step(dm, params, c, m, st, un, lk)
+                if events is not None:
+                    events[t][1].record()
+            return m
+
+        trajectory()
+        torch.cuda.synchronize()
+        # the decode is over once nothing is masked; time the calls up to that step
+        m.copy_(m0)
+        st.zero_()
+        T = 0
+        for c in confs:
+            plk.slowfast_step(dm, params, c, m, st, un, lk)
+            T += 1
+            if not bool(m.any()):
+                break
+        confs = confs[:T]
+        for _ in range(max(args.warmup, 3) - 1):
+            trajectory()
+        torch.cuda.synchronize()
+        E = lambda: torch.cuda.Event(enable_timing=True)
+        reps = max(3, min(20, args.steps // max(T, 1) + 1))
+        us = []
+        with ClockSampler(0) as clk:
+            for _ in range(reps):
+                ev = [(E(), E()) for _ in range(T)]
+                trajectory(ev)
+                torch.cuda.synchronize()
+                us += [a.elapsed_time(b) * 1e3 for a, b in ev]
+        assert not bool(m.any()), "trajectory did not finish"
+        us_mean = statistics.mean(us)
+        alg = 8 * B * N  # conf 4 B, masked read + write, unmask and lock 1 B each per position
+        gbs = alg / (us_mean * 1e-6) / 1e9
+        # cpu baseline: the oracle over the first steps of the same trajectory (about 10 s at most)
+        mo = synth.generation_mask(B, N, prompt)
+        so = [oracle.SpanState() for _ in range(B)]
+        t0, n = time.perf_counter(), 0
+        for c in confs:
+            mo, _, _, so = oracle.slowfast_step(c.cpu().numpy(), mo, so, op)
+            n += 1
+            if time.perf_counter() - t0 > 10.0:
+                break
+        cpu_s = (time.perf_counter() - t0) / n
+        lines.append({"metric": "SlowFast policy steps/s", "value": 1e6 / us_mean, "unit": "steps/s",
+                      "n_gpus": 1, "steps": len(us), "warmup": args.warmup, "us_per_call": us_mean,
+                      "us_per_call_median": statistics.median(us), "higher_is_better": True, "dtype": "f32",
+                      "data": "synthetic",
+                      "config": {"workload": f"slowfast_step, B={B}, N={N}, {N - prompt} generated, "
+                                             f"{T} steps per decode, {reps} decodes",
+                                 **{kk: v for kk, v in SF_PARAMS.items()}},
+                      "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                                   "frac": gbs / hbm, "traffic": None, "kernel": "slowfast_kernel",
+                                   "alg_bytes_per_call": alg,
+                                   "note": "one CTA per sequence: launch- and latency-bound at these sizes"},
+                      "clocks": clk.summary(),
+                      "cpu_baseline": {"value": 1.0 / cpu_s, "unit": "steps/s", "cores": 1, "kind": "oracle",
+                                       "sample": f"the first {n} steps of the same decode"}})
+    s_ = plk.get_status()
+    if s_ != plk.OK:
+        raise RuntimeError(f"device status {plk.error_string(s_)}")
+    for ln in lines:
+        print(json.dumps(ln), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -615,9 +715,10 @@ def main():
                     help="replay the step as one captured CUDA graph (default)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="enqueue the step's library calls directly every step")
-    ap.add_argument("--kernel", choices=["step", "kl_lock", "configs"], default="step",
-                    help="step: the headline layer step; kl_lock: the KL lock rule alone; configs: scoring "
-                         "and the all-active stack step at the shapes where their rooflines are judged")
+    ap.add_argument("--kernel", choices=["step", "kl_lock", "slowfast", "configs"], default="step",
+                    help="step: the headline layer step; kl_lock: the KL lock rule alone; slowfast: the SlowFast "
+                         "span policy over whole decodes; configs: scoring and the all-active stack step at the "
+                         "shapes where their rooflines are judged")
     ap.add_argument("--profile", action="store_true",
                     help="set up and run --steps steps without timing or output (for ncu)")
     args = ap.parse_args()
@@ -628,6 +729,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.kernel == "kl_lock":
         return run_kl_lock(args) if rank == 0 else 0
+    if args.kernel == "slowfast":
+        return run_slowfast(args) if rank == 0 else 0
     if args.kernel == "configs":
         return run_kernel_configs(args) if rank == 0 else 0
     if args.impl == "reference":

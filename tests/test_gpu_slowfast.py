@@ -63,6 +63,7 @@ def _trajectory(B, N, prompt, steps, seed, rate=16.0, nan_every=0, outputs=True,
     (3, 2500, 100, dict(k=2, tau_conv=0.6, tau_high=0.85)),                 # ragged N, several tiles
     (2, 1000, 0, dict(k=1, w_hist=3, k_max=4, var_stable=50.0)),
     (5, 77, 5, dict(k=100, w_hist=1, k_max=1, tau_high=-np.inf)),            # k above the masked count
+    (5, 77, 5, dict(k=3, w_hist=1, k_max=1, tau_high=-np.inf)),              # every span decoded at once
     (2, 300, 30, dict(k=3, tau_high=np.inf, var_stable=np.inf)),             # always the fallback
     (4, 1024, 64, dict(k=4, w_hist=16, k_max=16, var_stable=400.0)),         # the largest window
 ])
