@@ -20,10 +20,13 @@
 //   lock_out marks the rows the next forward pass may skip: outside the span in
 //   the fast phase, none in the slow phase, all once nothing is masked.
 //
-// One CTA of 1024 threads per sequence, a handful of block-wide passes over the
-// sequence's N positions (counts, the end point, a radix select for the top-k,
-// the ordered write pass): latency-bound by design (a few microseconds for
-// N <= 8192), so no attempt is made to spread one sequence over several CTAs.
+// One CTA of 1024 threads per sequence (latency-bound: a few microseconds).
+// Up to 16384 positions the sequence's confidences and mask flags are staged
+// in shared memory in one pass whose loads are all independent, so the later
+// passes cost shared-memory latency only; reductions combine four values per
+// block barrier pair; k <= 16 positions are picked by k rounds of a block-wide
+// arg-max over (preference key, lower index) instead of the four-pass radix
+// select, which serves larger k and sequences too long to stage.
 // The variance test is exact: with end points below 2^20 and W_hist <= 16 the
 // integer W*S2 - S1^2 and var_stable*W^2 are exact doubles.
 #include <limits.h>
@@ -34,42 +37,68 @@
 namespace plk {
 
 constexpr int kSfThreads = 1024;
+constexpr int kSfStageMaxN = 16384;  // positions staged in shared memory (5 bytes each)
+constexpr int kSfRoundsMaxK = 16;    // top-k by repeated block arg-max up to this k
 
 struct SfArgs {
   int k, w_hist, k_max;
   float tau_conv, tau_high, var_stable;
 };
 
-__device__ __forceinline__ int block_max_int(int v, int* sh) {
+// Block reduction of (sum, sum, max, max) with one barrier pair; every thread
+// gets the result.  sh4 holds one entry per warp.
+__device__ __forceinline__ int4 block_reduce_ssmm(int4 v, int4* sh4) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
-  for (int o = 16; o; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
-  __syncthreads();
-  if (lane == 0) sh[warp] = v;
-  __syncthreads();
-  int t = (threadIdx.x < nw) ? sh[threadIdx.x] : INT_MIN;
-  if (warp == 0) {
-#pragma unroll
-    for (int o = 16; o; o >>= 1) t = max(t, __shfl_xor_sync(0xffffffffu, t, o));
-    if (lane == 0) sh[32] = t;
+  for (int o = 16; o; o >>= 1) {
+    v.x += __shfl_xor_sync(0xffffffffu, v.x, o);
+    v.y += __shfl_xor_sync(0xffffffffu, v.y, o);
+    v.z = max(v.z, __shfl_xor_sync(0xffffffffu, v.z, o));
+    v.w = max(v.w, __shfl_xor_sync(0xffffffffu, v.w, o));
   }
+  __syncthreads();  // earlier readers of sh4 are done
+  if (lane == 0) sh4[warp] = v;
   __syncthreads();
-  return sh[32];
+  int4 r = sh4[0];
+  for (int j = 1; j < nw; ++j) {
+    const int4 t = sh4[j];
+    r.x += t.x, r.y += t.y, r.z = max(r.z, t.z), r.w = max(r.w, t.w);
+  }
+  return r;
 }
 
+__device__ __forceinline__ unsigned long long block_max_u64(unsigned long long v, unsigned long long* sh8) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const unsigned long long t = __shfl_xor_sync(0xffffffffu, v, o);
+    v = t > v ? t : v;
+  }
+  __syncthreads();
+  if (lane == 0) sh8[warp] = v;
+  __syncthreads();
+  unsigned long long r = sh8[0];
+  for (int j = 1; j < nw; ++j) r = sh8[j] > r ? sh8[j] : r;
+  return r;
+}
+
+template <bool kStaged>
 __global__ void __launch_bounds__(kSfThreads) slowfast_kernel(const float* __restrict__ conf_all, uint8_t* masked_all,
                                                               plk_sf_state* states, int N, SfArgs p,
                                                               uint8_t* unmask_out, uint8_t* lock_out) {
+  extern __shared__ __align__(16) uint8_t sf_dyn[];
   __shared__ int hist[256];
   __shared__ int sh[33];
+  __shared__ int4 sh4[32];
+  __shared__ unsigned long long sh8[32];
   __shared__ uint32_t s_prefix;
   __shared__ int s_remaining;
   pdl_wait();
   pdl_trigger();
   const int b = blockIdx.x;
   const long long base = (long long)b * N;
-  const float* conf = conf_all + base;
-  uint8_t* masked = masked_all + base;
+  const float* conf_g = conf_all + base;
+  uint8_t* masked_g = masked_all + base;
   plk_sf_state* stp = states + b;
 
   // every thread reads the state; thread 0 writes it back at the end (after the
@@ -77,11 +106,21 @@ __global__ void __launch_bounds__(kSfThreads) slowfast_kernel(const float* __res
   int phase = stp->phase, s = stp->s, e = stp->e, nslow = stp->nslow;
   if ((phase != 0 && phase != 1) || nslow < 0) phase = 0, s = 0, e = 0, nslow = 0;
 
-  // pass 1: masked count and the first masked position
+  // pass 1 (staging): masked count and the first masked position
+  float* s_conf = reinterpret_cast<float*>(sf_dyn);
+  uint8_t* s_mask = sf_dyn + 4 * ((N + 15) & ~15);
   int cnt = 0, first = INT_MAX;
-  for (int i = threadIdx.x; i < N; i += blockDim.x)
-    if (masked[i]) ++cnt, first = min(first, i);
-  const int npend = block_sum(cnt, sh);
+#pragma unroll 4
+  for (int i = threadIdx.x; i < N; i += blockDim.x) {
+    const uint8_t mv = masked_g[i];
+    if (kStaged) {
+      s_conf[i] = conf_g[i];
+      s_mask[i] = mv;
+    }
+    if (mv) ++cnt, first = min(first, i);
+  }
+  const int4 r1 = block_reduce_ssmm(make_int4(cnt, 0, -first, INT_MIN), sh4);  // also publishes the staging
+  const int npend = r1.x;
   if (npend == 0) {  // nothing to decode: state unchanged, nothing to recompute
     for (int i = threadIdx.x; i < N; i += blockDim.x) {
       if (unmask_out) unmask_out[base + i] = 0;
@@ -89,25 +128,28 @@ __global__ void __launch_bounds__(kSfThreads) slowfast_kernel(const float* __res
     }
     return;
   }
-  first = -block_max_int(-first, sh);
+  first = -r1.z;
+  const float* cf = kStaged ? s_conf : conf_g;
+  const uint8_t* mk = kStaged ? s_mask : masked_g;
 
   const bool slow = phase == 0;
   if (slow && nslow == 0) s = first;
   const int lo = s, hi = slow ? N - 1 : e;
-  auto cand = [masked, lo, hi](int i) { return masked[i] != 0 && lo <= i && i <= hi; };
+  auto cand = [mk, lo, hi](int i) { return mk[i] != 0 && lo <= i && i <= hi; };
 
   // pass 2: candidates, the converged end point (slow) or the hot count (fast)
   int ccnt = 0, hcnt = 0, emax = -1;
   for (int i = threadIdx.x; i < N; i += blockDim.x) {
     if (!cand(i)) continue;
     ++ccnt;
-    const float c = conf[i];
+    const float c = cf[i];
     if (slow && c > p.tau_conv) emax = max(emax, i);  // NaN compares false
     if (!slow && c > p.tau_high) ++hcnt;
   }
-  const int ncand = block_sum(ccnt, sh);
-  const int nhot = slow ? 0 : block_sum(hcnt, sh);
-  const int end_t = slow ? block_max_int(emax, sh) : -1;
+  const int4 r2 = block_reduce_ssmm(make_int4(ccnt, hcnt, emax, INT_MIN), sh4);
+  const int ncand = r2.x;
+  const int nhot = slow ? 0 : r2.y;
+  const int end_t = slow ? r2.z : -1;
 
   // which rule unmasks: 0 nothing (empty span), 1 the hot positions, 2 top-k
   int rule = 2;
@@ -137,47 +179,73 @@ __global__ void __launch_bounds__(kSfThreads) slowfast_kernel(const float* __res
   }
   if (reset) phase = 0, s = 0, e = 0, nslow = 0;
 
-  // top-k threshold among the candidates
+  // the k most confident candidates (rule 2)
   const int keep_n = rule == 2 ? min(p.k, ncand) : 0;
-  const bool keep_all = keep_n == ncand;
+  const bool select = rule == 2 && keep_n > 0 && keep_n < ncand;  // else all candidates or none
+  const bool rounds = kStaged && select && keep_n <= kSfRoundsMaxK;
+  uint32_t mine = 0u;  // rounds: bit j = this thread's j-th position was picked
   uint32_t kth = 0u;
   int remaining = 0;
-  if (rule == 2 && keep_n > 0 && !keep_all)
-    block_radix_kth(conf, N, keep_n, true, cand, hist, &s_prefix, &s_remaining, &kth, &remaining);
+  if (rounds) {
+    // each round takes the most preferred candidate not yet taken: the largest
+    // (key << 32 | ~index), i.e. the largest key and among equal keys the lowest index
+    for (int r = 0; r < keep_n; ++r) {
+      unsigned long long best = 0ull;
+      int j = 0;
+      for (int i = threadIdx.x; i < N; i += blockDim.x, ++j) {
+        if (((mine >> j) & 1u) || !cand(i)) continue;
+        const unsigned long long v = ((unsigned long long)pref_key(cf[i], true) << 32) | (uint32_t)~i;
+        best = v > best ? v : best;
+      }
+      best = block_max_u64(best, sh8);  // > 0: keep_n < ncand leaves a candidate every round
+      const int w = (int)~(uint32_t)best;
+      if (w % (int)blockDim.x == (int)threadIdx.x) mine |= 1u << (w / (int)blockDim.x);
+    }
+  } else if (select) {
+    block_radix_kth(cf, N, keep_n, true, cand, hist, &s_prefix, &s_remaining, &kth, &remaining);
+  }
 
   // pass 3 (ordered): unmask, and count what is left in the span and overall
-  int taken_eq = 0, left_span = 0, left_all = 0;
-  for (int c0 = 0; c0 < N; c0 += blockDim.x) {
+  int taken_eq = 0, left_span = 0, left_all = 0, j = 0;
+  for (int c0 = 0; c0 < N; c0 += blockDim.x, ++j) {
     const int i = c0 + threadIdx.x;
     const bool in = i < N;
-    const bool m = in && masked[i] != 0;
+    const bool m = in && mk[i] != 0;
     const bool cd = in && cand(i);
-    const float c = in ? conf[i] : 0.f;
-    bool gt = false, eq = false;
-    if (rule == 2 && cd && keep_n > 0 && !keep_all) {
-      const uint32_t key = pref_key(c, true);
-      gt = key > kth;
-      eq = key == kth;
-    }
-    int total;
-    const int r = block_rank(eq ? 1 : 0, sh, &total);
+    const float c = in ? cf[i] : 0.f;
     bool take = false;
-    if (rule == 1) take = cd && c > p.tau_high;
-    if (rule == 2) take = cd && keep_n > 0 && (keep_all || gt || (eq && taken_eq + r < remaining));
-    taken_eq += total;
-    if (take) masked[i] = 0;
+    if (rule == 1) {
+      take = cd && c > p.tau_high;
+    } else if (rule == 2) {
+      if (!select) {
+        take = cd && keep_n > 0;
+      } else if (rounds) {
+        take = (mine >> j) & 1u;
+      } else {  // radix: keys above the k-th, then the first `remaining` equal ones in index order
+        bool gt = false, eq = false;
+        if (cd) {
+          const uint32_t key = pref_key(c, true);
+          gt = key > kth;
+          eq = key == kth;
+        }
+        int total;
+        const int r = block_rank(eq ? 1 : 0, sh, &total);
+        take = cd && (gt || (eq && taken_eq + r < remaining));
+        taken_eq += total;
+      }
+    }
+    if (take) masked_g[i] = 0;
     if (in && unmask_out) unmask_out[base + i] = take ? 1 : 0;
     const bool left = m && !take;
     left_all += left ? 1 : 0;
     left_span += (left && s <= i && i <= e) ? 1 : 0;
   }
-  left_all = block_sum(left_all, sh);
-  left_span = block_sum(left_span, sh);
-  if (phase == 1 && left_span == 0) phase = 0, s = 0, e = 0, nslow = 0;  // the span is decoded
+  const int4 r3 = block_reduce_ssmm(make_int4(left_all, left_span, INT_MIN, INT_MIN), sh4);
+  if (phase == 1 && r3.y == 0) phase = 0, s = 0, e = 0, nslow = 0;  // the span is decoded
 
   if (lock_out) {
     for (int i = threadIdx.x; i < N; i += blockDim.x)
-      lock_out[base + i] = left_all == 0 ? 1 : (phase == 1 ? ((s <= i && i <= e) ? 0 : 1) : 0);
+      lock_out[base + i] = r3.x == 0 ? 1 : (phase == 1 ? ((s <= i && i <= e) ? 0 : 1) : 0);
   }
   if (threadIdx.x == 0) {
     if (slot >= 0) stp->hist[slot] = end;
@@ -197,7 +265,17 @@ int launch_slowfast(const plk_dims* dims, const plk_sf_params* prm, const float*
   a.tau_conv = prm->tau_conv;
   a.tau_high = prm->tau_high;
   a.var_stable = prm->var_stable;
-  return launch_pdl(slowfast_kernel, dim3(dims->B), dim3(kSfThreads), 0, st, conf, masked, state, dims->N, a,
+  const int N = dims->N;
+  if (N <= kSfStageMaxN) {
+    const size_t dyn = (size_t)5 * ((N + 15) & ~15);
+    if (dyn > (40u << 10) &&
+        cudaFuncSetAttribute(slowfast_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn) !=
+            cudaSuccess)
+      return PLK_ERR_CUDA;
+    return launch_pdl(slowfast_kernel<true>, dim3(dims->B), dim3(kSfThreads), dyn, st, conf, masked, state, N, a,
+                      unmask_out, lock_out);
+  }
+  return launch_pdl(slowfast_kernel<false>, dim3(dims->B), dim3(kSfThreads), 0, st, conf, masked, state, N, a,
                     unmask_out, lock_out);
 }
 

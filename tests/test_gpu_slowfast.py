@@ -66,6 +66,8 @@ def _trajectory(B, N, prompt, steps, seed, rate=16.0, nan_every=0, outputs=True,
     (5, 77, 5, dict(k=3, w_hist=1, k_max=1, tau_high=-np.inf)),              # every span decoded at once
     (2, 300, 30, dict(k=3, tau_high=np.inf, var_stable=np.inf)),             # always the fallback
     (4, 1024, 64, dict(k=4, w_hist=16, k_max=16, var_stable=400.0)),         # the largest window
+    (2, 600, 40, dict(k=20, k_max=3, tau_conv=0.3, tau_high=0.97)),          # k > 16: radix select
+    (1, 20000, 19000, dict(k=3)),                                            # too long to stage in smem
 ])
 def test_slowfast_trajectory_matches_oracle(B, N, prompt, kw):
     steps, phases, left = _trajectory(B, N, prompt, 600, seed=B + N, **kw)
