@@ -20,7 +20,7 @@
 //   lock_out marks the rows the next forward pass may skip: outside the span in
 //   the fast phase, none in the slow phase, all once nothing is masked.
 //
-// One CTA of 1024 threads per sequence (latency-bound: a few microseconds).
+// One CTA of 512 threads per sequence (latency-bound: a few microseconds).
 // Up to 16384 positions the sequence's confidences and mask flags are staged
 // in shared memory in one pass whose loads are all independent, so the later
 // passes cost shared-memory latency only; reductions combine four values per
@@ -36,8 +36,8 @@
 
 namespace plk {
 
-constexpr int kSfThreads = 1024;
-constexpr int kSfStageMaxN = 16384;  // positions staged in shared memory (5 bytes each)
+constexpr int kSfThreads = 512;
+constexpr int kSfStageMaxN = 16384;  // positions staged in shared memory (5 bytes each): <= 32 per thread
 constexpr int kSfRoundsMaxK = 16;    // top-k by repeated block arg-max up to this k
 
 struct SfArgs {
@@ -45,10 +45,7 @@ struct SfArgs {
   float tau_conv, tau_high, var_stable;
 };
 
-// Block reduction of (sum, sum, max, max) with one barrier pair; every thread
-// gets the result.  sh4 holds one entry per warp.
-__device__ __forceinline__ int4 block_reduce_ssmm(int4 v, int4* sh4) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+__device__ __forceinline__ int4 warp_reduce_ssmm(int4 v) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) {
     v.x += __shfl_xor_sync(0xffffffffu, v.x, o);
@@ -56,30 +53,36 @@ __device__ __forceinline__ int4 block_reduce_ssmm(int4 v, int4* sh4) {
     v.z = max(v.z, __shfl_xor_sync(0xffffffffu, v.z, o));
     v.w = max(v.w, __shfl_xor_sync(0xffffffffu, v.w, o));
   }
+  return v;
+}
+
+// Block reduction of (sum, sum, max, max) with one barrier pair; every thread
+// gets the result (each warp re-reduces the per-warp partials, one per lane).
+__device__ __forceinline__ int4 block_reduce_ssmm(int4 v, int4* sh4) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_reduce_ssmm(v);
   __syncthreads();  // earlier readers of sh4 are done
   if (lane == 0) sh4[warp] = v;
   __syncthreads();
-  int4 r = sh4[0];
-  for (int j = 1; j < nw; ++j) {
-    const int4 t = sh4[j];
-    r.x += t.x, r.y += t.y, r.z = max(r.z, t.z), r.w = max(r.w, t.w);
-  }
-  return r;
+  return warp_reduce_ssmm(lane < nw ? sh4[lane] : make_int4(0, 0, INT_MIN, INT_MIN));
 }
 
-__device__ __forceinline__ unsigned long long block_max_u64(unsigned long long v, unsigned long long* sh8) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long v) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) {
     const unsigned long long t = __shfl_xor_sync(0xffffffffu, v, o);
     v = t > v ? t : v;
   }
+  return v;
+}
+
+__device__ __forceinline__ unsigned long long block_max_u64(unsigned long long v, unsigned long long* sh8) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_max_u64(v);
   __syncthreads();
   if (lane == 0) sh8[warp] = v;
   __syncthreads();
-  unsigned long long r = sh8[0];
-  for (int j = 1; j < nw; ++j) r = sh8[j] > r ? sh8[j] : r;
-  return r;
+  return warp_max_u64(lane < nw ? sh8[lane] : 0ull);
 }
 
 template <bool kStaged>
@@ -101,16 +104,19 @@ __global__ void __launch_bounds__(kSfThreads) slowfast_kernel(const float* __res
   uint8_t* masked_g = masked_all + base;
   plk_sf_state* stp = states + b;
 
-  // every thread reads the state; thread 0 writes it back at the end (after the
-  // last block-wide barrier, so no thread reads a half-written state)
+  // every thread reads the state (and the end-point ring, in flight with the
+  // staging loads); thread 0 writes it back at the end, after the last
+  // block-wide barrier, so no thread reads a half-written state
   int phase = stp->phase, s = stp->s, e = stp->e, nslow = stp->nslow;
-  if ((phase != 0 && phase != 1) || nslow < 0) phase = 0, s = 0, e = 0, nslow = 0;
+  int ring[PLK_SF_HIST_MAX];
+#pragma unroll
+  for (int j = 0; j < PLK_SF_HIST_MAX; ++j) ring[j] = j < p.w_hist ? stp->hist[j] : 0;
 
   // pass 1 (staging): masked count and the first masked position
   float* s_conf = reinterpret_cast<float*>(sf_dyn);
   uint8_t* s_mask = sf_dyn + 4 * ((N + 15) & ~15);
   int cnt = 0, first = INT_MAX;
-#pragma unroll 4
+#pragma unroll 8
   for (int i = threadIdx.x; i < N; i += blockDim.x) {
     const uint8_t mv = masked_g[i];
     if (kStaged) {
@@ -129,6 +135,7 @@ __global__ void __launch_bounds__(kSfThreads) slowfast_kernel(const float* __res
     return;
   }
   first = -r1.z;
+  if ((phase != 0 && phase != 1) || nslow < 0) phase = 0, s = 0, e = 0, nslow = 0;
   const float* cf = kStaged ? s_conf : conf_g;
   const uint8_t* mk = kStaged ? s_mask : masked_g;
 
@@ -167,8 +174,10 @@ __global__ void __launch_bounds__(kSfThreads) slowfast_kernel(const float* __res
       // population variance of the ring (the last w_hist end points) < var_stable,
       // as w*S2 - S1^2 < var_stable * w^2 (end points taken relative to s)
       double s1 = 0.0, s2 = 0.0;
-      for (int j = 0; j < p.w_hist; ++j) {
-        const double v = (double)((j == slot ? end : stp->hist[j]) - (long long)s);
+#pragma unroll
+      for (int j = 0; j < PLK_SF_HIST_MAX; ++j) {
+        if (j >= p.w_hist) break;
+        const double v = (double)((j == slot ? end : ring[j]) - (long long)s);
         s1 += v;
         s2 += v * v;
       }
