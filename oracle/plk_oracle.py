@@ -77,6 +77,12 @@ R9  SlowFast span policy ([SF] part 2), per sequence and per decoding step,
       caching): in the fast phase every row outside [s, e]; in the slow phase
       none; once nothing is masked, every row.  A sequence with nothing masked
       is left as it is.
+R10 Grouped-query attention (an optional layer variant, like R8): with
+    dims.Hkv > 0 dividing H, the projection makes H query heads and Hkv key and
+    value heads (w_qkv rows: d for Q, then Hkv*hd for K, then Hkv*hd for V) and
+    query head h attends with K/V head h // (H / Hkv), so consecutive query heads
+    share one K/V head.  The K/V caches hold Hkv*hd values per row.  Hkv = 0 or
+    Hkv = H is plain multi-head attention.
 R6  Precision policy "bf16": every tensor that the bf16 path stores in bf16
     between operations is rounded to bf16 here as well -- the normalised
     inputs of the projections (xn, hn), q, k, v (and so the K/V cache), the
@@ -101,7 +107,7 @@ __all__ = [
     "proxy_project", "drift_cosine", "drift_l2", "score_drift",
     "lock_threshold", "lock_topk", "compact", "log_softmax", "kl_divergence", "entropy", "kl_lock", "rope",
     "SpanParams", "SpanState", "population_variance", "slowfast_step_seq", "slowfast_step",
-    "full_layer_step", "layer_step_partial", "proxy_commit",
+    "full_layer_step", "layer_step_partial", "proxy_commit", "kv_heads",
     "LayerState", "tiny_run",
 ]
 
@@ -475,15 +481,26 @@ def rope(x, pos, H, hd, theta):
     return np.concatenate([x1 * c - x2 * s, x1 * s + x2 * c], axis=-1).reshape(-1, H * hd)
 
 
+def kv_heads(dims):
+    """R10: the layer's K/V heads, dims.Hkv when set, else H."""
+    return int(getattr(dims, "Hkv", 0) or dims.H)
+
+
 def _qk(qkv, dims, pos):
     """q and k of the projection output, rotated when the layer uses RoPE (R8)."""
-    d = dims.d
-    q, k = qkv[:, :d], qkv[:, d:2 * d]
+    d, dkv = dims.d, kv_heads(dims) * dims.hd
+    q, k = qkv[:, :d], qkv[:, d:d + dkv]
     theta = getattr(dims, "rope_theta", 0.0)
     if theta and theta > 0:
         q = rope(q, pos, dims.H, dims.hd, theta)
-        k = rope(k, pos, dims.H, dims.hd, theta)
+        k = rope(k, pos, kv_heads(dims), dims.hd, theta)
     return q, k
+
+
+def _kv_cols(h, dims):
+    """Columns of the K/V head that query head h attends with (R10)."""
+    g = h // (dims.H // kv_heads(dims))
+    return slice(g * dims.hd, (g + 1) * dims.hd)
 
 
 def _w(W, name):
@@ -498,30 +515,31 @@ def full_layer_step(dims, W, X, policy="f64"):
     Returns the LayerState (K, V, Y) of all rows.
     """
     B, N, d, H, hd, F = dims.B, dims.N, dims.d, dims.H, dims.hd, dims.F
+    dkv = kv_heads(dims) * hd
     x = np.asarray(X, dtype=np.float64).reshape(B * N, d)
     xn = _store(rmsnorm(x, W["g1"], dims.eps), policy)
     qkv = _mm(xn, _w(W, "w_qkv"))
     q, k = _qk(qkv, dims, np.arange(B * N) % N)
     q, k = _store(q, policy), _store(k, policy)
-    v = _store(qkv[:, 2 * d:], policy)
+    v = _store(qkv[:, d + dkv:], policy)
     a = np.zeros((B * N, d))
     scale = 1.0 / math.sqrt(hd)
     for b in range(B):
         rows = slice(b * N, (b + 1) * N)
         for h in range(H):
-            cols = slice(h * hd, (h + 1) * hd)
-            S = _mm(q[rows, cols], k[rows, cols]) * scale          # [N, N]
+            cols, kv = slice(h * hd, (h + 1) * hd), _kv_cols(h, dims)
+            S = _mm(q[rows, cols], k[rows, kv]) * scale          # [N, N]
             S = S - S.max(axis=1, keepdims=True)
             P = np.exp(S)
             P = P / P.sum(axis=1, keepdims=True)
-            a[rows, cols] = _mm(P, v[rows, cols].T)                # [N, hd]
+            a[rows, cols] = _mm(P, v[rows, kv].T)                # [N, hd]
     a = _store(a, policy)
     hres = x + _mm(a, _w(W, "w_o"))
     hn = _store(rmsnorm(hres, W["g2"], dims.eps), policy)
     gu = _mm(hn, _w(W, "w_gu"))
     act = _store(silu(gu[:, :F]) * gu[:, F:], policy)
     y = _store(hres + _mm(act, _w(W, "w_down")), policy)
-    return LayerState(k.reshape(B, N, d), v.reshape(B, N, d), y.reshape(B, N, d))
+    return LayerState(k.reshape(B, N, dkv), v.reshape(B, N, dkv), y.reshape(B, N, d))
 
 
 def layer_step_partial(dims, W, X, idx, seg_ptr, state, policy="f64", out_rows=None):
@@ -538,6 +556,7 @@ def layer_step_partial(dims, W, X, idx, seg_ptr, state, policy="f64", out_rows=N
     Returns a new LayerState; ``state`` is not modified.
     """
     B, N, d, H, hd, F = dims.B, dims.N, dims.d, dims.H, dims.hd, dims.F
+    dkv = kv_heads(dims) * hd
     idx = np.asarray(idx, dtype=np.int64)
     seg_ptr = np.asarray(seg_ptr, dtype=np.int64)
     out = state.copy()
@@ -552,10 +571,10 @@ def layer_step_partial(dims, W, X, idx, seg_ptr, state, policy="f64", out_rows=N
     qkv = _mm(xn, _w(W, "w_qkv"))
     q, k = _qk(qkv, dims, idx % N)
     q, k = _store(q, policy), _store(k, policy)
-    v = _store(qkv[:, 2 * d:], policy)
+    v = _store(qkv[:, d + dkv:], policy)
     # S6 K/V scatter into the cache rows of the active positions
-    Kf = out.K.reshape(B * N, d)
-    Vf = out.V.reshape(B * N, d)
+    Kf = out.K.reshape(B * N, dkv)
+    Vf = out.V.reshape(B * N, dkv)
     Kf[idx] = k
     Vf[idx] = v
     rows = np.arange(M) if out_rows is None else np.asarray(out_rows, dtype=np.int64)
@@ -568,12 +587,12 @@ def layer_step_partial(dims, W, X, idx, seg_ptr, state, policy="f64", out_rows=N
         Kb = Kf[b * N:(b + 1) * N]
         Vb = Vf[b * N:(b + 1) * N]
         for h in range(H):
-            cols = slice(h * hd, (h + 1) * hd)
-            s = _mm(q[j:j + 1, cols], Kb[:, cols])[0] * scale     # [N]
+            cols, kv = slice(h * hd, (h + 1) * hd), _kv_cols(h, dims)
+            s = _mm(q[j:j + 1, cols], Kb[:, kv])[0] * scale     # [N]
             s = s - s.max()
             p = np.exp(s)
             p = p / p.sum()
-            a[t, cols] = _mm(p[None, :], Vb[:, cols].T)[0]        # [hd]
+            a[t, cols] = _mm(p[None, :], Vb[:, kv].T)[0]        # [hd]
     a = _store(a, policy)
     # S8 output projection + residual
     hres = x[rows] + _mm(a, _w(W, "w_o"))

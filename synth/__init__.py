@@ -65,9 +65,16 @@ class Dims:
     eps: float = 1e-6
     dtype: str = "bf16"  # "bf16" or "f32"
     rope_theta: float = 0.0  # RoPE base for q and k; 0 = no rotary embedding
+    Hkv: int = 0  # K/V heads (grouped-query attention); 0 = one per query head
 
     def __post_init__(self):
         assert self.d == self.H * self.hd, "d must equal H*hd"
+        assert self.Hkv == 0 or (0 < self.Hkv <= self.H and self.H % self.Hkv == 0), "Hkv must divide H"
+
+    @property
+    def dkv(self) -> int:
+        """Width of the K and V rows: (Hkv or H) * hd."""
+        return (self.Hkv or self.H) * self.hd
 
 
 def _normal(rng, shape, std, dtype):
@@ -83,14 +90,15 @@ def _normal(rng, shape, std, dtype):
 def layer_weights(dims: Dims, std: float, seed: int = 0, layer: int = 0) -> dict:
     """Random-init weights of one layer, nn.Linear layout [out_features, in_features].
 
-    w_qkv [3d, d] (rows 0..d-1 produce Q, d..2d-1 K, 2d..3d-1 V), w_o [d, d],
+    w_qkv [d + 2 dkv, d] (rows 0..d-1 produce Q, then dkv rows K, then dkv rows V;
+    dkv = d unless the layer has fewer K/V heads), w_o [d, d],
     w_gu [2F, d] (rows 0..F-1 gate, F..2F-1 up), w_down [d, F]; RMSNorm gains g1, g2
     are ones.  Values are exactly representable in the workload's dtype.
     """
     rng = _rng(seed, S_WEIGHTS, layer)
     d, F, dt = dims.d, dims.F, dims.dtype
     w = {
-        "w_qkv": _normal(rng, (3 * d, d), std, dt),
+        "w_qkv": _normal(rng, (d + 2 * dims.dkv, d), std, dt),
         "w_o": _normal(rng, (d, d), std, dt),
         "w_gu": _normal(rng, (2 * F, d), std, dt),
         "w_down": _normal(rng, (d, F), std, dt),

@@ -21,8 +21,8 @@ import synth
 from oracle import plk_oracle as po
 
 
-def _dims(B=2, N=7, d=16, H=2, hd=8, F=24, dtype="f32"):
-    return synth.Dims(B=B, N=N, d=d, H=H, hd=hd, F=F, eps=1e-6, dtype=dtype)
+def _dims(B=2, N=7, d=16, H=2, hd=8, F=24, dtype="f32", Hkv=0, rope_theta=0.0):
+    return synth.Dims(B=B, N=N, d=d, H=H, hd=hd, F=F, eps=1e-6, dtype=dtype, Hkv=Hkv, rope_theta=rope_theta)
 
 
 def _weights(dims, std=None, seed=0):
@@ -75,10 +75,13 @@ def torch_block(dims, W, X):
     t = lambda a: torch.from_numpy(np.asarray(a, dtype=np.float64))
     x = t(X)
     xn = Fnn.rms_norm(x, (d,), t(W["g1"]), eps=dims.eps)
+    Hkv = dims.Hkv or H
     qkv = Fnn.linear(xn, t(W["w_qkv"]))
-    q, k, v = qkv.split(d, dim=-1)
-    heads = lambda z: z.reshape(B, N, H, hd).transpose(1, 2)
-    a = Fnn.scaled_dot_product_attention(heads(q), heads(k), heads(v), is_causal=False)
+    q, k, v = qkv.split([d, Hkv * hd, Hkv * hd], dim=-1)
+    heads = lambda z, n: z.reshape(B, N, n, hd).transpose(1, 2)
+    # grouped-query attention: torch repeats each K/V head for H / Hkv consecutive query heads
+    a = Fnn.scaled_dot_product_attention(heads(q, H), heads(k, Hkv), heads(v, Hkv), is_causal=False,
+                                         enable_gqa=Hkv != H)
     a = a.transpose(1, 2).reshape(B, N, d)
     h = x + Fnn.linear(a, t(W["w_o"]))
     hn = Fnn.rms_norm(h, (d,), t(W["g2"]), eps=dims.eps)
@@ -89,7 +92,10 @@ def torch_block(dims, W, X):
 
 @pytest.mark.parametrize("shape", [dict(B=1, N=9, d=16, H=2, hd=8, F=24),
                                    dict(B=3, N=5, d=12, H=3, hd=4, F=8),
-                                   dict(B=1, N=64, d=64, H=4, hd=16, F=256)])
+                                   dict(B=1, N=64, d=64, H=4, hd=16, F=256),
+                                   dict(B=2, N=7, d=16, H=4, hd=4, F=24, Hkv=2),   # grouped-query
+                                   dict(B=1, N=9, d=24, H=6, hd=4, F=8, Hkv=1),    # one K/V head
+                                   dict(B=2, N=6, d=24, H=6, hd=4, F=8, Hkv=3)])
 def test_full_step_matches_torch_composition(shape):
     dims = _dims(**shape)
     W = _weights(dims)
@@ -400,7 +406,7 @@ _PARTIAL_MUTANTS = [
     ("* scale     # [N]", "           # [N]"),
     ("q[j:j + 1, cols]", "q[0:1, cols]"),
     ("Kb = Kf[b * N:(b + 1) * N]", "Kb = Kf[0:N]"),
-    ("a[t, cols] = _mm(p[None, :], Vb[:, cols].T)[0]", "a[t, cols] = _mm(p[None, :], Kb[:, cols].T)[0]"),
+    ("a[t, cols] = _mm(p[None, :], Vb[:, kv].T)[0]", "a[t, cols] = _mm(p[None, :], Kb[:, kv].T)[0]"),
     ("out.Y.reshape(B * N, d)[idx[rows]] = y", "out.Y.reshape(B * N, d)[idx[rows]] = hres"),
 ]
 
@@ -565,3 +571,102 @@ def test_rope_partial_equals_full_and_keeps_locked_rows():
     part = oracle.layer_step_partial(dims, W, X, idx, seg, full, "f64")  # unchanged inputs
     for a, b in ((part.K, full.K), (part.V, full.V), (part.Y, full.Y)):
         assert np.max(np.abs(a - b)) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# grouped-query attention (an optional layer variant): fewer K/V heads than query heads
+# ---------------------------------------------------------------------------
+def _replicated_mha(dims, W):
+    """The MHA layer whose K and V weight rows repeat each K/V head for its group of query heads."""
+    d, hd, H, Hkv = dims.d, dims.hd, dims.H, dims.Hkv
+    g = H // Hkv
+    wq = np.asarray(W["w_qkv"], dtype=np.float64)
+    wk = wq[d:d + Hkv * hd].reshape(Hkv, hd, d)
+    wv = wq[d + Hkv * hd:].reshape(Hkv, hd, d)
+    rep = lambda w: np.repeat(w, g, axis=0).reshape(H * hd, d)
+    mdims = _dims(B=dims.B, N=dims.N, d=d, H=H, hd=hd, F=dims.F, rope_theta=dims.rope_theta)
+    return mdims, dict(W, w_qkv=np.concatenate([wq[:d], rep(wk), rep(wv)]))
+
+
+@pytest.mark.parametrize("H,Hkv,theta", [(4, 2, 0.0), (6, 1, 0.0), (6, 3, 100.0), (4, 4, 0.0)])
+def test_gqa_equals_mha_with_repeated_kv_heads(H, Hkv, theta):
+    hd = 4
+    dims = _dims(B=2, N=6, d=H * hd, H=H, hd=hd, F=12, Hkv=Hkv, rope_theta=theta)
+    W = _weights(dims, seed=21)
+    X = synth.hidden_states(dims, seed=21)
+    st = oracle.full_layer_step(dims, W, X, "f64")
+    mdims, mW = _replicated_mha(dims, W)
+    ref = oracle.full_layer_step(mdims, mW, X, "f64")
+    assert st.K.shape == (2, 6, Hkv * hd)
+    np.testing.assert_allclose(st.Y, ref.Y, rtol=0, atol=1e-12)
+    g = H // Hkv
+    heads = lambda z, n: z.reshape(2, 6, n, hd)
+    np.testing.assert_allclose(heads(st.K, Hkv), heads(ref.K, H)[:, :, ::g], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(heads(st.V, Hkv), heads(ref.V, H)[:, :, ::g], rtol=0, atol=1e-12)
+    # the partial step from the full step's caches, a subset active
+    lock = synth.bernoulli_active(2, 6, 0.5, seed=22)
+    idx, seg = oracle.compact(lock)
+    stale = oracle.LayerState(st.K * 0.5, st.V * 2.0, st.Y)
+    part = oracle.layer_step_partial(dims, W, X, idx, seg, stale, "f64")
+    mstale = oracle.LayerState(np.repeat(heads(stale.K, Hkv), g, axis=2).reshape(2, 6, H * hd),
+                               np.repeat(heads(stale.V, Hkv), g, axis=2).reshape(2, 6, H * hd), stale.Y)
+    mpart = oracle.layer_step_partial(mdims, mW, X, idx, seg, mstale, "f64")
+    np.testing.assert_allclose(part.Y, mpart.Y, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(heads(part.K, Hkv), heads(mpart.K, H)[:, :, ::g], rtol=0, atol=1e-12)
+
+
+def test_gqa_partial_with_all_rows_equals_full_and_keeps_locked_rows():
+    dims = _dims(B=2, N=8, d=16, H=4, hd=4, F=12, Hkv=2, rope_theta=50.0)
+    W = _weights(dims, seed=23)
+    X = synth.hidden_states(dims, seed=23)
+    full = oracle.full_layer_step(dims, W, X, "f64")
+    idx, seg = oracle.compact(np.zeros((2, 8), np.uint8))
+    zero = oracle.LayerState(np.zeros_like(full.K), np.zeros_like(full.V), np.zeros_like(full.Y))
+    part = oracle.layer_step_partial(dims, W, X, idx, seg, zero, "f64")
+    for a, b in ((part.K, full.K), (part.V, full.V), (part.Y, full.Y)):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-12)
+    lock = synth.bernoulli_active(2, 8, 0.4, seed=24)
+    idx, seg = oracle.compact(lock)
+    rng = np.random.default_rng(24)
+    st = oracle.LayerState(*(rng.standard_normal(a.shape) for a in (full.K, full.V, full.Y)))
+    out = oracle.layer_step_partial(dims, W, X, idx, seg, st, "f64")
+    locked = lock.astype(bool)
+    for new, old in ((out.K, st.K), (out.V, st.V), (out.Y, st.Y)):
+        assert _h(new[locked]) == _h(old[locked])
+
+
+@pytest.mark.parametrize("Hkv", [1, 2])
+def test_gqa_flop_count_closed_form(Hkv):
+    B, N, d, H, hd, F = 2, 8, 16, 4, 4, 12
+    dims = _dims(B=B, N=N, d=d, H=H, hd=hd, F=F, Hkv=Hkv)
+    dkv = Hkv * hd
+    W = _weights(dims)
+    X = synth.hidden_states(dims, seed=25)
+    with oracle.count_flops() as cf:
+        full = oracle.full_layer_step(dims, W, X, "f64")
+    per_row = 2 * d * (d + 2 * dkv) + 2 * d * d + 6 * d * F
+    assert cf.flops == B * (N * per_row + 4 * N * N * d)
+    lock = synth.bernoulli_active(B, N, 0.5, seed=25)
+    idx, seg = oracle.compact(lock)
+    with oracle.count_flops() as cp:
+        oracle.layer_step_partial(dims, W, X, idx, seg, full, "f64")
+    assert cp.flops == idx.size * per_row + 4 * idx.size * N * d
+
+
+@pytest.mark.parametrize("old,new", [
+    ("g = h // (dims.H // kv_heads(dims))", "g = h % kv_heads(dims)"),        # heads dealt round-robin
+    ("g = h // (dims.H // kv_heads(dims))", "g = h // kv_heads(dims)"),       # wrong group size
+])
+def test_gqa_head_mapping_mutants_are_caught(old, new):
+    dims = _dims(B=1, N=6, d=24, H=6, hd=4, F=8, Hkv=3)
+    W = _weights(dims, seed=26)
+    X = synth.hidden_states(dims, seed=26)
+    ns = dict(po.__dict__)
+    src = textwrap.dedent(inspect.getsource(po._kv_cols))
+    assert src.count(old) == 1
+    exec(compile(src.replace(old, new), "<mutant>", "exec"), ns)
+    for f in (po.full_layer_step, po.layer_step_partial):
+        exec(compile(textwrap.dedent(inspect.getsource(f)), "<oracle>", "exec"), ns)
+    st = ns["full_layer_step"](dims, W, X, "f64")
+    _, _, y = torch_block(dims, W, X)
+    assert np.max(np.abs(st.Y - y)) > 1e-6
