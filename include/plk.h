@@ -74,7 +74,8 @@ extern "C" {
 /* Shape of one layer: B sequences of N tokens, model dim d = H*hd, FFN dim F.
  * PLK_BF16 requires hd == 128, d % 256 == 0, F % 128 == 0 (the projection GEMM
  * computes 256-feature tiles on pairs of SMs).
- * PLK_F32 requires hd in {16, 32, 64, 128}.  B*N < 2^31. */
+ * PLK_F32 requires hd in {16, 32, 64, 128}.  B*N < 2^31.  0 <= Hkv <= H and,
+ * when Hkv > 0, H % Hkv == 0. */
 typedef struct {
   int B, N, d, H, hd, F;
   float eps;    /* RMSNorm epsilon                                      */
@@ -84,12 +85,18 @@ typedef struct {
                      * head of q and k of the token at position n of its
                      * sequence turns by n * theta^(-2i/hd) before it is
                      * stored (K is cached after the rotation).            */
+  int Hkv;      /* K/V heads (grouped-query attention): 0 or H = one per
+                 * query head; otherwise 0 < Hkv < H with H % Hkv == 0 and
+                 * query head h attends with K/V head h / (H / Hkv).  The
+                 * K/V rows are dkv = Hkv*hd wide (dkv = d when Hkv is 0). */
 } plk_dims;
 
 /* Layer weights, nn.Linear layout [out_features, in_features], row-major:
  *   g1, g2   [d]       RMSNorm gains
- *   w_qkv    [3d, d]   rows 0..d-1 -> Q, d..2d-1 -> K, 2d..3d-1 -> V;
- *                      head h of Q/K/V is columns h*hd .. h*hd+hd-1
+ *   w_qkv    [d + 2 dkv, d]  rows 0..d-1 -> Q, the next dkv rows -> K, the
+ *                      last dkv rows -> V (dkv = d without grouping: [3d, d]);
+ *                      head h of Q (K/V head g of K, V) is columns
+ *                      h*hd .. h*hd+hd-1 (g*hd .. g*hd+hd-1)
  *   w_o      [d, d]
  *   w_gu     [2F, d]   rows 0..F-1 gate, F..2F-1 up
  *   w_down   [d, F]
@@ -147,7 +154,9 @@ int plk_select_active(const plk_dims* dims, const float* score, const uint8_t* l
  *     h  = x_t + a W_o^T;  hn = RMSNorm(h) * g2
  *     Y[t] = h + (silu(hn W_g^T) * (hn W_u^T)) W_down^T
  *   Rows not in idx are not read as queries and their K_cache, V_cache and Y
- *   rows are never written.  K_cache, V_cache, Y: [B, N, d], in/out.
+ *   rows are never written.  K_cache, V_cache: [B, N, dkv]; Y: [B, N, d]; in/out.
+ *   With grouped-query attention (dims->Hkv > 0) the projection makes Hkv
+ *   K/V heads and query head h uses K/V head h / (H / Hkv).
  *   PLK_BF16 stores xn, q, k, v, a, hn and the SwiGLU product in bf16 (the
  *   residual stream h stays fp32).  M = 0 is a no-op.
  *   workspace: device buffer of at least plk_workspace_bytes(dims) bytes, any

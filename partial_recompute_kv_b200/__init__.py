@@ -35,7 +35,7 @@ EXPORTED = (
 class PlkDims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("N", ctypes.c_int), ("d", ctypes.c_int), ("H", ctypes.c_int),
                 ("hd", ctypes.c_int), ("F", ctypes.c_int), ("eps", ctypes.c_float), ("dtype", ctypes.c_int),
-                ("rope_theta", ctypes.c_float)]
+                ("rope_theta", ctypes.c_float), ("Hkv", ctypes.c_int)]
 
 
 class PlkWeights(ctypes.Structure):
@@ -123,8 +123,10 @@ def _check(code, where):
         raise PlkError(code, where)
 
 
-def dims(B, N, d, H, hd, F, eps=1e-6, dtype=BF16, rope_theta=0.0) -> PlkDims:
-    return PlkDims(int(B), int(N), int(d), int(H), int(hd), int(F), float(eps), int(dtype), float(rope_theta))
+def dims(B, N, d, H, hd, F, eps=1e-6, dtype=BF16, rope_theta=0.0, Hkv=0) -> PlkDims:
+    """Layer shape; Hkv > 0 selects grouped-query attention with Hkv K/V heads (K/V rows Hkv*hd wide)."""
+    return PlkDims(int(B), int(N), int(d), int(H), int(hd), int(F), float(eps), int(dtype), float(rope_theta),
+                   int(Hkv))
 
 
 def _ptr(t):

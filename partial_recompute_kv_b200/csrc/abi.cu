@@ -11,6 +11,7 @@ static int check_dims(const plk_dims* d) {
   if (d->dtype != PLK_F32 && d->dtype != PLK_BF16) return PLK_ERR_DTYPE;
   if (d->B < 1 || d->N < 1 || d->d < 1 || d->H < 1 || d->hd < 1 || d->F < 1) return PLK_ERR_SHAPE;
   if ((long long)d->H * d->hd != d->d) return PLK_ERR_SHAPE;
+  if (d->Hkv < 0 || d->Hkv > d->H || (d->Hkv > 0 && d->H % d->Hkv != 0)) return PLK_ERR_SHAPE;
   if ((long long)d->B * d->N >= (1LL << 31)) return PLK_ERR_SHAPE;
   if (!(d->eps >= 0.f)) return PLK_ERR_ARG;
   if (!(d->rope_theta >= 0.f) || d->rope_theta > 3.0e38f) return PLK_ERR_ARG;

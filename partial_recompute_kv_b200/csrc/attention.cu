@@ -19,7 +19,9 @@
 // query tiles alone leave SMs idle, the two CTAs of a cluster pair split a
 // tile's keys: the odd CTA hands its partial O, row max and row sum to the even
 // CTA through distributed shared memory, which merges and writes the tile.
-// Keys past N are masked.
+// Keys past N are masked.  Under grouped-query attention the K/V tiles of query
+// head h come from K/V head h / (H / Hkv) of the Hkv-head caches; the query
+// heads of a group are separate units whose K/V reads meet in L2.
 // fp32: one thread per (query row, head), online softmax, SIMT.
 #include <math.h>
 
@@ -143,7 +145,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
                                                                const __grid_constant__ CUtensorMap tmV,
                                                                __nv_bfloat16* __restrict__ Aout,
                                                                const int32_t* __restrict__ seg_ptr, int B, int N,
-                                                               int H, int d, float scale_log2) {
+                                                               int H, int d, int kv_group, float scale_log2) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // same offset in both CTAs
@@ -233,7 +235,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
       int t = 0;        // unit counter
       for (int u = plan.first; u < plan.units && !*s_abort; u += plan.stride, ++t) {
         const AttnUnit it = attn_unit(u, seg_ptr, B, H);
-        const int hc = it.h * kAttHD;
+        const int hc = it.h * kAttHD;                  // query head columns
+        const int kc = (it.h / kv_group) * kAttHD;     // its K/V head (grouped-query attention)
         if (!mbar_wait(q_free, (uint32_t)((t & 1) ^ 1))) {
           *s_abort = 1;
           break;
@@ -250,15 +253,15 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
             break;
           }
           mbar_expect_tx(&k_full[st], kAttKVBytes);
-          tma_load_2d(sK + st * kAttKVBytes, &tmK, hc, y, &k_full[st]);
-          tma_load_2d(sK + st * kAttKVBytes + kAttKVBytes / 2, &tmK, hc + 64, y, &k_full[st]);
+          tma_load_2d(sK + st * kAttKVBytes, &tmK, kc, y, &k_full[st]);
+          tma_load_2d(sK + st * kAttKVBytes + kAttKVBytes / 2, &tmK, kc + 64, y, &k_full[st]);
           if (!mbar_wait(&v_empty[st], ph ^ 1)) {
             *s_abort = 1;
             break;
           }
           mbar_expect_tx(&v_full[st], kAttKVBytes);
-          tma_load_2d(sV + st * kAttKVBytes, &tmV, hc, y, &v_full[st]);
-          tma_load_2d(sV + st * kAttKVBytes + kAttKVBytes / 2, &tmV, hc + 64, y, &v_full[st]);
+          tma_load_2d(sV + st * kAttKVBytes, &tmV, kc, y, &v_full[st]);
+          tma_load_2d(sV + st * kAttKVBytes + kAttKVBytes / 2, &tmV, kc + 64, y, &v_full[st]);
         }
       }
     }
@@ -542,7 +545,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
 template <int HD>
 __global__ void attn_f32_kernel(const float* __restrict__ Q, const float* __restrict__ K,
                                 const float* __restrict__ V, float* __restrict__ A,
-                                const int32_t* __restrict__ seg_ptr, int B, int N, int d, int H, float scale) {
+                                const int32_t* __restrict__ seg_ptr, int B, int N, int d, int H, int dkv,
+                                int kv_group, float scale) {
   const int gid = blockIdx.x * blockDim.x + threadIdx.x;
   const int j = gid / H, h = gid - j * H;
   const int M = seg_ptr[B];
@@ -557,8 +561,8 @@ __global__ void attn_f32_kernel(const float* __restrict__ Q, const float* __rest
   }
   float m = -INFINITY, l = 0.f;
   for (int n = 0; n < N; ++n) {
-    const float* kr = K + ((size_t)b * N + n) * d + h * HD;
-    const float* vr = V + ((size_t)b * N + n) * d + h * HD;
+    const float* kr = K + ((size_t)b * N + n) * dkv + (h / kv_group) * HD;
+    const float* vr = V + ((size_t)b * N + n) * dkv + (h / kv_group) * HD;
     float s = 0.f;
 #pragma unroll
     for (int c = 0; c < HD; ++c) s = fmaf(q[c], kr[c], s);
@@ -577,11 +581,11 @@ __global__ void attn_f32_kernel(const float* __restrict__ Q, const float* __rest
 
 int launch_attention_bf16(const plk_dims* dims, const void* q, const void* K_cache, const void* V_cache,
                           void* a_out, const int32_t* seg_ptr, int num_sms, cudaStream_t st) {
-  const int B = dims->B, N = dims->N, d = dims->d, H = dims->H;
+  const int B = dims->B, N = dims->N, d = dims->d, H = dims->H, dkv = kv_width(dims);
   CUtensorMap tmQ, tmK, tmV;
   if (make_tmap_bf16(&tmQ, q, (uint64_t)B * N, (uint64_t)d, kAttBQ) != PLK_OK) return PLK_ERR_CUDA;
-  if (make_tmap_bf16(&tmK, K_cache, (uint64_t)B * N, (uint64_t)d, kAttBK) != PLK_OK) return PLK_ERR_CUDA;
-  if (make_tmap_bf16(&tmV, V_cache, (uint64_t)B * N, (uint64_t)d, kAttBK) != PLK_OK) return PLK_ERR_CUDA;
+  if (make_tmap_bf16(&tmK, K_cache, (uint64_t)B * N, (uint64_t)dkv, kAttBK) != PLK_OK) return PLK_ERR_CUDA;
+  if (make_tmap_bf16(&tmV, V_cache, (uint64_t)B * N, (uint64_t)dkv, kAttBK) != PLK_OK) return PLK_ERR_CUDA;
   static int attr_done[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PLK_ERR_CUDA;
@@ -607,7 +611,7 @@ int launch_attention_bf16(const plk_dims* dims, const void* q, const void* K_cac
   cfg.attrs = at;
   cfg.numAttrs = 2;
   if (cudaLaunchKernelEx(&cfg, attn_tc_kernel, tmQ, tmK, tmV, (__nv_bfloat16*)a_out, seg_ptr, B, N, H, d,
-                         scale_log2) != cudaSuccess)
+                         H / kv_heads(dims), scale_log2) != cudaSuccess)
     return PLK_ERR_CUDA;
   return PLK_OK;
 }
@@ -615,13 +619,22 @@ int launch_attention_bf16(const plk_dims* dims, const void* q, const void* K_cac
 int launch_attention_f32(const plk_dims* dims, const float* q, const float* K_cache, const float* V_cache,
                          float* a_out, const int32_t* seg_ptr, int Mcap, cudaStream_t st) {
   const int B = dims->B, N = dims->N, d = dims->d, H = dims->H, hd = dims->hd;
+  const int dkv = kv_width(dims), g = H / kv_heads(dims);
   const float scale = (float)(1.0 / sqrt((double)hd));
   const int threads = 128, blocks = ceil_div(Mcap * H, threads);
   switch (hd) {
-    case 16: attn_f32_kernel<16><<<blocks, threads, 0, st>>>(q, K_cache, V_cache, a_out, seg_ptr, B, N, d, H, scale); break;
-    case 32: attn_f32_kernel<32><<<blocks, threads, 0, st>>>(q, K_cache, V_cache, a_out, seg_ptr, B, N, d, H, scale); break;
-    case 64: attn_f32_kernel<64><<<blocks, threads, 0, st>>>(q, K_cache, V_cache, a_out, seg_ptr, B, N, d, H, scale); break;
-    case 128: attn_f32_kernel<128><<<blocks, threads, 0, st>>>(q, K_cache, V_cache, a_out, seg_ptr, B, N, d, H, scale); break;
+    case 16:
+      attn_f32_kernel<16><<<blocks, threads, 0, st>>>(q, K_cache, V_cache, a_out, seg_ptr, B, N, d, H, dkv, g, scale);
+      break;
+    case 32:
+      attn_f32_kernel<32><<<blocks, threads, 0, st>>>(q, K_cache, V_cache, a_out, seg_ptr, B, N, d, H, dkv, g, scale);
+      break;
+    case 64:
+      attn_f32_kernel<64><<<blocks, threads, 0, st>>>(q, K_cache, V_cache, a_out, seg_ptr, B, N, d, H, dkv, g, scale);
+      break;
+    case 128:
+      attn_f32_kernel<128><<<blocks, threads, 0, st>>>(q, K_cache, V_cache, a_out, seg_ptr, B, N, d, H, dkv, g, scale);
+      break;
     default: return PLK_ERR_SHAPE;
   }
   return cudaPeekAtLastError() == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;

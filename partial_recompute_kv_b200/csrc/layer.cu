@@ -63,7 +63,7 @@ Workspace workspace_layout(const plk_dims* dm, int num_sms) {
   w.hn = take(es * Mcap * d);
   w.act = take(es * Mcap * F);
   w.num_sms = num_sms;
-  w.c32 = take(4 * Mcap * std::max((size_t)3 * d, 2 * F));
+  w.c32 = take(4 * Mcap * std::max(d + 2 * (size_t)kv_width(dm), 2 * F));
   w.total = off;
   return w;
 }
@@ -312,31 +312,38 @@ __device__ __forceinline__ void rope_cs(int pos, int i, int hd, float log2_theta
   sincosf((float)a, &s, &c);
 }
 
-// [q | k | v] sums of compact row j -> Q[j] (compact), K/V cache rows idx[j];
-// with RoPE (log2_theta > 0) q and k are rotated by the row's position idx[j] % N
+// [q | k | v] sums of compact row j (d + 2 dkv wide) -> Q[j] (compact, d wide) and
+// the K/V cache rows idx[j] (dkv wide: Hkv heads under grouped-query attention);
+// with RoPE (log2_theta > 0) the heads of q and k are rotated by the row's
+// position idx[j] % N
 __global__ void __launch_bounds__(256) finish_qkv_kernel(const float* __restrict__ qkv32,
                                                          const int32_t* __restrict__ idx,
                                                          const int32_t* __restrict__ seg_ptr, int B, int N, int d,
-                                                         int hd, float log2_theta, __nv_bfloat16* __restrict__ q,
+                                                         int dkv, int hd, float log2_theta,
+                                                         __nv_bfloat16* __restrict__ q,
                                                          __nv_bfloat16* __restrict__ Kc,
                                                          __nv_bfloat16* __restrict__ Vc) {
   pdl_wait();
   pdl_trigger();
   const int M = seg_ptr[B];
   const bool rope = log2_theta > 0.f;
-  const int npair = rope ? d / 8 : 0;  // q and k: 8 pairs (x_i, x_{i+hd/2}) per unit
-  const int nv = 3 * d / 8;
+  const int W = d + 2 * dkv;
+  const int qunits = d / 16;                        // 8 pairs (x_i, x_{i+hd/2}) per unit
+  const int npair = rope ? qunits + dkv / 16 : 0;  // the q heads, then the k heads
+  const int nv = W / 8;
   for (int j = blockIdx.x; j < M; j += gridDim.x) {
     const size_t row = (size_t)idx[j];
-    const float* src = qkv32 + (size_t)j * 3 * d;
+    const float* src = qkv32 + (size_t)j * W;
     const int pos = (int)(row % (size_t)N);
     for (int u = threadIdx.x; u < npair; u += blockDim.x) {
-      const int per_part = d / 16, part = u / per_part, rem = u - part * per_part;
+      const bool isq = u < qunits;
+      const int rem = isq ? u : u - qunits;
       const int h = rem / (hd / 16), i0 = (rem - h * (hd / 16)) * 8;
       const int c1 = h * hd + i0, c2 = c1 + hd / 2;
+      const float* part = src + (isq ? 0 : d);
       float x1[8], x2[8];
-      load8(src + part * d + c1, x1);
-      load8(src + part * d + c2, x2);
+      load8(part + c1, x1);
+      load8(part + c2, x2);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         float cs, sn;
@@ -345,16 +352,17 @@ __global__ void __launch_bounds__(256) finish_qkv_kernel(const float* __restrict
         x1[e] = a * cs - b * sn;
         x2[e] = a * sn + b * cs;
       }
-      __nv_bfloat16* dst = part == 0 ? q + (size_t)j * d : Kc + row * d;
+      __nv_bfloat16* dst = isq ? q + (size_t)j * d : Kc + row * dkv;
       store_vec<__nv_bfloat16, 8>(dst + c1, x1);
       store_vec<__nv_bfloat16, 8>(dst + c2, x2);
     }
-    for (int v = threadIdx.x + (rope ? d / 4 : 0); v < nv; v += blockDim.x) {  // with RoPE: v only
-      const int c = v * 8, part = c / d, col = c - part * d;
+    for (int v = threadIdx.x + (rope ? (d + dkv) / 8 : 0); v < nv; v += blockDim.x) {  // with RoPE: v only
+      const int c = v * 8;
       float f[8];
       load8(src + c, f);
-      __nv_bfloat16* dst = part == 0 ? q + (size_t)j * d : (part == 1 ? Kc : Vc) + row * d;
-      store_vec<__nv_bfloat16, 8>(dst + col, f);
+      __nv_bfloat16* dst = c < d ? q + (size_t)j * d + c
+                                 : (c < d + dkv ? Kc + row * dkv + (c - d) : Vc + row * dkv + (c - d - dkv));
+      store_vec<__nv_bfloat16, 8>(dst, f);
     }
   }
 }
@@ -446,31 +454,34 @@ __global__ void __launch_bounds__(256) epilogue_f32_kernel(int mode, const float
                                                            const int32_t* __restrict__ idx,
                                                            const int32_t* __restrict__ seg_ptr, int B, int d, int F,
                                                            float* q, float* kc, float* vc, const float* x, float* h32,
-                                                           float* act, float* y, int N, int hd, float log2_theta) {
+                                                           float* act, float* y, int N, int hd, float log2_theta,
+                                                           int dkv) {
   const int M = seg_ptr[B];
   const int j = blockIdx.x;
   if (j >= M) return;
   const size_t row = (size_t)idx[j];
-  if (mode == F32_QKV) {
-    const float* c = C + (size_t)j * 3 * d;
-    if (log2_theta > 0.f) {  // RoPE on q and k: pair (t, t + hd/2) of a head
+  if (mode == F32_QKV) {  // [q | k | v] row of width d + 2 dkv; K/V cache rows dkv wide
+    const float* c = C + (size_t)j * (d + 2 * dkv);
+    if (log2_theta > 0.f) {  // RoPE on the q heads, then the k heads: pair (t, t + hd/2) of a head
       const int pos = (int)(row % (size_t)N), half = hd / 2;
-      for (int u = threadIdx.x; u < d / 2; u += blockDim.x) {
-        const int h = u / half, i = u - h * half, t1 = h * hd + i, t2 = t1 + half;
+      for (int u = threadIdx.x; u < (d + dkv) / 2; u += blockDim.x) {
+        const bool isq = u < d / 2;
+        const int uu = isq ? u : u - d / 2;
+        const int h = uu / half, i = uu - h * half, t1 = h * hd + i, t2 = t1 + half;
         float cs, sn;
         rope_cs(pos, i, hd, log2_theta, cs, sn);
-        q[(size_t)j * d + t1] = c[t1] * cs - c[t2] * sn;
-        q[(size_t)j * d + t2] = c[t1] * sn + c[t2] * cs;
-        kc[row * d + t1] = c[d + t1] * cs - c[d + t2] * sn;
-        kc[row * d + t2] = c[d + t1] * sn + c[d + t2] * cs;
+        const float* src = c + (isq ? 0 : d);
+        float* dst = isq ? q + (size_t)j * d : kc + row * dkv;
+        dst[t1] = src[t1] * cs - src[t2] * sn;
+        dst[t2] = src[t1] * sn + src[t2] * cs;
       }
-      for (int t = threadIdx.x; t < d; t += blockDim.x) vc[row * d + t] = c[2 * d + t];
+      for (int t = threadIdx.x; t < dkv; t += blockDim.x) vc[row * dkv + t] = c[d + dkv + t];
       return;
     }
-    for (int t = threadIdx.x; t < d; t += blockDim.x) {
-      q[(size_t)j * d + t] = c[t];
-      kc[row * d + t] = c[d + t];
-      vc[row * d + t] = c[2 * d + t];
+    for (int t = threadIdx.x; t < d; t += blockDim.x) q[(size_t)j * d + t] = c[t];
+    for (int t = threadIdx.x; t < dkv; t += blockDim.x) {
+      kc[row * dkv + t] = c[d + t];
+      vc[row * dkv + t] = c[d + dkv + t];
     }
   } else if (mode == F32_O) {
     for (int t = threadIdx.x; t < d; t += blockDim.x)
@@ -501,7 +512,7 @@ __global__ void __launch_bounds__(256) epilogue_f32_kernel(int mode, const float
 static int run_layer_f32(const plk_dims* dm, const plk_weights* w, const float* X, const int32_t* idx,
                          const int32_t* seg, float* Kc, float* Vc, float* Y, uint8_t* ws, const Workspace& L,
                          cudaStream_t st) {
-  const int B = dm->B, d = dm->d, F = dm->F, Mcap = dm->B * dm->N;
+  const int B = dm->B, d = dm->d, F = dm->F, Mcap = dm->B * dm->N, dkv = kv_width(dm);
   float* xn = (float*)(ws + L.xn);
   float* q = (float*)(ws + L.q);
   float* a = (float*)(ws + L.a);
@@ -515,18 +526,19 @@ static int run_layer_f32(const plk_dims* dm, const plk_weights* w, const float* 
     gemm_f32_kernel<<<grid, 256, 0, st>>>(A, (const float*)Wt, c32, Nout, K, seg, B);
   };
   PLK_TRY(launch_rmsnorm<float, float, float>(X, idx, seg, B, (const float*)w->g1, dm->eps, d, xn, Mcap, st));
-  gemm(xn, w->w_qkv, 3 * d, d);
+  gemm(xn, w->w_qkv, d + 2 * dkv, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_QKV, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, dm->N,
-                                            dm->hd, dm->rope_theta > 0.f ? log2f(dm->rope_theta) : 0.f);
+                                            dm->hd, dm->rope_theta > 0.f ? log2f(dm->rope_theta) : 0.f, dkv);
   PLK_LAUNCHED();
   PLK_TRY(launch_attention_f32(dm, q, Kc, Vc, a, seg, Mcap, st));
   gemm(a, w->w_o, d, d);
-  epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_O, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, 0, 0, 0.f);
+  epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_O, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, 0, 0, 0.f, 0);
   PLK_TRY(launch_rmsnorm<float, float, float>(h32, nullptr, seg, B, (const float*)w->g2, dm->eps, d, hn, Mcap, st));
   gemm(hn, w->w_gu, 2 * F, d);
-  epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_GU, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, 0, 0, 0.f);
+  epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_GU, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, 0, 0, 0.f, 0);
   gemm(act, w->w_down, d, F);
-  epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_DOWN, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, 0, 0, 0.f);
+  epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_DOWN, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, 0, 0, 0.f,
+                                            0);
   PLK_LAUNCHED();
   return PLK_OK;
 }
@@ -534,7 +546,7 @@ static int run_layer_f32(const plk_dims* dm, const plk_weights* w, const float* 
 static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_bfloat16* X, const int32_t* idx,
                           const int32_t* seg, void* Kc, void* Vc, void* Y, uint8_t* ws, const Workspace& L,
                           cudaStream_t st) {
-  const int B = dm->B, d = dm->d, F = dm->F, Mcap = dm->B * dm->N;
+  const int B = dm->B, d = dm->d, F = dm->F, Mcap = dm->B * dm->N, dkv = kv_width(dm);
   __nv_bfloat16* xn = (__nv_bfloat16*)(ws + L.xn);
   __nv_bfloat16* q = (__nv_bfloat16*)(ws + L.q);
   __nv_bfloat16* a = (__nv_bfloat16*)(ws + L.a);
@@ -542,10 +554,10 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   __nv_bfloat16* hn = (__nv_bfloat16*)(ws + L.hn);
   __nv_bfloat16* act = (__nv_bfloat16*)(ws + L.act);
 
-  float* c32 = (float*)(ws + L.c32);  // [Mcap, 3d] QKV sums, later [Mcap, 2F] gate/up sums
+  float* c32 = (float*)(ws + L.c32);  // [Mcap, d + 2 dkv] QKV sums, later [Mcap, 2F] gate/up sums
 
   CUtensorMap tW_qkv, tW_o, tW_gu, tW_down, tX_xn, tX_a, tX_hn, tX_act, tO_qkv, tO_h, tO_gu;
-  PLK_TRY(make_tmap_bf16(&tW_qkv, w->w_qkv, 3ull * d, d, 64));
+  PLK_TRY(make_tmap_bf16(&tW_qkv, w->w_qkv, (uint64_t)d + 2ull * dkv, d, 64));
   PLK_TRY(make_tmap_bf16(&tW_o, w->w_o, (uint64_t)d, d, 64));
   PLK_TRY(make_tmap_bf16(&tW_gu, w->w_gu, 2ull * F, d, 64));
   PLK_TRY(make_tmap_bf16(&tW_down, w->w_down, (uint64_t)d, F, 64));
@@ -553,7 +565,7 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   PLK_TRY(make_tmap_bf16(&tX_a, a, (uint64_t)Mcap, d, 64));
   PLK_TRY(make_tmap_bf16(&tX_hn, hn, (uint64_t)Mcap, d, 64));
   PLK_TRY(make_tmap_bf16(&tX_act, act, (uint64_t)Mcap, F, 64));
-  PLK_TRY(make_tmap_f32(&tO_qkv, c32, (uint64_t)Mcap, 3ull * d));
+  PLK_TRY(make_tmap_f32(&tO_qkv, c32, (uint64_t)Mcap, (uint64_t)d + 2ull * dkv));
   PLK_TRY(make_tmap_f32(&tO_h, h32, (uint64_t)Mcap, d));
   PLK_TRY(make_tmap_f32(&tO_gu, c32, (uint64_t)Mcap, 2ull * F));
 
@@ -566,18 +578,19 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   trace_mark(0, st);
   // x (fp32) staged in h32 takes the O projection's adds; the QKV sums start at 0
   PLK_TRY(launch_rmsnorm<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(X, idx, seg, B, (const __nv_bfloat16*)w->g1,
-                                                                      dm->eps, d, xn, Mcap, st, h32, c32, 3 * d));
+                                                                      dm->eps, d, xn, Mcap, st, h32, c32,
+                                                                      d + 2 * dkv));
   trace_mark(1, st);
 
   g.K = d;
-  g.ftiles = 3 * d / kGemmBM;
+  g.ftiles = (d + 2 * dkv) / kGemmBM;
   g.gu_F = 0;
   PLK_TRY(launch_gemm_tc(tW_qkv, tX_xn, tO_qkv, g, st));
   trace_mark(2, st);
 
   const float log2_theta = dm->rope_theta > 0.f ? log2f(dm->rope_theta) : 0.f;
   PLK_TRY(launch_pdl(finish_qkv_kernel, dim3(rgrid), dim3(256), 0, st, (const float*)c32, idx, seg, B, dm->N, d,
-                     dm->hd, log2_theta, q, (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc));
+                     dkv, dm->hd, log2_theta, q, (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc));
   trace_mark(3, st);
 
   PLK_TRY(launch_attention_bf16(dm, q, Kc, Vc, a, seg, L.num_sms, st));

@@ -20,6 +20,10 @@ constexpr int kGemmBK = 64;       // K per stage: one 128-byte swizzle row of bf
 constexpr int kGemmStages = 6;
 constexpr int kGemmThreads = 192; // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 
+// ---- grouped-query attention --------------------------------------------------
+inline int kv_heads(const plk_dims* d) { return d->Hkv > 0 ? d->Hkv : d->H; }
+inline int kv_width(const plk_dims* d) { return kv_heads(d) * d->hd; }  // dkv: K and V row width
+
 // ---- launch with programmatic stream serialization ---------------------------
 // The kernel may start while its predecessor in the stream finishes; it orders
 // itself with pdl_wait() (plk_common.cuh).

@@ -60,6 +60,11 @@ def test_host_validation_without_gpu(built):
     assert lib.plk_workspace_bytes(ctypes.byref(bad_ffn)) == 0
     bad_split = plk.dims(1, 8, 64, 3, 16, 64, dtype=plk.F32)  # d != H * hd
     assert lib.plk_workspace_bytes(ctypes.byref(bad_split)) == 0
+    # grouped-query attention: 0 <= Hkv <= H and H % Hkv == 0 (checked before the null weights)
+    for hkv, code in ((3, plk.ERR_SHAPE), (8, plk.ERR_SHAPE), (-1, plk.ERR_SHAPE), (2, plk.ERR_ARG),
+                      (1, plk.ERR_ARG), (4, plk.ERR_ARG), (0, plk.ERR_ARG)):
+        g = plk.dims(1, 8, 64, 4, 16, 64, dtype=plk.F32, Hkv=hkv)
+        assert lib.plk_full_layer_step(ctypes.byref(g), None, None, None, None, None, None, 0, None) == code, hkv
     ok = plk.dims(2, 8, 64, 4, 16, 64, dtype=plk.F32)
     p = ctypes.c_void_p(16)
     assert lib.plk_select_active(ctypes.byref(ok), p, p, p, 9, 0.5, 1, p, p, None) == plk.ERR_ARG

@@ -29,7 +29,7 @@ def plk():
 
 def pdims(plk, D):
     return plk.dims(D.B, D.N, D.d, D.H, D.hd, D.F, D.eps, plk.BF16 if D.dtype == "bf16" else plk.F32,
-                    getattr(D, "rope_theta", 0.0))
+                    getattr(D, "rope_theta", 0.0), getattr(D, "Hkv", 0))
 
 
 def int_dev(a, n):
@@ -272,6 +272,61 @@ def test_rope_layer_fp32(plk):
     assert plk.get_status() == plk.OK
     act = lock == 0
     assert_f32_close(host(K)[act], ref.K[act], "K active")
+    assert_f32_close(host(Y)[act], ref.Y[act], "Y active")
+
+
+@pytest.mark.parametrize("shape", [dict(Hkv=1), dict(Hkv=2), dict(Hkv=2, rope_theta=10000.0),
+                                   dict(B=1, N=640, d=1024, H=8, F=1024, Hkv=2)])
+def test_gqa_layer_bf16(plk, shape):
+    """Grouped-query variant (fewer K/V heads than query heads; K/V caches Hkv*hd wide): full
+    step, then a partial step on perturbed active rows."""
+    D = synth.Dims(**{**SMALL.__dict__, **shape})
+    W = synth.layer_weights(D, 0.02, seed=12)
+    X = synth.hidden_states(D, seed=12)
+    base = oracle.full_layer_step(D, W, X, "bf16")
+    dm = pdims(plk, D)
+    K = torch.zeros((D.B, D.N, D.dkv), dtype=BF, device="cuda")
+    V = torch.zeros_like(K)
+    Y = torch.zeros((D.B, D.N, D.d), dtype=BF, device="cuda")
+    plk.full_layer_step(dm, weights_dev(W, D), dev(X, BF), K, V, Y, plk.alloc_workspace(dm))
+    assert plk.get_status() == plk.OK
+    assert_bf16_close(host(K), base.K, "K full")
+    assert_bf16_close(host(V), base.V, "V full")
+    assert_bf16_close(host(Y), base.Y, "Y full")
+    lock = synth.bernoulli_active(D.B, D.N, 0.3, seed=12)
+    idx, seg = oracle.compact(lock)
+    X2 = synth.perturb_rows(X, synth.step_noise((D.B, D.N, D.d), 0.01, seed=12), lock == 0, "bf16")
+    ref = oracle.layer_step_partial(D, W, X2, idx, seg, base, "bf16")
+    K, V, Y = _run_partial(plk, D, W, X2, idx, seg, base)
+    locked = lock.astype(bool)
+    for g, o0, name in ((K, base.K, "K"), (V, base.V, "V"), (Y, base.Y, "Y")):
+        assert np.array_equal(g[locked], o0[locked]), f"{name}: a locked row was written"
+    act = ~locked
+    assert_bf16_close(K[act], ref.K[act], "K active")
+    assert_bf16_close(V[act], ref.V[act], "V active")
+    assert_bf16_close(Y[act], ref.Y[act], "Y active")
+
+
+@pytest.mark.parametrize("Hkv,theta", [(1, 0.0), (2, 10000.0)])
+def test_gqa_layer_fp32(plk, Hkv, theta):
+    D = synth.Dims(B=2, N=100, d=64, H=4, hd=16, F=64, eps=1e-6, dtype="f32", rope_theta=theta, Hkv=Hkv)
+    W = synth.layer_weights(D, 1.0 / math.sqrt(D.d), seed=13)
+    X = synth.hidden_states(D, seed=13)
+    base = oracle.full_layer_step(D, W, X, "f64")
+    lock = synth.bernoulli_active(D.B, D.N, 0.4, seed=13)
+    idx, seg = oracle.compact(lock)
+    X2 = synth.perturb_rows(X, synth.step_noise((D.B, D.N, D.d), 0.01, seed=13), lock == 0, "f32")
+    ref = oracle.layer_step_partial(D, W, X2, idx, seg, base, "f64")
+    dm = pdims(plk, D)
+    K, V, Y = (dev(a, torch.float32) for a in (base.K, base.V, base.Y))
+    assert K.shape == (D.B, D.N, Hkv * D.hd)
+    plk.layer_step_partial(dm, weights_dev(W, D), dev(X2, torch.float32), int_dev(idx, D.B * D.N),
+                           int_dev(seg, D.B + 1), K, V, Y, plk.alloc_workspace(dm))
+    assert plk.get_status() == plk.OK
+    act = lock == 0
+    assert np.array_equal(host(K)[~act], base.K[~act])
+    assert_f32_close(host(K)[act], ref.K[act], "K active")
+    assert_f32_close(host(V)[act], ref.V[act], "V active")
     assert_f32_close(host(Y)[act], ref.Y[act], "Y active")
 
 
