@@ -594,6 +594,28 @@ def run_kernel_configs(args):
                 "finish_qkv_kernel (K/V scatter)": {"us": per["finish_qkv"], "GB/s": scat / (per["finish_qkv"] * 1e-6) / 1e9,
                                                     "frac_of_hbm": scat / (per["finish_qkv"] * 1e-6) / 1e9 / hbm},
                 "per_kernel_us_traced": per})
+    del W, pw, X, K, V, Y, ws
+    # grouped-query layer variant at a 7B-class shape (28 query heads, 4 K/V heads of 128,
+    # SwiGLU 18944), N = 1024, 256 active rows
+    d_, H_, Hkv_, F_, N_, M_ = 3584, 28, 4, 18944, 1024, 256
+    dkv_ = Hkv_ * 128
+    dm = plk.dims(1, N_, d_, H_, 128, F_, 1e-6, plk.BF16, 0.0, Hkv_)
+    W = {kk: (torch.randn(sh, device=dev) * 0.02).to(bf) if len(sh) == 2 else torch.ones(sh, device=dev).to(bf)
+         for kk, sh in (("g1", (d_,)), ("w_qkv", (d_ + 2 * dkv_, d_)), ("w_o", (d_, d_)), ("g2", (d_,)),
+                        ("w_gu", (2 * F_, d_)), ("w_down", (d_, F_)))}
+    pw = plk.weights(W)
+    X = torch.randn((1, N_, d_), device=dev).to(bf)
+    K, V = (torch.randn((1, N_, dkv_), device=dev).to(bf) for _ in range(2))
+    Y = torch.zeros((1, N_, d_), dtype=bf, device=dev)
+    rows = np.sort(np.random.default_rng(0).choice(N_, M_, replace=False)).astype(np.int32)
+    idx = torch.from_numpy(rows).to(dev)
+    seg = torch.tensor([0, M_], dtype=torch.int32, device=dev)
+    ws = plk.alloc_workspace(dm, device=dev)
+    us_g = _timed(torch, lambda: plk.layer_step_partial(dm, pw, X, idx, seg, K, V, Y, ws), args.steps, args.warmup)
+    fl = M_ * (2 * d_ * (d_ + 2 * dkv_) + 2 * d_ * d_ + 6 * d_ * F_) + 4 * M_ * N_ * d_
+    out.append({"kernel": "layer step, grouped-query attention", "config": f"d={d_} H={H_} Hkv={Hkv_} F={F_} "
+                f"N={N_} M={M_}", "us": us_g, "active_token_layers_per_s": M_ / (us_g * 1e-6),
+                "TFLOP/s": fl / (us_g * 1e-6) / 1e12, "frac_of_peak": fl / (us_g * 1e-6) / 1e12 / tfl})
     st = plk.get_status()
     if st != plk.OK:
         raise RuntimeError(f"device status {plk.error_string(st)}")
