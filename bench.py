@@ -738,6 +738,266 @@ def run_slowfast(args):
     return 0
 
 
+# ---------------------------------------------------------------------------
+# the 32-layer stack over a whole decode (--kernel stack): B = 4 sequences of
+# N = 2048, 32 independently drawn 8B-shape layers, 256 steps of the linear
+# active-count schedule M_t = N - floor(t (N - floor(N/20)) / 255).  Per step
+# and layer: drift score (rank 128, L2) -> the M_t most drifted rows among those
+# not yet locked stay active, the rest lock for good -> partial layer step ->
+# proxy refresh; each layer's output cache is the next layer's input.  The
+# layer-0 input takes N(0, 0.01) noise on its active rows every step (outside
+# the timed region).
+# ---------------------------------------------------------------------------
+STACK_LAYERS, STACK_STEPS, STACK_RANK = 32, 256, 128
+
+
+def _stack_state(torch, plk, D, dev, seed):
+    import synth
+
+    bf = torch.bfloat16
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed)
+    rnd = lambda shape, std: (torch.randn(shape, generator=g, device=dev) * std).to(bf)
+    d, F, r = D.d, D.F, STACK_RANK
+    layers = []
+    for l in range(STACK_LAYERS):
+        W = {"g1": torch.ones(d, device=dev, dtype=bf), "w_qkv": rnd((3 * d, d), 0.02), "w_o": rnd((d, d), 0.02),
+             "g2": torch.ones(d, device=dev, dtype=bf), "w_gu": rnd((2 * F, d), 0.02), "w_down": rnd((d, F), 0.02)}
+        layers.append({"W": W, "pw": plk.weights(W),
+                       "Ut": torch.from_numpy(synth.proxy_basis(d, r, seed=l)).to(dev).to(bf),
+                       "pc": torch.zeros((D.B, D.N, r), device=dev), "pn": torch.empty((D.B, D.N, r), device=dev),
+                       "K": torch.zeros((D.B, D.N, d), device=dev, dtype=bf),
+                       "V": torch.zeros((D.B, D.N, d), device=dev, dtype=bf),
+                       "Y": torch.zeros((D.B, D.N, d), device=dev, dtype=bf),
+                       "lock": torch.zeros((D.B, D.N), device=dev, dtype=torch.uint8)})
+    X0 = rnd((D.B, D.N, d), 1.0)
+    noise = [torch.randn((D.B, D.N, d), generator=g, device=dev) * 0.1 for _ in range(4)]
+    return layers, X0, noise
+
+
+def _stack_reset(layers, X0, X0_init):
+    for Ly in layers:
+        Ly["pc"].zero_()
+        Ly["K"].zero_()
+        Ly["V"].zero_()
+        Ly["Y"].zero_()
+        Ly["lock"].zero_()
+    X0.copy_(X0_init)
+
+
+def run_stack(args):
+    import torch
+    import partial_recompute_kv_b200 as plk
+    import oracle
+    import synth
+
+    dev = torch.device("cuda", 0)
+    D = synth.STACK_8B
+    B, N, d, F, r = D.B, D.N, D.d, D.F, STACK_RANK
+    dm = plk.dims(B, N, d, D.H, D.hd, F, D.eps, plk.BF16)
+    layers, X0, noise = _stack_state(torch, plk, D, dev, seed=0)
+    X0_init = X0.clone()
+    ws = plk.alloc_workspace(dm, device=dev)
+    score = torch.empty((B, N), device=dev)
+    idx = torch.empty(B * N, dtype=torch.int32, device=dev)
+    seg = torch.empty(B + 1, dtype=torch.int32, device=dev)
+    sched = synth.linear_schedule(N, STACK_STEPS)
+
+    def step(t):
+        M = int(sched[t])
+        X = X0
+        for Ly in layers:
+            plk.score_drift(dm, X, Ly["Ut"], r, Ly["pc"], plk.METRIC_L2, score, proxy_out=Ly["pn"])
+            plk.select_active(dm, score, Ly["lock"], Ly["lock"], plk.SEL_TOPK_LARGEST, 0.0, M, idx, seg)
+            plk.layer_step_partial(dm, Ly["pw"], X, idx, seg, Ly["K"], Ly["V"], Ly["Y"], ws)
+            plk.proxy_commit(dm, r, idx, seg, Ly["pn"], Ly["pc"])
+            X = Ly["Y"]
+
+    def perturb(t):  # the layer-0 input process: noise on the rows still active at layer 0
+        act0 = (layers[0]["lock"] == 0).unsqueeze(-1)
+        X0.copy_((X0.float() + noise[t % len(noise)] * act0).to(torch.bfloat16))
+
+    warm = max(args.warmup, 3)
+    for t in range(warm):
+        perturb(t)
+        step(t)
+    torch.cuda.synchronize()
+    _stack_reset(layers, X0, X0_init)
+    E = lambda: torch.cuda.Event(enable_timing=True)
+    ev = [(E(), E()) for _ in range(STACK_STEPS)]
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clk:
+        for t in range(STACK_STEPS):
+            perturb(t)
+            ev[t][0].record()
+            step(t)
+            ev[t][1].record()
+        torch.cuda.synchronize()
+    st_ = plk.get_status()
+    if st_ != plk.OK:
+        raise RuntimeError(f"device status {plk.error_string(st_)}")
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_s = sum(step_ms) * 1e-3
+    # every layer ends with B * M_255 active rows: the schedule was followed
+    M_last = int(sched[-1])
+    for Ly in layers:
+        assert int((Ly["lock"] == 0).sum()) == B * M_last, "schedule not followed"
+    atl = int(sched.sum()) * B * STACK_LAYERS
+    flops = sum(int(m) * B * (8 * d * d + 6 * d * F + 4 * N * d) for m in sched) * STACK_LAYERS
+    pk = peaks()
+    tf = flops / total_s / 1e12
+    # cpu baseline: the oracle on one layer at the schedule's last step (B * M_255 active rows),
+    # extrapolated to the run by FLOP count
+    Dn = synth.Dims(B=B, N=N, d=d, H=D.H, hd=D.hd, F=F, eps=D.eps, dtype="bf16")
+    Wn = synth.layer_weights(Dn, 0.02, seed=0)
+    Xn = synth.hidden_states(Dn, seed=0)
+    rng = np.random.default_rng(0)
+    lock = np.ones((B, N), np.uint8)
+    for b in range(B):
+        lock[b, rng.choice(N, M_last, replace=False)] = 0
+    oidx, oseg = oracle.compact(lock)
+    zeros = np.zeros((B, N, d))
+    stn = oracle.LayerState(zeros, zeros.copy(), zeros.copy())
+    t0 = time.perf_counter()
+    oracle.layer_step_partial(Dn, Wn, Xn, oidx, oseg, stn, "bf16")
+    cpu_s = time.perf_counter() - t0
+    cpu_flops = B * M_last * (8 * d * d + 6 * d * F + 4 * N * d)
+    cpu_steps_per_s = (cpu_flops / cpu_s) / (flops / STACK_STEPS)
+    line = {"metric": "decode steps/s, 32-layer stack, B=4 x N=2048, linear 100%->5% active schedule",
+            "value": STACK_STEPS / total_s, "unit": "steps/s", "n_gpus": 1, "steps": STACK_STEPS,
+            "warmup": warm, "ms_per_step": total_s * 1e3 / STACK_STEPS,
+            "ms_per_step_first_last": [step_ms[0], step_ms[-1]],
+            "active_token_layers_per_s": atl / total_s, "active_token_layers_per_run": atl,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (random-init weights, N(0,1) layer-0 input + N(0,0.01) noise per step)",
+            "config": {"workload": f"32-layer 8B-shape stack, B={B}, N={N}, d={d}, F={F}, rank-{r} L2 drift, "
+                                   f"top-M_t among unlocked rows (permanent), M_t from {int(sched[0])} to {M_last}, "
+                                   f"{STACK_STEPS} steps", "l2": "weights 14 GB, streamed every step"},
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": float(pk["bf16_tflops_sustained"]),
+                         "unit": "TFLOP/s", "frac": tf / float(pk["bf16_tflops_sustained"]), "traffic": None,
+                         "kernel": "whole step (all kernels): algorithmic FLOP of the run / run time, against "
+                                   "the sustained bf16 peak"},
+            "clocks": clk.summary(),
+            "cpu_baseline": {"value": cpu_steps_per_s, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"one oracle layer step with {B * M_last} active rows (the last step), "
+                                       f"extrapolated to the run by FLOP count"}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# long context (--kernel long): one 8B-shape layer, N = 8192 (7936 prompt rows),
+# 8 block steps of 32 generated rows; block step i recomputes its 32 rows and
+# M_i - 32 earlier positions drawn uniformly, M_i = 32 + min(G, 480),
+# G ~ Geometric(1/64).  Caches come from one untimed full step.  Reports block
+# steps/s (the 8 steps captured as one CUDA graph) and the attention roofline
+# of each block (its K/V read of 2 N d bf16 values is what bounds it).
+# ---------------------------------------------------------------------------
+def run_long(args):
+    import torch
+    import partial_recompute_kv_b200 as plk
+    import oracle
+    import synth
+
+    dev = torch.device("cuda", 0)
+    bf = torch.bfloat16
+    D = synth.LONG_8B
+    N, d, F, prompt, nblk = D.N, D.d, D.F, 7936, 8
+    dm = plk.dims(1, N, d, D.H, D.hd, F, D.eps, plk.BF16)
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    rnd = lambda shape, std: (torch.randn(shape, generator=g, device=dev) * std).to(bf)
+    W = {"g1": torch.ones(d, device=dev, dtype=bf), "w_qkv": rnd((3 * d, d), 0.02), "w_o": rnd((d, d), 0.02),
+         "g2": torch.ones(d, device=dev, dtype=bf), "w_gu": rnd((2 * F, d), 0.02), "w_down": rnd((d, F), 0.02)}
+    pw = plk.weights(W)
+    X = rnd((1, N, d), 1.0)
+    K, V, Y = (torch.zeros((1, N, d), device=dev, dtype=bf) for _ in range(3))
+    ws = plk.alloc_workspace(dm, device=dev)
+    plk.full_layer_step(dm, pw, X, K, V, Y, ws)
+    Ms = [int(m) for m in synth.geometric_block_m(nblk)]
+    blocks = []
+    for blk, M in enumerate(Ms):
+        b0 = prompt + 32 * blk
+        rows = np.concatenate([synth.uniform_positions(0, b0, M - 32, tag=100 + blk), np.arange(b0, b0 + 32)])
+        blocks.append((M, torch.from_numpy(np.sort(rows).astype(np.int32)).to(dev),
+                       torch.tensor([0, M], dtype=torch.int32, device=dev)))
+
+    def decode():
+        for M, idx, seg in blocks:
+            plk.layer_step_partial(dm, pw, X, idx, seg, K, V, Y, ws)
+
+    for _ in range(max(args.warmup, 3)):
+        decode()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        decode()
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    E = lambda: torch.cuda.Event(enable_timing=True)
+    reps = max(5, min(100, args.steps // nblk))
+    ev = [(E(), E()) for _ in range(reps)]
+    with ClockSampler(0) as clk:
+        for a, b in ev:
+            a.record()
+            graph.replay()
+            b.record()
+        torch.cuda.synchronize()
+    del graph
+    dec_ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    # traced pass: the attention kernel of every block (events between the library's kernels)
+    att_us = []
+    for M, idx, seg in blocks:
+        samples = []
+        for _ in range(5):
+            tr = [E() for _ in range(11)]
+            plk.trace_events(tr)
+            plk.layer_step_partial(dm, pw, X, idx, seg, K, V, Y, ws)
+            plk.trace_events([])
+            torch.cuda.synchronize()
+            samples.append(tr[3].elapsed_time(tr[4]) * 1e3)
+        att_us.append(statistics.median(samples))
+    st_ = plk.get_status()
+    if st_ != plk.OK:
+        raise RuntimeError(f"device status {plk.error_string(st_)}")
+    pk = peaks()
+    hbm, tfl = float(pk["hbm_gbs"]), float(pk["bf16_tflops"])
+    att = []
+    for (M, _, _), us in zip(blocks, att_us):
+        by = 2 * N * d * 2 + 2 * M * d * 2  # K and V of the sequence, q in and a out
+        att.append({"M": M, "us": us, "GB/s": by / (us * 1e-6) / 1e9, "frac_of_hbm": by / (us * 1e-6) / 1e9 / hbm,
+                    "TFLOP/s": 4 * M * N * d / (us * 1e-6) / 1e12})
+    gbs_mean = statistics.mean(a["GB/s"] for a in att)
+    # cpu baseline: the oracle on block 0's step from zero caches
+    Dn = synth.Dims(B=1, N=N, d=d, H=D.H, hd=D.hd, F=F, eps=D.eps, dtype="bf16")
+    Wn = synth.layer_weights(Dn, 0.02, seed=0)
+    Xn = synth.hidden_states(Dn, seed=0)
+    lock = np.ones((1, N), np.uint8)
+    lock[0, blocks[0][1].cpu().numpy()] = 0
+    oidx, oseg = oracle.compact(lock)
+    zeros = np.zeros((1, N, d))
+    t0 = time.perf_counter()
+    oracle.layer_step_partial(Dn, Wn, Xn, oidx, oseg, oracle.LayerState(zeros, zeros.copy(), zeros.copy()), "bf16")
+    cpu_s = time.perf_counter() - t0
+    line = {"metric": "block steps/s, long context (8B layer, N=8192, 8 blocks of 32, geometric M)",
+            "value": nblk / (dec_ms * 1e-3), "unit": "steps/s", "n_gpus": 1, "steps": reps * nblk,
+            "warmup": max(args.warmup, 3), "ms_per_step": dec_ms / nblk, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (random-init weights, N(0,1) input)",
+            "config": {"workload": f"long context, B=1, N={N}, prompt {prompt}, {nblk} blocks of 32, M per block "
+                                   f"{Ms}, one layer d={d} F={F}, the {nblk} block steps as one CUDA graph"},
+            "active_token_layers_per_s": sum(Ms) / (dec_ms * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": gbs_mean, "peak": hbm, "unit": "GB/s", "frac": gbs_mean / hbm,
+                         "traffic": None, "kernel": "attn_tc_kernel (mean over the 8 blocks, traced pass)",
+                         "per_block": att},
+            "clocks": clk.summary(),
+            "cpu_baseline": {"value": 1.0 / cpu_s, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"one oracle block step (block 0, M={Ms[0]}) from zero caches"}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -751,10 +1011,11 @@ def main():
                     help="replay the step as one captured CUDA graph (default)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="enqueue the step's library calls directly every step")
-    ap.add_argument("--kernel", choices=["step", "kl_lock", "slowfast", "configs"], default="step",
+    ap.add_argument("--kernel", choices=["step", "kl_lock", "slowfast", "configs", "stack", "long"], default="step",
                     help="step: the headline layer step; kl_lock: the KL lock rule alone; slowfast: the SlowFast "
                          "span policy over whole decodes; configs: scoring and the all-active stack step at the "
-                         "shapes where their rooflines are judged")
+                         "shapes where their rooflines are judged; stack: the 32-layer stack over the 256-step "
+                         "schedule; long: the long-context block decode at N = 8192")
     ap.add_argument("--profile", action="store_true",
                     help="set up and run --steps steps without timing or output (for ncu)")
     args = ap.parse_args()
@@ -767,6 +1028,10 @@ def main():
         return run_kl_lock(args) if rank == 0 else 0
     if args.kernel == "slowfast":
         return run_slowfast(args) if rank == 0 else 0
+    if args.kernel == "stack":
+        return run_stack(args) if rank == 0 else 0
+    if args.kernel == "long":
+        return run_long(args) if rank == 0 else 0
     if args.kernel == "configs":
         return run_kernel_configs(args) if rank == 0 else 0
     if args.impl == "reference":
