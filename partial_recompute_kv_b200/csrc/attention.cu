@@ -18,7 +18,10 @@
 // below 256, exact in fp32); only then is its O row rescaled in TMEM.  When the
 // query tiles alone leave SMs idle, the two CTAs of a cluster pair split a
 // tile's keys: the odd CTA hands its partial O, row max and row sum to the even
-// CTA through distributed shared memory, which merges and writes the tile.
+// CTA through distributed shared memory, which merges and writes the tile.  When
+// even that leaves pairs idle, a unit's keys are cut into up to 4 parts, one
+// pair each; the pairs store their partials in global scratch and the pair
+// that completes the unit last (a per-unit counter) merges them.
 // Keys past N are masked.  Under grouped-query attention the K/V tiles of query
 // head h come from K/V head h / (H / Hkv) of the Hkv-head caches; the query
 // heads of a group are separate units whose K/V reads meet in L2.
@@ -120,24 +123,53 @@ __device__ __forceinline__ AttnUnit attn_unit(int u, const int32_t* seg_ptr, int
 // (2 x units <= CTAs) the two CTAs of a cluster split the unit's keys in halves
 // and the odd CTA hands its partial (O, max, sum) to the even one through
 // distributed shared memory; otherwise every CTA takes whole units on its own.
+// When the units leave more than half of the pairs idle, each unit's keys are
+// further cut into `parts` ranges, one pair each: the even CTA of every pair
+// stores its merged partial in global scratch, and the pair that finishes a
+// unit last (a device-scope counter per unit) merges the parts and writes the
+// output.  The work items are then (unit, part) pairs, part fastest.
+constexpr int kAttMaxParts = 4;
 struct AttnPlan {
   int split;   // 1 or 2
-  int first;   // first unit of this CTA
-  int stride;  // unit stride
-  int units;
+  int parts;   // key ranges per unit, one CTA pair each (1 unless split == 2)
+  int first;   // first work item of this CTA
+  int stride;  // work-item stride
+  int units;   // (tile, head) units
+  int items;   // units * parts
 };
-__device__ __forceinline__ AttnPlan attn_plan(const int32_t* seg_ptr, int B, int H, int N) {
+__device__ __forceinline__ AttnPlan attn_plan(const int32_t* seg_ptr, int B, int H, int N, int part_cap) {
   AttnPlan p;
   p.units = attn_units(seg_ptr, B, H);
-  p.split = (2 * p.units <= (int)gridDim.x && ceil_div(N, kAttBK) >= 2) ? 2 : 1;
+  const int nch = ceil_div(N, kAttBK);
+  p.split = (2 * p.units <= (int)gridDim.x && nch >= 2) ? 2 : 1;
+  p.parts = 1;
   if (p.split == 2) {
+    const int pairs = (int)gridDim.x >> 1;
+    int parts = min(min(pairs / p.units, nch / 2), kAttMaxParts);
+    if (p.units > 0) parts = min(parts, part_cap / p.units);  // scratch tiles for the partials
+    if (parts >= 2 && p.units <= kAttPartCounters) p.parts = parts;  // units <= CTAs / 4 here
     p.first = blockIdx.x >> 1;
-    p.stride = gridDim.x >> 1;
+    p.stride = pairs;
   } else {
     p.first = blockIdx.x;
     p.stride = gridDim.x;
   }
+  p.items = p.units * p.parts;
   return p;
+}
+// Key chunks [c0, c1) of work item w for this CTA (rank in its cluster): the
+// item's part of the nch chunks, halved between the two CTAs of a split pair.
+// Every CTA gets at least one chunk (parts <= nch / 2).
+__device__ __forceinline__ void attn_chunks(const AttnPlan& p, int w, int rank, int nch, int& c0, int& c1) {
+  const int part = w % p.parts;
+  const int p0 = part * nch / p.parts, p1 = (part + 1) * nch / p.parts;
+  if (p.split == 2) {
+    c0 = p0 + rank * (p1 - p0) / 2;
+    c1 = p0 + (rank + 1) * (p1 - p0) / 2;
+  } else {
+    c0 = p0;
+    c1 = p1;
+  }
 }
 
 __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -145,7 +177,9 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
                                                                const __grid_constant__ CUtensorMap tmV,
                                                                __nv_bfloat16* __restrict__ Aout,
                                                                const int32_t* __restrict__ seg_ptr, int B, int N,
-                                                               int H, int d, int kv_group, float scale_log2) {
+                                                               int H, int d, int kv_group, float scale_log2,
+                                                               float* __restrict__ opart, int* __restrict__ part_cnt,
+                                                               int part_cap) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // same offset in both CTAs
@@ -175,18 +209,18 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
   uint64_t* xo_read = bars + 38;  // even CTA: all 8 softmax warps have read the odd CTA's partial
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 39);
   volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 40);
+  uint64_t* part_written = bars + 41;  // parts > 1: the 8 softmax warps stored this CTA's partial
+  uint64_t* part_decided = bars + 42;  // parts > 1: warp 2 took the unit's counter (s_last is set)
+  volatile int* s_last = reinterpret_cast<volatile int*>(bars + 43);
 
   pdl_wait();
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rank = (int)cluster_ctarank();
-  const AttnPlan plan = attn_plan(seg_ptr, B, H, N);
+  const AttnPlan plan = attn_plan(seg_ptr, B, H, N, part_cap);
   const int nch = ceil_div(N, kAttBK);
-  const int c0 = plan.split == 2 ? rank * nch / 2 : 0;  // this CTA's key chunks of every unit
-  const int c1 = plan.split == 2 ? (rank + 1) * nch / 2 : nch;
-  const int n = c1 - c0;
-  // the two CTAs of a cluster see the same plan; with a split they also see the same units
-  if (plan.first >= plan.units) return;
+  // the two CTAs of a cluster see the same plan; with a split they also see the same items
+  if (plan.first >= plan.items) return;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -210,6 +244,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
     for (int i = 0; i < 8; ++i) mbar_init(&xmb[i], 2);
     for (int i = 0; i < 4; ++i) mbar_init(&xlb[i], 2);
     mbar_init(xo_read, kAttSoftWarps);
+    mbar_init(part_written, kAttSoftWarps);
+    mbar_init(part_decided, 1);
     *s_abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
@@ -233,8 +269,10 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
     if (elect_one()) {
       long long g = 0;  // chunk counter over this CTA's units
       int t = 0;        // unit counter
-      for (int u = plan.first; u < plan.units && !*s_abort; u += plan.stride, ++t) {
-        const AttnUnit it = attn_unit(u, seg_ptr, B, H);
+      for (int w = plan.first; w < plan.items && !*s_abort; w += plan.stride, ++t) {
+        const AttnUnit it = attn_unit(w / plan.parts, seg_ptr, B, H);
+        int c0, c1;
+        attn_chunks(plan, w, rank, nch, c0, c1);
         const int hc = it.h * kAttHD;                  // query head columns
         const int kc = (it.h / kv_group) * kAttHD;     // its K/V head (grouped-query attention)
         if (!mbar_wait(q_free, (uint32_t)((t & 1) ^ 1))) {
@@ -295,7 +333,10 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
         umma_commit(&p_free[pb]);  // also: every earlier MMA, so O holds chunks <= gj
         return true;
       };
-      for (int u = plan.first; u < plan.units && !*s_abort; u += plan.stride, ++t) {
+      for (int w = plan.first; w < plan.items && !*s_abort; w += plan.stride, ++t) {
+        int c0, c1;
+        attn_chunks(plan, w, rank, nch, c0, c1);
+        const int n = c1 - c0;
         bool ok = mbar_wait(q_full, (uint32_t)(t & 1));
         tc_fence_after();
         for (int j = 0; j < n && ok; ++j) {
@@ -353,8 +394,12 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
     auto wait_pv = [&](long long k) -> bool {
       return k < 0 || mbar_wait(&p_free[k & 1], (uint32_t)((k >> 1) & 1));
     };
-    for (int u = plan.first; u < plan.units && ok; u += plan.stride, ++t) {
+    for (int w = plan.first; w < plan.items && ok; w += plan.stride, ++t) {
+      const int u = w / plan.parts;
       const AttnUnit it = attn_unit(u, seg_ptr, B, H);
+      int c0, c1;
+      attn_chunks(plan, w, rank, nch, c0, c1);
+      const int n = c1 - c0;
       float m_used = -INFINITY, l = 0.f;
       for (int j = 0; j < n; ++j) {
         const long long gj = g + j;
@@ -492,7 +537,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(dsmem_addr(smem_u32(xo_full), 0));
       } else {
-        float w_own = 1.f, inv;
+        float m_row = m_used, l_tot = l_row;
         if (plan.split == 2) {
           // my P region is free (every P V of this unit is done): the odd CTA may write its partial
           __syncwarp();
@@ -504,19 +549,77 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
           }
           const float2 pm = reinterpret_cast<const float2*>(ml)[row];  // odd CTA's (max, sum)
           const float m = fmaxf(m_used, pm.x);
-          w_own = exp2f(m_used - m);
+          const float w_own = exp2f(m_used - m);
           const float w_odd = exp2f(pm.x - m);
-          inv = 1.0f / (w_own * l_row + w_odd * pm.y);
+          m_row = m;
+          l_tot = w_own * l_row + w_odd * pm.y;
           const float* xo = reinterpret_cast<const float*>(sP) + row * kAttHD + hf * 64;
 #pragma unroll
           for (int e = 0; e < 64; ++e) o[e] = fmaf(w_own, o[e], w_odd * xo[e]);
           // the next unit's P may overwrite the partial once every softmax warp has read it
           __syncwarp();
           if (lane == 0) mbar_arrive(xo_read);
-        } else {
-          inv = 1.0f / l_row;
         }
-        if (row < it.nrows) {
+        float inv = 1.0f / l_tot;
+        bool write_out = true;
+        if (plan.parts > 1) {
+          // this pair's key range is one part of the unit: store (O, max, sum), unnormalised,
+          // and let the pair that completes the unit last merge the parts
+          float2* mlp = reinterpret_cast<float2*>(opart + (size_t)part_cap * kAttBQ * kAttHD);
+          float4* op = reinterpret_cast<float4*>(opart + ((size_t)w * kAttBQ + row) * kAttHD + hf * 64);
+#pragma unroll
+          for (int v = 0; v < 16; ++v) op[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+          if (hf == 0) mlp[(size_t)w * kAttBQ + row] = make_float2(m_row, l_tot);
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(part_written);
+          if (warp == 2) {
+            int okd = 1;
+            if (lane == 0) {
+              okd = mbar_wait(part_written, (uint32_t)(t & 1)) ? 1 : 0;
+              int last = 0;
+              if (okd) {
+                __threadfence();
+                last = atomicAdd(part_cnt + u, 1) == plan.parts - 1 ? 1 : 0;
+              }
+              *s_last = last;
+              mbar_arrive(part_decided);
+            }
+            ok = ok && __shfl_sync(0xffffffffu, okd, 0) != 0;
+          }
+          ok = ok && mbar_wait(part_decided, (uint32_t)(t & 1));
+          if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
+          }
+          write_out = *s_last != 0;
+          if (write_out) {
+            __threadfence();
+            const size_t w0 = (size_t)u * plan.parts;
+            float mm = -INFINITY;
+            for (int q2 = 0; q2 < plan.parts; ++q2) mm = fmaxf(mm, __ldcg(&mlp[(w0 + q2) * kAttBQ + row]).x);
+            float lt = 0.f;
+#pragma unroll
+            for (int e = 0; e < 64; ++e) o[e] = 0.f;
+            for (int q2 = 0; q2 < plan.parts; ++q2) {
+              const float2 pq = __ldcg(&mlp[(w0 + q2) * kAttBQ + row]);
+              const float wq = exp2f(pq.x - mm);
+              lt = fmaf(wq, pq.y, lt);
+              const float4* src = reinterpret_cast<const float4*>(opart + ((w0 + q2) * kAttBQ + row) * kAttHD + hf * 64);
+#pragma unroll
+              for (int v = 0; v < 16; ++v) {
+                const float4 x = __ldcg(src + v);
+                o[4 * v] = fmaf(wq, x.x, o[4 * v]);
+                o[4 * v + 1] = fmaf(wq, x.y, o[4 * v + 1]);
+                o[4 * v + 2] = fmaf(wq, x.z, o[4 * v + 2]);
+                o[4 * v + 3] = fmaf(wq, x.w, o[4 * v + 3]);
+              }
+            }
+            inv = 1.0f / lt;
+            if (warp == 2 && lane == 0) part_cnt[u] = 0;  // every part has counted: reset for the next launch
+          }
+        }
+        if (write_out && row < it.nrows) {
           uint4* dst = reinterpret_cast<uint4*>(Aout + (size_t)grow * d + it.h * kAttHD + hf * 64);
 #pragma unroll
           for (int v = 0; v < 8; ++v)
@@ -580,7 +683,8 @@ __global__ void attn_f32_kernel(const float* __restrict__ Q, const float* __rest
 }
 
 int launch_attention_bf16(const plk_dims* dims, const void* q, const void* K_cache, const void* V_cache,
-                          void* a_out, const int32_t* seg_ptr, int num_sms, cudaStream_t st) {
+                          void* a_out, const int32_t* seg_ptr, int num_sms, float* part_scratch,
+                          size_t part_bytes, int* part_cnt, cudaStream_t st) {
   const int B = dims->B, N = dims->N, d = dims->d, H = dims->H, dkv = kv_width(dims);
   CUtensorMap tmQ, tmK, tmV;
   if (make_tmap_bf16(&tmQ, q, (uint64_t)B * N, (uint64_t)d, kAttBQ) != PLK_OK) return PLK_ERR_CUDA;
@@ -610,8 +714,11 @@ int launch_attention_bf16(const plk_dims* dims, const void* q, const void* K_cac
   at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 2;
+  // partial tiles (128 x 128 fp32) and their (max, sum) rows that fit in the scratch
+  const size_t tile_bytes = (size_t)kAttBQ * kAttHD * 4 + (size_t)kAttBQ * 8;
+  const int part_cap = part_scratch ? (int)std::min(part_bytes / tile_bytes, (size_t)1 << 20) : 0;
   if (cudaLaunchKernelEx(&cfg, attn_tc_kernel, tmQ, tmK, tmV, (__nv_bfloat16*)a_out, seg_ptr, B, N, H, d,
-                         H / kv_heads(dims), scale_log2) != cudaSuccess)
+                         H / kv_heads(dims), scale_log2, part_scratch, part_cnt, part_cap) != cudaSuccess)
     return PLK_ERR_CUDA;
   return PLK_OK;
 }

@@ -63,7 +63,8 @@ Workspace workspace_layout(const plk_dims* dm, int num_sms) {
   w.hn = take(es * Mcap * d);
   w.act = take(es * Mcap * F);
   w.num_sms = num_sms;
-  w.c32 = take(4 * Mcap * std::max(d + 2 * (size_t)kv_width(dm), 2 * F));
+  w.c32_bytes = 4 * Mcap * std::max(d + 2 * (size_t)kv_width(dm), 2 * F);
+  w.c32 = take(w.c32_bytes);
   w.total = off;
   return w;
 }
@@ -322,9 +323,11 @@ __global__ void __launch_bounds__(256) finish_qkv_kernel(const float* __restrict
                                                          int dkv, int hd, float log2_theta,
                                                          __nv_bfloat16* __restrict__ q,
                                                          __nv_bfloat16* __restrict__ Kc,
-                                                         __nv_bfloat16* __restrict__ Vc) {
+                                                         __nv_bfloat16* __restrict__ Vc, int* part_cnt) {
   pdl_wait();
   pdl_trigger();
+  if (blockIdx.x == 0)  // the attention's per-unit counters (their buffer's reader, the QKV GEMM, is done)
+    for (int i = threadIdx.x; i < kAttPartCounters; i += blockDim.x) part_cnt[i] = 0;
   const int M = seg_ptr[B];
   const bool rope = log2_theta > 0.f;
   const int W = d + 2 * dkv;
@@ -589,11 +592,13 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   trace_mark(2, st);
 
   const float log2_theta = dm->rope_theta > 0.f ? log2f(dm->rope_theta) : 0.f;
+  int* part_cnt = (int*)(ws + L.xn);  // RMSNorm1's output, consumed by the QKV GEMM
   PLK_TRY(launch_pdl(finish_qkv_kernel, dim3(rgrid), dim3(256), 0, st, (const float*)c32, idx, seg, B, dm->N, d,
-                     dkv, dm->hd, log2_theta, q, (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc));
+                     dkv, dm->hd, log2_theta, q, (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc, part_cnt));
   trace_mark(3, st);
 
-  PLK_TRY(launch_attention_bf16(dm, q, Kc, Vc, a, seg, L.num_sms, st));
+  // the QKV sums are consumed: c32 holds the attention's partial outputs until the gate/up GEMM
+  PLK_TRY(launch_attention_bf16(dm, q, Kc, Vc, a, seg, L.num_sms, c32, L.c32_bytes, part_cnt, st));
   trace_mark(4, st);
 
   g.K = d;

@@ -20,6 +20,12 @@ constexpr int kGemmBK = 64;       // K per stage: one 128-byte swizzle row of bf
 constexpr int kGemmStages = 6;
 constexpr int kGemmThreads = 192; // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 
+// ---- attention key split over several CTA pairs --------------------------------
+// Per-unit arrival counters of the attention kernel (zeroed by the QKV
+// finishing kernel, which runs just before it, in the RMSNorm1 output buffer
+// that the QKV GEMM has consumed by then).
+constexpr int kAttPartCounters = 128;
+
 // ---- grouped-query attention --------------------------------------------------
 inline int kv_heads(const plk_dims* d) { return d->Hkv > 0 ? d->Hkv : d->H; }
 inline int kv_width(const plk_dims* d) { return kv_heads(d) * d->hd; }  // dkv: K and V row width
@@ -49,7 +55,9 @@ struct Workspace {
   // offsets (bytes)
   size_t iota = 0, seg = 0;              // identity active set for the full step
   size_t xn = 0, q = 0, a = 0, h32 = 0, hn = 0, act = 0;
-  size_t c32 = 0;                        // fp32 GEMM sums [Mcap, max(3d, 2F)] (QKV, then gate/up)
+  size_t c32 = 0;                        // fp32 GEMM sums [Mcap, max(d + 2 dkv, 2F)] (QKV, then gate/up;
+                                         // in between, the attention's partial outputs)
+  size_t c32_bytes = 0;
   int num_sms = 0;
 };
 Workspace workspace_layout(const plk_dims* d, int num_sms);
@@ -96,8 +104,12 @@ struct GemmArgs {
 int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const CUtensorMap& tmOut, const GemmArgs& a,
                    cudaStream_t st);
 
+// part_scratch / part_bytes: free device memory for the partial outputs of a key
+// split over several CTA pairs (used when the units leave pairs idle); part_cnt:
+// kAttPartCounters ints, zero on entry, zero again on exit.
 int launch_attention_bf16(const plk_dims* dims, const void* q, const void* K_cache, const void* V_cache,
-                          void* a_out, const int32_t* seg_ptr, int num_sms, cudaStream_t st);
+                          void* a_out, const int32_t* seg_ptr, int num_sms, float* part_scratch,
+                          size_t part_bytes, int* part_cnt, cudaStream_t st);
 int launch_attention_f32(const plk_dims* dims, const float* q, const float* K_cache, const float* V_cache,
                          float* a_out, const int32_t* seg_ptr, int Mcap, cudaStream_t st);
 
