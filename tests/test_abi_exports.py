@@ -99,3 +99,34 @@ def test_slowfast_state_layout_matches_header():
     assert "#define PLK_SF_HIST_MAX %d" % plk.SF_HIST_MAX in src
     assert plk.SF_STATE_WORDS == 4 + plk.SF_HIST_MAX
     assert ctypes.sizeof(plk.PlkSfParams) == 24
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """The ctypes structures of the binding have the C header's sizes and field offsets."""
+    import shutil
+    import subprocess
+
+    import partial_recompute_kv_b200 as plk
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    structs = {"plk_dims": plk.PlkDims, "plk_weights": plk.PlkWeights, "plk_sf_params": plk.PlkSfParams}
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "plk.h"', "int main(void) {"]
+    for cname, py in structs.items():
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for fname, _ in py._fields_:
+            lines.append(f'  printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
+    lines.append('  printf("plk_sf_state size %zu\\n", sizeof(plk_sf_state));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = dict(((ln.rsplit(" ", 1)[0]), int(ln.rsplit(" ", 1)[1]))
+               for ln in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+               if ln)
+    for cname, py in structs.items():
+        assert got[f"{cname} size"] == ctypes.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert got[f"{cname} {fname}"] == getattr(py, fname).offset, (cname, fname)
+    assert got["plk_sf_state size"] == 4 * plk.SF_STATE_WORDS
