@@ -1,7 +1,7 @@
 """GPU parity of the SureLock KL lock rule (plk_kl_lock) against the oracle.
 
 Tolerances: KL and H are fp32 results of sums over the V vocabulary entries;
-the benchmark spec's fp32 bound (1e-4 relative) applies, with an absolute floor for KL
+the fp32 parity bound of this library (1e-4 relative) applies, with an absolute floor for KL
 values near zero (2e-7) and for H (1e-5 nats: H = lse - E_p[z] carries the
 rounding of lse ~ |max z|).  The lock bit is decided on the GPU's own fp32 KL
 and H, so it is checked bit-exactly against the rule applied to those values,
