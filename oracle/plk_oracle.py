@@ -83,12 +83,13 @@ R10 Grouped-query attention (an optional layer variant, like R8): with
     query head h attends with K/V head h // (H / Hkv), so consecutive query heads
     share one K/V head.  The K/V caches hold Hkv*hd values per row.  Hkv = 0 or
     Hkv = H is plain multi-head attention.
-R6  Precision policy "bf16": every tensor that the bf16 path stores in bf16
-    between operations is rounded to bf16 here as well -- the normalised
-    inputs of the projections (xn, hn), q, k, v (and so the K/V cache), the
-    attention output a, the SwiGLU product, and the layer output y.  The
-    residual stream h stays unrounded.  All arithmetic is float64.  Policy
-    "f64" rounds nothing.
+R6  Precision policy "bf16": the layer reads bf16 tensors (X, the weights,
+    the cached K/V of locked rows) and stores bf16 tensors: the fresh K/V rows
+    it writes into the cache, which its attention then reads back, and the
+    output rows Y.  Exactly those stored values are rounded to bf16 here;
+    every value computed between them (the normalised inputs xn and hn, q,
+    the attention output, the residual stream, the SwiGLU product) stays
+    float64.  All arithmetic is float64.  Policy "f64" rounds nothing.
 
 Parity unpinned: the pages print no tensor values, so nothing here is pinned to
 a printed example; every function is pinned instead to library routines,
@@ -517,10 +518,10 @@ def full_layer_step(dims, W, X, policy="f64"):
     B, N, d, H, hd, F = dims.B, dims.N, dims.d, dims.H, dims.hd, dims.F
     dkv = kv_heads(dims) * hd
     x = np.asarray(X, dtype=np.float64).reshape(B * N, d)
-    xn = _store(rmsnorm(x, W["g1"], dims.eps), policy)
+    xn = rmsnorm(x, W["g1"], dims.eps)
     qkv = _mm(xn, _w(W, "w_qkv"))
     q, k = _qk(qkv, dims, np.arange(B * N) % N)
-    q, k = _store(q, policy), _store(k, policy)
+    k = _store(k, policy)                      # K/V rows are stored in the cache
     v = _store(qkv[:, d + dkv:], policy)
     a = np.zeros((B * N, d))
     scale = 1.0 / math.sqrt(hd)
@@ -533,12 +534,11 @@ def full_layer_step(dims, W, X, policy="f64"):
             P = np.exp(S)
             P = P / P.sum(axis=1, keepdims=True)
             a[rows, cols] = _mm(P, v[rows, kv].T)                # [N, hd]
-    a = _store(a, policy)
     hres = x + _mm(a, _w(W, "w_o"))
-    hn = _store(rmsnorm(hres, W["g2"], dims.eps), policy)
+    hn = rmsnorm(hres, W["g2"], dims.eps)
     gu = _mm(hn, _w(W, "w_gu"))
-    act = _store(silu(gu[:, :F]) * gu[:, F:], policy)
-    y = _store(hres + _mm(act, _w(W, "w_down")), policy)
+    act = silu(gu[:, :F]) * gu[:, F:]
+    y = _store(hres + _mm(act, _w(W, "w_down")), policy)   # the output rows are stored
     return LayerState(k.reshape(B, N, dkv), v.reshape(B, N, dkv), y.reshape(B, N, d))
 
 
@@ -566,11 +566,11 @@ def layer_step_partial(dims, W, X, idx, seg_ptr, state, policy="f64", out_rows=N
     x_all = np.asarray(X, dtype=np.float64).reshape(B * N, d)
     # S4 gather + RMSNorm1
     x = x_all[idx]
-    xn = _store(rmsnorm(x, W["g1"], dims.eps), policy)
+    xn = rmsnorm(x, W["g1"], dims.eps)
     # S5 projections (Q only for active rows: [SL] Sec. 2 skips Q of locked rows)
     qkv = _mm(xn, _w(W, "w_qkv"))
     q, k = _qk(qkv, dims, idx % N)
-    q, k = _store(q, policy), _store(k, policy)
+    k = _store(k, policy)                      # K/V rows are stored in the cache
     v = _store(qkv[:, d + dkv:], policy)
     # S6 K/V scatter into the cache rows of the active positions
     Kf = out.K.reshape(B * N, dkv)
@@ -593,14 +593,13 @@ def layer_step_partial(dims, W, X, idx, seg_ptr, state, policy="f64", out_rows=N
             p = np.exp(s)
             p = p / p.sum()
             a[t, cols] = _mm(p[None, :], Vb[:, kv].T)[0]        # [hd]
-    a = _store(a, policy)
     # S8 output projection + residual
     hres = x[rows] + _mm(a, _w(W, "w_o"))
     # S9 RMSNorm2 + SwiGLU + residual
-    hn = _store(rmsnorm(hres, W["g2"], dims.eps), policy)
+    hn = rmsnorm(hres, W["g2"], dims.eps)
     gu = _mm(hn, _w(W, "w_gu"))
-    act = _store(silu(gu[:, :F]) * gu[:, F:], policy)
-    y = _store(hres + _mm(act, _w(W, "w_down")), policy)
+    act = silu(gu[:, :F]) * gu[:, F:]
+    y = _store(hres + _mm(act, _w(W, "w_down")), policy)   # the output rows are stored
     # S10 output scatter (locked rows of Y untouched)
     out.Y.reshape(B * N, d)[idx[rows]] = y
     return out

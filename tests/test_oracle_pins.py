@@ -127,8 +127,12 @@ def test_attention_matches_sdpa_single_head():
 # ---------------------------------------------------------------------------
 # brute force: explicit scalar loops on a tiny input
 # ---------------------------------------------------------------------------
-def brute_block(dims, W, X, rows):
+def brute_block(dims, W, X, rows, store=None):
+    """Scalar-loop block.  ``store`` (optional) maps a list of floats to the values a
+    stored tensor holds: it is applied to the K and V rows (the cache) and to the
+    output rows, and nowhere else."""
     B, N, d, H, hd, F = dims.B, dims.N, dims.d, dims.H, dims.hd, dims.F
+    keep = store or (lambda vals: vals)
     Wq = W["w_qkv"]
     out = {}
 
@@ -144,7 +148,7 @@ def brute_block(dims, W, X, rows):
     kv = {}
     for (b, n), vec in xs.items():
         z = lin(Wq, norm(vec, W["g1"]))
-        kv[(b, n)] = (z[:d], z[d:2 * d], z[2 * d:])
+        kv[(b, n)] = (z[:d], keep(z[d:2 * d]), keep(z[2 * d:]))
     for (b, n) in rows:
         q = kv[(b, n)][0]
         a = [0.0] * d
@@ -163,7 +167,7 @@ def brute_block(dims, W, X, rows):
         gu = lin(W["w_gu"], hn)
         act = [gu[f] / (1.0 + math.exp(-gu[f])) * gu[F + f] for f in range(F)]
         dn = lin(W["w_down"], act)
-        out[(b, n)] = [hres[c] + dn[c] for c in range(d)]
+        out[(b, n)] = keep([hres[c] + dn[c] for c in range(d)])
     return kv, out
 
 
@@ -184,6 +188,75 @@ def test_full_and_partial_match_brute_force():
     sp = oracle.layer_step_partial(dims, W, X, idx, seg, zero, "f64")
     for (b, n) in rows:
         np.testing.assert_allclose(sp.Y[b, n], yb[(b, n)], rtol=0, atol=1e-12)
+
+
+def _torch_bf16(vals):
+    """Round to bf16 with torch's conversion (an implementation independent of the oracle's)."""
+    return torch.tensor(vals, dtype=torch.float64).to(torch.bfloat16).to(torch.float64).tolist()
+
+
+def _bf16_case():
+    dims = _dims(B=2, N=5, d=8, H=2, hd=4, F=12, dtype="bf16")
+    W = synth.layer_weights(dims, 0.35, seed=3)
+    X = synth.hidden_states(dims, seed=3)
+    return dims, W, X
+
+
+def _assert_within_one_ulp(a, b, what, frac=0.02):
+    """Equal up to a bf16 rounding that lands on the other side of a tie: at most one
+    bf16 step of the element, on a small fraction of the elements."""
+    ulp = np.ldexp(1.0, np.frexp(np.abs(b) + 1e-300)[1] - 8)
+    assert np.all(np.abs(a - b) <= ulp), what
+    assert np.mean(a != b) <= frac, (what, np.mean(a != b))
+
+
+def test_bf16_policy_rounds_exactly_the_stored_tensors():
+    # brute force with torch's bf16 rounding applied to the K/V cache rows and the
+    # output rows only: the oracle's bf16 policy must agree with it
+    dims, W, X = _bf16_case()
+    rows = [(b, n) for b in range(2) for n in range(5)]
+    kv, yb = brute_block(dims, W, X, rows, store=_torch_bf16)
+    st = oracle.full_layer_step(dims, W, X, "bf16")
+    K = np.array([[kv[(b, n)][1] for n in range(5)] for b in range(2)])
+    V = np.array([[kv[(b, n)][2] for n in range(5)] for b in range(2)])
+    Y = np.array([[yb[(b, n)] for n in range(5)] for b in range(2)])
+    _assert_within_one_ulp(st.K, K, "K")
+    _assert_within_one_ulp(st.V, V, "V")
+    _assert_within_one_ulp(st.Y, Y, "Y")
+    # stored values are bf16 numbers; the f64 policy differs from them by at most half a step
+    for a in (st.K, st.V, st.Y):
+        np.testing.assert_array_equal(a, _torch_bf16_arr(a))
+    f = oracle.full_layer_step(dims, W, X, "f64")
+    assert np.max(np.abs(st.K - f.K) / np.ldexp(1.0, np.frexp(np.abs(f.K))[1] - 8)) <= 0.5 + 1e-9
+    # the partial step with every row active agrees with the brute force too
+    idx, seg = oracle.compact(np.zeros((2, 5), np.uint8))
+    zero = oracle.LayerState(np.zeros_like(st.K), np.zeros_like(st.V), np.zeros_like(st.Y))
+    part = oracle.layer_step_partial(dims, W, X, idx, seg, zero, "bf16")
+    _assert_within_one_ulp(part.Y, Y, "partial Y")
+
+
+def _torch_bf16_arr(a):
+    return torch.from_numpy(np.asarray(a, dtype=np.float64)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+@pytest.mark.parametrize("old,new", [
+    ("k = _store(k, policy)", "k = k"),                                          # cache rows not rounded
+    ("y = _store(hres + _mm(act, _w(W, \"w_down\")), policy)",
+     "y = hres + _mm(act, _w(W, \"w_down\"))"),                                 # output not rounded
+    ("hres = x + _mm(a, ", "hres = x + _mm(to_bf16(a), "),                      # attention output rounded
+    ("act = silu(gu[:, :F]) * gu[:, F:]", "act = to_bf16(silu(gu[:, :F]) * gu[:, F:])"),  # SwiGLU product rounded
+    ("hn = rmsnorm(hres, W[\"g2\"], dims.eps)", "hn = to_bf16(rmsnorm(hres, W[\"g2\"], dims.eps))"),
+])
+def test_bf16_policy_mutants_are_caught(old, new):
+    dims, W, X = _bf16_case()
+    rows = [(b, n) for b in range(2) for n in range(5)]
+    kv, yb = brute_block(dims, W, X, rows, store=_torch_bf16)
+    K = np.array([[kv[(b, n)][1] for n in range(5)] for b in range(2)])
+    Y = np.array([[yb[(b, n)] for n in range(5)] for b in range(2)])
+    st = _mutant(po.full_layer_step, old, new)(dims, W, X, "bf16")
+    with pytest.raises(AssertionError):
+        _assert_within_one_ulp(st.K, K, "K")
+        _assert_within_one_ulp(st.Y, Y, "Y")
 
 
 # ---------------------------------------------------------------------------
@@ -312,6 +385,57 @@ def test_proxy_identity_basis_and_score_cases():
 
 
 # ---------------------------------------------------------------------------
+# S10 proxy half: the refreshed rows take the fresh proxy as float32 (SPA-Cache part 1:
+# the low-resolution snapshot is refreshed where the row was recomputed)
+# ---------------------------------------------------------------------------
+def _proxy_commit_case():
+    rng = np.random.default_rng(18)
+    B, N, r = 3, 11, 5
+    cache = rng.standard_normal((B, N, r)).astype(np.float32).astype(np.float64)
+    fresh = rng.standard_normal((B, N, r)) * 3.0  # float64 values, not float32-representable
+    lock = (rng.random((B, N)) < 0.55).astype(np.uint8)
+    idx, _ = oracle.compact(lock)
+    assert 0 < idx.size < B * N
+    return cache, fresh, lock, idx
+
+
+def _proxy_commit_reference(cache, fresh, lock):
+    """Row by row with Python scalars: active rows get struct-packed float32 values."""
+    import struct
+    out = cache.copy()
+    B, N, r = cache.shape
+    for b in range(B):
+        for n in range(N):
+            if lock[b, n] == 0:
+                for c in range(r):
+                    out[b, n, c] = struct.unpack("f", struct.pack("f", float(fresh[b, n, c])))[0]
+    return out
+
+
+def test_proxy_commit_refreshes_active_rows_as_float32():
+    cache, fresh, lock, idx = _proxy_commit_case()
+    got = oracle.proxy_commit(cache, fresh, idx)
+    ref = _proxy_commit_reference(cache, fresh, lock)
+    np.testing.assert_array_equal(got, ref)
+    locked = lock.astype(bool)
+    assert got[locked].tobytes() == cache[locked].tobytes()      # the other rows: byte-identical
+    assert np.all(got[~locked] != fresh[~locked])                # fresh values were rounded ...
+    assert np.max(np.abs(got[~locked] - fresh[~locked]) / np.abs(fresh[~locked])) <= 2.0 ** -24  # ... to float32
+    assert np.array_equal(cache, _proxy_commit_case()[0])       # the input is not modified
+
+
+@pytest.mark.parametrize("old,new", [
+    ("flat[np.asarray(idx, dtype=np.int64)] = to_f32(", "_unused = ("),   # never writes the fresh proxy
+    ("= to_f32(np.asarray(p)", "= (np.asarray(p)"),                     # writes the unrounded value
+    ("[idx])", "[idx[::-1]])"),                                          # rows paired with the wrong fresh rows
+])
+def test_proxy_commit_mutants_are_caught(old, new):
+    cache, fresh, lock, idx = _proxy_commit_case()
+    got = _mutant(po.proxy_commit, old, new)(cache, fresh, idx)
+    assert not np.array_equal(got, _proxy_commit_reference(cache, fresh, lock))
+
+
+# ---------------------------------------------------------------------------
 # S2/S3 integer semantics against numpy sorts
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("ties", [False, True])
@@ -374,7 +498,7 @@ _FULL_MUTANTS = [
     ("silu(gu[:, :F]) * gu[:, F:]", "silu(gu[:, F:]) * gu[:, :F]"),       # gate/up swapped
     ("S = S - S.max(axis=1, keepdims=True)", "S = S - S.max(axis=0, keepdims=True)"),
     ("P = P / P.sum(axis=1, keepdims=True)", "P = P / P.sum(axis=0, keepdims=True)"),
-    ("hn = _store(rmsnorm(hres, W[\"g2\"]", "hn = _store(rmsnorm(x, W[\"g2\"]"),
+    ("hn = rmsnorm(hres, W[\"g2\"]", "hn = rmsnorm(x, W[\"g2\"]"),
 ]
 
 
