@@ -157,8 +157,11 @@ int plk_select_active(const plk_dims* dims, const float* score, const uint8_t* l
  *   rows are never written.  K_cache, V_cache: [B, N, dkv]; Y: [B, N, d]; in/out.
  *   With grouped-query attention (dims->Hkv > 0) the projection makes Hkv
  *   K/V heads and query head h uses K/V head h / (H / Hkv).
- *   PLK_BF16 stores xn, q, k, v, a, hn and the SwiGLU product in bf16 (the
- *   residual stream h stays fp32).  M = 0 is a no-op.
+ *   PLK_BF16 rounds to bf16 only the values it stores in the caller's tensors
+ *   (the K/V cache rows and Y).  The activations that feed tensor-core products
+ *   (xn, q, a, hn and the SwiGLU product) are held as bf16 pairs hi + lo with
+ *   lo = bf16(v - hi), ~16 significant bits; the residual stream h and every
+ *   sum are fp32.  M = 0 is a no-op.
  *   workspace: device buffer of at least plk_workspace_bytes(dims) bytes, any
  *   content, 256-byte aligned; it must not be used by another call that runs
  *   concurrently.
@@ -267,10 +270,16 @@ int plk_proxy_commit(const plk_dims* dims, int r, const int32_t* idx, const int3
  * PLK_STATIC_WS_BYTES, which every GPU that loads the library holds until the
  * process exits.  Arguments and results are those of plk_layer_step_partial.
  *   - It calls no cudaMalloc, cudaFree or allocating library routine.
- *   - Returns PLK_ERR_WORKSPACE, enqueueing nothing, when plk_workspace_bytes(dims)
- *     exceeds PLK_STATIC_WS_BYTES.
+ *   - Errors: first every error plk_layer_step_partial reports for the same
+ *     arguments (dims, weights, inputs, caches); then PLK_ERR_WORKSPACE,
+ *     enqueueing nothing, when plk_workspace_bytes(dims) exceeds
+ *     PLK_STATIC_WS_BYTES.
  *   - The first call on a device resolves the array's device address
  *     (cudaGetSymbolAddress); make that first call outside any stream capture.
+ *     The address is kept per device together with the id of the CUDA context
+ *     it belongs to; after a device reset the next call resolves it again (so
+ *     that call, too, belongs outside a capture).  Host threads may call
+ *     concurrently; the set-up is serialised internally.
  *   - All calls on a device share the array, which keeps the last call's
  *     contents (every kernel initialises what it reads): calls that overlap on
  *     the GPU, e.g. on two streams, race and must be serialised by the caller.

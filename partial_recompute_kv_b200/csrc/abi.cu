@@ -23,6 +23,17 @@ static int check_dims(const plk_dims* d) {
   return PLK_OK;
 }
 
+// The argument checks of plk_layer_step_partial (dims, weights, inputs and caches;
+// the workspace is checked where it is laid out).
+int check_layer_args(const plk_dims* dims, const plk_weights* w, const void* X, const int32_t* idx,
+                     const int32_t* seg_ptr, const void* K_cache, const void* V_cache, const void* Y) {
+  const int e = check_dims(dims);
+  if (e != PLK_OK) return e;
+  if (!w || !w->g1 || !w->w_qkv || !w->w_o || !w->g2 || !w->w_gu || !w->w_down) return PLK_ERR_ARG;
+  if (!X || !idx || !seg_ptr || !K_cache || !V_cache || !Y) return PLK_ERR_ARG;
+  return PLK_OK;
+}
+
 }  // namespace plk
 
 using namespace plk;
@@ -105,10 +116,8 @@ int plk_slowfast_step(const plk_dims* dims, const plk_sf_params* params, const f
 int plk_layer_step_partial(const plk_dims* dims, const plk_weights* w, const void* X, const int32_t* idx,
                            const int32_t* seg_ptr, void* K_cache, void* V_cache, void* Y, void* workspace,
                            size_t ws_bytes, void* stream) {
-  const int e = check_dims(dims);
+  const int e = check_layer_args(dims, w, X, idx, seg_ptr, K_cache, V_cache, Y);
   if (e != PLK_OK) return e;
-  if (!w || !w->g1 || !w->w_qkv || !w->w_o || !w->g2 || !w->w_gu || !w->w_down) return PLK_ERR_ARG;
-  if (!X || !idx || !seg_ptr || !K_cache || !V_cache || !Y) return PLK_ERR_ARG;
   return run_layer(dims, w, X, idx, seg_ptr, false, K_cache, V_cache, Y, workspace, ws_bytes,
                    (cudaStream_t)stream);
 }

@@ -5,10 +5,12 @@
 // O(M N d) instead of O(N^2 d), Sec. 2 "Algorithmic Complexity").
 //
 // bf16, hd = 128, on the tcgen05 tensor cores: a CTA takes 128 active queries
-// of one sequence and one head and a contiguous range of 64-key chunks.  Warp
-// 0 stages Q once and K, V chunk by chunk with TMA (128-byte swizzle, 3-stage
-// rings); one thread of warp 1 issues S = Q K^T into TMEM (double-buffered,
-// 64 columns each) and O += P V into TMEM (128 columns); warps 2-5 own one
+// of one sequence and one head and a contiguous range of 64-key chunks.  The
+// queries come as a bf16 pair q = q_hi + q_lo (q_lo = bf16(q - q_hi)), so the
+// scores see ~16 significant bits of q.  Warp 0 stages both Q tiles once and K,
+// V chunk by chunk with TMA (128-byte swizzle, 2-stage rings); one thread of
+// warp 1 issues S = Q_hi K^T + Q_lo K^T into TMEM (double-buffered, 64 columns
+// each) and O += P V into TMEM (128 columns); warps 2-5 own one
 // query row per thread: they read the row's scores from TMEM, keep the running
 // row max and sum (online softmax), and write P to shared memory as a bf16 high
 // part and a bf16 residual, both multiplied with V, so the softmax weights
@@ -22,6 +24,7 @@
 // even that leaves pairs idle, a unit's keys are cut into up to 4 parts, one
 // pair each; the pairs store their partials in global scratch and the pair
 // that completes the unit last (a per-unit counter) merges them.
+// The output a goes out as a bf16 hi/lo pair as well.
 // Keys past N are masked.  Under grouped-query attention the K/V tiles of query
 // head h come from K/V head h / (H / Hkv) of the Hkv-head caches; the query
 // heads of a group are separate units whose K/V reads meet in L2.
@@ -39,13 +42,13 @@ namespace {
 constexpr int kAttHD = 128;
 constexpr int kAttBQ = 128;                    // queries per CTA (UMMA M, one TMEM lane each)
 constexpr int kAttBK = 64;                     // keys per chunk (UMMA N of S, K of P V)
-constexpr int kAttStages = 3;                  // K and V ring depth
+constexpr int kAttStages = 2;                  // K and V ring depth
 constexpr int kAttSoftWarps = 8;               // two warps per TMEM lane quarter, one per half row
 constexpr int kAttThreads = 32 * (2 + kAttSoftWarps);  // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
-constexpr int kAttQBytes = kAttBQ * kAttHD * 2;   // 32 KB
+constexpr int kAttQBytes = kAttBQ * kAttHD * 2;   // 32 KB (hi or lo part)
 constexpr int kAttKVBytes = kAttBK * kAttHD * 2;  // 16 KB
 constexpr int kAttPBytes = kAttBQ * kAttBK * 2;   // 16 KB (high or low part)
-constexpr size_t kAttOffK = kAttQBytes;
+constexpr size_t kAttOffK = 2 * (size_t)kAttQBytes;
 constexpr size_t kAttOffV = kAttOffK + (size_t)kAttStages * kAttKVBytes;
 constexpr size_t kAttOffP = kAttOffV + (size_t)kAttStages * kAttKVBytes;  // [2 buffers][high, low]
 constexpr size_t kAttOffML = kAttOffP + 4 * (size_t)kAttPBytes;            // [128] (max, sum) of the odd CTA
@@ -53,6 +56,7 @@ constexpr size_t kAttOffXM = kAttOffML + kAttBQ * 8;                       // [2
 constexpr size_t kAttOffXL = kAttOffXM + 2 * 2 * kAttBQ * 4;               // [2 halves][128] row sum
 constexpr size_t kAttOffBar = kAttOffXL + 2 * kAttBQ * 4;
 constexpr int kAttSmem = (int)kAttOffBar + 512 + 1024;
+static_assert(kAttSmem <= 232448, "shared memory budget");
 constexpr uint32_t kAttTmemCols = 256;         // O: 0..127, S buffers: 128..191, 192..255
 constexpr float kAttStaleMax = 8.f;            // log2 headroom before a row's O is rescaled
 static_assert(4 * kAttPBytes == kAttBQ * kAttHD * 4, "the P region holds one fp32 O tile");
@@ -173,9 +177,11 @@ __device__ __forceinline__ void attn_chunks(const AttnPlan& p, int w, int rank, 
 }
 
 __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                                                               const __grid_constant__ CUtensorMap tmQlo,
                                                                const __grid_constant__ CUtensorMap tmK,
                                                                const __grid_constant__ CUtensorMap tmV,
                                                                __nv_bfloat16* __restrict__ Aout,
+                                                               __nv_bfloat16* __restrict__ Aout_lo,
                                                                const int32_t* __restrict__ seg_ptr, int B, int N,
                                                                int H, int d, int kv_group, float scale_log2,
                                                                float* __restrict__ opart, int* __restrict__ part_cnt,
@@ -183,7 +189,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // same offset in both CTAs
-  uint8_t* sQ = smem;
+  uint8_t* sQ = smem;                  // q_hi tile; the q_lo tile follows at + kAttQBytes
   uint8_t* sK = smem + kAttOffK;
   uint8_t* sV = smem + kAttOffV;
   uint8_t* sP = smem + kAttOffP;  // buffer x: high part at 2x, low part at 2x + 1 (16 KB each)
@@ -192,10 +198,10 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAttOffBar);
   uint64_t* q_full = bars + 0;
   uint64_t* q_free = bars + 1;
-  uint64_t* k_full = bars + 2;    // [3]
-  uint64_t* k_empty = bars + 5;   // [3]
-  uint64_t* v_full = bars + 8;    // [3]
-  uint64_t* v_empty = bars + 11;  // [3]
+  uint64_t* k_full = bars + 2;    // [kAttStages <= 3]
+  uint64_t* k_empty = bars + 5;   // [kAttStages <= 3]
+  uint64_t* v_full = bars + 8;    // [kAttStages <= 3]
+  uint64_t* v_empty = bars + 11;  // [kAttStages <= 3]
   uint64_t* s_full = bars + 14;   // [2] scores of a chunk in TMEM
   uint64_t* s_free = bars + 16;   // [2] scores read by the 8 softmax warps
   uint64_t* p_full = bars + 18;   // [2] P of a chunk in shared memory (8 softmax warps)
@@ -249,6 +255,7 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
     *s_abort = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmQlo);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
@@ -279,9 +286,11 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
           *s_abort = 1;
           break;
         }
-        mbar_expect_tx(q_full, kAttQBytes);
+        mbar_expect_tx(q_full, 2 * kAttQBytes);
         tma_load_2d(sQ, &tmQ, hc, it.r0, q_full);
         tma_load_2d(sQ + kAttQBytes / 2, &tmQ, hc + 64, it.r0, q_full);
+        tma_load_2d(sQ + kAttQBytes, &tmQlo, hc, it.r0, q_full);
+        tma_load_2d(sQ + kAttQBytes + kAttQBytes / 2, &tmQlo, hc + 64, it.r0, q_full);
         for (int c = c0; c < c1; ++c, ++g) {
           const int st = (int)(g % kAttStages);
           const uint32_t ph = (uint32_t)((g / kAttStages) & 1);
@@ -350,8 +359,9 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
 #pragma unroll
           for (int k = 0; k < kAttHD / 16; ++k) {  // 16 dims per step: box k / 4, +32 B within it
             const uint32_t qa = q0 + (k >> 2) * (kAttQBytes / 2), ka = kb + (k >> 2) * (kAttKVBytes / 2);
-            umma_bf16(tmem_base + 128 + sb * 64, sdesc_sw128(qa) + 2 * (k & 3), sdesc_sw128(ka) + 2 * (k & 3),
-                      idesc_s, k > 0 ? 1u : 0u);
+            const uint64_t kdesc = sdesc_sw128(ka) + 2 * (k & 3);
+            umma_bf16(tmem_base + 128 + sb * 64, sdesc_sw128(qa) + 2 * (k & 3), kdesc, idesc_s, k > 0 ? 1u : 0u);
+            umma_bf16(tmem_base + 128 + sb * 64, sdesc_sw128(qa + kAttQBytes) + 2 * (k & 3), kdesc, idesc_s, 1u);
           }
           any = true;
           umma_commit(&s_full[sb]);
@@ -620,13 +630,17 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
           }
         }
         if (write_out && row < it.nrows) {
-          uint4* dst = reinterpret_cast<uint4*>(Aout + (size_t)grow * d + it.h * kAttHD + hf * 64);
+          const size_t off = (size_t)grow * d + it.h * kAttHD + hf * 64;
+          uint4* dst = reinterpret_cast<uint4*>(Aout + off);
+          uint4* dst_lo = reinterpret_cast<uint4*>(Aout_lo + off);
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            dst[v] = make_uint4(pack_bf16(o[8 * v + 0] * inv, o[8 * v + 1] * inv),
-                                pack_bf16(o[8 * v + 2] * inv, o[8 * v + 3] * inv),
-                                pack_bf16(o[8 * v + 4] * inv, o[8 * v + 5] * inv),
-                                pack_bf16(o[8 * v + 6] * inv, o[8 * v + 7] * inv));
+          for (int v = 0; v < 8; ++v) {
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) split_pair(o[8 * v + 2 * e] * inv, o[8 * v + 2 * e + 1] * inv, hi[e], lo[e]);
+            dst[v] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            dst_lo[v] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          }
         }
       }
       g += n;
@@ -682,12 +696,13 @@ __global__ void attn_f32_kernel(const float* __restrict__ Q, const float* __rest
   for (int c = 0; c < HD; ++c) A[(size_t)j * d + h * HD + c] = o[c] * inv;
 }
 
-int launch_attention_bf16(const plk_dims* dims, const void* q, const void* K_cache, const void* V_cache,
-                          void* a_out, const int32_t* seg_ptr, int num_sms, float* part_scratch,
-                          size_t part_bytes, int* part_cnt, cudaStream_t st) {
+int launch_attention_bf16(const plk_dims* dims, const void* q, const void* q_lo, const void* K_cache,
+                          const void* V_cache, void* a_out, void* a_lo, const int32_t* seg_ptr, int num_sms,
+                          float* part_scratch, size_t part_bytes, int* part_cnt, cudaStream_t st) {
   const int B = dims->B, N = dims->N, d = dims->d, H = dims->H, dkv = kv_width(dims);
-  CUtensorMap tmQ, tmK, tmV;
+  CUtensorMap tmQ, tmQlo, tmK, tmV;
   if (make_tmap_bf16(&tmQ, q, (uint64_t)B * N, (uint64_t)d, kAttBQ) != PLK_OK) return PLK_ERR_CUDA;
+  if (make_tmap_bf16(&tmQlo, q_lo, (uint64_t)B * N, (uint64_t)d, kAttBQ) != PLK_OK) return PLK_ERR_CUDA;
   if (make_tmap_bf16(&tmK, K_cache, (uint64_t)B * N, (uint64_t)dkv, kAttBK) != PLK_OK) return PLK_ERR_CUDA;
   if (make_tmap_bf16(&tmV, V_cache, (uint64_t)B * N, (uint64_t)dkv, kAttBK) != PLK_OK) return PLK_ERR_CUDA;
   static int attr_done[64] = {0};
@@ -717,7 +732,8 @@ int launch_attention_bf16(const plk_dims* dims, const void* q, const void* K_cac
   // partial tiles (128 x 128 fp32) and their (max, sum) rows that fit in the scratch
   const size_t tile_bytes = (size_t)kAttBQ * kAttHD * 4 + (size_t)kAttBQ * 8;
   const int part_cap = part_scratch ? (int)std::min(part_bytes / tile_bytes, (size_t)1 << 20) : 0;
-  if (cudaLaunchKernelEx(&cfg, attn_tc_kernel, tmQ, tmK, tmV, (__nv_bfloat16*)a_out, seg_ptr, B, N, H, d,
+  if (cudaLaunchKernelEx(&cfg, attn_tc_kernel, tmQ, tmQlo, tmK, tmV, (__nv_bfloat16*)a_out, (__nv_bfloat16*)a_lo,
+                         seg_ptr, B, N, H, d,
                          H / kv_heads(dims), scale_log2, part_scratch, part_cnt, part_cap) != cudaSuccess)
     return PLK_ERR_CUDA;
   return PLK_OK;

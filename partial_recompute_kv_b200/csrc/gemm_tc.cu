@@ -8,13 +8,17 @@
 //  * CTA pairs (cta_group::2): the even CTA issues one tcgen05.mma of
 //    M = 256 feature rows x N = 128 or 256 tokens that runs on the tensor cores
 //    of both SMs.  Each CTA stages its own 128 weight rows and HALF of the
-//    token tile, so an SM ingests 32 KB per 64-deep k-block instead of 48 KB
-//    for a one-CTA 128 x 256 tile: the operand feed (L2 -> SM), not the tensor
-//    pipe, bounds this GEMM at M <= 256 tokens.  Accumulation is fp32 in TMEM;
-//    each CTA's TMEM holds its 128 rows x N columns.
+//    token tile, so an SM ingests 16 KB of weights and 32 KB of activations
+//    (hi and lo, below) per 64-deep k-block instead of 16 + 64 KB for a one-CTA
+//    128 x 256 tile.  Accumulation is fp32 in TMEM; each CTA's TMEM holds its
+//    128 rows x N columns.
 //  * Weights are the A operand and the compacted activations the B operand;
-//    at M <= 256 every weight byte is read from HBM once.  Both are K-major
-//    bf16 tiles loaded by TMA with a 128-byte swizzle into a 6-stage ring.
+//    at M <= 256 every weight byte is read from HBM once.  The activation comes
+//    as a bf16 pair, X = Xhi + Xlo (Xlo = bf16(X - Xhi)), so that it enters the
+//    product with ~16 significant bits: every k-block stages one weight tile and
+//    both activation tiles, and the pair MMA runs W Xhi^T and W Xlo^T into the
+//    same fp32 accumulator.  All tiles are K-major bf16, loaded by TMA with a
+//    128-byte swizzle into a 4-stage ring of 48 KB stages.
 //  * Warp roles: warp 0 issues TMA in both CTAs, every load counting its bytes
 //    on the even CTA's stage barrier; one thread of warp 1 of the even CTA
 //    issues the pair MMAs; warps 2-5 of both CTAs drain their TMEM.
@@ -26,7 +30,8 @@
 //    (O and down projections) or a zeroed fp32 buffer that a finishing kernel
 //    turns into bf16 (QKV -> Q and the K/V cache rows; gate/up -> silu(g) u).
 //    The order of the adds is not fixed: results may differ in the last fp32
-//    bit between runs.
+//    bit between runs.  A tile piece accumulates its whole k range in TMEM
+//    before its one reduce-add.
 //  * Two 256-column TMEM accumulators per CTA: the epilogue drains one tile
 //    piece while the MMA fills the next; the producers run ahead across
 //    pieces.
@@ -45,9 +50,10 @@ namespace {
 
 constexpr int kHalfTok = kGemmBNMax / 2;            // token rows of B staged per CTA
 constexpr int kStageA = kGemmBM * kGemmBK * 2;      // 16 KB
-constexpr int kStageB = kHalfTok * kGemmBK * 2;     // 16 KB
+constexpr int kStageB = kHalfTok * kGemmBK * 2;     // 16 KB (hi part; the lo part the same)
 constexpr size_t kOffB = (size_t)kGemmStages * kStageA;
-constexpr size_t kOffBar = kOffB + (size_t)kGemmStages * kStageB;
+constexpr size_t kOffBlo = kOffB + (size_t)kGemmStages * kStageB;
+constexpr size_t kOffBar = kOffBlo + (size_t)kGemmStages * kStageB;
 constexpr size_t kOffStg = kOffBar + 256;
 constexpr int kBlk = 32 * 32;                       // a warp's block: 32 tokens x 32 features (fp32)
 constexpr size_t kSmemUsed = kOffStg + 4 * 2 * kBlk * 4;
@@ -55,14 +61,13 @@ constexpr size_t kSmemBytes = kSmemUsed + 1024;     // slack for 1024-byte align
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert((size_t)4 * 8 * kBlk * 4 <= kOffBar, "the last piece's blocks fit the operand ring");
 // Longest run of k-blocks accumulated in one TMEM chain before its partial is
-// added into the fp32 output.  The tensor core's fp32 accumulation loses a
-// little precision per step (measured: 0.14% of bf16-rounded q values differ
-// from an fp64 reference over 256 steps, 0.06% over 64, against 0.017% for
-// fp32 in sequence on the CPU); shorter chains summed by the L2 in fp32 keep
-// that loss small, but every chain is one more fp32 read-modify-write of its
-// tile (measured over the four projections: 16 k-blocks cost 5% at 256 tokens
-// and 15% at 2048 tokens against no limit).
-constexpr int kGemmChainKB = 32;
+// added into the fp32 output.  Every chain is one more fp32 read-modify-write
+// of its tile (measured over the four projections: chains of 16 k-blocks cost
+// 5% at 256 tokens and 15% at 2048 tokens against no limit).  With the
+// activations split into hi/lo pairs no bf16 rounding follows a sum before the
+// layer's stored outputs, so the small per-step drift of the tensor core's fp32
+// accumulation stays small against the bf16 step of K, V and Y: no limit.
+constexpr int kGemmChainKB = 1 << 20;
 
 // bulk reduce-add of a [32 rows][32 fp32] smem block into the tensor at (x, y)
 __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* tm, int x, int y, const void* smem_src) {
@@ -123,15 +128,17 @@ struct TileGeom {
 
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                   const __grid_constant__ CUtensorMap tmOut, const GemmArgs args) {
+                   const __grid_constant__ CUtensorMap tmXlo, const __grid_constant__ CUtensorMap tmOut,
+                   const GemmArgs args) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);  // same offset in both CTAs of a pair
   uint8_t* sA = smem;
   uint8_t* sB = smem + kOffB;
+  uint8_t* sBlo = smem + kOffBlo;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
-  uint64_t* full = bars;                        // [6] stage landed, both halves (even CTA's used)
-  uint64_t* empty = bars + kGemmStages;         // [6] stage consumed by the pair MMA
+  uint64_t* full = bars;                        // [stages] stage landed, both halves (even CTA's used)
+  uint64_t* empty = bars + kGemmStages;         // [stages] stage consumed by the pair MMA
   uint64_t* tfull = bars + 2 * kGemmStages;     // [2] accumulator ready for the epilogue
   uint64_t* tempty = bars + 2 * kGemmStages + 2;  // [2] accumulator drained (even CTA: 8 warps)
   uint64_t* drain = bars + 2 * kGemmStages + 4;   // MMA completion on the abort path
@@ -166,6 +173,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmXlo);
     tma_prefetch_desc(&tmOut);
   }
   if (warp == 1) {
@@ -194,9 +202,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tma_load_2d_pair(a, &tmW, kb * kGemmBK, yA0, fb);
         tma_load_2d_pair(a + 8192, &tmW, kb * kGemmBK, yA1, fb);
       };
-      // bytes of one stage, both CTAs: 2 x (A rows + half of the token rows)
+      // bytes of one stage, both CTAs: 2 x (A rows + hi and lo of half of the token rows)
       auto stage_bytes = [](const TileGeom& t) {
-        return (uint32_t)(2 * (kStageA + (t.ncols >> 7) * (64 * kGemmBK * 2)));
+        return (uint32_t)(2 * (kStageA + 2 * (t.ncols >> 7) * (64 * kGemmBK * 2)));
       };
       SegWalk w(pair, npairs, tiles, KB);
       int u, kb0, kb1, stage = 0;
@@ -231,8 +239,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             load_a(stage, t, kb);
           }
           uint8_t* b = sB + stage * kStageB;
-          for (int j = 0; j < nbox; ++j)
+          uint8_t* blo = sBlo + stage * kStageB;
+          for (int j = 0; j < nbox; ++j) {
             tma_load_2d_pair(b + j * 8192, &tmX, kb * kGemmBK, trow + j * 64, lead_full0 + (uint32_t)(stage * 8));
+            tma_load_2d_pair(blo + j * 8192, &tmXlo, kb * kGemmBK, trow + j * 64,
+                             lead_full0 + (uint32_t)(stage * 8));
+          }
           ++issued;
           if (++stage == kGemmStages) {
             stage = 0;
@@ -276,9 +288,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tc_fence_after();
             const uint64_t adesc = sdesc_sw128(smem_u32(sA + stage * kStageA));
             const uint64_t bdesc = sdesc_sw128(smem_u32(sB + stage * kStageB));
+            const uint64_t bdesc_lo = sdesc_sw128(smem_u32(sBlo + stage * kStageB));
 #pragma unroll
-            for (int k = 0; k < kGemmBK / 16; ++k)  // +32 bytes of K per step = 2 descriptor units
+            for (int k = 0; k < kGemmBK / 16; ++k) {  // +32 bytes of K per step = 2 descriptor units
               umma_bf16_pair(acc, adesc + 2 * k, bdesc + 2 * k, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+              umma_bf16_pair(acc, adesc + 2 * k, bdesc_lo + 2 * k, idesc, 1u);
+            }
             any = true;
             umma_commit_pair(smem_u32(&empty[stage]));  // the stage is free in both CTAs
             umma_commit_pair(peer_empty0 + (uint32_t)(stage * 8));
@@ -395,8 +410,8 @@ static int resident_pairs(int num_sms) {
   return n;
 }
 
-int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const CUtensorMap& tmOut, const GemmArgs& a,
-                   cudaStream_t st) {
+int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const CUtensorMap& tmXlo,
+                   const CUtensorMap& tmOut, const GemmArgs& a, cudaStream_t st) {
   if (a.ftiles <= 0 || (a.ftiles & 1) || a.K % kGemmBK != 0) return PLK_ERR_SHAPE;
   static int attr_done[64] = {0};
   int dev = 0;
@@ -424,7 +439,7 @@ int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const CUtenso
   at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
   cfg.numAttrs = 2;
-  if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel, tmW, tmX, tmOut, a) != cudaSuccess) return PLK_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel, tmW, tmX, tmXlo, tmOut, a) != cudaSuccess) return PLK_ERR_CUDA;
   return PLK_OK;
 }
 

@@ -4,21 +4,27 @@
 // "Algorithmic Complexity"), and the full-recompute baseline (Sec. 1).
 //
 // bf16 chain (10 launches, M read on the device, no host synchronisation):
-//   1 gather rows idx[j] of X, RMSNorm1 -> xn (bf16), x -> h (fp32), zero the QKV sums
+//   1 gather rows idx[j] of X, RMSNorm1 -> xn, x -> h (fp32), zero the QKV sums
 //   2 tcgen05 GEMM  xn W_qkv^T -> QKV sums (fp32, split-K reduce-adds)
-//   3 QKV sums -> Q (compact bf16), K and V scattered into the cache rows idx[j]
-//   4 attention of the M queries over all N cached keys -> a (bf16)
+//   3 QKV sums -> q (compact), K and V scattered into the cache rows idx[j] (bf16)
+//   4 attention of the M queries over all N cached keys -> a
 //   5 tcgen05 GEMM  h += a W_o^T (fp32)
-//   6 RMSNorm2(h) -> hn (bf16), zero the gate/up sums
+//   6 RMSNorm2(h) -> hn, zero the gate/up sums
 //   7 tcgen05 GEMM  hn [W_g; W_u]^T -> gate/up sums (fp32)
-//   8 act = silu(g) * u (bf16)
+//   8 act = silu(g) * u
 //   9 tcgen05 GEMM  h += act W_down^T (fp32)
 //  10 h -> Y rows idx[j] (bf16)
+// The layer stores bf16 only where its results land in the caller's tensors (the
+// K/V cache rows and Y).  Every activation that feeds a tensor-core product (xn,
+// q, a, hn, act) is held as a pair of bf16 tensors, hi = bf16(v) and
+// lo = bf16(v - hi), and enters the product as hi + lo: ~16 significant bits,
+// so the fp32 values between the stored tensors are not cut to bf16's 8.
 // fp32 chain: the same steps with SIMT GEMMs into an fp32 scratch and
 // elementwise epilogue kernels.
 #include <math.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "plk_common.cuh"
 #include "plk_internal.h"
@@ -56,12 +62,18 @@ Workspace workspace_layout(const plk_dims* dm, int num_sms) {
   };
   w.iota = take(4 * Mcap);
   w.seg = take(4 * ((size_t)dm->B + 1));
+  const size_t lo = dm->dtype == PLK_BF16 ? 1 : 0;  // bf16: low halves of the split activations
   w.xn = take(es * Mcap * d);
+  w.xn_lo = take(lo * es * Mcap * d);
   w.q = take(es * Mcap * d);
+  w.q_lo = take(lo * es * Mcap * d);
   w.a = take(es * Mcap * d);
+  w.a_lo = take(lo * es * Mcap * d);
   w.h32 = take(4 * Mcap * d);
   w.hn = take(es * Mcap * d);
+  w.hn_lo = take(lo * es * Mcap * d);
   w.act = take(es * Mcap * F);
+  w.act_lo = take(lo * es * Mcap * F);
   w.num_sms = num_sms;
   w.c32_bytes = 4 * Mcap * std::max(d + 2 * (size_t)kv_width(dm), 2 * F);
   w.c32 = take(w.c32_bytes);
@@ -139,13 +151,15 @@ __device__ __forceinline__ void clear_row(float* row, int zcols) {
 // out[j] = RMSNorm(src_row(j)) * g for j < M.  src_row(j) = X[idx[j]] (gather)
 // or H[j] (idx == nullptr); res_out (optional) receives the fp32 source row;
 // zero_out (optional) gets row j of a [Mcap, zcols] fp32 buffer cleared for the
-// reduce-adds of the GEMM that follows.
+// reduce-adds of the GEMM that follows.  With a bf16 output, out receives
+// hi = bf16(v) and out_lo (when given) lo = bf16(v - hi).
 template <typename Tin, typename Tg, typename Tout>
 __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const Tin* __restrict__ X, const int32_t* __restrict__ idx,
                                                            const int32_t* __restrict__ seg_ptr, int B,
                                                            const Tg* __restrict__ g, float eps, int d,
-                                                           Tout* __restrict__ out, float* __restrict__ res_out,
-                                                           float* __restrict__ zero_out, int zcols) {
+                                                           Tout* __restrict__ out, Tout* __restrict__ out_lo,
+                                                           float* __restrict__ res_out, float* __restrict__ zero_out,
+                                                           int zcols) {
   __shared__ float sh[33];
   pdl_wait();
   pdl_trigger();
@@ -164,7 +178,12 @@ __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const Tin* __restrict
   ss = block_sum_f(ss, sh);
   const float inv = 1.0f / sqrtf(ss / (float)d + eps);
   Tout* o = out + (size_t)j * d;
-  for (int c = threadIdx.x; c < d; c += blockDim.x) o[c] = from_f<Tout>(to_f(x[c]) * inv * to_f(g[c]));
+  for (int c = threadIdx.x; c < d; c += blockDim.x) {
+    const float v = to_f(x[c]) * inv * to_f(g[c]);
+    const Tout hi = from_f<Tout>(v);
+    o[c] = hi;
+    if (out_lo) out_lo[(size_t)j * d + c] = from_f<Tout>(v - to_f(hi));
+  }
 }
 
 // Same as rmsnorm_rows_kernel with the row held in registers: each thread loads
@@ -226,12 +245,27 @@ __device__ __forceinline__ void store_vec<float, 8>(float* dst, const float* y) 
   reinterpret_cast<float4*>(dst)[1] = make_float4(y[4], y[5], y[6], y[7]);
 }
 
+// The split of an activation that feeds a tensor-core product: hi = bf16(v) and
+// lo = bf16(v - hi), E consecutive values each.
+template <int E>
+__device__ __forceinline__ void store_hilo(__nv_bfloat16* hi, __nv_bfloat16* lo, const float* y) {
+  float h[E], l[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    h[e] = __bfloat162float(__float2bfloat16_rn(y[e]));
+    l[e] = y[e] - h[e];  // exact in fp32
+  }
+  store_vec<__nv_bfloat16, E>(hi, h);  // h is already a bf16 value
+  store_vec<__nv_bfloat16, E>(lo, l);
+}
+
 template <typename Tin, typename Tg, typename Tout, int NV>
 __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict__ X, const int32_t* __restrict__ idx,
                                                           const int32_t* __restrict__ seg_ptr, int B,
                                                           const Tg* __restrict__ g, float eps, int d,
-                                                          Tout* __restrict__ out, float* __restrict__ res_out,
-                                                          float* __restrict__ zero_out, int zcols) {
+                                                          Tout* __restrict__ out, Tout* __restrict__ out_lo,
+                                                          float* __restrict__ res_out, float* __restrict__ zero_out,
+                                                          int zcols) {
   constexpr int E = Vec16<Tin>::E;
   __shared__ float sh[33];
   pdl_wait();
@@ -271,6 +305,12 @@ __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict_
       if (res_out) store_vec<float, E>(res_out + (size_t)j * d + vi * E, f);
 #pragma unroll
       for (int e = 0; e < E; ++e) f[e] = f[e] * inv * to_f(g[vi * E + e]);
+      if constexpr (std::is_same<Tout, __nv_bfloat16>::value) {
+        if (out_lo) {
+          store_hilo<E>(o + vi * E, out_lo + (size_t)j * d + vi * E, f);
+          continue;
+        }
+      }
       store_vec<Tout, E>(o + vi * E, f);
     }
   }
@@ -279,14 +319,14 @@ __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict_
 // Picks the register-resident kernel when the row fits, else the looping one.
 template <typename Tin, typename Tg, typename Tout>
 static int launch_rmsnorm(const Tin* X, const int32_t* idx, const int32_t* seg, int B, const Tg* g, float eps,
-                           int d, Tout* out, int grid, cudaStream_t st, float* res_out = nullptr,
+                           int d, Tout* out, Tout* out_lo, int grid, cudaStream_t st, float* res_out = nullptr,
                            float* zero_out = nullptr, int zcols = 0) {
   constexpr int E = Vec16<Tin>::E;
   if (d % E == 0 && d <= 4 * 256 * E)
     return launch_pdl(rmsnorm_vec_kernel<Tin, Tg, Tout, 4>, dim3(grid), dim3(256), 0, st, X, idx, seg, B, g, eps, d,
-                      out, res_out, zero_out, zcols);
+                      out, out_lo, res_out, zero_out, zcols);
   return launch_pdl(rmsnorm_rows_kernel<Tin, Tg, Tout>, dim3(grid), dim3(256), 0, st, X, idx, seg, B, g, eps, d, out,
-                    res_out, zero_out, zcols);
+                    out_lo, res_out, zero_out, zcols);
 }
 
 // ---------------------------------------------------------------------------
@@ -313,8 +353,9 @@ __device__ __forceinline__ void rope_cs(int pos, int i, int hd, float log2_theta
   sincosf((float)a, &s, &c);
 }
 
-// [q | k | v] sums of compact row j (d + 2 dkv wide) -> Q[j] (compact, d wide) and
-// the K/V cache rows idx[j] (dkv wide: Hkv heads under grouped-query attention);
+// [q | k | v] sums of compact row j (d + 2 dkv wide) -> q[j] (compact, d wide, as
+// the hi/lo pair q, q_lo) and the K/V cache rows idx[j] (bf16, dkv wide: Hkv heads
+// under grouped-query attention);
 // with RoPE (log2_theta > 0) the heads of q and k are rotated by the row's
 // position idx[j] % N
 __global__ void __launch_bounds__(256) finish_qkv_kernel(const float* __restrict__ qkv32,
@@ -322,6 +363,7 @@ __global__ void __launch_bounds__(256) finish_qkv_kernel(const float* __restrict
                                                          const int32_t* __restrict__ seg_ptr, int B, int N, int d,
                                                          int dkv, int hd, float log2_theta,
                                                          __nv_bfloat16* __restrict__ q,
+                                                         __nv_bfloat16* __restrict__ q_lo,
                                                          __nv_bfloat16* __restrict__ Kc,
                                                          __nv_bfloat16* __restrict__ Vc, int* part_cnt) {
   pdl_wait();
@@ -355,25 +397,31 @@ __global__ void __launch_bounds__(256) finish_qkv_kernel(const float* __restrict
         x1[e] = a * cs - b * sn;
         x2[e] = a * sn + b * cs;
       }
-      __nv_bfloat16* dst = isq ? q + (size_t)j * d : Kc + row * dkv;
-      store_vec<__nv_bfloat16, 8>(dst + c1, x1);
-      store_vec<__nv_bfloat16, 8>(dst + c2, x2);
+      if (isq) {
+        store_hilo<8>(q + (size_t)j * d + c1, q_lo + (size_t)j * d + c1, x1);
+        store_hilo<8>(q + (size_t)j * d + c2, q_lo + (size_t)j * d + c2, x2);
+      } else {
+        store_vec<__nv_bfloat16, 8>(Kc + row * dkv + c1, x1);
+        store_vec<__nv_bfloat16, 8>(Kc + row * dkv + c2, x2);
+      }
     }
     for (int v = threadIdx.x + (rope ? (d + dkv) / 8 : 0); v < nv; v += blockDim.x) {  // with RoPE: v only
       const int c = v * 8;
       float f[8];
       load8(src + c, f);
-      __nv_bfloat16* dst = c < d ? q + (size_t)j * d + c
-                                 : (c < d + dkv ? Kc + row * dkv + (c - d) : Vc + row * dkv + (c - d - dkv));
-      store_vec<__nv_bfloat16, 8>(dst, f);
+      if (c < d)
+        store_hilo<8>(q + (size_t)j * d + c, q_lo + (size_t)j * d + c, f);
+      else
+        store_vec<__nv_bfloat16, 8>(c < d + dkv ? Kc + row * dkv + (c - d) : Vc + row * dkv + (c - d - dkv), f);
     }
   }
 }
 
-// [g | u] sums of compact row j -> act[j] = silu(g) * u
+// [g | u] sums of compact row j -> act[j] = silu(g) * u, as the hi/lo pair act, act_lo
 __global__ void __launch_bounds__(256) finish_gu_kernel(const float* __restrict__ gu32,
                                                         const int32_t* __restrict__ seg_ptr, int B, int F,
-                                                        __nv_bfloat16* __restrict__ act) {
+                                                        __nv_bfloat16* __restrict__ act,
+                                                        __nv_bfloat16* __restrict__ act_lo) {
   pdl_wait();
   pdl_trigger();
   const int M = seg_ptr[B];
@@ -386,7 +434,7 @@ __global__ void __launch_bounds__(256) finish_gu_kernel(const float* __restrict_
       load8(src + F + v * 8, u);
 #pragma unroll
       for (int e = 0; e < 8; ++e) g[e] = silu_f(g[e]) * u[e];
-      store_vec<__nv_bfloat16, 8>(act + (size_t)j * F + v * 8, g);
+      store_hilo<8>(act + (size_t)j * F + v * 8, act_lo + (size_t)j * F + v * 8, g);
     }
   }
 }
@@ -528,7 +576,8 @@ static int run_layer_f32(const plk_dims* dm, const plk_weights* w, const float* 
     dim3 grid(ceil_div(Nout, 64), ceil_div(Mcap, 64));
     gemm_f32_kernel<<<grid, 256, 0, st>>>(A, (const float*)Wt, c32, Nout, K, seg, B);
   };
-  PLK_TRY(launch_rmsnorm<float, float, float>(X, idx, seg, B, (const float*)w->g1, dm->eps, d, xn, Mcap, st));
+  PLK_TRY(launch_rmsnorm<float, float, float>(X, idx, seg, B, (const float*)w->g1, dm->eps, d, xn, nullptr, Mcap,
+                                              st));
   gemm(xn, w->w_qkv, d + 2 * dkv, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_QKV, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, dm->N,
                                             dm->hd, dm->rope_theta > 0.f ? log2f(dm->rope_theta) : 0.f, dkv);
@@ -536,7 +585,8 @@ static int run_layer_f32(const plk_dims* dm, const plk_weights* w, const float* 
   PLK_TRY(launch_attention_f32(dm, q, Kc, Vc, a, seg, Mcap, st));
   gemm(a, w->w_o, d, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_O, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, 0, 0, 0.f, 0);
-  PLK_TRY(launch_rmsnorm<float, float, float>(h32, nullptr, seg, B, (const float*)w->g2, dm->eps, d, hn, Mcap, st));
+  PLK_TRY(launch_rmsnorm<float, float, float>(h32, nullptr, seg, B, (const float*)w->g2, dm->eps, d, hn, nullptr,
+                                              Mcap, st));
   gemm(hn, w->w_gu, 2 * F, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_GU, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, 0, 0, 0.f, 0);
   gemm(act, w->w_down, d, F);
@@ -550,24 +600,35 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
                           const int32_t* seg, void* Kc, void* Vc, void* Y, uint8_t* ws, const Workspace& L,
                           cudaStream_t st) {
   const int B = dm->B, d = dm->d, F = dm->F, Mcap = dm->B * dm->N, dkv = kv_width(dm);
+  // activations that feed tensor-core products: hi/lo bf16 pairs
   __nv_bfloat16* xn = (__nv_bfloat16*)(ws + L.xn);
+  __nv_bfloat16* xn_lo = (__nv_bfloat16*)(ws + L.xn_lo);
   __nv_bfloat16* q = (__nv_bfloat16*)(ws + L.q);
+  __nv_bfloat16* q_lo = (__nv_bfloat16*)(ws + L.q_lo);
   __nv_bfloat16* a = (__nv_bfloat16*)(ws + L.a);
+  __nv_bfloat16* a_lo = (__nv_bfloat16*)(ws + L.a_lo);
   float* h32 = (float*)(ws + L.h32);
   __nv_bfloat16* hn = (__nv_bfloat16*)(ws + L.hn);
+  __nv_bfloat16* hn_lo = (__nv_bfloat16*)(ws + L.hn_lo);
   __nv_bfloat16* act = (__nv_bfloat16*)(ws + L.act);
+  __nv_bfloat16* act_lo = (__nv_bfloat16*)(ws + L.act_lo);
 
   float* c32 = (float*)(ws + L.c32);  // [Mcap, d + 2 dkv] QKV sums, later [Mcap, 2F] gate/up sums
 
-  CUtensorMap tW_qkv, tW_o, tW_gu, tW_down, tX_xn, tX_a, tX_hn, tX_act, tO_qkv, tO_h, tO_gu;
+  CUtensorMap tW_qkv, tW_o, tW_gu, tW_down, tO_qkv, tO_h, tO_gu;
+  CUtensorMap tX_xn[2], tX_a[2], tX_hn[2], tX_act[2];  // {hi, lo}
   PLK_TRY(make_tmap_bf16(&tW_qkv, w->w_qkv, (uint64_t)d + 2ull * dkv, d, 64));
   PLK_TRY(make_tmap_bf16(&tW_o, w->w_o, (uint64_t)d, d, 64));
   PLK_TRY(make_tmap_bf16(&tW_gu, w->w_gu, 2ull * F, d, 64));
   PLK_TRY(make_tmap_bf16(&tW_down, w->w_down, (uint64_t)d, F, 64));
-  PLK_TRY(make_tmap_bf16(&tX_xn, xn, (uint64_t)Mcap, d, 64));
-  PLK_TRY(make_tmap_bf16(&tX_a, a, (uint64_t)Mcap, d, 64));
-  PLK_TRY(make_tmap_bf16(&tX_hn, hn, (uint64_t)Mcap, d, 64));
-  PLK_TRY(make_tmap_bf16(&tX_act, act, (uint64_t)Mcap, F, 64));
+  PLK_TRY(make_tmap_bf16(&tX_xn[0], xn, (uint64_t)Mcap, d, 64));
+  PLK_TRY(make_tmap_bf16(&tX_xn[1], xn_lo, (uint64_t)Mcap, d, 64));
+  PLK_TRY(make_tmap_bf16(&tX_a[0], a, (uint64_t)Mcap, d, 64));
+  PLK_TRY(make_tmap_bf16(&tX_a[1], a_lo, (uint64_t)Mcap, d, 64));
+  PLK_TRY(make_tmap_bf16(&tX_hn[0], hn, (uint64_t)Mcap, d, 64));
+  PLK_TRY(make_tmap_bf16(&tX_hn[1], hn_lo, (uint64_t)Mcap, d, 64));
+  PLK_TRY(make_tmap_bf16(&tX_act[0], act, (uint64_t)Mcap, F, 64));
+  PLK_TRY(make_tmap_bf16(&tX_act[1], act_lo, (uint64_t)Mcap, F, 64));
   PLK_TRY(make_tmap_f32(&tO_qkv, c32, (uint64_t)Mcap, (uint64_t)d + 2ull * dkv));
   PLK_TRY(make_tmap_f32(&tO_h, h32, (uint64_t)Mcap, d));
   PLK_TRY(make_tmap_f32(&tO_gu, c32, (uint64_t)Mcap, 2ull * F));
@@ -581,48 +642,49 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   trace_mark(0, st);
   // x (fp32) staged in h32 takes the O projection's adds; the QKV sums start at 0
   PLK_TRY(launch_rmsnorm<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(X, idx, seg, B, (const __nv_bfloat16*)w->g1,
-                                                                      dm->eps, d, xn, Mcap, st, h32, c32,
-                                                                      d + 2 * dkv));
+                                                                      dm->eps, d, xn, xn_lo, Mcap, st, h32,
+                                                                      c32, d + 2 * dkv));
   trace_mark(1, st);
 
   g.K = d;
   g.ftiles = (d + 2 * dkv) / kGemmBM;
   g.gu_F = 0;
-  PLK_TRY(launch_gemm_tc(tW_qkv, tX_xn, tO_qkv, g, st));
+  PLK_TRY(launch_gemm_tc(tW_qkv, tX_xn[0], tX_xn[1], tO_qkv, g, st));
   trace_mark(2, st);
 
   const float log2_theta = dm->rope_theta > 0.f ? log2f(dm->rope_theta) : 0.f;
   int* part_cnt = (int*)(ws + L.xn);  // RMSNorm1's output, consumed by the QKV GEMM
   PLK_TRY(launch_pdl(finish_qkv_kernel, dim3(rgrid), dim3(256), 0, st, (const float*)c32, idx, seg, B, dm->N, d,
-                     dkv, dm->hd, log2_theta, q, (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc, part_cnt));
+                     dkv, dm->hd, log2_theta, q, q_lo, (__nv_bfloat16*)Kc, (__nv_bfloat16*)Vc, part_cnt));
   trace_mark(3, st);
 
   // the QKV sums are consumed: c32 holds the attention's partial outputs until the gate/up GEMM
-  PLK_TRY(launch_attention_bf16(dm, q, Kc, Vc, a, seg, L.num_sms, c32, L.c32_bytes, part_cnt, st));
+  PLK_TRY(launch_attention_bf16(dm, q, q_lo, Kc, Vc, a, a_lo, seg, L.num_sms, c32, L.c32_bytes, part_cnt, st));
   trace_mark(4, st);
 
   g.K = d;
   g.ftiles = d / kGemmBM;
-  PLK_TRY(launch_gemm_tc(tW_o, tX_a, tO_h, g, st));  // h = x + a W_o^T
+  PLK_TRY(launch_gemm_tc(tW_o, tX_a[0], tX_a[1], tO_h, g, st));  // h = x + a W_o^T
   trace_mark(5, st);
 
   PLK_TRY(launch_rmsnorm<float, __nv_bfloat16, __nv_bfloat16>(h32, nullptr, seg, B, (const __nv_bfloat16*)w->g2,
-                                                              dm->eps, d, hn, Mcap, st, nullptr, c32, 2 * F));
+                                                              dm->eps, d, hn, hn_lo, Mcap, st, nullptr, c32,
+                                                              2 * F));
   trace_mark(6, st);
 
   g.K = d;
   g.ftiles = F / 64;
   g.gu_F = F;
-  PLK_TRY(launch_gemm_tc(tW_gu, tX_hn, tO_gu, g, st));
+  PLK_TRY(launch_gemm_tc(tW_gu, tX_hn[0], tX_hn[1], tO_gu, g, st));
   trace_mark(7, st);
 
-  PLK_TRY(launch_pdl(finish_gu_kernel, dim3(rgrid), dim3(256), 0, st, (const float*)c32, seg, B, F, act));
+  PLK_TRY(launch_pdl(finish_gu_kernel, dim3(rgrid), dim3(256), 0, st, (const float*)c32, seg, B, F, act, act_lo));
   trace_mark(8, st);
 
   g.K = F;
   g.ftiles = d / kGemmBM;
   g.gu_F = 0;
-  PLK_TRY(launch_gemm_tc(tW_down, tX_act, tO_h, g, st));  // y = h + act W_down^T
+  PLK_TRY(launch_gemm_tc(tW_down, tX_act[0], tX_act[1], tO_h, g, st));  // y = h + act W_down^T
   trace_mark(9, st);
 
   PLK_TRY(launch_pdl(finish_y_kernel, dim3(rgrid), dim3(256), 0, st, (const float*)h32, idx, seg, B, d,

@@ -17,7 +17,7 @@ namespace plk {
 constexpr int kGemmBM = 128;      // feature rows per CTA (a CTA pair computes 256)
 constexpr int kGemmBNMax = 256;   // tokens per tile (UMMA N, runtime 128 or 256; each CTA loads half)
 constexpr int kGemmBK = 64;       // K per stage: one 128-byte swizzle row of bf16
-constexpr int kGemmStages = 6;
+constexpr int kGemmStages = 4;  // 48 KB each: weight tile + the hi and lo activation tiles
 constexpr int kGemmThreads = 192; // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 
 // ---- attention key split over several CTA pairs --------------------------------
@@ -55,6 +55,7 @@ struct Workspace {
   // offsets (bytes)
   size_t iota = 0, seg = 0;              // identity active set for the full step
   size_t xn = 0, q = 0, a = 0, h32 = 0, hn = 0, act = 0;
+  size_t xn_lo = 0, q_lo = 0, a_lo = 0, hn_lo = 0, act_lo = 0;  // bf16: low halves (v - bf16(v))
   size_t c32 = 0;                        // fp32 GEMM sums [Mcap, max(d + 2 dkv, 2F)] (QKV, then gate/up;
                                          // in between, the attention's partial outputs)
   size_t c32_bytes = 0;
@@ -87,12 +88,17 @@ int launch_kl_lock(const plk_dims* dims, int V, const void* logits_t, const void
 int launch_slowfast(const plk_dims* dims, const plk_sf_params* prm, const float* conf, uint8_t* masked,
                     plk_sf_state* state, uint8_t* unmask_out, uint8_t* lock_out, cudaStream_t st);
 
+// The argument checks shared by the layer-step entry points (PLK_OK or the error code).
+int check_layer_args(const plk_dims* dims, const plk_weights* w, const void* X, const int32_t* idx,
+                     const int32_t* seg_ptr, const void* K_cache, const void* V_cache, const void* Y);
+
 int run_layer(const plk_dims* dims, const plk_weights* w, const void* X, const int32_t* idx,
               const int32_t* seg_ptr, bool full, void* K_cache, void* V_cache, void* Y, void* ws,
               size_t ws_bytes, cudaStream_t st);
 
-// Arguments of the tcgen05 GEMM out[t, f] += sum_k X[t, k] W[f, k] over the
-// M = seg_ptr[B] compact tokens (fp32 out, added with bulk reduce-adds).
+// Arguments of the tcgen05 GEMM out[t, f] += sum_k (Xhi[t, k] + Xlo[t, k]) W[f, k]
+// over the M = seg_ptr[B] compact tokens (fp32 out, added with bulk reduce-adds;
+// the activation enters as its bf16 hi/lo pair).
 struct GemmArgs {
   int K;                   // reduction length, multiple of 64
   int ftiles;              // 128-row feature tiles (even: a CTA pair takes two)
@@ -101,15 +107,16 @@ struct GemmArgs {
   int B;
   int num_sms;             // SM count: at most one persistent CTA per SM, in pairs
 };
-int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmX, const CUtensorMap& tmOut, const GemmArgs& a,
-                   cudaStream_t st);
+int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmXhi, const CUtensorMap& tmXlo,
+                   const CUtensorMap& tmOut, const GemmArgs& a, cudaStream_t st);
 
 // part_scratch / part_bytes: free device memory for the partial outputs of a key
 // split over several CTA pairs (used when the units leave pairs idle); part_cnt:
 // kAttPartCounters ints, zero on entry, zero again on exit.
-int launch_attention_bf16(const plk_dims* dims, const void* q, const void* K_cache, const void* V_cache,
-                          void* a_out, const int32_t* seg_ptr, int num_sms, float* part_scratch,
-                          size_t part_bytes, int* part_cnt, cudaStream_t st);
+// q, q_lo: the queries as a bf16 hi/lo pair; a_out, a_lo: the output as one.
+int launch_attention_bf16(const plk_dims* dims, const void* q, const void* q_lo, const void* K_cache,
+                          const void* V_cache, void* a_out, void* a_lo, const int32_t* seg_ptr, int num_sms,
+                          float* part_scratch, size_t part_bytes, int* part_cnt, cudaStream_t st);
 int launch_attention_f32(const plk_dims* dims, const float* q, const float* K_cache, const float* V_cache,
                          float* a_out, const int32_t* seg_ptr, int Mcap, cudaStream_t st);
 

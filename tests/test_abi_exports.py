@@ -117,6 +117,7 @@ def test_struct_layouts_match_the_header(tmp_path):
         for fname, _ in py._fields_:
             lines.append(f'  printf("{cname} {fname} %zu\\n", offsetof({cname}, {fname}));')
     lines.append('  printf("plk_sf_state size %zu\\n", sizeof(plk_sf_state));')
+    lines.append('  printf("PLK_STATIC_WS_BYTES %zu\\n", (size_t)PLK_STATIC_WS_BYTES);')
     lines += ["  return 0;", "}"]
     src = tmp_path / "layout.c"
     src.write_text("\n".join(lines) + "\n")
@@ -130,3 +131,4 @@ def test_struct_layouts_match_the_header(tmp_path):
         for fname, _ in py._fields_:
             assert got[f"{cname} {fname}"] == getattr(py, fname).offset, (cname, fname)
     assert got["plk_sf_state size"] == 4 * plk.SF_STATE_WORDS
+    assert got["PLK_STATIC_WS_BYTES"] == plk.STATIC_WS_BYTES  # the binding's copy of the static array's size
