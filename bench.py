@@ -45,14 +45,18 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # workload (seeded synthetic inputs shared by both arms)
 # ---------------------------------------------------------------------------
 class Workload:
-    def __init__(self, frac=0.25, rank=128, seed=0):
+    def __init__(self, frac=0.25, rank=128, seed=0, share=None):
+        """share: another Workload of the same seed and rank whose weights, X and U are reused."""
         import synth
         self.D = synth.LAYER_8B
         self.frac, self.r = frac, rank
         self.M = synth.active_count(self.D.N, frac)
-        self.W = synth.layer_weights(self.D, synth.LAYER_8B_WSTD, seed=seed)
-        self.X = synth.hidden_states(self.D, seed=seed)
-        self.Ut = synth.proxy_basis(self.D.d, rank, seed=seed)
+        if share is not None:
+            self.W, self.X, self.Ut = share.W, share.X, share.Ut
+        else:
+            self.W = synth.layer_weights(self.D, synth.LAYER_8B_WSTD, seed=seed)
+            self.X = synth.hidden_states(self.D, seed=seed)
+            self.Ut = synth.proxy_basis(self.D.d, rank, seed=seed)
         self.pos = synth.layer_8b_positions(self.D.N, frac, seed=seed)
         mask = np.zeros((self.D.B, self.D.N), bool)
         mask[0, self.pos] = True
@@ -70,6 +74,12 @@ class Workload:
     def weight_bytes(self):
         D = self.D
         return 2 * (4 * D.d * D.d + 3 * D.d * D.F)
+
+    def gemm_bytes(self):
+        """Algorithmic DRAM bytes of the four projections of one step: every weight once, the
+        activations read once as bf16, the fp32 sums written once."""
+        D, M = self.D, self.M
+        return self.weight_bytes() + M * (2 * (3 * D.d + D.F) + 4 * (5 * D.d + 2 * D.F))
 
     def config(self, l2="stream"):
         D = self.D
@@ -246,8 +256,8 @@ def run_reference(args, wl):
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline(wl, budget_s=15.0):
-    run = OracleRunner(wl)
+def cpu_baseline(wl, budget_s=15.0, run=None):
+    run = run or OracleRunner(wl)
     t0 = time.perf_counter()
     units, steps = 0, 0
     while True:
@@ -546,15 +556,19 @@ def run_kernel_configs(args):
     by = 2 * D.B * D.N * D.d + 8 * D.B * D.N * r + 2 * D.d * r
     out.append({"kernel": "score_tc_kernel", "config": f"B={D.B} N={D.N} d={D.d} r={r} L2", "us": us,
                 "GB/s": by / (us * 1e-6) / 1e9, "frac_of_hbm": by / (us * 1e-6) / 1e9 / hbm})
-    k = D.N * 10 // 100
+    score_us = us
     lk_in = torch.zeros((D.B, D.N), dtype=torch.uint8, device=dev)
     lk, idx = torch.empty_like(lk_in), torch.empty(D.B * D.N, dtype=torch.int32, device=dev)
     seg = torch.empty(D.B + 1, dtype=torch.int32, device=dev)
-    us = _timed(torch, lambda: plk.select_active(dm, score, lk_in, lk, plk.SEL_TOPK_LARGEST, 0.0, k, idx, seg),
-                args.steps, args.warmup)
-    by = 6 * D.B * D.N + 4 * D.B * k
-    out.append({"kernel": "topk_compact_kernel", "config": f"B={D.B} N={D.N} k={k}", "us": us,
-                "GB/s": by / (us * 1e-6) / 1e9, "frac_of_hbm": by / (us * 1e-6) / 1e9 / hbm})
+    for pct in synth.SCORE_PCTS:  # the per-layer budget k = {5, 10, 20}% of N (SPA-Cache part 2)
+        k = D.N * pct // 100
+        us = _timed(torch, lambda: plk.select_active(dm, score, lk_in, lk, plk.SEL_TOPK_LARGEST, 0.0, k, idx, seg),
+                    args.steps, args.warmup)
+        by = 6 * D.B * D.N + 4 * D.B * k
+        out.append({"kernel": "topk_compact_kernel", "config": f"B={D.B} N={D.N} k={k} ({pct}% of N)", "us": us,
+                    "GB/s": by / (us * 1e-6) / 1e9, "frac_of_hbm": by / (us * 1e-6) / 1e9 / hbm,
+                    "scoring_layer_us": score_us + us,
+                    "scoring_32_layers_us": 32 * (score_us + us)})
     del X, pc, pnew
     # stack step 0: B = 4, N = 2048, every row active
     D = synth.STACK_8B
@@ -998,6 +1012,53 @@ def run_long(args):
     return 0
 
 
+# ---------------------------------------------------------------------------
+# the active-fraction sweep (--kernel sweep): the headline step at every active
+# fraction of the 8B-shape layer, M/N in {1, 1/2, 1/4, 1/10, 1/20} (SureLock page,
+# Sec. 2 "Algorithmic Complexity": the per-step work falls with the active count
+# M_t <= N); one JSON line per fraction with the projections' roofline taken
+# against the tensor peak where their arithmetic intensity is above the ridge
+# and against HBM below it, and the CPU oracle beside it
+# ---------------------------------------------------------------------------
+def run_sweep(args):
+    import synth
+
+    base = Workload(frac=synth.LAYER_8B_FRACTIONS[0])
+    oracle_base = None
+    for frac in synth.LAYER_8B_FRACTIONS:
+        wl = Workload(frac=frac, share=base)
+        res = run_gpu(args, wl, None, 0, 1, 0)
+        pk = res["peaks"]
+        per = res["per_kernel_us"]
+        gemm_us = per["gemm_qkv"] + per["gemm_o"] + per["gemm_gu"] + per["gemm_down"]
+        flops, by = wl.M * wl.gemm_flops_per_row(), wl.gemm_bytes()
+        tfl, hbm = float(pk["bf16_tflops"]), float(pk["hbm_gbs"])
+        ridge = tfl * 1e12 / (hbm * 1e9)
+        t_achieved = flops / (gemm_us * 1e-6) / 1e12
+        b_achieved = by / (gemm_us * 1e-6) / 1e9
+        if flops / by >= ridge:
+            roof = {"bound": "tensor", "achieved": t_achieved, "peak": tfl, "unit": "TFLOP/s", "frac": t_achieved / tfl}
+        else:
+            roof = {"bound": "hbm", "achieved": b_achieved, "peak": hbm, "unit": "GB/s", "frac": b_achieved / hbm}
+        roof.update({"kernel": "gemm_tc_kernel (4 launches)", "intensity_flop_per_byte": flops / by, "ridge": ridge,
+                     "tensor_frac": t_achieved / tfl, "hbm_frac": b_achieved / hbm, "alg_flops": flops,
+                     "alg_bytes": by, "peak_source": pk.get("source"), "traffic": None})
+        if oracle_base is None:
+            oracle_base = OracleRunner(wl)
+        run = OracleRunner.__new__(OracleRunner)
+        run.__dict__.update(oracle_base.__dict__)
+        run.wl, run.pc = wl, oracle_base.pc.copy()
+        line = {"metric": f"active-token-layers/sec at 8B-shape, M/N={frac}", "value": res["value"], "unit": UNIT,
+                "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
+                "decode_steps_per_s": 1e3 / res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": wl.config(args.l2),
+                "roofline": roof, "step_tflops": res["step_tflops"], "per_kernel_us": per,
+                "e2e": res["e2e"], "clocks": res["clocks"],
+                "cpu_baseline": cpu_baseline(wl, budget_s=6.0, run=run)}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1011,8 +1072,12 @@ def main():
                     help="replay the step as one captured CUDA graph (default)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="enqueue the step's library calls directly every step")
-    ap.add_argument("--kernel", choices=["step", "kl_lock", "slowfast", "configs", "stack", "long"], default="step",
-                    help="step: the headline layer step; kl_lock: the KL lock rule alone; slowfast: the SlowFast "
+    ap.add_argument("--frac", type=float, default=0.25,
+                    help="active fraction M/N of the headline step (the metric is quoted at 0.25)")
+    ap.add_argument("--kernel", choices=["step", "sweep", "kl_lock", "slowfast", "configs", "stack", "long"],
+                    default="step",
+                    help="step: the headline layer step; sweep: the step at every active fraction 1, 1/2, 1/4, "
+                         "1/10, 1/20; kl_lock: the KL lock rule alone; slowfast: the SlowFast "
                          "span policy over whole decodes; configs: scoring and the all-active stack step at the "
                          "shapes where their rooflines are judged; stack: the 32-layer stack over the 256-step "
                          "schedule; long: the long-context block decode at N = 8192")
@@ -1034,10 +1099,12 @@ def main():
         return run_long(args) if rank == 0 else 0
     if args.kernel == "configs":
         return run_kernel_configs(args) if rank == 0 else 0
+    if args.kernel == "sweep":
+        return run_sweep(args) if rank == 0 else 0
     if args.impl == "reference":
         if rank != 0:
             return 0
-        run_reference(args, Workload())
+        run_reference(args, Workload(frac=args.frac))
         return 0
 
     dist = None
@@ -1049,7 +1116,7 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
-    wl = Workload()
+    wl = Workload(frac=args.frac)
     try:
         res = run_gpu(args, wl, dist, rank, world, local_rank)
     finally:
@@ -1058,7 +1125,8 @@ def main():
     if res is None or rank != 0:
         return 0
     launches_per_step = 1 + 1 + 10 + 1  # score, select, layer, commit
-    line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+    metric = METRIC if args.frac == 0.25 else f"active-token-layers/sec at 8B-shape, M/N={args.frac}"
+    line = {"metric": metric, "value": res["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": dict(wl.config(args.l2), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),

@@ -62,3 +62,50 @@ def tdtype(dims):
 def weights_dev(W, dims):
     dt = tdtype(dims)
     return {k: dev(v, dt) for k, v in W.items()}
+
+
+class Guarded:
+    """A device tensor with guard bands of a known byte pattern on both sides.
+
+    compute-sanitizer is not available to these tests, so a write past either end
+    of a buffer would go unseen; the guard bands catch it: ``check()`` asserts
+    that every guard byte still holds the pattern.  The tensor starts at a
+    4096-byte offset into its allocation (alignment kept for TMA and vector
+    accesses)."""
+
+    PATTERN = 0xA5
+    GUARD = 4096
+
+    def __init__(self, shape, dtype, init=None, fill=None, device="cuda"):
+        shape = tuple(int(s) for s in shape)
+        n = int(np.prod(shape)) if shape else 1
+        esize = torch.empty((), dtype=dtype).element_size()
+        self.nbytes = n * esize
+        body = (self.nbytes + 1023) // 1024 * 1024
+        self.raw = torch.full((2 * self.GUARD + body,), self.PATTERN, dtype=torch.uint8, device=device)
+        self.t = self.raw[self.GUARD:self.GUARD + self.nbytes].view(dtype).view(shape)
+        if init is not None:
+            self.t.copy_(init if isinstance(init, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(init)))
+        elif fill is not None:
+            self.t.fill_(fill)
+
+    def check(self, what):
+        if self.raw.is_cuda:
+            torch.cuda.synchronize()
+        head = self.raw[:self.GUARD]
+        tail = self.raw[self.GUARD + self.nbytes:]
+        bad_h = int((head != self.PATTERN).sum())
+        bad_t = int((tail != self.PATTERN).sum())
+        assert bad_h == 0 and bad_t == 0, f"{what}: {bad_h} guard bytes before and {bad_t} after the tensor changed"
+
+
+def check_guards(guards, what):
+    for name, g in guards.items():
+        g.check(f"{what}: {name}")
+
+
+def guarded_workspace(plk, dm):
+    n = plk.workspace_bytes(dm)
+    if n == 0:
+        raise plk.PlkError(plk.ERR_SHAPE, "workspace_bytes")
+    return Guarded((n,), torch.uint8)

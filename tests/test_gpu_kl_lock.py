@@ -16,7 +16,7 @@ import torch
 
 import oracle
 import synth
-from tests.parity_util import dev, host
+from tests.parity_util import Guarded, check_guards, dev, host
 
 pytestmark = pytest.mark.gpu
 
@@ -31,11 +31,12 @@ def _run(plk, zt, zp, lock_in, eps, h_max, dtype):
     B, N, V = zt.shape
     dm = plk.dims(B, N, 256, 2, 128, 512, dtype=plk.BF16 if dtype == "bf16" else plk.F32)
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
-    lk = torch.from_numpy(lock_in.copy()).cuda()
-    kl = torch.full((B, N), -7.0, dtype=torch.float32, device="cuda")
-    h = torch.full((B, N), -7.0, dtype=torch.float32, device="cuda")
+    g = {"lock": Guarded((B, N), torch.uint8, init=lock_in), "kl": Guarded((B, N), torch.float32, fill=-7.0),
+         "h": Guarded((B, N), torch.float32, fill=-7.0)}
+    lk, kl, h = g["lock"].t, g["kl"].t, g["h"].t
     plk.kl_lock(dm, V, dev(zt, tdt), dev(zp, tdt), lk, lk, eps, h_max, kl, h)  # lock in place
     assert plk.get_status() == plk.OK
+    check_guards(g, "kl_lock")
     return host(lk), host(kl), host(h)
 
 

@@ -13,7 +13,8 @@ import torch
 
 import oracle
 import synth
-from tests.parity_util import assert_bf16_close, assert_f32_close, dev, host, metrics, tdtype, weights_dev
+from tests.parity_util import (Guarded, assert_bf16_close, assert_f32_close, check_guards, dev, guarded_workspace,
+                               host, metrics, tdtype, weights_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -38,10 +39,15 @@ def int_dev(a, n):
     return t
 
 
+_SEL_GUARDS = {}
+
+
 def sel_bufs(B, N):
-    idx = torch.full((B * N,), -1, dtype=torch.int32, device="cuda")
-    seg = torch.full((B + 1,), -7, dtype=torch.int32, device="cuda")
-    return idx, seg
+    gi = Guarded((B * N,), torch.int32, fill=-1)
+    gs = Guarded((B + 1,), torch.int32, fill=-7)
+    _SEL_GUARDS[gi.t.data_ptr()] = gi
+    _SEL_GUARDS[gs.t.data_ptr()] = gs
+    return gi.t, gs.t
 
 
 def check_compaction(idx, seg, ref_lock):
@@ -51,6 +57,10 @@ def check_compaction(idx, seg, ref_lock):
     hi = host(idx)
     assert np.array_equal(hi[:M], ref_idx)
     assert np.all(hi[M:] == -1), "nothing past M is written"
+    for t, name in ((idx, "idx"), (seg, "seg_ptr")):  # and nothing outside the buffers
+        g = _SEL_GUARDS.get(t.data_ptr())
+        if g is not None:
+            g.check(name)
 
 
 # ---------------------------------------------------------------------------
@@ -68,14 +78,18 @@ def test_select_threshold_bitexact(plk, B, N, gt, inplace):
     tau = np.float32(0.5)
     ref = oracle.lock_threshold(s.astype(np.float64), lock, float(tau), greater=gt)
     dm = plk.dims(B, N, 64, 4, 16, 64, dtype=plk.F32)
-    score, lin = dev(s, torch.float32), dev(lock, torch.uint8)
-    lout = lin if inplace else torch.full_like(lin, 9)
+    score = dev(s, torch.float32)
+    glin = Guarded((B, N), torch.uint8, init=lock)
+    lin = glin.t
+    glout = glin if inplace else Guarded((B, N), torch.uint8, fill=9)
+    lout = glout.t
     idx, seg = sel_bufs(B, N)
     plk.select_active(dm, score, lin, lout, plk.SEL_THRESH_GT if gt else plk.SEL_THRESH_LT, float(tau), 0,
                       idx, seg)
     torch.cuda.synchronize()
     assert np.array_equal(host(lout), ref)
     check_compaction(idx, seg, ref)
+    check_guards({"lock_in": glin, "lock_out": glout}, "threshold select")
 
 
 @pytest.mark.parametrize("B,N", [(1, 5), (2, 777), (8, 4096)])
@@ -96,13 +110,15 @@ def test_select_topk_bitexact(plk, B, N, kind, largest):
     score, lin = dev(s, torch.float32), dev(lock, torch.uint8)
     for k in sorted({0, 1, max(N // 10, 1), N // 2, N, N + 5}):
         ref = oracle.lock_topk(s.astype(np.float64), lock, k, largest)
-        lout = torch.full_like(lin, 9)
+        glout = Guarded((B, N), torch.uint8, fill=9)
+        lout = glout.t
         idx, seg = sel_bufs(B, N)
         plk.select_active(dm, score, lin, lout, plk.SEL_TOPK_LARGEST if largest else plk.SEL_TOPK_SMALLEST,
                           0.0, k, idx, seg)
         torch.cuda.synchronize()
         assert np.array_equal(host(lout), ref), f"k={k}"
         check_compaction(idx, seg, ref)
+        glout.check(f"top-k select k={k}: lock_out")
 
 
 # ---------------------------------------------------------------------------
@@ -127,13 +143,15 @@ def test_score_drift(plk, dtype, metric):
     pc = pc.astype(np.float32).reshape(D.B, D.N, r)
     ref_s, ref_p = oracle.score_drift(X.astype(np.float64), Ut.astype(np.float64), pc, metric)
     dm = pdims(plk, D)
-    score = torch.empty((D.B, D.N), dtype=torch.float32, device="cuda")
-    pout = torch.empty((D.B, D.N, r), dtype=torch.float32, device="cuda")
+    gs = Guarded((D.B, D.N), torch.float32)
+    gp = Guarded((D.B, D.N, r), torch.float32)
+    score, pout = gs.t, gp.t
     plk.score_drift(dm, dev(X, tdtype(D)), dev(Ut, tdtype(D)), r, dev(pc, torch.float32),
                     plk.METRIC_COS if metric == "cos" else plk.METRIC_L2, score, proxy_out=pout)
     torch.cuda.synchronize()
     assert_f32_close(host(pout), ref_p, "proxy", tol=1e-5)
     assert_f32_close(host(score), ref_s, "score", tol=1e-4)
+    check_guards({"score": gs, "proxy_out": gp}, "score_drift")
 
 
 def test_score_drift_8b_shape_repeated(plk):
@@ -168,10 +186,11 @@ def test_proxy_commit(plk):
     idx, seg = oracle.compact(lock)
     ref = oracle.proxy_commit(pc, pn, idx)
     dm = plk.dims(B, N, 64, 4, 16, 64, dtype=plk.F32)
-    pcd = dev(pc, torch.float32)
-    plk.proxy_commit(dm, r, int_dev(idx, B * N), int_dev(seg, B + 1), dev(pn, torch.float32), pcd)
+    gpc = Guarded((B, N, r), torch.float32, init=pc)
+    plk.proxy_commit(dm, r, int_dev(idx, B * N), int_dev(seg, B + 1), dev(pn, torch.float32), gpc.t)
     torch.cuda.synchronize()
-    assert np.array_equal(host(pcd), ref)
+    assert np.array_equal(host(gpc.t), ref)
+    gpc.check("proxy_commit: proxy_cache")
 
 
 # ---------------------------------------------------------------------------
@@ -180,14 +199,34 @@ def test_proxy_commit(plk):
 SMALL = synth.Dims(B=2, N=320, d=512, H=4, hd=128, F=1536, dtype="bf16")
 
 
-def _run_partial(plk, D, W, X, idx, seg, st):
+def _run_layer_guarded(plk, D, Wd, X, idx, seg, st, dt=BF, what="layer step"):
+    """plk_layer_step_partial with the caches, the active set and the workspace inside guard bands;
+    returns the caches (host, float64) after checking that no guard byte changed."""
     dm = pdims(plk, D)
-    K, V, Y = dev(st.K, BF), dev(st.V, BF), dev(st.Y, BF)
-    ws = plk.alloc_workspace(dm)
-    plk.layer_step_partial(dm, weights_dev(W, D), dev(X, BF), int_dev(idx, D.B * D.N), int_dev(seg, D.B + 1),
-                           K, V, Y, ws)
+    g = {"K": Guarded(st.K.shape, dt, init=dev(st.K, dt)), "V": Guarded(st.V.shape, dt, init=dev(st.V, dt)),
+         "Y": Guarded(st.Y.shape, dt, init=dev(st.Y, dt)),
+         "idx": Guarded((D.B * D.N,), torch.int32, init=int_dev(idx, D.B * D.N)),
+         "seg_ptr": Guarded((D.B + 1,), torch.int32, init=int_dev(seg, D.B + 1)),
+         "workspace": guarded_workspace(plk, dm)}
+    plk.layer_step_partial(dm, Wd, dev(X, dt), g["idx"].t, g["seg_ptr"].t, g["K"].t, g["V"].t, g["Y"].t,
+                           g["workspace"].t)
     assert plk.get_status() == plk.OK
-    return host(K), host(V), host(Y)
+    check_guards(g, what)
+    return host(g["K"].t), host(g["V"].t), host(g["Y"].t)
+
+
+def _run_full_guarded(plk, D, Wd, X, dt=BF, what="full step"):
+    dm = pdims(plk, D)
+    g = {"K": Guarded((D.B, D.N, D.dkv), dt, fill=0), "V": Guarded((D.B, D.N, D.dkv), dt, fill=0),
+         "Y": Guarded((D.B, D.N, D.d), dt, fill=0), "workspace": guarded_workspace(plk, dm)}
+    plk.full_layer_step(dm, Wd, dev(X, dt), g["K"].t, g["V"].t, g["Y"].t, g["workspace"].t)
+    assert plk.get_status() == plk.OK
+    check_guards(g, what)
+    return host(g["K"].t), host(g["V"].t), host(g["Y"].t)
+
+
+def _run_partial(plk, D, W, X, idx, seg, st):
+    return _run_layer_guarded(plk, D, weights_dev(W, D), X, idx, seg, st)
 
 
 def test_full_layer_step_bf16(plk):
@@ -195,15 +234,10 @@ def test_full_layer_step_bf16(plk):
     W = synth.layer_weights(D, 0.02, seed=1)
     X = synth.hidden_states(D, seed=1)
     ref = oracle.full_layer_step(D, W, X, "bf16")
-    dm = pdims(plk, D)
-    K = torch.zeros((D.B, D.N, D.d), dtype=BF, device="cuda")
-    V, Y = torch.zeros_like(K), torch.zeros_like(K)
-    ws = plk.alloc_workspace(dm)
-    plk.full_layer_step(dm, weights_dev(W, D), dev(X, BF), K, V, Y, ws)
-    assert plk.get_status() == plk.OK
-    assert_bf16_close(host(K), ref.K, "K")
-    assert_bf16_close(host(V), ref.V, "V")
-    assert_bf16_close(host(Y), ref.Y, "Y")
+    K, V, Y = _run_full_guarded(plk, D, weights_dev(W, D), X)
+    assert_bf16_close(K, ref.K, "K")
+    assert_bf16_close(V, ref.V, "V")
+    assert_bf16_close(Y, ref.Y, "Y")
 
 
 @pytest.mark.parametrize("p_active", [0.05, 0.3, 1.0])
@@ -355,14 +389,18 @@ def test_workspace_too_small_is_rejected(plk):
 # ---------------------------------------------------------------------------
 # the tiny fp32 workload: 20 denoising steps, every step checked
 # ---------------------------------------------------------------------------
-def test_tiny_fp32_driver(plk):
+@pytest.mark.parametrize("noise_var", [synth.TINY_NOISE_VAR, 0.1])
+def test_tiny_fp32_driver(plk, noise_var):
+    """The tiny fp32 workload step by step.  With its own noise (variance 0.01) the active set
+    empties within four steps; with variance 0.1 it shrinks from 13 rows to 1 over the 20 steps,
+    so the fp32 layer runs on several rows at every step (decision margins >= 2e-4 from tau)."""
     D = synth.TINY
     r = synth.TINY_RANK
     W = synth.layer_weights(D, 1.0 / math.sqrt(D.d))
     X0 = synth.hidden_states(D)
     Ut = synth.proxy_basis(D.d, r, dtype="f32")
     lock0 = synth.bernoulli_active(D.B, D.N, synth.TINY_P_ACTIVE)
-    noises = [synth.step_noise((D.B, D.N, D.d), synth.TINY_NOISE_VAR, step=t) for t in range(synth.TINY_STEPS)]
+    noises = [synth.step_noise((D.B, D.N, D.d), noise_var, step=t) for t in range(synth.TINY_STEPS)]
     perturb = lambda X, e, m: synth.perturb_rows(X, e, m, "f32")
     recs = oracle.tiny_run(D, W, X0, Ut.astype(np.float64), lock0, noises, synth.TINY_TAU, perturb)
 
@@ -426,13 +464,9 @@ def _check_layer_rows(K, V, Y, ref, base, lock, what):
 def test_layer_8b_full_step(plk, layer_8b):
     """The full-recompute baseline at the 8B shape: every row of K, V and Y."""
     D, base = layer_8b["D"], layer_8b["base"]
-    dm = pdims(plk, D)
-    K = torch.zeros((D.B, D.N, D.d), dtype=BF, device="cuda")
-    V, Y = torch.zeros_like(K), torch.zeros_like(K)
-    plk.full_layer_step(dm, layer_8b["Wd"], dev(layer_8b["X"], BF), K, V, Y, plk.alloc_workspace(dm))
-    assert plk.get_status() == plk.OK
+    K, V, Y = _run_full_guarded(plk, D, layer_8b["Wd"], layer_8b["X"], what="8B full step")
     for g, o, name in ((K, base.K, "K"), (V, base.V, "V"), (Y, base.Y, "Y")):
-        assert_bf16_close(host(g), o, f"8B full step {name}")
+        assert_bf16_close(g, o, f"8B full step {name}")
 
 
 @pytest.mark.parametrize("frac", synth.LAYER_8B_FRACTIONS)
@@ -448,12 +482,7 @@ def test_layer_8b_fraction(plk, layer_8b, frac, record_property):
     assert idx.size == synth.active_count(D.N, frac)
     X2 = synth.perturb_rows(layer_8b["X"], synth.step_noise((1, D.N, D.d), 0.01), lock == 0, "bf16")
     ref = oracle.layer_step_partial(D, W, X2, idx, seg, base, "bf16")
-    dm = pdims(plk, D)
-    K, V, Y = dev(base.K, BF), dev(base.V, BF), dev(base.Y, BF)
-    plk.layer_step_partial(dm, layer_8b["Wd"], dev(X2, BF), int_dev(idx, D.N), int_dev(seg, 2), K, V, Y,
-                           plk.alloc_workspace(dm))
-    assert plk.get_status() == plk.OK
-    K, V, Y = host(K), host(V), host(Y)
+    K, V, Y = _run_layer_guarded(plk, D, layer_8b["Wd"], X2, idx, seg, base, what=f"8B M/N={frac}")
     res = _check_layer_rows(K, V, Y, ref, base, lock, f"8B M/N={frac}")
     for name, (mr, mae) in res.items():
         record_property(f"{name}_max_rel", mr)
@@ -492,12 +521,8 @@ def test_layer_8b_stack_last_step(plk):
         lock[b, rng.choice(D.N, Mt, replace=False)] = 0
     idx, seg = oracle.compact(lock)
     ref = oracle.layer_step_partial(D, W, X, idx, seg, st, "bf16")
-    dm = pdims(plk, D)
-    K, V, Y = dev(st.K, BF), dev(st.V, BF), dev(st.Y, BF)
-    plk.layer_step_partial(dm, weights_dev(W, D), dev(X, BF), int_dev(idx, D.B * D.N), int_dev(seg, D.B + 1),
-                           K, V, Y, plk.alloc_workspace(dm))
-    assert plk.get_status() == plk.OK
-    _check_layer_rows(host(K), host(V), host(Y), ref, st, lock, "stack t=255")
+    K, V, Y = _run_layer_guarded(plk, D, weights_dev(W, D), X, idx, seg, st, what="stack t=255")
+    _check_layer_rows(K, V, Y, ref, st, lock, "stack t=255")
 
 
 def test_layer_8b_long_context_block(plk):
@@ -514,12 +539,8 @@ def test_layer_8b_long_context_block(plk):
     idx, seg = oracle.compact(lock)
     assert idx.size == M
     ref = oracle.layer_step_partial(D, W, X, idx, seg, st, "bf16")
-    dm = pdims(plk, D)
-    K, V, Y = dev(st.K, BF), dev(st.V, BF), dev(st.Y, BF)
-    plk.layer_step_partial(dm, weights_dev(W, D), dev(X, BF), int_dev(idx, D.N), int_dev(seg, 2), K, V, Y,
-                           plk.alloc_workspace(dm))
-    assert plk.get_status() == plk.OK
-    _check_layer_rows(host(K), host(V), host(Y), ref, st, lock, "long-context block 0")
+    K, V, Y = _run_layer_guarded(plk, D, weights_dev(W, D), X, idx, seg, st, what="long-context block 0")
+    _check_layer_rows(K, V, Y, ref, st, lock, "long-context block 0")
 
 
 # ---------------------------------------------------------------------------

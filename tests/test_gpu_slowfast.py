@@ -11,6 +11,7 @@ import torch
 
 import synth
 from oracle import plk_oracle as po
+from tests.parity_util import Guarded, check_guards
 
 pytestmark = pytest.mark.gpu
 
@@ -33,10 +34,14 @@ def _trajectory(B, N, prompt, steps, seed, rate=16.0, nan_every=0, outputs=True,
     prm.update(kw)
     dm, params, op = _dims(B, N), plk.sf_params(**prm), po.SpanParams(**prm)
     m_or = synth.generation_mask(B, N, prompt)
-    m_dev = torch.from_numpy(m_or.copy()).cuda()
-    st_dev = plk.sf_state(B)
-    un = torch.full((B, N), 7, dtype=torch.uint8, device="cuda") if outputs else None
-    lk = torch.full((B, N), 7, dtype=torch.uint8, device="cuda") if outputs else None
+    guards = {"masked": Guarded((B, N), torch.uint8, init=m_or), "state": Guarded((B, plk.SF_STATE_WORDS), torch.int32,
+                                                                                  fill=0)}
+    if outputs:
+        guards["unmask"] = Guarded((B, N), torch.uint8, fill=7)
+        guards["lock"] = Guarded((B, N), torch.uint8, fill=7)
+    m_dev, st_dev = guards["masked"].t, guards["state"].t
+    un = guards["unmask"].t if outputs else None
+    lk = guards["lock"].t if outputs else None
     states = [po.SpanState() for _ in range(B)]
     phases = set()
     for t in range(steps):
@@ -56,6 +61,7 @@ def _trajectory(B, N, prompt, steps, seed, rate=16.0, nan_every=0, outputs=True,
             phases.add(states[b].phase)
         if not m_or.any():
             break
+    check_guards(guards, "slowfast trajectory")
     return t + 1, phases, m_or
 
 
