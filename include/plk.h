@@ -306,6 +306,12 @@ int plk_set_wait_limit(long long cycles);
  * word.  Exists to test the timeout path without faulting or hanging a GPU. */
 int plk_selftest_wait_timeout(void* stream);
 
+/* out[i] = 2^t[i] (n values, device pointers) by the exponential the attention
+ * softmax computes on the FMA pipe for part of its weights (range reduction to
+ * [-1/2, 1/2] and a degree-4 minimax polynomial; relative error <= 3e-6; t < -126
+ * gives 0).  Exists so that the polynomial can be tested against exp2 on a GPU. */
+int plk_selftest_exp2(const float* t, float* out, int n, void* stream);
+
 /* Tracing.  Registers up to 16 cudaEvent_t handles (passed as void*).  While
  * registered, plk_layer_step_partial and plk_full_layer_step record events[0]
  * on their stream before their first kernel and events[i] after their i-th

@@ -28,7 +28,7 @@ EXPORTED = (
     "plk_proxy_commit", "plk_layer_step_partial_static", "plk_kl_lock", "plk_slowfast_step", "plk_workspace_bytes",
     "plk_get_status",
     "plk_set_wait_limit",
-    "plk_selftest_wait_timeout", "plk_trace_events", "plk_error_string", "plk_version",
+    "plk_selftest_wait_timeout", "plk_selftest_exp2", "plk_trace_events", "plk_error_string", "plk_version",
 )
 
 
@@ -78,6 +78,7 @@ def _load():
         "plk_get_status": (I, [P]),
         "plk_set_wait_limit": (I, [L]),
         "plk_selftest_wait_timeout": (I, [P]),
+        "plk_selftest_exp2": (I, [P, P, I, P]),
         "plk_trace_events": (I, [ctypes.POINTER(ctypes.c_void_p), I]),
         "plk_error_string": (ctypes.c_char_p, [I]),
         "plk_version": (I, []),
@@ -244,6 +245,13 @@ def trace_events(events):
 
 def selftest_wait_timeout(stream=None):
     _check(lib.plk_selftest_wait_timeout(_stream(stream)), "selftest_wait_timeout")
+
+
+def selftest_exp2(t, out, stream=None):
+    """out = 2^t by the attention softmax's FMA-pipe exponential (fp32 tensors of equal size)."""
+    if t.dtype != torch.float32 or out.dtype != torch.float32 or t.numel() != out.numel():
+        raise ValueError("t and out must be float32 tensors of the same size")
+    _check(lib.plk_selftest_exp2(_ptr(t), _ptr(out), int(t.numel()), _stream(stream)), "selftest_exp2")
 
 
 def alloc_workspace(dm, device="cuda"):

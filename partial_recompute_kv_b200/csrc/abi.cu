@@ -173,6 +173,12 @@ __global__ void selftest_wait_kernel() {
 }
 }  // namespace plk
 
+extern "C" int plk_selftest_exp2(const float* t, float* out, int n, void* stream) {
+  if (n < 0 || (n > 0 && (!t || !out))) return PLK_ERR_ARG;
+  if (n == 0) return PLK_OK;
+  return plk::launch_exp2_selftest(t, out, n, (cudaStream_t)stream);
+}
+
 extern "C" int plk_selftest_wait_timeout(void* stream) {
   plk::selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>();
   return cudaPeekAtLastError() == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;

@@ -7,10 +7,12 @@
 // bf16, hd = 128, on the tcgen05 tensor cores: a CTA takes 128 active queries
 // of one sequence and one head and a contiguous range of 64-key chunks.  The
 // queries come as a bf16 pair q = q_hi + q_lo (q_lo = bf16(q - q_hi)), so the
-// scores see ~16 significant bits of q.  Warp 0 stages both Q tiles once and K,
-// V chunk by chunk with TMA (128-byte swizzle, 2-stage rings); one thread of
-// warp 1 issues S = Q_hi K^T + Q_lo K^T into TMEM (double-buffered, 64 columns
-// each) and O += P V into TMEM (128 columns); warps 2-5 own one
+// scores see ~16 significant bits of q.  Warp 0 stages both Q tiles once and K
+// chunk by chunk, warp 10 stages V chunk by chunk, with TMA (128-byte swizzle;
+// a 3-stage K ring and a 2-stage V ring, each with its own producer so a K load
+// never waits behind a V stage); one thread of warp 1 issues
+// S = Q_hi K^T + Q_lo K^T into TMEM (double-buffered, 64 columns each) and
+// O += P V into TMEM (128 columns); warps 2-5 own one
 // query row per thread: they read the row's scores from TMEM, keep the running
 // row max and sum (online softmax), and write P to shared memory as a bf16 high
 // part and a bf16 residual, both multiplied with V, so the softmax weights
@@ -42,15 +44,17 @@ namespace {
 constexpr int kAttHD = 128;
 constexpr int kAttBQ = 128;                    // queries per CTA (UMMA M, one TMEM lane each)
 constexpr int kAttBK = 64;                     // keys per chunk (UMMA N of S, K of P V)
-constexpr int kAttStages = 2;                  // K and V ring depth
+constexpr int kAttKStages = 3;                 // K ring depth
+constexpr int kAttVStages = 2;                 // V ring depth
 constexpr int kAttSoftWarps = 8;               // two warps per TMEM lane quarter, one per half row
-constexpr int kAttThreads = 32 * (2 + kAttSoftWarps);  // warp 0 TMA, warp 1 MMA, warps 2-9 softmax
+constexpr int kAttVWarp = 2 + kAttSoftWarps;   // warp 10: the V producer
+constexpr int kAttThreads = 32 * (3 + kAttSoftWarps);  // warp 0 Q/K TMA, warp 1 MMA, warps 2-9 softmax, warp 10 V TMA
 constexpr int kAttQBytes = kAttBQ * kAttHD * 2;   // 32 KB (hi or lo part)
 constexpr int kAttKVBytes = kAttBK * kAttHD * 2;  // 16 KB
 constexpr int kAttPBytes = kAttBQ * kAttBK * 2;   // 16 KB (high or low part)
 constexpr size_t kAttOffK = 2 * (size_t)kAttQBytes;
-constexpr size_t kAttOffV = kAttOffK + (size_t)kAttStages * kAttKVBytes;
-constexpr size_t kAttOffP = kAttOffV + (size_t)kAttStages * kAttKVBytes;  // [2 buffers][high, low]
+constexpr size_t kAttOffV = kAttOffK + (size_t)kAttKStages * kAttKVBytes;
+constexpr size_t kAttOffP = kAttOffV + (size_t)kAttVStages * kAttKVBytes;  // [2 buffers][high, low]
 constexpr size_t kAttOffML = kAttOffP + 4 * (size_t)kAttPBytes;            // [128] (max, sum) of the odd CTA
 constexpr size_t kAttOffXM = kAttOffML + kAttBQ * 8;                       // [2][2 halves][128] row max
 constexpr size_t kAttOffXL = kAttOffXM + 2 * 2 * kAttBQ * 4;               // [2 halves][128] row sum
@@ -65,6 +69,41 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+// The softmax weights as a bf16 pair without conversion instructions: hi keeps
+// the upper 16 bits of each fp32 weight (bf16 by truncation), the remainder
+// x - hi is exact in fp32, and lo keeps its upper 16 bits.  For 0 <= x the pair
+// hi + lo is within 2^-15 x below x (16 significant bits), computed on the
+// integer and FMA pipes only; the packed element order matches bf16x2 (x0 low).
+__device__ __forceinline__ void split_pair_trunc(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const uint32_t u0 = __float_as_uint(x0), u1 = __float_as_uint(x1);
+  hi = __byte_perm(u0, u1, 0x7632);
+  const float r0 = x0 - __uint_as_float(u0 & 0xFFFF0000u);
+  const float r1 = x1 - __uint_as_float(u1 & 0xFFFF0000u);
+  lo = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
+}
+
+// 2^t on the FMA and integer pipes, for a share of the softmax's exponentials
+// (the rest go to the MUFU unit's ex2): Cody-Waite style reduction t = n + f with
+// n = round(t) (1.5 * 2^23 added and subtracted in fp32) and f in [-1/2, 1/2];
+// 2^f by the degree-4 polynomial minimising the relative error on that interval
+// (Remez exchange fit; 2.7e-6 maximum in fp32 Horner form, against 2^-15 of the
+// bf16 pair the weights are stored in); 2^n added to the exponent field.
+// t < -126 gives 0 (below any weight that matters: weights are <= 2^8 here).
+__device__ __forceinline__ float exp2_fma(float t) {
+  const float tc = fmaxf(t, -126.0f);
+  const float j = tc + 12582912.0f;  // the low mantissa bits of j hold n
+  const float f = tc - (j - 12582912.0f);
+  float p = 9.5701022e-3f;
+  p = fmaf(p, f, 5.5917859e-2f);
+  p = fmaf(p, f, 2.4024744e-1f);
+  p = fmaf(p, f, 6.9312179e-1f);
+  p = fmaf(p, f, 9.9999928e-1f);
+  const float r = __int_as_float(__float_as_int(p) + (__float_as_int(j) << 23));
+  return t >= -126.0f ? r : 0.0f;
+}
+// every kAttPolyEvery-th exponential of a thread's chunk row goes to exp2_fma
+constexpr int kAttPolyEvery = 4;
+
 // hi = bf16(x) packed, lo = bf16(x - hi) packed
 __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uint32_t& lo) {
   const __nv_bfloat16 h0 = __float2bfloat16_rn(x0), h1 = __float2bfloat16_rn(x1);
@@ -198,10 +237,10 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAttOffBar);
   uint64_t* q_full = bars + 0;
   uint64_t* q_free = bars + 1;
-  uint64_t* k_full = bars + 2;    // [kAttStages <= 3]
-  uint64_t* k_empty = bars + 5;   // [kAttStages <= 3]
-  uint64_t* v_full = bars + 8;    // [kAttStages <= 3]
-  uint64_t* v_empty = bars + 11;  // [kAttStages <= 3]
+  uint64_t* k_full = bars + 2;    // [kAttKStages <= 3]
+  uint64_t* k_empty = bars + 5;   // [kAttKStages <= 3]
+  uint64_t* v_full = bars + 8;    // [kAttVStages <= 3]
+  uint64_t* v_empty = bars + 11;  // [kAttVStages <= 3]
   uint64_t* s_full = bars + 14;   // [2] scores of a chunk in TMEM
   uint64_t* s_free = bars + 16;   // [2] scores read by the 8 softmax warps
   uint64_t* p_full = bars + 18;   // [2] P of a chunk in shared memory (8 softmax warps)
@@ -231,9 +270,11 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     mbar_init(q_free, 1);
-    for (int i = 0; i < kAttStages; ++i) {
+    for (int i = 0; i < kAttKStages; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
+    }
+    for (int i = 0; i < kAttVStages; ++i) {
       mbar_init(&v_full[i], 1);
       mbar_init(&v_empty[i], 1);
     }
@@ -292,8 +333,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
         tma_load_2d(sQ + kAttQBytes, &tmQlo, hc, it.r0, q_full);
         tma_load_2d(sQ + kAttQBytes + kAttQBytes / 2, &tmQlo, hc + 64, it.r0, q_full);
         for (int c = c0; c < c1; ++c, ++g) {
-          const int st = (int)(g % kAttStages);
-          const uint32_t ph = (uint32_t)((g / kAttStages) & 1);
+          const int st = (int)(g % kAttKStages);
+          const uint32_t ph = (uint32_t)((g / kAttKStages) & 1);
           const int y = it.b * N + c * kAttBK;
           if (!mbar_wait(&k_empty[st], ph ^ 1)) {
             *s_abort = 1;
@@ -302,6 +343,23 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
           mbar_expect_tx(&k_full[st], kAttKVBytes);
           tma_load_2d(sK + st * kAttKVBytes, &tmK, kc, y, &k_full[st]);
           tma_load_2d(sK + st * kAttKVBytes + kAttKVBytes / 2, &tmK, kc + 64, y, &k_full[st]);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == kAttVWarp) {
+    // ------------------------------------------------------------ V producer
+    if (elect_one()) {
+      long long g = 0;
+      for (int w = plan.first; w < plan.items && !*s_abort; w += plan.stride) {
+        const AttnUnit it = attn_unit(w / plan.parts, seg_ptr, B, H);
+        int c0, c1;
+        attn_chunks(plan, w, rank, nch, c0, c1);
+        const int kc = (it.h / kv_group) * kAttHD;
+        for (int c = c0; c < c1; ++c, ++g) {
+          const int st = (int)(g % kAttVStages);
+          const uint32_t ph = (uint32_t)((g / kAttVStages) & 1);
+          const int y = it.b * N + c * kAttBK;
           if (!mbar_wait(&v_empty[st], ph ^ 1)) {
             *s_abort = 1;
             break;
@@ -324,10 +382,10 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
       bool any = false;
       // O += P_hi V + P_lo V for global chunk gj (first: the unit's first chunk overwrites O)
       auto issue_pv = [&](long long gj, bool first) -> bool {
-        const int pb = (int)(gj & 1), st = (int)(gj % kAttStages);
+        const int pb = (int)(gj & 1), st = (int)(gj % kAttVStages);
         if (first && !mbar_wait(o_free, (uint32_t)((t & 1) ^ 1))) return false;  // last unit's O read
         if (!mbar_wait(&p_full[pb], (uint32_t)((gj >> 1) & 1))) return false;
-        if (!mbar_wait(&v_full[st], (uint32_t)((gj / kAttStages) & 1))) return false;
+        if (!mbar_wait(&v_full[st], (uint32_t)((gj / kAttVStages) & 1))) return false;
         tc_fence_after();
         const uint32_t vb = smem_u32(sV + st * kAttKVBytes);
 #pragma unroll
@@ -350,9 +408,9 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
         tc_fence_after();
         for (int j = 0; j < n && ok; ++j) {
           const long long gj = g + j;
-          const int sb = (int)(gj & 1), st = (int)(gj % kAttStages);
+          const int sb = (int)(gj & 1), st = (int)(gj % kAttKStages);
           ok = mbar_wait(&s_free[sb], (uint32_t)(((gj >> 1) & 1) ^ 1)) &&
-               mbar_wait(&k_full[st], (uint32_t)((gj / kAttStages) & 1));
+               mbar_wait(&k_full[st], (uint32_t)((gj / kAttKStages) & 1));
           if (!ok) break;
           tc_fence_after();
           const uint32_t kb = smem_u32(sK + st * kAttKVBytes);
@@ -490,10 +548,12 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
           uint32_t hi[4], lo[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float p0 = exp2f(fmaf(sc[cc * 8 + 2 * e], scale_log2, -m_used));
-            const float p1 = exp2f(fmaf(sc[cc * 8 + 2 * e + 1], scale_log2, -m_used));
+            const int i0 = cc * 8 + 2 * e, i1 = i0 + 1;
+            const float t0 = fmaf(sc[i0], scale_log2, -m_used), t1 = fmaf(sc[i1], scale_log2, -m_used);
+            const float p0 = (i0 % kAttPolyEvery == kAttPolyEvery - 1) ? exp2_fma(t0) : exp2f(t0);
+            const float p1 = (i1 % kAttPolyEvery == kAttPolyEvery - 1) ? exp2_fma(t1) : exp2f(t1);
             l += p0 + p1;
-            split_pair(p0, p1, hi[e], lo[e]);
+            split_pair_trunc(p0, p1, hi[e], lo[e]);
           }
           const uint32_t off = rowoff + ((uint32_t)((hf * 4 + cc) ^ (row & 7)) << 4);
           *reinterpret_cast<uint4*>(ph + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
@@ -538,10 +598,14 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
           ok = false;
           break;
         }
-        const uint32_t xo = dsmem_addr(smem_u32(sP), 0) + (uint32_t)(row * kAttHD + hf * 64) * 4;
+        // row r's 32 16-byte slots, slot c at r * 32 + (c ^ (r & 7)): the 32 rows of a warp's
+        // store cover every bank (a plain row-major tile would put all 32 on the same banks)
+        const uint32_t xo = dsmem_addr(smem_u32(sP), 0);
 #pragma unroll
-        for (int v = 0; v < 16; ++v)
-          st_dsmem_v4(xo + v * 16, make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]));
+        for (int v = 0; v < 16; ++v) {
+          const int slot = row * 32 + ((hf * 16 + v) ^ (row & 7));
+          st_dsmem_v4(xo + (uint32_t)slot * 16, make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]));
+        }
         if (hf == 0) st_dsmem_v2(dsmem_addr(smem_u32(ml), 0) + row * 8, make_float2(m_used, l_row));
         asm volatile("fence.acq_rel.cluster;" ::: "memory");
         __syncwarp();
@@ -563,9 +627,15 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
           const float w_odd = exp2f(pm.x - m);
           m_row = m;
           l_tot = w_own * l_row + w_odd * pm.y;
-          const float* xo = reinterpret_cast<const float*>(sP) + row * kAttHD + hf * 64;
+          const float4* xo = reinterpret_cast<const float4*>(sP);
 #pragma unroll
-          for (int e = 0; e < 64; ++e) o[e] = fmaf(w_own, o[e], w_odd * xo[e]);
+          for (int v = 0; v < 16; ++v) {
+            const float4 x = xo[row * 32 + ((hf * 16 + v) ^ (row & 7))];
+            o[4 * v] = fmaf(w_own, o[4 * v], w_odd * x.x);
+            o[4 * v + 1] = fmaf(w_own, o[4 * v + 1], w_odd * x.y);
+            o[4 * v + 2] = fmaf(w_own, o[4 * v + 2], w_odd * x.z);
+            o[4 * v + 3] = fmaf(w_own, o[4 * v + 3], w_odd * x.w);
+          }
           // the next unit's P may overwrite the partial once every softmax warp has read it
           __syncwarp();
           if (lane == 0) mbar_arrive(xo_read);
@@ -575,10 +645,12 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
         if (plan.parts > 1) {
           // this pair's key range is one part of the unit: store (O, max, sum), unnormalised,
           // and let the pair that completes the unit last merge the parts
+          // column-major partial tiles ([item][column][row]): a warp's store of one column is
+          // 32 consecutive rows, 128 contiguous bytes
           float2* mlp = reinterpret_cast<float2*>(opart + (size_t)part_cap * kAttBQ * kAttHD);
-          float4* op = reinterpret_cast<float4*>(opart + ((size_t)w * kAttBQ + row) * kAttHD + hf * 64);
+          float* op = opart + ((size_t)w * kAttHD + hf * 64) * kAttBQ + row;
 #pragma unroll
-          for (int v = 0; v < 16; ++v) op[v] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+          for (int e = 0; e < 64; ++e) op[(size_t)e * kAttBQ] = o[e];
           if (hf == 0) mlp[(size_t)w * kAttBQ + row] = make_float2(m_row, l_tot);
           __threadfence();
           __syncwarp();
@@ -615,15 +687,9 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
               const float2 pq = __ldcg(&mlp[(w0 + q2) * kAttBQ + row]);
               const float wq = exp2f(pq.x - mm);
               lt = fmaf(wq, pq.y, lt);
-              const float4* src = reinterpret_cast<const float4*>(opart + ((w0 + q2) * kAttBQ + row) * kAttHD + hf * 64);
+              const float* src = opart + ((w0 + q2) * kAttHD + hf * 64) * kAttBQ + row;
 #pragma unroll
-              for (int v = 0; v < 16; ++v) {
-                const float4 x = __ldcg(src + v);
-                o[4 * v] = fmaf(wq, x.x, o[4 * v]);
-                o[4 * v + 1] = fmaf(wq, x.y, o[4 * v + 1]);
-                o[4 * v + 2] = fmaf(wq, x.z, o[4 * v + 2]);
-                o[4 * v + 3] = fmaf(wq, x.w, o[4 * v + 3]);
-              }
+              for (int e = 0; e < 64; ++e) o[e] = fmaf(wq, __ldcg(src + (size_t)e * kAttBQ), o[e]);
             }
             inv = 1.0f / lt;
             if (warp == 2 && lane == 0) part_cnt[u] = 0;  // every part has counted: reset for the next launch
@@ -737,6 +803,15 @@ int launch_attention_bf16(const plk_dims* dims, const void* q, const void* q_lo,
                          H / kv_heads(dims), scale_log2, part_scratch, part_cnt, part_cap) != cudaSuccess)
     return PLK_ERR_CUDA;
   return PLK_OK;
+}
+
+__global__ void exp2_selftest_kernel(const float* __restrict__ t, float* __restrict__ out, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) out[i] = exp2_fma(t[i]);
+}
+
+int launch_exp2_selftest(const float* t, float* out, int n, cudaStream_t st) {
+  exp2_selftest_kernel<<<std::min(ceil_div(std::max(n, 1), 256), 1024), 256, 0, st>>>(t, out, n);
+  return cudaPeekAtLastError() == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;
 }
 
 int launch_attention_f32(const plk_dims* dims, const float* q, const float* K_cache, const float* V_cache,

@@ -117,6 +117,8 @@ int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmXhi, const CUten
 int launch_attention_bf16(const plk_dims* dims, const void* q, const void* q_lo, const void* K_cache,
                           const void* V_cache, void* a_out, void* a_lo, const int32_t* seg_ptr, int num_sms,
                           float* part_scratch, size_t part_bytes, int* part_cnt, cudaStream_t st);
+// out[i] = 2^t[i] by the attention softmax's FMA-pipe exponential (test hook)
+int launch_exp2_selftest(const float* t, float* out, int n, cudaStream_t st);
 int launch_attention_f32(const plk_dims* dims, const float* q, const float* K_cache, const float* V_cache,
                          float* a_out, const int32_t* seg_ptr, int Mcap, cudaStream_t st);
 

@@ -669,3 +669,24 @@ def test_wait_timeout_reports_status(plk):
         plk.set_wait_limit(4_000_000_000)
     x = torch.ones(4, device="cuda")
     assert float((x + 1).sum()) == 8.0  # the context is still usable
+
+
+# ---------------------------------------------------------------------------
+# the softmax's FMA-pipe exponential against exp2 (float64) and against CUDA's exp2f bound
+# ---------------------------------------------------------------------------
+def test_exp2_fma_error_bound(plk):
+    """Every t the softmax can produce (-inf .. 8: the weights are kept below 2^8) on a dense
+    grid plus the interval ends and the rounding ties of the range reduction; relative error
+    <= 3e-6 (the polynomial's minimax error is 2.7e-6 in fp32), 0 below 2^-126."""
+    t = np.concatenate([np.linspace(-126.0, 8.0, 2_000_001), np.arange(-126, 9) + 0.5, np.arange(-125, 9) - 0.5,
+                        np.arange(-126, 9).astype(np.float64), [-126.0, -0.0, 0.0, 1e-30, -1e-30]]).astype(np.float32)
+    below = np.array([-126.5, -127.0, -200.0, -1e30, -np.inf], np.float32)
+    td = torch.from_numpy(np.concatenate([t, below])).cuda()
+    out = torch.empty_like(td)
+    plk.selftest_exp2(td, out)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy().astype(np.float64)
+    ref = np.exp2(t.astype(np.float64))
+    rel = np.abs(got[: t.size] - ref) / ref
+    assert rel.max() <= 3e-6, rel.max()
+    assert np.all(got[t.size:] == 0.0)
