@@ -127,6 +127,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128_mn(uint32_t saddr, uint32_t mn_b
   d |= (uint64_t)2 << 61;
   return d;
 }
+// Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory to another CTA's of
+// the cluster, completing the bytes on an mbarrier of that CTA (shared::cluster addresses).
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t mbar) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "r"(src), "r"(bytes), "r"(mbar)
+               : "memory");
+}
 __device__ __forceinline__ void st_dsmem_v4(uint32_t addr, float4 v) {
   asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
                "f"(v.w)
@@ -247,16 +254,17 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
   uint64_t* p_free = bars + 20;   // [2] the P V that read P buffer x has completed
   uint64_t* o_free = bars + 22;   // O read out by the 8 softmax warps
   uint64_t* drain = bars + 23;
-  uint64_t* xo_full = bars + 24;  // even CTA: the odd CTA's partial is in my P region (8 warps)
-  uint64_t* xo_free = bars + 25;  // odd CTA: the even CTA's P region is free for my partial (8 warps)
+  uint64_t* xo_full = bars + 24;  // even CTA: the odd CTA's partial is in my P region (bulk copy bytes)
+  uint64_t* xo_free = bars + 25;  // odd CTA: the even CTA's P region is free and armed for my partial
   uint64_t* xmb = bars + 26;      // [4 quarters][2] row-max exchange of the two warps of a quarter
   uint64_t* xlb = bars + 34;      // [4 quarters] row-sum exchange
-  uint64_t* xo_read = bars + 38;  // even CTA: all 8 softmax warps have read the odd CTA's partial
+  uint64_t* xo_done = bars + 38;  // odd CTA: my bulk copies to the even CTA have landed (source free)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 39);
   volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 40);
   uint64_t* part_written = bars + 41;  // parts > 1: the 8 softmax warps stored this CTA's partial
   uint64_t* part_decided = bars + 42;  // parts > 1: warp 2 took the unit's counter (s_last is set)
   volatile int* s_last = reinterpret_cast<volatile int*>(bars + 43);
+  uint64_t* sm_bar = bars + 44;        // the 8 softmax warps meet (one arrival per warp)
 
   pdl_wait();
   pdl_trigger();
@@ -286,11 +294,12 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
     }
     mbar_init(o_free, kAttSoftWarps);
     mbar_init(drain, 1);
-    mbar_init(xo_full, kAttSoftWarps);
-    mbar_init(xo_free, kAttSoftWarps);
+    mbar_init(xo_full, 1);
+    mbar_init(xo_free, 1);
     for (int i = 0; i < 8; ++i) mbar_init(&xmb[i], 2);
     for (int i = 0; i < 4; ++i) mbar_init(&xlb[i], 2);
-    mbar_init(xo_read, kAttSoftWarps);
+    mbar_init(xo_done, 1);
+    mbar_init(sm_bar, kAttSoftWarps);
     mbar_init(part_written, kAttSoftWarps);
     mbar_init(part_decided, 1);
     *s_abort = 0;
@@ -457,6 +466,15 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
     long long g = 0;
     int t = 0;
     bool ok = true;
+    // the 8 softmax warps meet: lane 0 of each arrives, every lane waits (bounded)
+    uint32_t sm_phase = 0;
+    auto soft_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm_bar);
+      const bool r = mbar_wait(sm_bar, sm_phase);
+      sm_phase ^= 1u;
+      return r;
+    };
     // waits until the P V of global chunk k (and every MMA before it) has completed; k's
     // buffer cannot have moved on, its next P V needs P of chunk k + 2 from these warps
     auto wait_pv = [&](long long k) -> bool {
@@ -533,8 +551,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
         }
         l *= factor;
         ok = wait_pv(gj - 2);  // the P V that read P buffer sb has completed
-        // even CTA with a split: the odd CTA's last partial, which sat in the P region, is consumed
-        if (plan.split == 2 && rank == 0 && j == 0 && t > 0) ok = ok && mbar_wait(xo_read, (uint32_t)((t - 1) & 1));
+        // odd CTA with a split: the last unit's partial, staged in the P region, has been copied out
+        if (plan.split == 2 && rank == 1 && j == 0 && t > 0) ok = ok && mbar_wait_cluster(xo_done, (uint32_t)((t - 1) & 1));
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
@@ -590,37 +608,53 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(o_free);
-      const int grow = it.r0 + row;
       if (plan.split == 2 && rank == 1) {
-        // hand (O, max, sum) of my key half to the even CTA, into its P region
-        ok = mbar_wait_cluster(xo_free, (uint32_t)(t & 1));
+        // hand (O, max, sum) of my key half to the even CTA: stage it in my own P region (free:
+        // every P V of this unit has completed), row r's 32 16-byte slots at r * 32 + (c ^ (r & 7))
+        // so that a warp's 32 rows cover every bank, then one thread moves the 64 KB (and the
+        // 1 KB of (max, sum)) into the even CTA's P region with bulk copies that complete on its
+        // xo_full barrier
+        float4* xs = reinterpret_cast<float4*>(sP);
+#pragma unroll
+        for (int v = 0; v < 16; ++v)
+          xs[row * 32 + ((hf * 16 + v) ^ (row & 7))] = make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]);
+        if (hf == 0) reinterpret_cast<float2*>(ml)[row] = make_float2(m_used, l_row);
+        fence_proxy_async_smem();  // the bulk copy reads these through the async proxy
+        ok = soft_sync();
         if (!__all_sync(0xffffffffu, ok)) {
           ok = false;
           break;
         }
-        // row r's 32 16-byte slots, slot c at r * 32 + (c ^ (r & 7)): the 32 rows of a warp's
-        // store cover every bank (a plain row-major tile would put all 32 on the same banks)
-        const uint32_t xo = dsmem_addr(smem_u32(sP), 0);
-#pragma unroll
-        for (int v = 0; v < 16; ++v) {
-          const int slot = row * 32 + ((hf * 16 + v) ^ (row & 7));
-          st_dsmem_v4(xo + (uint32_t)slot * 16, make_float4(o[4 * v], o[4 * v + 1], o[4 * v + 2], o[4 * v + 3]));
+        if (warp == 2 && lane == 0) {
+          if (mbar_wait_cluster(xo_free, (uint32_t)(t & 1))) {  // its P region is free, the bytes expected
+            const uint32_t full_r = dsmem_addr(smem_u32(xo_full), 0);
+            bulk_copy_to_peer(dsmem_addr(smem_u32(sP), 0), smem_u32(sP), kAttBQ * kAttHD * 4, full_r);
+            bulk_copy_to_peer(dsmem_addr(smem_u32(ml), 0), smem_u32(ml), kAttBQ * 8, full_r);
+          } else {
+            *s_abort = 1;
+          }
         }
-        if (hf == 0) st_dsmem_v2(dsmem_addr(smem_u32(ml), 0) + row * 8, make_float2(m_used, l_row));
-        asm volatile("fence.acq_rel.cluster;" ::: "memory");
-        __syncwarp();
-        if (lane == 0) mbar_arrive_remote(dsmem_addr(smem_u32(xo_full), 0));
       } else {
         float m_row = m_used, l_tot = l_row;
         if (plan.split == 2) {
-          // my P region is free (every P V of this unit is done): the odd CTA may write its partial
-          __syncwarp();
-          if (lane == 0) mbar_arrive_remote(dsmem_addr(smem_u32(xo_free), 1));
-          ok = mbar_wait_cluster(xo_full, (uint32_t)(t & 1));
+          // my P region is free once every softmax warp is here (every P V of this unit has
+          // completed): one thread arms xo_full for the odd CTA's 64 KB + 1 KB and lets it send
+          ok = soft_sync();
           if (!__all_sync(0xffffffffu, ok)) {
             ok = false;
             break;
           }
+          if (warp == 2 && lane == 0) {
+            mbar_expect_tx(xo_full, kAttBQ * kAttHD * 4 + kAttBQ * 8);
+            mbar_arrive_remote(dsmem_addr(smem_u32(xo_free), 1));
+          }
+          ok = mbar_wait(xo_full, (uint32_t)(t & 1));
+          if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
+          }
+          // the copies have landed, so they have read their source: the odd CTA may reuse its P region
+          if (warp == 2 && lane == 0) mbar_arrive_remote(dsmem_addr(smem_u32(xo_done), 1));
           const float2 pm = reinterpret_cast<const float2*>(ml)[row];  // odd CTA's (max, sum)
           const float m = fmaxf(m_used, pm.x);
           const float w_own = exp2f(m_used - m);
@@ -636,9 +670,6 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
             o[4 * v + 2] = fmaf(w_own, o[4 * v + 2], w_odd * x.z);
             o[4 * v + 3] = fmaf(w_own, o[4 * v + 3], w_odd * x.w);
           }
-          // the next unit's P may overwrite the partial once every softmax warp has read it
-          __syncwarp();
-          if (lane == 0) mbar_arrive(xo_read);
         }
         float inv = 1.0f / l_tot;
         bool write_out = true;
@@ -695,17 +726,46 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
             if (warp == 2 && lane == 0) part_cnt[u] = 0;  // every part has counted: reset for the next launch
           }
         }
-        if (write_out && row < it.nrows) {
-          const size_t off = (size_t)grow * d + it.h * kAttHD + hf * 64;
-          uint4* dst = reinterpret_cast<uint4*>(Aout + off);
-          uint4* dst_lo = reinterpret_cast<uint4*>(Aout_lo + off);
+        if (write_out) {
+          // the normalised tile as hi/lo bf16 pairs, staged in the P region (rows of 16 16-byte
+          // chunks, chunk c of row r at r * 16 + (c ^ (r & 7)): conflict-free both ways) and
+          // stored two rows per warp instruction, each row 256 contiguous bytes of hi and of lo
+          ok = soft_sync();  // every warp is done with the P region (and the odd CTA's partial in it)
+          if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
+          }
+          uint4* sh = reinterpret_cast<uint4*>(sP);
+          uint4* sl = reinterpret_cast<uint4*>(sP + kAttBQ * kAttHD * 2);
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
             uint32_t hi[4], lo[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) split_pair(o[8 * v + 2 * e] * inv, o[8 * v + 2 * e + 1] * inv, hi[e], lo[e]);
-            dst[v] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            dst_lo[v] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            const int slot = row * 16 + ((hf * 8 + v) ^ (row & 7));
+            sh[slot] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            sl[slot] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          }
+          ok = soft_sync();
+          if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
+          }
+          const int sw = warp - 2, ch = lane & 15;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = sw * 16 + 2 * i + (lane >> 4);
+            if (r < it.nrows) {
+              const size_t off = (size_t)(it.r0 + r) * d + it.h * kAttHD + ch * 8;
+              const int slot = r * 16 + (ch ^ (r & 7));
+              *reinterpret_cast<uint4*>(Aout + off) = sh[slot];
+              *reinterpret_cast<uint4*>(Aout_lo + off) = sl[slot];
+            }
+          }
+          ok = soft_sync();  // the P region may take the next unit's weights
+          if (!__all_sync(0xffffffffu, ok)) {
+            ok = false;
+            break;
           }
         }
       }
