@@ -293,6 +293,32 @@ int plk_layer_step_partial_static(const plk_dims* dims, const plk_weights* w, co
  * dims on the current device (0 for invalid dims). */
 size_t plk_workspace_bytes(const plk_dims* dims);
 
+/*
+ * The whole denoising step of one layer from host memory: the step S1..S10 as the
+ * calls above chain it, with the layer input coming from and the output going to
+ * host buffers ([SL] Sec. 2; [SPA] part 1 for the proxy refresh).  In stream order:
+ *   X_host [B, N, d] (host memory, layer dtype) is copied into the workspace;
+ *   plk_score_drift(X, Ut, r, proxy_cache, metric) -> score and fresh proxies;
+ *   plk_select_active(score, lock, mode, tau, k) -> lock (in place), idx, seg_ptr;
+ *   plk_layer_step_partial -> K_cache, V_cache, Y (device, in/out);
+ *   plk_proxy_commit -> proxy_cache (device [B, N, r] fp32, in/out);
+ *   Y [B, N, d] is copied to Y_host (host memory).
+ * One cudaMemcpyAsync each way on `stream`; the call returns after enqueueing
+ * (synchronise the stream before reading Y_host).  Host buffers should be pinned
+ * (cudaHostAlloc / cudaHostRegister) for the copies to be asynchronous.
+ * lock [B, N] uint8 is device memory (in/out).  The argument rules of the calls it
+ * chains apply (r, metric, mode, k).  workspace: device buffer of at least
+ * plk_step_workspace_bytes(dims, r) bytes, 256-byte aligned, not shared with a
+ * concurrent call.  Errors: those of the chained calls, checked before anything
+ * is enqueued, and PLK_ERR_WORKSPACE.
+ */
+int plk_denoise_step_host(const plk_dims* dims, const plk_weights* w, const void* Ut, int r, int metric,
+                          int mode, float tau, int k, float* proxy_cache, uint8_t* lock,
+                          void* K_cache, void* V_cache, void* Y, const void* X_host, void* Y_host,
+                          void* workspace, size_t ws_bytes, void* stream);
+/* Workspace of plk_denoise_step_host (0 for invalid dims or r). */
+size_t plk_step_workspace_bytes(const plk_dims* dims, int r);
+
 /* Synchronises `stream`, returns the device status word of the current device
  * (PLK_OK or PLK_ERR_TIMEOUT) and clears it. */
 int plk_get_status(void* stream);

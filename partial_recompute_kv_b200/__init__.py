@@ -26,6 +26,7 @@ SEL_THRESH_GT, SEL_THRESH_LT, SEL_TOPK_LARGEST, SEL_TOPK_SMALLEST = 0, 1, 2, 3
 EXPORTED = (
     "plk_score_drift", "plk_select_active", "plk_layer_step_partial", "plk_full_layer_step",
     "plk_proxy_commit", "plk_layer_step_partial_static", "plk_kl_lock", "plk_slowfast_step", "plk_workspace_bytes",
+    "plk_denoise_step_host", "plk_step_workspace_bytes",
     "plk_get_status",
     "plk_set_wait_limit",
     "plk_selftest_wait_timeout", "plk_selftest_exp2", "plk_trace_events", "plk_error_string", "plk_version",
@@ -75,6 +76,8 @@ def _load():
         "plk_kl_lock": (I, [V, I, P, P, P, P, F, F, P, P, P]),
         "plk_slowfast_step": (I, [V, ctypes.POINTER(PlkSfParams), P, P, P, P, P, P]),
         "plk_workspace_bytes": (S, [V]),
+        "plk_denoise_step_host": (I, [V, W, P, I, I, I, F, I, P, P, P, P, P, P, P, P, S, P]),
+        "plk_step_workspace_bytes": (S, [V, I]),
         "plk_get_status": (I, [P]),
         "plk_set_wait_limit": (I, [L]),
         "plk_selftest_wait_timeout": (I, [P]),
@@ -182,6 +185,35 @@ def layer_step_partial_static(dm, w, X, idx, seg_ptr, K_cache, V_cache, Y, strea
     _check(lib.plk_layer_step_partial_static(ctypes.byref(dm), ctypes.byref(pw), _ptr(X), _ptr(idx),
                                              _ptr(seg_ptr), _ptr(K_cache), _ptr(V_cache), _ptr(Y),
                                              _stream(stream)), "layer_step_partial_static")
+
+
+def _hptr(t):
+    if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_contiguous():
+        raise ValueError("host buffers must be contiguous CPU tensors (pinned for asynchronous copies)")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def step_workspace_bytes(dm, r) -> int:
+    return int(lib.plk_step_workspace_bytes(ctypes.byref(dm), int(r)))
+
+
+def alloc_step_workspace(dm, r, device="cuda"):
+    n = step_workspace_bytes(dm, r)
+    if n == 0:
+        raise PlkError(ERR_SHAPE, "step_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def denoise_step_host(dm, w, Ut, r, metric, mode, tau, k, proxy_cache, lock, K_cache, V_cache, Y, X_host, Y_host,
+                      workspace, stream=None):
+    """The whole step from host memory (see plk_denoise_step_host): X_host -> device, score, select,
+    layer step, proxy refresh, Y -> Y_host.  X_host / Y_host are CPU tensors (pinned)."""
+    pw = w if isinstance(w, PlkWeights) else weights(w)
+    _check(lib.plk_denoise_step_host(ctypes.byref(dm), ctypes.byref(pw), _ptr(Ut), int(r), int(metric), int(mode),
+                                     float(tau), int(k), _ptr(proxy_cache), _ptr(lock), _ptr(K_cache),
+                                     _ptr(V_cache), _ptr(Y), _hptr(X_host), _hptr(Y_host), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(stream)),
+           "denoise_step_host")
 
 
 def full_layer_step(dm, w, X, K_cache, V_cache, Y, workspace, stream=None):

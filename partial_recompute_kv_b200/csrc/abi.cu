@@ -140,6 +140,84 @@ int plk_proxy_commit(const plk_dims* dims, int r, const int32_t* idx, const int3
   return launch_proxy_commit(dims, r, idx, seg_ptr, proxy_new, proxy_cache, (cudaStream_t)stream);
 }
 
+}  // extern "C"
+
+namespace plk {
+// Layout of the workspace of plk_denoise_step_host behind the layer step's own:
+// score [B*N] fp32, fresh proxies [B*N*r] fp32, idx [B*N], seg_ptr [B+1], X [B*N*d].
+struct StepWs {
+  size_t layer = 0, score = 0, pnew = 0, idx = 0, seg = 0, x = 0, total = 0;
+};
+static size_t up256(size_t v) { return (v + 255) / 256 * 256; }
+static StepWs step_ws_layout(const plk_dims* d, int r) {
+  StepWs s;
+  const size_t BN = (size_t)d->B * d->N, es = d->dtype == PLK_BF16 ? 2 : 4;
+  s.layer = 0;
+  size_t off = up256(plk_workspace_bytes(d));
+  s.score = off;
+  off = up256(off + 4 * BN);
+  s.pnew = off;
+  off = up256(off + 4 * BN * (size_t)r);
+  s.idx = off;
+  off = up256(off + 4 * BN);
+  s.seg = off;
+  off = up256(off + 4 * ((size_t)d->B + 1));
+  s.x = off;
+  off = up256(off + es * BN * (size_t)d->d);
+  s.total = off;
+  return s;
+}
+static int check_score_args(const plk_dims* dims, int r, int metric) {
+  if (metric != PLK_METRIC_COS && metric != PLK_METRIC_L2) return PLK_ERR_ARG;
+  if (dims->dtype == PLK_BF16) {
+    if (r < 16 || r > 256 || r % 16 != 0 || dims->d % 64 != 0) return PLK_ERR_ARG;
+  } else {
+    if (r < 1 || r > 256) return PLK_ERR_ARG;
+  }
+  return PLK_OK;
+}
+}  // namespace plk
+
+extern "C" {
+
+size_t plk_step_workspace_bytes(const plk_dims* dims, int r) {
+  if (check_dims(dims) != PLK_OK || check_score_args(dims, r, PLK_METRIC_L2) != PLK_OK) return 0;
+  if (plk_workspace_bytes(dims) == 0) return 0;
+  return step_ws_layout(dims, r).total;
+}
+
+int plk_denoise_step_host(const plk_dims* dims, const plk_weights* w, const void* Ut, int r, int metric,
+                          int mode, float tau, int k, float* proxy_cache, uint8_t* lock, void* K_cache,
+                          void* V_cache, void* Y, const void* X_host, void* Y_host, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  int e = check_dims(dims);
+  if (e != PLK_OK) return e;
+  if ((e = check_score_args(dims, r, metric)) != PLK_OK) return e;
+  if (!Ut || !proxy_cache || !lock || !X_host || !Y_host) return PLK_ERR_ARG;
+  if (mode < PLK_SEL_THRESH_GT || mode > PLK_SEL_TOPK_SMALLEST) return PLK_ERR_ARG;
+  if ((mode == PLK_SEL_TOPK_LARGEST || mode == PLK_SEL_TOPK_SMALLEST) && k < 0) return PLK_ERR_ARG;
+  if (!w || !w->g1 || !w->w_qkv || !w->w_o || !w->g2 || !w->w_gu || !w->w_down) return PLK_ERR_ARG;
+  if (!K_cache || !V_cache || !Y) return PLK_ERR_ARG;
+  if (plk_workspace_bytes(dims) == 0) return PLK_ERR_CUDA;
+  const StepWs L = step_ws_layout(dims, r);
+  if (!workspace || ws_bytes < L.total) return PLK_ERR_WORKSPACE;
+  uint8_t* ws = (uint8_t*)workspace;
+  float* score = (float*)(ws + L.score);
+  float* pnew = (float*)(ws + L.pnew);
+  int32_t* idx = (int32_t*)(ws + L.idx);
+  int32_t* seg = (int32_t*)(ws + L.seg);
+  void* X = ws + L.x;
+  const size_t BN = (size_t)dims->B * dims->N, es = dims->dtype == PLK_BF16 ? 2 : 4;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(X, X_host, es * BN * dims->d, cudaMemcpyHostToDevice, st) != cudaSuccess) return PLK_ERR_CUDA;
+  if ((e = launch_score(dims, X, Ut, r, proxy_cache, metric, pnew, score, st)) != PLK_OK) return e;
+  if ((e = launch_select(dims, score, lock, lock, mode, tau, k, idx, seg, st)) != PLK_OK) return e;
+  if ((e = run_layer(dims, w, X, idx, seg, false, K_cache, V_cache, Y, ws, L.score, st)) != PLK_OK) return e;
+  if ((e = launch_proxy_commit(dims, r, idx, seg, pnew, proxy_cache, st)) != PLK_OK) return e;
+  if (cudaMemcpyAsync(Y_host, Y, es * BN * dims->d, cudaMemcpyDeviceToHost, st) != cudaSuccess) return PLK_ERR_CUDA;
+  return PLK_OK;
+}
+
 int plk_get_status(void* stream) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return PLK_ERR_CUDA;
   int v = PLK_OK;

@@ -690,3 +690,47 @@ def test_exp2_fma_error_bound(plk):
     rel = np.abs(got[: t.size] - ref) / ref
     assert rel.max() <= 3e-6, rel.max()
     assert np.all(got[t.size:] == 0.0)
+
+
+# ---------------------------------------------------------------------------
+# the whole step from host memory (plk_denoise_step_host) against the oracle
+# ---------------------------------------------------------------------------
+def test_denoise_step_host_matches_oracle(plk):
+    D = synth.Dims(B=2, N=320, d=512, H=4, hd=128, F=1536, dtype="bf16")
+    r, k = 128, 96
+    W = synth.layer_weights(D, 0.02, seed=14)
+    X = synth.hidden_states(D, seed=14)
+    Ut = synth.proxy_basis(D.d, r, seed=14)
+    base = oracle.full_layer_step(D, W, X, "bf16")
+    pc = oracle.to_f32(oracle.proxy_project(X.reshape(-1, D.d).astype(np.float64), Ut.astype(np.float64)))
+    pc = pc.astype(np.float32).reshape(D.B, D.N, r)
+    moved = np.zeros((D.B, D.N), bool)
+    for b in range(D.B):
+        moved[b, synth.uniform_positions(0, D.N, k, seed=14, tag=b)] = True
+    X2 = synth.perturb_rows(X, synth.step_noise((D.B, D.N, D.d), 0.25, seed=14), moved, "bf16")
+    # oracle: score -> top-k (the k moved rows of each sequence) -> layer step -> proxy refresh
+    s, p = oracle.score_drift(X2.astype(np.float64), Ut.astype(np.float64), pc, "l2")
+    ref_lock = oracle.lock_topk(s.astype(np.float32).astype(np.float64), np.zeros((D.B, D.N), np.uint8), k, True)
+    assert np.array_equal(ref_lock == 0, moved)
+    idx, seg = oracle.compact(ref_lock)
+    ref = oracle.layer_step_partial(D, W, X2, idx, seg, base, "bf16")
+    ref_pc = oracle.proxy_commit(pc, p, idx)
+
+    dm = pdims(plk, D)
+    g = {"K": Guarded(base.K.shape, BF, init=dev(base.K, BF)), "V": Guarded(base.V.shape, BF, init=dev(base.V, BF)),
+         "Y": Guarded(base.Y.shape, BF, init=dev(base.Y, BF)), "proxy": Guarded(pc.shape, torch.float32, init=pc),
+         "lock": Guarded((D.B, D.N), torch.uint8, fill=0)}
+    n = plk.step_workspace_bytes(dm, r)
+    assert n > plk.workspace_bytes(dm)
+    g["workspace"] = Guarded((n,), torch.uint8)
+    X_host = torch.from_numpy(np.ascontiguousarray(X2)).to(BF).pin_memory()
+    Y_host = torch.full(base.Y.shape, -3.0, dtype=BF).pin_memory()
+    plk.denoise_step_host(dm, weights_dev(W, D), dev(Ut, BF), r, plk.METRIC_L2, plk.SEL_TOPK_LARGEST, 0.0, k,
+                          g["proxy"].t, g["lock"].t, g["K"].t, g["V"].t, g["Y"].t, X_host, Y_host, g["workspace"].t)
+    assert plk.get_status() == plk.OK
+    check_guards(g, "denoise_step_host")
+    assert np.array_equal(host(g["lock"].t), ref_lock)
+    Yd = host(g["Y"].t)
+    assert np.array_equal(Y_host.to(torch.float64).numpy(), Yd), "Y_host is the device Y"
+    _check_layer_rows(host(g["K"].t), host(g["V"].t), Yd, ref, base, ref_lock, "host step")
+    assert_f32_close(host(g["proxy"].t), ref_pc, "proxy cache", tol=1e-5)
