@@ -11,10 +11,11 @@
 // The kernel streams X once from HBM; Ut stays in L2.  When there are too few
 // 128-row tiles to fill the GPU, the K dimension is split over a thread-block
 // cluster of S CTAs: once every CTA's loads and MMAs are done (a cluster
-// barrier), each CTA pushes the row slices of its partial projection into the
-// idle stage buffers of the CTA that finishes those rows (distributed shared
-// memory stores), and after a second barrier every CTA sums its S slices
-// locally (no global scratch, no remote loads).
+// barrier), each CTA stages its partial projection in its own shared memory and
+// moves each 128/S-row slice with one bulk copy into the idle stage buffers of
+// the CTA that finishes those rows (the copies complete on that CTA's
+// mbarrier); every CTA then sums its S slices locally (no global scratch, no
+// remote loads, no thread-issued remote stores).
 // fp32: a SIMT kernel, one warp per row.
 #include "plk_common.cuh"
 #include "plk_internal.h"
@@ -61,6 +62,7 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
   uint64_t* done = bars + 2 * kScStagesMax;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bars + 2 * kScStagesMax + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(bars + 2 * kScStagesMax + 2);
+  uint64_t* slices = bars + 2 * kScStagesMax + 3;  // split-K: the S row slices of my rows have landed
 
   pdl_wait();
   pdl_trigger();
@@ -76,6 +78,7 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
       mbar_init(&empty[i], 1);
     }
     mbar_init(done, 1);
+    mbar_init(slices, 1);
     *s_abort = 0;
     fence_mbar_init();
   }
@@ -146,39 +149,56 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
   const bool ok = mbar_wait(done, 0);
   tc_fence_after();
   if (S > 1) {
-    // split-K over the cluster: every CTA pushes the row slices of its partial projection to
-    // the CTA that finishes those rows (distributed shared memory stores, nothing waits on a
-    // round trip); the receiver's idle stage buffers hold slots [sender][rows_per][r]
+    // split-K over the cluster.  Layout of a row block of r fp32 values: 16-byte chunk c of row
+    // k sits at chunk c ^ (k & 7) of the row (c ^ (k & 3) when r / 4 is not a multiple of 8), so
+    // a warp's 32 rows spread over the banks.  Each CTA
+    // stages its whole partial [128 rows][r] in its own stage buffers, then one thread sends
+    // slice q (rows q * rows_per ..) with one bulk copy to slot [ks] of CTA q; CTA q's slice
+    // barrier counts the S copies' bytes.
     const int rows_per = 128 / S, tpr = 128 / rows_per;
-    float* slots = reinterpret_cast<float*>(smem);
+    const int nch = r / 4;                                   // 16-byte chunks per row
+    const int swz = (nch % 8 == 0) ? 7 : 3;                  // XOR key mask: stays inside the row
+    float4* stage = reinterpret_cast<float4*>(smem);         // [128][nch] my partial (sender side)
+    float* slots = reinterpret_cast<float*>(smem + (size_t)128 * r * 4);  // [S][rows_per][r] (receiver)
     const int rl = warp * 32 + lane;
-    const uint32_t dst = dsmem_addr(smem_u32(slots + ((size_t)ks * rows_per + rl % rows_per) * r),
-                                    (uint32_t)(rl / rows_per));
     const bool good = __all_sync(0xffffffffu, ok && !*s_abort);
-    // the receivers' stage buffers must be idle: every CTA's loads and MMAs are done
-    cluster_sync_all();
-    for (int c0 = 0; c0 < r; c0 += 16) {
-      uint32_t v[16];
-      if (good) {
+    if (good) {
+      for (int c0 = 0; c0 < r; c0 += 16) {
+        uint32_t v[16];
         tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)c0, v);
         tmem_ld_wait();
-      }
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        st_dsmem_f32x4(dst + 4u * (c0 + 4 * u),
-                       good ? make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
-                                          __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3]))
-                            : make_float4(0.f, 0.f, 0.f, 0.f));
+        for (int u = 0; u < 4; ++u)
+          stage[rl * nch + ((c0 / 4 + u) ^ (rl & swz))] =
+              make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]), __uint_as_float(v[4 * u + 2]),
+                          __uint_as_float(v[4 * u + 3]));
+      }
+    } else {
+      for (int c = 0; c < nch; ++c) stage[rl * nch + c] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    tc_fence_before();
-    cluster_sync_all();  // every slice has landed; nobody touches another CTA's memory after this
+    fence_proxy_async_smem();  // the bulk copies read the staged partial through the async proxy
+    if (threadIdx.x == 0) mbar_expect_tx(slices, (uint32_t)(S * rows_per * r * 4));
+    // the receivers' slot buffers (behind their staged partials) are idle and armed: every
+    // CTA's loads and MMAs are done and every CTA has staged its partial
+    cluster_sync_all();
+    if (threadIdx.x == 0) {
+      for (int q = 0; q < S; ++q)
+        asm volatile(
+            "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                dsmem_addr(smem_u32(slots + (size_t)ks * rows_per * r), (uint32_t)q)),
+            "r"(smem_u32(stage + (size_t)q * rows_per * nch)), "r"((uint32_t)(rows_per * r * 4)),
+            "r"(dsmem_addr(smem_u32(slices), (uint32_t)q))
+            : "memory");
+    }
+    const bool landed = mbar_wait(slices, 0);
     const int lrow = (int)threadIdx.x / tpr, sub = (int)threadIdx.x % tpr;
     const int row = row0 + ks * rows_per + lrow;
+    const int krow = ks * rows_per + lrow;  // the row's index in its sender's block (swizzle key)
     float dot = 0.f, pp = 0.f, cc = 0.f, dd = 0.f;
-    for (int c = sub * 4; c < r; c += 4 * tpr) {
+    for (int c = sub * 4; c < r && landed; c += 4 * tpr) {
       float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int sr = 0; sr < S; ++sr) {
-        const float4 x = *reinterpret_cast<const float4*>(slots + ((size_t)sr * rows_per + lrow) * r + c);
+        const float4 x = reinterpret_cast<const float4*>(slots + ((size_t)sr * rows_per + lrow) * r)[(c / 4) ^ (krow & swz)];
         p.x += x.x;
         p.y += x.y;
         p.z += x.z;
@@ -204,8 +224,10 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
       cc += __shfl_xor_sync(0xffffffffu, cc, o);
       dd += __shfl_xor_sync(0xffffffffu, dd, o);
     }
-    if (sub == 0 && row < rows)
+    if (sub == 0 && row < rows && landed)
       score[row] = metric == PLK_METRIC_COS ? dot / fmaxf(sqrtf(pp) * sqrtf(cc), 1e-30f) : sqrtf(dd);
+    tc_fence_before();
+    cluster_sync_all();  // every copy has landed, so every source was read: CTAs may leave
     if (warp == 2) {
       tc_fence_after();
       tmem_dealloc(tmem, (uint32_t)tmem_cols);
@@ -324,10 +346,15 @@ int launch_score(const plk_dims* dims, const void* X, const void* Ut, int r, con
       return PLK_ERR_CUDA;
     attr_smem[dev] = smem;
   }
-  // K slices: grow the cluster while it still fits the GPU and leaves >= 2 k-blocks per slice
+  // K slices: grow the cluster while it still fits the GPU and leaves >= 2 k-blocks per slice.
+  // The split needs the staged partial and the received slices ([128][r] fp32 each) inside the
+  // stage ring: at r = 256 the ring is too small, and the kernel runs unsplit.
   const int tiles = ceil_div(rows, 128), nkb = d / 64;
+  const int ring = sc_stages(r) * (kScA + ((r * 128 + 1023) & ~1023));
   int S = 1;
-  while (S < 8 && tiles * S * 2 <= device_sm_count() && nkb % (S * 2) == 0 && nkb / (S * 2) >= 2) S *= 2;
+  while (S < 8 && tiles * S * 2 <= device_sm_count() && nkb % (S * 2) == 0 && nkb / (S * 2) >= 2 &&
+         2 * 128 * r * 4 <= ring)
+    S *= 2;
   if (S == 1) {
     return launch_pdl(score_tc_kernel, dim3(tiles), dim3(128), smem, st, tmX, tmU, rows, d, r, tcols, proxy_cache,
                       proxy_out, score_out, metric);

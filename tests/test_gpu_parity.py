@@ -130,10 +130,14 @@ def _score_case(dtype):
     return synth.Dims(B=2, N=300, d=512, H=4, hd=128, F=512, dtype="bf16"), 128
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype,rank", [("f32", None), ("bf16", None), ("bf16", 16), ("bf16", 48), ("bf16", 256)])
 @pytest.mark.parametrize("metric", ["cos", "l2"])
-def test_score_drift(plk, dtype, metric):
+def test_score_drift(plk, dtype, rank, metric):
+    """Ranks 16 and 48 (row blocks whose 16-byte chunk count is not a multiple of 8) run the
+    K split over a cluster of 4 at d = 1024; rank 256 runs unsplit."""
     D, r = _score_case(dtype)
+    if rank is not None:
+        D, r = synth.Dims(B=2, N=300, d=1024, H=8, hd=128, F=512, dtype="bf16"), rank
     X = synth.hidden_states(D, seed=3)
     Ut = synth.proxy_basis(D.d, r, seed=3, dtype=dtype)
     p_exact = oracle.proxy_project(X.reshape(-1, D.d).astype(np.float64), Ut.astype(np.float64))
