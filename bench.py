@@ -574,7 +574,7 @@ def run_kernel_configs(args):
         us = _timed(torch, lambda: plk.select_active(dm, score, lk_in, lk, plk.SEL_TOPK_LARGEST, 0.0, k, idx, seg),
                     args.steps, args.warmup)
         by = 6 * D.B * D.N + 4 * D.B * k
-        out.append({"kernel": "topk_compact_kernel", "config": f"B={D.B} N={D.N} k={k} ({pct}% of N)", "us": us,
+        out.append({"kernel": "select_active (top-k decide + compaction)", "config": f"B={D.B} N={D.N} k={k} ({pct}% of N)", "us": us,
                     "GB/s": by / (us * 1e-6) / 1e9, "frac_of_hbm": by / (us * 1e-6) / 1e9 / hbm,
                     "scoring_layer_us": score_us + us,
                     "scoring_32_layers_us": 32 * (score_us + us)})

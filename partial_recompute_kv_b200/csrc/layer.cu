@@ -164,8 +164,7 @@ __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const Tin* __restrict
   pdl_wait();
   pdl_trigger();
   const int M = seg_ptr[B];
-  const int j = blockIdx.x;
-  if (j >= M) return;
+  for (int j = blockIdx.x; j < M; j += gridDim.x) {  // grid-stride over the live rows (uniform per block)
   if (zero_out) clear_row(zero_out + (size_t)j * zcols, zcols);
   const size_t row = idx ? (size_t)idx[j] : (size_t)j;
   const Tin* x = X + row * d;
@@ -183,6 +182,7 @@ __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const Tin* __restrict
     const Tout hi = from_f<Tout>(v);
     o[c] = hi;
     if (out_lo) out_lo[(size_t)j * d + c] = from_f<Tout>(v - to_f(hi));
+  }
   }
 }
 
@@ -271,8 +271,7 @@ __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict_
   pdl_wait();
   pdl_trigger();
   const int M = seg_ptr[B];
-  const int j = blockIdx.x;
-  if (j >= M) return;
+  for (int j = blockIdx.x; j < M; j += gridDim.x) {  // grid-stride over the live rows (uniform per block)
   if (zero_out) clear_row(zero_out + (size_t)j * zcols, zcols);
   const size_t row = idx ? (size_t)idx[j] : (size_t)j;
   const uint4* xv = reinterpret_cast<const uint4*>(X + row * d);
@@ -313,6 +312,7 @@ __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict_
       }
       store_vec<Tout, E>(o + vi * E, f);
     }
+  }
   }
 }
 
@@ -576,7 +576,8 @@ static int run_layer_f32(const plk_dims* dm, const plk_weights* w, const float* 
     dim3 grid(ceil_div(Nout, 64), ceil_div(Mcap, 64));
     gemm_f32_kernel<<<grid, 256, 0, st>>>(A, (const float*)Wt, c32, Nout, K, seg, B);
   };
-  PLK_TRY(launch_rmsnorm<float, float, float>(X, idx, seg, B, (const float*)w->g1, dm->eps, d, xn, nullptr, Mcap,
+  const int ngrid = std::min(Mcap, 2 * L.num_sms);  // row kernels: grid-stride over the M live rows
+  PLK_TRY(launch_rmsnorm<float, float, float>(X, idx, seg, B, (const float*)w->g1, dm->eps, d, xn, nullptr, ngrid,
                                               st));
   gemm(xn, w->w_qkv, d + 2 * dkv, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_QKV, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, dm->N,
@@ -586,7 +587,7 @@ static int run_layer_f32(const plk_dims* dm, const plk_weights* w, const float* 
   gemm(a, w->w_o, d, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_O, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, 0, 0, 0.f, 0);
   PLK_TRY(launch_rmsnorm<float, float, float>(h32, nullptr, seg, B, (const float*)w->g2, dm->eps, d, hn, nullptr,
-                                              Mcap, st));
+                                              ngrid, st));
   gemm(hn, w->w_gu, 2 * F, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_GU, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, 0, 0, 0.f, 0);
   gemm(act, w->w_down, d, F);
@@ -642,7 +643,7 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   trace_mark(0, st);
   // x (fp32) staged in h32 takes the O projection's adds; the QKV sums start at 0
   PLK_TRY(launch_rmsnorm<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(X, idx, seg, B, (const __nv_bfloat16*)w->g1,
-                                                                      dm->eps, d, xn, xn_lo, Mcap, st, h32,
+                                                                      dm->eps, d, xn, xn_lo, rgrid, st, h32,
                                                                       c32, d + 2 * dkv));
   trace_mark(1, st);
 
@@ -668,7 +669,7 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   trace_mark(5, st);
 
   PLK_TRY(launch_rmsnorm<float, __nv_bfloat16, __nv_bfloat16>(h32, nullptr, seg, B, (const __nv_bfloat16*)w->g2,
-                                                              dm->eps, d, hn, hn_lo, Mcap, st, nullptr, c32,
+                                                              dm->eps, d, hn, hn_lo, rgrid, st, nullptr, c32,
                                                               2 * F));
   trace_mark(6, st);
 

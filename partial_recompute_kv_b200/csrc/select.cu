@@ -6,11 +6,16 @@
 // page ("SPA-Cache: Singular Proxies for Adaptive Caching in Diffusion Language
 // Models", part 2) / Polestar-Cache's most-drifted refresh.
 //
-// Compaction: one CTA per sequence.  A CTA first counts the active rows of the
-// sequences before it (re-deriving their lock state, which is idempotent, so no
-// inter-CTA wait and no scratch memory is needed), then compacts its own
-// sequence chunk by chunk with warp ballots, popcounts and a block scan of the
-// 32 warp counts.  Indices come out ascending and deterministic.
+// One CTA per sequence decides every row's lock (threshold: compare; top-k:
+// radix select of the k-th key, then an ordered tie-break) and compacts its active rows chunk by chunk with warp
+// ballots, popcounts and a block scan of the 32 warp counts.  A single
+// sequence is done in that one launch.  With B > 1 sequences the decide launch
+// leaves each sequence's active count in seg_ptr[b + 1] (encoded as -(count+1))
+// and a second launch compacts: CTA b finds its output offset by walking
+// seg_ptr down from b, adding encoded counts until it meets an entry another
+// CTA has already turned into its final prefix sum (no inter-CTA waiting, no
+// scratch memory, O(B) reads per CTA).  Indices come out ascending and
+// deterministic.
 #include "plk_common.cuh"
 #include "plk_internal.h"
 
@@ -68,35 +73,79 @@ __device__ __forceinline__ int block_rank(int flag, int* sh, int* total) {
   return r;
 }
 
-// mode: PLK_SEL_THRESH_GT / PLK_SEL_THRESH_LT derive lock_out from lock_in and
-// the score; any other value takes lock_src as the final lock (after top-k).
-__global__ void __launch_bounds__(kSelThreads) compact_kernel(int mode, const float* __restrict__ score,
-                                                              const uint8_t* lock_src, uint8_t* lock_out,
-                                                              int N, float tau, int32_t* __restrict__ idx_out,
-                                                              int32_t* __restrict__ seg_ptr) {
+// The threshold rules, one CTA per sequence: lock_out = lock_in | (score > tau)
+// [or < tau].  direct (a single sequence): the active rows are compacted here and
+// seg_ptr is final; otherwise seg_ptr[b + 1] = -(active count + 1) for the
+// compaction launch.
+__global__ void __launch_bounds__(kSelThreads) thresh_decide_kernel(int mode, const float* __restrict__ score,
+                                                                    const uint8_t* lock_src, uint8_t* lock_out,
+                                                                    int N, float tau, int direct,
+                                                                    int32_t* __restrict__ idx_out,
+                                                                    int32_t* __restrict__ seg_ptr) {
   __shared__ int sh[33];
   pdl_wait();
   pdl_trigger();
   const int b = blockIdx.x;
-  const bool writes_lock = (mode == PLK_SEL_THRESH_GT || mode == PLK_SEL_THRESH_LT);
-  // active rows of the sequences before this one
-  int cnt = 0;
-  const long long before = (long long)b * N;
-  for (long long i = threadIdx.x; i < before; i += blockDim.x)
-    cnt += derive_lock(mode, score, lock_src, tau, i) ? 0 : 1;
-  const int offset = block_sum(cnt, sh);
+  const long long base = (long long)b * N;
   int running = 0;
   for (int c0 = 0; c0 < N; c0 += blockDim.x) {
     const int i = c0 + threadIdx.x;
     int act = 0;
     if (i < N) {
-      const uint8_t l = derive_lock(mode, score, lock_src, tau, before + i);
-      if (writes_lock) lock_out[before + i] = l;
+      const uint8_t l = derive_lock(mode, score, lock_src, tau, base + i);
+      lock_out[base + i] = l;
       act = l ? 0 : 1;
     }
     int total;
     const int r = block_rank(act, sh, &total);
-    if (act) idx_out[offset + running + r] = (int32_t)(before + i);
+    if (direct && act) idx_out[running + r] = (int32_t)(base + i);
+    running += total;
+  }
+  if (threadIdx.x == 0) {
+    if (direct) {
+      seg_ptr[0] = 0;
+      seg_ptr[1] = running;
+    } else {
+      seg_ptr[b + 1] = -(running + 1);
+    }
+  }
+}
+
+// Output offset of sequence b: the active rows of sequences 0 .. b-1.  seg_ptr[j]
+// (j >= 1) holds either -(count of sequence j-1) - 1, left by the decide launch,
+// or the final prefix count of sequences 0 .. j-1, written by CTA j-1 of this
+// launch; both are single 32-bit writes, so any value read is one of the two.
+__device__ __forceinline__ int sel_offset(const int32_t* seg_ptr, int b) {
+  int total = 0;
+  for (int j = b; j >= 1; --j) {
+    const int v = *reinterpret_cast<const volatile int32_t*>(seg_ptr + j);
+    if (v >= 0) return total + v;
+    total += -v - 1;
+  }
+  return total;
+}
+
+// Compaction of sequence b's rows with lock[b, i] == 0 into idx_out at its
+// offset; seg_ptr[b + 1] becomes the final prefix count.
+__global__ void __launch_bounds__(kSelThreads) compact_lock_kernel(const uint8_t* __restrict__ lock, int N,
+                                                                   int32_t* __restrict__ idx_out,
+                                                                   int32_t* __restrict__ seg_ptr) {
+  __shared__ int sh[33];
+  __shared__ int s_off;
+  pdl_wait();
+  pdl_trigger();
+  const int b = blockIdx.x;
+  const long long base = (long long)b * N;
+  if (threadIdx.x == 0) s_off = sel_offset(seg_ptr, b);
+  __syncthreads();
+  const int offset = s_off;
+  int running = 0;
+  for (int c0 = 0; c0 < N; c0 += blockDim.x) {
+    const int i = c0 + threadIdx.x;
+    const int act = (i < N && lock[base + i] == 0) ? 1 : 0;
+    int total;
+    const int r = block_rank(act, sh, &total);
+    if (act) idx_out[offset + running + r] = (int32_t)(base + i);
     running += total;
   }
   if (threadIdx.x == 0) {
@@ -175,18 +224,17 @@ __device__ void block_radix_kth(const float* __restrict__ score, int N, int keep
 }
 
 // One CTA per sequence: among rows with lock_in == 0 keep the k most preferred
-// (ties to the lower index), lock every other row, and compact the kept rows.
-// Radix select on 8-bit digits finds the k-th key (warp-parallel bin search);
-// an ordered block scan breaks ties and produces the ascending indices.  The
-// output offset of sequence b is sum_{b'<b} min(k, candidates(b')), which each
-// CTA computes from lock_in itself; when lock_in and lock_out alias, a
-// sequence's min(k, unlocked) count is the same before, during and after its
-// CTA rewrites it, so no inter-CTA ordering is needed.
-__global__ void __launch_bounds__(kSelThreads) topk_compact_kernel(const float* __restrict__ score,
-                                                                   const uint8_t* lock_in, uint8_t* lock_out,
-                                                                   int N, int k, int largest,
-                                                                   int32_t* __restrict__ idx_out,
-                                                                   int32_t* __restrict__ seg_ptr) {
+// (ties to the lower index) and lock every other row.  Radix select on 8-bit
+// digits finds the k-th key (warp-parallel bin search); an ordered block scan
+// breaks ties.  direct (a single sequence): the
+// kept rows are compacted here; otherwise seg_ptr[b + 1] = -(kept + 1) for the
+// compaction launch.  lock_in and lock_out may alias: a CTA reads only its own
+// sequence, and each row's lock_in before its lock_out.
+__global__ void __launch_bounds__(kSelThreads) topk_decide_kernel(const float* __restrict__ score,
+                                                                  const uint8_t* lock_in, uint8_t* lock_out,
+                                                                  int N, int k, int largest, int direct,
+                                                                  int32_t* __restrict__ idx_out,
+                                                                  int32_t* __restrict__ seg_ptr) {
   __shared__ int hist[256];
   __shared__ int sh[33];
   __shared__ uint32_t s_prefix;
@@ -196,14 +244,6 @@ __global__ void __launch_bounds__(kSelThreads) topk_compact_kernel(const float* 
   const int b = blockIdx.x;
   const long long base = (long long)b * N;
   const bool lg = largest != 0;
-  int offset = 0;
-  if (k > 0) {
-    for (int bp = 0; bp < b; ++bp) {
-      int c = 0;
-      for (int i = threadIdx.x; i < N; i += blockDim.x) c += lock_in[(long long)bp * N + i] ? 0 : 1;
-      offset += min(k, block_sum(c, sh));
-    }
-  }
   int c = 0;
   for (int i = threadIdx.x; i < N; i += blockDim.x) c += lock_in[base + i] ? 0 : 1;
   const int ncand = block_sum(c, sh);
@@ -237,23 +277,32 @@ __global__ void __launch_bounds__(kSelThreads) topk_compact_kernel(const float* 
     if (i < N) lock_out[base + i] = keep ? 0 : 1;
     int kt;
     const int kr = block_rank(keep ? 1 : 0, sh, &kt);
-    if (keep) idx_out[offset + running + kr] = (int32_t)(base + i);
+    if (direct && keep) idx_out[running + kr] = (int32_t)(base + i);
     running += kt;
   }
   if (threadIdx.x == 0) {
-    seg_ptr[b + 1] = offset + running;
-    if (b == 0) seg_ptr[0] = 0;
+    if (direct) {
+      seg_ptr[0] = 0;
+      seg_ptr[1] = running;
+    } else {
+      seg_ptr[b + 1] = -(running + 1);
+    }
   }
 }
 
 int launch_select(const plk_dims* dims, const float* score, const uint8_t* lock_in, uint8_t* lock_out,
                   int mode, float tau, int k, int32_t* idx_out, int32_t* seg_ptr, cudaStream_t st) {
   const int B = dims->B, N = dims->N;
+  const int direct = B == 1 ? 1 : 0;
+  int e;
   if (mode == PLK_SEL_TOPK_LARGEST || mode == PLK_SEL_TOPK_SMALLEST) {
-    return launch_pdl(topk_compact_kernel, dim3(B), dim3(kSelThreads), 0, st, score, lock_in, lock_out, N, k,
-                      (int)(mode == PLK_SEL_TOPK_LARGEST), idx_out, seg_ptr);
-  }
-  return launch_pdl(compact_kernel, dim3(B), dim3(kSelThreads), 0, st, mode, score, lock_in, lock_out, N, tau, idx_out,
+    e = launch_pdl(topk_decide_kernel, dim3(B), dim3(kSelThreads), 0, st, score, lock_in, lock_out, N, k,
+                   (int)(mode == PLK_SEL_TOPK_LARGEST), direct, idx_out, seg_ptr);
+  } else
+    e = launch_pdl(thresh_decide_kernel, dim3(B), dim3(kSelThreads), 0, st, mode, score, lock_in, lock_out, N, tau,
+                   direct, idx_out, seg_ptr);
+  if (e != PLK_OK || direct) return e;
+  return launch_pdl(compact_lock_kernel, dim3(B), dim3(kSelThreads), 0, st, (const uint8_t*)lock_out, N, idx_out,
                     seg_ptr);
 }
 
