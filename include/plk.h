@@ -145,7 +145,9 @@ int plk_select_active(const plk_dims* dims, const float* score, const uint8_t* l
  * S4..S10  One partial-recompute layer step ([SL] Sec. 2 "Permanent
  * Deactivation", "Continued Attention", "Algorithmic Complexity").
  *   X [B, N, d]: layer input hidden states.  idx / seg_ptr: the active rows
- *   as written by plk_select_active (M = seg_ptr[B], read on the device).
+ *   as written by plk_select_active (M = seg_ptr[B], read on the device); idx
+ *   is a [B*N] buffer: entries past M are read (so that their loads overlap
+ *   the read of M) but never used.
  *   For every active row j (token row t = idx[j] of sequence b):
  *     xn = RMSNorm(x_t) * g1;   [q|k|v] = xn W_qkv^T
  *     K_cache[t] = k, V_cache[t] = v          (before attention)
@@ -254,6 +256,7 @@ int plk_slowfast_step(const plk_dims* dims, const plk_sf_params* params, const f
 
 /*
  * S10 (proxy half)  proxy_cache[idx[j]] = proxy_new[idx[j]] for j < M = seg_ptr[B].
+ * idx is a [B*N] buffer (entries past M are read, never used).
  * Both [B, N, r] fp32; rows not in idx are untouched.
  */
 int plk_proxy_commit(const plk_dims* dims, int r, const int32_t* idx, const int32_t* seg_ptr,

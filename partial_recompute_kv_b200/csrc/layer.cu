@@ -261,7 +261,7 @@ __device__ __forceinline__ void store_hilo(__nv_bfloat16* hi, __nv_bfloat16* lo,
 
 template <typename Tin, typename Tg, typename Tout, int NV>
 __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict__ X, const int32_t* __restrict__ idx,
-                                                          const int32_t* __restrict__ seg_ptr, int B,
+                                                          const int32_t* __restrict__ seg_ptr, int B, int Mcap,
                                                           const Tg* __restrict__ g, float eps, int d,
                                                           Tout* __restrict__ out, Tout* __restrict__ out_lo,
                                                           float* __restrict__ res_out, float* __restrict__ zero_out,
@@ -270,61 +270,83 @@ __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict_
   __shared__ float sh[33];
   pdl_wait();
   pdl_trigger();
+  // M, the gains and the first row are loaded without waiting for one another
   const int M = seg_ptr[B];
-  for (int j = blockIdx.x; j < M; j += gridDim.x) {  // grid-stride over the live rows (uniform per block)
-  if (zero_out) clear_row(zero_out + (size_t)j * zcols, zcols);
-  const size_t row = idx ? (size_t)idx[j] : (size_t)j;
-  const uint4* xv = reinterpret_cast<const uint4*>(X + row * d);
   const int nvec = d / E;
-  uint4 buf[NV];
+  float gf[NV][E];
 #pragma unroll
   for (int u = 0; u < NV; ++u) {
     const int vi = threadIdx.x + u * 256;
-    if (vi < nvec) buf[u] = __ldg(xv + vi);
+#pragma unroll
+    for (int e = 0; e < E; ++e) gf[u][e] = vi < nvec ? to_f(g[vi * E + e]) : 0.f;
   }
-  float ss = 0.f;
+  // Rows j < Mcap exist in idx (B*N entries) and in an un-gathered source
+  // ([Mcap, d]), so their loads are issued before M is known; nothing of a row
+  // j >= M is used.
+  for (int j = blockIdx.x; j < Mcap; j += gridDim.x) {  // grid-stride over the rows (uniform per block)
+    uint4 buf[NV];
+    if (idx) {
+      const size_t row = (size_t)idx[j];
+      if (j >= M) return;
+      const uint4* xv = reinterpret_cast<const uint4*>(X + row * d);
 #pragma unroll
-  for (int u = 0; u < NV; ++u) {
-    if (threadIdx.x + u * 256 < nvec) {
-      float f[E];
-      Vec16<Tin>::unpack(buf[u], f);
-#pragma unroll
-      for (int e = 0; e < E; ++e) ss = fmaf(f[e], f[e], ss);
-    }
-  }
-  ss = block_sum_f(ss, sh);
-  const float inv = 1.0f / sqrtf(ss / (float)d + eps);
-  Tout* o = out + (size_t)j * d;
-#pragma unroll
-  for (int u = 0; u < NV; ++u) {
-    const int vi = threadIdx.x + u * 256;
-    if (vi < nvec) {
-      float f[E];
-      Vec16<Tin>::unpack(buf[u], f);
-      if (res_out) store_vec<float, E>(res_out + (size_t)j * d + vi * E, f);
-#pragma unroll
-      for (int e = 0; e < E; ++e) f[e] = f[e] * inv * to_f(g[vi * E + e]);
-      if constexpr (std::is_same<Tout, __nv_bfloat16>::value) {
-        if (out_lo) {
-          store_hilo<E>(o + vi * E, out_lo + (size_t)j * d + vi * E, f);
-          continue;
-        }
+      for (int u = 0; u < NV; ++u) {
+        const int vi = threadIdx.x + u * 256;
+        if (vi < nvec) buf[u] = __ldg(xv + vi);
       }
-      store_vec<Tout, E>(o + vi * E, f);
+    } else {
+      const uint4* xv = reinterpret_cast<const uint4*>(X + (size_t)j * d);
+#pragma unroll
+      for (int u = 0; u < NV; ++u) {
+        const int vi = threadIdx.x + u * 256;
+        if (vi < nvec) buf[u] = __ldg(xv + vi);
+      }
+      if (j >= M) return;
     }
-  }
+    if (zero_out) clear_row(zero_out + (size_t)j * zcols, zcols);
+    float ss = 0.f;
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+      if (threadIdx.x + u * 256 < nvec) {
+        float f[E];
+        Vec16<Tin>::unpack(buf[u], f);
+#pragma unroll
+        for (int e = 0; e < E; ++e) ss = fmaf(f[e], f[e], ss);
+      }
+    }
+    ss = block_sum_f(ss, sh);
+    const float inv = 1.0f / sqrtf(ss / (float)d + eps);
+    Tout* o = out + (size_t)j * d;
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+      const int vi = threadIdx.x + u * 256;
+      if (vi < nvec) {
+        float f[E];
+        Vec16<Tin>::unpack(buf[u], f);
+        if (res_out) store_vec<float, E>(res_out + (size_t)j * d + vi * E, f);
+#pragma unroll
+        for (int e = 0; e < E; ++e) f[e] = f[e] * inv * gf[u][e];
+        if constexpr (std::is_same<Tout, __nv_bfloat16>::value) {
+          if (out_lo) {
+            store_hilo<E>(o + vi * E, out_lo + (size_t)j * d + vi * E, f);
+            continue;
+          }
+        }
+        store_vec<Tout, E>(o + vi * E, f);
+      }
+    }
   }
 }
 
 // Picks the register-resident kernel when the row fits, else the looping one.
 template <typename Tin, typename Tg, typename Tout>
-static int launch_rmsnorm(const Tin* X, const int32_t* idx, const int32_t* seg, int B, const Tg* g, float eps,
-                           int d, Tout* out, Tout* out_lo, int grid, cudaStream_t st, float* res_out = nullptr,
-                           float* zero_out = nullptr, int zcols = 0) {
+static int launch_rmsnorm(const Tin* X, const int32_t* idx, const int32_t* seg, int B, int Mcap, const Tg* g,
+                          float eps, int d, Tout* out, Tout* out_lo, int grid, cudaStream_t st,
+                          float* res_out = nullptr, float* zero_out = nullptr, int zcols = 0) {
   constexpr int E = Vec16<Tin>::E;
   if (d % E == 0 && d <= 4 * 256 * E)
-    return launch_pdl(rmsnorm_vec_kernel<Tin, Tg, Tout, 4>, dim3(grid), dim3(256), 0, st, X, idx, seg, B, g, eps, d,
-                      out, out_lo, res_out, zero_out, zcols);
+    return launch_pdl(rmsnorm_vec_kernel<Tin, Tg, Tout, 4>, dim3(grid), dim3(256), 0, st, X, idx, seg, B, Mcap, g,
+                      eps, d, out, out_lo, res_out, zero_out, zcols);
   return launch_pdl(rmsnorm_rows_kernel<Tin, Tg, Tout>, dim3(grid), dim3(256), 0, st, X, idx, seg, B, g, eps, d, out,
                     out_lo, res_out, zero_out, zcols);
 }
@@ -577,7 +599,7 @@ static int run_layer_f32(const plk_dims* dm, const plk_weights* w, const float* 
     gemm_f32_kernel<<<grid, 256, 0, st>>>(A, (const float*)Wt, c32, Nout, K, seg, B);
   };
   const int ngrid = std::min(Mcap, 2 * L.num_sms);  // row kernels: grid-stride over the M live rows
-  PLK_TRY(launch_rmsnorm<float, float, float>(X, idx, seg, B, (const float*)w->g1, dm->eps, d, xn, nullptr, ngrid,
+  PLK_TRY(launch_rmsnorm<float, float, float>(X, idx, seg, B, Mcap, (const float*)w->g1, dm->eps, d, xn, nullptr, ngrid,
                                               st));
   gemm(xn, w->w_qkv, d + 2 * dkv, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_QKV, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, dm->N,
@@ -586,7 +608,7 @@ static int run_layer_f32(const plk_dims* dm, const plk_weights* w, const float* 
   PLK_TRY(launch_attention_f32(dm, q, Kc, Vc, a, seg, Mcap, st));
   gemm(a, w->w_o, d, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_O, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, 0, 0, 0.f, 0);
-  PLK_TRY(launch_rmsnorm<float, float, float>(h32, nullptr, seg, B, (const float*)w->g2, dm->eps, d, hn, nullptr,
+  PLK_TRY(launch_rmsnorm<float, float, float>(h32, nullptr, seg, B, Mcap, (const float*)w->g2, dm->eps, d, hn, nullptr,
                                               ngrid, st));
   gemm(hn, w->w_gu, 2 * F, d);
   epilogue_f32_kernel<<<rows, 256, 0, st>>>(F32_GU, c32, idx, seg, B, d, F, q, Kc, Vc, X, h32, act, Y, 0, 0, 0.f, 0);
@@ -642,7 +664,7 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
 
   trace_mark(0, st);
   // x (fp32) staged in h32 takes the O projection's adds; the QKV sums start at 0
-  PLK_TRY(launch_rmsnorm<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(X, idx, seg, B, (const __nv_bfloat16*)w->g1,
+  PLK_TRY(launch_rmsnorm<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(X, idx, seg, B, Mcap, (const __nv_bfloat16*)w->g1,
                                                                       dm->eps, d, xn, xn_lo, rgrid, st, h32,
                                                                       c32, d + 2 * dkv));
   trace_mark(1, st);
@@ -668,7 +690,7 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   PLK_TRY(launch_gemm_tc(tW_o, tX_a[0], tX_a[1], tO_h, g, st));  // h = x + a W_o^T
   trace_mark(5, st);
 
-  PLK_TRY(launch_rmsnorm<float, __nv_bfloat16, __nv_bfloat16>(h32, nullptr, seg, B, (const __nv_bfloat16*)w->g2,
+  PLK_TRY(launch_rmsnorm<float, __nv_bfloat16, __nv_bfloat16>(h32, nullptr, seg, B, Mcap, (const __nv_bfloat16*)w->g2,
                                                               dm->eps, d, hn, hn_lo, rgrid, st, nullptr, c32,
                                                               2 * F));
   trace_mark(6, st);

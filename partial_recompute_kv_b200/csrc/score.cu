@@ -308,15 +308,25 @@ __global__ void __launch_bounds__(256) score_f32_kernel(const float* __restrict_
   if (lane == 0) score[row] = metric == PLK_METRIC_COS ? dot / fmaxf(sqrtf(pp) * sqrtf(cc), 1e-30f) : sqrtf(dd);
 }
 
+// One warp per compact row j: idx has B*N entries, so idx[j] is loaded beside
+// M = seg_ptr[B]; the row's r <= 256 values are all loaded before any store.
 __global__ void proxy_commit_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ seg_ptr, int B,
-                                    int r, const float* __restrict__ pnew, float* __restrict__ pc) {
+                                    int rows, int r, const float* __restrict__ pnew, float* __restrict__ pc) {
   pdl_wait();
   pdl_trigger();
-  const int M = seg_ptr[B];
   const int j = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (j >= M) return;
+  if (j >= rows) return;
+  const int M = seg_ptr[B];
   const size_t row = (size_t)idx[j];
-  for (int c = threadIdx.x & 31; c < r; c += 32) pc[row * r + c] = pnew[row * r + c];
+  if (j >= M) return;
+  const int lane = threadIdx.x & 31;
+  float v[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+    if (lane + u * 32 < r) v[u] = pnew[row * r + lane + u * 32];
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+    if (lane + u * 32 < r) pc[row * r + lane + u * 32] = v[u];
 }
 
 static int score_tc_smem(int r) {
@@ -383,7 +393,7 @@ int launch_score(const plk_dims* dims, const void* X, const void* Ut, int r, con
 int launch_proxy_commit(const plk_dims* dims, int r, const int32_t* idx, const int32_t* seg_ptr,
                         const float* proxy_new, float* proxy_cache, cudaStream_t st) {
   const int rows = dims->B * dims->N;
-  return launch_pdl(proxy_commit_kernel, dim3(ceil_div(rows, 8)), dim3(256), 0, st, idx, seg_ptr, dims->B, r,
+  return launch_pdl(proxy_commit_kernel, dim3(ceil_div(rows, 8)), dim3(256), 0, st, idx, seg_ptr, dims->B, rows, r,
                     proxy_new, proxy_cache);
 }
 
