@@ -8,14 +8,18 @@
 //
 // One CTA per sequence decides every row's lock (threshold: compare; top-k:
 // radix select of the k-th key, then an ordered tie-break) and compacts its active rows chunk by chunk with warp
-// ballots, popcounts and a block scan of the 32 warp counts.  A single
-// sequence is done in that one launch.  With B > 1 sequences the decide launch
+// ballots, popcounts and a block scan of the 32 warp counts; top-k on sequences
+// of 2049 .. 32768 rows runs on a cluster of up to 8 CTAs per sequence instead
+// (keys in registers, histograms merged through distributed shared memory).  A
+// single sequence is done in that one launch.  With B > 1 sequences the decide launch
 // leaves each sequence's active count in seg_ptr[b + 1] (encoded as -(count+1))
 // and a second launch compacts: CTA b finds its output offset by walking
 // seg_ptr down from b, adding encoded counts until it meets an entry another
 // CTA has already turned into its final prefix sum (no inter-CTA waiting, no
 // scratch memory, O(B) reads per CTA).  Indices come out ascending and
 // deterministic.
+#include <algorithm>
+
 #include "plk_common.cuh"
 #include "plk_internal.h"
 
@@ -290,14 +294,244 @@ __global__ void __launch_bounds__(kSelThreads) topk_decide_kernel(const float* _
   }
 }
 
+// ---------------------------------------------------------------------------
+// The top-k rule with the keys in registers, on a cluster of 2 <= S <= 8 CTAs of
+// NT threads per sequence (sequences of more than 2048 rows).  CTA s owns rows
+// [s L, min((s + 1) L, N)), L = ceil(N / S); thread t keeps the keys of rows
+// s L + t + NT j (j < KPT), so the scores are read once.  Every radix pass
+// builds a 256-bin histogram per CTA (two buffers, alternating, so one cluster
+// barrier per pass suffices) and every CTA sums the S histograms through
+// distributed shared memory and finds the same digit; the first pass's bins
+// also count the candidates.  Then each CTA publishes its count of rows kept
+// for sure and of ties at the k-th key: the ties kept are the lowest indices,
+// so a CTA's ties and kept rows come after those of the CTAs of lower rank and
+// the result equals the one-CTA kernel's.  direct (one sequence): the CTAs
+// compact their kept rows at their offsets; otherwise rank 0 leaves
+// seg_ptr[b + 1] = -(kept + 1) for the compaction launch.
+__device__ __forceinline__ int ld_dsmem_s32(const int* p, uint32_t rank) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(dsmem_addr(smem_u32(p), rank)));
+  return v;
+}
+// p's value summed over the S CTAs of the cluster (the loads are all issued before the adds)
+__device__ __forceinline__ int cluster_sum(const int* p, int S, int upto) {
+  int v[8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r) v[r] = ld_dsmem_s32(p, (uint32_t)(r < S ? r : 0));
+  int tot = 0;
+#pragma unroll
+  for (int r = 0; r < 8; ++r) tot += r < upto ? v[r] : 0;
+  return tot;
+}
+
+constexpr int kSelClusterThreads = 256;
+
+template <int KPT, int NT>
+__global__ void __launch_bounds__(NT) topk_cluster_kernel(const float* __restrict__ score,
+                                                                          const uint8_t* lock_in, uint8_t* lock_out,
+                                                                          int N, int k, int largest, int direct,
+                                                                          int S, int32_t* __restrict__ idx_out,
+                                                                          int32_t* __restrict__ seg_ptr) {
+  __shared__ int hist[2][256];
+  __shared__ int gh[256];    // the cluster's histogram of the current pass
+  __shared__ int pub[2];     // published to the cluster: rows kept for sure, ties at the k-th key
+  __shared__ int sh[33];
+  __shared__ uint32_t s_prefix;
+  __shared__ int s_rem, s_ncand;
+  pdl_wait();
+  pdl_trigger();
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int s = (int)cluster_ctarank();
+  const int b = blockIdx.y;
+  const long long base = (long long)b * N;
+  const int L = (N + S - 1) / S;
+  const int lo = s * L, hi = min(N, lo + L);
+  const bool lg = largest != 0;
+  uint32_t key[KPT];
+  bool cand[KPT];
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    const int i = lo + t + NT * j;
+    cand[j] = i < hi && lock_in[base + i] == 0;
+    key[j] = cand[j] ? pref_key(score[base + i], lg) : 0u;
+  }
+  uint32_t prefix = 0u, pmask = 0u;
+  int rem = 0, ncand = 0, keep_n = 0;
+  bool keep_none = true, keep_all = false;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    int* hb = hist[pass & 1];  // the other buffer may still be read by the cluster
+    if (t < 256) hb[t] = 0;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < KPT; ++j)
+      if (cand[j] && (key[j] & pmask) == prefix) atomicAdd(&hb[(key[j] >> shift) & 255u], 1);
+    cluster_sync_all();  // every CTA's histogram of this pass is complete
+    if (t < 256) gh[t] = cluster_sum(&hb[t], S, S);
+    __syncthreads();
+    if (pass == 0) {  // every candidate is in the first pass's histogram
+      if (warp == 0) {
+        int c = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) c += gh[lane * 8 + q];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        if (lane == 0) s_ncand = c;
+      }
+      __syncthreads();
+      ncand = s_ncand;
+      keep_n = k <= 0 ? 0 : min(k, ncand);
+      keep_none = keep_n == 0;
+      keep_all = !keep_none && keep_n == ncand;
+      rem = keep_n;
+      if (keep_none || keep_all) break;  // the same in every CTA
+    }
+    if (warp == 0) {
+      // lane l owns bins 255-8l .. 248-8l (descending); find the bin holding the
+      // rem-th most preferred key
+      int cnt[8], tt = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        cnt[q] = gh[255 - 8 * lane - q];
+        tt += cnt[q];
+      }
+      int inc = tt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += n;
+      }
+      int above = inc - tt;
+      if (above < rem && rem <= inc) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (above + cnt[q] >= rem) {
+            s_prefix = prefix | ((uint32_t)(255 - 8 * lane - q) << shift);
+            s_rem = rem - above;
+            break;
+          }
+          above += cnt[q];
+        }
+      }
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    rem = s_rem;
+    pmask |= 0xFFu << shift;
+  }
+  const bool sel = !keep_none && !keep_all;
+  const uint32_t kth = prefix;
+  const int remaining = sel ? rem : 0;  // ties at kth that are kept, lowest indices first
+  // this CTA's rows kept for sure (every candidate, or the keys above the k-th) and its ties
+  int gtc = 0, eqc = 0;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    gtc += (cand[j] && (keep_all || (sel && key[j] > kth))) ? 1 : 0;
+    eqc += (sel && cand[j] && key[j] == kth) ? 1 : 0;
+  }
+  gtc = block_sum(gtc, sh);
+  eqc = block_sum(eqc, sh);
+  if (t == 0) {
+    pub[0] = gtc;
+    pub[1] = eqc;
+  }
+  cluster_sync_all();
+  // kept rows of CTA r: its sure rows plus its share of the ties, taken in rank order
+  int before = 0, all = 0, eq_before = 0;
+  {
+    int gv[8], ev[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      gv[r] = ld_dsmem_s32(&pub[0], (uint32_t)(r < S ? r : 0));
+      ev[r] = ld_dsmem_s32(&pub[1], (uint32_t)(r < S ? r : 0));
+    }
+    int taken = 0;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      if (r < S) {
+        const int kr = gv[r] + max(0, min(ev[r], remaining - taken));
+        if (r < s) {
+          before += kr;
+          eq_before += ev[r];
+        }
+        all += kr;
+        taken += ev[r];
+      }
+    }
+  }
+  int taken_eq = eq_before, running = before;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {  // row order: j, then t
+    const bool eq = sel && cand[j] && key[j] == kth;
+    const bool gt = sel && cand[j] && key[j] > kth;
+    int total;
+    const int r = block_rank(eq ? 1 : 0, sh, &total);
+    const bool keep = cand[j] && !keep_none && (keep_all || gt || (eq && taken_eq + r < remaining));
+    taken_eq += total;
+    const int i = lo + t + NT * j;
+    if (i < hi) lock_out[base + i] = keep ? 0 : 1;
+    if (direct) {
+      int kt;
+      const int kr = block_rank(keep ? 1 : 0, sh, &kt);
+      if (keep) idx_out[running + kr] = (int32_t)(base + i);
+      running += kt;
+    }
+  }
+  if (s == 0 && t == 0) {
+    if (direct) {
+      seg_ptr[0] = 0;
+      seg_ptr[1] = all;
+    } else {
+      seg_ptr[b + 1] = -(all + 1);
+    }
+  }
+  cluster_sync_all();  // no CTA leaves while another can still read its shared memory
+}
+
 int launch_select(const plk_dims* dims, const float* score, const uint8_t* lock_in, uint8_t* lock_out,
                   int mode, float tau, int k, int32_t* idx_out, int32_t* seg_ptr, cudaStream_t st) {
   const int B = dims->B, N = dims->N;
   const int direct = B == 1 ? 1 : 0;
   int e;
-  if (mode == PLK_SEL_TOPK_LARGEST || mode == PLK_SEL_TOPK_SMALLEST) {
-    e = launch_pdl(topk_decide_kernel, dim3(B), dim3(kSelThreads), 0, st, score, lock_in, lock_out, N, k,
-                   (int)(mode == PLK_SEL_TOPK_LARGEST), direct, idx_out, seg_ptr);
+  const int largest = (int)(mode == PLK_SEL_TOPK_LARGEST);
+  const bool topk = mode == PLK_SEL_TOPK_LARGEST || mode == PLK_SEL_TOPK_SMALLEST;
+  // sequences of more than 2048 rows: keys in registers on a cluster of S CTAs of
+  // 256 threads (512 rows each and more, at most 4096 each); shorter ones (and
+  // longer than 8 x 4096) on one CTA of 1024 threads, which is faster there
+  const int S = std::min(8, ceil_div(N, 512));
+  const int NT = kSelClusterThreads;
+  const int kpt = ceil_div(ceil_div(N, S), NT);
+  if (topk && N > 2048 && kpt <= 16) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)S, (unsigned)B, 1);
+    cfg.blockDim = dim3((unsigned)NT, 1, 1);
+    cfg.stream = st;
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    at[1].id = cudaLaunchAttributeClusterDimension;
+    at[1].val.clusterDim.x = (unsigned)S;
+    at[1].val.clusterDim.y = 1;
+    at[1].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 2;
+    cudaError_t ce;
+#define PLK_TOPK_LAUNCH(KPT_, NT_)                                                                            \
+  ce = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<KPT_, NT_>, score, lock_in, lock_out, N, k, largest, direct, S, \
+                          idx_out, seg_ptr)
+    if (kpt <= 2)
+      PLK_TOPK_LAUNCH(2, kSelClusterThreads);
+    else if (kpt <= 4)
+      PLK_TOPK_LAUNCH(4, kSelClusterThreads);
+    else if (kpt <= 8)
+      PLK_TOPK_LAUNCH(8, kSelClusterThreads);
+    else
+      PLK_TOPK_LAUNCH(16, kSelClusterThreads);
+#undef PLK_TOPK_LAUNCH
+    e = ce == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;
+  } else if (topk) {  // longer sequences: the one-CTA kernel that reads the scores per pass
+    e = launch_pdl(topk_decide_kernel, dim3(B), dim3(kSelThreads), 0, st, score, lock_in, lock_out, N, k, largest,
+                   direct, idx_out, seg_ptr);
   } else
     e = launch_pdl(thresh_decide_kernel, dim3(B), dim3(kSelThreads), 0, st, mode, score, lock_in, lock_out, N, tau,
                    direct, idx_out, seg_ptr);

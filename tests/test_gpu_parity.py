@@ -92,7 +92,9 @@ def test_select_threshold_bitexact(plk, B, N, gt, inplace):
     check_guards({"lock_in": glin, "lock_out": glout}, "threshold select")
 
 
-@pytest.mark.parametrize("B,N", [(1, 5), (2, 777), (8, 4096)])
+# N <= 256: one CTA per sequence; larger N: a cluster of up to 8 CTAs per sequence (up to 4096 rows
+# each; (1, 40000) is past that and goes back to one CTA)
+@pytest.mark.parametrize("B,N", [(1, 5), (2, 777), (8, 4096), (1, 1024), (1, 8192), (1, 32000), (3, 40000)])
 @pytest.mark.parametrize("kind", ["random", "ties", "nan"])
 @pytest.mark.parametrize("largest", [True, False])
 def test_select_topk_bitexact(plk, B, N, kind, largest):
