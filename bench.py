@@ -529,23 +529,37 @@ def run_kl_lock(args):
 # compute-bound GEMMs and attention, the K/V scatter at 67 MB)
 # ---------------------------------------------------------------------------
 def _timed(torch, fn, steps, warmup):
+    """Device time of one call of fn: `reps` calls captured in a CUDA graph (so host launch
+    time is not measured), the graph replayed with events around every replay; median."""
     for _ in range(max(warmup, 3)):
         fn()
     torch.cuda.synchronize()
+    reps = max(1, min(steps, 20))
+    stream = torch.cuda.Stream()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for _ in range(reps):
+            fn()
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
     E = lambda: torch.cuda.Event(enable_timing=True)
-    ev = [(E(), E()) for _ in range(steps)]
+    ev = [(E(), E()) for _ in range(max(3, steps // reps))]
     for a, b in ev:
         a.record()
-        fn()
+        graph.replay()
         b.record()
     torch.cuda.synchronize()
-    return statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
+    del graph
+    return statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3 / reps
 
 
 def run_kernel_configs(args):
     import torch
     import partial_recompute_kv_b200 as plk
     import synth
+
+    clk = ClockSampler(0).__enter__()  # SM clock and throttle reasons over every config below
 
     dev = torch.device("cuda", 0)
     bf = torch.bfloat16
@@ -642,7 +656,9 @@ def run_kernel_configs(args):
     st = plk.get_status()
     if st != plk.OK:
         raise RuntimeError(f"device status {plk.error_string(st)}")
+    clk.__exit__(None, None, None)
     for o in out:
+        o["clocks_over_all_configs"] = clk.summary()
         print(json.dumps(o), flush=True)
     return 0
 
