@@ -22,16 +22,20 @@
 //  * Warp roles: warp 0 issues TMA in both CTAs, every load counting its bytes
 //    on the even CTA's stage barrier; one thread of warp 1 of the even CTA
 //    issues the pair MMAs; warps 2-5 of both CTAs drain their TMEM.
-//  * Persistent stream-K without inter-CTA waiting: each pair owns an equal,
-//    contiguous share of the (256-feature tile) x (k-block) iteration space
-//    and adds the fp32 partial of each tile piece it covers into the fp32
-//    output with TMA bulk reduce-add (cp.reduce.async.bulk.tensor .add.f32),
-//    which the L2 applies atomically.  The output is the residual stream h
-//    (O and down projections) or a zeroed fp32 buffer that a finishing kernel
-//    turns into bf16 (QKV -> Q and the K/V cache rows; gate/up -> silu(g) u).
-//    The order of the adds is not fixed: results may differ in the last fp32
-//    bit between runs.  A tile piece accumulates its whole k range in TMEM
-//    before its one reduce-add.
+//  * Persistent stream-K: each pair owns an equal, contiguous share of the
+//    (256-feature tile) x (k-block) iteration space and adds the fp32 partial
+//    of each tile piece it covers into the fp32 output with TMA bulk
+//    reduce-add (cp.reduce.async.bulk.tensor .add.f32), which the L2 applies
+//    atomically.  The output is the residual stream h (O and down projections)
+//    or an fp32 sums buffer that a finishing kernel turns into bf16 (QKV -> Q
+//    and the K/V cache rows; gate/up -> silu(g) u).  The sums buffer is not
+//    zeroed: a whole-tile piece stores its partial (TMA bulk store); in a split
+//    tile the piece whose warp arrives first stores and raises a ready flag once
+//    the store is complete, and the later pieces' warps wait for that flag (a
+//    bounded wait on a CTA that is already running and waits on nothing) before
+//    they add.  The order of the adds is not fixed: results may differ in the
+//    last fp32 bit between runs.  A tile piece accumulates its whole k range in
+//    TMEM before its one store or reduce-add.
 //  * Two 256-column TMEM accumulators per CTA: the epilogue drains one tile
 //    piece while the MMA fills the next; the producers run ahead across
 //    pieces.
@@ -76,6 +80,13 @@ __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* tm, int x, 
           reinterpret_cast<uint64_t>(tm)),
       "r"(x), "r"(y), "r"(smem_u32(smem_src))
       : "memory");
+}
+// bulk store of a [32 rows][32 fp32] smem block into the tensor at (x, y)
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, int x, int y, const void* smem_src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(tm)),
+               "r"(x), "r"(y), "r"(smem_u32(smem_src))
+               : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // waits until at most n committed bulk groups still read their shared-memory source
@@ -335,6 +346,34 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                 : t.ft * kGemmBM + q * 32;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * 256);
       const int nchunks = t.ncols >> 5;
+      // Into an output that starts undefined (args.arrive set), the piece of a tile that gets
+      // there first stores its partial and the later pieces add theirs once that store is
+      // complete (a per-(tile, CTA, warp) arrival count and ready flag); a whole tile is stored.
+      bool store = false;
+      uint32_t* ready = nullptr;
+      if (args.arrive) {
+        if (kb0 == 0 && kb1 == KB) {
+          store = true;
+        } else {
+          const int slot = (2 * u + rank) * 4 + q;
+          int old = 0;
+          if (lane == 0) old = atomicAdd(args.arrive + slot, 1);
+          old = __shfl_sync(0xffffffffu, old, 0);
+          ready = args.ready + slot;
+          store = old == 0;
+          if (!store) {
+            bool got = true;
+            if (lane == 0) {
+              got = spin_until_geq(ready, 1u);  // the first piece's CTA is running: bounded, short
+              fence_proxy_async_global();       // its stored values before this warp's bulk adds
+            }
+            if (!__all_sync(0xffffffffu, __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0)) {
+              if (lane == 0) *s_abort = 1;
+            }
+            ready = nullptr;
+          }
+        }
+      }
       for (int c = 0; c < nchunks; ++c) {
         float* blk;
         if (last) {
@@ -366,9 +405,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         fence_proxy_async_smem();  // make the block visible to the bulk-copy unit
         __syncwarp();
         if (lane == 0) {
-          tma_reduce_add_2d(&tmOut, col, t.tok0 + c * 32, blk);
+          if (store)
+            tma_store_2d(&tmOut, col, t.tok0 + c * 32, blk);
+          else
+            tma_reduce_add_2d(&tmOut, col, t.tok0 + c * 32, blk);
           bulk_commit();
         }
+      }
+      if (ready) {  // first piece of a split tile: its store is complete, the others may add
+        if (lane == 0) {
+          bulk_wait_all();
+          fence_proxy_async_global();
+          red_release_add_u32(ready, 1u);
+        }
+        __syncwarp();
       }
       ++j;
     }

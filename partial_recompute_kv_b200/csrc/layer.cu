@@ -77,6 +77,14 @@ Workspace workspace_layout(const plk_dims* dm, int num_sms) {
   w.num_sms = num_sms;
   w.c32_bytes = 4 * Mcap * std::max(d + 2 * (size_t)kv_width(dm), 2 * F);
   w.c32 = take(w.c32_bytes);
+  if (dm->dtype == PLK_BF16) {
+    // arrival counts and ready flags of the QKV and gate/up GEMMs: 8 per pair tile each
+    const size_t tt = (Mcap + kGemmBNMax - 1) / kGemmBNMax;
+    w.gsync_tiles[0] = (int)(((d + 2 * (size_t)kv_width(dm)) / 256) * tt);
+    w.gsync_tiles[1] = (int)((F / 128) * tt);
+    w.gsync_ints = 16 * (w.gsync_tiles[0] + w.gsync_tiles[1]);
+    w.gsync = take(4 * (size_t)w.gsync_ints);
+  }
   w.total = off;
   return w;
 }
@@ -142,30 +150,26 @@ __device__ __forceinline__ float block_sum_f(float v, float* sh) {
   return sh[32];
 }
 
-// zcols % 4 == 0, row 16-byte aligned
-__device__ __forceinline__ void clear_row(float* row, int zcols) {
-  float4* r4 = reinterpret_cast<float4*>(row);
-  for (int c = threadIdx.x; c < (zcols >> 2); c += blockDim.x) r4[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-}
 
 // out[j] = RMSNorm(src_row(j)) * g for j < M.  src_row(j) = X[idx[j]] (gather)
 // or H[j] (idx == nullptr); res_out (optional) receives the fp32 source row;
-// zero_out (optional) gets row j of a [Mcap, zcols] fp32 buffer cleared for the
-// reduce-adds of the GEMM that follows.  With a bf16 output, out receives
+// zero_ints (optional): nzero ints that the grid clears (counters and flags of
+// later kernels of the step).  With a bf16 output, out receives
 // hi = bf16(v) and out_lo (when given) lo = bf16(v - hi).
 template <typename Tin, typename Tg, typename Tout>
 __global__ void __launch_bounds__(256) rmsnorm_rows_kernel(const Tin* __restrict__ X, const int32_t* __restrict__ idx,
                                                            const int32_t* __restrict__ seg_ptr, int B,
                                                            const Tg* __restrict__ g, float eps, int d,
                                                            Tout* __restrict__ out, Tout* __restrict__ out_lo,
-                                                           float* __restrict__ res_out, float* __restrict__ zero_out,
-                                                           int zcols) {
+                                                           float* __restrict__ res_out, int* __restrict__ zero_ints,
+                                                           int nzero) {
   __shared__ float sh[33];
   pdl_wait();
   pdl_trigger();
+  if (zero_ints)
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nzero; i += gridDim.x * blockDim.x) zero_ints[i] = 0;
   const int M = seg_ptr[B];
   for (int j = blockIdx.x; j < M; j += gridDim.x) {  // grid-stride over the live rows (uniform per block)
-  if (zero_out) clear_row(zero_out + (size_t)j * zcols, zcols);
   const size_t row = idx ? (size_t)idx[j] : (size_t)j;
   const Tin* x = X + row * d;
   float ss = 0.f;
@@ -264,12 +268,14 @@ __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict_
                                                           const int32_t* __restrict__ seg_ptr, int B, int Mcap,
                                                           const Tg* __restrict__ g, float eps, int d,
                                                           Tout* __restrict__ out, Tout* __restrict__ out_lo,
-                                                          float* __restrict__ res_out, float* __restrict__ zero_out,
-                                                          int zcols) {
+                                                          float* __restrict__ res_out, int* __restrict__ zero_ints,
+                                                          int nzero) {
   constexpr int E = Vec16<Tin>::E;
   __shared__ float sh[33];
   pdl_wait();
   pdl_trigger();
+  if (zero_ints)
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < nzero; i += gridDim.x * blockDim.x) zero_ints[i] = 0;
   // M, the gains and the first row are loaded without waiting for one another
   const int M = seg_ptr[B];
   const int nvec = d / E;
@@ -303,8 +309,7 @@ __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict_
       }
       if (j >= M) return;
     }
-    if (zero_out) clear_row(zero_out + (size_t)j * zcols, zcols);
-    float ss = 0.f;
+      float ss = 0.f;
 #pragma unroll
     for (int u = 0; u < NV; ++u) {
       if (threadIdx.x + u * 256 < nvec) {
@@ -342,13 +347,13 @@ __global__ void __launch_bounds__(256) rmsnorm_vec_kernel(const Tin* __restrict_
 template <typename Tin, typename Tg, typename Tout>
 static int launch_rmsnorm(const Tin* X, const int32_t* idx, const int32_t* seg, int B, int Mcap, const Tg* g,
                           float eps, int d, Tout* out, Tout* out_lo, int grid, cudaStream_t st,
-                          float* res_out = nullptr, float* zero_out = nullptr, int zcols = 0) {
+                          float* res_out = nullptr, int* zero_ints = nullptr, int nzero = 0) {
   constexpr int E = Vec16<Tin>::E;
   if (d % E == 0 && d <= 4 * 256 * E)
     return launch_pdl(rmsnorm_vec_kernel<Tin, Tg, Tout, 4>, dim3(grid), dim3(256), 0, st, X, idx, seg, B, Mcap, g,
-                      eps, d, out, out_lo, res_out, zero_out, zcols);
+                      eps, d, out, out_lo, res_out, zero_ints, nzero);
   return launch_pdl(rmsnorm_rows_kernel<Tin, Tg, Tout>, dim3(grid), dim3(256), 0, st, X, idx, seg, B, g, eps, d, out,
-                    out_lo, res_out, zero_out, zcols);
+                    out_lo, res_out, zero_ints, nzero);
 }
 
 // ---------------------------------------------------------------------------
@@ -662,17 +667,28 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   g.num_sms = L.num_sms;
   const int rgrid = std::min(Mcap, 2 * L.num_sms);  // finishing kernels: grid-stride over M rows
 
+  // the QKV and gate/up sums need no zeroing: the first piece of a tile stores, later pieces add
+  int* gsync = (int*)(ws + L.gsync);
+  int* arrive_qkv = gsync;
+  uint32_t* ready_qkv = (uint32_t*)(gsync + 8 * L.gsync_tiles[0]);
+  int* arrive_gu = gsync + 16 * L.gsync_tiles[0];
+  uint32_t* ready_gu = (uint32_t*)(arrive_gu + 8 * L.gsync_tiles[1]);
+
   trace_mark(0, st);
-  // x (fp32) staged in h32 takes the O projection's adds; the QKV sums start at 0
+  // x (fp32) staged in h32 takes the O projection's adds; the GEMMs' arrival counts start at 0
   PLK_TRY(launch_rmsnorm<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(X, idx, seg, B, Mcap, (const __nv_bfloat16*)w->g1,
                                                                       dm->eps, d, xn, xn_lo, rgrid, st, h32,
-                                                                      c32, d + 2 * dkv));
+                                                                      gsync, L.gsync_ints));
   trace_mark(1, st);
 
   g.K = d;
   g.ftiles = (d + 2 * dkv) / kGemmBM;
   g.gu_F = 0;
+  g.arrive = arrive_qkv;
+  g.ready = ready_qkv;
   PLK_TRY(launch_gemm_tc(tW_qkv, tX_xn[0], tX_xn[1], tO_qkv, g, st));
+  g.arrive = nullptr;  // the O projection adds into h
+  g.ready = nullptr;
   trace_mark(2, st);
 
   const float log2_theta = dm->rope_theta > 0.f ? log2f(dm->rope_theta) : 0.f;
@@ -691,14 +707,17 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   trace_mark(5, st);
 
   PLK_TRY(launch_rmsnorm<float, __nv_bfloat16, __nv_bfloat16>(h32, nullptr, seg, B, Mcap, (const __nv_bfloat16*)w->g2,
-                                                              dm->eps, d, hn, hn_lo, rgrid, st, nullptr, c32,
-                                                              2 * F));
+                                                              dm->eps, d, hn, hn_lo, rgrid, st));
   trace_mark(6, st);
 
   g.K = d;
   g.ftiles = F / 64;
   g.gu_F = F;
+  g.arrive = arrive_gu;
+  g.ready = ready_gu;
   PLK_TRY(launch_gemm_tc(tW_gu, tX_hn[0], tX_hn[1], tO_gu, g, st));
+  g.arrive = nullptr;  // the down projection adds into h
+  g.ready = nullptr;
   trace_mark(7, st);
 
   PLK_TRY(launch_pdl(finish_gu_kernel, dim3(rgrid), dim3(256), 0, st, (const float*)c32, seg, B, F, act, act_lo));
