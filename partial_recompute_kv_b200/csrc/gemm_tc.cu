@@ -74,18 +74,20 @@ static_assert((size_t)4 * 8 * kBlk * 4 <= kOffBar, "the last piece's blocks fit 
 constexpr int kGemmChainKB = 1 << 20;
 
 // bulk reduce-add of a [32 rows][32 fp32] smem block into the tensor at (x, y)
-__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* tm, int x, int y, const void* smem_src) {
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* tm, int x, int y, const void* smem_src,
+                                                  uint64_t policy) {
   asm volatile(
-      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+      "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group.L2::cache_hint [%0, {%1, %2}], [%3], %4;" ::"l"(
           reinterpret_cast<uint64_t>(tm)),
-      "r"(x), "r"(y), "r"(smem_u32(smem_src))
+      "r"(x), "r"(y), "r"(smem_u32(smem_src)), "l"(policy)
       : "memory");
 }
 // bulk store of a [32 rows][32 fp32] smem block into the tensor at (x, y)
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, int x, int y, const void* smem_src) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* tm, int x, int y, const void* smem_src,
+                                             uint64_t policy) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%1, %2}], [%3], %4;" ::"l"(
                    reinterpret_cast<uint64_t>(tm)),
-               "r"(x), "r"(y), "r"(smem_u32(smem_src))
+               "r"(x), "r"(y), "r"(smem_u32(smem_src)), "l"(policy)
                : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
@@ -203,6 +205,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer (both CTAs)
     if (elect_one()) {
+      // L2 policies: with a single token tile every weight tile is read by one pair only
+      // (streamed: evict first) and every pair reads the activations (evict last)
+      const uint64_t pol_w = ttiles == 1 ? l2_policy_evict_first() : l2_policy_evict_normal();
+      const uint64_t pol_x = ttiles == 1 ? l2_policy_evict_last() : l2_policy_evict_normal();
       // this CTA's 128 weight rows of tile t (gate/up tile: 64 gate rows, then the 64 up rows)
       const uint32_t lead_full0 = dsmem_addr(smem_u32(&full[0]), 0);
       auto load_a = [&](int stage, const TileGeom& t, int kb) {
@@ -210,8 +216,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int yA1 = args.gu_F ? args.gu_F + t.ft * 64 : t.ft * kGemmBM + 64;
         uint8_t* a = sA + stage * kStageA;
         const uint32_t fb = lead_full0 + (uint32_t)(stage * 8);
-        tma_load_2d_pair(a, &tmW, kb * kGemmBK, yA0, fb);
-        tma_load_2d_pair(a + 8192, &tmW, kb * kGemmBK, yA1, fb);
+        tma_load_2d_pair_hint(a, &tmW, kb * kGemmBK, yA0, fb, pol_w);
+        tma_load_2d_pair_hint(a + 8192, &tmW, kb * kGemmBK, yA1, fb, pol_w);
       };
       // bytes of one stage, both CTAs: 2 x (A rows + hi and lo of half of the token rows)
       auto stage_bytes = [](const TileGeom& t) {
@@ -252,9 +258,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           uint8_t* b = sB + stage * kStageB;
           uint8_t* blo = sBlo + stage * kStageB;
           for (int j = 0; j < nbox; ++j) {
-            tma_load_2d_pair(b + j * 8192, &tmX, kb * kGemmBK, trow + j * 64, lead_full0 + (uint32_t)(stage * 8));
-            tma_load_2d_pair(blo + j * 8192, &tmXlo, kb * kGemmBK, trow + j * 64,
-                             lead_full0 + (uint32_t)(stage * 8));
+            tma_load_2d_pair_hint(b + j * 8192, &tmX, kb * kGemmBK, trow + j * 64,
+                                  lead_full0 + (uint32_t)(stage * 8), pol_x);
+            tma_load_2d_pair_hint(blo + j * 8192, &tmXlo, kb * kGemmBK, trow + j * 64,
+                                  lead_full0 + (uint32_t)(stage * 8), pol_x);
           }
           ++issued;
           if (++stage == kGemmStages) {
@@ -329,6 +336,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;  // a warp reads TMEM lanes 32 * (warp % 4) ..
     const uint32_t lead_tempty0 = rank == 0 ? 0u : dsmem_addr(smem_u32(&tempty[0]), 0);
+    // the sums are read again soon (the finishing kernel, the next piece's adds): keep them in L2
+    // when the weights stream past them (a single token tile)
+    const uint64_t pol_out = ttiles == 1 ? l2_policy_evict_last() : l2_policy_evict_normal();
     SegWalk w(pair, npairs, tiles, KB);
     int u, kb0, kb1, j = 0, n = 0;
     while (w.next(u, kb0, kb1)) {
@@ -406,9 +416,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         __syncwarp();
         if (lane == 0) {
           if (store)
-            tma_store_2d(&tmOut, col, t.tok0 + c * 32, blk);
+            tma_store_2d(&tmOut, col, t.tok0 + c * 32, blk, pol_out);
           else
-            tma_reduce_add_2d(&tmOut, col, t.tok0 + c * 32, blk);
+            tma_reduce_add_2d(&tmOut, col, t.tok0 + c * 32, blk, pol_out);
           bulk_commit();
         }
       }
