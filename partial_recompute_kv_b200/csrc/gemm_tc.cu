@@ -23,19 +23,23 @@
 //    on the even CTA's stage barrier; one thread of warp 1 of the even CTA
 //    issues the pair MMAs; warps 2-5 of both CTAs drain their TMEM.
 //  * Persistent stream-K: each pair owns an equal, contiguous share of the
-//    (256-feature tile) x (k-block) iteration space and adds the fp32 partial
-//    of each tile piece it covers into the fp32 output with TMA bulk
-//    reduce-add (cp.reduce.async.bulk.tensor .add.f32), which the L2 applies
-//    atomically.  The output is the residual stream h (O and down projections)
-//    or an fp32 sums buffer that a finishing kernel turns into bf16 (QKV -> Q
-//    and the K/V cache rows; gate/up -> silu(g) u).  The sums buffer is not
-//    zeroed: a whole-tile piece stores its partial (TMA bulk store); in a split
-//    tile the piece whose warp arrives first stores and raises a ready flag once
-//    the store is complete, and the later pieces' warps wait for that flag (a
-//    bounded wait on a CTA that is already running and waits on nothing) before
-//    they add.  The order of the adds is not fixed: results may differ in the
-//    last fp32 bit between runs.  A tile piece accumulates its whole k range in
-//    TMEM before its one store or reduce-add.
+//    (256-feature tile) x (k-block) iteration space.  A tile piece
+//    accumulates its whole k range in TMEM, then goes into the fp32 output by
+//    TMA bulk store or bulk reduce-add (cp.reduce.async.bulk.tensor .add.f32,
+//    applied in the L2).  The output is the residual stream h (O and down
+//    projections: every piece adds, in the order the pieces arrive, so h may
+//    differ in the last fp32 bit between runs) or an fp32 sums buffer that a
+//    finishing kernel turns into bf16 (QKV -> Q and the K/V cache rows;
+//    gate/up -> silu(g) u), which is not zeroed: the piece of the last k range
+//    stores.  Into a sums buffer the pieces of a split tile land in a fixed
+//    order, last k range first (it is its pair's first piece, done early):
+//    each later piece waits (bounded) until the pieces of higher k have
+//    landed, a count per (tile, CTA, warp) that every piece but the first-k
+//    one raises once its bulk operation is complete.  A waiting pair waits
+//    only on pairs of higher index whose piece is their first, so no wait
+//    closes a cycle, and the sums are the same in every run.  (For the O and
+//    down projections, 16 tiles split 5-6 ways at 256 rows, such a chain
+//    costs ~18 us per launch.)
 //  * Two 256-column TMEM accumulators per CTA: the epilogue drains one tile
 //    piece while the MMA fills the next; the producers run ahead across
 //    pieces.
@@ -122,6 +126,21 @@ struct SegWalk {
     return true;
   }
   __device__ bool done() const { return i >= iend; }
+};
+
+// Order of the pieces of a split tile.  Pair c owns iterations [start(c), start(c + 1)),
+// start(c) = floor(c T / G); iteration x lies in the range of pair floor(((x + 1) G - 1) / T).
+// With T > G every range is nonempty and a tile's pieces belong to consecutive pairs; with
+// T <= G every nonempty range is one iteration, so every k-block of a tile is a piece.
+struct SplitPlan {
+  long long T;
+  int G, KB;
+  __device__ int pair_of(long long x) const { return (int)(((x + 1) * G - 1) / T); }
+  // pieces of tile u with a higher k range than the piece of `pair` starting at k-block kb0
+  __device__ int rank_from_tail(int u, int pair, int kb0) const {
+    if (T <= G) return KB - 1 - kb0;
+    return pair_of((long long)u * KB + KB - 1) - pair;
+  }
 };
 
 // Geometry of pair tile u as seen by CTA `rank` of the pair.
@@ -339,6 +358,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // the sums are read again soon (the finishing kernel, the next piece's adds): keep them in L2
     // when the weights stream past them (a single token tile)
     const uint64_t pol_out = ttiles == 1 ? l2_policy_evict_last() : l2_policy_evict_normal();
+    const SplitPlan plan{(long long)tiles * KB, npairs, KB};
     SegWalk w(pair, npairs, tiles, KB);
     int u, kb0, kb1, j = 0, n = 0;
     while (w.next(u, kb0, kb1)) {
@@ -356,33 +376,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                                 : t.ft * kGemmBM + q * 32;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * 256);
       const int nchunks = t.ncols >> 5;
-      // Into an output that starts undefined (args.arrive set), the piece of a tile that gets
-      // there first stores its partial and the later pieces add theirs once that store is
-      // complete (a per-(tile, CTA, warp) arrival count and ready flag); a whole tile is stored.
-      bool store = false;
-      uint32_t* ready = nullptr;
-      if (args.arrive) {
-        if (kb0 == 0 && kb1 == KB) {
-          store = true;
-        } else {
-          const int slot = (2 * u + rank) * 4 + q;
-          int old = 0;
-          if (lane == 0) old = atomicAdd(args.arrive + slot, 1);
-          old = __shfl_sync(0xffffffffu, old, 0);
-          ready = args.ready + slot;
-          store = old == 0;
-          if (!store) {
-            bool got = true;
-            if (lane == 0) {
-              got = spin_until_geq(ready, 1u);  // the first piece's CTA is running: bounded, short
-              fence_proxy_async_global();       // its stored values before this warp's bulk adds
-            }
-            if (!__all_sync(0xffffffffu, __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0)) {
-              if (lane == 0) *s_abort = 1;
-            }
-            ready = nullptr;
-          }
+      // The pieces of a split tile go into the output one after another in a fixed order, from
+      // the last k range (the tail, which is its pair's first piece and is done early) down to
+      // the first: the tail stores (an output that starts undefined) or adds, every other piece
+      // waits until the rho pieces of higher k have landed (a per-(tile, CTA, warp) count of the
+      // pieces done), then adds.  The fp32 sums therefore come out the same in every run.  A
+      // whole tile is one piece.
+      const int rho = plan.rank_from_tail(u, pair, kb0);
+      const bool store = args.store_first && kb1 == KB;
+      uint32_t* done = (args.done && kb0 > 0) ? args.done + ((2 * u + rank) * 4 + q) : nullptr;  // not the head
+      if (args.done && rho > 0) {
+        bool got = true;
+        if (lane == 0) {
+          got = spin_until_geq(args.done + ((2 * u + rank) * 4 + q), (uint32_t)rho);  // bounded; see above
+          fence_proxy_async_global();  // the landed pieces before this warp's bulk adds
         }
+        if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0 && lane == 0) *s_abort = 1;
       }
       for (int c = 0; c < nchunks; ++c) {
         float* blk;
@@ -422,11 +431,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           bulk_commit();
         }
       }
-      if (ready) {  // first piece of a split tile: its store is complete, the others may add
+      if (done) {  // every piece but the head: landed, the next lower k range may add
         if (lane == 0) {
           bulk_wait_all();
           fence_proxy_async_global();
-          red_release_add_u32(ready, 1u);
+          red_release_add_u32(done, 1u);
         }
         __syncwarp();
       }

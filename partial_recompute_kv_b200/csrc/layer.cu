@@ -78,11 +78,11 @@ Workspace workspace_layout(const plk_dims* dm, int num_sms) {
   w.c32_bytes = 4 * Mcap * std::max(d + 2 * (size_t)kv_width(dm), 2 * F);
   w.c32 = take(w.c32_bytes);
   if (dm->dtype == PLK_BF16) {
-    // arrival counts and ready flags of the QKV and gate/up GEMMs: 8 per pair tile each
+    // pieces-done counts of the QKV and gate/up GEMMs: 8 per pair tile
     const size_t tt = (Mcap + kGemmBNMax - 1) / kGemmBNMax;
     w.gsync_tiles[0] = (int)(((d + 2 * (size_t)kv_width(dm)) / 256) * tt);
     w.gsync_tiles[1] = (int)((F / 128) * tt);
-    w.gsync_ints = 16 * (w.gsync_tiles[0] + w.gsync_tiles[1]);
+    w.gsync_ints = 8 * (w.gsync_tiles[0] + w.gsync_tiles[1]);
     w.gsync = take(4 * (size_t)w.gsync_ints);
   }
   w.total = off;
@@ -667,15 +667,15 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   g.num_sms = L.num_sms;
   const int rgrid = std::min(Mcap, 2 * L.num_sms);  // finishing kernels: grid-stride over M rows
 
-  // the QKV and gate/up sums need no zeroing: the first piece of a tile stores, later pieces add
+  // in the QKV and gate/up GEMMs the pieces of a split tile land in a fixed order, counted per
+  // (tile, CTA, warp), and their sums need no zeroing: the last k range's piece stores, the
+  // others add
   int* gsync = (int*)(ws + L.gsync);
-  int* arrive_qkv = gsync;
-  uint32_t* ready_qkv = (uint32_t*)(gsync + 8 * L.gsync_tiles[0]);
-  int* arrive_gu = gsync + 16 * L.gsync_tiles[0];
-  uint32_t* ready_gu = (uint32_t*)(arrive_gu + 8 * L.gsync_tiles[1]);
+  uint32_t* done_qkv = (uint32_t*)gsync;
+  uint32_t* done_gu = done_qkv + 8 * L.gsync_tiles[0];
 
   trace_mark(0, st);
-  // x (fp32) staged in h32 takes the O projection's adds; the GEMMs' arrival counts start at 0
+  // x (fp32) staged in h32 takes the O projection's adds; the GEMMs' pieces-done counts start at 0
   PLK_TRY(launch_rmsnorm<__nv_bfloat16, __nv_bfloat16, __nv_bfloat16>(X, idx, seg, B, Mcap, (const __nv_bfloat16*)w->g1,
                                                                       dm->eps, d, xn, xn_lo, rgrid, st, h32,
                                                                       gsync, L.gsync_ints));
@@ -684,11 +684,9 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   g.K = d;
   g.ftiles = (d + 2 * dkv) / kGemmBM;
   g.gu_F = 0;
-  g.arrive = arrive_qkv;
-  g.ready = ready_qkv;
+  g.done = done_qkv;
+  g.store_first = 1;
   PLK_TRY(launch_gemm_tc(tW_qkv, tX_xn[0], tX_xn[1], tO_qkv, g, st));
-  g.arrive = nullptr;  // the O projection adds into h
-  g.ready = nullptr;
   trace_mark(2, st);
 
   const float log2_theta = dm->rope_theta > 0.f ? log2f(dm->rope_theta) : 0.f;
@@ -703,7 +701,11 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
 
   g.K = d;
   g.ftiles = d / kGemmBM;
-  PLK_TRY(launch_gemm_tc(tW_o, tX_a[0], tX_a[1], tO_h, g, st));  // h = x + a W_o^T
+  // h = x + a W_o^T: 16 tiles split 5-6 ways at 256 rows, where an ordered chain of their
+  // pieces costs ~18 us; the pieces add in the order they arrive
+  g.done = nullptr;
+  g.store_first = 0;
+  PLK_TRY(launch_gemm_tc(tW_o, tX_a[0], tX_a[1], tO_h, g, st));
   trace_mark(5, st);
 
   PLK_TRY(launch_rmsnorm<float, __nv_bfloat16, __nv_bfloat16>(h32, nullptr, seg, B, Mcap, (const __nv_bfloat16*)w->g2,
@@ -713,11 +715,9 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   g.K = d;
   g.ftiles = F / 64;
   g.gu_F = F;
-  g.arrive = arrive_gu;
-  g.ready = ready_gu;
+  g.done = done_gu;
+  g.store_first = 1;
   PLK_TRY(launch_gemm_tc(tW_gu, tX_hn[0], tX_hn[1], tO_gu, g, st));
-  g.arrive = nullptr;  // the down projection adds into h
-  g.ready = nullptr;
   trace_mark(7, st);
 
   PLK_TRY(launch_pdl(finish_gu_kernel, dim3(rgrid), dim3(256), 0, st, (const float*)c32, seg, B, F, act, act_lo));
@@ -726,7 +726,9 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   g.K = F;
   g.ftiles = d / kGemmBM;
   g.gu_F = 0;
-  PLK_TRY(launch_gemm_tc(tW_down, tX_act[0], tX_act[1], tO_h, g, st));  // y = h + act W_down^T
+  g.done = nullptr;  // y = h + act W_down^T, pieces in arrival order as for O
+  g.store_first = 0;
+  PLK_TRY(launch_gemm_tc(tW_down, tX_act[0], tX_act[1], tO_h, g, st));
   trace_mark(9, st);
 
   PLK_TRY(launch_pdl(finish_y_kernel, dim3(rgrid), dim3(256), 0, st, (const float*)h32, idx, seg, B, d,

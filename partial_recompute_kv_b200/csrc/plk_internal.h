@@ -59,8 +59,8 @@ struct Workspace {
   size_t c32 = 0;                        // fp32 GEMM sums [Mcap, max(d + 2 dkv, 2F)] (QKV, then gate/up;
                                          // in between, the attention's partial outputs)
   size_t c32_bytes = 0;
-  // bf16 path: arrival counts then ready flags ([8 x tiles] each) of the QKV GEMM, then those
-  // of the gate/up GEMM; cleared by RMSNorm1 at every step
+  // bf16 path: the pieces-done counts ([8 x tiles]) of the QKV and gate/up GEMMs in turn,
+  // cleared by RMSNorm1 at every step
   size_t gsync = 0;
   int gsync_ints = 0;
   int gsync_tiles[2] = {0, 0};
@@ -111,10 +111,10 @@ struct GemmArgs {
   const int32_t* seg_ptr;  // M = seg_ptr[B]
   int B;
   int num_sms;             // SM count: at most one persistent CTA per SM, in pairs
-  // Output that starts undefined (nullptr: the output holds values the GEMM adds to): per
-  // (pair tile, CTA, epilogue warp) arrival counts and ready flags, [tiles * 8] each, zero.
-  int* arrive = nullptr;
-  uint32_t* ready = nullptr;
+  // Per (pair tile, CTA, epilogue warp): the count of the tile's pieces that have landed in the
+  // output, [tiles * 8], zero on entry (nullptr: one piece per tile only, e.g. no split).
+  uint32_t* done = nullptr;
+  int store_first = 0;     // 1: the output starts undefined, the tail piece stores; 0: every piece adds
 };
 int launch_gemm_tc(const CUtensorMap& tmW, const CUtensorMap& tmXhi, const CUtensorMap& tmXlo,
                    const CUtensorMap& tmOut, const GemmArgs& a, cudaStream_t st);

@@ -475,6 +475,26 @@ def test_layer_8b_full_step(plk, layer_8b):
         assert_bf16_close(g, o, f"8B full step {name}")
 
 
+@pytest.mark.parametrize("frac", [0.25, 0.05])
+def test_layer_8b_kv_are_deterministic(plk, layer_8b, frac):
+    """The QKV projection lands the pieces of a split tile in a fixed order (at M = 256 its tiles
+    split over 2-3 CTA pairs): identical calls give bit-identical K and V.  The O and down
+    projections add their pieces into the residual stream in arrival order, so Y agrees up to the
+    last bits."""
+    D, base = layer_8b["D"], layer_8b["base"]
+    pos = synth.layer_8b_positions(D.N, frac)
+    lock = np.ones((1, D.N), np.uint8)
+    lock[0, pos] = 0
+    idx, seg = oracle.compact(lock)
+    X2 = synth.perturb_rows(layer_8b["X"], synth.step_noise((1, D.N, D.d), 0.01), lock == 0, "bf16")
+    runs = [_run_layer_guarded(plk, D, layer_8b["Wd"], X2, idx, seg, base, what=f"8B M/N={frac} run {i}")
+            for i in range(3)]
+    for r in runs[1:]:
+        for a, b, name in zip(runs[0][:2], r[:2], "KV"):
+            assert np.array_equal(a, b), f"8B M/N={frac}: {name} differs between identical calls"
+        assert_bf16_close(r[2], runs[0][2], f"8B M/N={frac}: Y of identical calls")
+
+
 @pytest.mark.parametrize("frac", synth.LAYER_8B_FRACTIONS)
 def test_layer_8b_fraction(plk, layer_8b, frac, record_property):
     """Partial step from the full step's caches with the active rows perturbed: all M active rows of
