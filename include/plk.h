@@ -330,6 +330,16 @@ int plk_get_status(void* stream);
  * about two seconds).  Values < 1 are rejected. */
 int plk_set_wait_limit(long long cycles);
 
+/* Reproducible mode for the bf16 layer step (host-side setting, process-wide;
+ * default off).  Off: the O and down projections add the pieces of a split tile
+ * into the residual stream in the order they arrive, so h and Y may differ in
+ * the last bits between runs (q, K, V and the SwiGLU input never do).  On: those
+ * pieces land in a fixed order too, and every output of plk_layer_step_partial,
+ * plk_full_layer_step and plk_denoise_step_host is bit-reproducible for the same
+ * inputs on the same GPU model, at ~35 us more per step at the 8B shape with 256
+ * rows (the pieces of a tile wait for one another).  on is 0 or 1. */
+int plk_set_deterministic(int on);
+
 /* Launches one block that waits on a device flag nothing ever sets, bounded by
  * the current wait limit; the wait then records PLK_ERR_TIMEOUT in the status
  * word.  Exists to test the timeout path without faulting or hanging a GPU. */

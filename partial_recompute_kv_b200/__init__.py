@@ -28,7 +28,7 @@ EXPORTED = (
     "plk_proxy_commit", "plk_layer_step_partial_static", "plk_kl_lock", "plk_slowfast_step", "plk_workspace_bytes",
     "plk_denoise_step_host", "plk_step_workspace_bytes",
     "plk_get_status",
-    "plk_set_wait_limit",
+    "plk_set_wait_limit", "plk_set_deterministic",
     "plk_selftest_wait_timeout", "plk_selftest_exp2", "plk_trace_events", "plk_error_string", "plk_version",
 )
 
@@ -80,6 +80,7 @@ def _load():
         "plk_step_workspace_bytes": (S, [V, I]),
         "plk_get_status": (I, [P]),
         "plk_set_wait_limit": (I, [L]),
+        "plk_set_deterministic": (I, [I]),
         "plk_selftest_wait_timeout": (I, [P]),
         "plk_selftest_exp2": (I, [P, P, I, P]),
         "plk_trace_events": (I, [ctypes.POINTER(ctypes.c_void_p), I]),
@@ -260,6 +261,10 @@ def get_status(stream=None) -> int:
 
 def set_wait_limit(cycles: int):
     _check(lib.plk_set_wait_limit(int(cycles)), "set_wait_limit")
+
+
+def set_deterministic(on: bool):
+    _check(lib.plk_set_deterministic(1 if on else 0), "set_deterministic")
 
 
 def trace_events(events):

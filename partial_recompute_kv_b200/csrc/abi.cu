@@ -234,6 +234,12 @@ int plk_trace_events(void* const* events, int n) {
   return PLK_OK;
 }
 
+int plk_set_deterministic(int on) {
+  if (on != 0 && on != 1) return PLK_ERR_ARG;
+  g_deterministic = on;
+  return PLK_OK;
+}
+
 int plk_set_wait_limit(long long cycles) {
   if (cycles < 1) return PLK_ERR_ARG;
   return cudaMemcpyToSymbol(g_wait_limit, &cycles, sizeof(cycles)) == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;

@@ -37,6 +37,7 @@ namespace plk {
 // events registered by plk_trace_events, recorded between the step's kernels
 cudaEvent_t g_trace[16];
 int g_ntrace = 0;
+int g_deterministic = 0;
 static inline void trace_mark(int i, cudaStream_t st) {
   if (i < g_ntrace && g_trace[i]) cudaEventRecord(g_trace[i], st);
 }
@@ -78,11 +79,13 @@ Workspace workspace_layout(const plk_dims* dm, int num_sms) {
   w.c32_bytes = 4 * Mcap * std::max(d + 2 * (size_t)kv_width(dm), 2 * F);
   w.c32 = take(w.c32_bytes);
   if (dm->dtype == PLK_BF16) {
-    // pieces-done counts of the QKV and gate/up GEMMs: 8 per pair tile
+    // pieces-done counts of the QKV, O, gate/up and down GEMMs: 8 per pair tile
     const size_t tt = (Mcap + kGemmBNMax - 1) / kGemmBNMax;
     w.gsync_tiles[0] = (int)(((d + 2 * (size_t)kv_width(dm)) / 256) * tt);
-    w.gsync_tiles[1] = (int)((F / 128) * tt);
-    w.gsync_ints = 8 * (w.gsync_tiles[0] + w.gsync_tiles[1]);
+    w.gsync_tiles[1] = (int)((d / 256) * tt);
+    w.gsync_tiles[2] = (int)((F / 128) * tt);
+    w.gsync_tiles[3] = (int)((d / 256) * tt);
+    w.gsync_ints = 8 * (w.gsync_tiles[0] + w.gsync_tiles[1] + w.gsync_tiles[2] + w.gsync_tiles[3]);
     w.gsync = take(4 * (size_t)w.gsync_ints);
   }
   w.total = off;
@@ -672,7 +675,9 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   // others add
   int* gsync = (int*)(ws + L.gsync);
   uint32_t* done_qkv = (uint32_t*)gsync;
-  uint32_t* done_gu = done_qkv + 8 * L.gsync_tiles[0];
+  uint32_t* done_o = done_qkv + 8 * L.gsync_tiles[0];
+  uint32_t* done_gu = done_o + 8 * L.gsync_tiles[1];
+  uint32_t* done_down = done_gu + 8 * L.gsync_tiles[2];
 
   trace_mark(0, st);
   // x (fp32) staged in h32 takes the O projection's adds; the GEMMs' pieces-done counts start at 0
@@ -702,8 +707,8 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   g.K = d;
   g.ftiles = d / kGemmBM;
   // h = x + a W_o^T: 16 tiles split 5-6 ways at 256 rows, where an ordered chain of their
-  // pieces costs ~18 us; the pieces add in the order they arrive
-  g.done = nullptr;
+  // pieces costs ~18 us; the pieces add in the order they arrive unless reproducible mode is on
+  g.done = g_deterministic ? done_o : nullptr;
   g.store_first = 0;
   PLK_TRY(launch_gemm_tc(tW_o, tX_a[0], tX_a[1], tO_h, g, st));
   trace_mark(5, st);
@@ -726,7 +731,7 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   g.K = F;
   g.ftiles = d / kGemmBM;
   g.gu_F = 0;
-  g.done = nullptr;  // y = h + act W_down^T, pieces in arrival order as for O
+  g.done = g_deterministic ? done_down : nullptr;  // y = h + act W_down^T, as for O
   g.store_first = 0;
   PLK_TRY(launch_gemm_tc(tW_down, tX_act[0], tX_act[1], tO_h, g, st));
   trace_mark(9, st);

@@ -59,14 +59,16 @@ struct Workspace {
   size_t c32 = 0;                        // fp32 GEMM sums [Mcap, max(d + 2 dkv, 2F)] (QKV, then gate/up;
                                          // in between, the attention's partial outputs)
   size_t c32_bytes = 0;
-  // bf16 path: the pieces-done counts ([8 x tiles]) of the QKV and gate/up GEMMs in turn,
-  // cleared by RMSNorm1 at every step
+  // bf16 path: the pieces-done counts ([8 x tiles]) of the QKV, O, gate/up and down GEMMs in
+  // turn (O and down used in reproducible mode only), cleared by RMSNorm1 at every step
   size_t gsync = 0;
   int gsync_ints = 0;
-  int gsync_tiles[2] = {0, 0};
+  int gsync_tiles[4] = {0, 0, 0, 0};
   int num_sms = 0;
 };
 Workspace workspace_layout(const plk_dims* d, int num_sms);
+// plk_set_deterministic: the O and down projections land split-tile pieces in a fixed order too
+extern int g_deterministic;
 int device_sm_count();
 
 // ---- TMA descriptors ---------------------------------------------------------

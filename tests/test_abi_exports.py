@@ -74,6 +74,8 @@ def test_host_validation_without_gpu(built):
     assert lib.plk_score_drift(ctypes.byref(ok), p, p, 8, p, 5, None, p, None) == plk.ERR_ARG
     assert lib.plk_score_drift(ctypes.byref(ok), p, p, 8, p, 0, p, p, None) == plk.ERR_ARG  # out aliases cache
     assert lib.plk_set_wait_limit(0) == plk.ERR_ARG
+    assert lib.plk_set_deterministic(2) == plk.ERR_ARG
+    assert lib.plk_set_deterministic(0) == plk.OK
     assert lib.plk_proxy_commit(ctypes.byref(ok), 0, p, p, p, p, None) == plk.ERR_ARG
     # SlowFast policy: bad params, shapes and aliasing are refused before any launch
     q = ctypes.c_void_p(32)

@@ -495,6 +495,29 @@ def test_layer_8b_kv_are_deterministic(plk, layer_8b, frac):
         assert_bf16_close(r[2], runs[0][2], f"8B M/N={frac}: Y of identical calls")
 
 
+def test_layer_8b_reproducible_mode(plk, layer_8b):
+    """plk_set_deterministic(1): the O and down projections land their split-tile pieces in a
+    fixed order too, so identical calls give bit-identical K, V and Y; the outputs still meet the
+    oracle."""
+    D, W, base = layer_8b["D"], layer_8b["W"], layer_8b["base"]
+    pos = synth.layer_8b_positions(D.N, 0.25)
+    lock = np.ones((1, D.N), np.uint8)
+    lock[0, pos] = 0
+    idx, seg = oracle.compact(lock)
+    X2 = synth.perturb_rows(layer_8b["X"], synth.step_noise((1, D.N, D.d), 0.01), lock == 0, "bf16")
+    plk.set_deterministic(True)
+    try:
+        runs = [_run_layer_guarded(plk, D, layer_8b["Wd"], X2, idx, seg, base, what=f"8B reproducible run {i}")
+                for i in range(3)]
+    finally:
+        plk.set_deterministic(False)
+    for r in runs[1:]:
+        for a, b, name in zip(runs[0], r, "KVY"):
+            assert np.array_equal(a, b), f"reproducible mode: {name} differs between identical calls"
+    ref = oracle.layer_step_partial(D, W, X2, idx, seg, base, "bf16")
+    _check_layer_rows(*runs[0], ref, base, lock, "8B reproducible mode")
+
+
 @pytest.mark.parametrize("frac", synth.LAYER_8B_FRACTIONS)
 def test_layer_8b_fraction(plk, layer_8b, frac, record_property):
     """Partial step from the full step's caches with the active rows perturbed: all M active rows of
