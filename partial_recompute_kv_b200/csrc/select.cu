@@ -326,7 +326,7 @@ __device__ __forceinline__ int cluster_sum(const int* p, int S, int upto) {
 
 constexpr int kSelClusterThreads = 256;
 
-template <int KPT, int NT>
+template <int KPT, int NT, bool CL>
 __global__ void __launch_bounds__(NT) topk_cluster_kernel(const float* __restrict__ score,
                                                                           const uint8_t* lock_in, uint8_t* lock_out,
                                                                           int N, int k, int largest, int direct,
@@ -341,7 +341,7 @@ __global__ void __launch_bounds__(NT) topk_cluster_kernel(const float* __restric
   pdl_wait();
   pdl_trigger();
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int s = (int)cluster_ctarank();
+  const int s = CL ? (int)cluster_ctarank() : 0;
   const int b = blockIdx.y;
   const long long base = (long long)b * N;
   const int L = (N + S - 1) / S;
@@ -366,8 +366,13 @@ __global__ void __launch_bounds__(NT) topk_cluster_kernel(const float* __restric
 #pragma unroll
     for (int j = 0; j < KPT; ++j)
       if (cand[j] && (key[j] & pmask) == prefix) atomicAdd(&hb[(key[j] >> shift) & 255u], 1);
-    cluster_sync_all();  // every CTA's histogram of this pass is complete
-    if (t < 256) gh[t] = cluster_sum(&hb[t], S, S);
+    if (CL) {
+      cluster_sync_all();  // every CTA's histogram of this pass is complete
+      if (t < 256) gh[t] = cluster_sum(&hb[t], S, S);
+    } else {
+      __syncthreads();
+      if (t < 256) gh[t] = hb[t];
+    }
     __syncthreads();
     if (pass == 0) {  // every candidate is in the first pass's histogram
       if (warp == 0) {
@@ -435,15 +440,18 @@ __global__ void __launch_bounds__(NT) topk_cluster_kernel(const float* __restric
     pub[0] = gtc;
     pub[1] = eqc;
   }
-  cluster_sync_all();
+  if (CL)
+    cluster_sync_all();
+  else
+    __syncthreads();
   // kept rows of CTA r: its sure rows plus its share of the ties, taken in rank order
   int before = 0, all = 0, eq_before = 0;
   {
     int gv[8], ev[8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
-      gv[r] = ld_dsmem_s32(&pub[0], (uint32_t)(r < S ? r : 0));
-      ev[r] = ld_dsmem_s32(&pub[1], (uint32_t)(r < S ? r : 0));
+      gv[r] = CL ? ld_dsmem_s32(&pub[0], (uint32_t)(r < S ? r : 0)) : pub[0];
+      ev[r] = CL ? ld_dsmem_s32(&pub[1], (uint32_t)(r < S ? r : 0)) : pub[1];
     }
     int taken = 0;
 #pragma unroll
@@ -485,7 +493,7 @@ __global__ void __launch_bounds__(NT) topk_cluster_kernel(const float* __restric
       seg_ptr[b + 1] = -(all + 1);
     }
   }
-  cluster_sync_all();  // no CTA leaves while another can still read its shared memory
+  if (CL) cluster_sync_all();  // no CTA leaves while another can still read its shared memory
 }
 
 int launch_select(const plk_dims* dims, const float* score, const uint8_t* lock_in, uint8_t* lock_out,
@@ -495,13 +503,19 @@ int launch_select(const plk_dims* dims, const float* score, const uint8_t* lock_
   int e;
   const int largest = (int)(mode == PLK_SEL_TOPK_LARGEST);
   const bool topk = mode == PLK_SEL_TOPK_LARGEST || mode == PLK_SEL_TOPK_SMALLEST;
-  // sequences of more than 2048 rows: keys in registers on a cluster of S CTAs of
-  // 256 threads (512 rows each and more, at most 4096 each); shorter ones (and
-  // longer than 8 x 4096) on one CTA of 1024 threads, which is faster there
+  // keys in registers: sequences of up to 2048 rows on one CTA of 1024 threads, longer
+  // ones on a cluster of S CTAs of 256 threads (512 rows each and more, at most 4096
+  // each); longer than 8 x 4096 rows: the one-CTA kernel that reads the scores per pass
   const int S = std::min(8, ceil_div(N, 512));
   const int NT = kSelClusterThreads;
   const int kpt = ceil_div(ceil_div(N, S), NT);
-  if (topk && N > 2048 && kpt <= 16) {
+  if (topk && N <= kSelThreads) {
+    e = launch_pdl(topk_cluster_kernel<1, kSelThreads, false>, dim3(1, B), dim3(kSelThreads), 0, st, score,
+                   lock_in, lock_out, N, k, largest, direct, 1, idx_out, seg_ptr);
+  } else if (topk && N <= 2 * kSelThreads) {
+    e = launch_pdl(topk_cluster_kernel<2, kSelThreads, false>, dim3(1, B), dim3(kSelThreads), 0, st, score,
+                   lock_in, lock_out, N, k, largest, direct, 1, idx_out, seg_ptr);
+  } else if (topk && kpt <= 16) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)S, (unsigned)B, 1);
     cfg.blockDim = dim3((unsigned)NT, 1, 1);
@@ -516,9 +530,9 @@ int launch_select(const plk_dims* dims, const float* score, const uint8_t* lock_
     cfg.attrs = at;
     cfg.numAttrs = 2;
     cudaError_t ce;
-#define PLK_TOPK_LAUNCH(KPT_, NT_)                                                                            \
-  ce = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<KPT_, NT_>, score, lock_in, lock_out, N, k, largest, direct, S, \
-                          idx_out, seg_ptr)
+#define PLK_TOPK_LAUNCH(KPT_, NT_)                                                                        \
+  ce = cudaLaunchKernelEx(&cfg, topk_cluster_kernel<KPT_, NT_, true>, score, lock_in, lock_out, N, k, largest, \
+                          direct, S, idx_out, seg_ptr)
     if (kpt <= 2)
       PLK_TOPK_LAUNCH(2, kSelClusterThreads);
     else if (kpt <= 4)
