@@ -103,6 +103,14 @@ __device__ __forceinline__ float exp2_fma(float t) {
 }
 // every kAttPolyEvery-th exponential of a thread's chunk row goes to exp2_fma
 constexpr int kAttPolyEvery = 4;
+// 2^t by the MUFU unit's approximate ex2 alone (PTX ex2.approx.ftz.f32: relative error about
+// 2^-22, subnormal results flushed to 0), for the softmax weights: they are stored with ~16
+// significant bits and weights below 2^-126 do not matter.
+__device__ __forceinline__ float exp2_mufu(float t) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(t));
+  return r;
+}
 
 // hi = bf16(x) packed, lo = bf16(x - hi) packed
 __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uint32_t& lo) {
@@ -568,8 +576,8 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
           for (int e = 0; e < 4; ++e) {
             const int i0 = cc * 8 + 2 * e, i1 = i0 + 1;
             const float t0 = fmaf(sc[i0], scale_log2, -m_used), t1 = fmaf(sc[i1], scale_log2, -m_used);
-            const float p0 = (i0 % kAttPolyEvery == kAttPolyEvery - 1) ? exp2_fma(t0) : exp2f(t0);
-            const float p1 = (i1 % kAttPolyEvery == kAttPolyEvery - 1) ? exp2_fma(t1) : exp2f(t1);
+            const float p0 = (i0 % kAttPolyEvery == kAttPolyEvery - 1) ? exp2_fma(t0) : exp2_mufu(t0);
+            const float p1 = (i1 % kAttPolyEvery == kAttPolyEvery - 1) ? exp2_fma(t1) : exp2_mufu(t1);
             l += p0 + p1;
             split_pair_trunc(p0, p1, hi[e], lo[e]);
           }
