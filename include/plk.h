@@ -345,10 +345,11 @@ int plk_set_deterministic(int on);
  * word.  Exists to test the timeout path without faulting or hanging a GPU. */
 int plk_selftest_wait_timeout(void* stream);
 
-/* out[i] = 2^t[i] (n values, device pointers) by the exponential the attention
- * softmax computes on the FMA pipe for part of its weights (range reduction to
+/* out[i] = 2^t[i] (n values, device pointers) by the FMA-pipe exponential the
+ * attention softmax can compute for a share of its weights (range reduction to
  * [-1/2, 1/2] and a degree-4 minimax polynomial; relative error <= 3e-6; t < -126
- * gives 0).  Exists so that the polynomial can be tested against exp2 on a GPU. */
+ * gives 0; the build gives it no share: the MUFU ex2 alone measured faster).
+ * Exists so that the polynomial can be tested against exp2 on a GPU. */
 int plk_selftest_exp2(const float* t, float* out, int n, void* stream);
 
 /* Tracing.  Registers up to 16 cudaEvent_t handles (passed as void*).  While

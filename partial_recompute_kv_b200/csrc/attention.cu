@@ -101,8 +101,11 @@ __device__ __forceinline__ float exp2_fma(float t) {
   const float r = __int_as_float(__float_as_int(p) + (__float_as_int(j) << 23));
   return t >= -126.0f ? r : 0.0f;
 }
-// every kAttPolyEvery-th exponential of a thread's chunk row goes to exp2_fma
-constexpr int kAttPolyEvery = 4;
+// every kAttPolyEvery-th exponential of a thread's chunk row goes to exp2_fma (0: none).  With
+// the MUFU path a bare ex2 instruction (exp2_mufu) the FMA share no longer pays: at 1024 keys
+// the kernel took 21.4 us with every 4th exponential on the FMA pipe, 20.8 with every 8th and
+// 20.5 with none (52.3 against 54.8 us at 8192 keys).
+constexpr int kAttPolyEvery = 0;
 // 2^t by the MUFU unit's approximate ex2 alone (PTX ex2.approx.ftz.f32: relative error about
 // 2^-22, subnormal results flushed to 0), for the softmax weights: they are stored with ~16
 // significant bits and weights below 2^-126 do not matter.
@@ -576,8 +579,10 @@ __global__ void __launch_bounds__(kAttThreads, 1) attn_tc_kernel(const __grid_co
           for (int e = 0; e < 4; ++e) {
             const int i0 = cc * 8 + 2 * e, i1 = i0 + 1;
             const float t0 = fmaf(sc[i0], scale_log2, -m_used), t1 = fmaf(sc[i1], scale_log2, -m_used);
-            const float p0 = (i0 % kAttPolyEvery == kAttPolyEvery - 1) ? exp2_fma(t0) : exp2_mufu(t0);
-            const float p1 = (i1 % kAttPolyEvery == kAttPolyEvery - 1) ? exp2_fma(t1) : exp2_mufu(t1);
+            const bool f0 = kAttPolyEvery > 0 && i0 % (kAttPolyEvery > 0 ? kAttPolyEvery : 1) == kAttPolyEvery - 1;
+            const bool f1 = kAttPolyEvery > 0 && i1 % (kAttPolyEvery > 0 ? kAttPolyEvery : 1) == kAttPolyEvery - 1;
+            const float p0 = f0 ? exp2_fma(t0) : exp2_mufu(t0);
+            const float p1 = f1 ? exp2_fma(t1) : exp2_mufu(t1);
             l += p0 + p1;
             split_pair_trunc(p0, p1, hi[e], lo[e]);
           }
