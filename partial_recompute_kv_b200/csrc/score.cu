@@ -190,12 +190,21 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
             "r"(dsmem_addr(smem_u32(slices), (uint32_t)q))
             : "memory");
     }
-    const bool landed = mbar_wait(slices, 0);
     const int lrow = (int)threadIdx.x / tpr, sub = (int)threadIdx.x % tpr;
     const int row = row0 + ks * rows_per + lrow;
     const int krow = ks * rows_per + lrow;  // the row's index in its sender's block (swizzle key)
+    // the cached proxies of this thread's first 4 column groups, loaded while the slices travel
+    float4 cpre[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = sub * 4 + i * 4 * tpr;
+      cpre[i] = (c < r && row < rows) ? __ldg(reinterpret_cast<const float4*>(cache + (size_t)row * r + c))
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    const bool landed = mbar_wait(slices, 0);
     float dot = 0.f, pp = 0.f, cc = 0.f, dd = 0.f;
-    for (int c = sub * 4; c < r && landed; c += 4 * tpr) {
+    int ci = 0;
+    for (int c = sub * 4; c < r && landed; c += 4 * tpr, ++ci) {
       float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int sr = 0; sr < S; ++sr) {
         const float4 x = reinterpret_cast<const float4*>(slots + ((size_t)sr * rows_per + lrow) * r)[(c / 4) ^ (krow & swz)];
@@ -205,7 +214,11 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
         p.w += x.w;
       }
       if (row < rows) {
-        const float4 cv = __ldg(reinterpret_cast<const float4*>(cache + (size_t)row * r + c));
+        const float4 cv = ci == 0   ? cpre[0]
+                          : ci == 1 ? cpre[1]
+                          : ci == 2 ? cpre[2]
+                          : ci == 3 ? cpre[3]
+                                    : __ldg(reinterpret_cast<const float4*>(cache + (size_t)row * r + c));
         const float pv[4] = {p.x, p.y, p.z, p.w};
         const float cvv[4] = {cv.x, cv.y, cv.z, cv.w};
 #pragma unroll
