@@ -309,14 +309,15 @@ def run_gpu(args, wl, dist, rank, world, local_rank):
     pc0 = pnew.clone()
     pc.copy_(pc0)
 
-    def step(xin):
-        plk.score_drift(dm, xin, Ut, r, pc, plk.METRIC_L2, score, proxy_out=pnew)
-        plk.select_active(dm, score, lock_in, lock, plk.SEL_TOPK_LARGEST, 0.0, M, idx, seg)
-        plk.layer_step_partial(dm, pw, xin, idx, seg, K, V, Y, ws)
-        plk.proxy_commit(dm, r, idx, seg, pnew, pc)
+    sws = plk.alloc_step_workspace(dm, r, device=dev)
+    lock_s = torch.zeros_like(lock_in)  # the whole-step call locks in place
+
+    def step(xin):  # one call: score, select, layer step with the proxy refresh folded in
+        plk.denoise_step(dm, pw, Ut, r, plk.METRIC_L2, plk.SEL_TOPK_LARGEST, 0.0, M, pc, lock_s, K, V, Y, xin, sws)
 
     def prep():
         pc.copy_(pc0)
+        lock_s.zero_()
         if flush is not None:
             flush.zero_()
 
@@ -325,8 +326,8 @@ def run_gpu(args, wl, dist, rank, world, local_rank):
     st = plk.get_status()
     if st != plk.OK:
         raise RuntimeError(f"device status {plk.error_string(st)}")
-    got = idx[:M].cpu().numpy()
-    if int(seg[-1]) != M or not np.array_equal(np.sort(got), np.sort(wl.pos)):
+    got = np.flatnonzero(lock_s.cpu().numpy().reshape(-1) == 0)
+    if got.size != M or not np.array_equal(got, np.sort(wl.pos)):
         raise RuntimeError("the top-k did not select the perturbed rows")
     if args.profile:
         for _ in range(args.steps):
@@ -434,7 +435,6 @@ def run_gpu(args, wl, dist, rank, world, local_rank):
     e2e_steps = min(K_, 50)
     Xp_host = torch.from_numpy(np.ascontiguousarray(wl.Xp)).to(bf).pin_memory()
     Y_host = torch.empty(Y.shape, dtype=bf).pin_memory()
-    sws = plk.alloc_step_workspace(dm, r, device=dev)
     lock_e = torch.empty_like(lock_in)
     ee = [(E(), E()) for _ in range(e2e_steps)]
     torch.cuda.synchronize()
@@ -1149,7 +1149,7 @@ def main():
             dist.destroy_process_group()
     if res is None or rank != 0:
         return 0
-    launches_per_step = 1 + 1 + 10 + 1  # score, select, layer, commit
+    launches_per_step = 1 + 1 + 10  # score, select (B = 1: one launch), layer step (proxy refresh folded in)
     metric = METRIC if args.frac == 0.25 else f"active-token-layers/sec at 8B-shape, M/N={args.frac}"
     line = {"metric": metric, "value": res["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,

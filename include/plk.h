@@ -297,6 +297,21 @@ int plk_layer_step_partial_static(const plk_dims* dims, const plk_weights* w, co
 size_t plk_workspace_bytes(const plk_dims* dims);
 
 /*
+ * The whole denoising step of one layer on device buffers: in stream order
+ *   plk_score_drift(X, Ut, r, proxy_cache, metric) -> score and fresh proxies;
+ *   plk_select_active(score, lock, mode, tau, k) -> lock (in place), idx, seg_ptr;
+ *   plk_layer_step_partial -> K_cache, V_cache, Y (device, in/out), with
+ *   plk_proxy_commit -> proxy_cache folded into the layer step's last kernel
+ *   (bf16; fp32 runs it as a separate launch).
+ * X [B, N, d] device (layer dtype).  Same arguments, rules, workspace
+ * (plk_step_workspace_bytes) and errors as plk_denoise_step_host below, without
+ * the host copies.
+ */
+int plk_denoise_step(const plk_dims* dims, const plk_weights* w, const void* Ut, int r, int metric, int mode,
+                     float tau, int k, float* proxy_cache, uint8_t* lock, void* K_cache, void* V_cache, void* Y,
+                     const void* X, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * The whole denoising step of one layer from host memory: the step S1..S10 as the
  * calls above chain it, with the layer input coming from and the output going to
  * host buffers ([SL] Sec. 2; [SPA] part 1 for the proxy refresh).  In stream order:

@@ -26,7 +26,7 @@ SEL_THRESH_GT, SEL_THRESH_LT, SEL_TOPK_LARGEST, SEL_TOPK_SMALLEST = 0, 1, 2, 3
 EXPORTED = (
     "plk_score_drift", "plk_select_active", "plk_layer_step_partial", "plk_full_layer_step",
     "plk_proxy_commit", "plk_layer_step_partial_static", "plk_kl_lock", "plk_slowfast_step", "plk_workspace_bytes",
-    "plk_denoise_step_host", "plk_step_workspace_bytes",
+    "plk_denoise_step", "plk_denoise_step_host", "plk_step_workspace_bytes",
     "plk_get_status",
     "plk_set_wait_limit", "plk_set_deterministic",
     "plk_selftest_wait_timeout", "plk_selftest_exp2", "plk_trace_events", "plk_error_string", "plk_version",
@@ -76,6 +76,7 @@ def _load():
         "plk_kl_lock": (I, [V, I, P, P, P, P, F, F, P, P, P]),
         "plk_slowfast_step": (I, [V, ctypes.POINTER(PlkSfParams), P, P, P, P, P, P]),
         "plk_workspace_bytes": (S, [V]),
+        "plk_denoise_step": (I, [V, W, P, I, I, I, F, I, P, P, P, P, P, P, P, S, P]),
         "plk_denoise_step_host": (I, [V, W, P, I, I, I, F, I, P, P, P, P, P, P, P, P, S, P]),
         "plk_step_workspace_bytes": (S, [V, I]),
         "plk_get_status": (I, [P]),
@@ -203,6 +204,17 @@ def alloc_step_workspace(dm, r, device="cuda"):
     if n == 0:
         raise PlkError(ERR_SHAPE, "step_workspace_bytes")
     return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def denoise_step(dm, w, Ut, r, metric, mode, tau, k, proxy_cache, lock, K_cache, V_cache, Y, X, workspace,
+                 stream=None):
+    """The whole step on device buffers (see plk_denoise_step): score, select (lock in place),
+    layer step with the proxy refresh folded in."""
+    pw = w if isinstance(w, PlkWeights) else weights(w)
+    _check(lib.plk_denoise_step(ctypes.byref(dm), ctypes.byref(pw), _ptr(Ut), int(r), int(metric), int(mode),
+                                float(tau), int(k), _ptr(proxy_cache), _ptr(lock), _ptr(K_cache), _ptr(V_cache),
+                                _ptr(Y), _ptr(X), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                _stream(stream)), "denoise_step")
 
 
 def denoise_step_host(dm, w, Ut, r, metric, mode, tau, k, proxy_cache, lock, K_cache, V_cache, Y, X_host, Y_host,

@@ -186,34 +186,75 @@ size_t plk_step_workspace_bytes(const plk_dims* dims, int r) {
   return step_ws_layout(dims, r).total;
 }
 
-int plk_denoise_step_host(const plk_dims* dims, const plk_weights* w, const void* Ut, int r, int metric,
-                          int mode, float tau, int k, float* proxy_cache, uint8_t* lock, void* K_cache,
-                          void* V_cache, void* Y, const void* X_host, void* Y_host, void* workspace,
-                          size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace plk {
+// The checks of the whole-step entry points (PLK_OK or the error code); X may be a host or a
+// device pointer (only checked for null).
+static int check_step_args(const plk_dims* dims, const plk_weights* w, const void* Ut, int r, int metric, int mode,
+                           int k, const float* proxy_cache, const uint8_t* lock, const void* K_cache,
+                           const void* V_cache, const void* Y, const void* X) {
   int e = check_dims(dims);
   if (e != PLK_OK) return e;
   if ((e = check_score_args(dims, r, metric)) != PLK_OK) return e;
-  if (!Ut || !proxy_cache || !lock || !X_host || !Y_host) return PLK_ERR_ARG;
+  if (!Ut || !proxy_cache || !lock || !X) return PLK_ERR_ARG;
   if (mode < PLK_SEL_THRESH_GT || mode > PLK_SEL_TOPK_SMALLEST) return PLK_ERR_ARG;
   if ((mode == PLK_SEL_TOPK_LARGEST || mode == PLK_SEL_TOPK_SMALLEST) && k < 0) return PLK_ERR_ARG;
   if (!w || !w->g1 || !w->w_qkv || !w->w_o || !w->g2 || !w->w_gu || !w->w_down) return PLK_ERR_ARG;
   if (!K_cache || !V_cache || !Y) return PLK_ERR_ARG;
   if (plk_workspace_bytes(dims) == 0) return PLK_ERR_CUDA;
-  const StepWs L = step_ws_layout(dims, r);
-  if (!workspace || ws_bytes < L.total) return PLK_ERR_WORKSPACE;
-  uint8_t* ws = (uint8_t*)workspace;
+  return PLK_OK;
+}
+
+// score -> select (in place) -> layer step with the proxy refresh folded into its last kernel
+static int run_step(const plk_dims* dims, const plk_weights* w, const void* Ut, int r, int metric, int mode,
+                    float tau, int k, float* proxy_cache, uint8_t* lock, void* K_cache, void* V_cache, void* Y,
+                    const void* X, uint8_t* ws, const StepWs& L, cudaStream_t st) {
   float* score = (float*)(ws + L.score);
   float* pnew = (float*)(ws + L.pnew);
   int32_t* idx = (int32_t*)(ws + L.idx);
   int32_t* seg = (int32_t*)(ws + L.seg);
+  int e;
+  if ((e = launch_score(dims, X, Ut, r, proxy_cache, metric, pnew, score, st)) != PLK_OK) return e;
+  if ((e = launch_select(dims, score, lock, lock, mode, tau, k, idx, seg, st)) != PLK_OK) return e;
+  ProxyRefresh pr;
+  pr.r = r;
+  pr.proxy_new = pnew;
+  pr.proxy_cache = proxy_cache;
+  return run_layer(dims, w, X, idx, seg, false, K_cache, V_cache, Y, ws, L.score, st, &pr);
+}
+}  // namespace plk
+
+extern "C" {
+
+int plk_denoise_step(const plk_dims* dims, const plk_weights* w, const void* Ut, int r, int metric, int mode,
+                     float tau, int k, float* proxy_cache, uint8_t* lock, void* K_cache, void* V_cache, void* Y,
+                     const void* X, void* workspace, size_t ws_bytes, void* stream) {
+  int e = check_step_args(dims, w, Ut, r, metric, mode, k, proxy_cache, lock, K_cache, V_cache, Y, X);
+  if (e != PLK_OK) return e;
+  const StepWs L = step_ws_layout(dims, r);
+  if (!workspace || ws_bytes < L.total) return PLK_ERR_WORKSPACE;
+  return run_step(dims, w, Ut, r, metric, mode, tau, k, proxy_cache, lock, K_cache, V_cache, Y, X,
+                  (uint8_t*)workspace, L, (cudaStream_t)stream);
+}
+
+int plk_denoise_step_host(const plk_dims* dims, const plk_weights* w, const void* Ut, int r, int metric,
+                          int mode, float tau, int k, float* proxy_cache, uint8_t* lock, void* K_cache,
+                          void* V_cache, void* Y, const void* X_host, void* Y_host, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  int e = check_step_args(dims, w, Ut, r, metric, mode, k, proxy_cache, lock, K_cache, V_cache, Y, X_host);
+  if (e != PLK_OK) return e;
+  if (!Y_host) return PLK_ERR_ARG;
+  const StepWs L = step_ws_layout(dims, r);
+  if (!workspace || ws_bytes < L.total) return PLK_ERR_WORKSPACE;
+  uint8_t* ws = (uint8_t*)workspace;
   void* X = ws + L.x;
   const size_t BN = (size_t)dims->B * dims->N, es = dims->dtype == PLK_BF16 ? 2 : 4;
   cudaStream_t st = (cudaStream_t)stream;
   if (cudaMemcpyAsync(X, X_host, es * BN * dims->d, cudaMemcpyHostToDevice, st) != cudaSuccess) return PLK_ERR_CUDA;
-  if ((e = launch_score(dims, X, Ut, r, proxy_cache, metric, pnew, score, st)) != PLK_OK) return e;
-  if ((e = launch_select(dims, score, lock, lock, mode, tau, k, idx, seg, st)) != PLK_OK) return e;
-  if ((e = run_layer(dims, w, X, idx, seg, false, K_cache, V_cache, Y, ws, L.score, st)) != PLK_OK) return e;
-  if ((e = launch_proxy_commit(dims, r, idx, seg, pnew, proxy_cache, st)) != PLK_OK) return e;
+  if ((e = run_step(dims, w, Ut, r, metric, mode, tau, k, proxy_cache, lock, K_cache, V_cache, Y, X, ws, L, st)) !=
+      PLK_OK)
+    return e;
   if (cudaMemcpyAsync(Y_host, Y, es * BN * dims->d, cudaMemcpyDeviceToHost, st) != cudaSuccess) return PLK_ERR_CUDA;
   return PLK_OK;
 }

@@ -469,10 +469,12 @@ __global__ void __launch_bounds__(256) finish_gu_kernel(const float* __restrict_
   }
 }
 
-// residual-stream sums of compact row j -> Y cache row idx[j]
+// residual-stream sums of compact row j -> Y cache row idx[j]; with pnew (the whole
+// step's proxy refresh folded in) also pc[idx[j]] = pnew[idx[j]] (r fp32 values)
 __global__ void __launch_bounds__(256) finish_y_kernel(const float* __restrict__ h32, const int32_t* __restrict__ idx,
                                                        const int32_t* __restrict__ seg_ptr, int B, int d,
-                                                       __nv_bfloat16* __restrict__ Y) {
+                                                       __nv_bfloat16* __restrict__ Y, int r,
+                                                       const float* __restrict__ pnew, float* __restrict__ pc) {
   pdl_wait();
   pdl_trigger();
   const int M = seg_ptr[B];
@@ -484,6 +486,8 @@ __global__ void __launch_bounds__(256) finish_y_kernel(const float* __restrict__
       load8(h32 + (size_t)j * d + v * 8, f);
       store_vec<__nv_bfloat16, 8>(Y + row * d + v * 8, f);
     }
+    if (pnew)
+      for (int c = threadIdx.x; c < r; c += blockDim.x) pc[row * r + c] = pnew[row * r + c];
   }
 }
 
@@ -629,7 +633,7 @@ static int run_layer_f32(const plk_dims* dm, const plk_weights* w, const float* 
 
 static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_bfloat16* X, const int32_t* idx,
                           const int32_t* seg, void* Kc, void* Vc, void* Y, uint8_t* ws, const Workspace& L,
-                          cudaStream_t st) {
+                          cudaStream_t st, const ProxyRefresh* pr) {
   const int B = dm->B, d = dm->d, F = dm->F, Mcap = dm->B * dm->N, dkv = kv_width(dm);
   // activations that feed tensor-core products: hi/lo bf16 pairs
   __nv_bfloat16* xn = (__nv_bfloat16*)(ws + L.xn);
@@ -737,13 +741,15 @@ static int run_layer_bf16(const plk_dims* dm, const plk_weights* w, const __nv_b
   trace_mark(9, st);
 
   PLK_TRY(launch_pdl(finish_y_kernel, dim3(rgrid), dim3(256), 0, st, (const float*)h32, idx, seg, B, d,
-                     (__nv_bfloat16*)Y));
+                     (__nv_bfloat16*)Y, pr ? pr->r : 0, pr ? pr->proxy_new : nullptr,
+                     pr ? pr->proxy_cache : nullptr));
   trace_mark(10, st);
   return PLK_OK;
 }
 
 int run_layer(const plk_dims* dm, const plk_weights* w, const void* X, const int32_t* idx, const int32_t* seg_ptr,
-              bool full, void* Kc, void* Vc, void* Y, void* ws, size_t ws_bytes, cudaStream_t st) {
+              bool full, void* Kc, void* Vc, void* Y, void* ws, size_t ws_bytes, cudaStream_t st,
+              const ProxyRefresh* pr) {
   const int nsm = device_sm_count();
   if (nsm <= 0) return PLK_ERR_CUDA;
   const Workspace L = workspace_layout(dm, nsm);
@@ -758,9 +764,12 @@ int run_layer(const plk_dims* dm, const plk_weights* w, const void* X, const int
     idx = iota;
     seg_ptr = seg;
   }
-  if (dm->dtype == PLK_F32)
-    return run_layer_f32(dm, w, (const float*)X, idx, seg_ptr, (float*)Kc, (float*)Vc, (float*)Y, wsb, L, st);
-  return run_layer_bf16(dm, w, (const __nv_bfloat16*)X, idx, seg_ptr, Kc, Vc, Y, wsb, L, st);
+  if (dm->dtype == PLK_F32) {
+    PLK_TRY(run_layer_f32(dm, w, (const float*)X, idx, seg_ptr, (float*)Kc, (float*)Vc, (float*)Y, wsb, L, st));
+    if (pr) return launch_proxy_commit(dm, pr->r, idx, seg_ptr, pr->proxy_new, pr->proxy_cache, st);
+    return PLK_OK;
+  }
+  return run_layer_bf16(dm, w, (const __nv_bfloat16*)X, idx, seg_ptr, Kc, Vc, Y, wsb, L, st, pr);
 }
 
 }  // namespace plk

@@ -99,9 +99,16 @@ int launch_slowfast(const plk_dims* dims, const plk_sf_params* prm, const float*
 int check_layer_args(const plk_dims* dims, const plk_weights* w, const void* X, const int32_t* idx,
                      const int32_t* seg_ptr, const void* K_cache, const void* V_cache, const void* Y);
 
+// Optional proxy refresh folded into the layer step's last kernel (bf16 path):
+// proxy_cache[idx[j]] = proxy_new[idx[j]] (r fp32 values per row) for j < M.
+struct ProxyRefresh {
+  int r = 0;
+  const float* proxy_new = nullptr;
+  float* proxy_cache = nullptr;
+};
 int run_layer(const plk_dims* dims, const plk_weights* w, const void* X, const int32_t* idx,
               const int32_t* seg_ptr, bool full, void* K_cache, void* V_cache, void* Y, void* ws,
-              size_t ws_bytes, cudaStream_t st);
+              size_t ws_bytes, cudaStream_t st, const ProxyRefresh* pr = nullptr);
 
 // Arguments of the tcgen05 GEMM out[t, f] += sum_k (Xhi[t, k] + Xlo[t, k]) W[f, k]
 // over the M = seg_ptr[B] compact tokens (fp32 out, added with bulk reduce-adds;

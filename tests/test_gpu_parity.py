@@ -744,7 +744,10 @@ def test_exp2_fma_error_bound(plk):
 # ---------------------------------------------------------------------------
 # the whole step from host memory (plk_denoise_step_host) against the oracle
 # ---------------------------------------------------------------------------
-def test_denoise_step_host_matches_oracle(plk):
+@pytest.mark.parametrize("entry", ["host", "device"])
+def test_denoise_step_matches_oracle(plk, entry):
+    """The whole step through plk_denoise_step_host (host X in, host Y out) or plk_denoise_step
+    (device buffers); the proxy refresh runs inside the layer step's last kernel."""
     D = synth.Dims(B=2, N=320, d=512, H=4, hd=128, F=1536, dtype="bf16")
     r, k = 128, 96
     W = synth.layer_weights(D, 0.02, seed=14)
@@ -772,14 +775,21 @@ def test_denoise_step_host_matches_oracle(plk):
     n = plk.step_workspace_bytes(dm, r)
     assert n > plk.workspace_bytes(dm)
     g["workspace"] = Guarded((n,), torch.uint8)
-    X_host = torch.from_numpy(np.ascontiguousarray(X2)).to(BF).pin_memory()
-    Y_host = torch.full(base.Y.shape, -3.0, dtype=BF).pin_memory()
-    plk.denoise_step_host(dm, weights_dev(W, D), dev(Ut, BF), r, plk.METRIC_L2, plk.SEL_TOPK_LARGEST, 0.0, k,
-                          g["proxy"].t, g["lock"].t, g["K"].t, g["V"].t, g["Y"].t, X_host, Y_host, g["workspace"].t)
+    if entry == "host":
+        X_host = torch.from_numpy(np.ascontiguousarray(X2)).to(BF).pin_memory()
+        Y_host = torch.full(base.Y.shape, -3.0, dtype=BF).pin_memory()
+        plk.denoise_step_host(dm, weights_dev(W, D), dev(Ut, BF), r, plk.METRIC_L2, plk.SEL_TOPK_LARGEST, 0.0, k,
+                              g["proxy"].t, g["lock"].t, g["K"].t, g["V"].t, g["Y"].t, X_host, Y_host,
+                              g["workspace"].t)
+    else:
+        g["X"] = Guarded(X2.shape, BF, init=dev(X2, BF))
+        plk.denoise_step(dm, weights_dev(W, D), dev(Ut, BF), r, plk.METRIC_L2, plk.SEL_TOPK_LARGEST, 0.0, k,
+                         g["proxy"].t, g["lock"].t, g["K"].t, g["V"].t, g["Y"].t, g["X"].t, g["workspace"].t)
     assert plk.get_status() == plk.OK
-    check_guards(g, "denoise_step_host")
+    check_guards(g, f"denoise_step ({entry})")
     assert np.array_equal(host(g["lock"].t), ref_lock)
     Yd = host(g["Y"].t)
-    assert np.array_equal(Y_host.to(torch.float64).numpy(), Yd), "Y_host is the device Y"
-    _check_layer_rows(host(g["K"].t), host(g["V"].t), Yd, ref, base, ref_lock, "host step")
+    if entry == "host":
+        assert np.array_equal(Y_host.to(torch.float64).numpy(), Yd), "Y_host is the device Y"
+    _check_layer_rows(host(g["K"].t), host(g["V"].t), Yd, ref, base, ref_lock, f"{entry} step")
     assert_f32_close(host(g["proxy"].t), ref_pc, "proxy cache", tol=1e-5)
