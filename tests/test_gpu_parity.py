@@ -396,10 +396,12 @@ def test_workspace_too_small_is_rejected(plk):
 # the tiny fp32 workload: 20 denoising steps, every step checked
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("noise_var", [synth.TINY_NOISE_VAR, 0.1])
-def test_tiny_fp32_driver(plk, noise_var):
+@pytest.mark.parametrize("entry", ["calls", "step"])
+def test_tiny_fp32_driver(plk, noise_var, entry):
     """The tiny fp32 workload step by step.  With its own noise (variance 0.01) the active set
     empties within four steps; with variance 0.1 it shrinks from 13 rows to 1 over the 20 steps,
-    so the fp32 layer runs on several rows at every step (decision margins >= 2e-4 from tau)."""
+    so the fp32 layer runs on several rows at every step (decision margins >= 2e-4 from tau).
+    entry "calls": the four API calls of a step; "step": one plk_denoise_step per step."""
     D = synth.TINY
     r = synth.TINY_RANK
     W = synth.layer_weights(D, 1.0 / math.sqrt(D.d))
@@ -425,20 +427,26 @@ def test_tiny_fp32_driver(plk, noise_var):
     pc.copy_(pnew)
     lock = dev(lock0, torch.uint8)
     idx, seg = sel_bufs(D.B, D.N)
+    sws = plk.alloc_step_workspace(dm, r) if entry == "step" else None
     X = X0.copy()
     for t, eps in enumerate(noises):
         X = perturb(X, eps, host(lock) == 0)
         Xd = dev(X, f32)
-        plk.score_drift(dm, Xd, Utd, r, pc, plk.METRIC_COS, score, proxy_out=pnew)
-        plk.select_active(dm, score, lock, lock, plk.SEL_THRESH_GT, synth.TINY_TAU, 0, idx, seg)
-        plk.layer_step_partial(dm, Wd, Xd, idx, seg, K, V, Y, ws)
-        plk.proxy_commit(dm, r, idx, seg, pnew, pc)
+        if entry == "calls":
+            plk.score_drift(dm, Xd, Utd, r, pc, plk.METRIC_COS, score, proxy_out=pnew)
+            plk.select_active(dm, score, lock, lock, plk.SEL_THRESH_GT, synth.TINY_TAU, 0, idx, seg)
+            plk.layer_step_partial(dm, Wd, Xd, idx, seg, K, V, Y, ws)
+            plk.proxy_commit(dm, r, idx, seg, pnew, pc)
+        else:
+            plk.denoise_step(dm, Wd, Utd, r, plk.METRIC_COS, plk.SEL_THRESH_GT, synth.TINY_TAU, 0, pc, lock, K, V,
+                             Y, Xd, sws)
         assert plk.get_status() == plk.OK
         rec = recs[t]
         assert np.array_equal(host(lock), rec["lock"]), f"step {t}: lock"
-        M = int(rec["seg_ptr"][-1])
-        assert np.array_equal(host(seg), rec["seg_ptr"]) and np.array_equal(host(idx)[:M], rec["idx"])
-        assert_f32_close(host(score), rec["score"], f"step {t}: score")
+        if entry == "calls":
+            M = int(rec["seg_ptr"][-1])
+            assert np.array_equal(host(seg), rec["seg_ptr"]) and np.array_equal(host(idx)[:M], rec["idx"])
+            assert_f32_close(host(score), rec["score"], f"step {t}: score")
         for name, g in (("K", K), ("V", V), ("Y", Y), ("proxy", pc)):
             assert_f32_close(host(g), rec[name], f"step {t}: {name}")
 
