@@ -409,6 +409,30 @@ __global__ void __launch_bounds__(256) finish_qkv_kernel(const float* __restrict
   for (int j = blockIdx.x; j < M; j += gridDim.x) {
     const size_t row = (size_t)idx[j];
     const float* src = qkv32 + (size_t)j * W;
+    if (!rope) {
+      // every thread loads its (up to) 6 vectors of the row before it stores any: one round of
+      // memory latency per row instead of one per vector
+      constexpr int KV = 6;
+      for (int base = 0; base < nv; base += KV * 256) {
+        float f[KV][8];
+#pragma unroll
+        for (int k = 0; k < KV; ++k) {
+          const int v = base + threadIdx.x + k * 256;
+          if (v < nv) load8(src + v * 8, f[k]);
+        }
+#pragma unroll
+        for (int k = 0; k < KV; ++k) {
+          const int c = (base + threadIdx.x + k * 256) * 8;
+          if (c >= W) continue;
+          if (c < d)
+            store_hilo<8>(q + (size_t)j * d + c, q_lo + (size_t)j * d + c, f[k]);
+          else
+            store_vec<__nv_bfloat16, 8>(c < d + dkv ? Kc + row * dkv + (c - d) : Vc + row * dkv + (c - d - dkv),
+                                        f[k]);
+        }
+      }
+      continue;
+    }
     const int pos = (int)(row % (size_t)N);
     for (int u = threadIdx.x; u < npair; u += blockDim.x) {
       const bool isq = u < qunits;
@@ -456,15 +480,27 @@ __global__ void __launch_bounds__(256) finish_gu_kernel(const float* __restrict_
   pdl_trigger();
   const int M = seg_ptr[B];
   const int nv = F / 8;
+  constexpr int KV = 6;  // vectors a thread loads before it stores any (one memory latency per row)
   for (int j = blockIdx.x; j < M; j += gridDim.x) {
     const float* src = gu32 + (size_t)j * 2 * F;
-    for (int v = threadIdx.x; v < nv; v += blockDim.x) {
-      float g[8], u[8];
-      load8(src + v * 8, g);
-      load8(src + F + v * 8, u);
+    for (int base = 0; base < nv; base += KV * 256) {
+      float g[KV][8], u[KV][8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) g[e] = silu_f(g[e]) * u[e];
-      store_hilo<8>(act + (size_t)j * F + v * 8, act_lo + (size_t)j * F + v * 8, g);
+      for (int k = 0; k < KV; ++k) {
+        const int v = base + threadIdx.x + k * 256;
+        if (v < nv) {
+          load8(src + v * 8, g[k]);
+          load8(src + F + v * 8, u[k]);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < KV; ++k) {
+        const int v = base + threadIdx.x + k * 256;
+        if (v >= nv) continue;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) g[k][e] = silu_f(g[k][e]) * u[k][e];
+        store_hilo<8>(act + (size_t)j * F + v * 8, act_lo + (size_t)j * F + v * 8, g[k]);
+      }
     }
   }
 }
@@ -479,12 +515,21 @@ __global__ void __launch_bounds__(256) finish_y_kernel(const float* __restrict__
   pdl_trigger();
   const int M = seg_ptr[B];
   const int nv = d / 8;
+  constexpr int KV = 2;  // vectors a thread loads before it stores any
   for (int j = blockIdx.x; j < M; j += gridDim.x) {
     const size_t row = (size_t)idx[j];
-    for (int v = threadIdx.x; v < nv; v += blockDim.x) {
-      float f[8];
-      load8(h32 + (size_t)j * d + v * 8, f);
-      store_vec<__nv_bfloat16, 8>(Y + row * d + v * 8, f);
+    for (int base = 0; base < nv; base += KV * 256) {
+      float f[KV][8];
+#pragma unroll
+      for (int k = 0; k < KV; ++k) {
+        const int v = base + threadIdx.x + k * 256;
+        if (v < nv) load8(h32 + (size_t)j * d + v * 8, f[k]);
+      }
+#pragma unroll
+      for (int k = 0; k < KV; ++k) {
+        const int v = base + threadIdx.x + k * 256;
+        if (v < nv) store_vec<__nv_bfloat16, 8>(Y + row * d + v * 8, f[k]);
+      }
     }
     if (pnew)
       for (int c = threadIdx.x; c < r; c += blockDim.x) pc[row * r + c] = pnew[row * r + c];
