@@ -752,6 +752,33 @@ def test_exp2_fma_error_bound(plk):
 # ---------------------------------------------------------------------------
 # the whole step from host memory (plk_denoise_step_host) against the oracle
 # ---------------------------------------------------------------------------
+def test_denoise_step_k_zero_is_noop(plk):
+    """Top-k with k = 0 keeps no row: every row locks, and K, V, Y and the proxy cache are left
+    as they were (the layer step and the folded proxy refresh see M = 0)."""
+    D = synth.Dims(B=2, N=320, d=512, H=4, hd=128, F=1536, dtype="bf16")
+    r = 64
+    rng = np.random.default_rng(15)
+    W = synth.layer_weights(D, 0.02, seed=15)
+    X = synth.hidden_states(D, seed=15)
+    caches = [synth.round_bf16(rng.standard_normal((D.B, D.N, D.d)).astype(np.float32)) for _ in range(3)]
+    pc = rng.standard_normal((D.B, D.N, r)).astype(np.float32)
+    dm = pdims(plk, D)
+    g = {name: Guarded(c.shape, BF, init=dev(c, BF)) for name, c in zip("KVY", caches)}
+    g["proxy"] = Guarded(pc.shape, torch.float32, init=pc)
+    g["lock"] = Guarded((D.B, D.N), torch.uint8, fill=0)
+    g["X"] = Guarded(X.shape, BF, init=dev(X, BF))
+    g["workspace"] = Guarded((plk.step_workspace_bytes(dm, r),), torch.uint8)
+    plk.denoise_step(dm, weights_dev(W, D), dev(synth.proxy_basis(D.d, r, seed=15), BF), r, plk.METRIC_L2,
+                     plk.SEL_TOPK_LARGEST, 0.0, 0, g["proxy"].t, g["lock"].t, g["K"].t, g["V"].t, g["Y"].t, g["X"].t,
+                     g["workspace"].t)
+    assert plk.get_status() == plk.OK
+    check_guards(g, "denoise_step k = 0")
+    assert np.all(host(g["lock"].t) == 1)
+    for name, ref in (("K", caches[0]), ("V", caches[1]), ("Y", caches[2])):
+        assert np.array_equal(host(g[name].t), ref.astype(np.float64)), f"{name} changed"
+    assert np.array_equal(host(g["proxy"].t), pc.astype(np.float64)), "proxy cache changed"
+
+
 @pytest.mark.parametrize("entry", ["host", "device"])
 def test_denoise_step_matches_oracle(plk, entry):
     """The whole step through plk_denoise_step_host (host X in, host Y out) or plk_denoise_step
