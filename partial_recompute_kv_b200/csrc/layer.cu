@@ -4,16 +4,17 @@
 // "Algorithmic Complexity"), and the full-recompute baseline (Sec. 1).
 //
 // bf16 chain (10 launches, M read on the device, no host synchronisation):
-//   1 gather rows idx[j] of X, RMSNorm1 -> xn, x -> h (fp32), zero the QKV sums
-//   2 tcgen05 GEMM  xn W_qkv^T -> QKV sums (fp32, split-K reduce-adds)
+//   1 gather rows idx[j] of X, RMSNorm1 -> xn, x -> h (fp32); clear the GEMMs'
+//     split-tile counts
+//   2 tcgen05 GEMM  xn W_qkv^T -> QKV sums (fp32; split tiles land in a fixed order)
 //   3 QKV sums -> q (compact), K and V scattered into the cache rows idx[j] (bf16)
 //   4 attention of the M queries over all N cached keys -> a
 //   5 tcgen05 GEMM  h += a W_o^T (fp32)
-//   6 RMSNorm2(h) -> hn, zero the gate/up sums
-//   7 tcgen05 GEMM  hn [W_g; W_u]^T -> gate/up sums (fp32)
+//   6 RMSNorm2(h) -> hn
+//   7 tcgen05 GEMM  hn [W_g; W_u]^T -> gate/up sums (fp32, fixed order as in 2)
 //   8 act = silu(g) * u
 //   9 tcgen05 GEMM  h += act W_down^T (fp32)
-//  10 h -> Y rows idx[j] (bf16)
+//  10 h -> Y rows idx[j] (bf16); in the whole-step call also the proxy refresh
 // The layer stores bf16 only where its results land in the caller's tensors (the
 // K/V cache rows and Y).  Every activation that feeds a tensor-core product (xn,
 // q, a, hn, act) is held as a pair of bf16 tensors, hi = bf16(v) and
