@@ -426,8 +426,12 @@ def run_gpu(args, wl, dist, rank, world, local_rank):
     d_, F_, r_, BN = D.d, D.F, r, D.B * D.N
     alg_bytes = {"score": 2 * BN * d_ + 8 * BN * r_ + 2 * d_ * r_,
                  "select": 6 * BN + 4 * M,
-                 "rmsnorm1": 20 * M * d_, "finish_qkv": 18 * M * d_,
-                 "rmsnorm2": 6 * M * d_ + 8 * M * F_, "finish_gu": 10 * M * F_,
+                 # x in (bf16), the hi/lo pair and the fp32 residual out
+                 "rmsnorm1": 10 * M * d_,
+                 # the fp32 q, k and v sums in, q as a hi/lo pair and the K/V rows (bf16) out
+                 "finish_qkv": 20 * M * d_,
+                 "rmsnorm2": 8 * M * d_,  # h in (fp32), the hi/lo pair out
+                 "finish_gu": 12 * M * F_,  # gate and up sums in, silu(g) u as a hi/lo pair out
                  "finish_y": 6 * M * d_, "proxy_commit": 8 * M * r_}
     hbm = float(pk["hbm_gbs"])
     hbm_kernels = {k: {"bytes": v, "GB/s": v / (per[k] * 1e-6) / 1e9, "frac": v / (per[k] * 1e-6) / 1e9 / hbm}
@@ -624,7 +628,7 @@ def run_kernel_configs(args):
     gemm_flops = M * (8 * D.d * D.d + 6 * D.d * D.F)
     gemm_us = per["gemm_qkv"] + per["gemm_o"] + per["gemm_gu"] + per["gemm_down"]
     att_flops = 4 * D.B * D.N * D.N * D.d  # QK^T and PV over every (query, key) pair of a sequence
-    scat = 18 * M * D.d
+    scat = 20 * M * D.d  # the fp32 q, k and v sums in; q (hi/lo) and the K/V rows out
     out.append({"kernel": "layer step, every row active", "config": f"B={D.B} N={D.N} (stack step 0)",
                 "us": us_step, "active_token_layers_per_s": M / (us_step * 1e-6),
                 "gemm_tc_kernel": {"us": gemm_us, "TFLOP/s": gemm_flops / (gemm_us * 1e-6) / 1e12,

@@ -32,6 +32,11 @@
  *     later by plk_get_status().
  *   - Tensors are dense row-major.  Token row (b, i) of a [B, N, ...] tensor is
  *     flattened row b*N + i.
+ *   - The tensors the kernels move with 16-byte vectors or TMA start on a
+ *     16-byte boundary: X, Ut, proxy_cache and proxy_out of the score, the
+ *     weights and the K_cache, V_cache and Y of the layer steps (cudaMalloc and
+ *     PyTorch allocations are 256-byte aligned); idx and seg_ptr on a 4-byte
+ *     one.  A misaligned pointer returns PLK_ERR_ARG with nothing enqueued.
  *   - dtype PLK_BF16: hidden states, weights, Ut, K/V/Y caches are bf16;
  *     proxies and scores are fp32; accumulation is fp32.  dtype PLK_F32: all
  *     of those are fp32 (fp32 arithmetic, no tensor cores).

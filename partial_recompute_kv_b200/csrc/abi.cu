@@ -23,14 +23,27 @@ static int check_dims(const plk_dims* d) {
   return PLK_OK;
 }
 
+// The kernels move these tensors with 16-byte vectors or TMA: their base addresses must be
+// 16-byte aligned (rows stay aligned: d, F and bf16 proxy ranks are multiples of 16 elements).
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool weights_ok(const plk_weights* w) {
+  if (!w || !w->g1 || !w->w_qkv || !w->w_o || !w->g2 || !w->w_gu || !w->w_down) return false;
+  return aligned16(w->g1) && aligned16(w->w_qkv) && aligned16(w->w_o) && aligned16(w->g2) && aligned16(w->w_gu) &&
+         aligned16(w->w_down);
+}
+static bool caches_ok(const void* K_cache, const void* V_cache, const void* Y) {
+  return K_cache && V_cache && Y && aligned16(K_cache) && aligned16(V_cache) && aligned16(Y);
+}
+
 // The argument checks of plk_layer_step_partial (dims, weights, inputs and caches;
 // the workspace is checked where it is laid out).
 int check_layer_args(const plk_dims* dims, const plk_weights* w, const void* X, const int32_t* idx,
                      const int32_t* seg_ptr, const void* K_cache, const void* V_cache, const void* Y) {
   const int e = check_dims(dims);
   if (e != PLK_OK) return e;
-  if (!w || !w->g1 || !w->w_qkv || !w->w_o || !w->g2 || !w->w_gu || !w->w_down) return PLK_ERR_ARG;
-  if (!X || !idx || !seg_ptr || !K_cache || !V_cache || !Y) return PLK_ERR_ARG;
+  if (!weights_ok(w)) return PLK_ERR_ARG;
+  if (!X || !aligned16(X) || !idx || !seg_ptr || !caches_ok(K_cache, V_cache, Y)) return PLK_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(idx) | reinterpret_cast<uintptr_t>(seg_ptr)) & 3u) return PLK_ERR_ARG;
   return PLK_OK;
 }
 
@@ -67,6 +80,7 @@ int plk_score_drift(const plk_dims* dims, const void* X, const void* Ut, int r, 
   const int e = check_dims(dims);
   if (e != PLK_OK) return e;
   if (!X || !Ut || !proxy_cache || !score_out) return PLK_ERR_ARG;
+  if (!aligned16(X) || !aligned16(Ut) || !aligned16(proxy_cache) || !aligned16(proxy_out)) return PLK_ERR_ARG;
   if (metric != PLK_METRIC_COS && metric != PLK_METRIC_L2) return PLK_ERR_ARG;
   if (proxy_out && proxy_out == proxy_cache) return PLK_ERR_ARG;
   if (dims->dtype == PLK_BF16) {
@@ -126,8 +140,8 @@ int plk_full_layer_step(const plk_dims* dims, const plk_weights* w, const void* 
                         void* Y, void* workspace, size_t ws_bytes, void* stream) {
   const int e = check_dims(dims);
   if (e != PLK_OK) return e;
-  if (!w || !w->g1 || !w->w_qkv || !w->w_o || !w->g2 || !w->w_gu || !w->w_down) return PLK_ERR_ARG;
-  if (!X || !K_cache || !V_cache || !Y) return PLK_ERR_ARG;
+  if (!weights_ok(w)) return PLK_ERR_ARG;
+  if (!X || !aligned16(X) || !caches_ok(K_cache, V_cache, Y)) return PLK_ERR_ARG;
   return run_layer(dims, w, X, nullptr, nullptr, true, K_cache, V_cache, Y, workspace, ws_bytes,
                    (cudaStream_t)stream);
 }
@@ -190,7 +204,7 @@ size_t plk_step_workspace_bytes(const plk_dims* dims, int r) {
 
 namespace plk {
 // The checks of the whole-step entry points (PLK_OK or the error code); X may be a host or a
-// device pointer (only checked for null).
+// device pointer (only checked for null here).
 static int check_step_args(const plk_dims* dims, const plk_weights* w, const void* Ut, int r, int metric, int mode,
                            int k, const float* proxy_cache, const uint8_t* lock, const void* K_cache,
                            const void* V_cache, const void* Y, const void* X) {
@@ -198,10 +212,10 @@ static int check_step_args(const plk_dims* dims, const plk_weights* w, const voi
   if (e != PLK_OK) return e;
   if ((e = check_score_args(dims, r, metric)) != PLK_OK) return e;
   if (!Ut || !proxy_cache || !lock || !X) return PLK_ERR_ARG;
+  if (!aligned16(Ut) || !aligned16(proxy_cache)) return PLK_ERR_ARG;
   if (mode < PLK_SEL_THRESH_GT || mode > PLK_SEL_TOPK_SMALLEST) return PLK_ERR_ARG;
   if ((mode == PLK_SEL_TOPK_LARGEST || mode == PLK_SEL_TOPK_SMALLEST) && k < 0) return PLK_ERR_ARG;
-  if (!w || !w->g1 || !w->w_qkv || !w->w_o || !w->g2 || !w->w_gu || !w->w_down) return PLK_ERR_ARG;
-  if (!K_cache || !V_cache || !Y) return PLK_ERR_ARG;
+  if (!weights_ok(w) || !caches_ok(K_cache, V_cache, Y)) return PLK_ERR_ARG;
   if (plk_workspace_bytes(dims) == 0) return PLK_ERR_CUDA;
   return PLK_OK;
 }
@@ -232,6 +246,7 @@ int plk_denoise_step(const plk_dims* dims, const plk_weights* w, const void* Ut,
                      const void* X, void* workspace, size_t ws_bytes, void* stream) {
   int e = check_step_args(dims, w, Ut, r, metric, mode, k, proxy_cache, lock, K_cache, V_cache, Y, X);
   if (e != PLK_OK) return e;
+  if (!aligned16(X)) return PLK_ERR_ARG;
   const StepWs L = step_ws_layout(dims, r);
   if (!workspace || ws_bytes < L.total) return PLK_ERR_WORKSPACE;
   return run_step(dims, w, Ut, r, metric, mode, tau, k, proxy_cache, lock, K_cache, V_cache, Y, X,

@@ -15,7 +15,9 @@
 // moves each 128/S-row slice with one bulk copy into the idle stage buffers of
 // the CTA that finishes those rows (the copies complete on that CTA's
 // mbarrier); every CTA then sums its S slices locally (no global scratch, no
-// remote loads, no thread-issued remote stores).
+// remote loads, no thread-issued remote stores).  When there are more 128-row tiles
+// than SMs, two CTAs share each SM with half the stage ring each, so that every tile
+// runs in the first wave.
 // fp32: a SIMT kernel, one warp per row.
 #include "plk_common.cuh"
 #include "plk_internal.h"
@@ -29,7 +31,7 @@ constexpr int kScRingBudget = 200 * 1024;
 
 // Ring depth for proxy rank r: as many (X, U) stages as fit 200 KB, 2..6.  The
 // X loads are HBM-latency bound, so the more stages in flight the better.
-__host__ __device__ inline int sc_stages(int r) {
+inline int sc_stages(int r) {
   const int stage_bytes = kScA + ((r * 128 + 1023) & ~1023);
   const int n = kScRingBudget / stage_bytes;
   return n < 2 ? 2 : (n > kScStagesMax ? kScStagesMax : n);
@@ -49,14 +51,13 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
                                                        const __grid_constant__ CUtensorMap tmU, int rows, int d,
                                                        int r, int tmem_cols, const float* __restrict__ cache,
                                                        float* __restrict__ pout, float* __restrict__ score,
-                                                       int metric) {
+                                                       int metric, int stages, int x_stream) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   const int stageB = r * 128;
   const int stage_bytes = kScA + ((stageB + 1023) & ~1023);
-  const int kScStages = sc_stages(r);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kScStages * stage_bytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + stages * stage_bytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + kScStagesMax;
   uint64_t* done = bars + 2 * kScStagesMax;
@@ -73,7 +74,7 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
   const int kb0 = ks * nkb_all / S;
   const int nkb = (ks + 1) * nkb_all / S - kb0;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kScStages; ++i) {
+    for (int i = 0; i < stages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
@@ -91,8 +92,17 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
 
+  if (S == 1 && warp == 3 && lane == 0) {
+    // the cached proxies of this tile's rows, read by the epilogue: into L2 while X streams
+    const int nrows = min(128, rows - row0);
+    const char* src = reinterpret_cast<const char*>(cache + (size_t)row0 * r);
+    for (uint32_t off = 0, bytes = (uint32_t)(nrows * r * 4); off < bytes; off += 16384u)
+      bulk_prefetch_l2(src + off, min(16384u, bytes - off));
+  }
   if (warp == 0) {
     if (elect_one()) {
+      // X larger than the L2 is read once: evict first, so that the proxies and Ut stay
+      const uint64_t pol_x = x_stream ? l2_policy_evict_first() : l2_policy_evict_normal();
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
@@ -103,18 +113,18 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
         }
         uint8_t* a = smem + stage * stage_bytes;
         mbar_expect_tx(&full[stage], (uint32_t)(kScA + stageB));
-        tma_load_2d(a, &tmX, (kb0 + kb) * 64, row0, &full[stage]);
+        tma_load_2d_hint(a, &tmX, (kb0 + kb) * 64, row0, &full[stage], pol_x);
         tma_load_2d(a + kScA, &tmU, (kb0 + kb) * 64, 0, &full[stage]);
         ++issued;
-        if (++stage == kScStages) {
+        if (++stage == stages) {
           stage = 0;
           phase ^= 1;
         }
       }
       if (*s_abort) {  // let started copies land before exit
-        for (int i = 0; i < kScStages && i < issued; ++i) {
+        for (int i = 0; i < stages && i < issued; ++i) {
           const int kb = issued - 1 - i;
-          (void)mbar_wait(&full[kb % kScStages], (uint32_t)((kb / kScStages) & 1));
+          (void)mbar_wait(&full[kb % stages], (uint32_t)((kb / stages) & 1));
         }
       }
     }
@@ -136,7 +146,7 @@ __global__ void __launch_bounds__(128) score_tc_kernel(const __grid_constant__ C
 #pragma unroll
         for (int k = 0; k < 4; ++k) umma_bf16(tmem, adesc + 2 * k, bdesc + 2 * k, idesc, (kb | k) ? 1u : 0u);
         umma_commit(&empty[stage]);
-        if (++stage == kScStages) {
+        if (++stage == stages) {
           stage = 0;
           phase ^= 1;
         }
@@ -342,9 +352,24 @@ __global__ void proxy_commit_kernel(const int32_t* __restrict__ idx, const int32
     if (lane + u * 32 < r) pc[row * r + lane + u * 32] = v[u];
 }
 
-static int score_tc_smem(int r) {
+static int score_tc_smem(int r, int stages) {
   const int stage_bytes = kScA + ((r * 128 + 1023) & ~1023);
-  return sc_stages(r) * stage_bytes + 128 + 1024;
+  return stages * stage_bytes + 128 + 1024;
+}
+
+// Dynamic shared memory one CTA may take so that two CTAs share an SM (per device, cached).
+static int score_tc_half_sm_smem() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  int per_sm = 0, reserved = 0;
+  if (cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
+    return 0;
+  const int v = per_sm / 2 - reserved;
+  if (dev < 64) cached[dev] = v;
+  return v;
 }
 
 int launch_score(const plk_dims* dims, const void* X, const void* Ut, int r, const float* proxy_cache,
@@ -360,27 +385,37 @@ int launch_score(const plk_dims* dims, const void* X, const void* Ut, int r, con
   if (make_tmap_bf16(&tmU, Ut, (uint64_t)r, (uint64_t)d, (uint32_t)r) != PLK_OK) return PLK_ERR_CUDA;
   int tcols = 32;
   while (tcols < r) tcols <<= 1;
-  const int smem = score_tc_smem(r);
+  const int smem_max = score_tc_smem(r, sc_stages(r));
   static int attr_smem[64] = {0};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return PLK_ERR_CUDA;
-  if (dev < 64 && attr_smem[dev] < smem) {
-    if (cudaFuncSetAttribute(score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  if (dev < 64 && attr_smem[dev] < smem_max) {
+    if (cudaFuncSetAttribute(score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_max) != cudaSuccess)
       return PLK_ERR_CUDA;
-    attr_smem[dev] = smem;
+    attr_smem[dev] = smem_max;
   }
   // K slices: grow the cluster while it still fits the GPU and leaves >= 2 k-blocks per slice.
   // The split needs the staged partial and the received slices ([128][r] fp32 each) inside the
   // stage ring: at r = 256 the ring is too small, and the kernel runs unsplit.
-  const int tiles = ceil_div(rows, 128), nkb = d / 64;
-  const int ring = sc_stages(r) * (kScA + ((r * 128 + 1023) & ~1023));
+  const int tiles = ceil_div(rows, 128), nkb = d / 64, sms = device_sm_count();
+  const int stage_bytes = kScA + ((r * 128 + 1023) & ~1023);
+  int stages = sc_stages(r);
+  const int ring = stages * stage_bytes;
   int S = 1;
-  while (S < 8 && tiles * S * 2 <= device_sm_count() && nkb % (S * 2) == 0 && nkb / (S * 2) >= 2 &&
-         2 * 128 * r * 4 <= ring)
+  while (S < 8 && tiles * S * 2 <= sms && nkb % (S * 2) == 0 && nkb / (S * 2) >= 2 && 2 * 128 * r * 4 <= ring)
     S *= 2;
+  // More row tiles than SMs: with one CTA per SM the tiles past the first wave run in a second,
+  // partly idle one.  Two CTAs per SM with half the ring each keep as many X loads in flight
+  // per SM and take every tile (up to two per SM) in one wave.
+  if (S == 1 && tiles > sms) {
+    const int fit = (score_tc_half_sm_smem() - 128 - 1024) / stage_bytes;
+    if (fit >= 2 && fit < stages) stages = fit;
+  }
+  const int smem = score_tc_smem(r, stages);
+  const int x_stream = (size_t)rows * d * 2 > ((size_t)64 << 20);  // more than half of the 126 MB L2
   if (S == 1) {
     return launch_pdl(score_tc_kernel, dim3(tiles), dim3(128), smem, st, tmX, tmU, rows, d, r, tcols, proxy_cache,
-                      proxy_out, score_out, metric);
+                      proxy_out, score_out, metric, stages, x_stream);
   } else {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(tiles, S, 1);
@@ -397,7 +432,7 @@ int launch_score(const plk_dims* dims, const void* X, const void* Ut, int r, con
     cfg.attrs = at;
     cfg.numAttrs = 2;
     if (cudaLaunchKernelEx(&cfg, score_tc_kernel, tmX, tmU, rows, d, r, tcols, proxy_cache, proxy_out, score_out,
-                           metric) != cudaSuccess)
+                           metric, stages, x_stream) != cudaSuccess)
       return PLK_ERR_CUDA;
   }
   return cudaPeekAtLastError() == cudaSuccess ? PLK_OK : PLK_ERR_CUDA;

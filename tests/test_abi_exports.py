@@ -73,6 +73,24 @@ def test_host_validation_without_gpu(built):
     assert lib.plk_score_drift(ctypes.byref(ok), p, p, 300, p, 0, None, p, None) == plk.ERR_ARG
     assert lib.plk_score_drift(ctypes.byref(ok), p, p, 8, p, 5, None, p, None) == plk.ERR_ARG
     assert lib.plk_score_drift(ctypes.byref(ok), p, p, 8, p, 0, p, p, None) == plk.ERR_ARG  # out aliases cache
+    # base addresses the kernels read with 16-byte vectors or TMA must be 16-byte aligned
+    odd, p48 = ctypes.c_void_p(24), ctypes.c_void_p(48)
+    for args in ((odd, p, p, None), (p, odd, p, None), (p, p, odd, None), (p, p, p48, odd)):
+        X, U, pc, po = args
+        assert lib.plk_score_drift(ctypes.byref(ok), X, U, 8, pc, 0, po, p, None) == plk.ERR_ARG, args
+    w_ok = plk.PlkWeights(*(16 * (i + 1) for i in range(6)))
+    for i in range(6):
+        w_bad = plk.PlkWeights(*(16 * (j + 1) + (8 if j == i else 0) for j in range(6)))
+        assert lib.plk_full_layer_step(ctypes.byref(ok), ctypes.byref(w_bad), p, p, p, p, None, 0, None) == \
+            plk.ERR_ARG, i
+    for pos in range(4):  # X, K_cache, V_cache, Y
+        a = [p, p, p, p]
+        a[pos] = odd
+        assert lib.plk_full_layer_step(ctypes.byref(ok), ctypes.byref(w_ok), *a, None, 0, None) == plk.ERR_ARG, pos
+        assert lib.plk_layer_step_partial(ctypes.byref(ok), ctypes.byref(w_ok), a[0], p, p, *a[1:], None, 0,
+                                          None) == plk.ERR_ARG, pos
+    assert lib.plk_layer_step_partial(ctypes.byref(ok), ctypes.byref(w_ok), p, ctypes.c_void_p(18), p, p, p, p,
+                                      None, 0, None) == plk.ERR_ARG  # idx on a 2-byte boundary
     assert lib.plk_set_wait_limit(0) == plk.ERR_ARG
     assert lib.plk_set_deterministic(2) == plk.ERR_ARG
     assert lib.plk_set_deterministic(0) == plk.OK

@@ -183,6 +183,55 @@ def test_score_drift_8b_shape_repeated(plk):
         assert_f32_close(host(score), ref_s, f"score, run {run}", tol=1e-4)
 
 
+@pytest.mark.parametrize("rank,metric", [(128, "l2"), (256, "cos"), (16, "cos")])
+def test_score_drift_more_tiles_than_sms(plk, rank, metric):
+    """21000 rows at d = 1024: 165 row tiles (the last one ragged) against 148 SMs, so the
+    launch runs unsplit with two CTAs per SM and a shallower stage ring (3 stages at rank 128,
+    2 at rank 256; rank 16 keeps its full ring).  Every row against the oracle."""
+    D, r = synth.Dims(B=3, N=7000, d=1024, H=8, hd=128, F=512, dtype="bf16"), rank
+    X = synth.hidden_states(D, seed=7)
+    Ut = synth.proxy_basis(D.d, r, seed=7)
+    p_exact = oracle.proxy_project(X.reshape(-1, D.d).astype(np.float64), Ut.astype(np.float64))
+    rng = np.random.default_rng(7)
+    pc = p_exact + (rng.random(D.B * D.N) < 0.3)[:, None] * rng.standard_normal(p_exact.shape) * 0.5
+    pc = pc.astype(np.float32).reshape(D.B, D.N, r)
+    ref_s, ref_p = oracle.score_drift(X.astype(np.float64), Ut.astype(np.float64), pc, metric)
+    gs = Guarded((D.B, D.N), torch.float32)
+    gp = Guarded((D.B, D.N, r), torch.float32)
+    plk.score_drift(pdims(plk, D), dev(X, BF), dev(Ut, BF), r, dev(pc, torch.float32),
+                    plk.METRIC_COS if metric == "cos" else plk.METRIC_L2, gs.t, proxy_out=gp.t)
+    torch.cuda.synchronize()
+    assert_f32_close(host(gp.t), ref_p, "proxy", tol=1e-5)
+    assert_f32_close(host(gs.t), ref_s, "score", tol=1e-4)
+    check_guards({"score": gs, "proxy_out": gp}, "score_drift")
+
+
+def test_score_drift_scoring_shape_sampled(plk):
+    """The scoring launch at its full size (8 sequences x 4096 rows x 4096, rank 128, L2 drift:
+    256 row tiles, two CTAs per SM), checked against the oracle on 1024 sampled rows plus the
+    first and last row of every sequence; every score finite.  Both outputs are fp32 and take the
+    fp32 bound (1e-4): over 4096 bf16 products the tensor cores' fp32 accumulation reaches ~1.6e-5
+    of the proxies' rms on some of these rows."""
+    D, r = synth.SCORE_8B, synth.PROXY_RANK_8B
+    X = synth.hidden_states(D, seed=6).reshape(-1, D.d)
+    Ut = synth.proxy_basis(D.d, r, seed=6)
+    rng = np.random.default_rng(6)
+    pc = rng.standard_normal((D.B * D.N, r)).astype(np.float32)
+    rows = np.unique(np.concatenate([rng.choice(D.B * D.N, 1024, replace=False),
+                                     np.arange(0, D.B * D.N, D.N), np.arange(D.N - 1, D.B * D.N, D.N)]))
+    ref_s, ref_p = oracle.score_drift(X[rows][None].astype(np.float64), Ut.astype(np.float64), pc[rows][None], "l2")
+    score = torch.full((D.B, D.N), float("nan"), dtype=torch.float32, device="cuda")
+    pout = torch.full((D.B, D.N, r), float("nan"), dtype=torch.float32, device="cuda")
+    Xd = dev(X, BF)
+    del X
+    plk.score_drift(pdims(plk, D), Xd, dev(Ut, BF), r, dev(pc, torch.float32), plk.METRIC_L2, score, proxy_out=pout)
+    torch.cuda.synchronize()
+    s_all = host(score).reshape(-1)
+    assert np.all(np.isfinite(s_all)), "score: non-finite values"
+    assert_f32_close(s_all[rows], ref_s[0], "score (sampled rows)", tol=1e-4)
+    assert_f32_close(host(pout).reshape(-1, r)[rows], ref_p[0], "proxy (sampled rows)")
+
+
 def test_proxy_commit(plk):
     B, N, r = 3, 50, 16
     rng = np.random.default_rng(4)
