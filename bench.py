@@ -561,7 +561,7 @@ def _timed(torch, fn, steps, warmup):
     return statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3 / reps
 
 
-def run_kernel_configs(args):
+def run_kernel_configs(args, scoring_only=False):
     import torch
     import partial_recompute_kv_b200 as plk
     import synth
@@ -600,6 +600,8 @@ def run_kernel_configs(args):
                     "scoring_layer_us": score_us + us,
                     "scoring_32_layers_us": 32 * (score_us + us)})
     del X, pc, pnew
+    if scoring_only:
+        return _configs_done(torch, plk, clk, out)
     # stack step 0: B = 4, N = 2048, every row active
     D = synth.STACK_8B
     dm = plk.dims(D.B, D.N, D.d, D.H, D.hd, D.F, D.eps, plk.BF16)
@@ -660,6 +662,10 @@ def run_kernel_configs(args):
     out.append({"kernel": "layer step, grouped-query attention", "config": f"d={d_} H={H_} Hkv={Hkv_} F={F_} "
                 f"N={N_} M={M_}", "us": us_g, "active_token_layers_per_s": M_ / (us_g * 1e-6),
                 "TFLOP/s": fl / (us_g * 1e-6) / 1e12, "frac_of_peak": fl / (us_g * 1e-6) / 1e12 / tfl})
+    return _configs_done(torch, plk, clk, out)
+
+
+def _configs_done(torch, plk, clk, out):
     st = plk.get_status()
     if st != plk.OK:
         raise RuntimeError(f"device status {plk.error_string(st)}")
@@ -1106,12 +1112,14 @@ def main():
                     help="enqueue the step's library calls directly every step")
     ap.add_argument("--frac", type=float, default=0.25,
                     help="active fraction M/N of the headline step (the metric is quoted at 0.25)")
-    ap.add_argument("--kernel", choices=["step", "sweep", "kl_lock", "slowfast", "configs", "stack", "long"],
+    ap.add_argument("--kernel", choices=["step", "sweep", "kl_lock", "slowfast", "configs", "scoring", "stack",
+                                         "long"],
                     default="step",
                     help="step: the headline layer step; sweep: the step at every active fraction 1, 1/2, 1/4, "
                          "1/10, 1/20; kl_lock: the KL lock rule alone; slowfast: the SlowFast "
                          "span policy over whole decodes; configs: scoring and the all-active stack step at the "
-                         "shapes where their rooflines are judged; stack: the 32-layer stack over the 256-step "
+                         "shapes where their rooflines are judged; scoring: the first of those alone (score and "
+                         "top-k at 8 x 4096); stack: the 32-layer stack over the 256-step "
                          "schedule; long: the long-context block decode at N = 8192")
     ap.add_argument("--profile", action="store_true",
                     help="set up and run --steps steps without timing or output (for ncu)")
@@ -1129,8 +1137,8 @@ def main():
         return run_stack(args) if rank == 0 else 0
     if args.kernel == "long":
         return run_long(args) if rank == 0 else 0
-    if args.kernel == "configs":
-        return run_kernel_configs(args) if rank == 0 else 0
+    if args.kernel in ("configs", "scoring"):
+        return run_kernel_configs(args, scoring_only=args.kernel == "scoring") if rank == 0 else 0
     if args.kernel == "sweep":
         return run_sweep(args) if rank == 0 else 0
     if args.impl == "reference":
