@@ -342,6 +342,41 @@ int plk_denoise_step_host(const plk_dims* dims, const plk_weights* w, const void
 /* Workspace of plk_denoise_step_host (0 for invalid dims or r). */
 size_t plk_step_workspace_bytes(const plk_dims* dims, int r);
 
+/*
+ * T consecutive denoising steps of one layer from host memory, with the host
+ * copies overlapped with the compute of neighbouring steps.  Step t (t < T) is
+ * plk_denoise_step_host with X_hosts[t] in and Y_hosts[t] out: it reads the
+ * layer input X_hosts[t] ([B, N, d], host, layer dtype) and leaves in
+ * Y_hosts[t] ([B, N, d], host) the output cache Y as it stands after step t.
+ * lock, proxy_cache, K_cache, V_cache and Y carry over from step to step as in
+ * T separate calls, and the results are those of T separate calls.
+ *   - upload_stream copies X_hosts[t + 1] into a second device buffer while
+ *     step t computes on `stream`;
+ *   - after step t, Y is copied on the device into one of two snapshot buffers
+ *     (step t + 1 updates Y in place), and download_stream copies the snapshot
+ *     to Y_hosts[t] while step t + 1 computes.
+ * Each step still moves its whole X in and its whole Y out; the copies of
+ * consecutive steps run concurrently with the compute (on separate copy
+ * engines when the host buffers are pinned).  The three streams are the
+ * caller's (upload_stream and download_stream should be two further streams;
+ * passing `stream` for them runs everything in order).  The copies start after
+ * the work already enqueued on `stream`, and `stream` waits for the last
+ * download: synchronise `stream` before reading any Y_hosts[t].  Y_hosts[t]
+ * may repeat (the downloads run in step order).  workspace: at least
+ * plk_steps_workspace_bytes(dims, r) bytes, 256-byte aligned, not shared with
+ * a concurrent call.  Errors: PLK_ERR_ARG for T < 1 or a null X_hosts[t] or
+ * Y_hosts[t], then those of plk_denoise_step_host, all checked before anything
+ * is enqueued; PLK_ERR_CUDA when a copy or launch fails part way (synchronise
+ * all three streams before reusing the buffers).
+ */
+int plk_denoise_steps_host(const plk_dims* dims, const plk_weights* w, const void* Ut, int r, int metric,
+                           int mode, float tau, int k, float* proxy_cache, uint8_t* lock,
+                           void* K_cache, void* V_cache, void* Y, int T, const void* const* X_hosts,
+                           void* const* Y_hosts, void* workspace, size_t ws_bytes, void* stream,
+                           void* upload_stream, void* download_stream);
+/* Workspace of plk_denoise_steps_host (0 for invalid dims or r). */
+size_t plk_steps_workspace_bytes(const plk_dims* dims, int r);
+
 /* Synchronises `stream`, returns the device status word of the current device
  * (PLK_OK or PLK_ERR_TIMEOUT) and clears it. */
 int plk_get_status(void* stream);

@@ -26,7 +26,8 @@ SEL_THRESH_GT, SEL_THRESH_LT, SEL_TOPK_LARGEST, SEL_TOPK_SMALLEST = 0, 1, 2, 3
 EXPORTED = (
     "plk_score_drift", "plk_select_active", "plk_layer_step_partial", "plk_full_layer_step",
     "plk_proxy_commit", "plk_layer_step_partial_static", "plk_kl_lock", "plk_slowfast_step", "plk_workspace_bytes",
-    "plk_denoise_step", "plk_denoise_step_host", "plk_step_workspace_bytes",
+    "plk_denoise_step", "plk_denoise_step_host", "plk_step_workspace_bytes", "plk_denoise_steps_host",
+    "plk_steps_workspace_bytes",
     "plk_get_status",
     "plk_set_wait_limit", "plk_set_deterministic",
     "plk_selftest_wait_timeout", "plk_selftest_exp2", "plk_trace_events", "plk_error_string", "plk_version",
@@ -79,6 +80,9 @@ def _load():
         "plk_denoise_step": (I, [V, W, P, I, I, I, F, I, P, P, P, P, P, P, P, S, P]),
         "plk_denoise_step_host": (I, [V, W, P, I, I, I, F, I, P, P, P, P, P, P, P, P, S, P]),
         "plk_step_workspace_bytes": (S, [V, I]),
+        "plk_denoise_steps_host": (I, [V, W, P, I, I, I, F, I, P, P, P, P, P, I, ctypes.POINTER(P),
+                                       ctypes.POINTER(P), P, S, P, P, P]),
+        "plk_steps_workspace_bytes": (S, [V, I]),
         "plk_get_status": (I, [P]),
         "plk_set_wait_limit": (I, [L]),
         "plk_set_deterministic": (I, [I]),
@@ -227,6 +231,37 @@ def denoise_step_host(dm, w, Ut, r, metric, mode, tau, k, proxy_cache, lock, K_c
                                      _ptr(V_cache), _ptr(Y), _hptr(X_host), _hptr(Y_host), _ptr(workspace),
                                      workspace.numel() * workspace.element_size(), _stream(stream)),
            "denoise_step_host")
+
+
+def steps_workspace_bytes(dm, r) -> int:
+    return int(lib.plk_steps_workspace_bytes(ctypes.byref(dm), int(r)))
+
+
+def alloc_steps_workspace(dm, r, device="cuda"):
+    n = steps_workspace_bytes(dm, r)
+    if n == 0:
+        raise PlkError(ERR_SHAPE, "steps_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def denoise_steps_host(dm, w, Ut, r, metric, mode, tau, k, proxy_cache, lock, K_cache, V_cache, Y, X_hosts,
+                       Y_hosts, workspace, upload_stream, download_stream, stream=None):
+    """len(X_hosts) consecutive whole steps from host memory (see plk_denoise_steps_host): step t
+    reads X_hosts[t] and leaves Y after it in Y_hosts[t]; the uploads and downloads run on
+    upload_stream / download_stream (torch.cuda.Stream) beside the compute on `stream`.  Host
+    tensors are CPU tensors (pinned)."""
+    if len(X_hosts) != len(Y_hosts):
+        raise ValueError("X_hosts and Y_hosts differ in length")
+    pw = w if isinstance(w, PlkWeights) else weights(w)
+    T = len(X_hosts)
+    xs = (ctypes.c_void_p * T)(*(_hptr(x) for x in X_hosts))
+    ys = (ctypes.c_void_p * T)(*(_hptr(y) for y in Y_hosts))
+    _check(lib.plk_denoise_steps_host(ctypes.byref(dm), ctypes.byref(pw), _ptr(Ut), int(r), int(metric), int(mode),
+                                      float(tau), int(k), _ptr(proxy_cache), _ptr(lock), _ptr(K_cache),
+                                      _ptr(V_cache), _ptr(Y), T, xs, ys, _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(), _stream(stream),
+                                      _stream(upload_stream), _stream(download_stream)),
+           "denoise_steps_host")
 
 
 def full_layer_step(dm, w, X, K_cache, V_cache, Y, workspace, stream=None):

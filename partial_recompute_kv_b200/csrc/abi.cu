@@ -274,6 +274,103 @@ int plk_denoise_step_host(const plk_dims* dims, const plk_weights* w, const void
   return PLK_OK;
 }
 
+}  // extern "C"
+
+namespace plk {
+// Workspace of plk_denoise_steps_host: the one-step layout, then a second X buffer and two
+// snapshots of Y (the inputs and outputs of consecutive steps in flight).
+struct StepsWs {
+  StepWs one;
+  size_t x2 = 0, y0 = 0, y1 = 0, total = 0;
+};
+static StepsWs steps_ws_layout(const plk_dims* d, int r) {
+  StepsWs s;
+  s.one = step_ws_layout(d, r);
+  const size_t bytes = (size_t)d->B * d->N * d->d * (d->dtype == PLK_BF16 ? 2 : 4);
+  s.x2 = up256(s.one.total);
+  s.y0 = up256(s.x2 + bytes);
+  s.y1 = up256(s.y0 + bytes);
+  s.total = up256(s.y1 + bytes);
+  return s;
+}
+
+// The events of one plk_denoise_steps_host call, destroyed with it (a recorded event that has
+// not completed is released by the driver once it does).
+struct StepEvents {
+  cudaEvent_t up[2] = {}, comp[2] = {}, down[2] = {}, start = nullptr;
+  bool ok = true;
+  StepEvents() {
+    for (cudaEvent_t* e : {&up[0], &up[1], &comp[0], &comp[1], &down[0], &down[1], &start})
+      ok = ok && cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
+  }
+  ~StepEvents() {
+    for (cudaEvent_t e : {up[0], up[1], comp[0], comp[1], down[0], down[1], start})
+      if (e) cudaEventDestroy(e);
+  }
+};
+}  // namespace plk
+
+extern "C" {
+
+size_t plk_steps_workspace_bytes(const plk_dims* dims, int r) {
+  if (plk_step_workspace_bytes(dims, r) == 0) return 0;
+  return steps_ws_layout(dims, r).total;
+}
+
+int plk_denoise_steps_host(const plk_dims* dims, const plk_weights* w, const void* Ut, int r, int metric,
+                           int mode, float tau, int k, float* proxy_cache, uint8_t* lock, void* K_cache,
+                           void* V_cache, void* Y, int T, const void* const* X_hosts, void* const* Y_hosts,
+                           void* workspace, size_t ws_bytes, void* stream, void* upload_stream,
+                           void* download_stream) {
+  if (T < 1 || !X_hosts || !Y_hosts) return PLK_ERR_ARG;
+  for (int t = 0; t < T; ++t)
+    if (!X_hosts[t] || !Y_hosts[t]) return PLK_ERR_ARG;
+  int e = check_step_args(dims, w, Ut, r, metric, mode, k, proxy_cache, lock, K_cache, V_cache, Y, X_hosts[0]);
+  if (e != PLK_OK) return e;
+  const StepsWs L = steps_ws_layout(dims, r);
+  if (!workspace || ws_bytes < L.total) return PLK_ERR_WORKSPACE;
+  uint8_t* ws = (uint8_t*)workspace;
+  void* Xb[2] = {ws + L.one.x, ws + L.x2};
+  void* Ys[2] = {ws + L.y0, ws + L.y1};
+  const size_t bytes = (size_t)dims->B * dims->N * dims->d * (dims->dtype == PLK_BF16 ? 2 : 4);
+  cudaStream_t S = (cudaStream_t)stream, U = (cudaStream_t)upload_stream, D = (cudaStream_t)download_stream;
+  StepEvents ev;
+  if (!ev.ok) return PLK_ERR_CUDA;
+#define PLK_CU(x) \
+  if ((x) != cudaSuccess) return PLK_ERR_CUDA
+  // the copy streams start after the work already on `stream` (an earlier call's use of the
+  // workspace included)
+  PLK_CU(cudaEventRecord(ev.start, S));
+  PLK_CU(cudaStreamWaitEvent(U, ev.start, 0));
+  PLK_CU(cudaStreamWaitEvent(D, ev.start, 0));
+  PLK_CU(cudaMemcpyAsync(Xb[0], X_hosts[0], bytes, cudaMemcpyHostToDevice, U));
+  PLK_CU(cudaEventRecord(ev.up[0], U));
+  for (int t = 0; t < T; ++t) {
+    const int b = t & 1, nb = b ^ 1;
+    if (t + 1 < T) {  // the next input, into the buffer step t - 1 read
+      if (t >= 1) PLK_CU(cudaStreamWaitEvent(U, ev.comp[nb], 0));
+      PLK_CU(cudaMemcpyAsync(Xb[nb], X_hosts[t + 1], bytes, cudaMemcpyHostToDevice, U));
+      PLK_CU(cudaEventRecord(ev.up[nb], U));
+    }
+    PLK_CU(cudaStreamWaitEvent(S, ev.up[b], 0));
+    if ((e = run_step(dims, w, Ut, r, metric, mode, tau, k, proxy_cache, lock, K_cache, V_cache, Y, Xb[b], ws,
+                      L.one, S)) != PLK_OK)
+      return e;
+    // Y after step t, snapshotted (step t + 1 updates Y in place) once the download of step
+    // t - 2 has read that snapshot buffer
+    if (t >= 2) PLK_CU(cudaStreamWaitEvent(S, ev.down[b], 0));
+    PLK_CU(cudaMemcpyAsync(Ys[b], Y, bytes, cudaMemcpyDeviceToDevice, S));
+    PLK_CU(cudaEventRecord(ev.comp[b], S));
+    PLK_CU(cudaStreamWaitEvent(D, ev.comp[b], 0));
+    PLK_CU(cudaMemcpyAsync(Y_hosts[t], Ys[b], bytes, cudaMemcpyDeviceToHost, D));
+    PLK_CU(cudaEventRecord(ev.down[b], D));
+  }
+  // `stream` ends after the last download (the downloads run in step order on one stream)
+  PLK_CU(cudaStreamWaitEvent(S, ev.down[(T - 1) & 1], 0));
+#undef PLK_CU
+  return PLK_OK;
+}
+
 int plk_get_status(void* stream) {
   if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return PLK_ERR_CUDA;
   int v = PLK_OK;

@@ -91,6 +91,14 @@ def test_host_validation_without_gpu(built):
                                           None) == plk.ERR_ARG, pos
     assert lib.plk_layer_step_partial(ctypes.byref(ok), ctypes.byref(w_ok), p, ctypes.c_void_p(18), p, p, p, p,
                                       None, 0, None) == plk.ERR_ARG  # idx on a 2-byte boundary
+    # the pipelined steps: T >= 1 and a host buffer for every step's X and Y
+    hs = (ctypes.c_void_p * 2)(16, 32)
+    hole = (ctypes.c_void_p * 2)(16, None)
+    steps = lib.plk_denoise_steps_host
+    for T, xs, ys in ((0, hs, hs), (2, None, hs), (2, hs, None), (2, hole, hs), (2, hs, hole)):
+        assert steps(ctypes.byref(ok), ctypes.byref(w_ok), p, 8, 0, plk.SEL_TOPK_LARGEST, 0.0, 1, p, p, p, p, p, T,
+                     xs, ys, p, 1 << 30, None, None, None) == plk.ERR_ARG, (T, xs, ys)
+    assert lib.plk_steps_workspace_bytes(ctypes.byref(bad_width), 8) == 0
     assert lib.plk_set_wait_limit(0) == plk.ERR_ARG
     assert lib.plk_set_deterministic(2) == plk.ERR_ARG
     assert lib.plk_set_deterministic(0) == plk.OK

@@ -877,3 +877,106 @@ def test_denoise_step_matches_oracle(plk, entry):
         assert np.array_equal(Y_host.to(torch.float64).numpy(), Yd), "Y_host is the device Y"
     _check_layer_rows(host(g["K"].t), host(g["V"].t), Yd, ref, base, ref_lock, f"{entry} step")
     assert_f32_close(host(g["proxy"].t), ref_pc, "proxy cache", tol=1e-5)
+
+
+def _steps_case():
+    """Four denoising steps at a small bf16 shape: step t moves a shrinking subset of the rows the
+    previous step moved, so threshold locking (L2 drift below tau) shrinks the active set
+    120 -> 80 -> 40 -> 8 rows per sequence."""
+    D = synth.Dims(B=2, N=320, d=512, H=4, hd=128, F=1536, dtype="bf16")
+    r, tau = 128, 0.05
+    W = synth.layer_weights(D, 0.02, seed=15)
+    X0 = synth.hidden_states(D, seed=15)
+    Ut = synth.proxy_basis(D.d, r, seed=15)
+    base = oracle.full_layer_step(D, W, X0, "bf16")
+    pc0 = oracle.to_f32(oracle.proxy_project(X0.reshape(-1, D.d).astype(np.float64), Ut.astype(np.float64)))
+    pc0 = pc0.astype(np.float32).reshape(D.B, D.N, r)
+    Xs, moved, Xc = [], np.ones((D.B, D.N), bool), X0
+    for t, cnt in enumerate((120, 80, 40, 8)):
+        m = np.zeros((D.B, D.N), bool)
+        for b in range(D.B):
+            pool = np.flatnonzero(moved[b])
+            m[b, pool[synth.uniform_positions(0, pool.size, cnt, seed=15 + t, tag=b)]] = True
+        Xc = synth.perturb_rows(Xc, synth.step_noise((D.B, D.N, D.d), 0.25, seed=15, step=t), m, "bf16")
+        Xs.append(Xc)
+        moved = m
+    return D, r, tau, W, Ut, base, pc0, Xs
+
+
+@pytest.mark.parametrize("streams", ["separate", "same"])
+def test_denoise_steps_host_pipelined(plk, streams):
+    """plk_denoise_steps_host (each step's upload and download on their own streams beside the
+    compute of the neighbouring steps) against the same steps as separate plk_denoise_step_host
+    calls, bit for bit in reproducible mode, and against the oracle's chain of steps (threshold
+    lock bit-exact, K, V and every step's Y within the bf16 bounds).  "same": all three streams
+    are one, and every step's Y goes to the same host buffer (it ends with the last step's Y)."""
+    D, r, tau, W, Ut, base, pc0, Xs = _steps_case()
+    T = len(Xs)
+    # the oracle's chain: score -> lock (drift below tau) -> partial layer step -> proxy refresh
+    state, pc, lock = base, pc0, np.zeros((D.B, D.N), np.uint8)
+    ref_Y, ref_locks = [], []
+    for X in Xs:
+        s, p = oracle.score_drift(X.astype(np.float64), Ut.astype(np.float64), pc, "l2")
+        lock = oracle.lock_threshold(s.astype(np.float32).astype(np.float64), lock, tau, greater=False)
+        idx, seg = oracle.compact(lock)
+        state = oracle.layer_step_partial(D, W, X, idx, seg, state, "bf16")
+        pc = oracle.proxy_commit(pc, p, idx).astype(np.float32)
+        ref_Y.append(state.Y)
+        ref_locks.append(lock.copy())
+    assert [int((l == 0).sum()) for l in ref_locks] == [240, 160, 80, 16]
+
+    dm, Wd, Ud = pdims(plk, D), weights_dev(W, D), dev(Ut, BF)
+    X_hosts = [torch.from_numpy(np.ascontiguousarray(X)).to(BF).pin_memory() for X in Xs]
+
+    def fresh():
+        return {"K": Guarded(base.K.shape, BF, init=dev(base.K, BF)), "V": Guarded(base.V.shape, BF, init=dev(base.V, BF)),
+                "Y": Guarded(base.Y.shape, BF, init=dev(base.Y, BF)),
+                "proxy": Guarded(pc0.shape, torch.float32, init=pc0),
+                "lock": Guarded((D.B, D.N), torch.uint8, fill=0)}
+
+    plk.set_deterministic(True)
+    try:
+        # the same steps as separate calls
+        gs = fresh()
+        sws = plk.alloc_step_workspace(dm, r)
+        seq_Y = []
+        for t in range(T):
+            Yh = torch.full(base.Y.shape, -3.0, dtype=BF).pin_memory()
+            plk.denoise_step_host(dm, Wd, Ud, r, plk.METRIC_L2, plk.SEL_THRESH_LT, tau, 0, gs["proxy"].t,
+                                  gs["lock"].t, gs["K"].t, gs["V"].t, gs["Y"].t, X_hosts[t], Yh, sws)
+            torch.cuda.synchronize()
+            assert np.array_equal(host(gs["lock"].t), ref_locks[t]), f"separate calls: lock after step {t}"
+            seq_Y.append(Yh.to(torch.float64).numpy())
+        # pipelined
+        g = fresh()
+        n = plk.steps_workspace_bytes(dm, r)
+        assert n > plk.step_workspace_bytes(dm, r)
+        g["workspace"] = Guarded((n,), torch.uint8)
+        if streams == "separate":
+            up, down = torch.cuda.Stream(), torch.cuda.Stream()
+            Y_hosts = [torch.full(base.Y.shape, -3.0, dtype=BF).pin_memory() for _ in range(T)]
+        else:
+            up = down = torch.cuda.current_stream()
+            Y_hosts = [torch.full(base.Y.shape, -3.0, dtype=BF).pin_memory()] * T
+        plk.denoise_steps_host(dm, Wd, Ud, r, plk.METRIC_L2, plk.SEL_THRESH_LT, tau, 0, g["proxy"].t, g["lock"].t,
+                               g["K"].t, g["V"].t, g["Y"].t, X_hosts, Y_hosts, g["workspace"].t, up, down)
+        torch.cuda.current_stream().synchronize()  # the call's stream waits for the last download
+        assert plk.get_status() == plk.OK
+    finally:
+        plk.set_deterministic(False)
+    check_guards(g, f"denoise_steps_host ({streams})")
+    assert np.array_equal(host(g["lock"].t), ref_locks[-1])
+    for name in ("K", "V", "Y", "proxy"):
+        assert np.array_equal(host(g[name].t), host(gs[name].t)), f"{name} differs from the separate calls"
+    got = [y.to(torch.float64).numpy() for y in Y_hosts]
+    steps = range(T) if streams == "separate" else [T - 1]
+    for t in steps:
+        assert np.array_equal(got[t], seq_Y[t]), f"Y_hosts[{t}] differs from the separate call's Y"
+        never = ref_locks[0].astype(bool)  # locked at step 0: Y keeps the base rows
+        assert np.array_equal(got[t][never], base.Y[never]), f"step {t}: a row locked from the start was written"
+        act = ~never
+        assert_bf16_close(got[t][act], ref_Y[t][act], f"pipelined step {t} Y")
+    K, V = host(g["K"].t), host(g["V"].t)
+    act = ~ref_locks[0].astype(bool)
+    assert_bf16_close(K[act], state.K[act], "pipelined K")
+    assert_bf16_close(V[act], state.V[act], "pipelined V")
