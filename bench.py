@@ -475,10 +475,11 @@ def run_gpu(args, wl, dist, rank, world, local_rank):
     steps_call(3)  # warm-up
     torch.cuda.synchronize()
     pa, pb = E(), E()
-    pa.record()
-    steps_call(e2e_steps)
-    pb.record()
-    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk_e2e:  # a short run: its clocks may differ from the value's
+        pa.record()
+        steps_call(e2e_steps)
+        pb.record()
+        torch.cuda.synchronize()
     if plk.get_status() != plk.OK:
         raise RuntimeError("device status after the pipelined host-buffer steps")
     if int((lock_e == 0).sum()) != M:
@@ -488,7 +489,7 @@ def run_gpu(args, wl, dist, rank, world, local_rank):
            "h2d_bytes_per_step": Xp_host.numel() * Xp_host.element_size(),
            "d2h_bytes_per_step": Y_pair[0].numel() * Y_pair[0].element_size(), "ms_per_step": e2e_ms,
            "api": f"plk_denoise_steps_host over {e2e_steps} consecutive steps (host X in, host Y out every "
-                  "step; the copies overlap the neighbouring steps' compute)",
+                  "step; the copies overlap the neighbouring steps' compute)", "clocks": clk_e2e.summary(),
            "single_call_per_step": {"value": world * M / (single_ms / 1e3), "ms_per_step": single_ms,
                                     "api": "plk_denoise_step_host, one call per step (copies in line)"}}
     step_flops = M * wl.flops_per_row()
