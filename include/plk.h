@@ -60,7 +60,7 @@ extern "C" {
 #define PLK_ERR_DTYPE     -3  /* unknown dtype                                 */
 #define PLK_ERR_CUDA      -4  /* a CUDA runtime/driver call failed             */
 #define PLK_ERR_TIMEOUT   -5  /* a device wait gave up (from plk_get_status)   */
-#define PLK_ERR_WORKSPACE -6  /* workspace missing or smaller than required    */
+#define PLK_ERR_WORKSPACE -6  /* workspace missing, not 256-byte aligned, or smaller than required */
 
 /* dtypes */
 #define PLK_F32  0

@@ -63,7 +63,7 @@ const char* plk_error_string(int code) {
     case PLK_ERR_DTYPE: return "unknown dtype";
     case PLK_ERR_CUDA: return "CUDA call failed";
     case PLK_ERR_TIMEOUT: return "device wait exceeded its limit";
-    case PLK_ERR_WORKSPACE: return "workspace missing or too small";
+    case PLK_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     default: return "unknown error code";
   }
 }
@@ -248,7 +248,7 @@ int plk_denoise_step(const plk_dims* dims, const plk_weights* w, const void* Ut,
   if (e != PLK_OK) return e;
   if (!aligned16(X)) return PLK_ERR_ARG;
   const StepWs L = step_ws_layout(dims, r);
-  if (!workspace || ws_bytes < L.total) return PLK_ERR_WORKSPACE;
+  if (!workspace || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return PLK_ERR_WORKSPACE;
   return run_step(dims, w, Ut, r, metric, mode, tau, k, proxy_cache, lock, K_cache, V_cache, Y, X,
                   (uint8_t*)workspace, L, (cudaStream_t)stream);
 }
@@ -261,7 +261,7 @@ int plk_denoise_step_host(const plk_dims* dims, const plk_weights* w, const void
   if (e != PLK_OK) return e;
   if (!Y_host) return PLK_ERR_ARG;
   const StepWs L = step_ws_layout(dims, r);
-  if (!workspace || ws_bytes < L.total) return PLK_ERR_WORKSPACE;
+  if (!workspace || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return PLK_ERR_WORKSPACE;
   uint8_t* ws = (uint8_t*)workspace;
   void* X = ws + L.x;
   const size_t BN = (size_t)dims->B * dims->N, es = dims->dtype == PLK_BF16 ? 2 : 4;
@@ -328,7 +328,7 @@ int plk_denoise_steps_host(const plk_dims* dims, const plk_weights* w, const voi
   int e = check_step_args(dims, w, Ut, r, metric, mode, k, proxy_cache, lock, K_cache, V_cache, Y, X_hosts[0]);
   if (e != PLK_OK) return e;
   const StepsWs L = steps_ws_layout(dims, r);
-  if (!workspace || ws_bytes < L.total) return PLK_ERR_WORKSPACE;
+  if (!workspace || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return PLK_ERR_WORKSPACE;
   uint8_t* ws = (uint8_t*)workspace;
   void* Xb[2] = {ws + L.one.x, ws + L.x2};
   void* Ys[2] = {ws + L.y0, ws + L.y1};

@@ -799,7 +799,7 @@ int run_layer(const plk_dims* dm, const plk_weights* w, const void* X, const int
   const int nsm = device_sm_count();
   if (nsm <= 0) return PLK_ERR_CUDA;
   const Workspace L = workspace_layout(dm, nsm);
-  if (!ws || ws_bytes < L.total) return PLK_ERR_WORKSPACE;
+  if (!ws || ws_bytes < L.total || (reinterpret_cast<uintptr_t>(ws) & 255u)) return PLK_ERR_WORKSPACE;
   uint8_t* wsb = (uint8_t*)ws;
   if (full) {
     int32_t* iota = (int32_t*)(wsb + L.iota);

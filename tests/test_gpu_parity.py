@@ -439,6 +439,15 @@ def test_workspace_too_small_is_rejected(plk):
     with pytest.raises(plk.PlkError) as e:
         plk.full_layer_step(dm, W, X, X.clone(), X.clone(), X.clone(), small)
     assert e.value.code == plk.ERR_WORKSPACE
+    # large enough but not on a 256-byte boundary: refused as well, nothing enqueued
+    n = plk.workspace_bytes(dm)
+    raw = torch.empty(n + 256, dtype=torch.uint8, device="cuda")
+    for off in (16, 128):
+        with pytest.raises(plk.PlkError) as e:
+            plk.full_layer_step(dm, W, X, X.clone(), X.clone(), X.clone(), raw[off:off + n])
+        assert e.value.code == plk.ERR_WORKSPACE, off
+    torch.cuda.synchronize()
+    assert plk.get_status() == plk.OK
 
 
 # ---------------------------------------------------------------------------
