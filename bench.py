@@ -1136,7 +1136,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["plk", "reference"], default="plk")
     ap.add_argument("--l2", choices=["stream", "flush"], default="stream",
-                    help="stream: no flush between steps (the weights alone are 3.4x L2); "
+                    help="stream: no flush between steps (the weights alone are 3.5x L2); "
                          "flush: write 256 MiB before every step")
     ap.add_argument("--graph", dest="graph", action="store_true", default=True,
                     help="replay the step as one captured CUDA graph (default)")
