@@ -454,12 +454,15 @@ def test_workspace_too_small_is_rejected(plk):
 # the tiny fp32 workload: 20 denoising steps, every step checked
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("noise_var", [synth.TINY_NOISE_VAR, 0.1])
-@pytest.mark.parametrize("entry", ["calls", "step"])
+@pytest.mark.parametrize("entry", ["calls", "step", "steps"])
 def test_tiny_fp32_driver(plk, noise_var, entry):
     """The tiny fp32 workload step by step.  With its own noise (variance 0.01) the active set
     empties within four steps; with variance 0.1 it shrinks from 13 rows to 1 over the 20 steps,
     so the fp32 layer runs on several rows at every step (decision margins >= 2e-4 from tau).
-    entry "calls": the four API calls of a step; "step": one plk_denoise_step per step."""
+    entry "calls": the four API calls of a step; "step": one plk_denoise_step per step; "steps":
+    all 20 steps in one plk_denoise_steps_host call from host buffers (the inputs built up front
+    from the oracle's locks, which the other entries match bit for bit), every step's Y
+    checked."""
     D = synth.TINY
     r = synth.TINY_RANK
     W = synth.layer_weights(D, 1.0 / math.sqrt(D.d))
@@ -487,6 +490,26 @@ def test_tiny_fp32_driver(plk, noise_var, entry):
     idx, seg = sel_bufs(D.B, D.N)
     sws = plk.alloc_step_workspace(dm, r) if entry == "step" else None
     X = X0.copy()
+    if entry == "steps":
+        X_hosts, act = [], lock0 == 0
+        for t, eps in enumerate(noises):
+            X = perturb(X, eps, act)
+            X_hosts.append(torch.from_numpy(np.ascontiguousarray(X, dtype=np.float32)).pin_memory())
+            act = recs[t]["lock"] == 0
+        Y_hosts = [torch.full((D.B, D.N, D.d), float("nan"), dtype=f32).pin_memory() for _ in noises]
+        gws = Guarded((plk.steps_workspace_bytes(dm, r),), torch.uint8)
+        plk.denoise_steps_host(dm, Wd, Utd, r, plk.METRIC_COS, plk.SEL_THRESH_GT, synth.TINY_TAU, 0, pc, lock, K, V,
+                               Y, X_hosts, Y_hosts, gws.t, torch.cuda.Stream(), torch.cuda.Stream())
+        torch.cuda.current_stream().synchronize()
+        assert plk.get_status() == plk.OK
+        gws.check("denoise_steps_host: workspace")
+        for t, rec in enumerate(recs):
+            assert_f32_close(Y_hosts[t].numpy().astype(np.float64), rec["Y"], f"step {t}: Y_hosts")
+        rec = recs[-1]
+        assert np.array_equal(host(lock), rec["lock"]), "lock after the last step"
+        for name, g in (("K", K), ("V", V), ("Y", Y), ("proxy", pc)):
+            assert_f32_close(host(g), rec[name], f"last step: {name}")
+        return
     for t, eps in enumerate(noises):
         X = perturb(X, eps, host(lock) == 0)
         Xd = dev(X, f32)
