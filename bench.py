@@ -565,7 +565,7 @@ def run_kl_lock(args):
 # kernels at the configurations where their rooflines are judged (not the
 # headline): scoring at the 8 x 4096 scoring shape (HBM-bound), and the layer
 # step with every row active at B = 4, N = 2048 (step 0 of the 32-layer stack:
-# compute-bound GEMMs and attention, the K/V scatter at 67 MB)
+# compute-bound GEMMs and attention, the K/V scatter kernel moving 671 MB)
 # ---------------------------------------------------------------------------
 def _timed(torch, fn, steps, warmup):
     """Device time of one call of fn: `reps` calls captured in a CUDA graph (so host launch
