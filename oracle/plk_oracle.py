@@ -91,9 +91,9 @@ R6  Precision policy "bf16": the layer reads bf16 tensors (X, the weights,
     the attention output, the residual stream, the SwiGLU product) stays
     float64.  All arithmetic is float64.  Policy "f64" rounds nothing.
 
-Parity unpinned: the pages print no tensor values, so nothing here is pinned to
-a printed example; every function is pinned instead to library routines,
-brute force, closed forms and invariants in ``tests/test_oracle_*.py``.
+Pins: the pages print no tensor values, so no function here is pinned to a
+printed example; every function is pinned instead to library routines, brute
+force, closed forms and invariants in ``tests/test_oracle_*.py``.
 """
 from __future__ import annotations
 
