@@ -357,7 +357,10 @@ size_t plk_step_workspace_bytes(const plk_dims* dims, int r);
  *     to Y_hosts[t] while step t + 1 computes.
  * Each step still moves its whole X in and its whole Y out; the copies of
  * consecutive steps run concurrently with the compute (on separate copy
- * engines when the host buffers are pinned).  The three streams are the
+ * engines when the host buffers are pinned).  For T >= 3 the call captures the
+ * step as CUDA graphs (one per X buffer) and launches one graph per step; with
+ * tracing on (plk_trace_events) or if the capture fails it launches the
+ * kernels directly.  The results are the same either way.  The three streams are the
  * caller's (upload_stream and download_stream should be two further streams;
  * passing `stream` for them runs everything in order).  The copies start after
  * the work already enqueued on `stream`, and `stream` waits for the last

@@ -294,6 +294,63 @@ static StepsWs steps_ws_layout(const plk_dims* d, int r) {
   return s;
 }
 
+// dst = src in 16-byte vectors (the snapshot of Y after a step): a grid-stride copy on the SMs,
+// chained to the step's last kernel by programmatic dependent launch
+__global__ void snapshot_kernel(const uint4* __restrict__ src, uint4* __restrict__ dst, size_t n16) {
+  pdl_wait();
+  pdl_trigger();
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += (size_t)gridDim.x * blockDim.x)
+    dst[i] = __ldcs(src + i);
+}
+
+// One step of plk_denoise_steps_host on `st`: the step, then Y copied into the snapshot buffer
+// that the download of this step reads.
+static int run_step_snapshot(const plk_dims* dims, const plk_weights* w, const void* Ut, int r, int metric, int mode,
+                             float tau, int k, float* proxy_cache, uint8_t* lock, void* K_cache, void* V_cache,
+                             void* Y, const void* X, uint8_t* ws, const StepWs& L, void* Ysnap, cudaStream_t st) {
+  const int e = run_step(dims, w, Ut, r, metric, mode, tau, k, proxy_cache, lock, K_cache, V_cache, Y, X, ws, L, st);
+  if (e != PLK_OK) return e;
+  const size_t bytes = (size_t)dims->B * dims->N * dims->d * (dims->dtype == PLK_BF16 ? 2 : 4);
+  return launch_pdl(snapshot_kernel, dim3(4 * (unsigned)device_sm_count()), dim3(256), 0, st, (const uint4*)Y,
+                    (uint4*)Ysnap, bytes / 16);
+}
+
+// The step captured as a CUDA graph, one per X buffer, for the duration of one
+// plk_denoise_steps_host call: one launch per step instead of the step's dozen
+// kernel launches and their descriptor set-up on the host, which would otherwise
+// take a large share of the step's device time and let host jitter idle the GPU.
+struct StepGraphs {
+  cudaGraphExec_t exec[2] = {nullptr, nullptr};
+  bool ok = false;
+  ~StepGraphs() {
+    for (cudaGraphExec_t e : exec)
+      if (e) cudaGraphExecDestroy(e);  // an instance still in flight is freed when it completes
+  }
+  // Captures run_step for both X buffers on a private stream (nothing runs during capture).
+  // Any failure leaves ok false and the caller launches the steps directly.
+  void build(const plk_dims* dims, const plk_weights* w, const void* Ut, int r, int metric, int mode, float tau,
+             int k, float* proxy_cache, uint8_t* lock, void* K_cache, void* V_cache, void* Y, void* const Xb[2],
+             void* const Ys[2], uint8_t* ws, const StepWs& L) {
+    cudaStream_t cs = nullptr;
+    if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return;
+    bool good = true;
+    for (int b = 0; b < 2 && good; ++b) {
+      cudaGraph_t graph = nullptr;
+      good = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+      if (!good) break;
+      const int e = run_step_snapshot(dims, w, Ut, r, metric, mode, tau, k, proxy_cache, lock, K_cache, V_cache, Y,
+                                      Xb[b], ws, L, Ys[b], cs);
+      const bool ended = cudaStreamEndCapture(cs, &graph) == cudaSuccess;
+      good = e == PLK_OK && ended && graph != nullptr &&
+             cudaGraphInstantiate(&exec[b], graph, 0) == cudaSuccess;
+      if (graph) cudaGraphDestroy(graph);
+    }
+    cudaStreamDestroy(cs);
+    (void)cudaGetLastError();  // a failed capture is not the caller's error: the direct path follows
+    ok = good;
+  }
+};
+
 // The events of one plk_denoise_steps_host call, destroyed with it (a recorded event that has
 // not completed is released by the driver once it does).
 struct StepEvents {
@@ -336,8 +393,15 @@ int plk_denoise_steps_host(const plk_dims* dims, const plk_weights* w, const voi
   cudaStream_t S = (cudaStream_t)stream, U = (cudaStream_t)upload_stream, D = (cudaStream_t)download_stream;
   StepEvents ev;
   if (!ev.ok) return PLK_ERR_CUDA;
-#define PLK_CU(x) \
-  if ((x) != cudaSuccess) return PLK_ERR_CUDA
+  // from three steps on, capture the step once per X buffer and launch it as a graph (not while
+  // plk_trace_events records events between the kernels)
+  StepGraphs graphs;
+  if (T >= 3 && g_ntrace == 0)
+    graphs.build(dims, w, Ut, r, metric, mode, tau, k, proxy_cache, lock, K_cache, V_cache, Y, Xb, Ys, ws, L.one);
+#define PLK_CU(x)                                 \
+  do {                                            \
+    if ((x) != cudaSuccess) return PLK_ERR_CUDA;  \
+  } while (0)
   // the copy streams start after the work already on `stream` (an earlier call's use of the
   // workspace included)
   PLK_CU(cudaEventRecord(ev.start, S));
@@ -352,14 +416,16 @@ int plk_denoise_steps_host(const plk_dims* dims, const plk_weights* w, const voi
       PLK_CU(cudaMemcpyAsync(Xb[nb], X_hosts[t + 1], bytes, cudaMemcpyHostToDevice, U));
       PLK_CU(cudaEventRecord(ev.up[nb], U));
     }
+    // step t reads X buffer b, and ends by snapshotting Y (step t + 1 updates Y in place) into
+    // snapshot buffer b, which the download of step t - 2 must have read by then
     PLK_CU(cudaStreamWaitEvent(S, ev.up[b], 0));
-    if ((e = run_step(dims, w, Ut, r, metric, mode, tau, k, proxy_cache, lock, K_cache, V_cache, Y, Xb[b], ws,
-                      L.one, S)) != PLK_OK)
-      return e;
-    // Y after step t, snapshotted (step t + 1 updates Y in place) once the download of step
-    // t - 2 has read that snapshot buffer
     if (t >= 2) PLK_CU(cudaStreamWaitEvent(S, ev.down[b], 0));
-    PLK_CU(cudaMemcpyAsync(Ys[b], Y, bytes, cudaMemcpyDeviceToDevice, S));
+    if (graphs.ok) {
+      PLK_CU(cudaGraphLaunch(graphs.exec[b], S));
+    } else if ((e = run_step_snapshot(dims, w, Ut, r, metric, mode, tau, k, proxy_cache, lock, K_cache, V_cache, Y,
+                                      Xb[b], ws, L.one, Ys[b], S)) != PLK_OK) {
+      return e;
+    }
     PLK_CU(cudaEventRecord(ev.comp[b], S));
     PLK_CU(cudaStreamWaitEvent(D, ev.comp[b], 0));
     PLK_CU(cudaMemcpyAsync(Y_hosts[t], Ys[b], bytes, cudaMemcpyDeviceToHost, D));

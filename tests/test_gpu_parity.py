@@ -935,13 +935,15 @@ def _steps_case():
     return D, r, tau, W, Ut, base, pc0, Xs
 
 
-@pytest.mark.parametrize("streams", ["separate", "same"])
+@pytest.mark.parametrize("streams", ["separate", "same", "direct"])
 def test_denoise_steps_host_pipelined(plk, streams):
     """plk_denoise_steps_host (each step's upload and download on their own streams beside the
     compute of the neighbouring steps) against the same steps as separate plk_denoise_step_host
     calls, bit for bit in reproducible mode, and against the oracle's chain of steps (threshold
-    lock bit-exact, K, V and every step's Y within the bf16 bounds).  "same": all three streams
-    are one, and every step's Y goes to the same host buffer (it ends with the last step's Y)."""
+    lock bit-exact, K, V and every step's Y within the bf16 bounds).  The call captures the step
+    as CUDA graphs and launches those; "direct": a trace event is set, so the call launches the
+    step's kernels directly instead.  "same": all three streams are one, and every step's Y goes
+    to the same host buffer (it ends with the last step's Y)."""
     D, r, tau, W, Ut, base, pc0, Xs = _steps_case()
     T = len(Xs)
     # the oracle's chain: score -> lock (drift below tau) -> partial layer step -> proxy refresh
@@ -984,14 +986,20 @@ def test_denoise_steps_host_pipelined(plk, streams):
         n = plk.steps_workspace_bytes(dm, r)
         assert n > plk.step_workspace_bytes(dm, r)
         g["workspace"] = Guarded((n,), torch.uint8)
-        if streams == "separate":
+        if streams in ("separate", "direct"):
             up, down = torch.cuda.Stream(), torch.cuda.Stream()
             Y_hosts = [torch.full(base.Y.shape, -3.0, dtype=BF).pin_memory() for _ in range(T)]
         else:
             up = down = torch.cuda.current_stream()
             Y_hosts = [torch.full(base.Y.shape, -3.0, dtype=BF).pin_memory()] * T
-        plk.denoise_steps_host(dm, Wd, Ud, r, plk.METRIC_L2, plk.SEL_THRESH_LT, tau, 0, g["proxy"].t, g["lock"].t,
-                               g["K"].t, g["V"].t, g["Y"].t, X_hosts, Y_hosts, g["workspace"].t, up, down)
+        trace = [torch.cuda.Event(enable_timing=True)] if streams == "direct" else []
+        plk.trace_events(trace)
+        try:
+            plk.denoise_steps_host(dm, Wd, Ud, r, plk.METRIC_L2, plk.SEL_THRESH_LT, tau, 0, g["proxy"].t,
+                                   g["lock"].t, g["K"].t, g["V"].t, g["Y"].t, X_hosts, Y_hosts, g["workspace"].t, up,
+                                   down)
+        finally:
+            plk.trace_events([])
         torch.cuda.current_stream().synchronize()  # the call's stream waits for the last download
         assert plk.get_status() == plk.OK
     finally:
@@ -1001,7 +1009,7 @@ def test_denoise_steps_host_pipelined(plk, streams):
     for name in ("K", "V", "Y", "proxy"):
         assert np.array_equal(host(g[name].t), host(gs[name].t)), f"{name} differs from the separate calls"
     got = [y.to(torch.float64).numpy() for y in Y_hosts]
-    steps = range(T) if streams == "separate" else [T - 1]
+    steps = [T - 1] if streams == "same" else range(T)
     for t in steps:
         assert np.array_equal(got[t], seq_Y[t]), f"Y_hosts[{t}] differs from the separate call's Y"
         never = ref_locks[0].astype(bool)  # locked at step 0: Y keeps the base rows
