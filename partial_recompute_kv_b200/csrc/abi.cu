@@ -317,8 +317,8 @@ static int run_step_snapshot(const plk_dims* dims, const plk_weights* w, const v
 
 // The step captured as a CUDA graph, one per X buffer, for the duration of one
 // plk_denoise_steps_host call: one launch per step instead of the step's dozen
-// kernel launches and their descriptor set-up on the host, which would otherwise
-// take a large share of the step's device time and let host jitter idle the GPU.
+// kernel launches and their descriptor set-up, whose host time comes close to the
+// step's device time and would let host jitter idle the GPU.
 struct StepGraphs {
   cudaGraphExec_t exec[2] = {nullptr, nullptr};
   bool ok = false;
@@ -326,7 +326,8 @@ struct StepGraphs {
     for (cudaGraphExec_t e : exec)
       if (e) cudaGraphExecDestroy(e);  // an instance still in flight is freed when it completes
   }
-  // Captures run_step for both X buffers on a private stream (nothing runs during capture).
+  // Captures the step and its snapshot copy for both X buffers on a private stream (nothing runs
+  // during capture).
   // Any failure leaves ok false and the caller launches the steps directly.
   void build(const plk_dims* dims, const plk_weights* w, const void* Ut, int r, int metric, int mode, float tau,
              int k, float* proxy_cache, uint8_t* lock, void* K_cache, void* V_cache, void* Y, void* const Xb[2],
